@@ -1,0 +1,251 @@
+// Host side of the C ABI declared in include/apr.h: argument checks, workspace
+// layout, dispatch to the kernel launchers, status plumbing.  Nothing here
+// allocates device memory.
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <atomic>
+
+#include "apr_internal.cuh"
+
+namespace apr {
+
+static thread_local char g_err[512] = "";
+static std::atomic<uint64_t> g_launches{0};
+
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+void set_error(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+}
+
+bool merge_supported(int k, int r, int nproj);
+
+static apr_status fail(apr_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+static apr_status cuda_fail(cudaError_t e, const char* where) {
+  return fail(APR_ERR_CUDA, "%s: %s (%s)", where, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static apr_status check_ws(void* ws, size_t ws_bytes, size_t need, const char* who) {
+  if (ws == nullptr) return fail(APR_ERR_WORKSPACE, "%s: workspace is NULL", who);
+  if (reinterpret_cast<uintptr_t>(ws) % kAlign)
+    return fail(APR_ERR_WORKSPACE, "%s: workspace must be %zu-byte aligned", who, kAlign);
+  if (ws_bytes < need)
+    return fail(APR_ERR_WORKSPACE, "%s: workspace has %zu bytes, needs %zu", who, ws_bytes, need);
+  return APR_OK;
+}
+
+static apr_status check_route_dims(int T, int k, int E, const char* who) {
+  if (T < 0) return fail(APR_ERR_INVALID_ARG, "%s: T=%d < 0", who, T);
+  if (E < 1 || E > APR_MAX_E) return fail(APR_ERR_INVALID_ARG, "%s: E=%d outside [1, %d]", who, E, APR_MAX_E);
+  if (k < 1 || k > E || k > APR_MAX_K)
+    return fail(APR_ERR_INVALID_ARG, "%s: k=%d outside [1, min(E, %d)]", who, k, APR_MAX_K);
+  if ((long)T * k > (1L << 30)) return fail(APR_ERR_UNSUPPORTED, "%s: T*k too large", who);
+  return APR_OK;
+}
+
+}  // namespace apr
+
+using namespace apr;
+
+extern "C" {
+
+size_t apr_workspace_size(int T, int k, int E, int max_rank, int max_d_in) {
+  if (T < 0 || k < 1 || k > APR_MAX_K || E < 1 || E > APR_MAX_E || max_rank < 8 ||
+      max_rank > APR_MAX_RANK || (max_rank & 7) || max_d_in < 8 || (max_d_in & 7))
+    return 0;
+  const WsLayout L = ws_layout(T, k, E);
+  size_t scratch = route_scratch_bytes(T, E);
+  const size_t sg = sgmm_scratch_bytes(T, k, max_rank, max_d_in);
+  if (sg > scratch) scratch = sg;
+  return L.scratch + align_up(scratch) + kAlign;
+}
+
+apr_status apr_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+  if (ws == nullptr || ws_bytes < sizeof(WsHeader)) return fail(APR_ERR_WORKSPACE, "workspace_init: too small");
+  if (reinterpret_cast<uintptr_t>(ws) % kAlign) return fail(APR_ERR_WORKSPACE, "workspace_init: misaligned");
+  cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(WsHeader), (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "workspace_init");
+  return APR_OK;
+}
+
+apr_status apr_pregate_route(const void* h, const void* Wr, int dtype, int T, int d, int E, int k,
+                             int32_t* idx, float* gate, void* ws, size_t ws_bytes, void* stream) {
+  apr_status st = check_route_dims(T, k, E, "pregate_route");
+  if (st) return st;
+  if (dtype != APR_F32 && dtype != APR_BF16) return fail(APR_ERR_INVALID_ARG, "pregate_route: bad dtype %d", dtype);
+  if (d < 8 || (d & 7)) return fail(APR_ERR_INVALID_ARG, "pregate_route: d=%d must be a positive multiple of 8", d);
+  if (T == 0) return APR_OK;
+  if (!h || !Wr || !idx || !gate) return fail(APR_ERR_INVALID_ARG, "pregate_route: NULL pointer");
+  if (!aligned16(h) || !aligned16(Wr)) return fail(APR_ERR_INVALID_ARG, "pregate_route: h/Wr not 16-byte aligned");
+  const WsLayout L = ws_layout(T, k, E);
+  st = check_ws(ws, ws_bytes, L.scratch + route_scratch_bytes(T, E), "pregate_route");
+  if (st) return st;
+  cudaError_t e = launch_route(h, Wr, dtype, T, d, E, k, idx, gate, ws, L.scratch, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "pregate_route launch");
+  return APR_OK;
+}
+
+apr_status apr_segment_tokens(const int32_t* idx, int T, int k, int E, int32_t* seg_off,
+                              int32_t* perm, void* ws, size_t ws_bytes, void* stream) {
+  apr_status st = check_route_dims(T, k, E, "segment_tokens");
+  if (st) return st;
+  if (!seg_off) return fail(APR_ERR_INVALID_ARG, "segment_tokens: NULL seg_off");
+  const WsLayout L = ws_layout(T, k, E);
+  st = check_ws(ws, ws_bytes, L.scratch, "segment_tokens");
+  if (st) return st;
+  if (T > 0 && (!idx || !perm)) return fail(APR_ERR_INVALID_ARG, "segment_tokens: NULL pointer");
+  if (T == 0) {
+    cudaError_t e = cudaMemsetAsync(seg_off, 0, sizeof(int32_t) * (E + 1), (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "segment_tokens");
+    return APR_OK;
+  }
+  cudaError_t e = launch_segment(idx, T, k, E, seg_off, perm, ws, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "segment_tokens launch");
+  return APR_OK;
+}
+
+apr_status apr_sgmm_shrink_expand(const void* x, int d_in, const apr_proj* projs, int nproj,
+                                  int dtype, int T, int k, int E, const int32_t* ranks,
+                                  int max_rank, const int32_t* idx, const float* gate,
+                                  const int32_t* seg_off, const int32_t* perm, void* ws,
+                                  size_t ws_bytes, int kernel, void* stream) {
+  apr_status st = check_route_dims(T, k, E, "sgmm");
+  if (st) return st;
+  if (dtype != APR_F32 && dtype != APR_BF16) return fail(APR_ERR_INVALID_ARG, "sgmm: bad dtype %d", dtype);
+  if (nproj < 1 || nproj > APR_MAX_PROJ) return fail(APR_ERR_INVALID_ARG, "sgmm: nproj=%d outside [1, %d]", nproj, APR_MAX_PROJ);
+  if (!projs) return fail(APR_ERR_INVALID_ARG, "sgmm: NULL projs");
+  if (d_in < 8 || (d_in & 7)) return fail(APR_ERR_INVALID_ARG, "sgmm: d_in=%d must be a positive multiple of 8", d_in);
+  if (max_rank < 8 || max_rank > APR_MAX_RANK || (max_rank & 7))
+    return fail(APR_ERR_INVALID_ARG, "sgmm: max_rank=%d must be a multiple of 8 in [8, %d]", max_rank, APR_MAX_RANK);
+  if (kernel < APR_SGMM_AUTO || kernel > APR_SGMM_TENSOR) return fail(APR_ERR_INVALID_ARG, "sgmm: bad kernel %d", kernel);
+  for (int p = 0; p < nproj; ++p) {
+    const apr_proj& pj = projs[p];
+    if (pj.d_out < 8 || (pj.d_out & 7)) return fail(APR_ERR_INVALID_ARG, "sgmm: proj %d d_out=%d must be a positive multiple of 8", p, pj.d_out);
+    if (T > 0 && (!pj.y || !pj.y_base || !pj.A || !pj.B)) return fail(APR_ERR_INVALID_ARG, "sgmm: proj %d has a NULL pointer", p);
+    if (T > 0 && (!aligned16(pj.y) || !aligned16(pj.y_base))) return fail(APR_ERR_INVALID_ARG, "sgmm: proj %d y/y_base not 16-byte aligned", p);
+  }
+  if (T == 0) return APR_OK;
+  if (!x || !ranks || !idx || !gate || !seg_off || !perm) return fail(APR_ERR_INVALID_ARG, "sgmm: NULL pointer");
+  if (!aligned16(x)) return fail(APR_ERR_INVALID_ARG, "sgmm: x not 16-byte aligned");
+  const WsLayout L = ws_layout(T, k, E);
+  st = check_ws(ws, ws_bytes, L.scratch + sgmm_scratch_bytes(T, k, max_rank, d_in), "sgmm");
+  if (st) return st;
+
+  SgmmArgs a;
+  memset(&a, 0, sizeof(a));
+  a.x = x;
+  a.d_in = d_in;
+  a.nproj = nproj;
+  for (int p = 0; p < nproj; ++p) {
+    a.proj[p].y = projs[p].y;
+    a.proj[p].y_base = projs[p].y_base;
+    a.proj[p].d_out = projs[p].d_out;
+    a.proj[p].A = projs[p].A;
+    a.proj[p].B = projs[p].B;
+  }
+  a.T = T;
+  a.k = k;
+  a.E = E;
+  a.ranks = ranks;
+  a.max_rank = max_rank;
+  a.idx = idx;
+  a.gate = gate;
+  a.seg_off = seg_off;
+  a.perm = perm;
+  a.ws = ws;
+
+  int use = kernel;
+  if (use == APR_SGMM_AUTO) {
+    // mean pairs per adapter, known on the host without reading the routing
+    const double mean_seg = (double)T * k / E;
+    use = (mean_seg >= 256.0 && sgmm_tensor_supported(a, dtype)) ? APR_SGMM_TENSOR : APR_SGMM_SKINNY;
+  }
+  cudaError_t e;
+  if (use == APR_SGMM_TENSOR) {
+    if (!sgmm_tensor_supported(a, dtype))
+      return fail(APR_ERR_UNSUPPORTED, "sgmm: tensor-core kernel needs bf16, k<=2, max_rank<=64, d_in%%64==0, d_out%%16==0");
+    e = launch_sgmm_tensor(a, (cudaStream_t)stream);
+  } else {
+    e = launch_sgmm_skinny(a, dtype, L.scratch, (cudaStream_t)stream);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "sgmm launch");
+  return APR_OK;
+}
+
+apr_status apr_merge_adapters(const apr_merge_proj* projs, int nproj, int E, int r,
+                              const int32_t* idx, const float* gate, int k, void* ws,
+                              size_t ws_bytes, void* stream) {
+  if (nproj < 1) return fail(APR_ERR_INVALID_ARG, "merge: nproj=%d < 1", nproj);
+  if (E < 1 || E > APR_MAX_E) return fail(APR_ERR_INVALID_ARG, "merge: E=%d outside [1, %d]", E, APR_MAX_E);
+  if (k < 1 || k > E || k > APR_MAX_K) return fail(APR_ERR_INVALID_ARG, "merge: k=%d outside [1, min(E, %d)]", k, APR_MAX_K);
+  if (r < 8 || (r & 7) || r > APR_MAX_RANK) return fail(APR_ERR_INVALID_ARG, "merge: r=%d must be a multiple of 8 in [8, %d]", r, APR_MAX_RANK);
+  if (!merge_supported(k, r, nproj)) return fail(APR_ERR_UNSUPPORTED, "merge: k*r=%d > 64 or nproj=%d > 4096", k * r, nproj);
+  if (!projs || !idx || !gate) return fail(APR_ERR_INVALID_ARG, "merge: NULL pointer");
+  apr_status st = check_ws(ws, ws_bytes, sizeof(WsHeader), "merge");
+  if (st) return st;
+  cudaError_t e = launch_merge(projs, nproj, E, r, idx, gate, k, ws, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "merge launch");
+  return APR_OK;
+}
+
+apr_status apr_gemv(const void* W, const void* x, void* y, int d_in, int d_out, void* stream) {
+  if (d_in < 8 || (d_in & 7)) return fail(APR_ERR_INVALID_ARG, "gemv: d_in=%d must be a positive multiple of 8", d_in);
+  if (d_in > 48 * 1024) return fail(APR_ERR_UNSUPPORTED, "gemv: d_in=%d > 49152", d_in);
+  if (d_out < 0) return fail(APR_ERR_INVALID_ARG, "gemv: d_out=%d < 0", d_out);
+  if (d_out == 0) return APR_OK;
+  if (!W || !x || !y) return fail(APR_ERR_INVALID_ARG, "gemv: NULL pointer");
+  if (!aligned16(W) || !aligned16(x)) return fail(APR_ERR_INVALID_ARG, "gemv: W/x not 16-byte aligned");
+  cudaError_t e = launch_gemv(W, x, y, d_in, d_out, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "gemv launch");
+  return APR_OK;
+}
+
+apr_status apr_stream_status(void* ws, void* stream) {
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "stream_status");
+  if (ws == nullptr) return APR_OK;
+  int words[2] = {0, 0};
+  e = cudaMemcpy(words, ws, sizeof(words), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "stream_status read");
+  if (words[0] != 0) {
+    const int zero[2] = {0, 0};
+    e = cudaMemcpy(ws, zero, sizeof(zero), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_fail(e, "stream_status clear");
+    return fail((apr_status)words[0], "device reported %s (kernel %d, value %d)",
+                apr_status_string(words[0]), (words[1] >> 24) & 0xFF, words[1] & 0xFFFFFF);
+  }
+  return APR_OK;
+}
+
+const char* apr_last_error(void) { return g_err; }
+
+const char* apr_status_string(int s) {
+  switch (s) {
+    case APR_OK: return "APR_OK";
+    case APR_ERR_INVALID_ARG: return "APR_ERR_INVALID_ARG";
+    case APR_ERR_UNSUPPORTED: return "APR_ERR_UNSUPPORTED";
+    case APR_ERR_WORKSPACE: return "APR_ERR_WORKSPACE";
+    case APR_ERR_CUDA: return "APR_ERR_CUDA";
+    case APR_ERR_DEVICE_INDEX: return "APR_ERR_DEVICE_INDEX";
+    case APR_ERR_TIMEOUT: return "APR_ERR_TIMEOUT";
+    default: return "APR_ERR_UNKNOWN";
+  }
+}
+
+uint64_t apr_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
+}  // extern "C"

@@ -1,0 +1,222 @@
+// Internal definitions shared by the libapr translation units: workspace
+// layout, device error reporting, launch helpers and element conversions.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <utility>
+
+#include "../../include/apr.h"
+
+namespace apr {
+
+// ---------------------------------------------------------------- workspace
+
+constexpr size_t kAlign = 256;
+constexpr int kPairTile = 32;       // pairs per shrink tile of the skinny kernel
+constexpr int kSetTile = 128;       // tokens per tensor-core tile (one adapter set)
+constexpr int kShrinkKC = 2048;     // input columns per skinny shrink item
+constexpr int kRouteKC = 256;       // minimum router split-K chunk
+
+struct WsHeader {
+  int err;          // first device-side apr_status recorded (0 = none)
+  int err_info;     // detail (kernel id << 24 | value)
+  int n_ptiles;     // shrink pair tiles written by the segment kernel
+  int n_stiles;     // tensor-core set tiles written by the segment kernel
+  int T, k, E;      // routing the plan was built for
+  int pad[57];
+};
+static_assert(sizeof(WsHeader) == 256, "header is one alignment unit");
+
+struct PairTile {   // a run of <= kPairTile consecutive sorted pairs of one adapter
+  int e, start, len, pad;
+};
+struct SetTile {    // a run of <= kSetTile tokens (in set order) sharing one adapter set
+  int start, len;
+};
+
+__host__ __device__ inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+__host__ __device__ inline int max_ptiles(int T, int k, int E) {
+  long n = (long)T * k;
+  long m = n < E ? n : E;
+  return (int)((n + kPairTile - 1) / kPairTile + m + 1);
+}
+
+struct WsLayout {
+  size_t inv, tok_order, tok_tmp, ptiles, stiles, scratch;
+};
+
+__host__ __device__ inline WsLayout ws_layout(int T, int k, int E) {
+  WsLayout L;
+  size_t o = align_up(sizeof(WsHeader));
+  L.inv = o;       o = align_up(o + sizeof(int) * (size_t)T * k);
+  L.tok_order = o; o = align_up(o + sizeof(int) * (size_t)T);
+  L.tok_tmp = o;   o = align_up(o + sizeof(int) * (size_t)T);
+  L.ptiles = o;    o = align_up(o + sizeof(PairTile) * (size_t)max_ptiles(T, k, E));
+  L.stiles = o;    o = align_up(o + sizeof(SetTile) * (size_t)(T + 1));
+  L.scratch = o;
+  (void)E;
+  return L;
+}
+
+inline int route_max_chunks(int T, int E) {
+  long te = (long)T * E;
+  long cap = te > 0 ? (1L << 18) / te : 16;
+  if (cap < 1) cap = 1;
+  if (cap > 16) cap = 16;
+  return (int)cap;
+}
+
+inline size_t route_scratch_bytes(int T, int E) {
+  return sizeof(float) * (size_t)route_max_chunks(T, E) * T * E;
+}
+
+inline int shrink_kchunks(int d_in) { return (d_in + kShrinkKC - 1) / kShrinkKC; }
+
+inline size_t sgmm_scratch_bytes(int T, int k, int max_rank, int d_in) {
+  return sizeof(float) * (size_t)shrink_kchunks(d_in) * T * k * max_rank;
+}
+
+template <typename P>
+__host__ __device__ inline P* ws_at(void* ws, size_t off) {
+  return reinterpret_cast<P*>(reinterpret_cast<char*>(ws) + off);
+}
+
+// ---------------------------------------------------------------- device helpers
+
+// Record the first device-side fault; later ones keep the first code.
+__device__ inline void report(void* ws, int code, int kernel_id, int value) {
+  WsHeader* h = reinterpret_cast<WsHeader*>(ws);
+  if (atomicCAS(&h->err, 0, code) == 0) {
+    atomicExch(&h->err_info, (kernel_id << 24) | (value & 0xFFFFFF));
+  }
+}
+
+// Programmatic dependent launch: wait for the preceding grid on the stream
+// (and its memory) before reading inputs; then let the next grid launch.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float v);
+template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) {
+  return __float2bfloat16_rn(v);
+}
+
+// Unpack 8 consecutive elements starting at a 16-byte aligned address.
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&f)[8]) {
+  uint4 u = *reinterpret_cast<const uint4*>(p);
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 t = __bfloat1622float2(h[i]);
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
+__device__ __forceinline__ void load8(const float* p, float (&f)[8]) {
+  float4 a = reinterpret_cast<const float4*>(p)[0];
+  float4 b = reinterpret_cast<const float4*>(p)[1];
+  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+  f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+
+// Streaming (evict-first) variant for data read once per step.
+__device__ __forceinline__ void load8_stream(const __nv_bfloat16* p, float (&f)[8]) {
+  uint4 u = __ldcs(reinterpret_cast<const uint4*>(p));
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 t = __bfloat1622float2(h[i]);
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
+__device__ __forceinline__ void load8_stream(const float* p, float (&f)[8]) {
+  float4 a = __ldcs(reinterpret_cast<const float4*>(p));
+  float4 b = __ldcs(reinterpret_cast<const float4*>(p) + 1);
+  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+  f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+
+__device__ __forceinline__ void store8(__nv_bfloat16* p, const float (&f)[8]) {
+  uint4 u;
+  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+  *reinterpret_cast<uint4*>(p) = u;
+}
+__device__ __forceinline__ void store8(float* p, const float (&f)[8]) {
+  reinterpret_cast<float4*>(p)[0] = make_float4(f[0], f[1], f[2], f[3]);
+  reinterpret_cast<float4*>(p)[1] = make_float4(f[4], f[5], f[6], f[7]);
+}
+
+// Kernel ids used in WsHeader::err_info.
+enum KernelId { K_ROUTE = 1, K_TOPK = 2, K_SEGMENT = 3, K_SHRINK = 4, K_EXPAND = 5, K_MERGE = 6, K_TC = 7 };
+
+}  // namespace apr
+
+// ---------------------------------------------------------------- launchers (host)
+namespace apr {
+
+void count_launch();
+void set_error(const char* fmt, ...);
+
+// Launch with programmatic stream serialization allowed (PDL).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  count_launch();
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// Host-side launchers implemented in the kernel translation units.
+cudaError_t launch_route(const void* h, const void* Wr, int dtype, int T, int d, int E, int k,
+                         int32_t* idx, float* gate, void* ws, size_t scratch_off, cudaStream_t s);
+cudaError_t launch_segment(const int32_t* idx, int T, int k, int E, int32_t* seg_off,
+                           int32_t* perm, void* ws, cudaStream_t s);
+struct ProjArgs {
+  void* y;
+  const void* y_base;
+  int d_out;
+  const void* const* A;
+  const void* const* B;
+};
+struct SgmmArgs {
+  const void* x;
+  int d_in;
+  ProjArgs proj[APR_MAX_PROJ];
+  int nproj;
+  int T, k, E;
+  const int32_t* ranks;
+  int max_rank;
+  const int32_t* idx;
+  const float* gate;
+  const int32_t* seg_off;
+  const int32_t* perm;
+  void* ws;
+};
+cudaError_t launch_sgmm_skinny(const SgmmArgs& a, int dtype, size_t scratch_off, cudaStream_t s);
+cudaError_t launch_sgmm_tensor(const SgmmArgs& a, cudaStream_t s);
+bool sgmm_tensor_supported(const SgmmArgs& a, int dtype);
+cudaError_t launch_merge(const apr_merge_proj* projs, int nproj, int E, int r, const int32_t* idx,
+                         const float* gate, int k, void* ws, cudaStream_t s);
+cudaError_t launch_gemv(const void* W, const void* x, void* y, int d_in, int d_out, cudaStream_t s);
+
+}  // namespace apr

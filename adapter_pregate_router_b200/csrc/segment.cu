@@ -1,0 +1,278 @@
+// Segments of the segmented gather product (AdaFuse summary, gist.science,
+// Resumen tecnico §2.B: SGMM gathers the tokens of each adapter and runs one
+// batched product).  One CTA of 1024 threads builds, bit-exactly and
+// deterministically:
+//   seg_off [E+1]  exclusive prefix sum of the per-adapter pair counts
+//   perm    [T*k]  pair ids q = t*k+j grouped by adapter, ascending q inside
+//                  a segment (stable counting sort)
+// and the routing plan in the workspace:
+//   inv      [T*k] sorted position of pair q
+//   tiles    pair tiles (<= kPairTile pairs of one adapter) for the shrink
+//   tok_order[T]   tokens ordered by their sorted adapter tuple (LSD radix of
+//                  k stable counting sorts), so that tokens sharing an adapter
+//                  set are contiguous
+//   set tiles      runs of <= kSetTile tokens with one adapter set
+// The histograms use shared-memory atomics (order-free counts); every order-
+// dependent step runs in one warp, 32 elements at a time, with __match_any_sync
+// ranking equal keys by lane, so the result is unique.
+#include "apr_internal.cuh"
+
+namespace apr {
+
+constexpr int SEG_THREADS = 1024;
+
+__device__ __forceinline__ unsigned lanemask_lt() {
+  unsigned m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+// Exclusive scan of one value per thread over the whole block; *total gets the sum.
+__device__ int block_exclusive_scan(int v, int* warp_sums, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nwarps = blockDim.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, off);
+    if (lane >= off) x += y;
+  }
+  if (lane == 31) warp_sums[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int s = lane < nwarps ? warp_sums[lane] : 0;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, s, off);
+      if (lane >= off) s += y;
+    }
+    warp_sums[lane] = s;
+  }
+  __syncthreads();
+  const int before = (warp > 0 ? warp_sums[warp - 1] : 0) + x - v;
+  *total = warp_sums[nwarps - 1];
+  __syncthreads();
+  return before;
+}
+
+// The p-th smallest adapter of token t (its tuple sorted ascending).
+__device__ __forceinline__ int sorted_key(const int32_t* idx, int t, int k, int p) {
+  if (k == 1) return idx[t];
+  if (k == 2) {
+    const int a0 = idx[2 * (size_t)t], a1 = idx[2 * (size_t)t + 1];
+    return p == 0 ? min(a0, a1) : max(a0, a1);
+  }
+  int a[APR_MAX_K];
+#pragma unroll
+  for (int j = 0; j < APR_MAX_K; ++j) a[j] = j < k ? idx[(size_t)t * k + j] : 0x7FFFFFFF;
+#pragma unroll
+  for (int i = 1; i < APR_MAX_K; ++i) {
+#pragma unroll
+    for (int j = APR_MAX_K - 1; j >= 1; --j) {
+      if (j <= i && a[j - 1] > a[j]) {
+        const int tmp = a[j];
+        a[j] = a[j - 1];
+        a[j - 1] = tmp;
+      }
+    }
+  }
+  int r = a[0];
+#pragma unroll
+  for (int j = 1; j < APR_MAX_K; ++j)
+    if (j == p) r = a[j];
+  return r;
+}
+
+__device__ __forceinline__ bool same_set(const int32_t* idx, int t0, int t1, int k) {
+  for (int p = 0; p < k; ++p)
+    if (sorted_key(idx, t0, k, p) != sorted_key(idx, t1, k, p)) return false;
+  return true;
+}
+
+__global__ void __launch_bounds__(SEG_THREADS) segment_kernel(const int32_t* __restrict__ idx, int T,
+                                                              int k, int E,
+                                                              int32_t* __restrict__ seg_off,
+                                                              int32_t* __restrict__ perm, void* ws) {
+  pdl_wait();
+  pdl_trigger();
+  extern __shared__ int sm[];
+  int* hist = sm;          // [E]
+  int* base = sm + E;      // [E]
+  __shared__ int warp_sums[32];
+  __shared__ int bad;
+  __shared__ int carry[2];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int n = T * k;
+  const WsLayout L = ws_layout(T, k, E);
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
+  int* inv = ws_at<int>(ws, L.inv);
+  int* tok_order = ws_at<int>(ws, L.tok_order);
+  int* tok_tmp = ws_at<int>(ws, L.tok_tmp);
+  PairTile* ptiles = ws_at<PairTile>(ws, L.ptiles);
+  SetTile* stiles = ws_at<SetTile>(ws, L.stiles);
+
+  // 1. counts and validation
+  for (int e = tid; e < E; e += SEG_THREADS) hist[e] = 0;
+  if (tid == 0) bad = 0;
+  __syncthreads();
+  for (int q = tid; q < n; q += SEG_THREADS) {
+    const int e = idx[q];
+    if (e < 0 || e >= E) {
+      bad = 1;
+    } else {
+      atomicAdd(&hist[e], 1);
+    }
+  }
+  __syncthreads();
+  if (bad) {
+    for (int e = tid; e <= E; e += SEG_THREADS) seg_off[e] = 0;
+    if (tid == 0) {
+      report(ws, APR_ERR_DEVICE_INDEX, K_SEGMENT, 0);
+      hdr->n_ptiles = 0;
+      hdr->n_stiles = 0;
+    }
+    return;
+  }
+  // 2. segment offsets
+  int total;
+  {
+    const int c = tid < E ? hist[tid] : 0;
+    const int off = block_exclusive_scan(c, warp_sums, &total);
+    if (tid < E) {
+      base[tid] = off;
+      seg_off[tid] = off;
+    }
+    if (tid == 0) seg_off[E] = total;
+  }
+  __syncthreads();
+  // 3. shrink pair tiles: ceil(count / kPairTile) per adapter, in adapter order
+  {
+    const int c = tid < E ? hist[tid] : 0;
+    const int nt = (c + kPairTile - 1) / kPairTile;
+    int ntiles;
+    const int toff = block_exclusive_scan(nt, warp_sums, &ntiles);
+    if (tid < E) {
+      const int s0 = base[tid];
+      for (int i = 0; i < nt; ++i) {
+        PairTile p;
+        p.e = tid;
+        p.start = s0 + i * kPairTile;
+        p.len = min(kPairTile, c - i * kPairTile);
+        p.pad = 0;
+        ptiles[toff + i] = p;
+      }
+    }
+    if (tid == 0) {
+      hdr->n_ptiles = ntiles;
+      hdr->T = T;
+      hdr->k = k;
+      hdr->E = E;
+    }
+  }
+  __syncthreads();
+  // 4. stable scatter of the pairs (one warp, in order)
+  if (warp == 0) {
+    for (int q0 = 0; q0 < n; q0 += 32) {
+      const int q = q0 + lane;
+      const bool valid = q < n;
+      const int e = valid ? idx[q] : -1 - lane;
+      const unsigned peers = __match_any_sync(0xffffffffu, e);
+      if (valid) {
+        const int pos = base[e] + __popc(peers & lanemask_lt());
+        perm[pos] = q;
+        inv[q] = pos;
+      }
+      __syncwarp();
+      if (valid && lane == __ffs(peers) - 1) base[e] += __popc(peers);
+      __syncwarp();
+    }
+  }
+  __syncthreads();
+  // 5. tokens ordered by sorted adapter tuple: LSD, k stable counting sorts
+  int* src = tok_tmp;
+  int* dst = tok_order;
+  for (int i = tid; i < T; i += SEG_THREADS) src[i] = i;
+  for (int p = k - 1; p >= 0; --p) {
+    for (int e = tid; e < E; e += SEG_THREADS) hist[e] = 0;
+    __syncthreads();
+    for (int i = tid; i < T; i += SEG_THREADS) atomicAdd(&hist[sorted_key(idx, i, k, p)], 1);
+    __syncthreads();
+    {
+      const int c = tid < E ? hist[tid] : 0;
+      int tot;
+      const int off = block_exclusive_scan(c, warp_sums, &tot);
+      if (tid < E) base[tid] = off;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      for (int i0 = 0; i0 < T; i0 += 32) {
+        const int i = i0 + lane;
+        const bool valid = i < T;
+        const int t = valid ? src[i] : 0;
+        const int key = valid ? sorted_key(idx, t, k, p) : -1 - lane;
+        const unsigned peers = __match_any_sync(0xffffffffu, key);
+        if (valid) dst[base[key] + __popc(peers & lanemask_lt())] = t;
+        __syncwarp();
+        if (valid && lane == __ffs(peers) - 1) base[key] += __popc(peers);
+        __syncwarp();
+      }
+    }
+    __syncthreads();
+    int* tmp = src;
+    src = dst;
+    dst = tmp;
+  }
+  // src holds the final order
+  if (src != tok_order) {
+    for (int i = tid; i < T; i += SEG_THREADS) tok_order[i] = src[i];
+    __syncthreads();
+  }
+  // 6. set tiles: split runs of equal adapter sets into <= kSetTile tokens
+  if (warp == 0) {
+    if (lane == 0) {
+      carry[0] = 0;  // start of the current run
+      carry[1] = 0;  // tiles written
+    }
+    __syncwarp();
+    for (int i0 = 0; i0 < T; i0 += 32) {
+      const int i = i0 + lane;
+      const bool valid = i < T;
+      bool head = false;
+      if (valid) head = (i == 0) || !same_set(idx, tok_order[i - 1], tok_order[i], k);
+      const unsigned heads = __ballot_sync(0xffffffffu, head);
+      const unsigned upto = heads & (lanemask_lt() | (1u << lane));
+      const int run_start = upto ? i0 + (31 - __clz(upto)) : carry[0];
+      const bool tstart = valid && (head || ((i - run_start) % kSetTile) == 0);
+      const unsigned starts = __ballot_sync(0xffffffffu, tstart);
+      const int wbase = carry[1];
+      if (tstart) {
+        SetTile st;
+        st.start = i;
+        st.len = 0;
+        stiles[wbase + __popc(starts & lanemask_lt())] = st;
+      }
+      __syncwarp();
+      if (lane == 31) {
+        carry[0] = run_start;
+        carry[1] = wbase + __popc(starts);
+      }
+      __syncwarp();
+    }
+  }
+  __syncthreads();
+  const int nst = carry[1];
+  for (int j = tid; j < nst; j += SEG_THREADS) {
+    const int end = (j + 1 < nst) ? stiles[j + 1].start : T;
+    stiles[j].len = end - stiles[j].start;
+  }
+  if (tid == 0) hdr->n_stiles = nst;
+}
+
+cudaError_t launch_segment(const int32_t* idx, int T, int k, int E, int32_t* seg_off,
+                           int32_t* perm, void* ws, cudaStream_t s) {
+  const size_t smem = sizeof(int) * 2 * (size_t)E;
+  return launch_pdl(segment_kernel, dim3(1), dim3(SEG_THREADS), smem, s, idx, T, k, E, seg_off,
+                    perm, ws);
+}
+
+}  // namespace apr

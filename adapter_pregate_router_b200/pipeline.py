@@ -1,0 +1,192 @@
+"""One step of the pre-gated mixture-of-LoRA hot path on device buffers.
+
+A ``Step`` holds the device tensors of one named workload (see ``workloads``)
+and runs, through the C ABI only:
+
+* ``apr_pregate_route``   once per step (the router of the first adapted layer
+  fixes every layer's adapters, AdaFuse summary §2.A);
+* ``apr_segment_tokens``  once per step;
+* ``apr_sgmm_shrink_expand`` once per (layer, shared-input group);
+
+or, for the batch-1 merge workload, the route, one ``apr_merge_adapters``
+over every weight and one ``apr_gemv`` per weight (§2.B steps 1-5).
+
+Tensors are built once from the seeded pools (``workloads.device_tensor``) and
+stay resident; ``run()`` enqueues the step on the current stream.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from . import apr
+from . import workloads as W
+
+
+def _dt(cfg):
+    return torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+
+
+class Step:
+    def __init__(self, cfg: W.Config, device="cuda", layers=None, zero_y_base=False,
+                 kernel=apr.SGMM_AUTO, out_of_place=True):
+        self.cfg = cfg
+        self.device = device
+        self.kernel = kernel
+        self.layers = list(range(cfg.layers)) if layers is None else list(layers)
+        dt = _dt(cfg)
+        T, E, k = cfg.T, cfg.E, cfg.k
+        self.ranks_np = W.ranks(cfg)
+        self.max_rank = int(self.ranks_np.max())
+        self.ranks = torch.from_numpy(self.ranks_np).to(device)
+        h, Wr, self.forced = W.router_inputs(cfg)
+        self.h = torch.from_numpy(h).to(device=device, dtype=dt)
+        self.Wr = torch.from_numpy(Wr).to(device=device, dtype=dt)
+        self.idx = torch.empty((T, k), dtype=torch.int32, device=device)
+        self.gate = torch.empty((T, k), dtype=torch.float32, device=device)
+        self.seg_off = torch.empty(E + 1, dtype=torch.int32, device=device)
+        self.perm = torch.empty(T * k, dtype=torch.int32, device=device)
+        max_d_in = max(g.d_in for g in cfg.groups)
+        self.ws = apr.workspace(T, k, E, self.max_rank, max_d_in, device=device)
+        self.keep = []
+        if cfg.merge:
+            self._build_merge(dt)
+        else:
+            self._build_sgmm(dt, zero_y_base, out_of_place)
+
+    # ------------------------------------------------------------ SGMM workload
+    def _build_sgmm(self, dt, zero_y_base, out_of_place):
+        cfg, dev = self.cfg, self.device
+        T = cfg.T
+        self.calls = []          # (x, [Proj...], (l, g))
+        self.outputs = {}        # (l, g, p) -> (y, y_base)
+        self.adapters = {}       # (l, g, p) -> (A list, B list)
+        # Activations live in two flat arenas so that a step's inputs (router
+        # hidden, x, y_base) and outputs (y) move host<->device in one copy each.
+        n_in = T * cfg.d_router
+        n_out = 0
+        for _ in self.layers:
+            for g in cfg.groups:
+                n_in += T * g.d_in + sum(T * d for d in g.d_outs)
+                n_out += sum(T * d for d in g.d_outs)
+        self.act_in = torch.empty(n_in, dtype=dt, device=dev)
+        self.act_out = self.act_in if not out_of_place else torch.empty(n_out, dtype=dt, device=dev)
+        pos_in = [0]
+
+        def take_in(shape):
+            n = int(np.prod(shape))
+            v = self.act_in[pos_in[0]:pos_in[0] + n].view(shape)
+            pos_in[0] += n
+            return v
+        h = take_in(tuple(self.h.shape))
+        h.copy_(self.h)
+        self.h = h
+        pos_out = 0
+        for l in self.layers:
+            for g in cfg.groups:
+                x = take_in((T, g.d_in))
+                x.copy_(W.device_tensor(cfg, W.x_key(l, g.name), (T, g.d_in), dev))
+                projs = []
+                for p, d_out in zip(g.proj_names, g.d_outs):
+                    A = [W.device_tensor(cfg, W.a_key(l, g.name, p, e), (int(self.ranks_np[e]), g.d_in), dev)
+                         for e in range(cfg.E)]
+                    B = [W.device_tensor(cfg, W.b_key(l, g.name, p, e), (d_out, int(self.ranks_np[e])), dev)
+                         for e in range(cfg.E)]
+                    At, Bt = apr.ptr_array(A, dev), apr.ptr_array(B, dev)
+                    yb = take_in((T, d_out))
+                    if zero_y_base:
+                        yb.zero_()
+                    else:
+                        yb.copy_(W.device_tensor(cfg, W.ybase_key(l, g.name, p), (T, d_out), dev))
+                    if out_of_place:
+                        y = self.act_out[pos_out:pos_out + T * d_out].view(T, d_out)
+                        pos_out += T * d_out
+                    else:
+                        y = yb
+                    projs.append(apr.make_proj(y, yb, At, Bt))
+                    self.outputs[(l, g.name, p)] = (y, yb)
+                    self.adapters[(l, g.name, p)] = (A, B)
+                    self.keep += [At, Bt]
+                self.calls.append((x, projs, (l, g.name)))
+        W.clear_device_pools()
+
+    # ------------------------------------------------------------ merge workload
+    def _build_merge(self, dt):
+        cfg, dev = self.cfg, self.device
+        entries = []
+        self.weights = {}    # (l, g, p) -> (W, Wp, x, y)
+        self.adapters = {}
+        for l in self.layers:
+            for g in cfg.groups:
+                for p, d_out in zip(g.proj_names, g.d_outs):
+                    Wt = W.device_tensor(cfg, W.w_key(l, g.name, p), (d_out, g.d_in), dev)
+                    Wp = torch.empty_like(Wt)
+                    A = [W.device_tensor(cfg, W.a_key(l, g.name, p, e), (int(self.ranks_np[e]), g.d_in), dev)
+                         for e in range(cfg.E)]
+                    B = [W.device_tensor(cfg, W.b_key(l, g.name, p, e), (d_out, int(self.ranks_np[e])), dev)
+                         for e in range(cfg.E)]
+                    At, Bt = apr.ptr_array(A, dev), apr.ptr_array(B, dev)
+                    x = W.device_tensor(cfg, W.xm_key(l, g.name, p), (g.d_in,), dev)
+                    y = torch.empty(d_out, dtype=dt, device=dev)
+                    entries.append((Wt, Wp, At, Bt))
+                    self.weights[(l, g.name, p)] = (Wt, Wp, x, y)
+                    self.adapters[(l, g.name, p)] = (A, B)
+                    self.keep += [At, Bt]
+        self.merge_tab = apr.merge_table(entries, dev)
+        self.nmerge = len(entries)
+        W.clear_device_pools()
+
+    # ------------------------------------------------------------ running
+    def route(self, stream=None):
+        cfg = self.cfg
+        apr.pregate_route(self.h, self.Wr, cfg.k, self.idx, self.gate, self.ws, stream)
+        apr.segment_tokens(self.idx, cfg.E, self.seg_off, self.perm, self.ws, stream)
+
+    def layers_only(self, stream=None):
+        cfg = self.cfg
+        if cfg.merge:
+            apr.merge_adapters(self.merge_tab, self.nmerge, cfg.E, self.max_rank, self.idx, self.gate,
+                               cfg.k, self.ws, stream)
+            for (Wt, Wp, x, y) in self.weights.values():
+                apr.gemv(Wp, x, y, stream)
+            return
+        for x, projs, _ in self.calls:
+            apr.sgmm_shrink_expand(x, projs, cfg.k, cfg.E, self.ranks, self.max_rank, self.idx,
+                                   self.gate, self.seg_off, self.perm, self.ws, self.kernel, stream)
+
+    def run(self, stream=None):
+        self.route(stream)
+        self.layers_only(stream)
+
+    def launches_per_step(self) -> int:
+        before = apr.kernel_launches()
+        s = torch.cuda.Stream()
+        with torch.cuda.stream(s):
+            self.run()
+        s.synchronize()
+        return apr.kernel_launches() - before
+
+    # ------------------------------------------------------------ bytes moved
+    def algorithmic_bytes(self, idx_np=None) -> int:
+        """Bytes the step must move at least once (inputs read once, outputs written once)."""
+        cfg = self.cfg
+        el = 2 if cfg.dtype == "bf16" else 4
+        T = cfg.T
+        if idx_np is None:
+            idx_np = self.idx.cpu().numpy()
+        touched = np.unique(idx_np.reshape(-1))
+        b = 0
+        b += T * cfg.d_router * el + cfg.E * cfg.d_router * el    # router h, Wr
+        for l in self.layers:
+            for g in cfg.groups:
+                if cfg.merge:
+                    for d_out in g.d_outs:
+                        b += 2 * d_out * g.d_in * el                              # W read, Wp write
+                        b += sum(int(self.ranks_np[e]) * (g.d_in + d_out) * el for e in touched)
+                        b += d_out * g.d_in * el + g.d_in * el + d_out * el       # GEMV
+                    continue
+                b += T * g.d_in * el                                               # x once per group
+                for d_out in g.d_outs:
+                    b += sum(int(self.ranks_np[e]) * (g.d_in + d_out) * el for e in touched)
+                    b += 2 * T * d_out * el                                        # y_base read, y write
+        return b

@@ -1,0 +1,431 @@
+"""Benchmark of the pre-gated mixture-of-LoRA hot path (one JSON line on rank 0).
+
+A step is one pass of the whole path over one batch of synthetic tokens:
+router + top-k + gates (once), segments (once), then the SGMM shrink/expand
+fused into the base-output add for every (layer, shared-input group) of the
+workload.  The default workload is ``decode`` (Llama-2-7B layer set, 32
+tokens, 8 rank-16 adapters, top-2).  The step is captured once in a CUDA graph
+and replayed.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+With N > 1 (torchrun, one process per GPU) every rank runs its own batch
+(weak scaling: tokens are independent and the path has no exchange step);
+timing is the max over ranks of the CUDA-event time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "mixture-of-LoRA SGMM tokens/s at 1 B200; % of HBM / tensor-core roofline"
+DESCR = {
+    "decode": "decode: Llama-2-7B layer set (32 layers; q,k,v,o 4096->4096; gate,up 4096->11008; "
+              "down 11008->4096), 8 adapters rank 16, top-2 pre-gate, 32 tokens/step, uniform, bf16",
+    "prefill": "prefill: same layers, 16 adapters rank 16, top-2, 8192 tokens, Zipf(1.1) popularity, bf16",
+    "multitenant": "multi-tenant: 32 layers q,v 4096->4096, 256 adapters ranks {8,16,32,64}, top-1, "
+                   "4096 tokens uniform, bf16",
+    "merge": "batch-1 merge: 224 decode-shaped weights, top-2 merged W' = W + sum g B A in one launch, "
+             "then one GEMV per weight, bf16",
+    "tiny": "tiny: 4 layers x 256->256, 8 adapters rank 8, top-2, 64 tokens, fp32",
+}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+        return False
+
+    def summary(self):
+        if not self.lines:
+            return None
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in self.lines:
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(value, world):
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- CPU oracle leg
+
+
+class OracleSample:
+    """The fp64 oracle on a bounded sample of one step of ``cfg``.
+
+    Inputs of the first ``n_layers`` layers are prepared once, outside the
+    clock; one pass times the route + segments over all tokens and those
+    layers (every projection, every token), and the step time is scaled to
+    all layers.  BLAS is held to one thread, so ``cores`` is 1.
+    """
+
+    def __init__(self, cfg, layer_budget_s):
+        from adapter_pregate_router_b200 import workloads as W
+        from oracle import apr_oracle as O
+        self.cfg, self.W, self.O = cfg, W, O
+        self.ranks = W.ranks(cfg)
+        self.h, self.Wr, _ = W.router_inputs(cfg)
+        idx, gate, _ = O.pregate_route(self.h, self.Wr, cfg.k)
+        self.sel = set(idx.reshape(-1).tolist())
+        self.layers = [self._prepare(0)]
+        t = self._time_layer(self.layers[0], idx, gate)
+        n = int(max(1, min(cfg.layers, layer_budget_s / max(t, 1e-6))))
+        for l in range(1, n):
+            self.layers.append(self._prepare(l))
+
+    def _prepare(self, l):
+        cfg, W = self.cfg, self.W
+        items = []
+        for g in cfg.groups:
+            if cfg.merge:
+                for p, d_out in zip(g.proj_names, g.d_outs):
+                    Wt = W.host_tensor(cfg, W.w_key(l, g.name, p), (d_out, g.d_in))
+                    A = [W.host_tensor(cfg, W.a_key(l, g.name, p, e), (int(self.ranks[e]), g.d_in))
+                         if e in self.sel else None for e in range(cfg.E)]
+                    B = [W.host_tensor(cfg, W.b_key(l, g.name, p, e), (d_out, int(self.ranks[e])))
+                         if e in self.sel else None for e in range(cfg.E)]
+                    items.append(("merge", Wt, A, B, W.host_tensor(cfg, W.xm_key(l, g.name, p), (g.d_in,))))
+                continue
+            x = W.host_tensor(cfg, W.x_key(l, g.name), (cfg.T, g.d_in))
+            for p, d_out in zip(g.proj_names, g.d_outs):
+                A = [W.host_tensor(cfg, W.a_key(l, g.name, p, e), (int(self.ranks[e]), g.d_in))
+                     if e in self.sel else None for e in range(cfg.E)]
+                B = [W.host_tensor(cfg, W.b_key(l, g.name, p, e), (d_out, int(self.ranks[e])))
+                     if e in self.sel else None for e in range(cfg.E)]
+                yb = W.host_tensor(cfg, W.ybase_key(l, g.name, p), (cfg.T, d_out))
+                items.append(("sgmm", x, A, B, yb))
+        return items
+
+    def _time_layer(self, items, idx, gate):
+        O = self.O
+        t0 = time.perf_counter()
+        for it in items:
+            if it[0] == "merge":
+                _, Wt, A, B, xv = it
+                O.gemv(O.merge_adapters(Wt, A, B, idx[0], gate[0]), xv)
+            else:
+                _, x, A, B, yb = it
+                O.sgmm_shrink_expand(x, A, B, idx, gate, yb)
+        return time.perf_counter() - t0
+
+    def step_seconds(self):
+        from threadpoolctl import threadpool_limits
+        O, cfg = self.O, self.cfg
+        with threadpool_limits(limits=1):
+            t0 = time.perf_counter()
+            idx, gate, _ = O.pregate_route(self.h, self.Wr, cfg.k)
+            O.segment_tokens(idx, cfg.E)
+            t_route = time.perf_counter() - t0
+            t_layers = sum(self._time_layer(items, idx, gate) for items in self.layers)
+        return t_route + t_layers * cfg.layers / len(self.layers)
+
+    def describe(self):
+        c = self.cfg
+        return (f"route+segments over all {c.T} tokens plus {len(self.layers)} of {c.layers} layers "
+                f"(every projection and token) timed, scaled to {c.layers} layers; fp64 numpy oracle, 1 BLAS thread")
+
+
+def cpu_baseline(cfg, budget_s):
+    """Repeat oracle passes for about ``budget_s`` seconds of CPU work."""
+    smp = OracleSample(cfg, layer_budget_s=budget_s / 4)
+    times, spent = [], 0.0
+    while spent < budget_s or not times:
+        t = smp.step_seconds()
+        times.append(t)
+        spent += t * len(smp.layers) / cfg.layers + 1e-3
+        if len(times) >= 50:
+            break
+    step_s = float(np.median(times))
+    return {"value": cfg.T / step_s, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": smp.describe() + f"; median of {len(times)} passes"}
+
+
+def run_reference(args, world, rank):
+    """The reference arm: the fp64 CPU oracle, timed on the host cores."""
+    if rank != 0:
+        return
+    from adapter_pregate_router_b200 import workloads as W
+    cfg = W.CONFIGS[args.workload]
+    per_step_budget = min(args.ref_budget, 150.0 / (args.steps + args.warmup))
+    smp = OracleSample(cfg, layer_budget_s=per_step_budget)
+    for _ in range(args.warmup):
+        smp.step_seconds()
+    per_step = [smp.step_seconds() for _ in range(args.steps)]
+    step_s = float(np.mean(per_step))
+    value = cfg.T / step_s
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_block(cfg, world),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": smp.describe()},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_block(cfg, world):
+    return {"workload": DESCR.get(cfg.name, cfg.name), "name": cfg.name, "tokens_per_step": cfg.T,
+            "adapters": cfg.E, "top_k": cfg.k, "ranks": list(cfg.rank_choices), "layers": cfg.layers,
+            "parallelism": f"replicas x{world} (token batches, no collective)",
+            "l2": "working set larger than the 126 MB L2 (every layer has its own buffers); no flush"}
+
+
+# ---------------------------------------------------------------- GPU leg
+
+
+def run_gpu(args, world, rank, local):
+    import torch
+    from adapter_pregate_router_b200 import apr, pipeline
+    from adapter_pregate_router_b200 import workloads as W
+
+    cfg = W.scaled(W.CONFIGS[args.workload], seed=W.CONFIGS[args.workload].seed + rank)
+    peaks = load_peaks()
+    dev = torch.device("cuda", local)
+    step = pipeline.Step(cfg, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    stream.wait_stream(torch.cuda.current_stream(dev))
+
+    # launches per step (eager, counted by the library)
+    with torch.cuda.stream(stream):
+        before = apr.kernel_launches()
+        step.run()
+        launches = apr.kernel_launches() - before
+    stream.synchronize()
+    apr.stream_status(step.ws, stream)
+
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        step.run()
+        stream.synchronize()
+        with torch.cuda.graph(graph, stream=stream):
+            step.run()
+    layer_graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(layer_graph, stream=stream):
+            step.layers_only()
+    stream.synchronize()
+
+    # ---- warm-up
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            graph.replay()
+    stream.synchronize()
+    apr.stream_status(step.ws, stream)
+
+    # ---- timed region: K whole steps
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        with torch.cuda.stream(stream):
+            ev0.record(stream)
+            for _ in range(args.steps):
+                graph.replay()
+            ev1.record(stream)
+        stream.synchronize()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    ms = ev0.elapsed_time(ev1)
+    ms = max_over_ranks(ms, world)
+    ms_step = ms / args.steps
+    tokens_total = cfg.T * args.steps * world
+    value = tokens_total / (ms / 1e3)
+    apr.stream_status(step.ws, stream)
+
+    # ---- the dominant kernel class timed alone (every layer call, no route)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            layer_graph.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        nrep = max(10, min(args.steps, 500))
+        for _ in range(nrep):
+            layer_graph.replay()
+        e1.record(stream)
+    stream.synchronize()
+    layer_ms = e0.elapsed_time(e1) / nrep
+    idx_np = step.idx.cpu().numpy()
+    step_bytes = step.algorithmic_bytes(idx_np)
+    router_bytes = cfg.T * cfg.d_router * (2 if cfg.dtype == "bf16" else 4) + cfg.E * cfg.d_router * (
+        2 if cfg.dtype == "bf16" else 4)
+    layer_bytes = step_bytes - router_bytes
+    ncalls = len(step.calls) if not cfg.merge else 1 + step.nmerge
+    achieved_gbs = layer_bytes / (layer_ms * 1e-3) / 1e9
+    roof = {
+        "bound": "hbm", "kernel": "apr_sgmm_shrink_expand (shrink+expand launches of every layer call)",
+        "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+        "frac": achieved_gbs / peaks["hbm_gbs"], "peak_source": f"{peaks['source']} copy bandwidth",
+        "traffic": None, "bytes_per_call": layer_bytes / ncalls, "calls_per_step": ncalls,
+        "us_per_call": layer_ms * 1e3 / ncalls, "step_bytes": step_bytes,
+        "step_frac": step_bytes / (ms_step * 1e-3) / 1e9 / peaks["hbm_gbs"],
+    }
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not cfg.merge:
+        host_in = torch.empty(step.act_in.numel(), dtype=step.act_in.dtype, pin_memory=True)
+        host_out = torch.empty(step.act_out.numel(), dtype=step.act_out.dtype, pin_memory=True)
+        host_in.copy_(step.act_in)
+        ke = max(3, min(args.steps, 50))
+        with torch.cuda.stream(stream):
+            for _ in range(2):
+                step.act_in.copy_(host_in, non_blocking=True)
+                graph.replay()
+                host_out.copy_(step.act_out, non_blocking=True)
+            stream.synchronize()
+            barrier(world)
+            x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            x0.record(stream)
+            for _ in range(ke):
+                step.act_in.copy_(host_in, non_blocking=True)
+                graph.replay()
+                host_out.copy_(step.act_out, non_blocking=True)
+            x1.record(stream)
+        stream.synchronize()
+        e_ms = max_over_ranks(x0.elapsed_time(x1), world)
+        e2e = {"value": cfg.T * ke * world / (e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": host_in.numel() * host_in.element_size(),
+               "d2h_bytes_per_step": host_out.numel() * host_out.element_size(),
+               "steps": ke, "ms_per_step": e_ms / ke}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(W.CONFIGS[args.workload], budget_s=args.ref_budget)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if cfg.dtype == "bf16" else "f32", "data": "synthetic",
+        "config": config_block(cfg, world), "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+        "clocks": clk.summary(), "gpu_launches": launches * args.steps,
+        "launches_per_step": launches,
+    }
+    graph.reset()
+    layer_graph.reset()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "multitenant", "merge", "tiny"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--ref-budget", type=float, default=12.0, help="seconds of oracle work per reference step")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, world, rank)
+        return
+    world, rank, local = dist_setup(args)
+    try:
+        run_gpu(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

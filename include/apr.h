@@ -1,0 +1,205 @@
+/*
+ * apr.h -- C ABI of libapr: token-level pre-gated mixture-of-LoRA with a
+ * segmented gather product (SGMM), for NVIDIA B200 (sm_100a).
+ *
+ * The operations follow the AdaFuse summary ("AdaFuse: Accelerating Dynamic
+ * Adapter Inference via Token-Level Pre-Gating and Fused Kernel
+ * Optimization", gist.science, Resumen tecnico):
+ *   - section 2.A: one light router, run once per token at the first adapted
+ *     layer, fixes the adapters of every later layer of that token;
+ *   - section 2.B, decoding steps 1-2: one router pass, top-K selection;
+ *   - section 2.B, SGMM: one batched product over the tokens gathered per
+ *     adapter applies (fuses) the selected adapters in a single kernel call;
+ *   - section 2.B, steps 3-5: merge the selected adapters into the backbone,
+ *     run the base model, unmerge for the next token.
+ *
+ * Conventions (all entry points):
+ *   - Every buffer belongs to the caller.  The library never allocates or
+ *     frees device memory.  Pointers named "device" must be device (or
+ *     managed) memory of the current device; "host" pointers are read before
+ *     the call returns.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL is the legacy default stream).  Host-side argument checks happen
+ *     before anything is launched and return an error status with nothing
+ *     enqueued.  Faults the device detects (an adapter index out of range, a
+ *     rank above the declared maximum) set an error word in the workspace
+ *     and the offending rows are skipped; they never trap.  Read and clear
+ *     that word with apr_stream_status().
+ *   - Kernels are launched with programmatic dependent launch allowed: each
+ *     waits for its predecessor on the stream before touching any input, so
+ *     stream order is kept; consecutive calls may overlap their launch.
+ *   - Layouts are row-major and dense.  Element type is given by `dtype`
+ *     (APR_F32 or APR_BF16) for activations and adapter weights; router
+ *     logits are accumulated and gates are produced in fp32.
+ *   - Device pointers to activations and weights must be 16-byte aligned and
+ *     every row length a multiple of 8 elements.
+ *   - No C++ exception crosses this boundary.  apr_last_error() returns a
+ *     thread-local description of the last failure.
+ */
+#ifndef APR_H_
+#define APR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum apr_status {
+  APR_OK = 0,
+  APR_ERR_INVALID_ARG = 1,  /* a host-checkable argument is wrong            */
+  APR_ERR_UNSUPPORTED = 2,  /* valid but outside this build's limits         */
+  APR_ERR_WORKSPACE = 3,    /* workspace missing, misaligned or too small    */
+  APR_ERR_CUDA = 4,         /* a CUDA runtime call failed                     */
+  APR_ERR_DEVICE_INDEX = 5, /* device saw an adapter index/rank out of range */
+  APR_ERR_TIMEOUT = 6       /* a bounded device-side wait gave up            */
+} apr_status;
+
+typedef enum apr_dtype { APR_F32 = 0, APR_BF16 = 1 } apr_dtype;
+
+/* Limits of this build. */
+#define APR_MAX_E 1024        /* adapters                                   */
+#define APR_MAX_K 8           /* adapters per token                         */
+#define APR_MAX_RANK 128      /* LoRA rank, a multiple of 8                 */
+#define APR_MAX_PROJ 4        /* projections sharing one input per SGMM call */
+
+/* Kernel choice for apr_sgmm_shrink_expand. */
+typedef enum apr_sgmm_kernel {
+  APR_SGMM_AUTO = 0,    /* by the mean segment size T*k/E (known on the host) */
+  APR_SGMM_SKINNY = 1,  /* CUDA-core kernel for few tokens per adapter        */
+  APR_SGMM_TENSOR = 2   /* tcgen05 tensor-core kernel for long segments       */
+} apr_sgmm_kernel;
+
+/* ------------------------------------------------------------------------
+ * Workspace.  One device buffer of apr_workspace_size() bytes, 256-byte
+ * aligned, serves a whole step: apr_pregate_route uses it as scratch,
+ * apr_segment_tokens writes the routing plan into it, and every
+ * apr_sgmm_shrink_expand of the step reads that plan (so it must be the same
+ * buffer, untouched in between).  It starts with an error word: zero it once
+ * with apr_workspace_init() before first use.  Calls that share a workspace
+ * must be ordered on one stream.
+ *   T, k, E      : largest token count, top-k and adapter count of the step
+ *   max_rank     : largest adapter rank
+ *   max_d_in     : largest SGMM input width
+ * Returns 0 when an argument is out of range.
+ * ---------------------------------------------------------------------- */
+size_t apr_workspace_size(int T, int k, int E, int max_rank, int max_d_in);
+apr_status apr_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Token-level pre-gate (section 2.A; section 2.B steps 1-2).
+ *   L[t,e]   = sum_i h[t,i] * Wr[e,i]           (fp32 accumulation)
+ *   idx[t,:] = the k adapters with the largest L[t,.], in descending order;
+ *              equal logits go to the lower adapter index
+ *   gate[t,j]= exp(L[t,idx[t,j]] - L[t,idx[t,0]]) / sum_j' exp(...)
+ * h        device [T, d]  dtype     router input (hidden state of the token)
+ * Wr       device [E, d]  dtype     router weight
+ * idx      device [T, k]  int32     out
+ * gate     device [T, k]  fp32      out
+ * ws       device workspace (scratch for split-K partial logits)
+ * Limits: 1 <= k <= min(E, APR_MAX_K), E <= APR_MAX_E, d % 8 == 0.  T == 0
+ * is a no-op.  Logits must be finite; sums of products stay exact when the
+ * inputs are small integers scaled by powers of two.
+ * ---------------------------------------------------------------------- */
+apr_status apr_pregate_route(const void* h, const void* Wr, int dtype, int T, int d, int E,
+                             int k, int32_t* idx, float* gate, void* ws, size_t ws_bytes,
+                             void* stream);
+
+/* ------------------------------------------------------------------------
+ * Segments (the "segmented gather" of section 2.B's SGMM).
+ * Pair q = t*k + j belongs to adapter idx[t,j].
+ *   seg_off  device [E+1] int32  out: seg_off[0] = 0, seg_off[e+1]-seg_off[e] =
+ *                                pairs of adapter e (exclusive prefix sum)
+ *   perm     device [T*k] int32  out: pair ids grouped by adapter, ascending
+ *                                q inside each segment (a stable counting sort)
+ * Also writes the routing plan that apr_sgmm_shrink_expand reads from `ws`
+ * (inverse permutation, tokens ordered by adapter set, tile lists).
+ * An index outside [0, E) sets APR_ERR_DEVICE_INDEX in the workspace and
+ * leaves every segment empty.  Deterministic; bit-exact.
+ * ---------------------------------------------------------------------- */
+apr_status apr_segment_tokens(const int32_t* idx, int T, int k, int E, int32_t* seg_off,
+                              int32_t* perm, void* ws, size_t ws_bytes, void* stream);
+
+/* One projection of a shared-input group. */
+typedef struct apr_proj {
+  void* y;                /* device [T, d_out] out; may equal y_base (in place)   */
+  const void* y_base;     /* device [T, d_out] base projection output             */
+  int d_out;              /* output width, a multiple of 8                        */
+  const void* const* A;   /* device array [E] of device pointers, A[e] -> [r_e, d_in] */
+  const void* const* B;   /* device array [E] of device pointers, B[e] -> [d_out, r_e] */
+} apr_proj;
+
+/* ------------------------------------------------------------------------
+ * SGMM shrink/expand fused into the add onto the base output (section 2.B).
+ * For every projection p of the group and every token t:
+ *   y_p[t] = y_base_p[t] + sum_j gate[t,j] * B_e (A_e x[t]),  e = idx[t,j]
+ * with fp32 accumulation and one rounding to dtype per output element.
+ * x        device [T, d_in] dtype, shared by the nproj projections
+ * projs    host   [nproj] (1 <= nproj <= APR_MAX_PROJ)
+ * ranks    device [E] int32, r_e in [8, max_rank], multiples of 8
+ * max_rank host   bound on ranks (multiple of 8, <= APR_MAX_RANK)
+ * idx,gate device [T,k]: the outputs of apr_pregate_route (the same routing
+ *          is reused by every layer, section 2.A)
+ * seg_off,perm device: the outputs of apr_segment_tokens for this idx; `ws`
+ *          must be the workspace that call wrote.
+ * kernel   APR_SGMM_AUTO, or a forced kernel class.  The tensor-core kernel
+ *          needs dtype == APR_BF16, k <= 2, max_rank <= 64, d_in % 64 == 0 and
+ *          d_out % 16 == 0; it returns APR_ERR_UNSUPPORTED otherwise.
+ * T == 0 is a no-op.  Empty segments are legal.
+ * ---------------------------------------------------------------------- */
+apr_status apr_sgmm_shrink_expand(const void* x, int d_in, const apr_proj* projs, int nproj,
+                                  int dtype, int T, int k, int E, const int32_t* ranks,
+                                  int max_rank, const int32_t* idx, const float* gate,
+                                  const int32_t* seg_off, const int32_t* perm, void* ws,
+                                  size_t ws_bytes, int kernel, void* stream);
+
+/* One weight of the merge step. */
+typedef struct apr_merge_proj {
+  const void* W;          /* device [d_out, d_in] bf16 base weight (never written) */
+  void* Wp;               /* device [d_out, d_in] bf16 merged weight, out         */
+  int d_in, d_out;        /* multiples of 8                                       */
+  const void* const* A;   /* device array [E] of device pointers, A[e] -> [r, d_in]  */
+  const void* const* B;   /* device array [E] of device pointers, B[e] -> [d_out, r] */
+} apr_merge_proj;
+
+/* ------------------------------------------------------------------------
+ * Batch-1 merge (section 2.B steps 3 and 5), all weights in ONE launch:
+ *   Wp = W + sum_j gate[j] * B_{idx[j]} A_{idx[j]}
+ * written out of place, so W is never modified and unmerging is free.
+ * projs    device [nproj] apr_merge_proj
+ * r        rank shared by the merged adapters (multiple of 8, <= 64)
+ * idx,gate device [k]: one token's pre-gate (row 0 of apr_pregate_route)
+ * fp32 accumulation, one rounding to bf16 per element.
+ * ---------------------------------------------------------------------- */
+apr_status apr_merge_adapters(const apr_merge_proj* projs, int nproj, int E, int r,
+                              const int32_t* idx, const float* gate, int k, void* ws,
+                              size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Base inference on the merged weight (section 2.B step 4): y = W x.
+ * W device [d_out, d_in] bf16, x device [d_in] bf16, y device [d_out] bf16.
+ * fp32 accumulation, one rounding per output.
+ * ---------------------------------------------------------------------- */
+apr_status apr_gemv(const void* W, const void* x, void* y, int d_in, int d_out, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Status plumbing.
+ * apr_stream_status: synchronizes `stream`, then reads and clears the device
+ *   error word of `ws`; returns APR_OK, the first device-side error recorded
+ *   since the last call, or APR_ERR_CUDA if the stream itself failed.
+ * apr_last_error: thread-local text of the last non-OK status of this thread.
+ * apr_status_string: fixed name of a status code.
+ * apr_kernel_launches: number of kernels this library has launched in the
+ *   process (all threads), for accounting.
+ * ---------------------------------------------------------------------- */
+apr_status apr_stream_status(void* ws, void* stream);
+const char* apr_last_error(void);
+const char* apr_status_string(int status);
+uint64_t apr_kernel_launches(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* APR_H_ */

@@ -1,0 +1,118 @@
+"""The C ABI library: it builds, loads without a GPU, exports every declared
+symbol, and rejects bad arguments on the host before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def apr():
+    from adapter_pregate_router_b200 import build
+    build.build()
+    from adapter_pregate_router_b200 import apr as mod
+    return mod
+
+
+def declared_symbols():
+    names = []
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if not h.endswith(".h"):
+            continue
+        text = open(os.path.join(ROOT, "include", h)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names += re.findall(r"\b(apr_[a-z0-9_]+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(apr):
+    lib = ctypes.CDLL(apr.LIB_PATH)
+    names = declared_symbols()
+    assert "apr_sgmm_shrink_expand" in names and "apr_pregate_route" in names
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+    assert set(apr.EXPORTED) <= set(names)
+
+
+def test_library_has_no_libcuda_dependency(apr):
+    import subprocess
+    out = subprocess.run(["ldd", apr.LIB_PATH], capture_output=True, text=True).stdout
+    assert "libcuda.so" not in out and "libcudart.so" not in out
+
+
+def test_workspace_size(apr):
+    assert apr.workspace_size(32, 2, 8, 16, 11008) > 0
+    assert apr.workspace_size(32, 2, 8, 12, 4096) == 0          # rank not a multiple of 8
+    assert apr.workspace_size(32, 9, 16, 16, 4096) == 0          # k > 8
+    assert apr.workspace_size(32, 2, 2048, 16, 4096) == 0        # E too large
+    a = apr.workspace_size(8192, 2, 16, 16, 11008)
+    b = apr.workspace_size(8192, 2, 16, 64, 11008)
+    assert b > a
+
+
+def test_status_strings(apr):
+    assert apr.status_string(0) == "APR_OK"
+    assert apr.status_string(5) == "APR_ERR_DEVICE_INDEX"
+    assert apr.status_string(99) == "APR_ERR_UNKNOWN"
+
+
+def _route(apr, **kw):
+    args = dict(h=0x1000, Wr=0x1000, dtype=1, T=4, d=64, E=8, k=2, idx=0x1000, gate=0x1000,
+                ws=0x100000, ws_bytes=1 << 30, stream=None)
+    args.update(kw)
+    return apr._pregate_route(*args.values())
+
+
+def test_route_host_validation(apr):
+    assert _route(apr, k=9) == apr.APR_ERR_INVALID_ARG
+    assert _route(apr, k=0) == apr.APR_ERR_INVALID_ARG
+    assert _route(apr, E=4, k=5) == apr.APR_ERR_INVALID_ARG
+    assert _route(apr, E=2000) == apr.APR_ERR_INVALID_ARG
+    assert _route(apr, d=60) == apr.APR_ERR_INVALID_ARG
+    assert _route(apr, dtype=7) == apr.APR_ERR_INVALID_ARG
+    assert _route(apr, h=None) == apr.APR_ERR_INVALID_ARG
+    assert _route(apr, h=0x1008) == apr.APR_ERR_INVALID_ARG       # not 16-byte aligned
+    assert _route(apr, ws=None) == apr.APR_ERR_WORKSPACE
+    assert _route(apr, ws=0x100010) == apr.APR_ERR_WORKSPACE      # not 256-byte aligned
+    assert _route(apr, ws_bytes=16) == apr.APR_ERR_WORKSPACE
+    assert _route(apr, T=0, h=None, idx=None) == apr.APR_OK        # empty batch: no-op
+    assert "k=9" in (_route(apr, k=9) and apr.last_error())
+
+
+def test_sgmm_host_validation(apr):
+    P = apr.Proj(0x1000, 0x1000, 64, 0x1000, 0x1000)
+    arr = (apr.Proj * 1)(P)
+
+    def call(**kw):
+        a = dict(x=0x1000, d_in=64, projs=arr, nproj=1, dtype=1, T=4, k=2, E=8, ranks=0x1000,
+                 max_rank=16, idx=0x1000, gate=0x1000, seg_off=0x1000, perm=0x1000, ws=0x100000,
+                 ws_bytes=1 << 30, kernel=0, stream=None)
+        a.update(kw)
+        return apr._sgmm(*a.values())
+
+    assert call(nproj=0) == apr.APR_ERR_INVALID_ARG
+    assert call(nproj=5) == apr.APR_ERR_INVALID_ARG
+    assert call(max_rank=12) == apr.APR_ERR_INVALID_ARG
+    assert call(max_rank=136) == apr.APR_ERR_INVALID_ARG
+    assert call(d_in=20) == apr.APR_ERR_INVALID_ARG
+    assert call(kernel=3) == apr.APR_ERR_INVALID_ARG
+    assert call(x=None) == apr.APR_ERR_INVALID_ARG
+    assert call(ws_bytes=256) == apr.APR_ERR_WORKSPACE
+    bad = (apr.Proj * 1)(apr.Proj(0x1000, 0x1000, 60, 0x1000, 0x1000))
+    assert call(projs=bad) == apr.APR_ERR_INVALID_ARG
+    assert call(T=0) == apr.APR_OK
+    # the tensor-core kernel refuses shapes outside its limits before launching
+    assert call(kernel=2, dtype=0) == apr.APR_ERR_UNSUPPORTED
+
+
+def test_merge_and_gemv_host_validation(apr):
+    assert apr._merge(0x1000, 0, 8, 16, 0x1000, 0x1000, 2, 0x100000, 1 << 20, None) == apr.APR_ERR_INVALID_ARG
+    assert apr._merge(0x1000, 4, 8, 12, 0x1000, 0x1000, 2, 0x100000, 1 << 20, None) == apr.APR_ERR_INVALID_ARG
+    assert apr._merge(0x1000, 4, 8, 64, 0x1000, 0x1000, 2, 0x100000, 1 << 20, None) == apr.APR_ERR_UNSUPPORTED
+    assert apr._merge(0x1000, 4, 8, 16, 0x1000, 0x1000, 2, None, 1 << 20, None) == apr.APR_ERR_WORKSPACE
+    assert apr._gemv(0x1000, 0x1000, 0x1000, 60, 8, None) == apr.APR_ERR_INVALID_ARG
+    assert apr._gemv(0x1000, 0x1000, 0x1000, 64, 0, None) == apr.APR_OK
+    assert apr._gemv(None, 0x1000, 0x1000, 64, 8, None) == apr.APR_ERR_INVALID_ARG

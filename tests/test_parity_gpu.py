@@ -1,0 +1,312 @@
+"""GPU parity: every entry point of the C ABI against the fp64 oracle.
+
+Indices, offsets and permutations must match bit for bit; gates within 1e-6;
+floating outputs within relative Frobenius 5e-3 and max-abs 1e-2*max|ref| per
+tensor; small-integer cases must be exact.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import apr_oracle as O
+from adapter_pregate_router_b200 import workloads as W
+from tests.apr_testlib import (GATE_ATOL, bf16_exact, close, oracle_group, run_route, run_segment,
+                               run_sgmm, to_np)
+
+pytestmark = pytest.mark.gpu
+
+BF16, F32 = torch.bfloat16, torch.float32
+
+
+@pytest.fixture(scope="module")
+def apr():
+    from adapter_pregate_router_b200 import build
+    build.build()
+    from adapter_pregate_router_b200 import apr as mod
+    assert torch.cuda.is_available()
+    return mod
+
+
+# ------------------------------------------------------------------ router
+
+
+@pytest.mark.parametrize("name", ["tiny", "decode", "prefill", "multitenant", "merge"])
+def test_route_configs_bit_exact(apr, name):
+    cfg = W.CONFIGS[name]
+    h, Wr, forced = W.router_inputs(cfg)
+    dt = BF16 if cfg.dtype == "bf16" else F32
+    idx, gate = run_route(apr, h, Wr, cfg.k, dt)
+    ridx, rgate, _ = O.pregate_route(h, Wr, cfg.k)
+    assert np.array_equal(idx, ridx)
+    assert np.abs(gate - rgate).max() <= GATE_ATOL
+    if forced is not None:
+        assert np.array_equal(idx, forced)
+
+
+@pytest.mark.parametrize("E,k,d,T", [(8, 2, 64, 100), (5, 5, 32, 33), (256, 3, 256, 70), (1024, 8, 128, 40),
+                                     (33, 1, 512, 1), (64, 4, 4096, 300)])
+def test_route_ties_and_shapes(apr, E, k, d, T):
+    rng = np.random.default_rng(E + k + d)
+    # few distinct integer values -> many exact ties among logits
+    h = rng.integers(-1, 2, size=(T, d)).astype(np.float32)
+    Wr = rng.integers(-1, 2, size=(E, d)).astype(np.float32)
+    Wr[E // 2] = Wr[0]                         # two identical adapters: always tied
+    for dt in (F32, BF16):
+        idx, gate = run_route(apr, h, Wr, k, dt)
+        ridx, rgate, L = O.pregate_route(h, Wr, k)
+        assert np.array_equal(idx, ridx)
+        assert np.abs(gate - rgate).max() <= GATE_ATOL
+        assert np.allclose(gate.sum(axis=1), 1.0, atol=1e-6)
+
+
+def test_route_equal_logits_give_half_gates(apr):
+    h = np.ones((4, 16), np.float32)
+    Wr = np.zeros((6, 16), np.float32)
+    Wr[2] = 1.0
+    Wr[4] = 1.0
+    idx, gate = run_route(apr, h, Wr, 2, F32)
+    assert idx.tolist() == [[2, 4]] * 4
+    assert np.all(gate == 0.5)
+    idx1, gate1 = run_route(apr, h, Wr, 1, F32)
+    assert idx1.tolist() == [[2]] * 4 and np.all(gate1 == 1.0)
+
+
+# ------------------------------------------------------------------ segments
+
+
+@pytest.mark.parametrize("T,k,E", [(1, 1, 1), (7, 2, 3), (64, 2, 8), (1000, 3, 40), (4096, 1, 256),
+                                   (8192, 2, 16), (333, 8, 1024), (5000, 2, 2)])
+def test_segments_bit_exact(apr, T, k, E):
+    rng = np.random.default_rng(T * 7 + k + E)
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+    seg_off, perm, _ = run_segment(apr, idx, E)
+    rs, rp = O.segment_tokens(idx, E)
+    assert np.array_equal(seg_off, rs)
+    assert np.array_equal(perm, rp)
+
+
+def test_segments_skewed_and_empty(apr):
+    # one adapter takes almost everything, several are empty
+    idx = np.zeros((3000, 1), np.int32)
+    idx[::97] = 5
+    idx[1] = 9
+    seg_off, perm, _ = run_segment(apr, idx, 12)
+    rs, rp = O.segment_tokens(idx, 12)
+    assert np.array_equal(seg_off, rs) and np.array_equal(perm, rp)
+
+
+def test_segment_rejects_out_of_range_index(apr):
+    idx = np.array([[0, 1], [2, 7]], np.int32)
+    T, k, E = 2, 2, 4
+    ws = apr.workspace(T, k, E, 8, 8)
+    d_idx = torch.from_numpy(idx).cuda()
+    seg_off = torch.full((E + 1,), 5, dtype=torch.int32, device="cuda")
+    perm = torch.zeros(4, dtype=torch.int32, device="cuda")
+    apr.segment_tokens(d_idx, E, seg_off, perm, ws)
+    assert apr.raw_stream_status(ws) == apr.APR_ERR_DEVICE_INDEX
+    assert seg_off.cpu().tolist() == [0] * (E + 1)
+    assert apr.raw_stream_status(ws) == apr.APR_OK          # the error word was cleared
+
+
+# ------------------------------------------------------------------ SGMM, explicit cases
+
+
+def _case(rng, T, d_in, d_outs, ranks, k, dist="uniform", pool=None, ints=False):
+    E = len(ranks)
+    if pool is None:
+        pool = np.arange(E)
+    if dist == "uniform":
+        idx = np.stack([rng.choice(pool, size=k, replace=False) for _ in range(T)]).astype(np.int32)
+    else:
+        idx = dist
+    if ints:
+        x = rng.integers(-1, 2, size=(T, d_in)).astype(np.float32)
+        As = [[rng.integers(-1, 2, size=(r, d_in)).astype(np.float32) for r in ranks] for _ in d_outs]
+        Bs = [[rng.integers(-1, 2, size=(d, r)).astype(np.float32) for r in ranks] for d in d_outs]
+        gate = np.full((T, k), 1.0 / k, np.float32)
+        ybs = [rng.integers(-4, 5, size=(T, d)).astype(np.float32) for d in d_outs]
+    else:
+        x = rng.normal(size=(T, d_in)).astype(np.float32)
+        As = [[(0.02 * rng.normal(size=(r, d_in))).astype(np.float32) for r in ranks] for _ in d_outs]
+        Bs = [[(0.02 * rng.normal(size=(d, r))).astype(np.float32) for r in ranks] for d in d_outs]
+        gate = rng.dirichlet(np.ones(k), size=T).astype(np.float32)
+        ybs = [rng.normal(size=(T, d)).astype(np.float32) for d in d_outs]
+    return x, As, Bs, idx, gate, ybs
+
+
+def _rounded(x, As, Bs, ybs):
+    return (bf16_exact(x), [[bf16_exact(a) for a in P] for P in As], [[bf16_exact(b) for b in P] for P in Bs],
+            [bf16_exact(y) for y in ybs])
+
+
+@pytest.mark.parametrize("dtype", [F32, BF16])
+@pytest.mark.parametrize("T,d_in,d_outs,ranks,k", [
+    (64, 256, (256,), (8,) * 8, 2),                       # the tiny shape
+    (32, 4096, (4096, 4096, 4096), (16,) * 8, 2),         # a decode qkv group
+    (37, 1000, (1000, 520), (8, 16, 32, 64, 128, 8), 2),  # ragged widths, every rank
+    (129, 4104, (136,), (16, 24, 40), 1),                 # three column chunks, odd ranks
+    (300, 512, (256,), (16,) * 5, 3),
+    (16, 64, (64,), (8,) * 16, 8),                        # k = 8
+    (1, 2048, (4096,), (16,) * 8, 2),                     # one token
+])
+def test_sgmm_skinny_parity(apr, dtype, T, d_in, d_outs, ranks, k):
+    rng = np.random.default_rng(T + d_in + k)
+    x, As, Bs, idx, gate, ybs = _case(rng, T, d_in, d_outs, ranks, k)
+    if dtype == BF16:
+        x, As, Bs, ybs = _rounded(x, As, Bs, ybs)
+    for zero in (True, False):
+        yb = [np.zeros_like(y) for y in ybs] if zero else ybs
+        got = run_sgmm(apr, x, As, Bs, idx, gate, yb, dtype, kernel=apr.SGMM_SKINNY)
+        ref = oracle_group(x, As, Bs, idx, gate.astype(np.float64), yb)
+        for p in range(len(d_outs)):
+            close(got[p], ref[p], f"proj {p} zero_ybase={zero}")
+
+
+def test_sgmm_adversarial_segments(apr):
+    """Empty, size-1 and 127/128/129-pair segments; one huge segment; ragged T."""
+    rng = np.random.default_rng(5)
+    counts = {1: 1, 2: 127, 3: 128, 4: 129, 5: 2000}
+    idx = np.concatenate([np.full(c, e, np.int32) for e, c in counts.items()])
+    rng.shuffle(idx)
+    idx = idx[:, None]
+    T = idx.shape[0]
+    ranks = (16, 8, 16, 32, 64, 16, 8)           # adapters 0 and 6 are empty
+    x, As, Bs, _, _, ybs = _case(rng, T, 512, (328,), ranks, 1)
+    gate = np.ones((T, 1), np.float32)
+    x, As, Bs, ybs = _rounded(x, As, Bs, ybs)
+    got = run_sgmm(apr, x, As, Bs, idx, gate, ybs, BF16, kernel=apr.SGMM_SKINNY)
+    ref = oracle_group(x, As, Bs, idx, gate.astype(np.float64), ybs)
+    close(got[0], ref[0], "adversarial")
+
+
+def test_sgmm_all_tokens_one_adapter_pair(apr):
+    rng = np.random.default_rng(6)
+    T = 777
+    idx = np.tile(np.array([[3, 1]], np.int32), (T, 1))
+    x, As, Bs, _, gate, ybs = _case(rng, T, 256, (264,), (16,) * 4, 2)
+    x, As, Bs, ybs = _rounded(x, As, Bs, ybs)
+    got = run_sgmm(apr, x, As, Bs, idx, gate, ybs, BF16, kernel=apr.SGMM_SKINNY)
+    close(got[0], oracle_group(x, As, Bs, idx, gate.astype(np.float64), ybs)[0], "one pair")
+
+
+@pytest.mark.parametrize("dtype", [F32, BF16])
+def test_sgmm_integer_inputs_exact(apr, dtype):
+    """Small integers and gates of 1/2: every product and sum is exact in fp32,
+    so the device result must equal the oracle's exact value rounded once to the
+    output type, bit for bit (pins the gather/scatter indexing)."""
+    rng = np.random.default_rng(7)
+    x, As, Bs, idx, gate, ybs = _case(rng, 150, 1000, (72, 40), (8, 16, 8, 24), 2, ints=True)
+    got = run_sgmm(apr, x, As, Bs, idx, gate, ybs, dtype, kernel=apr.SGMM_SKINNY)
+    ref = oracle_group(x, As, Bs, idx, gate.astype(np.float64), ybs)
+    for p in range(2):
+        want = ref[p] if dtype == F32 else bf16_exact(ref[p]).astype(np.float64)
+        assert np.array_equal(got[p], want), f"proj {p}: max diff {np.abs(got[p] - want).max()}"
+
+
+def test_sgmm_zero_B_leaves_base_bit_exact(apr):
+    rng = np.random.default_rng(8)
+    x, As, Bs, idx, gate, ybs = _case(rng, 40, 512, (256,), (16,) * 6, 2)
+    x, As, Bs, ybs = _rounded(x, As, Bs, ybs)
+    Bz = [[np.zeros_like(b) for b in P] for P in Bs]
+    got = run_sgmm(apr, x, As, Bz, idx, gate, ybs, BF16, kernel=apr.SGMM_SKINNY)
+    assert np.array_equal(got[0], ybs[0].astype(np.float64))
+
+
+def test_sgmm_in_place_and_token_order(apr):
+    rng = np.random.default_rng(9)
+    x, As, Bs, idx, gate, ybs = _case(rng, 90, 256, (128,), (16,) * 5, 2)
+    x, As, Bs, ybs = _rounded(x, As, Bs, ybs)
+    a = run_sgmm(apr, x, As, Bs, idx, gate, ybs, BF16, kernel=apr.SGMM_SKINNY, in_place=True)[0]
+    b = run_sgmm(apr, x, As, Bs, idx, gate, ybs, BF16, kernel=apr.SGMM_SKINNY)[0]
+    assert np.array_equal(a, b)
+    p = rng.permutation(90)
+    c = run_sgmm(apr, x[p], As, Bs, idx[p], gate[p], [ybs[0][p]], BF16, kernel=apr.SGMM_SKINNY)[0]
+    assert np.array_equal(c, b[p])                 # the same bits: no order dependence
+
+
+def test_sgmm_deterministic(apr):
+    rng = np.random.default_rng(10)
+    x, As, Bs, idx, gate, ybs = _case(rng, 200, 4096, (512,), (16,) * 8, 2)
+    x, As, Bs, ybs = _rounded(x, As, Bs, ybs)
+    a = run_sgmm(apr, x, As, Bs, idx, gate, ybs, BF16, kernel=apr.SGMM_SKINNY)[0]
+    b = run_sgmm(apr, x, As, Bs, idx, gate, ybs, BF16, kernel=apr.SGMM_SKINNY)[0]
+    assert np.array_equal(a, b)
+
+
+def test_sgmm_device_index_fault_is_reported(apr):
+    """A rank above the declared maximum is caught on the device: error word, no trap."""
+    rng = np.random.default_rng(11)
+    x, As, Bs, idx, gate, ybs = _case(rng, 20, 256, (128,), (16, 16, 32), 2)
+    x, As, Bs, ybs = _rounded(x, As, Bs, ybs)
+    with pytest.raises(apr.AprError) as ei:
+        run_sgmm(apr, x, As, Bs, idx, gate, ybs, BF16, kernel=apr.SGMM_SKINNY, max_rank=16)
+    assert ei.value.status == apr.APR_ERR_DEVICE_INDEX
+    # the context is still usable afterwards
+    ok = run_sgmm(apr, x, As, Bs, idx, gate, ybs, BF16, kernel=apr.SGMM_SKINNY)
+    close(ok[0], oracle_group(x, As, Bs, idx, gate.astype(np.float64), ybs)[0], "after fault")
+
+
+# ------------------------------------------------------------------ merge and GEMV
+
+
+def test_merge_and_gemv_small(apr):
+    rng = np.random.default_rng(12)
+    E, r, k = 5, 16, 2
+    shapes = [(264, 136), (40, 1000), (1000, 64)]
+    Ws = [bf16_exact(0.02 * rng.normal(size=s)) for s in shapes]
+    As = [[bf16_exact(0.02 * rng.normal(size=(r, s[1]))) for _ in range(E)] for s in shapes]
+    Bs = [[bf16_exact(0.02 * rng.normal(size=(s[0], r))) for _ in range(E)] for s in shapes]
+    xs = [bf16_exact(rng.normal(size=s[1])) for s in shapes]
+    idx1 = np.array([3, 1], np.int32)
+    g1 = np.array([0.625, 0.375], np.float32)
+    dW = [torch.from_numpy(w).cuda().to(BF16) for w in Ws]
+    dWp = [torch.full_like(w, float("nan")) for w in dW]
+    keep = []
+    entries = []
+    for p in range(len(shapes)):
+        A = [torch.from_numpy(a).cuda().to(BF16) for a in As[p]]
+        B = [torch.from_numpy(b).cuda().to(BF16) for b in Bs[p]]
+        At, Bt = apr.ptr_array(A), apr.ptr_array(B)
+        keep += [A, B, At, Bt]
+        entries.append((dW[p], dWp[p], At, Bt))
+    tab = apr.merge_table(entries)
+    ws = apr.workspace(1, k, E, r, 8)
+    apr.merge_adapters(tab, len(shapes), E, r, torch.from_numpy(idx1).cuda(), torch.from_numpy(g1).cuda(), k, ws)
+    ys = []
+    for p in range(len(shapes)):
+        y = torch.empty(shapes[p][0], dtype=BF16, device="cuda")
+        apr.gemv(dWp[p], torch.from_numpy(xs[p]).cuda().to(BF16), y)
+        ys.append(y)
+    apr.stream_status(ws)
+    for p in range(len(shapes)):
+        ref = O.merge_adapters(Ws[p], As[p], Bs[p], idx1, g1.astype(np.float64))
+        close(to_np(dWp[p]), ref, f"merged weight {p}")
+        close(to_np(ys[p]), O.gemv(ref, xs[p]), f"gemv {p}")
+
+
+def test_merge_zero_B_is_bit_exact_copy(apr):
+    rng = np.random.default_rng(13)
+    E, r = 3, 16
+    Wt = bf16_exact(0.02 * rng.normal(size=(96, 512)))
+    A = [torch.from_numpy(bf16_exact(rng.normal(size=(r, 512)))).cuda().to(BF16) for _ in range(E)]
+    B = [torch.zeros((96, r), dtype=BF16, device="cuda") for _ in range(E)]
+    At, Bt = apr.ptr_array(A), apr.ptr_array(B)
+    dW = torch.from_numpy(Wt).cuda().to(BF16)
+    dWp = torch.empty_like(dW)
+    tab = apr.merge_table([(dW, dWp, At, Bt)])
+    ws = apr.workspace(1, 2, E, r, 8)
+    apr.merge_adapters(tab, 1, E, r, torch.tensor([2, 0], dtype=torch.int32, device="cuda"),
+                       torch.tensor([0.7, 0.3], dtype=torch.float32, device="cuda"), 2, ws)
+    apr.stream_status(ws)
+    assert torch.equal(dWp, dW)
+
+
+@pytest.mark.parametrize("d_out,d_in", [(4096, 4096), (11008, 4096), (4096, 11008), (37, 72)])
+def test_gemv_parity(apr, d_out, d_in):
+    rng = np.random.default_rng(d_out + d_in)
+    Wt = bf16_exact(0.02 * rng.normal(size=(d_out, d_in)))
+    x = bf16_exact(rng.normal(size=d_in))
+    y = torch.empty(d_out, dtype=BF16, device="cuda")
+    apr.gemv(torch.from_numpy(Wt).cuda().to(BF16), torch.from_numpy(x).cuda().to(BF16), y)
+    torch.cuda.synchronize()
+    close(to_np(y), O.gemv(Wt, x), "gemv")

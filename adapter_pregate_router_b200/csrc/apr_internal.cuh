@@ -17,7 +17,7 @@ namespace apr {
 constexpr size_t kAlign = 256;
 constexpr int kPairTile = 32;       // pairs per shrink tile of the skinny kernel
 constexpr int kSetTile = 128;       // tokens per tensor-core tile (one adapter set)
-constexpr int kShrinkKC = 2048;     // input columns per skinny shrink item
+constexpr int kShrinkKC = 1024;     // input columns per skinny shrink item (128 threads x 8)
 constexpr int kRouteKC = 256;       // minimum router split-K chunk
 
 struct WsHeader {
@@ -76,8 +76,9 @@ inline size_t route_scratch_bytes(int T, int E) {
 
 inline int shrink_kchunks(int d_in) { return (d_in + kShrinkKC - 1) / kShrinkKC; }
 
+// Shrink partial sums: [projection][column chunk][sorted pair][rank] fp32.
 inline size_t sgmm_scratch_bytes(int T, int k, int max_rank, int d_in) {
-  return sizeof(float) * (size_t)shrink_kchunks(d_in) * T * k * max_rank;
+  return sizeof(float) * APR_MAX_PROJ * (size_t)shrink_kchunks(d_in) * T * k * max_rank;
 }
 
 template <typename P>
@@ -156,6 +157,16 @@ __device__ __forceinline__ void store8(float* p, const float (&f)[8]) {
   reinterpret_cast<float4*>(p)[0] = make_float4(f[0], f[1], f[2], f[3]);
   reinterpret_cast<float4*>(p)[1] = make_float4(f[4], f[5], f[6], f[7]);
 }
+
+// Asynchronous 16-byte global -> shared copies (L2 only), grouped and awaited.
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 // Kernel ids used in WsHeader::err_info.
 enum KernelId { K_ROUTE = 1, K_TOPK = 2, K_SEGMENT = 3, K_SHRINK = 4, K_EXPAND = 5, K_MERGE = 6, K_TC = 7 };

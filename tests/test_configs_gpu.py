@@ -90,6 +90,9 @@ def test_config_parity(mods, name, nrows):
 
 
 def test_config_parity_merge(mods):
+    """Merged weights on sampled rows for every weight; for two full layers the
+    whole merged weight and the whole GEMV output (the merged path rounds W'
+    to bf16 before the GEMV, so the GEMV is judged over its full output)."""
     apr, pipeline = mods
     cfg = W.CONFIGS["merge"]
     step = pipeline.Step(cfg)
@@ -99,9 +102,10 @@ def test_config_parity_merge(mods):
     ranks = W.ranks(cfg)
     e_sel = ridx[0]
     rng = np.random.default_rng(3)
+    full_layers = {0, 25}
     for (l, g, p), (Wt, Wp, x, y) in step.weights.items():
         d_out, d_in = Wt.shape
-        rows = np.sort(rng.choice(d_out, size=8, replace=False))
+        rows = np.arange(d_out) if l in full_layers else np.sort(rng.choice(d_out, size=8, replace=False))
         Wr_rows = W.host_rows(cfg, W.w_key(l, g, p), (d_out, d_in), rows)
         A = {e: W.host_tensor(cfg, W.a_key(l, g, p, e), (int(ranks[e]), d_in)) for e in e_sel}
         Bfull = {e: W.host_tensor(cfg, W.b_key(l, g, p, e), (d_out, int(ranks[e]))) for e in e_sel}
@@ -110,8 +114,9 @@ def test_config_parity_merge(mods):
         ref_rows = O.merge_adapters(Wr_rows, Al, Bl, e_sel, rgate[0])
         got = to_np(Wp[torch.from_numpy(rows).to(Wp.device)])
         close(got, ref_rows, f"merged {l}/{p}")
-        xv = W.host_tensor(cfg, W.xm_key(l, g, p), (d_in,))
-        close(to_np(y[torch.from_numpy(rows).to(y.device)]), O.gemv(ref_rows, xv), f"gemv {l}/{p}")
+        if l in full_layers:
+            xv = W.host_tensor(cfg, W.xm_key(l, g, p), (d_in,))
+            close(to_np(y), O.gemv(ref_rows, xv), f"gemv {l}/{p}")
 
 
 def test_graph_replay_matches_eager(mods):

@@ -310,3 +310,66 @@ def test_gemv_parity(apr, d_out, d_in):
     apr.gemv(torch.from_numpy(Wt).cuda().to(BF16), torch.from_numpy(x).cuda().to(BF16), y)
     torch.cuda.synchronize()
     close(to_np(y), O.gemv(Wt, x), "gemv")
+
+
+# ------------------------------------------------------------------ SGMM, tensor-core kernel
+
+
+def _zipf_idx(rng, T, E, k, s=1.1):
+    p = 1.0 / np.arange(1, E + 1) ** s
+    p /= p.sum()
+    return np.stack([rng.choice(E, size=k, replace=False, p=p) for _ in range(T)]).astype(np.int32)
+
+
+@pytest.mark.parametrize("T,d_in,d_outs,ranks,k,zipf", [
+    (300, 512, (256,), (16,) * 4, 2, False),               # many small sets, partial tiles
+    (1000, 1024, (512, 1008), (16,) * 6, 2, True),         # sets longer than one tile, ragged d_out
+    (700, 256, (128,), (8, 16, 32, 64), 1, False),         # top-1, every rank up to 64
+    (517, 4096, (4096,), (16,) * 16, 2, True),             # prefill-shaped projection
+    (129, 192, (64, 64, 64, 64), (32,) * 3, 2, False),     # four projections, k * rank = 64
+    (1, 128, (16,), (16, 16), 2, False),                   # one token
+])
+def test_sgmm_tensor_parity(apr, T, d_in, d_outs, ranks, k, zipf):
+    rng = np.random.default_rng(T + d_in + k + 1)
+    idx = _zipf_idx(rng, T, len(ranks), k) if zipf else "uniform"
+    x, As, Bs, idx, gate, ybs = _case(rng, T, d_in, d_outs, ranks, k, dist=idx)
+    x, As, Bs, ybs = _rounded(x, As, Bs, ybs)
+    for zero in (True, False):
+        yb = [np.zeros_like(y) for y in ybs] if zero else ybs
+        got = run_sgmm(apr, x, As, Bs, idx, gate, yb, BF16, kernel=apr.SGMM_TENSOR)
+        ref = oracle_group(x, As, Bs, idx, gate.astype(np.float64), yb)
+        for p in range(len(d_outs)):
+            close(got[p], ref[p], f"tensor proj {p} zero_ybase={zero}")
+
+
+def test_sgmm_tensor_integer_inputs_exact(apr):
+    """Small integers, gates of 1/2: the tensor-core result is the exact value
+    rounded once to bf16."""
+    rng = np.random.default_rng(21)
+    x, As, Bs, idx, gate, ybs = _case(rng, 400, 512, (128, 256), (16, 16, 16, 16, 16), 2, ints=True)
+    got = run_sgmm(apr, x, As, Bs, idx, gate, ybs, BF16, kernel=apr.SGMM_TENSOR)
+    ref = oracle_group(x, As, Bs, idx, gate.astype(np.float64), ybs)
+    for p in range(2):
+        want = bf16_exact(ref[p]).astype(np.float64)
+        assert np.array_equal(got[p], want), f"proj {p}: max diff {np.abs(got[p] - want).max()}"
+
+
+def test_sgmm_tensor_matches_skinny(apr):
+    rng = np.random.default_rng(22)
+    idx = _zipf_idx(rng, 2000, 8, 2)
+    x, As, Bs, idx, gate, ybs = _case(rng, 2000, 1024, (512,), (16,) * 8, 2, dist=idx)
+    x, As, Bs, ybs = _rounded(x, As, Bs, ybs)
+    a = run_sgmm(apr, x, As, Bs, idx, gate, ybs, BF16, kernel=apr.SGMM_TENSOR)[0]
+    b = run_sgmm(apr, x, As, Bs, idx, gate, ybs, BF16, kernel=apr.SGMM_SKINNY)[0]
+    # both within one bf16 rounding of each other almost everywhere
+    assert np.mean(a == b) > 0.95
+    close(a, b, "tensor vs skinny")
+
+
+def test_sgmm_tensor_rejects_unsupported(apr):
+    rng = np.random.default_rng(23)
+    x, As, Bs, idx, gate, ybs = _case(rng, 50, 100 * 8, (64,), (16,) * 4, 2)   # d_in % 64 != 0
+    x, As, Bs, ybs = _rounded(x, As, Bs, ybs)
+    with pytest.raises(apr.AprError) as ei:
+        run_sgmm(apr, x, As, Bs, idx, gate, ybs, BF16, kernel=apr.SGMM_TENSOR)
+    assert ei.value.status == apr.APR_ERR_UNSUPPORTED

@@ -72,6 +72,7 @@ def _sig(name, res, args):
 _workspace_size = _sig("apr_workspace_size", _sz, [_i, _i, _i, _i, _i])
 _workspace_init = _sig("apr_workspace_init", _i, [_vp, _sz, _vp])
 _pregate_route = _sig("apr_pregate_route", _i, [_vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _sz, _vp])
+_pregate_route_noalloc = _sig("apr_pregate_route_noalloc", _i, [_vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp])
 _segment_tokens = _sig("apr_segment_tokens", _i, [_vp, _i, _i, _i, _vp, _vp, _vp, _sz, _vp])
 _sgmm = _sig("apr_sgmm_shrink_expand", _i,
              [_vp, _i, ctypes.POINTER(Proj), _i, _i, _i, _i, _i, _vp, _i, _vp, _vp, _vp, _vp, _vp, _sz, _i, _vp])
@@ -82,7 +83,8 @@ _last_error = _sig("apr_last_error", ctypes.c_char_p, [])
 _status_string = _sig("apr_status_string", ctypes.c_char_p, [_i])
 _kernel_launches = _sig("apr_kernel_launches", ctypes.c_uint64, [])
 
-EXPORTED = ("apr_workspace_size", "apr_workspace_init", "apr_pregate_route", "apr_segment_tokens",
+EXPORTED = ("apr_workspace_size", "apr_workspace_init", "apr_pregate_route", "apr_pregate_route_noalloc",
+            "apr_segment_tokens",
             "apr_sgmm_shrink_expand", "apr_merge_adapters", "apr_gemv", "apr_stream_status",
             "apr_last_error", "apr_status_string", "apr_kernel_launches")
 
@@ -153,6 +155,14 @@ def pregate_route(h, Wr, k, idx, gate, ws, stream=None):
     E = Wr.shape[0]
     _check(_pregate_route(_ptr(h), _ptr(Wr), _dtype_code(h), T, d, E, k, _ptr(idx), _ptr(gate),
                           _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def pregate_route_noalloc(h, Wr, k, idx, gate, stream=None):
+    """``pregate_route`` for callers that cannot allocate a workspace (library-owned scratch)."""
+    T, d = h.shape
+    E = Wr.shape[0]
+    _check(_pregate_route_noalloc(_ptr(h), _ptr(Wr), _dtype_code(h), T, d, E, k, _ptr(idx), _ptr(gate),
+                                  _stream(stream)))
 
 
 def segment_tokens(idx, E, seg_off, perm, ws, stream=None):

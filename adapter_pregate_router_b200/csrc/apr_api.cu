@@ -99,6 +99,23 @@ apr_status apr_pregate_route(const void* h, const void* Wr, int dtype, int T, in
   return APR_OK;
 }
 
+apr_status apr_pregate_route_noalloc(const void* h, const void* Wr, int dtype, int T, int d, int E,
+                                     int k, int32_t* idx, float* gate, void* stream) {
+  apr_status st = check_route_dims(T, k, E, "pregate_route_noalloc");
+  if (st) return st;
+  if (dtype != APR_F32 && dtype != APR_BF16) return fail(APR_ERR_INVALID_ARG, "pregate_route_noalloc: bad dtype %d", dtype);
+  if (d < 8 || (d & 7)) return fail(APR_ERR_INVALID_ARG, "pregate_route_noalloc: d=%d must be a positive multiple of 8", d);
+  if (T == 0) return APR_OK;
+  if (!h || !Wr || !idx || !gate) return fail(APR_ERR_INVALID_ARG, "pregate_route_noalloc: NULL pointer");
+  if (!aligned16(h) || !aligned16(Wr)) return fail(APR_ERR_INVALID_ARG, "pregate_route_noalloc: h/Wr not 16-byte aligned");
+  if ((size_t)T * E > route_noalloc_capacity_floats())
+    return fail(APR_ERR_UNSUPPORTED, "pregate_route_noalloc: T*E=%zu exceeds the fixed scratch (%zu)",
+                (size_t)T * E, route_noalloc_capacity_floats());
+  cudaError_t e = launch_route_noalloc(h, Wr, dtype, T, d, E, k, idx, gate, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "pregate_route_noalloc launch");
+  return APR_OK;
+}
+
 apr_status apr_segment_tokens(const int32_t* idx, int T, int k, int E, int32_t* seg_off,
                               int32_t* perm, void* ws, size_t ws_bytes, void* stream) {
   apr_status st = check_route_dims(T, k, E, "segment_tokens");

@@ -200,6 +200,9 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
 // Host-side launchers implemented in the kernel translation units.
 cudaError_t launch_route(const void* h, const void* Wr, int dtype, int T, int d, int E, int k,
                          int32_t* idx, float* gate, void* ws, size_t scratch_off, cudaStream_t s);
+cudaError_t launch_route_noalloc(const void* h, const void* Wr, int dtype, int T, int d, int E, int k,
+                                 int32_t* idx, float* gate, cudaStream_t s);
+size_t route_noalloc_capacity_floats();
 cudaError_t launch_segment(const int32_t* idx, int T, int k, int E, int32_t* seg_off,
                            int32_t* perm, void* ws, cudaStream_t s);
 struct ProjArgs {

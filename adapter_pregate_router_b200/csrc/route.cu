@@ -15,6 +15,8 @@
 //                        lower index winning ties, softmax over the k winners.
 #include <math.h>
 
+#include <mutex>
+
 #include "apr_internal.cuh"
 
 namespace apr {
@@ -194,6 +196,86 @@ cudaError_t launch_route(const void* h, const void* Wr, int dtype, int T, int d,
   dim3 g2((T + warps_per_block - 1) / warps_per_block);
   return launch_pdl(route_topk_kernel, g2, dim3(32 * warps_per_block), 0, s, (const float*)part,
                     nch, T, E, k, idx, gate, ws);
+}
+
+
+// ---------------------------------------------------------------- no-allocation variant
+//
+// apr_pregate_route_noalloc serves callers that cannot hand the library a
+// workspace: code with no device allocator of its own (a plug-in whose host
+// application owns every byte of device memory, or a latency-critical loop in
+// which cudaMalloc and the device-wide synchronisation it can cause are not
+// acceptable).  Its scratch is the file-scope array below: a 256-byte header
+// (the device error word) followed by the split-K partial logits of one call.
+// Every GPU that loads the library keeps these 8 MiB until the process exits.
+// All calls share the array, so calls that overlap on the GPU (different
+// streams without ordering) race on it.
+
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;
+constexpr size_t kNoAllocHeaderBytes = 256;
+static __device__ __align__(256) unsigned char g_route_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+static std::mutex g_noalloc_mu;
+static void* g_noalloc_ptr[kMaxDevices];
+
+// Device address of the scratch array on the current device.  Looked up once
+// per device (with that device current) on the first call there.
+static cudaError_t noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    err = cudaGetSymbolAddress(&p, g_route_noalloc_scratch);
+    if (err != cudaSuccess) return err;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return cudaSuccess;
+}
+
+size_t route_noalloc_capacity_floats() { return (kNoAllocScratchBytes - kNoAllocHeaderBytes) / sizeof(float); }
+
+cudaError_t launch_route_noalloc(const void* h, const void* Wr, int dtype, int T, int d, int E, int k,
+                                 int32_t* idx, float* gate, cudaStream_t s) {
+  void* base = nullptr;
+  cudaError_t err = noalloc_scratch(&base);
+  if (err != cudaSuccess) return err;
+  const size_t cap = route_noalloc_capacity_floats();
+  const size_t te = (size_t)T * E;
+  // the error word must start at zero; the partial sums are fully overwritten
+  err = cudaMemsetAsync(base, 0, kNoAllocHeaderBytes, s);
+  if (err != cudaSuccess) return err;
+  const int tiles_t = (T + RT_M - 1) / RT_M;
+  const int tiles_e = (E + RT_N - 1) / RT_N;
+  const int tiles = tiles_t * tiles_e;
+  int nch = (2 * 148 + tiles - 1) / tiles;
+  int by_k = d / kRouteKC;
+  if (by_k < 1) by_k = 1;
+  if (nch > by_k) nch = by_k;
+  if (nch > route_max_chunks(T, E)) nch = route_max_chunks(T, E);
+  if ((size_t)nch * te > cap) nch = (int)(cap / te);
+  if (nch < 1) nch = 1;
+  int chunk = (d + nch - 1) / nch;
+  chunk = (chunk + RT_K - 1) / RT_K * RT_K;
+  nch = (d + chunk - 1) / chunk;
+  float* part = reinterpret_cast<float*>(static_cast<unsigned char*>(base) + kNoAllocHeaderBytes);
+  dim3 grid(tiles_t, tiles_e, nch);
+  if (dtype == APR_BF16) {
+    err = launch_pdl(route_logits_kernel<__nv_bfloat16>, grid, dim3(256), 0, s, (const __nv_bfloat16*)h,
+                     (const __nv_bfloat16*)Wr, T, d, E, chunk, part);
+  } else {
+    err = launch_pdl(route_logits_kernel<float>, grid, dim3(256), 0, s, (const float*)h, (const float*)Wr, T,
+                     d, E, chunk, part);
+  }
+  if (err != cudaSuccess) return err;
+  const int warps_per_block = 8;
+  dim3 g2((T + warps_per_block - 1) / warps_per_block);
+  return launch_pdl(route_topk_kernel, g2, dim3(32 * warps_per_block), 0, s, (const float*)part, nch, T, E, k,
+                    idx, gate, base);
 }
 
 }  // namespace apr

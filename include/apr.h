@@ -107,6 +107,28 @@ apr_status apr_pregate_route(const void* h, const void* Wr, int dtype, int T, in
                              void* stream);
 
 /* ------------------------------------------------------------------------
+ * apr_pregate_route with no workspace: the paper has no counterpart; this is
+ * a convenience of this library.  It exists for callers that cannot allocate
+ * device memory for a workspace -- code without an allocator of its own (a
+ * plug-in whose host application owns every byte of device memory) or a
+ * latency-critical loop in which cudaMalloc and the device-wide
+ * synchronisation it can trigger are not acceptable.
+ * Same arguments (minus the workspace), same results as apr_pregate_route.
+ * Its scratch is one fixed 8 MiB array inside libapr, which every GPU that
+ * loads the library keeps until the process exits; it holds the split-K
+ * partial logits, so T*E must not exceed 2,097,088, else the call returns
+ * APR_ERR_UNSUPPORTED with nothing enqueued.  The first call on a device
+ * looks the array up on that device (cudaGetSymbolAddress); make that first
+ * call before any stream capture.  Every call uses the same array and leaves
+ * its contents behind, so calls that overlap on the GPU (for example on two
+ * streams with no ordering between them) race with each other.  Nothing is
+ * allocated or freed.  A token whose logits are all NaN gets adapter 0; there
+ * is no workspace in which to report that.
+ * ---------------------------------------------------------------------- */
+apr_status apr_pregate_route_noalloc(const void* h, const void* Wr, int dtype, int T, int d, int E,
+                                     int k, int32_t* idx, float* gate, void* stream);
+
+/* ------------------------------------------------------------------------
  * Segments (the "segmented gather" of section 2.B's SGMM).
  * Pair q = t*k + j belongs to adapter idx[t,j].
  *   seg_off  device [E+1] int32  out: seg_off[0] = 0, seg_off[e+1]-seg_off[e] =

@@ -115,7 +115,7 @@ def _case(rng, T, d_in, d_outs, ranks, k, dist="uniform", pool=None, ints=False)
     E = len(ranks)
     if pool is None:
         pool = np.arange(E)
-    if dist == "uniform":
+    if isinstance(dist, str):
         idx = np.stack([rng.choice(pool, size=k, replace=False) for _ in range(T)]).astype(np.int32)
     else:
         idx = dist

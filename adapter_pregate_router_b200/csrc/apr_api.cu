@@ -210,11 +210,14 @@ apr_status apr_merge_adapters(const apr_merge_proj* projs, int nproj, int E, int
   if (E < 1 || E > APR_MAX_E) return fail(APR_ERR_INVALID_ARG, "merge: E=%d outside [1, %d]", E, APR_MAX_E);
   if (k < 1 || k > E || k > APR_MAX_K) return fail(APR_ERR_INVALID_ARG, "merge: k=%d outside [1, min(E, %d)]", k, APR_MAX_K);
   if (r < 8 || (r & 7) || r > APR_MAX_RANK) return fail(APR_ERR_INVALID_ARG, "merge: r=%d must be a multiple of 8 in [8, %d]", r, APR_MAX_RANK);
-  if (!merge_supported(k, r, nproj)) return fail(APR_ERR_UNSUPPORTED, "merge: k*r=%d > 64 or nproj=%d > 4096", k * r, nproj);
+  const bool on_tensor = merge_tensor_supported(k, r, nproj);
+  if (!on_tensor && !merge_supported(k, r, nproj))
+    return fail(APR_ERR_UNSUPPORTED, "merge: k*r=%d > 64 or nproj=%d > 4096", k * r, nproj);
   if (!projs || !idx || !gate) return fail(APR_ERR_INVALID_ARG, "merge: NULL pointer");
   apr_status st = check_ws(ws, ws_bytes, sizeof(WsHeader), "merge");
   if (st) return st;
-  cudaError_t e = launch_merge(projs, nproj, E, r, idx, gate, k, ws, (cudaStream_t)stream);
+  cudaError_t e = on_tensor ? launch_merge_tensor(projs, nproj, E, r, idx, gate, k, ws, (cudaStream_t)stream)
+                            : launch_merge(projs, nproj, E, r, idx, gate, k, ws, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "merge launch");
   return APR_OK;
 }
@@ -239,8 +242,9 @@ apr_status apr_stream_status(void* ws, void* stream) {
   e = cudaMemcpy(words, ws, sizeof(words), cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return cuda_fail(e, "stream_status read");
   if (words[0] != 0) {
-    const int zero[2] = {0, 0};
-    e = cudaMemcpy(ws, zero, sizeof(zero), cudaMemcpyHostToDevice);
+    // clear the error word and the grid-barrier arrivals a failed wait may have left behind
+    e = cudaMemset(ws, 0, 2 * sizeof(int));
+    if (e == cudaSuccess) e = cudaMemset(&reinterpret_cast<WsHeader*>(ws)->bar_count, 0, sizeof(unsigned));
     if (e != cudaSuccess) return cuda_fail(e, "stream_status clear");
     return fail((apr_status)words[0], "device reported %s (kernel %d, value %d)",
                 apr_status_string(words[0]), (words[1] >> 24) & 0xFF, words[1] & 0xFFFFFF);

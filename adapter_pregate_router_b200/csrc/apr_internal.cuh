@@ -17,7 +17,7 @@ namespace apr {
 constexpr size_t kAlign = 256;
 constexpr int kPairTile = 32;       // pairs per shrink tile of the skinny kernel
 constexpr int kSetTile = 128;       // tokens per tensor-core tile (one adapter set)
-constexpr int kShrinkKC = 1024;     // input columns per skinny shrink item (128 threads x 8)
+constexpr int kShrinkKC = 2048;     // input columns per skinny shrink item (256 threads x 8)
 constexpr int kRouteKC = 256;       // minimum router split-K chunk
 
 struct WsHeader {
@@ -26,7 +26,9 @@ struct WsHeader {
   int n_ptiles;     // shrink pair tiles written by the segment kernel
   int n_stiles;     // tensor-core set tiles written by the segment kernel
   int T, k, E;      // routing the plan was built for
-  int pad[57];
+  unsigned bar_count;   // grid barrier of the fused skinny kernel: arrivals
+  unsigned bar_gen;     //   and generation
+  int pad[55];
 };
 static_assert(sizeof(WsHeader) == 256, "header is one alignment unit");
 
@@ -231,6 +233,9 @@ cudaError_t launch_sgmm_tensor(const SgmmArgs& a, cudaStream_t s);
 bool sgmm_tensor_supported(const SgmmArgs& a, int dtype);
 cudaError_t launch_merge(const apr_merge_proj* projs, int nproj, int E, int r, const int32_t* idx,
                          const float* gate, int k, void* ws, cudaStream_t s);
+bool merge_tensor_supported(int k, int r, int nproj);
+cudaError_t launch_merge_tensor(const apr_merge_proj* projs, int nproj, int E, int r, const int32_t* idx,
+                                const float* gate, int k, void* ws, cudaStream_t s);
 cudaError_t launch_gemv(const void* W, const void* x, void* y, int d_in, int d_out, cudaStream_t s);
 
 }  // namespace apr

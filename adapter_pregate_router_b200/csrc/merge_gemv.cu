@@ -10,8 +10,8 @@
 // 4-byte-per-lane coalesced accesses.
 //
 // apr_gemv: y = W x for the merged weight, a streaming HBM-bound kernel: each
-// warp owns 4 rows, 128-bit evict-first loads of W, x staged in shared memory,
-// warp-shuffle reduction.
+// warp owns one row with eight 128-bit evict-first loads of W in flight per
+// lane, x staged in shared memory, warp-shuffle reduction.
 #include "apr_internal.cuh"
 
 namespace apr {
@@ -148,8 +148,10 @@ __global__ void __launch_bounds__(MG_THREADS) merge_kernel(const apr_merge_proj*
 }
 
 constexpr int GV_THREADS = 256;
-constexpr int GV_ROWS_PER_WARP = 4;
+constexpr int GV_UNROLL = 8;     // 16-byte loads of W in flight per lane
 
+// One warp per output row: 8 x 128-bit evict-first loads of W in flight per
+// lane, x from shared memory, warp-shuffle reduction.
 __global__ void __launch_bounds__(GV_THREADS) gemv_kernel(const __nv_bfloat16* __restrict__ W,
                                                           const __nv_bfloat16* __restrict__ x,
                                                           __nv_bfloat16* __restrict__ y, int d_in,
@@ -161,40 +163,36 @@ __global__ void __launch_bounds__(GV_THREADS) gemv_kernel(const __nv_bfloat16* _
     *reinterpret_cast<uint4*>(xs + c) = *reinterpret_cast<const uint4*>(x + c);
   __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int row0 = (blockIdx.x * (GV_THREADS / 32) + warp) * GV_ROWS_PER_WARP;
-  if (row0 >= d_out) return;
-  float acc[GV_ROWS_PER_WARP];
+  const int row = blockIdx.x * (GV_THREADS / 32) + warp;
+  if (row >= d_out) return;
+  const __nv_bfloat16* __restrict__ wr = W + (size_t)row * d_in;
+  float acc = 0.f;
+  for (int c0 = lane * 8; c0 < d_in; c0 += 256 * GV_UNROLL) {
+    uint4 wv[GV_UNROLL];
 #pragma unroll
-  for (int rr = 0; rr < GV_ROWS_PER_WARP; ++rr) acc[rr] = 0.f;
-#pragma unroll 2
-  for (int c = lane * 8; c < d_in; c += 256) {
-    float xv[8];
-    load8(xs + c, xv);
+    for (int u = 0; u < GV_UNROLL; ++u) {
+      const int c = c0 + u * 256;
+      wv[u] = c < d_in ? __ldcs(reinterpret_cast<const uint4*>(wr + c)) : make_uint4(0, 0, 0, 0);
+    }
 #pragma unroll
-    for (int rr = 0; rr < GV_ROWS_PER_WARP; ++rr) {
-      const int n = row0 + rr;
-      if (n < d_out) {
-        float wv[8];
-        load8_stream(W + (size_t)n * d_in + c, wv);
+    for (int u = 0; u < GV_UNROLL; ++u) {
+      const int c = c0 + u * 256;
+      if (c < d_in) {
+        float xv[8];
+        load8(xs + c, xv);
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&wv[u]);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[rr] = fmaf(wv[i], xv[i], acc[rr]);
+        for (int i = 0; i < 4; ++i) {
+          const float2 f = __bfloat1622float2(h[i]);
+          acc = fmaf(f.x, xv[2 * i], acc);
+          acc = fmaf(f.y, xv[2 * i + 1], acc);
+        }
       }
     }
   }
 #pragma unroll
-  for (int rr = 0; rr < GV_ROWS_PER_WARP; ++rr) {
-    float v = acc[rr];
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-    acc[rr] = v;
-  }
-  if (lane < GV_ROWS_PER_WARP && row0 + lane < d_out) {
-    float v = acc[0];
-#pragma unroll
-    for (int rr = 1; rr < GV_ROWS_PER_WARP; ++rr)
-      if (lane == rr) v = acc[rr];
-    y[row0 + lane] = __float2bfloat16_rn(v);
-  }
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (lane == 0) y[row] = __float2bfloat16_rn(acc);
 }
 
 cudaError_t launch_merge(const apr_merge_proj* projs, int nproj, int E, int r, const int32_t* idx,
@@ -208,7 +206,7 @@ cudaError_t launch_merge(const apr_merge_proj* projs, int nproj, int E, int r, c
 }
 
 cudaError_t launch_gemv(const void* W, const void* x, void* y, int d_in, int d_out, cudaStream_t s) {
-  const int rows_per_block = (GV_THREADS / 32) * GV_ROWS_PER_WARP;
+  const int rows_per_block = GV_THREADS / 32;
   const size_t smem = sizeof(__nv_bfloat16) * (size_t)d_in;
   static size_t configured = 0;
   if (smem > 48 * 1024 && smem > configured) {

@@ -7,26 +7,33 @@
 // The routing plan orders tokens by their adapter set; a work item is one
 // set tile (<= 128 tokens that share the same k <= 2 adapters {e0, e1}) and
 // one projection.  Per item, in one CTA of 128 threads (1 CTA per SM, TMEM
-// fully owned):
+// fully owned, persistent over the items):
 //
 //  shrink  D1[128 x N1] = X_tile[128 x d_in] . [A_e0 ; A_e1]^T on tcgen05
 //          (kind::f16, bf16 in, fp32 accumulate in TMEM), N1 = k * R16 where
 //          R16 is the rank rounded up to 16 (zero rows pad the smaller ranks).
-//          The gathered x rows and the A rows are staged with 16-byte cp.async
-//          into 128B-swizzled K-major tiles, 3 stages in flight, one elected
-//          thread issues the MMAs and commits each stage to an mbarrier.
+//          Every thread copies its token's x row and a share of the A rows
+//          with 16-byte cp.async (each warp fetches whole 128-byte row segments)
+//          into 128B-swizzled K-major stages; the copies arrive on the stage's
+//          "full" mbarrier when they land (6 stages in flight, no block
+//          barrier per stage); thread 0 issues the MMAs of a
+//          stage once it is full and commits them to the stage's "empty"
+//          mbarrier, which frees the stage for the next fill.
 //  gate    D1 is read back with tcgen05.ld (one TMEM lane per token), scaled
 //          by the token's gates and split into bf16 hi + lo parts (so the
 //          expand keeps ~16 mantissa bits of v), written to shared memory as
 //          the K-major A operand of the expand.
 //  expand  for every 128-column tile of d_out: D2[128 x 128] = V_hi.Bcat^T +
 //          V_lo.Bcat^T with Bcat[n] = [B_e0[n] | B_e1[n]] (K2 = N1), TMEM
-//          double buffered.  The epilogue adds y_base (fetched with bulk
-//          async copies one tile ahead, completion on an mbarrier), rounds to
-//          bf16 once and writes each token row back with a bulk async store.
+//          double buffered.  Bcat and the y_base rows of a tile are fetched two
+//          tiles ahead with cp.async into 3-deep rings that reuse the shrink
+//          stages' shared memory (each warp loads and stores whole row
+//          segments, 2 rows per instruction); the epilogue adds D2 in its
+//          token's row, rounds to bf16 once, and the warp writes its 32 rows
+//          back with coalesced 128-bit stores.
 //
 // Every mbarrier wait is bounded by the global timer (1 s); on expiry the CTA
-// records APR_ERR_TIMEOUT, drains its own bulk copies and frees its TMEM.
+// records APR_ERR_TIMEOUT, drains its own copies and frees its TMEM.
 #include "apr_internal.cuh"
 
 namespace apr {
@@ -34,26 +41,36 @@ namespace apr {
 constexpr int TC_THREADS = 128;
 constexpr int TC_BM = 128;       // tokens per tile (= kSetTile)
 constexpr int TC_BK = 64;        // input columns per stage (one 128-byte swizzle row)
-constexpr int TC_STAGES = 3;
+constexpr int TC_STAGES = 6;
 constexpr int TC_MAXN1 = 64;     // k * R16
 constexpr int TC_NT = 128;       // output columns per expand tile
+constexpr int TC_NY = 3;         // depth of the Bcat / y_base rings (prefetch distance 2)
 constexpr int TC_YSTRIDE = TC_NT * 2 + 16;   // bytes per staged y row (padding against bank conflicts)
 constexpr uint32_t TC_TMEM_COLS = 512;
 constexpr uint32_t TC_D2_COL = 128;           // D2 buffers at columns 128 and 256
+constexpr int TC_STAGE_BYTES = TC_BM * 128 + TC_MAXN1 * 128;   // x tile + A rows
+constexpr int TC_YBUF_BYTES = TC_BM * TC_YSTRIDE;
+constexpr int TC_BBUF_BYTES = TC_NT * TC_MAXN1 * 2;
 
 struct TcSmem {
-  static constexpr size_t X = 0;                                              // 3 x 16 KB
-  static constexpr size_t A = X + (size_t)TC_STAGES * TC_BM * 128;            // 3 x 8 KB
-  static constexpr size_t VH = A + (size_t)TC_STAGES * TC_MAXN1 * 128;        // 16 KB
+  // the shrink stages and the expand's rings are never live at the same time
+  static constexpr size_t STAGE_AREA = (size_t)TC_STAGES * TC_STAGE_BYTES;
+  static constexpr size_t RING_AREA = (size_t)TC_NY * (TC_YBUF_BYTES + TC_BBUF_BYTES);
+  static constexpr size_t U = 0;
+  static constexpr size_t U_BYTES = STAGE_AREA > RING_AREA ? STAGE_AREA : RING_AREA;
+  static constexpr size_t YR = U;                                             // y ring
+  static constexpr size_t BR = U + (size_t)TC_NY * TC_YBUF_BYTES;             // Bcat ring
+  static constexpr size_t VH = U + (U_BYTES + 1023) / 1024 * 1024;            // 16 KB
   static constexpr size_t VL = VH + (size_t)TC_BM * TC_MAXN1 * 2;             // 16 KB
-  static constexpr size_t BB = VL + (size_t)TC_BM * TC_MAXN1 * 2;             // 2 x 16 KB
-  static constexpr size_t Y = BB + 2 * (size_t)TC_NT * TC_MAXN1 * 2;          // 2 x 34 KB
-  static constexpr size_t BAR = Y + 2 * (size_t)TC_BM * TC_YSTRIDE;           // mbarriers
-  static constexpr size_t META = BAR + 16 * 8;
+  static constexpr size_t BAR = VL + (size_t)TC_BM * TC_MAXN1 * 2;            // mbarriers
+  static constexpr int NBARS = 2 * TC_STAGES + 1 + 2;
+  static constexpr size_t META = BAR + (size_t)NBARS * 8;
   static constexpr size_t TOTAL = META + 3 * TC_BM * 4 + 64;
   static constexpr size_t ALLOC = TOTAL + 1024;                               // for 1024-byte alignment
 };
 static_assert(TcSmem::ALLOC <= 227 * 1024, "shared memory budget");
+static_assert(TC_STAGE_BYTES % 1024 == 0, "stages keep 1024-byte alignment");
+static_assert(TcSmem::BR % 16 == 0 && TC_YBUF_BYTES % 16 == 0, "16-byte aligned rings");
 
 // ---------------------------------------------------------------- PTX wrappers
 
@@ -94,24 +111,18 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
   }
 }
 
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+
+
+
+// 16-byte cp.async; with `valid` false nothing is read and the destination is zero-filled.
+__device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0) : "memory");
 }
 
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-      "l"(src), "r"(bytes), "r"(bar)
-      : "memory");
+// The mbarrier receives one arrival once every cp.async this thread issued so far has landed.
+__device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
-
-__device__ __forceinline__ void bulk_store(void* dst, uint32_t src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -191,28 +202,30 @@ __global__ void __launch_bounds__(TC_THREADS, 1) sgmm_tc_kernel(TcArgs args) {
   const int tid = threadIdx.x, warp = tid >> 5;
   const int K = a.k, R16 = args.R16, N1 = args.N1, K2 = N1;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + TcSmem::BAR);
-  // barriers: [0..2] stage MMA done, [3..4] expand MMA done, [5..6] y_base arrived
-  const uint32_t bar_stage = smem_u32(bars);
-  const uint32_t bar_mma2 = smem_u32(bars + 3);
-  const uint32_t bar_y = smem_u32(bars + 5);
+  // barriers: full[S], empty[S], d1, mma2[2]
+  const uint32_t bar_full = smem_u32(bars);
+  const uint32_t bar_empty = smem_u32(bars + TC_STAGES);
+  const uint32_t bar_d1 = smem_u32(bars + 2 * TC_STAGES);
+  const uint32_t bar_mma2 = smem_u32(bars + 2 * TC_STAGES + 1);
   int* s_tok = reinterpret_cast<int*>(smem + TcSmem::META);
   float* s_g0 = reinterpret_cast<float*>(s_tok + TC_BM);
   float* s_g1 = s_g0 + TC_BM;
-  volatile int* s_flags = reinterpret_cast<volatile int*>(s_g1 + TC_BM);   // [0] tmem base, [1] abort, [2..3] set
-  const uint32_t sX = smem_u32(smem + TcSmem::X);
-  const uint32_t sA = smem_u32(smem + TcSmem::A);
+  volatile int* s_flags = reinterpret_cast<volatile int*>(s_g1 + TC_BM);   // [0] tmem base, [2..3] set
+  const uint32_t sU = smem_u32(smem + TcSmem::U);
   const uint32_t sVH = smem_u32(smem + TcSmem::VH);
   const uint32_t sVL = smem_u32(smem + TcSmem::VL);
-  const uint32_t sB = smem_u32(smem + TcSmem::BB);
-  unsigned char* sYp = smem + TcSmem::Y;
+  unsigned char* sYp = smem + TcSmem::YR;     // rings overlay the stages
   const uint32_t sY = smem_u32(sYp);
+  const uint32_t sB = smem_u32(smem + TcSmem::BR);
 
   if (tid == 0) {
-    for (int i = 0; i < TC_STAGES; ++i) mbar_init(bar_stage + 8 * i, 1);
+    for (int i = 0; i < TC_STAGES; ++i) {
+      mbar_init(bar_full + 8 * i, TC_THREADS);
+      mbar_init(bar_empty + 8 * i, 1);
+    }
+    mbar_init(bar_d1, 1);
     for (int i = 0; i < 2; ++i) mbar_init(bar_mma2 + 8 * i, 1);
-    for (int i = 0; i < 2; ++i) mbar_init(bar_y + 8 * i, TC_THREADS);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    s_flags[1] = 0;
   }
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -241,8 +254,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) sgmm_tc_kernel(TcArgs args) {
   const uint32_t id1 = idesc_bf16(TC_BM, N1);
   const uint32_t id2 = idesc_bf16(TC_BM, TC_NT);
   const uint32_t sbo_v = (uint32_t)(K2 / 8) * 128;   // V and Bcat: next 8-row group
-  uint32_t ph_stage = 0;                              // bit s: parity of stage barrier s
-  uint32_t ph_mma2 = 0, ph_y = 0;
+  uint32_t gchunk = 0;       // shrink chunks issued by this CTA so far (stage = gchunk % S)
+  uint32_t ph_d1 = 0, ph_mma2 = 0;
   bool abort = false;
 
   for (long item = blockIdx.x; item < nitems && !abort; item += gridDim.x) {
@@ -297,62 +310,58 @@ __global__ void __launch_bounds__(TC_THREADS, 1) sgmm_tc_kernel(TcArgs args) {
     const int my_tok = s_tok[tid];
 
     // ------------------------------------------------------------ shrink
-    for (int c = 0; c < nk + TC_STAGES - 1 && !abort; ++c) {
-      if (c < nk && !abort) {
-        const int s = c % TC_STAGES;
-        if (c >= TC_STAGES) {
-          if (!mbar_wait(bar_stage + 8 * s, (ph_stage >> s) & 1)) abort = true;
-          ph_stage ^= 1u << s;
-        }
-        // x row of this thread's token: 8 x 16 bytes into the swizzled row
-        const uint32_t xrow = sX + (uint32_t)s * TC_BM * 128 + (uint32_t)tid * 128;
-        if (my_tok >= 0) {
-          const __nv_bfloat16* src = x + (size_t)my_tok * d_in + (size_t)c * TC_BK;
+    auto consume = [&](uint32_t g, int c) {      // thread 0: MMAs of chunk c (global index g)
+      const uint32_t s = g % TC_STAGES;
+      if (!mbar_wait(bar_full + 8 * s, (g / TC_STAGES) & 1)) { abort = true; return; }
+      tc_fence_after();
+      const uint32_t xs = sU + s * TC_STAGE_BYTES;
+      const uint32_t as = xs + TC_BM * 128;
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(xrow + ((q ^ (tid & 7)) << 4)),
-                         "l"(src + q * 8)
-                         : "memory");
-          }
-        }
-        // A rows: row j of [A_e0 ; A_e1] (rank slots of R16 rows, zero padded)
-        const uint32_t abase = sA + (uint32_t)s * TC_MAXN1 * 128;
-        for (int w = tid; w < N1 * 8; w += TC_THREADS) {
-          const int j = w >> 3, q = w & 7;
-          const int slot = j / R16, r = j % R16;
-          const uint32_t dst = abase + (uint32_t)j * 128 + ((q ^ (j & 7)) << 4);
-          if (r < rk[slot]) {
-            const __nv_bfloat16* src = Aj[slot] + (size_t)r * d_in + (size_t)c * TC_BK + q * 8;
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-          } else {
-            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0) : "memory");
-          }
+      for (int kk = 0; kk < TC_BK / 16; ++kk)
+        mma_bf16(tmem, desc_k_sw128(xs + kk * 32), desc_k_sw128(as + kk * 32), id1, (c > 0 || kk > 0) ? 1u : 0u);
+      mma_commit(bar_empty + 8 * s);
+    };
+    const uint32_t g0 = gchunk;
+    constexpr int LAG = TC_STAGES - 1;
+    for (int c = 0; c < nk && !abort; ++c) {
+      const uint32_t g = g0 + c;
+      const uint32_t s = g % TC_STAGES;
+      if (g >= TC_STAGES) {                      // the MMAs of this stage's previous fill are done
+        if (!mbar_wait(bar_empty + 8 * s, ((g / TC_STAGES) - 1) & 1)) { abort = true; break; }
+      }
+      // x rows: 8 lanes cover one row's 128-byte segment, a warp 4 rows per instruction
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        const int w = tid + m * TC_THREADS;
+        const int row = w >> 3, q = w & 7;
+        const int tok = s_tok[row];
+        if (tok >= 0) {
+          const uint32_t dst = sU + s * TC_STAGE_BYTES + (uint32_t)row * 128 + ((q ^ (row & 7)) << 4);
+          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst),
+                       "l"(x + (size_t)tok * d_in + (size_t)c * TC_BK + q * 8)
+                       : "memory");
         }
       }
-      cp_async_commit();
-      const int m = c - (TC_STAGES - 1);
-      if (m >= 0) {
-        cp_async_wait<TC_STAGES - 1>();
-        fence_proxy_async();
-        abort = __syncthreads_or(abort);
-        if (abort) break;
-        if (tid == 0) {
-          tc_fence_after();
-          const int s = m % TC_STAGES;
-          const uint32_t xs = sX + (uint32_t)s * TC_BM * 128;
-          const uint32_t as = sA + (uint32_t)s * TC_MAXN1 * 128;
-#pragma unroll
-          for (int kk = 0; kk < TC_BK / 16; ++kk)
-            mma_bf16(tmem, desc_k_sw128(xs + kk * 32), desc_k_sw128(as + kk * 32), id1, (m > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(bar_stage + 8 * s);
-        }
+      const uint32_t abase = sU + s * TC_STAGE_BYTES + TC_BM * 128;
+      for (int w = tid; w < N1 * 8; w += TC_THREADS) {
+        const int j = w >> 3, q = w & 7;
+        const int slot = j / R16, r = j % R16;
+        const uint32_t dst = abase + (uint32_t)j * 128 + ((q ^ (j & 7)) << 4);
+        const bool valid = r < rk[slot];
+        cp_async16_zfill(dst, valid ? Aj[slot] + (size_t)r * d_in + (size_t)c * TC_BK + q * 8 : Aj[0], valid);
       }
+      cp_async_arrive(bar_full + 8 * s);
+      if (tid == 0 && c >= LAG) consume(g0 + c - LAG, c - LAG);
     }
-    // every stage with an outstanding commit: wait (keeps parities in step)
-    for (int s = 0; s < TC_STAGES && s < nk; ++s) {
-      if (!abort && !mbar_wait(bar_stage + 8 * s, (ph_stage >> s) & 1)) abort = true;
-      ph_stage ^= 1u << s;
+    if (tid == 0 && !abort) {
+      for (int c = max(0, nk - LAG); c < nk && !abort; ++c) consume(g0 + c, c);
+      if (!abort) mma_commit(bar_d1);
     }
+    gchunk = g0 + nk;
+    abort = __syncthreads_or(abort);
+    if (abort) break;
+    if (!mbar_wait(bar_d1, ph_d1)) abort = true;
+    ph_d1 ^= 1;
     abort = __syncthreads_or(abort);
     tc_fence_after();
     if (abort) break;
@@ -400,45 +409,53 @@ __global__ void __launch_bounds__(TC_THREADS, 1) sgmm_tc_kernel(TcArgs args) {
     __nv_bfloat16* __restrict__ y = reinterpret_cast<__nv_bfloat16*>(a.proj[p].y);
     const int nnt = (d_out + TC_NT - 1) / TC_NT;
 
-    auto issue_tile = [&](int nt, int b) {
+    // Bcat rows and y_base rows of tile nt into ring slot nt % NY (one cp.async group)
+    auto issue_tile = [&](int nt) {
+      const int slot = nt % TC_NY;
       const int n0 = nt * TC_NT;
       const int ncols = min(TC_NT, d_out - n0);
-      // Bcat rows n0..n0+127: K2 / 8 chunks of 16 bytes per row
-      const uint32_t bbase = sB + (uint32_t)b * TC_NT * TC_MAXN1 * 2;
+      const uint32_t bbase = sB + (uint32_t)slot * TC_BBUF_BYTES;
       const int cpr = K2 / 8;
       for (int w = tid; w < TC_NT * cpr; w += TC_THREADS) {
         const int n = w / cpr, q = w % cpr;
-        const int slot = q / (R16 / 8), cq = q % (R16 / 8);
+        const int kslot = q / (R16 / 8), cq = q % (R16 / 8);
         const uint32_t dst = bbase + (uint32_t)(n >> 3) * sbo_v + (uint32_t)q * 128 + (uint32_t)(n & 7) * 16;
-        if (n < ncols && cq * 8 < rk[slot]) {
-          const __nv_bfloat16* src = Bj[slot] + (size_t)(n0 + n) * rk[slot] + cq * 8;
-          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-        } else {
-          asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0) : "memory");
+        const bool valid = n < ncols && cq * 8 < rk[kslot];
+        cp_async16_zfill(dst, valid ? Bj[kslot] + (size_t)(n0 + n) * rk[kslot] + cq * 8 : Bj[0], valid);
+      }
+      // this warp's 32 token rows: 16 lanes per 256-byte row segment, 2 rows per instruction
+      const uint32_t ybase = sY + (uint32_t)slot * TC_YBUF_BYTES;
+      const int lane = tid & 31;
+      const int ch = lane & 15;
+      if (ch * 8 < ncols) {
+#pragma unroll 4
+        for (int k2 = 0; k2 < 16; ++k2) {
+          const int row = warp * 32 + 2 * k2 + (lane >> 4);
+          const int tok = s_tok[row];
+          if (tok >= 0)
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(ybase + (uint32_t)row * TC_YSTRIDE + ch * 16),
+                         "l"(yb + (size_t)tok * d_out + n0 + ch * 8)
+                         : "memory");
         }
       }
-      // y_base row of this thread's token (the previous store from this buffer row must be read out)
-      bulk_wait_read_all();
-      const uint32_t bytes = my_tok >= 0 ? (uint32_t)ncols * 2 : 0u;
-      mbar_arrive_expect_tx(bar_y + 8 * b, bytes);
-      if (bytes) bulk_load(sY + (uint32_t)b * TC_BM * TC_YSTRIDE + (uint32_t)tid * TC_YSTRIDE,
-                           yb + (size_t)my_tok * d_out + n0, bytes, bar_y + 8 * b);
     };
 
-    issue_tile(0, 0);
-    cp_async_commit();
+    for (int nt = 0; nt < TC_NY - 1; ++nt) {
+      if (nt < nnt) issue_tile(nt);
+      cp_async_commit();
+    }
     for (int nt = 0; nt < nnt; ++nt) {
       const int b = nt & 1;
+      const int slot = nt % TC_NY;
       const int n0 = nt * TC_NT;
       const int ncols = min(TC_NT, d_out - n0);
-      if (nt + 1 < nnt) issue_tile(nt + 1, b ^ 1);
+      if (nt + TC_NY - 1 < nnt) issue_tile(nt + TC_NY - 1);
       cp_async_commit();
-      cp_async_wait<1>();
-      fence_proxy_async();
-      __syncthreads();
+      cp_async_wait<TC_NY - 1>();                 // tile nt's group has landed (this thread)
+      __syncthreads();                            // ... and every thread's
       if (tid == 0) {
         tc_fence_after();
-        const uint32_t bb = sB + (uint32_t)b * TC_NT * TC_MAXN1 * 2;
+        const uint32_t bb = sB + (uint32_t)slot * TC_BBUF_BYTES;
         const uint32_t dcol = tmem + TC_D2_COL + (uint32_t)b * TC_NT;
         for (int kk = 0; kk < K2 / 16; ++kk)
           mma_bf16(dcol, desc_k_plain(sVH + kk * 256, 128, sbo_v), desc_k_plain(bb + kk * 256, 128, sbo_v), id2,
@@ -450,14 +467,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1) sgmm_tc_kernel(TcArgs args) {
       if (!mbar_wait(bar_mma2 + 8 * b, (ph_mma2 >> b) & 1)) abort = true;
       ph_mma2 ^= 1u << b;
       tc_fence_after();
-      if (!mbar_wait(bar_y + 8 * b, (ph_y >> b) & 1)) abort = true;
-      ph_y ^= 1u << b;
       abort = __syncthreads_or(abort);
       if (abort) break;
-      // epilogue: y = y_base + D2, one rounding, back into the staged row, then a bulk store
+      // epilogue: y = y_base + D2 in this thread's token row (one rounding) ...
       {
         const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16) + TC_D2_COL + (uint32_t)b * TC_NT;
-        unsigned char* yrow = sYp + (size_t)b * TC_BM * TC_YSTRIDE + (size_t)tid * TC_YSTRIDE;
+        unsigned char* yrow = sYp + (size_t)slot * TC_YBUF_BYTES + (size_t)tid * TC_YSTRIDE;
         for (int c0 = 0; c0 < ncols; c0 += 16) {
           float v[16];
           tmem_ld16(lane_addr + (uint32_t)c0, v);
@@ -477,22 +492,32 @@ __global__ void __launch_bounds__(TC_THREADS, 1) sgmm_tc_kernel(TcArgs args) {
             pr[1] = u1;
           }
         }
-        if (my_tok >= 0) {
-          fence_proxy_async();
-          bulk_store(y + (size_t)my_tok * d_out + n0,
-                     sY + (uint32_t)b * TC_BM * TC_YSTRIDE + (uint32_t)tid * TC_YSTRIDE, (uint32_t)ncols * 2);
-          bulk_commit();
+        __syncwarp();
+        // ... then the warp writes its 32 rows back, 2 rows (2 x 256 bytes) per instruction
+        const int lane = tid & 31;
+        const int ch = lane & 15;
+        if (ch * 8 < ncols) {
+#pragma unroll 4
+          for (int k2 = 0; k2 < 16; ++k2) {
+            const int row = warp * 32 + 2 * k2 + (lane >> 4);
+            const int tok = s_tok[row];
+            if (tok >= 0) {
+              const uint4 val = *reinterpret_cast<const uint4*>(sYp + (size_t)slot * TC_YBUF_BYTES +
+                                                               (size_t)row * TC_YSTRIDE + ch * 16);
+              __stcs(reinterpret_cast<uint4*>(y + (size_t)tok * d_out + n0 + ch * 8), val);
+            }
+          }
         }
       }
       tc_fence_before();
       __syncthreads();
     }
+    // the ring area is reused by the next item's shrink stages
     cp_async_wait_all();
     __syncthreads();
   }
   if (abort && tid == 0) report(a.ws, APR_ERR_TIMEOUT, K_TC, (int)blockIdx.x);
   cp_async_wait_all();
-  bulk_wait_all();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -536,6 +561,283 @@ cudaError_t launch_sgmm_tensor(const SgmmArgs& a, cudaStream_t s) {
   int grid = nsm;
   if (max_items < grid) grid = (int)max_items;
   return launch_pdl(sgmm_tc_kernel, dim3(grid), dim3(TC_THREADS), TcSmem::ALLOC, s, t);
+}
+
+
+// ---------------------------------------------------------------- merge on the tensor cores
+//
+// Batch-1 merge (AdaFuse summary §2.B decoding steps 3 and 5), every weight in
+// one launch, out of place:  W' = W + sum_j g_j B_{e_j} A_{e_j}.
+// A work item is a strip of 128 rows of one weight.  The strip's gated B rows
+// Bg[n][j*R16 + i] = g_j B_{e_j}[n][i] are formed once (fp32 -> bf16 hi + lo,
+// K-major), then for every 128-column tile: D[128 x 128] = Bg_hi.A^T +
+// Bg_lo.A^T on tcgen05 with A^T as an MN-major operand (rows of A_e are
+// contiguous along the output columns), TMEM double buffered; the W tile and
+// the A tile arrive two tiles ahead by cp.async into 3-deep rings, and the
+// epilogue adds D to W in fp32, rounds once and the warp writes its 32 rows
+// of W' back with coalesced 128-bit stores.
+
+constexpr int MT_BN = 128;                      // columns per tile
+constexpr int MT_NY = 3;                        // ring depth
+constexpr int MT_WSTRIDE = MT_BN * 2 + 16;      // bytes per staged W row
+constexpr int MT_WBUF = TC_BM * MT_WSTRIDE;
+constexpr int MT_ABUF = MT_BN * TC_MAXN1 * 2;   // MN-major A^T tile
+constexpr int MT_MAXPROJ = 4096;
+
+struct MtSmem {
+  static constexpr size_t GH = 0;                                        // 16 KB
+  static constexpr size_t GL = GH + (size_t)TC_BM * TC_MAXN1 * 2;        // 16 KB
+  static constexpr size_t WR = GL + (size_t)TC_BM * TC_MAXN1 * 2;        // W ring
+  static constexpr size_t AR = WR + (size_t)MT_NY * MT_WBUF;             // A ring
+  static constexpr size_t BAR = AR + (size_t)MT_NY * MT_ABUF;
+  static constexpr size_t META = BAR + 2 * 8;
+  static constexpr size_t PREF = META + 128;                             // [nproj + 1] strip prefix
+  static constexpr size_t fixed_bytes() { return PREF + 1024; }
+};
+
+// K-major A operand / MN-major B operand instruction descriptor (bf16 -> fp32).
+__host__ __device__ constexpr uint32_t idesc_bf16_bmn(int M, int N) { return idesc_bf16(M, N) | (1u << 16); }
+
+__global__ void __launch_bounds__(TC_THREADS, 1) merge_tc_kernel(const apr_merge_proj* __restrict__ projs,
+                                                                 int nproj, int E, int r, int R16,
+                                                                 const int32_t* __restrict__ idx,
+                                                                 const float* __restrict__ gate, int k,
+                                                                 void* ws) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem =
+      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int K = k * R16;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + MtSmem::BAR);
+  const uint32_t bar_mma = smem_u32(bars);                     // [2]
+  volatile int* s_flags = reinterpret_cast<volatile int*>(smem + MtSmem::META);   // [0] tmem, [1] bad
+  int* s_e = const_cast<int*>(s_flags) + 4;                    // [<= 8]
+  float* s_g = reinterpret_cast<float*>(s_e + 8);              // [<= 8]
+  int* s_pref = reinterpret_cast<int*>(smem + MtSmem::PREF);
+  const uint32_t sGH = smem_u32(smem + MtSmem::GH);
+  const uint32_t sGL = smem_u32(smem + MtSmem::GL);
+  unsigned char* sWp = smem + MtSmem::WR;
+  const uint32_t sW = smem_u32(sWp);
+  const uint32_t sA = smem_u32(smem + MtSmem::AR);
+
+  if (tid == 0) {
+    for (int i = 0; i < 2; ++i) mbar_init(bar_mma + 8 * i, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    s_flags[1] = 0;
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(const_cast<int*>(s_flags))),
+                 "r"(TC_TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = (uint32_t)s_flags[0];
+  pdl_wait();
+  pdl_trigger();
+
+  if (tid < k) {
+    const int e = idx[tid];
+    if (e < 0 || e >= E) s_flags[1] = 1;
+    s_e[tid] = e;
+    s_g[tid] = gate[tid];
+  }
+  // strips (128 rows) per weight, prefix over the weights
+  if (tid == 0) {
+    int acc = 0;
+    s_pref[0] = 0;
+    for (int p = 0; p < nproj; ++p) {
+      acc += (projs[p].d_out + TC_BM - 1) / TC_BM;
+      s_pref[p + 1] = acc;
+    }
+  }
+  __syncthreads();
+  bool abort = false;
+  if (s_flags[1]) {
+    if (tid == 0 && blockIdx.x == 0) report(ws, APR_ERR_DEVICE_INDEX, K_MERGE, 0);
+  } else {
+    const int total = s_pref[nproj];
+    const uint32_t sbo_g = (uint32_t)(K / 8) * 128;         // Bg: next 8-row group
+    const uint32_t id = idesc_bf16_bmn(TC_BM, MT_BN);
+    uint32_t ph_mma = 0;
+    for (int strip = blockIdx.x; strip < total && !abort; strip += gridDim.x) {
+      int lo = 0, hi = nproj;                                 // weight of this strip
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (s_pref[mid] <= strip) lo = mid; else hi = mid;
+      }
+      const apr_merge_proj pj = projs[lo];
+      const int row0 = (strip - s_pref[lo]) * TC_BM;
+      const int nrows = min(TC_BM, pj.d_out - row0);
+      const __nv_bfloat16* __restrict__ Wt = reinterpret_cast<const __nv_bfloat16*>(pj.W);
+      __nv_bfloat16* __restrict__ Wp = reinterpret_cast<__nv_bfloat16*>(pj.Wp);
+      // gated B rows of the strip, bf16 hi + lo, K-major
+      {
+        const int n = row0 + tid;
+        for (int j = 0; j < k; ++j) {
+          const __nv_bfloat16* B = reinterpret_cast<const __nv_bfloat16*>(pj.B[s_e[j]]);
+          for (int c8 = 0; c8 < R16; c8 += 8) {
+            float f[8];
+            if (tid < nrows && c8 < r) {
+              load8(B + (size_t)n * r + c8, f);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 8; ++i) f[i] = 0.f;
+            }
+            uint32_t h4[4], l4[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float a0 = f[2 * i] * s_g[j], a1 = f[2 * i + 1] * s_g[j];
+              const __nv_bfloat162 hh = __floats2bfloat162_rn(a0, a1);
+              const float2 hf = __bfloat1622float2(hh);
+              h4[i] = *reinterpret_cast<const uint32_t*>(&hh);
+              l4[i] = pack_bf16x2(a0 - hf.x, a1 - hf.y);
+            }
+            const int kc8 = (j * R16 + c8) >> 3;
+            const uint32_t off = (uint32_t)(tid >> 3) * sbo_g + (uint32_t)kc8 * 128 + (uint32_t)(tid & 7) * 16;
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(sGH + off), "r"(h4[0]), "r"(h4[1]),
+                         "r"(h4[2]), "r"(h4[3])
+                         : "memory");
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(sGL + off), "r"(l4[0]), "r"(l4[1]),
+                         "r"(l4[2]), "r"(l4[3])
+                         : "memory");
+          }
+        }
+      }
+      fence_proxy_async();                       // Bg was written by ordinary stores
+      const int nct = (pj.d_in + MT_BN - 1) / MT_BN;
+      auto issue_tile = [&](int ct) {
+        const int slot = ct % MT_NY;
+        const int c0 = ct * MT_BN;
+        const int ncols = min(MT_BN, pj.d_in - c0);
+        // A^T tile, MN-major: core matrix (8 columns x 8 rank rows) at (col/8)*128 + (kk/8)*2048
+        const uint32_t abase = sA + (uint32_t)slot * MT_ABUF;
+        for (int w = tid; w < K * (MT_BN / 8); w += TC_THREADS) {
+          const int kk = w / (MT_BN / 8), c = w % (MT_BN / 8);
+          const int j = kk / R16, i = kk % R16;
+          const uint32_t dst = abase + (uint32_t)c * 128 + (uint32_t)(kk >> 3) * 2048 + (uint32_t)(kk & 7) * 16;
+          const bool valid = i < r && c * 8 < ncols;
+          const __nv_bfloat16* A = reinterpret_cast<const __nv_bfloat16*>(pj.A[s_e[j]]);
+          cp_async16_zfill(dst, valid ? A + (size_t)i * pj.d_in + c0 + c * 8 : A, valid);
+        }
+        // W rows of the tile: 16 lanes per 256-byte row segment, 2 rows per instruction
+        const uint32_t wbase = sW + (uint32_t)slot * MT_WBUF;
+        const int ch = lane & 15;
+        if (ch * 8 < ncols) {
+#pragma unroll 4
+          for (int k2 = 0; k2 < 16; ++k2) {
+            const int row = warp * 32 + 2 * k2 + (lane >> 4);
+            if (row < nrows)
+              asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(wbase + (uint32_t)row * MT_WSTRIDE + ch * 16),
+                           "l"(Wt + (size_t)(row0 + row) * pj.d_in + c0 + ch * 8)
+                           : "memory");
+          }
+        }
+      };
+      for (int ct = 0; ct < MT_NY - 1; ++ct) {
+        if (ct < nct) issue_tile(ct);
+        cp_async_commit();
+      }
+      for (int ct = 0; ct < nct; ++ct) {
+        const int b = ct & 1;
+        const int slot = ct % MT_NY;
+        const int c0 = ct * MT_BN;
+        const int ncols = min(MT_BN, pj.d_in - c0);
+        if (ct + MT_NY - 1 < nct) issue_tile(ct + MT_NY - 1);
+        cp_async_commit();
+        cp_async_wait<MT_NY - 1>();
+        __syncthreads();
+        if (tid == 0) {
+          tc_fence_after();
+          const uint32_t ab = sA + (uint32_t)slot * MT_ABUF;
+          const uint32_t dcol = tmem + TC_D2_COL + (uint32_t)b * MT_BN;
+          for (int kk = 0; kk < K / 16; ++kk)
+            mma_bf16(dcol, desc_k_plain(sGH + kk * 256, 128, sbo_g), desc_k_plain(ab + kk * 4096, 2048, 128), id,
+                     kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < K / 16; ++kk)
+            mma_bf16(dcol, desc_k_plain(sGL + kk * 256, 128, sbo_g), desc_k_plain(ab + kk * 4096, 2048, 128), id, 1u);
+          mma_commit(bar_mma + 8 * b);
+        }
+        if (!mbar_wait(bar_mma + 8 * b, (ph_mma >> b) & 1)) abort = true;
+        ph_mma ^= 1u << b;
+        tc_fence_after();
+        abort = __syncthreads_or(abort);
+        if (abort) break;
+        {
+          const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16) + TC_D2_COL + (uint32_t)b * MT_BN;
+          unsigned char* wrow = sWp + (size_t)slot * MT_WBUF + (size_t)tid * MT_WSTRIDE;
+          for (int cc = 0; cc < ncols; cc += 16) {
+            float v[16];
+            tmem_ld16(lane_addr + (uint32_t)cc, v);
+            if (tid < nrows) {
+              uint4* pr = reinterpret_cast<uint4*>(wrow + cc * 2);
+              uint4 u0 = pr[0], u1 = pr[1];
+              __nv_bfloat162* h0 = reinterpret_cast<__nv_bfloat162*>(&u0);
+              __nv_bfloat162* h1 = reinterpret_cast<__nv_bfloat162*>(&u1);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const float2 f0 = __bfloat1622float2(h0[i]);
+                const float2 f1 = __bfloat1622float2(h1[i]);
+                h0[i] = __floats2bfloat162_rn(f0.x + v[2 * i], f0.y + v[2 * i + 1]);
+                h1[i] = __floats2bfloat162_rn(f1.x + v[8 + 2 * i], f1.y + v[8 + 2 * i + 1]);
+              }
+              pr[0] = u0;
+              pr[1] = u1;
+            }
+          }
+          __syncwarp();
+          const int ch = lane & 15;
+          if (ch * 8 < ncols) {
+#pragma unroll 4
+            for (int k2 = 0; k2 < 16; ++k2) {
+              const int row = warp * 32 + 2 * k2 + (lane >> 4);
+              if (row < nrows) {
+                const uint4 val = *reinterpret_cast<const uint4*>(sWp + (size_t)slot * MT_WBUF +
+                                                                 (size_t)row * MT_WSTRIDE + ch * 16);
+                __stcs(reinterpret_cast<uint4*>(Wp + (size_t)(row0 + row) * pj.d_in + c0 + ch * 8), val);
+              }
+            }
+          }
+        }
+        tc_fence_before();
+        __syncthreads();
+      }
+      cp_async_wait_all();
+      __syncthreads();
+    }
+  }
+  if (abort && tid == 0) report(ws, APR_ERR_TIMEOUT, K_MERGE, (int)blockIdx.x);
+  cp_async_wait_all();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TC_TMEM_COLS)
+                 : "memory");
+  }
+}
+
+bool merge_tensor_supported(int k, int r, int nproj) {
+  return k * round16(r) <= TC_MAXN1 && nproj <= MT_MAXPROJ;
+}
+
+cudaError_t launch_merge_tensor(const apr_merge_proj* projs, int nproj, int E, int r, const int32_t* idx,
+                                const float* gate, int k, void* ws, cudaStream_t s) {
+  const size_t smem = MtSmem::fixed_bytes() + sizeof(int) * ((size_t)nproj + 1);
+  static size_t configured = 0;
+  if (smem > configured) {
+    cudaError_t err = cudaFuncSetAttribute(merge_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    configured = smem;
+  }
+  int dev = 0, nsm = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  return launch_pdl(merge_tc_kernel, dim3(nsm), dim3(TC_THREADS), smem, s, projs, nproj, E, r, round16(r), idx,
+                    gate, k, ws);
 }
 
 }  // namespace apr

@@ -249,16 +249,18 @@ def test_sgmm_device_index_fault_is_reported(apr):
 # ------------------------------------------------------------------ merge and GEMV
 
 
-def test_merge_and_gemv_small(apr):
-    rng = np.random.default_rng(12)
-    E, r, k = 5, 16, 2
+@pytest.mark.parametrize("E,r,k", [(5, 16, 2), (8, 8, 5), (4, 32, 2), (3, 8, 1)])
+def test_merge_and_gemv_small(apr, E, r, k):
+    """Tensor-core merge (k * rank <= 64 after rounding the rank to 16) and the
+    CUDA-core merge (k=5, rank 8), on ragged weight shapes."""
+    rng = np.random.default_rng(12 + E + r + k)
     shapes = [(264, 136), (40, 1000), (1000, 64)]
     Ws = [bf16_exact(0.02 * rng.normal(size=s)) for s in shapes]
     As = [[bf16_exact(0.02 * rng.normal(size=(r, s[1]))) for _ in range(E)] for s in shapes]
     Bs = [[bf16_exact(0.02 * rng.normal(size=(s[0], r))) for _ in range(E)] for s in shapes]
     xs = [bf16_exact(rng.normal(size=s[1])) for s in shapes]
-    idx1 = np.array([3, 1], np.int32)
-    g1 = np.array([0.625, 0.375], np.float32)
+    idx1 = rng.permutation(E)[:k].astype(np.int32)
+    g1 = rng.dirichlet(np.ones(k)).astype(np.float32)
     dW = [torch.from_numpy(w).cuda().to(BF16) for w in Ws]
     dWp = [torch.full_like(w, float("nan")) for w in dW]
     keep = []

@@ -7,9 +7,8 @@
 //
 //   y_p[t] = y_base_p[t] + sum_j gate[t,j] * B_e (A_e x[t]),  e = idx[t,j]
 //
-// One launch per shared-input group, in two phases separated by a grid-wide
-// barrier (all CTAs are co-resident: the grid is sized from the occupancy;
-// the barrier's wait is bounded and reports APR_ERR_TIMEOUT):
+// Two launches per shared-input group, chained by programmatic dependent
+// launch (a kernel boundary costs less than a grid-wide barrier here):
 //
 // shrink  static items (projection, adapter e, 2048-column chunk, 4 rank rows
 //         of A_e, split of the segment).  Each thread holds an 8-column slice
@@ -23,7 +22,8 @@
 //         64 threads share the columns.  Token tiles follow the adapter-set
 //         order of the routing plan, so a tile touches few adapters.  B rows
 //         of the tile's adapters are staged in shared memory with cp.async,
-//         y_base rows are fetched asynchronously while the shrink runs, the
+//         the tile's routing plan and y_base rows are fetched before the wait
+//         (they are inputs of the call), the
 //         column-chunk partials of the tile's pairs are summed in a fixed
 //         order and gated, products accumulate in fp32, and y = y_base + delta
 //         is written with 128-bit stores, one rounding per element.  Each
@@ -89,10 +89,12 @@ __device__ __forceinline__ void zero8(Vec8<In>& r) {
 __device__ __forceinline__ bool rank_ok(int r, int max_rank) { return r > 0 && r <= max_rank && !(r & 7); }
 
 struct SkinnySmem {      // byte offsets inside the dynamic shared memory
-  size_t red, shtok, B, yb, v, acc, ints, flags, total;
+  size_t red, shtok, B, yb, v, acc, wh, wl, ints, flags, total;
 };
 
-__host__ __device__ inline SkinnySmem skinny_smem_layout(int TT, int k, int R, int elem, int bslots) {
+constexpr int DN_MAXK = 256;       // E * R handled by the dense tensor-core expand
+
+__host__ __device__ inline SkinnySmem skinny_smem_layout(int TT, int k, int R, int elem, int bslots, int dense_k) {
   SkinnySmem L;
   const int TK = TT * k;
   size_t o = 0;
@@ -102,6 +104,9 @@ __host__ __device__ inline SkinnySmem skinny_smem_layout(int TT, int k, int R, i
   L.yb = o;    o += (size_t)TT * EX_NT * elem;
   L.v = o;     o += sizeof(float) * (size_t)TK * R;
   L.acc = o;   o += sizeof(float) * (size_t)TT * EX_NT;
+  L.wh = o;    o += (size_t)TT * (dense_k + 8) * 2;       // dense gated v, bf16 hi
+  L.wl = o;    o += (size_t)TT * (dense_k + 8) * 2;       //   and lo parts
+  o = (o + 15) / 16 * 16;
   L.ints = o;  o += sizeof(int) * ((size_t)TT + 7 * (size_t)TK + 1);
   L.flags = o; o += sizeof(int) * 4;
   L.total = (o + 15) / 16 * 16;
@@ -113,38 +118,20 @@ struct SkinnyParams {
   int nkc, nrc, nsplit;   // shrink item space
   int TT, ntt, ntd;       // expand item space
   int bslots, prefetch_all;
+  int dense_k;            // > 0: expand as one dense [TT x E*R] x [E*R x 64] product on tensor cores
 };
 
-// Bounded grid-wide barrier on the workspace header (every CTA is resident).
-__device__ bool grid_barrier(WsHeader* hdr, unsigned nblocks, volatile int* s_flag) {
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int ok = 1;
-    const unsigned gen = *reinterpret_cast<volatile unsigned*>(&hdr->bar_gen);
-    __threadfence();
-    const unsigned arrived = atomicAdd(&hdr->bar_count, 1u);
-    if (arrived == nblocks - 1) {
-      atomicExch(&hdr->bar_count, 0u);
-      __threadfence();
-      atomicAdd(&hdr->bar_gen, 1u);
-    } else {
-      uint64_t t0;
-      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
-      while (*reinterpret_cast<volatile unsigned*>(&hdr->bar_gen) == gen) {
-        uint64_t t;
-        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-        if (t - t0 > 1000000000ull) { ok = 0; break; }
-        __nanosleep(64);
-      }
-    }
-    __threadfence();
-    *s_flag = ok;
-  }
-  __syncthreads();
-  return *s_flag != 0;
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-template <typename In>
+// PHASE 0: shrink (partial sums to the workspace); PHASE 1: expand.
+template <typename In, int PHASE>
 __global__ void __launch_bounds__(SK_THREADS) sgmm_skinny_kernel(SgmmArgs a, SkinnyParams P) {
   constexpr int SH_BATCH = sizeof(In) == 2 ? 8 : 4;   // x rows in flight per thread
   extern __shared__ __align__(16) unsigned char smem[];
@@ -153,7 +140,7 @@ __global__ void __launch_bounds__(SK_THREADS) sgmm_skinny_kernel(SgmmArgs a, Ski
   const int npairs = a.T * K;
   const int elem = (int)sizeof(In);
   const int TT = P.TT, TK = TT * K;
-  const SkinnySmem Ls = skinny_smem_layout(TT, K, R, elem, P.bslots);
+  const SkinnySmem Ls = skinny_smem_layout(TT, K, R, elem, P.bslots, P.dense_k);
   float (*red)[kPairTile][SH_RC] = reinterpret_cast<float (*)[kPairTile][SH_RC]>(smem + Ls.red);
   int* s_shtok = reinterpret_cast<int*>(smem + Ls.shtok);
   unsigned char* s_B = smem + Ls.B;
@@ -169,12 +156,10 @@ __global__ void __launch_bounds__(SK_THREADS) sgmm_skinny_kernel(SgmmArgs a, Ski
   int* s_Ur = s_U + TK;                                    // [TK] their ranks
   float* s_g = reinterpret_cast<float*>(s_Ur + TK);        // [TK] gate of the pair
   int* s_nU = reinterpret_cast<int*>(s_g + TK);            // [1]
-  volatile int* s_flag = reinterpret_cast<volatile int*>(smem + Ls.flags);
   const int stride_b = R * elem + 16;
   const In* __restrict__ x = reinterpret_cast<const In*>(a.x);
   const int d_in = a.d_in;
   float* vpart = ws_at<float>(a.ws, P.scratch_off);
-  WsHeader* hdr = reinterpret_cast<WsHeader*>(a.ws);
   const WsLayout L = ws_layout(a.T, a.k, a.E);
   const int* tok_order = ws_at<int>(a.ws, L.tok_order);
   const int* inv = ws_at<int>(a.ws, L.inv);
@@ -206,11 +191,24 @@ __global__ void __launch_bounds__(SK_THREADS) sgmm_skinny_kernel(SgmmArgs a, Ski
       const int row = v / vpr, c = v % vpr;
       cp_async16(dst + (size_t)row * stride_b + c * 16, src + ((size_t)row * vpr + c) * 16);
     }
+    if (P.dense_k) {               // the dense product reads every rank column: zero the tail
+      const int vfull = R * elem / 16;
+      for (int v = tid; v < EX_NT * (vfull - vpr); v += SK_THREADS) {
+        const int row = v / (vfull - vpr), c = vpr + v % (vfull - vpr);
+        *reinterpret_cast<uint4*>(dst + (size_t)row * stride_b + c * 16) = make_uint4(0, 0, 0, 0);
+      }
+    }
+  };
+  auto zero_slot = [&](int slot) {
+    unsigned char* dst = s_B + (size_t)slot * EX_NT * stride_b;
+    for (int v = tid; v < EX_NT * stride_b / 16; v += SK_THREADS)
+      reinterpret_cast<uint4*>(dst)[v] = make_uint4(0, 0, 0, 0);
   };
   auto prefetch_all_B = [&](const ExItem& it) {
     for (int e = 0; e < E; ++e) {
       const int r_e = a.ranks[e];
       if (rank_ok(r_e, R)) stage_B(it, e, r_e, e);
+      else if (P.dense_k) zero_slot(e);
     }
   };
   // routing plan of the tile and its y_base rows (after the wait)
@@ -284,30 +282,95 @@ __global__ void __launch_bounds__(SK_THREADS) sgmm_skinny_kernel(SgmmArgs a, Ski
     }
     // gated v of every pair of the tile: column-chunk partials summed in order
     const float* vp = vpart + (size_t)it.p * P.nkc * npairs * R;
-    constexpr int VB = 8;
+    constexpr int VB = 4, NKC = 8;               // column chunks summed with every load in flight
     for (int w0 = tid * VB; w0 < TK * R; w0 += SK_THREADS * VB) {
-      float part[VB];
+      float ld[NKC][VB];
 #pragma unroll
-      for (int u = 0; u < VB; ++u) part[u] = 0.f;
-      for (int c = 0; c < P.nkc; ++c) {
-        float ld[VB];
+      for (int c = 0; c < NKC; ++c)
 #pragma unroll
         for (int u = 0; u < VB; ++u) {
           const int w = w0 + u;
           const int pi = w / R, i = w % R;
-          ld[u] = (w < TK * R && i < s_pr[pi]) ? __ldcg(vp + ((size_t)c * npairs + s_pos[pi]) * R + i) : 0.f;
+          ld[c][u] = (c < P.nkc && w < TK * R && i < s_pr[pi])
+                         ? __ldcg(vp + ((size_t)c * npairs + s_pos[pi]) * R + i) : 0.f;
         }
+      for (int c = NKC; c < P.nkc; ++c)
 #pragma unroll
-        for (int u = 0; u < VB; ++u) part[u] += ld[u];
-      }
+        for (int u = 0; u < VB; ++u) {
+          const int w = w0 + u;
+          const int pi = w / R, i = w % R;
+          if (w < TK * R && i < s_pr[pi]) ld[NKC - 1][u] += __ldcg(vp + ((size_t)c * npairs + s_pos[pi]) * R + i);
+        }
 #pragma unroll
       for (int u = 0; u < VB; ++u) {
         const int w = w0 + u;
-        if (w < TK * R) s_v[w] = s_g[w / R] * part[u];
+        float part = 0.f;
+#pragma unroll
+        for (int c = 0; c < NKC; ++c) part += ld[c][u];
+        if (w < TK * R) s_v[w] = s_g[w / R] * part;
       }
     }
     for (int w = tid; w < TT * EX_NT; w += SK_THREADS) s_acc[w] = 0.f;
     __syncthreads();
+    if (P.dense_k) {
+      if constexpr (sizeof(In) == 2) {
+        // W[t][e*R + i] = sum of the gated v of token t's pairs on adapter e (bf16 hi + lo)
+        const int KD = P.dense_k, WS = KD + 8;
+        __nv_bfloat16* wh = reinterpret_cast<__nv_bfloat16*>(smem + Ls.wh);
+        __nv_bfloat16* wl = reinterpret_cast<__nv_bfloat16*>(smem + Ls.wl);
+        for (int w = tid; w < TT * KD; w += SK_THREADS) {
+          const int t = w / KD, kk = w % KD;
+          const int e = kk / R, i = kk % R;
+          float val = 0.f;
+          for (int j = 0; j < K; ++j) {
+            const int pi = t * K + j;
+            if (t < it.ntok && s_pe[pi] == e) val += s_v[(size_t)pi * R + i];
+          }
+          const __nv_bfloat16 h = __float2bfloat16_rn(val);
+          wh[t * WS + kk] = h;
+          wl[t * WS + kk] = __float2bfloat16_rn(val - __bfloat162float(h));
+        }
+        if (!prefetched) {
+          prefetch_all_B(it);
+          cp_async_commit();
+        }
+        cp_async_wait_all();
+        __syncthreads();
+        // [TT x KD] x [KD x 64] on mma.sync m16n8k16: (TT/16) x 8 tiles of 16 x 8 over 8 warps
+        const int g = lane >> 2, c = lane & 3;
+        const int mtiles = (TT + 15) / 16;
+        for (int tile = warp; tile < mtiles * (EX_NT / 8); tile += SK_THREADS / 32) {
+          const int mt = tile / (EX_NT / 8), n8 = tile % (EX_NT / 8);
+          float d[4] = {0.f, 0.f, 0.f, 0.f};
+          const int r0 = mt * 16 + g, r1 = r0 + 8;
+          const int n = n8 * 8 + g;
+          for (int k0 = 0; k0 < KD; k0 += 16) {
+            const int ka = k0 + 2 * c, kb = ka + 8;
+            const int e_a = ka / R, ia = ka % R, e_b = kb / R, ib = kb % R;
+            const uint32_t b0 = *reinterpret_cast<const uint32_t*>(s_B + (size_t)e_a * EX_NT * stride_b +
+                                                                   (size_t)n * stride_b + ia * 2);
+            const uint32_t b1 = *reinterpret_cast<const uint32_t*>(s_B + (size_t)e_b * EX_NT * stride_b +
+                                                                   (size_t)n * stride_b + ib * 2);
+            const bool v0 = r0 < TT, v1 = r1 < TT;
+            const uint32_t ah0 = v0 ? *reinterpret_cast<const uint32_t*>(wh + r0 * WS + ka) : 0u;
+            const uint32_t ah1 = v1 ? *reinterpret_cast<const uint32_t*>(wh + r1 * WS + ka) : 0u;
+            const uint32_t ah2 = v0 ? *reinterpret_cast<const uint32_t*>(wh + r0 * WS + kb) : 0u;
+            const uint32_t ah3 = v1 ? *reinterpret_cast<const uint32_t*>(wh + r1 * WS + kb) : 0u;
+            const uint32_t al0 = v0 ? *reinterpret_cast<const uint32_t*>(wl + r0 * WS + ka) : 0u;
+            const uint32_t al1 = v1 ? *reinterpret_cast<const uint32_t*>(wl + r1 * WS + ka) : 0u;
+            const uint32_t al2 = v0 ? *reinterpret_cast<const uint32_t*>(wl + r0 * WS + kb) : 0u;
+            const uint32_t al3 = v1 ? *reinterpret_cast<const uint32_t*>(wl + r1 * WS + kb) : 0u;
+            mma16816(d, ah0, ah1, ah2, ah3, b0, b1);
+            mma16816(d, al0, al1, al2, al3, b0, b1);
+          }
+          const int col0 = n8 * 8 + 2 * c;
+          if (r0 < TT) { s_acc[r0 * EX_NT + col0] = d[0]; s_acc[r0 * EX_NT + col0 + 1] = d[1]; }
+          if (r1 < TT) { s_acc[r1 * EX_NT + col0] = d[2]; s_acc[r1 * EX_NT + col0 + 1] = d[3]; }
+        }
+        __syncthreads();
+        nU = 0;                    // the per-pair loop below has nothing left to do
+      }
+    }
     const int ucap = P.prefetch_all ? E : P.bslots;
     const int col = tid % EX_NT, tg = tid / EX_NT;
     for (int u0 = 0; u0 < nU; u0 += ucap) {
@@ -369,16 +432,7 @@ __global__ void __launch_bounds__(SK_THREADS) sgmm_skinny_kernel(SgmmArgs a, Ski
     __syncthreads();
   };
 
-  // ---------------------------------------------------------------- before the wait
-  // first shrink item's A rows (registers) and first expand item's B slices (shared)
-  const bool have_ex = blockIdx.x < nB;
-  ExItem ex0 = {};
-  if (have_ex) {
-    ex0 = ex_item(blockIdx.x);
-    if (P.prefetch_all) prefetch_all_B(ex0);
-  }
-  cp_async_commit();
-
+  if constexpr (PHASE == 0) {
   auto shrink_item = [&](long it, bool first) {
     long rest = it;
     const int split = (int)(rest % P.nsplit); rest /= P.nsplit;
@@ -410,7 +464,6 @@ __global__ void __launch_bounds__(SK_THREADS) sgmm_skinny_kernel(SgmmArgs a, Ski
     if (first) {
       pdl_wait();
       pdl_trigger();
-      if (have_ex) plan(ex0);        // routing plan + y_base of the first expand item
     }
     if (bad) {
       if (tid == 0 && p == 0 && rc == 0 && kc == 0 && split == 0) report(a.ws, APR_ERR_DEVICE_INDEX, K_SHRINK, e);
@@ -462,31 +515,32 @@ __global__ void __launch_bounds__(SK_THREADS) sgmm_skinny_kernel(SgmmArgs a, Ski
     }
   };
 
-  // ---------------------------------------------------------------- shrink phase
-  bool first = true;
-  for (long it = blockIdx.x; it < nA; it += gridDim.x) {
-    shrink_item(it, first);
-    first = false;
-  }
-  if (first) {
+    bool first = true;
+    for (long it = blockIdx.x; it < nA; it += gridDim.x) {
+      shrink_item(it, first);
+      first = false;
+    }
+    // a CTA without items exits; that counts as its trigger for the next launch
+  } else {
+    // The preceding kernel is this call's shrink, which triggers this launch only
+    // after its own wait: every input of the call (weights, routing plan,
+    // y_base) is complete, only the shrink's partial sums need the wait.
+    const bool have_ex = blockIdx.x < nB;
+    if (!have_ex) return;
+    const ExItem ex0 = ex_item(blockIdx.x);
+    if (P.prefetch_all) prefetch_all_B(ex0);
+    cp_async_commit();
+    plan(ex0);
     pdl_wait();
     pdl_trigger();
-    if (have_ex) plan(ex0);
-  }
-  // ---------------------------------------------------------------- all partial sums written
-  if (!grid_barrier(hdr, gridDim.x, s_flag)) {
-    if (tid == 0) report(a.ws, APR_ERR_TIMEOUT, K_EXPAND, (int)blockIdx.x);
+    finish(ex0, P.prefetch_all != 0);
+    for (long it = (long)blockIdx.x + gridDim.x; it < nB; it += gridDim.x) {
+      const ExItem ex = ex_item(it);
+      plan(ex);
+      finish(ex, false);
+    }
     cp_async_wait_all();
-    return;
   }
-  // ---------------------------------------------------------------- expand phase
-  if (have_ex) finish(ex0, P.prefetch_all != 0);
-  for (long it = (long)blockIdx.x + gridDim.x; it < nB; it += gridDim.x) {
-    const ExItem ex = ex_item(it);
-    plan(ex);
-    finish(ex, false);
-  }
-  cp_async_wait_all();
 }
 
 static int expand_tokens_per_tile(int k, int max_rank) {
@@ -529,26 +583,25 @@ static cudaError_t launch_skinny_typed(const SgmmArgs& a, size_t scratch_off, cu
   P.prefetch_all = (size_t)a.E * per_slot <= (size_t)EX_BBUDGET ? 1 : 0;
   P.bslots = P.prefetch_all ? a.E : (int)(EX_BBUDGET / per_slot);
   if (P.bslots < 1) P.bslots = 1;
-  const size_t smem = skinny_smem_layout(P.TT, a.k, a.max_rank, elem, P.bslots).total;
+  P.dense_k = (sizeof(In) == 2 && P.prefetch_all && a.E * a.max_rank <= DN_MAXK && a.E * a.max_rank % 16 == 0)
+                  ? a.E * a.max_rank : 0;
+  const size_t smem = skinny_smem_layout(P.TT, a.k, a.max_rank, elem, P.bslots, P.dense_k).total;
+  const long nA = (long)a.nproj * a.E * P.nkc * P.nrc * P.nsplit;
+  const long nB = (long)a.nproj * P.ntt * P.ntd;
+  const long capA = 16L * sm_count();
+  const long gA = nA < capA ? (nA > 0 ? nA : 1) : capA;
+  const size_t smemA = skinny_smem_layout(P.TT, a.k, a.max_rank, elem, 0, 0).B;   // shrink: reduction buffers only
+  cudaError_t err = launch_pdl(sgmm_skinny_kernel<In, 0>, dim3((unsigned)gA), dim3(SK_THREADS), smemA, s, a, P);
+  if (err != cudaSuccess) return err;
   static size_t configured = 0;
   if (smem > 48 * 1024 && smem > configured) {
-    cudaError_t err =
-        cudaFuncSetAttribute(sgmm_skinny_kernel<In>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    err = cudaFuncSetAttribute(sgmm_skinny_kernel<In, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     configured = smem;
   }
-  // every CTA must be resident at once for the grid barrier
-  int per_sm = 0;
-  cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, sgmm_skinny_kernel<In>, SK_THREADS, smem);
-  if (err != cudaSuccess) return err;
-  if (per_sm < 1) return cudaErrorInvalidConfiguration;
-  const long nA = (long)a.nproj * a.E * P.nkc * P.nrc * P.nsplit;
-  const long nB = (long)a.nproj * P.ntt * P.ntd;
-  long grid = nA > nB ? nA : nB;
-  const long cap = (long)per_sm * sm_count();
-  if (grid > cap) grid = cap;
-  if (grid < 1) grid = 1;
-  return launch_pdl(sgmm_skinny_kernel<In>, dim3((unsigned)grid), dim3(SK_THREADS), smem, s, a, P);
+  const long capB = 64L * sm_count();
+  const long gB = nB < capB ? (nB > 0 ? nB : 1) : capB;
+  return launch_pdl(sgmm_skinny_kernel<In, 1>, dim3((unsigned)gB), dim3(SK_THREADS), smem, s, a, P);
 }
 
 cudaError_t launch_sgmm_skinny(const SgmmArgs& a, int dtype, size_t scratch_off, cudaStream_t s) {

@@ -12,28 +12,36 @@
 //  shrink  D1[128 x N1] = X_tile[128 x d_in] . [A_e0 ; A_e1]^T on tcgen05
 //          (kind::f16, bf16 in, fp32 accumulate in TMEM), N1 = k * R16 where
 //          R16 is the rank rounded up to 16 (zero rows pad the smaller ranks).
-//          Every thread copies its token's x row and a share of the A rows
-//          with 16-byte cp.async (each warp fetches whole 128-byte row segments)
-//          into 128B-swizzled K-major stages; the copies arrive on the stage's
-//          "full" mbarrier when they land (6 stages in flight, no block
-//          barrier per stage); thread 0 issues the MMAs of a
-//          stage once it is full and commits them to the stage's "empty"
-//          mbarrier, which frees the stage for the next fill.
+//          The gathered x rows arrive by TMA (tile::gather4: four token rows x
+//          128 bytes per instruction, 128B-swizzled, one issuing lane per warp
+//          for its 32 tokens, rows of absent tokens zero-filled) and the small
+//          A rows by 16-byte cp.async; both complete on the stage's "full"
+//          mbarrier (6 stages in flight).  One thread of the MMA warp issues
+//          the MMAs of a stage once it is full and commits them to the stage's
+//          "empty" mbarrier, which frees the stage for the next fill.
 //  gate    D1 is read back with tcgen05.ld (one TMEM lane per token), scaled
 //          by the token's gates and split into bf16 hi + lo parts (so the
 //          expand keeps ~16 mantissa bits of v), written to shared memory as
 //          the K-major A operand of the expand.
 //  expand  for every 128-column tile of d_out: D2[128 x 128] = V_hi.Bcat^T +
 //          V_lo.Bcat^T with Bcat[n] = [B_e0[n] | B_e1[n]] (K2 = N1), TMEM
-//          double buffered.  Bcat and the y_base rows of a tile are fetched two
-//          tiles ahead with cp.async into 3-deep rings that reuse the shrink
-//          stages' shared memory (each warp loads and stores whole row
-//          segments, 2 rows per instruction); the epilogue adds D2 in its
-//          token's row, rounds to bf16 once, and the warp writes its 32 rows
-//          back with coalesced 128-bit stores.
+//          double buffered.  Bcat (cp.async) and the y_base rows (TMA gather4)
+//          of a tile are fetched two tiles ahead into 3-deep rings that reuse
+//          the shrink stages' shared memory; the epilogue adds D2 in its
+//          token's row, rounds to bf16 once, and the rows leave by TMA
+//          scatter4 (plain stores for the one 4-row group a tile's end cuts).
+//
+// Warps 0-3 stage operands and run epilogues, warp 4 issues the MMAs; each
+// worker warp owns 32 token rows of every buffer, so reuse of a ring slot only
+// waits for that warp's own bulk stores.
 //
 // Every mbarrier wait is bounded by the global timer (1 s); on expiry the CTA
 // records APR_ERR_TIMEOUT, drains its own copies and frees its TMEM.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
 #include "apr_internal.cuh"
 
 namespace apr {
@@ -45,11 +53,10 @@ constexpr int TC_STAGES = 6;
 constexpr int TC_MAXN1 = 64;     // k * R16
 constexpr int TC_NT = 128;       // output columns per expand tile
 constexpr int TC_NY = 3;         // depth of the Bcat / y_base rings (prefetch distance 2)
-constexpr int TC_YSTRIDE = TC_NT * 2 + 16;   // bytes per staged y row (padding against bank conflicts)
 constexpr uint32_t TC_TMEM_COLS = 512;
 constexpr uint32_t TC_D2_COL = 128;           // D2 buffers at columns 128 and 256
 constexpr int TC_STAGE_BYTES = TC_BM * 128 + TC_MAXN1 * 128;   // x tile + A rows
-constexpr int TC_YBUF_BYTES = TC_BM * TC_YSTRIDE;
+constexpr int TC_YBUF_BYTES = 2 * TC_BM * 128;                  // two 64-column halves, 128B-swizzled rows
 constexpr int TC_BBUF_BYTES = TC_NT * TC_MAXN1 * 2;
 
 struct TcSmem {
@@ -58,19 +65,19 @@ struct TcSmem {
   static constexpr size_t RING_AREA = (size_t)TC_NY * (TC_YBUF_BYTES + TC_BBUF_BYTES);
   static constexpr size_t U = 0;
   static constexpr size_t U_BYTES = STAGE_AREA > RING_AREA ? STAGE_AREA : RING_AREA;
-  static constexpr size_t YR = U;                                             // y ring
+  static constexpr size_t YR = U;                                             // y ring (1024-aligned slots)
   static constexpr size_t BR = U + (size_t)TC_NY * TC_YBUF_BYTES;             // Bcat ring
   static constexpr size_t VH = U + (U_BYTES + 1023) / 1024 * 1024;            // 16 KB
   static constexpr size_t VL = VH + (size_t)TC_BM * TC_MAXN1 * 2;             // 16 KB
   static constexpr size_t BAR = VL + (size_t)TC_BM * TC_MAXN1 * 2;            // mbarriers
-  static constexpr int NBARS = 2 * TC_STAGES + 1 + 2;
+  static constexpr int NBARS = 2 * TC_STAGES + 2 + TC_NY + 4;
   static constexpr size_t META = BAR + (size_t)NBARS * 8;
   static constexpr size_t TOTAL = META + 3 * TC_BM * 4 + 64;
   static constexpr size_t ALLOC = TOTAL + 1024;                               // for 1024-byte alignment
 };
 static_assert(TcSmem::ALLOC <= 227 * 1024, "shared memory budget");
 static_assert(TC_STAGE_BYTES % 1024 == 0, "stages keep 1024-byte alignment");
-static_assert(TcSmem::BR % 16 == 0 && TC_YBUF_BYTES % 16 == 0, "16-byte aligned rings");
+static_assert(TcSmem::BR % 16 == 0 && TC_YBUF_BYTES % 1024 == 0, "aligned rings");
 
 // ---------------------------------------------------------------- PTX wrappers
 
@@ -123,6 +130,31 @@ __device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void* src, 
 __device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+// TMA: four rows (y0..y3) x one 64-column box of a 2-D tensor map, into / out of
+// four consecutive 128-byte (swizzled) shared rows.  Row coordinates past the
+// tensor's end load zeros; stores are only issued for rows that exist.
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* tm, int x, int y0, int y1, int y2,
+                                            int y3, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+      "%3, %4, %5, %6}], [%7];" ::"r"(dst),
+      "l"(tm), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void tma_scatter4(const CUtensorMap* tm, int x, int y0, int y1, int y2, int y3,
+                                             uint32_t src) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.tile::scatter4.bulk_group [%0, {%1, %2, %3, %4, %5}], [%6];" ::"l"(tm),
+      "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(src)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -189,28 +221,47 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
 // ---------------------------------------------------------------- the kernel
 
 struct TcArgs {
+  CUtensorMap tm_x;                    // x [T, d_in], box 64 x 1, 128B swizzle
+  CUtensorMap tm_yb[APR_MAX_PROJ];     // y_base [T, d_out]
+  CUtensorMap tm_y[APR_MAX_PROJ];      // y [T, d_out]
   SgmmArgs a;
   int R16;     // rank slot per adapter (multiple of 16)
   int N1;      // k * R16
 };
 
-__global__ void __launch_bounds__(TC_THREADS, 1) sgmm_tc_kernel(TcArgs args) {
+constexpr int TC_WORKERS = 128;                  // warps 0-3: loads and epilogues
+constexpr int TC_BLOCK = TC_WORKERS + 32;        // warp 4: MMA issue
+
+__device__ __forceinline__ void workers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(TC_WORKERS) : "memory"); }
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+// Warp-specialised: warps 0-3 stage operands with TMA and cp.async (completion
+// arrives on mbarriers) and run the epilogues; lane 0 of warp 4 issues every
+// tcgen05.mma and commits it to the barrier that releases the consumer.  No
+// block-wide barrier inside an item, so loads, MMAs and epilogues of different
+// chunks and tiles overlap.
+__global__ void __launch_bounds__(TC_BLOCK, 1) sgmm_tc_kernel(const __grid_constant__ TcArgs args) {
   const SgmmArgs& a = args.a;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const bool worker = tid < TC_WORKERS;
   const int K = a.k, R16 = args.R16, N1 = args.N1, K2 = N1;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + TcSmem::BAR);
-  // barriers: full[S], empty[S], d1, mma2[2]
-  const uint32_t bar_full = smem_u32(bars);
-  const uint32_t bar_empty = smem_u32(bars + TC_STAGES);
-  const uint32_t bar_d1 = smem_u32(bars + 2 * TC_STAGES);
-  const uint32_t bar_mma2 = smem_u32(bars + 2 * TC_STAGES + 1);
+  const uint32_t bar_full = smem_u32(bars);                              // [S]  stage loaded
+  const uint32_t bar_empty = smem_u32(bars + TC_STAGES);                 // [S]  stage consumed
+  const uint32_t bar_d1 = smem_u32(bars + 2 * TC_STAGES);                // shrink accumulator ready
+  const uint32_t bar_v = smem_u32(bars + 2 * TC_STAGES + 1);             // V written
+  const uint32_t bar_tfull = smem_u32(bars + 2 * TC_STAGES + 2);         // [NY] tile operands loaded
+  const uint32_t bar_d2full = smem_u32(bars + 2 * TC_STAGES + 2 + TC_NY);      // [2] expand accumulator ready
+  const uint32_t bar_d2empty = smem_u32(bars + 2 * TC_STAGES + 4 + TC_NY);     // [2] expand accumulator read
   int* s_tok = reinterpret_cast<int*>(smem + TcSmem::META);
   float* s_g0 = reinterpret_cast<float*>(s_tok + TC_BM);
   float* s_g1 = s_g0 + TC_BM;
-  volatile int* s_flags = reinterpret_cast<volatile int*>(s_g1 + TC_BM);   // [0] tmem base, [2..3] set
+  volatile int* s_flags = reinterpret_cast<volatile int*>(s_g1 + TC_BM);   // [0] tmem, [2..3] set, [4] bad
   const uint32_t sU = smem_u32(smem + TcSmem::U);
   const uint32_t sVH = smem_u32(smem + TcSmem::VH);
   const uint32_t sVL = smem_u32(smem + TcSmem::VL);
@@ -220,11 +271,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1) sgmm_tc_kernel(TcArgs args) {
 
   if (tid == 0) {
     for (int i = 0; i < TC_STAGES; ++i) {
-      mbar_init(bar_full + 8 * i, TC_THREADS);
+      mbar_init(bar_full + 8 * i, TC_WORKERS + 4);       // A copies of every worker + x rows of every warp
       mbar_init(bar_empty + 8 * i, 1);
     }
     mbar_init(bar_d1, 1);
-    for (int i = 0; i < 2; ++i) mbar_init(bar_mma2 + 8 * i, 1);
+    mbar_init(bar_v, TC_WORKERS);
+    for (int i = 0; i < TC_NY; ++i) mbar_init(bar_tfull + 8 * i, TC_WORKERS + 4);   // Bcat + y_base rows
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar_d2full + 8 * i, 1);
+      mbar_init(bar_d2empty + 8 * i, TC_WORKERS);
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 0) {
@@ -248,27 +304,27 @@ __global__ void __launch_bounds__(TC_THREADS, 1) sgmm_tc_kernel(TcArgs args) {
   const SetTile* stiles = ws_at<SetTile>(a.ws, L.stiles);
   const int nst = hdr->n_stiles;
   const long nitems = (long)nst * a.nproj;
-  const __nv_bfloat16* __restrict__ x = reinterpret_cast<const __nv_bfloat16*>(a.x);
   const int d_in = a.d_in;
   const int nk = d_in / TC_BK;
   const uint32_t id1 = idesc_bf16(TC_BM, N1);
   const uint32_t id2 = idesc_bf16(TC_BM, TC_NT);
   const uint32_t sbo_v = (uint32_t)(K2 / 8) * 128;   // V and Bcat: next 8-row group
-  uint32_t gchunk = 0;       // shrink chunks issued by this CTA so far (stage = gchunk % S)
-  uint32_t ph_d1 = 0, ph_mma2 = 0;
+  uint32_t gchunk = 0;      // shrink chunks so far (stage = gchunk % S, use = gchunk / S)
+  uint32_t gtile = 0;       // expand tiles so far (ring slot = gtile % NY, D2 buffer = gtile & 1)
+  uint32_t nitem = 0;       // items so far (parity of d1 / V barriers)
   bool abort = false;
 
-  for (long item = blockIdx.x; item < nitems && !abort; item += gridDim.x) {
+  for (long item = blockIdx.x; item < nitems; item += gridDim.x) {
     const int st = (int)(item / a.nproj);
     const int p = (int)(item % a.nproj);
-    const SetTile tile = stiles[st];
-    const int len = tile.len;
     const int d_out = a.proj[p].d_out;
-    // tokens, their adapter set (sorted) and gates in that order
-    {
+    const int nnt = (d_out + TC_NT - 1) / TC_NT;
+    if (worker) {
+      // tokens, their adapter set (sorted) and gates in that order
+      const SetTile tile = stiles[st];
       int tok = -1, e0 = 0, e1 = 0;
       float g0 = 0.f, g1 = 0.f;
-      if (tid < len) {
+      if (tid < tile.len) {
         tok = tok_order[tile.start + tid];
         e0 = a.idx[(size_t)tok * K];
         g0 = a.gate[(size_t)tok * K];
@@ -287,198 +343,155 @@ __global__ void __launch_bounds__(TC_THREADS, 1) sgmm_tc_kernel(TcArgs args) {
       if (tid == 0) {
         s_flags[2] = e0;
         s_flags[3] = e1;
+        bool bad = (e0 < 0 || e0 >= a.E || (K == 2 && (e1 < 0 || e1 >= a.E)));
+        if (!bad) {
+          const int r0 = a.ranks[e0], r1 = K == 2 ? a.ranks[e1] : 8;
+          bad = r0 <= 0 || r0 > R16 || (r0 & 7) || r1 <= 0 || r1 > R16 || (r1 & 7);
+        }
+        s_flags[4] = bad ? 1 : 0;
+        if (bad) report(a.ws, APR_ERR_DEVICE_INDEX, K_TC, e0);
       }
     }
     __syncthreads();
-    const int e0 = s_flags[2], e1 = s_flags[3];
-    int rk[2] = {0, 0};
-    bool bad = (e0 < 0 || e0 >= a.E || (K == 2 && (e1 < 0 || e1 >= a.E)));
-    if (!bad) {
-      rk[0] = a.ranks[e0];
-      rk[1] = K == 2 ? a.ranks[e1] : 0;
-      if (rk[0] <= 0 || rk[0] > R16 || (rk[0] & 7) || (K == 2 && (rk[1] <= 0 || rk[1] > R16 || (rk[1] & 7))))
-        bad = true;
-    }
-    if (bad) {
-      if (tid == 0) report(a.ws, APR_ERR_DEVICE_INDEX, K_TC, e0);
+    if (s_flags[4] || abort) {
       __syncthreads();
       continue;
     }
-    const __nv_bfloat16* Aj[2];
-    Aj[0] = reinterpret_cast<const __nv_bfloat16*>(a.proj[p].A[e0]);
-    Aj[1] = K == 2 ? reinterpret_cast<const __nv_bfloat16*>(a.proj[p].A[e1]) : Aj[0];
-    const int my_tok = s_tok[tid];
+    const int e0 = s_flags[2], e1 = s_flags[3];
+    const int rk[2] = {a.ranks[e0], K == 2 ? a.ranks[e1] : 0};
+    const uint32_t g0 = gchunk, t0 = gtile;
+    // this warp's 32 token rows as TMA row coordinates (T = past the end: zero fill)
+    int trow[32];
+    if (worker && lane == 0) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int tk = s_tok[warp * 32 + i];
+        trow[i] = tk >= 0 ? tk : a.T;
+      }
+    }
 
-    // ------------------------------------------------------------ shrink
-    auto consume = [&](uint32_t g, int c) {      // thread 0: MMAs of chunk c (global index g)
-      const uint32_t s = g % TC_STAGES;
-      if (!mbar_wait(bar_full + 8 * s, (g / TC_STAGES) & 1)) { abort = true; return; }
+    if (worker) {
+      // -------------------------------------------------------- shrink operands
+      const __nv_bfloat16* Aj[2];
+      Aj[0] = reinterpret_cast<const __nv_bfloat16*>(a.proj[p].A[e0]);
+      Aj[1] = K == 2 ? reinterpret_cast<const __nv_bfloat16*>(a.proj[p].A[e1]) : Aj[0];
+      for (int c = 0; c < nk && !abort; ++c) {
+        const uint32_t g = g0 + c;
+        const uint32_t s = g % TC_STAGES;
+        if (g >= TC_STAGES && !mbar_wait(bar_empty + 8 * s, ((g / TC_STAGES) - 1) & 1)) { abort = true; break; }
+        // x rows of this warp's 32 tokens: 8 TMA gathers of 4 rows x 128 bytes
+        if (lane == 0) {
+          const uint32_t fb = bar_full + 8 * s;
+          mbar_arrive_expect_tx(fb, 8 * 4 * 128);
+          const uint32_t xdst = sU + s * TC_STAGE_BYTES + (uint32_t)(warp * 32) * 128;
+#pragma unroll
+          for (int g4 = 0; g4 < 8; ++g4)
+            tma_gather4(xdst + g4 * 512, &args.tm_x, c * TC_BK, trow[4 * g4], trow[4 * g4 + 1], trow[4 * g4 + 2],
+                        trow[4 * g4 + 3], fb);
+        }
+        const uint32_t abase = sU + s * TC_STAGE_BYTES + TC_BM * 128;
+        for (int w = tid; w < N1 * 8; w += TC_WORKERS) {
+          const int j = w >> 3, q = w & 7;
+          const int slot = j / R16, r = j % R16;
+          const uint32_t dst = abase + (uint32_t)j * 128 + ((q ^ (j & 7)) << 4);
+          const bool valid = r < rk[slot];
+          cp_async16_zfill(dst, valid ? Aj[slot] + (size_t)r * d_in + (size_t)c * TC_BK + q * 8 : Aj[0], valid);
+        }
+        cp_async_arrive(bar_full + 8 * s);
+      }
+      // -------------------------------------------------------- gates -> V (bf16 hi + lo)
+      if (!abort && !mbar_wait(bar_d1, nitem & 1)) abort = true;
       tc_fence_after();
-      const uint32_t xs = sU + s * TC_STAGE_BYTES;
-      const uint32_t as = xs + TC_BM * 128;
+      if (!abort) {
+        const int row = tid;                       // TMEM lane = token row
+        const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+        const float ga = s_g0[row], gb = s_g1[row];
+        for (int c0 = 0; c0 < N1; c0 += 16) {
+          float v[16];
+          tmem_ld16(lane_addr + (uint32_t)c0, v);
+          const float gg = (c0 / R16) == 0 ? ga : gb;
+          uint32_t hi[8], lo[8];
 #pragma unroll
-      for (int kk = 0; kk < TC_BK / 16; ++kk)
-        mma_bf16(tmem, desc_k_sw128(xs + kk * 32), desc_k_sw128(as + kk * 32), id1, (c > 0 || kk > 0) ? 1u : 0u);
-      mma_commit(bar_empty + 8 * s);
-    };
-    const uint32_t g0 = gchunk;
-    constexpr int LAG = TC_STAGES - 1;
-    for (int c = 0; c < nk && !abort; ++c) {
-      const uint32_t g = g0 + c;
-      const uint32_t s = g % TC_STAGES;
-      if (g >= TC_STAGES) {                      // the MMAs of this stage's previous fill are done
-        if (!mbar_wait(bar_empty + 8 * s, ((g / TC_STAGES) - 1) & 1)) { abort = true; break; }
-      }
-      // x rows: 8 lanes cover one row's 128-byte segment, a warp 4 rows per instruction
+          for (int i = 0; i < 8; ++i) {
+            const float a0 = v[2 * i] * gg, a1 = v[2 * i + 1] * gg;
+            const __nv_bfloat162 h = __floats2bfloat162_rn(a0, a1);
+            const float2 hf = __bfloat1622float2(h);
+            hi[i] = *reinterpret_cast<const uint32_t*>(&h);
+            lo[i] = pack_bf16x2(a0 - hf.x, a1 - hf.y);
+          }
 #pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        const int w = tid + m * TC_THREADS;
-        const int row = w >> 3, q = w & 7;
-        const int tok = s_tok[row];
-        if (tok >= 0) {
-          const uint32_t dst = sU + s * TC_STAGE_BYTES + (uint32_t)row * 128 + ((q ^ (row & 7)) << 4);
-          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst),
-                       "l"(x + (size_t)tok * d_in + (size_t)c * TC_BK + q * 8)
-                       : "memory");
-        }
-      }
-      const uint32_t abase = sU + s * TC_STAGE_BYTES + TC_BM * 128;
-      for (int w = tid; w < N1 * 8; w += TC_THREADS) {
-        const int j = w >> 3, q = w & 7;
-        const int slot = j / R16, r = j % R16;
-        const uint32_t dst = abase + (uint32_t)j * 128 + ((q ^ (j & 7)) << 4);
-        const bool valid = r < rk[slot];
-        cp_async16_zfill(dst, valid ? Aj[slot] + (size_t)r * d_in + (size_t)c * TC_BK + q * 8 : Aj[0], valid);
-      }
-      cp_async_arrive(bar_full + 8 * s);
-      if (tid == 0 && c >= LAG) consume(g0 + c - LAG, c - LAG);
-    }
-    if (tid == 0 && !abort) {
-      for (int c = max(0, nk - LAG); c < nk && !abort; ++c) consume(g0 + c, c);
-      if (!abort) mma_commit(bar_d1);
-    }
-    gchunk = g0 + nk;
-    abort = __syncthreads_or(abort);
-    if (abort) break;
-    if (!mbar_wait(bar_d1, ph_d1)) abort = true;
-    ph_d1 ^= 1;
-    abort = __syncthreads_or(abort);
-    tc_fence_after();
-    if (abort) break;
-
-    // ------------------------------------------------------------ gates -> V (bf16 hi + lo)
-    {
-      const int row = tid;                       // TMEM lane = token row
-      const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
-      const float ga = s_g0[row], gb = s_g1[row];
-      for (int c0 = 0; c0 < N1; c0 += 16) {
-        float v[16];
-        tmem_ld16(lane_addr + (uint32_t)c0, v);
-        const float g = (c0 / R16) == 0 ? ga : gb;
-        uint32_t hi[8], lo[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float a0 = v[2 * i] * g, a1 = v[2 * i + 1] * g;
-          const __nv_bfloat162 h = __floats2bfloat162_rn(a0, a1);
-          const float2 hf = __bfloat1622float2(h);
-          hi[i] = *reinterpret_cast<const uint32_t*>(&h);
-          lo[i] = pack_bf16x2(a0 - hf.x, a1 - hf.y);
-        }
-#pragma unroll
-        for (int h8 = 0; h8 < 2; ++h8) {
-          const int kc8 = (c0 >> 3) + h8;          // core matrix index along K
-          const uint32_t off = (uint32_t)(row >> 3) * sbo_v + (uint32_t)kc8 * 128 + (uint32_t)(row & 7) * 16;
-          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(sVH + off), "r"(hi[4 * h8]),
-                       "r"(hi[4 * h8 + 1]), "r"(hi[4 * h8 + 2]), "r"(hi[4 * h8 + 3])
-                       : "memory");
-          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(sVL + off), "r"(lo[4 * h8]),
-                       "r"(lo[4 * h8 + 1]), "r"(lo[4 * h8 + 2]), "r"(lo[4 * h8 + 3])
-                       : "memory");
-        }
-      }
-    }
-    fence_proxy_async();
-    tc_fence_before();
-    __syncthreads();
-
-    // ------------------------------------------------------------ expand
-    const __nv_bfloat16* Bj[2];
-    Bj[0] = reinterpret_cast<const __nv_bfloat16*>(a.proj[p].B[e0]);
-    Bj[1] = K == 2 ? reinterpret_cast<const __nv_bfloat16*>(a.proj[p].B[e1]) : Bj[0];
-    const __nv_bfloat16* __restrict__ yb = reinterpret_cast<const __nv_bfloat16*>(a.proj[p].y_base);
-    __nv_bfloat16* __restrict__ y = reinterpret_cast<__nv_bfloat16*>(a.proj[p].y);
-    const int nnt = (d_out + TC_NT - 1) / TC_NT;
-
-    // Bcat rows and y_base rows of tile nt into ring slot nt % NY (one cp.async group)
-    auto issue_tile = [&](int nt) {
-      const int slot = nt % TC_NY;
-      const int n0 = nt * TC_NT;
-      const int ncols = min(TC_NT, d_out - n0);
-      const uint32_t bbase = sB + (uint32_t)slot * TC_BBUF_BYTES;
-      const int cpr = K2 / 8;
-      for (int w = tid; w < TC_NT * cpr; w += TC_THREADS) {
-        const int n = w / cpr, q = w % cpr;
-        const int kslot = q / (R16 / 8), cq = q % (R16 / 8);
-        const uint32_t dst = bbase + (uint32_t)(n >> 3) * sbo_v + (uint32_t)q * 128 + (uint32_t)(n & 7) * 16;
-        const bool valid = n < ncols && cq * 8 < rk[kslot];
-        cp_async16_zfill(dst, valid ? Bj[kslot] + (size_t)(n0 + n) * rk[kslot] + cq * 8 : Bj[0], valid);
-      }
-      // this warp's 32 token rows: 16 lanes per 256-byte row segment, 2 rows per instruction
-      const uint32_t ybase = sY + (uint32_t)slot * TC_YBUF_BYTES;
-      const int lane = tid & 31;
-      const int ch = lane & 15;
-      if (ch * 8 < ncols) {
-#pragma unroll 4
-        for (int k2 = 0; k2 < 16; ++k2) {
-          const int row = warp * 32 + 2 * k2 + (lane >> 4);
-          const int tok = s_tok[row];
-          if (tok >= 0)
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(ybase + (uint32_t)row * TC_YSTRIDE + ch * 16),
-                         "l"(yb + (size_t)tok * d_out + n0 + ch * 8)
+          for (int h8 = 0; h8 < 2; ++h8) {
+            const int kc8 = (c0 >> 3) + h8;
+            const uint32_t off = (uint32_t)(row >> 3) * sbo_v + (uint32_t)kc8 * 128 + (uint32_t)(row & 7) * 16;
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(sVH + off), "r"(hi[4 * h8]),
+                         "r"(hi[4 * h8 + 1]), "r"(hi[4 * h8 + 2]), "r"(hi[4 * h8 + 3])
                          : "memory");
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(sVL + off), "r"(lo[4 * h8]),
+                         "r"(lo[4 * h8 + 1]), "r"(lo[4 * h8 + 2]), "r"(lo[4 * h8 + 3])
+                         : "memory");
+          }
         }
+        fence_proxy_async();
+        tc_fence_before();
+        mbar_arrive(bar_v);
       }
-    };
-
-    for (int nt = 0; nt < TC_NY - 1; ++nt) {
-      if (nt < nnt) issue_tile(nt);
-      cp_async_commit();
-    }
-    for (int nt = 0; nt < nnt; ++nt) {
-      const int b = nt & 1;
-      const int slot = nt % TC_NY;
-      const int n0 = nt * TC_NT;
-      const int ncols = min(TC_NT, d_out - n0);
-      if (nt + TC_NY - 1 < nnt) issue_tile(nt + TC_NY - 1);
-      cp_async_commit();
-      cp_async_wait<TC_NY - 1>();                 // tile nt's group has landed (this thread)
-      __syncthreads();                            // ... and every thread's
-      if (tid == 0) {
+      // -------------------------------------------------------- expand operands and epilogues
+      const __nv_bfloat16* Bj[2];
+      Bj[0] = reinterpret_cast<const __nv_bfloat16*>(a.proj[p].B[e0]);
+      Bj[1] = K == 2 ? reinterpret_cast<const __nv_bfloat16*>(a.proj[p].B[e1]) : Bj[0];
+      __nv_bfloat16* __restrict__ y = reinterpret_cast<__nv_bfloat16*>(a.proj[p].y);
+      auto issue_tile = [&](int nt) {
+        const uint32_t slot = (t0 + nt) % TC_NY;
+        const int n0 = nt * TC_NT;
+        const int ncols = min(TC_NT, d_out - n0);
+        const uint32_t bbase = sB + slot * TC_BBUF_BYTES;
+        const int cpr = K2 / 8;
+        for (int w = tid; w < TC_NT * cpr; w += TC_WORKERS) {
+          const int n = w / cpr, q = w % cpr;
+          const int kslot = q / (R16 / 8), cq = q % (R16 / 8);
+          const uint32_t dst = bbase + (uint32_t)(n >> 3) * sbo_v + (uint32_t)q * 128 + (uint32_t)(n & 7) * 16;
+          const bool valid = n < ncols && cq * 8 < rk[kslot];
+          cp_async16_zfill(dst, valid ? Bj[kslot] + (size_t)(n0 + n) * rk[kslot] + cq * 8 : Bj[0], valid);
+        }
+        cp_async_arrive(bar_tfull + 8 * slot);
+        // y_base rows of this warp's tokens: TMA gathers into the two swizzled 64-column halves
+        if (lane == 0) {
+          bulk_wait_read_all();                    // this warp's stores from the slot are read out
+          const uint32_t tb = bar_tfull + 8 * slot;
+          const int nh = (ncols + 63) / 64;
+          mbar_arrive_expect_tx(tb, nh * 8 * 4 * 128);
+          for (int h = 0; h < nh; ++h) {
+            const uint32_t ydst = sY + slot * TC_YBUF_BYTES + h * (TC_BM * 128) + (uint32_t)(warp * 32) * 128;
+#pragma unroll
+            for (int g4 = 0; g4 < 8; ++g4)
+              tma_gather4(ydst + g4 * 512, &args.tm_yb[p], n0 + 64 * h, trow[4 * g4], trow[4 * g4 + 1],
+                          trow[4 * g4 + 2], trow[4 * g4 + 3], tb);
+          }
+        }
+      };
+      for (int nt = 0; nt < TC_NY - 1 && nt < nnt && !abort; ++nt) issue_tile(nt);
+      for (int nt = 0; nt < nnt && !abort; ++nt) {
+        const uint32_t g = t0 + nt;
+        const uint32_t slot = g % TC_NY, b = g & 1;
+        const int n0 = nt * TC_NT;
+        const int ncols = min(TC_NT, d_out - n0);
+        if (nt + TC_NY - 1 < nnt) issue_tile(nt + TC_NY - 1);   // slot of tile nt-1: consumed
+        if (!mbar_wait(bar_tfull + 8 * slot, (g / TC_NY) & 1)) { abort = true; break; }
+        if (!mbar_wait(bar_d2full + 8 * b, (g >> 1) & 1)) { abort = true; break; }
         tc_fence_after();
-        const uint32_t bb = sB + (uint32_t)slot * TC_BBUF_BYTES;
-        const uint32_t dcol = tmem + TC_D2_COL + (uint32_t)b * TC_NT;
-        for (int kk = 0; kk < K2 / 16; ++kk)
-          mma_bf16(dcol, desc_k_plain(sVH + kk * 256, 128, sbo_v), desc_k_plain(bb + kk * 256, 128, sbo_v), id2,
-                   kk > 0 ? 1u : 0u);
-        for (int kk = 0; kk < K2 / 16; ++kk)
-          mma_bf16(dcol, desc_k_plain(sVL + kk * 256, 128, sbo_v), desc_k_plain(bb + kk * 256, 128, sbo_v), id2, 1u);
-        mma_commit(bar_mma2 + 8 * b);
-      }
-      if (!mbar_wait(bar_mma2 + 8 * b, (ph_mma2 >> b) & 1)) abort = true;
-      ph_mma2 ^= 1u << b;
-      tc_fence_after();
-      abort = __syncthreads_or(abort);
-      if (abort) break;
-      // epilogue: y = y_base + D2 in this thread's token row (one rounding) ...
-      {
-        const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16) + TC_D2_COL + (uint32_t)b * TC_NT;
-        unsigned char* yrow = sYp + (size_t)slot * TC_YBUF_BYTES + (size_t)tid * TC_YSTRIDE;
+        const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16) + TC_D2_COL + b * TC_NT;
+        unsigned char* yslot = sYp + (size_t)slot * TC_YBUF_BYTES;
+        const int sw = tid & 7;
+        const bool mine = s_tok[tid] >= 0;
         for (int c0 = 0; c0 < ncols; c0 += 16) {
           float v[16];
           tmem_ld16(lane_addr + (uint32_t)c0, v);
-          if (my_tok >= 0) {
-            uint4* pr = reinterpret_cast<uint4*>(yrow + c0 * 2);
-            uint4 u0 = pr[0], u1 = pr[1];
+          if (mine) {
+            const int h = c0 >> 6, q = (c0 & 63) >> 3;
+            unsigned char* rbase = yslot + (size_t)h * (TC_BM * 128) + (size_t)tid * 128;
+            uint4* p0 = reinterpret_cast<uint4*>(rbase + ((q ^ sw) << 4));
+            uint4* p1 = reinterpret_cast<uint4*>(rbase + (((q + 1) ^ sw) << 4));
+            uint4 u0 = *p0, u1 = *p1;
             __nv_bfloat162* h0 = reinterpret_cast<__nv_bfloat162*>(&u0);
             __nv_bfloat162* h1 = reinterpret_cast<__nv_bfloat162*>(&u1);
 #pragma unroll
@@ -488,36 +501,84 @@ __global__ void __launch_bounds__(TC_THREADS, 1) sgmm_tc_kernel(TcArgs args) {
               h0[i] = __floats2bfloat162_rn(f0.x + v[2 * i], f0.y + v[2 * i + 1]);
               h1[i] = __floats2bfloat162_rn(f1.x + v[8 + 2 * i], f1.y + v[8 + 2 * i + 1]);
             }
-            pr[0] = u0;
-            pr[1] = u1;
+            *p0 = u0;
+            *p1 = u1;
           }
+        }
+        tc_fence_before();
+        mbar_arrive(bar_d2empty + 8 * b);          // D2[b] may be overwritten
+        // rows of a 4-row group with a missing token are written by their owners ...
+        const int g4 = (tid & 31) >> 2;
+        const bool full_group = s_tok[warp * 32 + 4 * g4] >= 0 && s_tok[warp * 32 + 4 * g4 + 1] >= 0 &&
+                                s_tok[warp * 32 + 4 * g4 + 2] >= 0 && s_tok[warp * 32 + 4 * g4 + 3] >= 0;
+        if (mine && !full_group) {
+          for (int qq = 0; qq < ncols / 8; ++qq) {
+            const int h = qq >> 3, q = qq & 7;
+            const uint4 val = *reinterpret_cast<const uint4*>(yslot + (size_t)h * (TC_BM * 128) + (size_t)tid * 128 +
+                                                              ((q ^ sw) << 4));
+            *reinterpret_cast<uint4*>(y + (size_t)s_tok[tid] * d_out + n0 + qq * 8) = val;
+          }
+        }
+        // ... and full groups leave by TMA scatter, 4 rows x 64 columns per instruction
+        fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) {
+          const int nh = (ncols + 63) / 64;
+          for (int gg = 0; gg < 8; ++gg) {
+            const int r = warp * 32 + 4 * gg;
+            if (s_tok[r] < 0 || s_tok[r + 1] < 0 || s_tok[r + 2] < 0 || s_tok[r + 3] < 0) continue;
+            for (int h = 0; h < nh; ++h)
+              tma_scatter4(&args.tm_y[p], n0 + 64 * h, s_tok[r], s_tok[r + 1], s_tok[r + 2], s_tok[r + 3],
+                           smem_u32(yslot + (size_t)h * (TC_BM * 128) + (size_t)r * 128));
+          }
+          bulk_commit();
         }
         __syncwarp();
-        // ... then the warp writes its 32 rows back, 2 rows (2 x 256 bytes) per instruction
-        const int lane = tid & 31;
-        const int ch = lane & 15;
-        if (ch * 8 < ncols) {
-#pragma unroll 4
-          for (int k2 = 0; k2 < 16; ++k2) {
-            const int row = warp * 32 + 2 * k2 + (lane >> 4);
-            const int tok = s_tok[row];
-            if (tok >= 0) {
-              const uint4 val = *reinterpret_cast<const uint4*>(sYp + (size_t)slot * TC_YBUF_BYTES +
-                                                               (size_t)row * TC_YSTRIDE + ch * 16);
-              __stcs(reinterpret_cast<uint4*>(y + (size_t)tok * d_out + n0 + ch * 8), val);
-            }
-          }
-        }
       }
-      tc_fence_before();
-      __syncthreads();
+      // the next item's stages overlay the y ring: this warp's stores must have read it out
+      if (lane == 0) bulk_wait_read_all();
+      cp_async_wait_all();
+    } else if (lane == 0) {
+      // -------------------------------------------------------- MMA issue (one thread)
+      for (int c = 0; c < nk && !abort; ++c) {
+        const uint32_t g = g0 + c;
+        const uint32_t s = g % TC_STAGES;
+        if (!mbar_wait(bar_full + 8 * s, (g / TC_STAGES) & 1)) { abort = true; break; }
+        tc_fence_after();
+        const uint32_t xs = sU + s * TC_STAGE_BYTES;
+        const uint32_t as = xs + TC_BM * 128;
+#pragma unroll
+        for (int kk = 0; kk < TC_BK / 16; ++kk)
+          mma_bf16(tmem, desc_k_sw128(xs + kk * 32), desc_k_sw128(as + kk * 32), id1, (c > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(bar_empty + 8 * s);
+      }
+      if (!abort) mma_commit(bar_d1);
+      if (!abort && !mbar_wait(bar_v, nitem & 1)) abort = true;
+      tc_fence_after();
+      for (int nt = 0; nt < nnt && !abort; ++nt) {
+        const uint32_t g = t0 + nt;
+        const uint32_t slot = g % TC_NY, b = g & 1;
+        if (!mbar_wait(bar_tfull + 8 * slot, (g / TC_NY) & 1)) { abort = true; break; }
+        if (g >= 2 && !mbar_wait(bar_d2empty + 8 * b, ((g >> 1) - 1) & 1)) { abort = true; break; }
+        tc_fence_after();
+        const uint32_t bb = sB + slot * TC_BBUF_BYTES;
+        const uint32_t dcol = tmem + TC_D2_COL + b * TC_NT;
+        for (int kk = 0; kk < K2 / 16; ++kk)
+          mma_bf16(dcol, desc_k_plain(sVH + kk * 256, 128, sbo_v), desc_k_plain(bb + kk * 256, 128, sbo_v), id2,
+                   kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < K2 / 16; ++kk)
+          mma_bf16(dcol, desc_k_plain(sVL + kk * 256, 128, sbo_v), desc_k_plain(bb + kk * 256, 128, sbo_v), id2, 1u);
+        mma_commit(bar_d2full + 8 * b);
+      }
     }
-    // the ring area is reused by the next item's shrink stages
-    cp_async_wait_all();
-    __syncthreads();
+    gchunk = g0 + nk;
+    gtile = t0 + nnt;
+    ++nitem;
+    abort = __syncthreads_or(abort);
   }
   if (abort && tid == 0) report(a.ws, APR_ERR_TIMEOUT, K_TC, (int)blockIdx.x);
   cp_async_wait_all();
+  if (lane == 0) bulk_wait_all();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -541,6 +602,33 @@ bool sgmm_tensor_supported(const SgmmArgs& a, int dtype) {
   return true;
 }
 
+// cuTensorMapEncodeTiled, fetched through the runtime (no link against libcuda).
+static PFN_cuTensorMapEncodeTiled tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled>(p);
+  });
+  return fn;
+}
+
+// Row-major bf16 [rows, cols] matrix seen by TMA as boxes of one row x 64
+// columns (128 bytes) with the 128-byte swizzle; reads past the last row or
+// column return zeros, writes there are dropped.
+static bool encode_rows(PFN_cuTensorMapEncodeTiled enc, CUtensorMap* m, const void* base, int rows, int cols) {
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  const cuuint32_t box[2] = {64, 1};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 cudaError_t launch_sgmm_tensor(const SgmmArgs& a, cudaStream_t s) {
   static bool configured = false;
   if (!configured) {
@@ -549,18 +637,27 @@ cudaError_t launch_sgmm_tensor(const SgmmArgs& a, cudaStream_t s) {
     if (err != cudaSuccess) return err;
     configured = true;
   }
+  PFN_cuTensorMapEncodeTiled enc = tensor_map_encoder();
+  if (!enc) return cudaErrorNotSupported;
   int dev = 0, nsm = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
   TcArgs t;
+  memset(&t, 0, sizeof(t));
   t.a = a;
   t.R16 = round16(a.max_rank);
   t.N1 = a.k * t.R16;
+  if (!encode_rows(enc, &t.tm_x, a.x, a.T, a.d_in)) return cudaErrorInvalidValue;
+  for (int p = 0; p < a.nproj; ++p) {
+    if (!encode_rows(enc, &t.tm_yb[p], a.proj[p].y_base, a.T, a.proj[p].d_out) ||
+        !encode_rows(enc, &t.tm_y[p], a.proj[p].y, a.T, a.proj[p].d_out))
+      return cudaErrorInvalidValue;
+  }
   // upper bound on items: set tiles <= T (one per token at worst); the kernel loops over the real count
   long max_items = (long)((a.T + TC_BM - 1) / TC_BM + a.T) * a.nproj;
   int grid = nsm;
   if (max_items < grid) grid = (int)max_items;
-  return launch_pdl(sgmm_tc_kernel, dim3(grid), dim3(TC_THREADS), TcSmem::ALLOC, s, t);
+  return launch_pdl(sgmm_tc_kernel, dim3(grid), dim3(TC_BLOCK), TcSmem::ALLOC, s, t);
 }
 
 

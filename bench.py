@@ -29,6 +29,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "mixture-of-LoRA SGMM tokens/s at 1 B200; % of HBM / tensor-core roofline"
+W_CONFIG_LAYERS = {"tiny": 4, "decode": 32, "prefill": 32, "multitenant": 32, "merge": 32}
 DESCR = {
     "decode": "decode: Llama-2-7B layer set (32 layers; q,k,v,o 4096->4096; gate,up 4096->11008; "
               "down 11008->4096), 8 adapters rank 16, top-2 pre-gate, 32 tokens/step, uniform, bf16",
@@ -131,14 +132,23 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(value, world):
+def max_over_ranks(value, world, device=None):
+    """Largest value over all ranks (the job's wall time is its slowest rank's)."""
     if world == 1:
         return value
     import torch
     import torch.distributed as dist
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    if device is None:
+        device = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate_throughput(units_per_rank, ms_local, world, device=None):
+    """Whole-job throughput: units processed by all ranks / the slowest rank's time."""
+    ms = max_over_ranks(ms_local, world, device)
+    return units_per_rank * world / (ms / 1e3), ms
 
 
 # ---------------------------------------------------------------- CPU oracle leg
@@ -259,7 +269,11 @@ def run_reference(args, world, rank):
 
 
 def config_block(cfg, world):
-    return {"workload": DESCR.get(cfg.name, cfg.name), "name": cfg.name, "tokens_per_step": cfg.T,
+    full = W_CONFIG_LAYERS.get(cfg.name, cfg.layers)
+    descr = DESCR.get(cfg.name, cfg.name)
+    if cfg.layers != full:
+        descr += f" [REDUCED: {cfg.layers} of {full} layers, profiling only]"
+    return {"workload": descr, "name": cfg.name, "tokens_per_step": cfg.T,
             "adapters": cfg.E, "top_k": cfg.k, "ranks": list(cfg.rank_choices), "layers": cfg.layers,
             "parallelism": f"replicas x{world} (token batches, no collective)",
             "l2": "working set larger than the 126 MB L2 (every layer has its own buffers); no flush"}
@@ -274,6 +288,8 @@ def run_gpu(args, world, rank, local):
     from adapter_pregate_router_b200 import workloads as W
 
     cfg = W.scaled(W.CONFIGS[args.workload], seed=W.CONFIGS[args.workload].seed + rank)
+    if args.layers:
+        cfg = W.scaled(cfg, layers=args.layers)
     peaks = load_peaks()
     dev = torch.device("cuda", local)
     step = pipeline.Step(cfg, device=dev)
@@ -320,11 +336,8 @@ def run_gpu(args, world, rank, local):
         stream.synchronize()
     torch.cuda.synchronize(dev)
     barrier(world)
-    ms = ev0.elapsed_time(ev1)
-    ms = max_over_ranks(ms, world)
+    value, ms = aggregate_throughput(cfg.T * args.steps, ev0.elapsed_time(ev1), world)
     ms_step = ms / args.steps
-    tokens_total = cfg.T * args.steps * world
-    value = tokens_total / (ms / 1e3)
     apr.stream_status(step.ws, stream)
 
     # ---- the dominant kernel class timed alone (every layer call, no route)
@@ -410,6 +423,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-budget", type=float, default=12.0, help="seconds of oracle work per reference step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="build only this many layers (a reduced workload for profiling; not the benchmark)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

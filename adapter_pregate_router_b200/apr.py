@@ -30,6 +30,7 @@ APR_BF16 = 1
 SGMM_AUTO = 0
 SGMM_SKINNY = 1
 SGMM_TENSOR = 2
+SGMM_DENSE = 3
 
 MAX_E = 1024
 MAX_K = 8

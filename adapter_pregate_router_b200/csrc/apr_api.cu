@@ -69,7 +69,7 @@ size_t apr_workspace_size(int T, int k, int E, int max_rank, int max_d_in) {
     return 0;
   const WsLayout L = ws_layout(T, k, E);
   size_t scratch = route_scratch_bytes(T, E);
-  const size_t sg = sgmm_scratch_bytes(T, k, max_rank, max_d_in);
+  const size_t sg = sgmm_scratch_bytes(T, k, E, max_rank, max_d_in);
   if (sg > scratch) scratch = sg;
   return L.scratch + align_up(scratch) + kAlign;
 }
@@ -148,7 +148,7 @@ apr_status apr_sgmm_shrink_expand(const void* x, int d_in, const apr_proj* projs
   if (d_in < 8 || (d_in & 7)) return fail(APR_ERR_INVALID_ARG, "sgmm: d_in=%d must be a positive multiple of 8", d_in);
   if (max_rank < 8 || max_rank > APR_MAX_RANK || (max_rank & 7))
     return fail(APR_ERR_INVALID_ARG, "sgmm: max_rank=%d must be a multiple of 8 in [8, %d]", max_rank, APR_MAX_RANK);
-  if (kernel < APR_SGMM_AUTO || kernel > APR_SGMM_TENSOR) return fail(APR_ERR_INVALID_ARG, "sgmm: bad kernel %d", kernel);
+  if (kernel < APR_SGMM_AUTO || kernel > APR_SGMM_DENSE) return fail(APR_ERR_INVALID_ARG, "sgmm: bad kernel %d", kernel);
   for (int p = 0; p < nproj; ++p) {
     const apr_proj& pj = projs[p];
     if (pj.d_out < 8 || (pj.d_out & 7)) return fail(APR_ERR_INVALID_ARG, "sgmm: proj %d d_out=%d must be a positive multiple of 8", p, pj.d_out);
@@ -159,7 +159,7 @@ apr_status apr_sgmm_shrink_expand(const void* x, int d_in, const apr_proj* projs
   if (!x || !ranks || !idx || !gate || !seg_off || !perm) return fail(APR_ERR_INVALID_ARG, "sgmm: NULL pointer");
   if (!aligned16(x)) return fail(APR_ERR_INVALID_ARG, "sgmm: x not 16-byte aligned");
   const WsLayout L = ws_layout(T, k, E);
-  st = check_ws(ws, ws_bytes, L.scratch + sgmm_scratch_bytes(T, k, max_rank, d_in), "sgmm");
+  st = check_ws(ws, ws_bytes, L.scratch + sgmm_scratch_bytes(T, k, E, max_rank, d_in), "sgmm");
   if (st) return st;
 
   SgmmArgs a;
@@ -187,12 +187,18 @@ apr_status apr_sgmm_shrink_expand(const void* x, int d_in, const apr_proj* projs
 
   int use = kernel;
   if (use == APR_SGMM_AUTO) {
-    // mean pairs per adapter, known on the host without reading the routing
+    // by the shapes and the mean pairs per adapter, known on the host without reading the routing
     const double mean_seg = (double)T * k / E;
-    use = (mean_seg >= 256.0 && sgmm_tensor_supported(a, dtype)) ? APR_SGMM_TENSOR : APR_SGMM_SKINNY;
+    if (sgmm_dense_supported(a, dtype)) use = APR_SGMM_DENSE;
+    else if (mean_seg >= 256.0 && sgmm_tensor_supported(a, dtype)) use = APR_SGMM_TENSOR;
+    else use = APR_SGMM_SKINNY;
   }
   cudaError_t e;
-  if (use == APR_SGMM_TENSOR) {
+  if (use == APR_SGMM_DENSE) {
+    if (!sgmm_dense_supported(a, dtype))
+      return fail(APR_ERR_UNSUPPORTED, "sgmm: dense kernel needs bf16, T<=64, E<=16, E*round16(max_rank)<=256");
+    e = launch_sgmm_dense(a, L.scratch, (cudaStream_t)stream);
+  } else if (use == APR_SGMM_TENSOR) {
     if (!sgmm_tensor_supported(a, dtype))
       return fail(APR_ERR_UNSUPPORTED, "sgmm: tensor-core kernel needs bf16, k<=2, max_rank<=64, d_in%%64==0, d_out%%16==0");
     e = launch_sgmm_tensor(a, (cudaStream_t)stream);

@@ -78,9 +78,28 @@ inline size_t route_scratch_bytes(int T, int E) {
 
 inline int shrink_kchunks(int d_in) { return (d_in + kShrinkKC - 1) / kShrinkKC; }
 
-// Shrink partial sums: [projection][column chunk][sorted pair][rank] fp32.
-inline size_t sgmm_scratch_bytes(int T, int k, int max_rank, int d_in) {
-  return sizeof(float) * APR_MAX_PROJ * (size_t)shrink_kchunks(d_in) * T * k * max_rank;
+// Dense small-batch path: up to 64 tokens and an adapter bank of at most 16
+// adapters whose rank slots (max rank rounded up to 16) add up to <= 256 rows;
+// d_in is split over clusters of 8 CTAs x 256 columns.
+constexpr int kDenseMaxT = 64;
+constexpr int kDenseMaxRows = 256;
+constexpr int kDenseClusterCols = 8 * 256;
+inline int round16i(int v) { return (v + 15) / 16 * 16; }
+inline bool dense_dims_ok(int T, int E, int max_rank) {
+  return T >= 1 && T <= kDenseMaxT && E <= 16 && E * round16i(max_rank) <= kDenseMaxRows;
+}
+inline int dense_clusters(int d_in) { return (d_in + kDenseClusterCols - 1) / kDenseClusterCols; }
+
+// Shrink partial sums.  Gather paths: [projection][column chunk][sorted pair][rank]
+// fp32; dense path: [projection][cluster][token (padded to 16)][adapter * rank slot].
+inline size_t sgmm_scratch_bytes(int T, int k, int E, int max_rank, int d_in) {
+  size_t b = sizeof(float) * APR_MAX_PROJ * (size_t)shrink_kchunks(d_in) * T * k * max_rank;
+  if (dense_dims_ok(T, E, max_rank)) {
+    const size_t d = sizeof(float) * APR_MAX_PROJ * (size_t)dense_clusters(d_in) * round16i(T) * E *
+                     round16i(max_rank);
+    if (d > b) b = d;
+  }
+  return b;
 }
 
 template <typename P>
@@ -230,6 +249,8 @@ struct SgmmArgs {
 };
 cudaError_t launch_sgmm_skinny(const SgmmArgs& a, int dtype, size_t scratch_off, cudaStream_t s);
 cudaError_t launch_sgmm_tensor(const SgmmArgs& a, cudaStream_t s);
+cudaError_t launch_sgmm_dense(const SgmmArgs& a, size_t scratch_off, cudaStream_t s);
+bool sgmm_dense_supported(const SgmmArgs& a, int dtype);
 bool sgmm_tensor_supported(const SgmmArgs& a, int dtype);
 cudaError_t launch_merge(const apr_merge_proj* projs, int nproj, int E, int r, const int32_t* idx,
                          const float* gate, int k, void* ws, cudaStream_t s);

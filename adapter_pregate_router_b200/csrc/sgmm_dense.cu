@@ -1,0 +1,434 @@
+// SGMM for small batches (decode) as two dense tcgen05 products over the whole
+// adapter bank.  AdaFuse summary (gist.science), Resumen tecnico §2.B: the
+// segmented gather product applies the pre-gated adapters of every token and
+// is fused into the add onto the base projection output.
+//
+// With a few dozen tokens the gather buys nothing: every adapter is selected
+// by some token, so all of A and B is read anyway, and the cost of a call is
+// its latency.  Both products therefore run densely over the E adapters
+// (rank slots padded to Rp, a multiple of 16), and the gates zero what a token
+// did not select:
+//
+//  shrink  U[e*Rp + i, t] = (A_e x_t)_i for all e, t.  The input columns are
+//          split over clusters of 8 CTAs, 256 columns per CTA; each CTA stages
+//          its slice of every A_e (before the PDL wait: weights never depend
+//          on the preceding launch) and of x (after it) in 128B-swizzled
+//          K-major tiles, and one thread issues the tcgen05 MMAs
+//          D[NR x Tp] = A_slice . x_slice^T (A as the M side, tokens as N).
+//          The 8 partial products are summed in a fixed order through
+//          distributed shared memory, gated
+//          V[t, e*Rp + i] = sum_j [idx[t,j] = e] g[t,j] U[e*Rp + i, t]
+//          and written as fp32 partials per cluster: [proj][cluster][Tp][NR].
+//  expand  one CTA per 128 output columns: D[128 x Tp] = Bslice . V^T with
+//          Bslice[n, e*Rp + i] = B_e[n, i] (staged before the wait, with the
+//          y_base columns) and V summed over the clusters in order and split
+//          into bf16 hi + lo halves (two MMAs keep ~16 mantissa bits of v).
+//          Thread n reads row n of D from TMEM and writes
+//          y[t, n] = y_base[t, n] + D[n, t], rounded to bf16 once.
+//
+// Every wait is bounded (1 s); an expired wait records APR_ERR_TIMEOUT and the
+// CTA still passes every cluster barrier and frees its TMEM.
+#include "apr_internal.cuh"
+#include "tc_ptx.cuh"
+
+namespace apr {
+
+constexpr int DN_THREADS = 256;
+constexpr int DN_KC = 256;        // input columns per shrink CTA (four 64-column swizzle atoms)
+constexpr int DN_CL = 8;          // shrink CTAs per cluster
+constexpr int DN_NT = 128;        // output columns per expand CTA
+
+struct DenseArgs {
+  SgmmArgs a;
+  int Tp;                              // tokens rounded up to 16 (MMA N)
+  int Rp;                              // rank slot per adapter (max rank rounded up to 16)
+  int NR;                              // E * Rp
+  int MR;                              // NR rounded up to 128 (shrink MMA M)
+  int ncl;                             // clusters along d_in
+  size_t vpart_off;                    // scratch offset of the gated partials
+  int tiles_before[APR_MAX_PROJ + 1];  // expand: prefix of 128-column tiles per projection
+};
+
+static_assert(DN_KC == 4 * 64, "four swizzle atoms per shrink CTA");
+
+__device__ __forceinline__ uint32_t tmem_cols_for(int n) {
+  uint32_t c = 32;
+  while ((int)c < n) c <<= 1;
+  return c;
+}
+
+__device__ __forceinline__ uint32_t cluster_map(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// ---------------------------------------------------------------- shrink
+
+__global__ void __launch_bounds__(DN_THREADS, 1) dense_shrink_kernel(const __grid_constant__ DenseArgs args) {
+  const SgmmArgs& a = args.a;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem =
+      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int rank = blockIdx.x;                    // rank in the cluster (cluster spans gridDim.x)
+  const int cl = blockIdx.y, p = blockIdx.z;
+  const int Tp = args.Tp, Rp = args.Rp, NR = args.NR, MR = args.MR;
+  const int T = a.T, K = a.k, E = a.E, d_in = a.d_in;
+  const int k0 = (cl * DN_CL + rank) * DN_KC;
+
+  // shared memory: A slice [4 atoms][MR][128 B], x slice [4 atoms][Tp][128 B];
+  // after the MMAs the A area holds this CTA's partial product P[Tp][MR] fp32.
+  unsigned char* sA = smem;
+  unsigned char* sX = smem + (size_t)MR * 512;
+  unsigned char* meta = sX + (size_t)Tp * 512;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(meta);
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(meta + 8);
+  const __nv_bfloat16** s_Ap = reinterpret_cast<const __nv_bfloat16**>(meta + 16);   // [E]
+  int* s_rk = reinterpret_cast<int*>(meta + 16 + 8 * 16);                             // [E]
+  int* s_idx = s_rk + 16;                                                              // [T*K]
+  float* s_gate = reinterpret_cast<float*>(s_idx + 64 * APR_MAX_K);                   // [T*K]
+  float* P = reinterpret_cast<float*>(sA);
+
+  const uint32_t cs = tmem_cols_for(Tp);            // TMEM columns per M tile (a power of two)
+  const uint32_t ncols = (uint32_t)(MR / 128) * cs;
+  if (tid == 0) {
+    mbar_init(smem_u32(bar), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) tmem_alloc(smem_u32(s_tmem), ncols);
+  if (tid < E) {
+    s_Ap[tid] = reinterpret_cast<const __nv_bfloat16*>(a.proj[p].A[tid]);
+    const int r = a.ranks[tid];
+    const bool ok = r >= 8 && r <= Rp && (r & 7) == 0;
+    if (!ok) report(a.ws, APR_ERR_DEVICE_INDEX, K_SHRINK, tid);
+    s_rk[tid] = ok ? r : 0;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+
+  // A slice of every adapter (rows beyond a rank, or columns beyond d_in, are zeros)
+  {
+    const int q = tid & 31;                 // 16-byte column chunk
+    const int col = k0 + q * 8;
+    const bool col_ok = col < d_in;
+    int r = tid >> 5;
+    int e = r / Rp, i = r - e * Rp;
+    const uint32_t base = smem_u32(sA) + (uint32_t)(q >> 3) * (uint32_t)(MR * 128);
+    for (; r < MR; r += 8) {
+      const bool valid = col_ok && e < E && i < s_rk[e];
+      const void* src = valid ? (const void*)(s_Ap[e] + (size_t)i * d_in + col) : (const void*)a.x;
+      cp_async16_zfill(base + (uint32_t)r * 128 + ((((uint32_t)q & 7) ^ ((uint32_t)r & 7)) << 4), src, valid);
+      i += 8;
+      if (i >= Rp) { i -= Rp; ++e; }
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  }
+
+  pdl_wait();
+  pdl_trigger();
+
+  // x slice of the tokens, and their routing
+  {
+    const __nv_bfloat16* x = reinterpret_cast<const __nv_bfloat16*>(a.x);
+    const int q = tid & 31;
+    const int col = k0 + q * 8;
+    const uint32_t base = smem_u32(sX) + (uint32_t)(q >> 3) * (uint32_t)(Tp * 128);
+    for (int t = tid >> 5; t < Tp; t += 8) {
+      const bool valid = t < T && col < d_in;
+      const void* src = valid ? (const void*)(x + (size_t)t * d_in + col) : (const void*)a.x;
+      cp_async16_zfill(base + (uint32_t)t * 128 + ((((uint32_t)q & 7) ^ ((uint32_t)t & 7)) << 4), src, valid);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    for (int w = tid; w < T * K; w += DN_THREADS) {
+      s_idx[w] = a.idx[w];
+      s_gate[w] = a.gate[w];
+    }
+  }
+  cp_async_wait_all();
+  fence_proxy_async();
+  __syncthreads();
+
+  // D[MR x Tp] = A_slice . x_slice^T, one M tile of 128 rows at a time
+  if (tid == 0) {
+    tc_fence_after();
+    const uint32_t id = idesc_bf16(128, Tp);
+    for (int mt = 0; mt < MR / 128; ++mt)
+      for (int kk = 0; kk < DN_KC / 16; ++kk) {
+        const uint32_t aa = smem_u32(sA) + (uint32_t)(kk >> 2) * (uint32_t)(MR * 128) + (uint32_t)mt * 16384 +
+                            (uint32_t)(kk & 3) * 32;
+        const uint32_t bb = smem_u32(sX) + (uint32_t)(kk >> 2) * (uint32_t)(Tp * 128) + (uint32_t)(kk & 3) * 32;
+        mma_bf16(tmem + (uint32_t)mt * cs, desc_k_sw128(aa), desc_k_sw128(bb), id, kk > 0 ? 1u : 0u);
+      }
+    mma_commit(smem_u32(bar));
+  }
+  const bool done = mbar_wait(smem_u32(bar), 0);
+  tc_fence_after();
+  if (!done) {
+    if (tid == 0) report(a.ws, APR_ERR_TIMEOUT, K_SHRINK, (int)blockIdx.x);
+  } else {
+    // TMEM -> P[t][r] (the A slice is no longer read)
+    const int wq = warp & 3, wg = warp >> 2;
+    const int r_in = wq * 32 + lane;
+    for (int mt = 0; mt < MR / 128; ++mt) {
+      if (MR == 256 && mt != wg) continue;
+      for (int c8 = 0; c8 < Tp / 8; ++c8) {
+        if (MR == 128 && (c8 & 1) != wg) continue;
+        float v[8];
+        tmem_ld8(tmem + ((uint32_t)(wq * 32) << 16) + (uint32_t)mt * cs + (uint32_t)(c8 * 8), v);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) P[(size_t)(c8 * 8 + u) * MR + mt * 128 + r_in] = v[u];
+      }
+    }
+  }
+  tc_fence_before();
+  cluster_sync_all();          // every CTA's P is complete
+
+  // this CTA's share of the rows, summed over the cluster in rank order, gated
+  {
+    const int RS = MR / DN_CL;               // rows per CTA (16 or 32)
+    const int groups = RS / 4;
+    float* vpart = ws_at<float>(a.ws, args.vpart_off) + ((size_t)(p * args.ncl + cl) * Tp) * NR;
+    for (int w = tid; w < groups * Tp; w += DN_THREADS) {
+      const int t = w / groups, r0 = rank * RS + (w % groups) * 4;
+      const uint32_t off = smem_u32(P + (size_t)t * MR + r0);
+      float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int c = 0; c < DN_CL; ++c) {
+        const float4 v = ld_cluster_f4(cluster_map(off, (uint32_t)c));
+        s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+      }
+      if (r0 >= NR) continue;
+      const int e = r0 / Rp;
+      float g = 0.f;
+      if (t < T) {
+        for (int j = 0; j < K; ++j) {
+          const int ej = s_idx[t * K + j];
+          if (ej < 0 || ej >= E) {
+            if (rank == 0 && cl == 0 && r0 == 0) report(a.ws, APR_ERR_DEVICE_INDEX, K_SHRINK, ej);
+          } else if (ej == e) {
+            g += s_gate[t * K + j];
+          }
+        }
+      }
+      *reinterpret_cast<float4*>(vpart + (size_t)t * NR + r0) = make_float4(g * s.x, g * s.y, g * s.z, g * s.w);
+    }
+  }
+  cluster_sync_all();          // remote reads of P are over before any CTA leaves
+  if (warp == 0) tmem_dealloc(tmem, ncols);
+}
+
+// ---------------------------------------------------------------- expand
+
+__global__ void __launch_bounds__(DN_THREADS, 1) dense_expand_kernel(const __grid_constant__ DenseArgs args) {
+  const SgmmArgs& a = args.a;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem =
+      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int Tp = args.Tp, Rp = args.Rp, NR = args.NR;
+  const int T = a.T, E = a.E;
+  int p = 0;
+  while (p + 1 < a.nproj && (int)blockIdx.x >= args.tiles_before[p + 1]) ++p;
+  const int n0 = ((int)blockIdx.x - args.tiles_before[p]) * DN_NT;
+  const int d_out = a.proj[p].d_out;
+  const uint32_t SBO = (uint32_t)(NR / 8) * 128;     // next 8-row group of a K-major no-swizzle operand
+
+  // shared memory: Bslice [128 x NR], V hi / lo [Tp x NR] (bf16, 8x16-byte core matrices),
+  // y_base columns [Tp][128] bf16
+  unsigned char* sB = smem;
+  unsigned char* sVH = sB + (size_t)DN_NT * NR * 2;
+  unsigned char* sVL = sVH + (size_t)Tp * NR * 2;
+  __nv_bfloat16* sYB = reinterpret_cast<__nv_bfloat16*>(sVL + (size_t)Tp * NR * 2);
+  unsigned char* meta = reinterpret_cast<unsigned char*>(sYB + (size_t)Tp * DN_NT);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(meta);
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(meta + 8);
+  const __nv_bfloat16** s_Bp = reinterpret_cast<const __nv_bfloat16**>(meta + 16);   // [E]
+  int* s_rk = reinterpret_cast<int*>(meta + 16 + 8 * 16);                             // [E]
+
+  const uint32_t ncols = tmem_cols_for(Tp);
+  if (tid == 0) {
+    mbar_init(smem_u32(bar), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) tmem_alloc(smem_u32(s_tmem), ncols);
+  if (tid < E) {
+    s_Bp[tid] = reinterpret_cast<const __nv_bfloat16*>(a.proj[p].B[tid]);
+    const int r = a.ranks[tid];
+    s_rk[tid] = (r >= 8 && r <= Rp && (r & 7) == 0) ? r : 0;    // a bad rank is reported by the shrink
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+
+  // B slice of every adapter and the y_base columns: before the wait
+  {
+    const int kq_n = NR / 8, cq_n = Rp / 8;
+    for (int w = tid; w < DN_NT * kq_n; w += DN_THREADS) {
+      const int n = w / kq_n, kq = w - n * kq_n;
+      const int e = kq / cq_n, cq = kq - e * cq_n;
+      const bool valid = n0 + n < d_out && cq * 8 < s_rk[e];
+      const void* src = valid ? (const void*)(s_Bp[e] + (size_t)(n0 + n) * s_rk[e] + cq * 8) : (const void*)a.x;
+      cp_async16_zfill(smem_u32(sB) + (uint32_t)(n >> 3) * SBO + (uint32_t)kq * 128 + (uint32_t)(n & 7) * 16, src,
+                       valid);
+    }
+    const __nv_bfloat16* yb = reinterpret_cast<const __nv_bfloat16*>(a.proj[p].y_base);
+    for (int w = tid; w < T * (DN_NT / 8); w += DN_THREADS) {
+      const int t = w >> 4, c = (w & 15) * 8;
+      const bool valid = n0 + c < d_out;
+      cp_async16_zfill(smem_u32(sYB + (size_t)t * DN_NT + c),
+                       valid ? (const void*)(yb + (size_t)t * d_out + n0 + c) : (const void*)a.x, valid);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  }
+
+  pdl_wait();
+  pdl_trigger();
+
+  // V = sum over the clusters' gated partials (in order), split into bf16 hi + lo
+  {
+    const float* vp = ws_at<float>(a.ws, args.vpart_off) + (size_t)p * args.ncl * Tp * NR;
+    const int kq_n = NR / 8;
+    for (int w = tid; w < Tp * kq_n; w += DN_THREADS) {
+      const int t = w / kq_n, kq = w - t * kq_n;
+      float f[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      for (int c = 0; c < args.ncl; ++c) {
+        const float4* src = reinterpret_cast<const float4*>(vp + ((size_t)c * Tp + t) * NR + kq * 8);
+        const float4 u0 = __ldcg(src), u1 = __ldcg(src + 1);
+        f[0] += u0.x; f[1] += u0.y; f[2] += u0.z; f[3] += u0.w;
+        f[4] += u1.x; f[5] += u1.y; f[6] += u1.z; f[7] += u1.w;
+      }
+      uint32_t hi[4], lo[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+        const float2 hf = __bfloat1622float2(h);
+        hi[i] = *reinterpret_cast<const uint32_t*>(&h);
+        lo[i] = pack_bf16x2(f[2 * i] - hf.x, f[2 * i + 1] - hf.y);
+      }
+      const uint32_t off = (uint32_t)(t >> 3) * SBO + (uint32_t)kq * 128 + (uint32_t)(t & 7) * 16;
+      asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(sVH) + off), "r"(hi[0]), "r"(hi[1]),
+                   "r"(hi[2]), "r"(hi[3])
+                   : "memory");
+      asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(sVL) + off), "r"(lo[0]), "r"(lo[1]),
+                   "r"(lo[2]), "r"(lo[3])
+                   : "memory");
+    }
+  }
+  cp_async_wait_all();
+  fence_proxy_async();
+  __syncthreads();
+
+  if (tid == 0) {
+    tc_fence_after();
+    const uint32_t id = idesc_bf16(128, Tp);
+    for (int kk = 0; kk < NR / 16; ++kk)
+      mma_bf16(tmem, desc_k_plain(smem_u32(sB) + kk * 256, 128, SBO), desc_k_plain(smem_u32(sVH) + kk * 256, 128, SBO),
+               id, kk > 0 ? 1u : 0u);
+    for (int kk = 0; kk < NR / 16; ++kk)
+      mma_bf16(tmem, desc_k_plain(smem_u32(sB) + kk * 256, 128, SBO), desc_k_plain(smem_u32(sVL) + kk * 256, 128, SBO),
+               id, 1u);
+    mma_commit(smem_u32(bar));
+  }
+  const bool done = mbar_wait(smem_u32(bar), 0);
+  tc_fence_after();
+  if (!done) {
+    if (tid == 0) report(a.ws, APR_ERR_TIMEOUT, K_EXPAND, (int)blockIdx.x);
+  } else {
+    // thread n holds D[n][t] for its column: y[t, n0 + n] = y_base[t, n0 + n] + D[n, t]
+    __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(a.proj[p].y);
+    const int wq = warp & 3, wg = warp >> 2;
+    const int n = wq * 32 + lane;
+    const bool col_ok = n0 + n < d_out;
+    for (int c8 = wg; c8 < Tp / 8; c8 += 2) {
+      float v[8];
+      tmem_ld8(tmem + ((uint32_t)(wq * 32) << 16) + (uint32_t)(c8 * 8), v);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int t = c8 * 8 + u;
+        if (t < T && col_ok)
+          y[(size_t)t * d_out + n0 + n] = __float2bfloat16_rn(__bfloat162float(sYB[(size_t)t * DN_NT + n]) + v[u]);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, ncols);
+}
+
+// ---------------------------------------------------------------- host side
+
+static int dn_round16(int v) { return (v + 15) / 16 * 16; }
+
+bool sgmm_dense_supported(const SgmmArgs& a, int dtype) {
+  return dtype == APR_BF16 && dense_dims_ok(a.T, a.E, a.max_rank) && a.E <= 16 && a.k <= APR_MAX_K;
+}
+
+static size_t shrink_smem(int MR, int Tp) { return (size_t)MR * 512 + (size_t)Tp * 512 + 16 + 8 * 16 + 4 * 16 + 8 * 64 * APR_MAX_K + 1024; }
+static size_t expand_smem(int NR, int Tp) {
+  return (size_t)DN_NT * NR * 2 + 2 * (size_t)Tp * NR * 2 + (size_t)Tp * DN_NT * 2 + 16 + 8 * 16 + 4 * 16 + 128;
+}
+
+cudaError_t launch_sgmm_dense(const SgmmArgs& a, size_t scratch_off, cudaStream_t s) {
+  DenseArgs d;
+  memset(&d, 0, sizeof(d));
+  d.a = a;
+  d.Tp = dn_round16(a.T);
+  d.Rp = dn_round16(a.max_rank);
+  d.NR = a.E * d.Rp;
+  d.MR = d.NR <= 128 ? 128 : 256;
+  d.ncl = dense_clusters(a.d_in);
+  d.vpart_off = scratch_off;
+  d.tiles_before[0] = 0;
+  for (int p = 0; p < a.nproj; ++p) d.tiles_before[p + 1] = d.tiles_before[p] + (a.proj[p].d_out + DN_NT - 1) / DN_NT;
+
+  const size_t sm1 = shrink_smem(d.MR, d.Tp), sm2 = expand_smem(d.NR, d.Tp);
+  static size_t conf1 = 0, conf2 = 0;
+  cudaError_t err;
+  if (sm1 > conf1) {
+    if ((err = cudaFuncSetAttribute(dense_shrink_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1)) != cudaSuccess)
+      return err;
+    conf1 = sm1;
+  }
+  if (sm2 > conf2) {
+    if ((err = cudaFuncSetAttribute(dense_expand_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2)) != cudaSuccess)
+      return err;
+    conf2 = sm2;
+  }
+  {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(DN_CL, d.ncl, a.nproj);
+    cfg.blockDim = dim3(DN_THREADS);
+    cfg.dynamicSmemBytes = sm1;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = DN_CL;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    count_launch();
+    if ((err = cudaLaunchKernelEx(&cfg, dense_shrink_kernel, d)) != cudaSuccess) return err;
+  }
+  return launch_pdl(dense_expand_kernel, dim3(d.tiles_before[a.nproj]), dim3(DN_THREADS), sm2, s, d);
+}
+
+}  // namespace apr

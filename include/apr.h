@@ -66,9 +66,10 @@ typedef enum apr_dtype { APR_F32 = 0, APR_BF16 = 1 } apr_dtype;
 
 /* Kernel choice for apr_sgmm_shrink_expand. */
 typedef enum apr_sgmm_kernel {
-  APR_SGMM_AUTO = 0,    /* by the mean segment size T*k/E (known on the host) */
+  APR_SGMM_AUTO = 0,    /* by T, E, the ranks and the mean segment size T*k/E */
   APR_SGMM_SKINNY = 1,  /* CUDA-core kernel for few tokens per adapter        */
-  APR_SGMM_TENSOR = 2   /* tcgen05 tensor-core kernel for long segments       */
+  APR_SGMM_TENSOR = 2,  /* tcgen05 tensor-core kernel for long segments       */
+  APR_SGMM_DENSE = 3    /* tcgen05 over the whole adapter bank, small batches */
 } apr_sgmm_kernel;
 
 /* ------------------------------------------------------------------------
@@ -167,7 +168,11 @@ typedef struct apr_proj {
  *          must be the workspace that call wrote.
  * kernel   APR_SGMM_AUTO, or a forced kernel class.  The tensor-core kernel
  *          needs dtype == APR_BF16, k <= 2, max_rank <= 64, d_in % 64 == 0 and
- *          d_out % 16 == 0; it returns APR_ERR_UNSUPPORTED otherwise.
+ *          d_out % 16 == 0; the dense kernel needs dtype == APR_BF16, T <= 64,
+ *          E <= 16 and E * (max_rank rounded up to 16) <= 256; a forced kernel
+ *          returns APR_ERR_UNSUPPORTED outside its range.  AUTO takes the
+ *          dense kernel where it applies, the tensor-core kernel where
+ *          T*k/E >= 256, and the CUDA-core kernel otherwise.
  * T == 0 is a no-op.  Empty segments are legal.
  * ---------------------------------------------------------------------- */
 apr_status apr_sgmm_shrink_expand(const void* x, int d_in, const apr_proj* projs, int nproj,

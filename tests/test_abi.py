@@ -98,7 +98,7 @@ def test_sgmm_host_validation(apr):
     assert call(max_rank=12) == apr.APR_ERR_INVALID_ARG
     assert call(max_rank=136) == apr.APR_ERR_INVALID_ARG
     assert call(d_in=20) == apr.APR_ERR_INVALID_ARG
-    assert call(kernel=3) == apr.APR_ERR_INVALID_ARG
+    assert call(kernel=4) == apr.APR_ERR_INVALID_ARG
     assert call(x=None) == apr.APR_ERR_INVALID_ARG
     assert call(ws_bytes=256) == apr.APR_ERR_WORKSPACE
     bad = (apr.Proj * 1)(apr.Proj(0x1000, 0x1000, 60, 0x1000, 0x1000))
@@ -106,6 +106,9 @@ def test_sgmm_host_validation(apr):
     assert call(T=0) == apr.APR_OK
     # the tensor-core kernel refuses shapes outside its limits before launching
     assert call(kernel=2, dtype=0) == apr.APR_ERR_UNSUPPORTED
+    # so does the dense kernel (fp32, or more than 64 tokens)
+    assert call(kernel=3, dtype=0) == apr.APR_ERR_UNSUPPORTED
+    assert call(kernel=3, T=65) == apr.APR_ERR_UNSUPPORTED
 
 
 def test_merge_and_gemv_host_validation(apr):

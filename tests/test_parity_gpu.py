@@ -375,3 +375,78 @@ def test_sgmm_tensor_rejects_unsupported(apr):
     with pytest.raises(apr.AprError) as ei:
         run_sgmm(apr, x, As, Bs, idx, gate, ybs, BF16, kernel=apr.SGMM_TENSOR)
     assert ei.value.status == apr.APR_ERR_UNSUPPORTED
+
+
+# ------------------------------------------------------------------ SGMM, dense small-batch kernel
+
+
+@pytest.mark.parametrize("T,d_in,d_outs,ranks,k", [
+    (32, 4096, (4096, 4096, 4096), (16,) * 8, 2),          # a decode qkv group
+    (32, 11008, (4096,), (16,) * 8, 2),                    # the down projection: six clusters, the last ragged
+    (32, 4096, (11008, 11008), (16,) * 8, 2),              # gate/up: a ragged last output tile
+    (1, 2048, (136,), (8, 16, 24, 16), 2),                 # one token, mixed ranks, an 8-column tail tile
+    (64, 200, (72,), (16,) * 16, 3),                       # 256 rank rows (two M tiles); d_in not a multiple of 64
+    (17, 520, (264, 8), (64, 32, 8, 64), 1),               # rank slots of 64, k = 1, an 8-wide projection
+    (50, 1024, (128,), (128, 8), 2),                       # rank 128: two adapters fill 256 rows
+    (5, 64, (16,), (8,) * 3, 3),                           # k = E, fewer rank rows than one M tile
+])
+def test_sgmm_dense_parity(apr, T, d_in, d_outs, ranks, k):
+    rng = np.random.default_rng(T + d_in + k + 3)
+    x, As, Bs, idx, gate, ybs = _case(rng, T, d_in, d_outs, ranks, k)
+    x, As, Bs, ybs = _rounded(x, As, Bs, ybs)
+    for zero in (True, False):
+        yb = [np.zeros_like(y) for y in ybs] if zero else ybs
+        got = run_sgmm(apr, x, As, Bs, idx, gate, yb, BF16, kernel=apr.SGMM_DENSE)
+        ref = oracle_group(x, As, Bs, idx, gate.astype(np.float64), yb)
+        for p in range(len(d_outs)):
+            close(got[p], ref[p], f"dense proj {p} zero_ybase={zero}")
+
+
+def test_sgmm_dense_integer_inputs_exact(apr):
+    """Small integers, gates of 1/2: the dense result is the exact value rounded
+    once to bf16 (pins the adapter-slot and token indexing of both products)."""
+    rng = np.random.default_rng(31)
+    x, As, Bs, idx, gate, ybs = _case(rng, 40, 2560, (72, 136), (8, 16, 8, 24, 16), 2, ints=True)
+    got = run_sgmm(apr, x, As, Bs, idx, gate, ybs, BF16, kernel=apr.SGMM_DENSE)
+    ref = oracle_group(x, As, Bs, idx, gate.astype(np.float64), ybs)
+    for p in range(2):
+        want = bf16_exact(ref[p]).astype(np.float64)
+        assert np.array_equal(got[p], want), f"proj {p}: max diff {np.abs(got[p] - want).max()}"
+
+
+def test_sgmm_dense_properties(apr):
+    """Zero B leaves y_base bit-exact; in place equals out of place; a token
+    permutation permutes the output bits; two runs agree bit for bit; the dense
+    and CUDA-core kernels agree within one bf16 rounding."""
+    rng = np.random.default_rng(32)
+    x, As, Bs, idx, gate, ybs = _case(rng, 50, 4096, (512,), (16,) * 8, 2)
+    x, As, Bs, ybs = _rounded(x, As, Bs, ybs)
+    Bz = [[np.zeros_like(b) for b in P] for P in Bs]
+    z = run_sgmm(apr, x, As, Bz, idx, gate, ybs, BF16, kernel=apr.SGMM_DENSE)[0]
+    assert np.array_equal(z, ybs[0].astype(np.float64))
+    a = run_sgmm(apr, x, As, Bs, idx, gate, ybs, BF16, kernel=apr.SGMM_DENSE, in_place=True)[0]
+    b = run_sgmm(apr, x, As, Bs, idx, gate, ybs, BF16, kernel=apr.SGMM_DENSE)[0]
+    c = run_sgmm(apr, x, As, Bs, idx, gate, ybs, BF16, kernel=apr.SGMM_DENSE)[0]
+    assert np.array_equal(a, b) and np.array_equal(b, c)
+    p = rng.permutation(50)
+    d = run_sgmm(apr, x[p], As, Bs, idx[p], gate[p], [ybs[0][p]], BF16, kernel=apr.SGMM_DENSE)[0]
+    assert np.array_equal(d, b[p])
+    s = run_sgmm(apr, x, As, Bs, idx, gate, ybs, BF16, kernel=apr.SGMM_SKINNY)[0]
+    assert np.mean(s == b) > 0.95
+    close(b, s, "dense vs skinny")
+
+
+def test_sgmm_dense_faults_and_limits(apr):
+    rng = np.random.default_rng(33)
+    x, As, Bs, idx, gate, ybs = _case(rng, 20, 256, (128,), (16, 16, 32), 2)
+    x, As, Bs, ybs = _rounded(x, As, Bs, ybs)
+    with pytest.raises(apr.AprError) as ei:                   # a rank above max_rank, caught on the device
+        run_sgmm(apr, x, As, Bs, idx, gate, ybs, BF16, kernel=apr.SGMM_DENSE, max_rank=16)
+    assert ei.value.status == apr.APR_ERR_DEVICE_INDEX
+    ok = run_sgmm(apr, x, As, Bs, idx, gate, ybs, BF16, kernel=apr.SGMM_DENSE)
+    close(ok[0], oracle_group(x, As, Bs, idx, gate.astype(np.float64), ybs)[0], "dense after fault")
+    x2, As2, Bs2, idx2, gate2, ybs2 = _case(rng, 65, 256, (128,), (16,) * 4, 2)   # T above the dense limit
+    x2, As2, Bs2, ybs2 = _rounded(x2, As2, Bs2, ybs2)
+    with pytest.raises(apr.AprError) as ei:
+        run_sgmm(apr, x2, As2, Bs2, idx2, gate2, ybs2, BF16, kernel=apr.SGMM_DENSE)
+    assert ei.value.status == apr.APR_ERR_UNSUPPORTED

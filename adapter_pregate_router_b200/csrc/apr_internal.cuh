@@ -85,20 +85,34 @@ constexpr int kDenseMaxT = 64;
 constexpr int kDenseMaxRows = 256;
 constexpr int kDenseClusterCols = 8 * 256;
 inline int round16i(int v) { return (v + 15) / 16 * 16; }
-inline bool dense_dims_ok(int T, int E, int max_rank) {
-  return T >= 1 && T <= kDenseMaxT && E <= 16 && E * round16i(max_rank) <= kDenseMaxRows;
-}
 inline int dense_clusters(int d_in) { return (d_in + kDenseClusterCols - 1) / kDenseClusterCols; }
+inline bool dense_dims_ok(int T, int E, int max_rank, int d_in = 0) {
+  return T >= 1 && T <= kDenseMaxT && E <= 16 && E * round16i(max_rank) <= kDenseMaxRows &&
+         dense_clusters(d_in) <= 8;
+}
+
+// Tensor-core path: gated V rows [projection][plan position][2 * k * R16] bf16
+// (hi | lo) and one 16-byte descriptor per set tile; k <= 2, k * R16 <= 64.
+constexpr int kTensorMaxK2 = 64;
+inline size_t tc_vprep_bytes(int T, int K2) { return (size_t)APR_MAX_PROJ * T * 4 * K2; }
+inline size_t tc_scratch_bytes(int T, int k, int max_rank) {
+  if (k < 1 || k > 2) return 0;
+  const int K2 = k * round16i(max_rank);
+  if (K2 > kTensorMaxK2) return 0;
+  return align_up(tc_vprep_bytes(T, K2)) + 16 * (size_t)(T + 1);
+}
 
 // Shrink partial sums.  Gather paths: [projection][column chunk][sorted pair][rank]
 // fp32; dense path: [projection][cluster][token (padded to 16)][adapter * rank slot].
 inline size_t sgmm_scratch_bytes(int T, int k, int E, int max_rank, int d_in) {
   size_t b = sizeof(float) * APR_MAX_PROJ * (size_t)shrink_kchunks(d_in) * T * k * max_rank;
-  if (dense_dims_ok(T, E, max_rank)) {
+  if (dense_dims_ok(T, E, max_rank, d_in)) {
     const size_t d = sizeof(float) * APR_MAX_PROJ * (size_t)dense_clusters(d_in) * round16i(T) * E *
                      round16i(max_rank);
     if (d > b) b = d;
   }
+  const size_t t = tc_scratch_bytes(T, k, max_rank);
+  if (t > b) b = t;
   return b;
 }
 
@@ -248,7 +262,7 @@ struct SgmmArgs {
   void* ws;
 };
 cudaError_t launch_sgmm_skinny(const SgmmArgs& a, int dtype, size_t scratch_off, cudaStream_t s);
-cudaError_t launch_sgmm_tensor(const SgmmArgs& a, cudaStream_t s);
+cudaError_t launch_sgmm_tensor(const SgmmArgs& a, size_t scratch_off, cudaStream_t s);
 cudaError_t launch_sgmm_dense(const SgmmArgs& a, size_t scratch_off, cudaStream_t s);
 bool sgmm_dense_supported(const SgmmArgs& a, int dtype);
 bool sgmm_tensor_supported(const SgmmArgs& a, int dtype);

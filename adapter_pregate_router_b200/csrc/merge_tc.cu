@@ -1,0 +1,289 @@
+// Batch-1 merge on the 5th-generation tensor cores (tcgen05).
+#include "apr_internal.cuh"
+#include "tc_ptx.cuh"
+
+namespace apr {
+
+constexpr int TC_THREADS = 128;
+constexpr int TC_BM = 128;                      // rows of W per strip
+constexpr int TC_MAXN1 = 64;                    // k * rank (rounded up to 16)
+constexpr uint32_t TC_TMEM_COLS = 512;
+constexpr uint32_t TC_D2_COL = 128;             // D buffers at columns 128 and 256
+
+static int round16(int r) { return (r + 15) / 16 * 16; }
+
+// Batch-1 merge (AdaFuse summary §2.B decoding steps 3 and 5), every weight in
+// one launch, out of place:  W' = W + sum_j g_j B_{e_j} A_{e_j}.
+// A work item is a strip of 128 rows of one weight.  The strip's gated B rows
+// Bg[n][j*R16 + i] = g_j B_{e_j}[n][i] are formed once (fp32 -> bf16 hi + lo,
+// K-major), then for every 128-column tile: D[128 x 128] = Bg_hi.A^T +
+// Bg_lo.A^T on tcgen05 with A^T as an MN-major operand (rows of A_e are
+// contiguous along the output columns), TMEM double buffered; the W tile and
+// the A tile arrive two tiles ahead by cp.async into 3-deep rings, and the
+// epilogue adds D to W in fp32, rounds once and the warp writes its 32 rows
+// of W' back with coalesced 128-bit stores.
+
+constexpr int MT_BN = 128;                      // columns per tile
+constexpr int MT_NY = 3;                        // ring depth
+constexpr int MT_WSTRIDE = MT_BN * 2 + 16;      // bytes per staged W row
+constexpr int MT_WBUF = TC_BM * MT_WSTRIDE;
+constexpr int MT_ABUF = MT_BN * TC_MAXN1 * 2;   // MN-major A^T tile
+constexpr int MT_MAXPROJ = 4096;
+
+struct MtSmem {
+  static constexpr size_t GH = 0;                                        // 16 KB
+  static constexpr size_t GL = GH + (size_t)TC_BM * TC_MAXN1 * 2;        // 16 KB
+  static constexpr size_t WR = GL + (size_t)TC_BM * TC_MAXN1 * 2;        // W ring
+  static constexpr size_t AR = WR + (size_t)MT_NY * MT_WBUF;             // A ring
+  static constexpr size_t BAR = AR + (size_t)MT_NY * MT_ABUF;
+  static constexpr size_t META = BAR + 2 * 8;
+  static constexpr size_t PREF = META + 128;                             // [nproj + 1] strip prefix
+  static constexpr size_t fixed_bytes() { return PREF + 1024; }
+};
+
+// K-major A operand / MN-major B operand instruction descriptor (bf16 -> fp32).
+__host__ __device__ constexpr uint32_t idesc_bf16_bmn(int M, int N) { return idesc_bf16(M, N) | (1u << 16); }
+
+__global__ void __launch_bounds__(TC_THREADS, 1) merge_tc_kernel(const apr_merge_proj* __restrict__ projs,
+                                                                 int nproj, int E, int r, int R16,
+                                                                 const int32_t* __restrict__ idx,
+                                                                 const float* __restrict__ gate, int k,
+                                                                 void* ws) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem =
+      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int K = k * R16;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + MtSmem::BAR);
+  const uint32_t bar_mma = smem_u32(bars);                     // [2]
+  volatile int* s_flags = reinterpret_cast<volatile int*>(smem + MtSmem::META);   // [0] tmem, [1] bad
+  int* s_e = const_cast<int*>(s_flags) + 4;                    // [<= 8]
+  float* s_g = reinterpret_cast<float*>(s_e + 8);              // [<= 8]
+  int* s_pref = reinterpret_cast<int*>(smem + MtSmem::PREF);
+  const uint32_t sGH = smem_u32(smem + MtSmem::GH);
+  const uint32_t sGL = smem_u32(smem + MtSmem::GL);
+  unsigned char* sWp = smem + MtSmem::WR;
+  const uint32_t sW = smem_u32(sWp);
+  const uint32_t sA = smem_u32(smem + MtSmem::AR);
+
+  if (tid == 0) {
+    for (int i = 0; i < 2; ++i) mbar_init(bar_mma + 8 * i, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    s_flags[1] = 0;
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(const_cast<int*>(s_flags))),
+                 "r"(TC_TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = (uint32_t)s_flags[0];
+  pdl_wait();
+  pdl_trigger();
+
+  if (tid < k) {
+    const int e = idx[tid];
+    if (e < 0 || e >= E) s_flags[1] = 1;
+    s_e[tid] = e;
+    s_g[tid] = gate[tid];
+  }
+  // strips (128 rows) per weight, prefix over the weights
+  if (tid == 0) {
+    int acc = 0;
+    s_pref[0] = 0;
+    for (int p = 0; p < nproj; ++p) {
+      acc += (projs[p].d_out + TC_BM - 1) / TC_BM;
+      s_pref[p + 1] = acc;
+    }
+  }
+  __syncthreads();
+  bool abort = false;
+  if (s_flags[1]) {
+    if (tid == 0 && blockIdx.x == 0) report(ws, APR_ERR_DEVICE_INDEX, K_MERGE, 0);
+  } else {
+    const int total = s_pref[nproj];
+    const uint32_t sbo_g = (uint32_t)(K / 8) * 128;         // Bg: next 8-row group
+    const uint32_t id = idesc_bf16_bmn(TC_BM, MT_BN);
+    uint32_t ph_mma = 0;
+    for (int strip = blockIdx.x; strip < total && !abort; strip += gridDim.x) {
+      int lo = 0, hi = nproj;                                 // weight of this strip
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (s_pref[mid] <= strip) lo = mid; else hi = mid;
+      }
+      const apr_merge_proj pj = projs[lo];
+      const int row0 = (strip - s_pref[lo]) * TC_BM;
+      const int nrows = min(TC_BM, pj.d_out - row0);
+      const __nv_bfloat16* __restrict__ Wt = reinterpret_cast<const __nv_bfloat16*>(pj.W);
+      __nv_bfloat16* __restrict__ Wp = reinterpret_cast<__nv_bfloat16*>(pj.Wp);
+      // gated B rows of the strip, bf16 hi + lo, K-major
+      {
+        const int n = row0 + tid;
+        for (int j = 0; j < k; ++j) {
+          const __nv_bfloat16* B = reinterpret_cast<const __nv_bfloat16*>(pj.B[s_e[j]]);
+          for (int c8 = 0; c8 < R16; c8 += 8) {
+            float f[8];
+            if (tid < nrows && c8 < r) {
+              load8(B + (size_t)n * r + c8, f);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 8; ++i) f[i] = 0.f;
+            }
+            uint32_t h4[4], l4[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float a0 = f[2 * i] * s_g[j], a1 = f[2 * i + 1] * s_g[j];
+              const __nv_bfloat162 hh = __floats2bfloat162_rn(a0, a1);
+              const float2 hf = __bfloat1622float2(hh);
+              h4[i] = *reinterpret_cast<const uint32_t*>(&hh);
+              l4[i] = pack_bf16x2(a0 - hf.x, a1 - hf.y);
+            }
+            const int kc8 = (j * R16 + c8) >> 3;
+            const uint32_t off = (uint32_t)(tid >> 3) * sbo_g + (uint32_t)kc8 * 128 + (uint32_t)(tid & 7) * 16;
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(sGH + off), "r"(h4[0]), "r"(h4[1]),
+                         "r"(h4[2]), "r"(h4[3])
+                         : "memory");
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(sGL + off), "r"(l4[0]), "r"(l4[1]),
+                         "r"(l4[2]), "r"(l4[3])
+                         : "memory");
+          }
+        }
+      }
+      fence_proxy_async();                       // Bg was written by ordinary stores
+      const int nct = (pj.d_in + MT_BN - 1) / MT_BN;
+      auto issue_tile = [&](int ct) {
+        const int slot = ct % MT_NY;
+        const int c0 = ct * MT_BN;
+        const int ncols = min(MT_BN, pj.d_in - c0);
+        // A^T tile, MN-major: core matrix (8 columns x 8 rank rows) at (col/8)*128 + (kk/8)*2048
+        const uint32_t abase = sA + (uint32_t)slot * MT_ABUF;
+        for (int w = tid; w < K * (MT_BN / 8); w += TC_THREADS) {
+          const int kk = w / (MT_BN / 8), c = w % (MT_BN / 8);
+          const int j = kk / R16, i = kk % R16;
+          const uint32_t dst = abase + (uint32_t)c * 128 + (uint32_t)(kk >> 3) * 2048 + (uint32_t)(kk & 7) * 16;
+          const bool valid = i < r && c * 8 < ncols;
+          const __nv_bfloat16* A = reinterpret_cast<const __nv_bfloat16*>(pj.A[s_e[j]]);
+          cp_async16_zfill(dst, valid ? A + (size_t)i * pj.d_in + c0 + c * 8 : A, valid);
+        }
+        // W rows of the tile: 16 lanes per 256-byte row segment, 2 rows per instruction
+        const uint32_t wbase = sW + (uint32_t)slot * MT_WBUF;
+        const int ch = lane & 15;
+        if (ch * 8 < ncols) {
+#pragma unroll 4
+          for (int k2 = 0; k2 < 16; ++k2) {
+            const int row = warp * 32 + 2 * k2 + (lane >> 4);
+            if (row < nrows)
+              asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(wbase + (uint32_t)row * MT_WSTRIDE + ch * 16),
+                           "l"(Wt + (size_t)(row0 + row) * pj.d_in + c0 + ch * 8)
+                           : "memory");
+          }
+        }
+      };
+      for (int ct = 0; ct < MT_NY - 1; ++ct) {
+        if (ct < nct) issue_tile(ct);
+        cp_async_commit();
+      }
+      for (int ct = 0; ct < nct; ++ct) {
+        const int b = ct & 1;
+        const int slot = ct % MT_NY;
+        const int c0 = ct * MT_BN;
+        const int ncols = min(MT_BN, pj.d_in - c0);
+        if (ct + MT_NY - 1 < nct) issue_tile(ct + MT_NY - 1);
+        cp_async_commit();
+        cp_async_wait<MT_NY - 1>();
+        __syncthreads();
+        if (tid == 0) {
+          tc_fence_after();
+          const uint32_t ab = sA + (uint32_t)slot * MT_ABUF;
+          const uint32_t dcol = tmem + TC_D2_COL + (uint32_t)b * MT_BN;
+          for (int kk = 0; kk < K / 16; ++kk)
+            mma_bf16(dcol, desc_k_plain(sGH + kk * 256, 128, sbo_g), desc_k_plain(ab + kk * 4096, 2048, 128), id,
+                     kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < K / 16; ++kk)
+            mma_bf16(dcol, desc_k_plain(sGL + kk * 256, 128, sbo_g), desc_k_plain(ab + kk * 4096, 2048, 128), id, 1u);
+          mma_commit(bar_mma + 8 * b);
+        }
+        if (!mbar_wait(bar_mma + 8 * b, (ph_mma >> b) & 1)) abort = true;
+        ph_mma ^= 1u << b;
+        tc_fence_after();
+        abort = __syncthreads_or(abort);
+        if (abort) break;
+        {
+          const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16) + TC_D2_COL + (uint32_t)b * MT_BN;
+          unsigned char* wrow = sWp + (size_t)slot * MT_WBUF + (size_t)tid * MT_WSTRIDE;
+          for (int cc = 0; cc < ncols; cc += 16) {
+            float v[16];
+            tmem_ld16(lane_addr + (uint32_t)cc, v);
+            if (tid < nrows) {
+              uint4* pr = reinterpret_cast<uint4*>(wrow + cc * 2);
+              uint4 u0 = pr[0], u1 = pr[1];
+              __nv_bfloat162* h0 = reinterpret_cast<__nv_bfloat162*>(&u0);
+              __nv_bfloat162* h1 = reinterpret_cast<__nv_bfloat162*>(&u1);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const float2 f0 = __bfloat1622float2(h0[i]);
+                const float2 f1 = __bfloat1622float2(h1[i]);
+                h0[i] = __floats2bfloat162_rn(f0.x + v[2 * i], f0.y + v[2 * i + 1]);
+                h1[i] = __floats2bfloat162_rn(f1.x + v[8 + 2 * i], f1.y + v[8 + 2 * i + 1]);
+              }
+              pr[0] = u0;
+              pr[1] = u1;
+            }
+          }
+          __syncwarp();
+          const int ch = lane & 15;
+          if (ch * 8 < ncols) {
+#pragma unroll 4
+            for (int k2 = 0; k2 < 16; ++k2) {
+              const int row = warp * 32 + 2 * k2 + (lane >> 4);
+              if (row < nrows) {
+                const uint4 val = *reinterpret_cast<const uint4*>(sWp + (size_t)slot * MT_WBUF +
+                                                                 (size_t)row * MT_WSTRIDE + ch * 16);
+                __stcs(reinterpret_cast<uint4*>(Wp + (size_t)(row0 + row) * pj.d_in + c0 + ch * 8), val);
+              }
+            }
+          }
+        }
+        tc_fence_before();
+        __syncthreads();
+      }
+      cp_async_wait_all();
+      __syncthreads();
+    }
+  }
+  if (abort && tid == 0) report(ws, APR_ERR_TIMEOUT, K_MERGE, (int)blockIdx.x);
+  cp_async_wait_all();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TC_TMEM_COLS)
+                 : "memory");
+  }
+}
+
+bool merge_tensor_supported(int k, int r, int nproj) {
+  return k * round16(r) <= TC_MAXN1 && nproj <= MT_MAXPROJ;
+}
+
+cudaError_t launch_merge_tensor(const apr_merge_proj* projs, int nproj, int E, int r, const int32_t* idx,
+                                const float* gate, int k, void* ws, cudaStream_t s) {
+  const size_t smem = MtSmem::fixed_bytes() + sizeof(int) * ((size_t)nproj + 1);
+  static size_t configured = 0;
+  if (smem > configured) {
+    cudaError_t err = cudaFuncSetAttribute(merge_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    configured = smem;
+  }
+  int dev = 0, nsm = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  return launch_pdl(merge_tc_kernel, dim3(nsm), dim3(TC_THREADS), smem, s, projs, nproj, E, r, round16(r), idx,
+                    gate, k, ws);
+}
+
+}  // namespace apr

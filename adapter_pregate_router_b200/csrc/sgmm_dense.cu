@@ -62,21 +62,25 @@ __device__ __forceinline__ uint32_t cluster_map(uint32_t saddr, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
   return r;
 }
+// A load from another CTA's shared memory; ordered by the cluster barriers
+// around it, it carries no memory clobber, so several stay in flight.
 __device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
   float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(addr)
-               : "memory");
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
   return v;
 }
+__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
 __device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+  cluster_arrive();
+  cluster_wait();
 }
 
 // ---------------------------------------------------------------- shrink
 
+// TP (tokens padded to 16) and MRT (rank rows padded to 128) are compile-time,
+// so the decode instantiation is short straight-line code.
+template <int TP, int MRT>
 __global__ void __launch_bounds__(DN_THREADS, 1) dense_shrink_kernel(const __grid_constant__ DenseArgs args) {
   const SgmmArgs& a = args.a;
   extern __shared__ unsigned char smem_raw[];
@@ -85,7 +89,8 @@ __global__ void __launch_bounds__(DN_THREADS, 1) dense_shrink_kernel(const __gri
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int rank = blockIdx.x;                    // rank in the cluster (cluster spans gridDim.x)
   const int cl = blockIdx.y, p = blockIdx.z;
-  const int Tp = args.Tp, Rp = args.Rp, NR = args.NR, MR = args.MR;
+  constexpr int Tp = TP, MR = MRT;
+  const int Rp = args.Rp, NR = args.NR;
   const int T = a.T, K = a.k, E = a.E, d_in = a.d_in;
   const int k0 = (cl * DN_CL + rank) * DN_KC;
 
@@ -200,16 +205,31 @@ __global__ void __launch_bounds__(DN_THREADS, 1) dense_shrink_kernel(const __gri
 
   // this CTA's share of the rows, summed over the cluster in rank order, gated
   {
-    const int RS = MR / DN_CL;               // rows per CTA (16 or 32)
-    const int groups = RS / 4;
+    constexpr int RS = MR / DN_CL;           // rows per CTA (16 or 32)
+    constexpr int groups = RS / 4;
     float* vpart = ws_at<float>(a.ws, args.vpart_off) + ((size_t)(p * args.ncl + cl) * Tp) * NR;
-    for (int w = tid; w < groups * Tp; w += DN_THREADS) {
+    constexpr int PER = 2;                   // float4 groups per thread: RS / 4 * Tp <= 8 * 64 = 2 * 256
+    float4 part[PER][DN_CL];
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+      const int w = tid + u * DN_THREADS;
+      if (w < groups * Tp) {
+        const int t = w / groups, r0 = rank * RS + (w % groups) * 4;
+        const uint32_t off = smem_u32(P + (size_t)t * MR + r0);
+#pragma unroll
+        for (int c = 0; c < DN_CL; ++c) part[u][c] = ld_cluster_f4(cluster_map(off, (uint32_t)c));
+      }
+    }
+    cluster_arrive();          // this CTA's reads of the cluster's P are issued and consumed below
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+      const int w = tid + u * DN_THREADS;
+      if (w >= groups * Tp) continue;
       const int t = w / groups, r0 = rank * RS + (w % groups) * 4;
-      const uint32_t off = smem_u32(P + (size_t)t * MR + r0);
-      float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int c = 0; c < DN_CL; ++c) {
-        const float4 v = ld_cluster_f4(cluster_map(off, (uint32_t)c));
-        s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+      float4 s = part[u][0];
+#pragma unroll
+      for (int c = 1; c < DN_CL; ++c) {
+        s.x += part[u][c].x; s.y += part[u][c].y; s.z += part[u][c].z; s.w += part[u][c].w;
       }
       if (r0 >= NR) continue;
       const int e = r0 / Rp;
@@ -227,19 +247,21 @@ __global__ void __launch_bounds__(DN_THREADS, 1) dense_shrink_kernel(const __gri
       *reinterpret_cast<float4*>(vpart + (size_t)t * NR + r0) = make_float4(g * s.x, g * s.y, g * s.z, g * s.w);
     }
   }
-  cluster_sync_all();          // remote reads of P are over before any CTA leaves
+  cluster_wait();              // every CTA's reads of this CTA's P are over before it leaves
   if (warp == 0) tmem_dealloc(tmem, ncols);
 }
 
 // ---------------------------------------------------------------- expand
 
+template <int TP>
 __global__ void __launch_bounds__(DN_THREADS, 1) dense_expand_kernel(const __grid_constant__ DenseArgs args) {
   const SgmmArgs& a = args.a;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int Tp = args.Tp, Rp = args.Rp, NR = args.NR;
+  constexpr int Tp = TP;
+  const int Rp = args.Rp, NR = args.NR;
   const int T = a.T, E = a.E;
   int p = 0;
   while (p + 1 < a.nproj && (int)blockIdx.x >= args.tiles_before[p + 1]) ++p;
@@ -303,22 +325,53 @@ __global__ void __launch_bounds__(DN_THREADS, 1) dense_expand_kernel(const __gri
   {
     const float* vp = ws_at<float>(a.ws, args.vpart_off) + (size_t)p * args.ncl * Tp * NR;
     const int kq_n = NR / 8;
-    for (int w = tid; w < Tp * kq_n; w += DN_THREADS) {
-      const int t = w / kq_n, kq = w - t * kq_n;
-      float f[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      for (int c = 0; c < args.ncl; ++c) {
-        const float4* src = reinterpret_cast<const float4*>(vp + ((size_t)c * Tp + t) * NR + kq * 8);
-        const float4 u0 = __ldcg(src), u1 = __ldcg(src + 1);
-        f[0] += u0.x; f[1] += u0.y; f[2] += u0.z; f[3] += u0.w;
-        f[4] += u1.x; f[5] += u1.y; f[6] += u1.z; f[7] += u1.w;
+    for (int w0 = tid; w0 < Tp * kq_n; w0 += DN_THREADS * 2) {
+      // two 8-value chunks per thread; the cluster partials are summed in order,
+      // two clusters' loads in flight per round
+      float f[2][8];
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) f[h][i] = 0.f;
+      for (int c0 = 0; c0 < args.ncl; c0 += 2) {
+        float4 ld[2][2][2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int w = w0 + h * DN_THREADS;
+          const int t = w / kq_n, kq = w - t * kq_n;
+#pragma unroll
+          for (int dc = 0; dc < 2; ++dc) {
+            const int c = c0 + dc;
+            if (w < Tp * kq_n && c < args.ncl) {
+              const float4* src = reinterpret_cast<const float4*>(vp + ((size_t)c * Tp + t) * NR + kq * 8);
+              ld[h][dc][0] = __ldcg(src);
+              ld[h][dc][1] = __ldcg(src + 1);
+            } else {
+              ld[h][dc][0] = ld[h][dc][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+          }
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int dc = 0; dc < 2; ++dc) {
+            const float4 u0 = ld[h][dc][0], u1 = ld[h][dc][1];
+            f[h][0] += u0.x; f[h][1] += u0.y; f[h][2] += u0.z; f[h][3] += u0.w;
+            f[h][4] += u1.x; f[h][5] += u1.y; f[h][6] += u1.z; f[h][7] += u1.w;
+          }
       }
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+      const int w = w0 + h * DN_THREADS;
+      if (w >= Tp * kq_n) continue;
+      const int t = w / kq_n, kq = w - t * kq_n;
       uint32_t hi[4], lo[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
-        const float2 hf = __bfloat1622float2(h);
-        hi[i] = *reinterpret_cast<const uint32_t*>(&h);
-        lo[i] = pack_bf16x2(f[2 * i] - hf.x, f[2 * i + 1] - hf.y);
+        const __nv_bfloat162 hv = __floats2bfloat162_rn(f[h][2 * i], f[h][2 * i + 1]);
+        const float2 hf = __bfloat1622float2(hv);
+        hi[i] = *reinterpret_cast<const uint32_t*>(&hv);
+        lo[i] = pack_bf16x2(f[h][2 * i] - hf.x, f[h][2 * i + 1] - hf.y);
       }
       const uint32_t off = (uint32_t)(t >> 3) * SBO + (uint32_t)kq * 128 + (uint32_t)(t & 7) * 16;
       asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(sVH) + off), "r"(hi[0]), "r"(hi[1]),
@@ -327,6 +380,7 @@ __global__ void __launch_bounds__(DN_THREADS, 1) dense_expand_kernel(const __gri
       asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(sVL) + off), "r"(lo[0]), "r"(lo[1]),
                    "r"(lo[2]), "r"(lo[3])
                    : "memory");
+      }
     }
   }
   cp_async_wait_all();
@@ -376,7 +430,7 @@ __global__ void __launch_bounds__(DN_THREADS, 1) dense_expand_kernel(const __gri
 static int dn_round16(int v) { return (v + 15) / 16 * 16; }
 
 bool sgmm_dense_supported(const SgmmArgs& a, int dtype) {
-  return dtype == APR_BF16 && dense_dims_ok(a.T, a.E, a.max_rank) && a.E <= 16 && a.k <= APR_MAX_K;
+  return dtype == APR_BF16 && dense_dims_ok(a.T, a.E, a.max_rank, a.d_in) && a.k <= APR_MAX_K;
 }
 
 static size_t shrink_smem(int MR, int Tp) { return (size_t)MR * 512 + (size_t)Tp * 512 + 16 + 8 * 16 + 4 * 16 + 8 * 64 * APR_MAX_K + 1024; }
@@ -398,17 +452,23 @@ cudaError_t launch_sgmm_dense(const SgmmArgs& a, size_t scratch_off, cudaStream_
   for (int p = 0; p < a.nproj; ++p) d.tiles_before[p + 1] = d.tiles_before[p] + (a.proj[p].d_out + DN_NT - 1) / DN_NT;
 
   const size_t sm1 = shrink_smem(d.MR, d.Tp), sm2 = expand_smem(d.NR, d.Tp);
-  static size_t conf1 = 0, conf2 = 0;
+  using Kern = void (*)(DenseArgs);
+  const int ti = d.Tp / 16 - 1, mi = d.MR / 128 - 1;
+  static const Kern shrinks[4][2] = {
+      {dense_shrink_kernel<16, 128>, dense_shrink_kernel<16, 256>}, {dense_shrink_kernel<32, 128>, dense_shrink_kernel<32, 256>},
+      {dense_shrink_kernel<48, 128>, dense_shrink_kernel<48, 256>}, {dense_shrink_kernel<64, 128>, dense_shrink_kernel<64, 256>}};
+  static const Kern expands[4] = {dense_expand_kernel<16>, dense_expand_kernel<32>, dense_expand_kernel<48>,
+                                  dense_expand_kernel<64>};
+  static size_t conf1[4][2] = {}, conf2[4] = {};
+  const Kern k1 = shrinks[ti][mi], k2 = expands[ti];
   cudaError_t err;
-  if (sm1 > conf1) {
-    if ((err = cudaFuncSetAttribute(dense_shrink_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1)) != cudaSuccess)
-      return err;
-    conf1 = sm1;
+  if (sm1 > conf1[ti][mi]) {
+    if ((err = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1)) != cudaSuccess) return err;
+    conf1[ti][mi] = sm1;
   }
-  if (sm2 > conf2) {
-    if ((err = cudaFuncSetAttribute(dense_expand_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2)) != cudaSuccess)
-      return err;
-    conf2 = sm2;
+  if (sm2 > conf2[ti]) {
+    if ((err = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2)) != cudaSuccess) return err;
+    conf2[ti] = sm2;
   }
   {
     cudaLaunchConfig_t cfg = {};
@@ -426,9 +486,9 @@ cudaError_t launch_sgmm_dense(const SgmmArgs& a, size_t scratch_off, cudaStream_
     cfg.attrs = attr;
     cfg.numAttrs = 2;
     count_launch();
-    if ((err = cudaLaunchKernelEx(&cfg, dense_shrink_kernel, d)) != cudaSuccess) return err;
+    if ((err = cudaLaunchKernelEx(&cfg, k1, d)) != cudaSuccess) return err;
   }
-  return launch_pdl(dense_expand_kernel, dim3(d.tiles_before[a.nproj]), dim3(DN_THREADS), sm2, s, d);
+  return launch_pdl(k2, dim3(d.tiles_before[a.nproj]), dim3(DN_THREADS), sm2, s, d);
 }
 
 }  // namespace apr

@@ -1,153 +1,114 @@
 // SGMM on the 5th-generation tensor cores (tcgen05) for long segments
-// (prefill).  AdaFuse summary (gist.science), Resumen tecnico §2.B: the
-// segmented gather product applies the selected low-rank adapters to the
-// tokens gathered per adapter in one batched product, fused into the add onto
-// the base projection output, with prefetching and tiling.
+// (prefill, many tenants).  AdaFuse summary (gist.science), Resumen tecnico
+// §2.B: the segmented gather product applies the selected low-rank adapters to
+// the tokens gathered per adapter in one batched product, fused into the add
+// onto the base projection output.
 //
-// The routing plan orders tokens by their adapter set; a work item is one
-// set tile (<= 128 tokens that share the same k <= 2 adapters {e0, e1}) and
-// one projection.  Per item, in one CTA of 128 threads (1 CTA per SM, TMEM
-// fully owned, persistent over the items):
+// The routing plan orders the tokens by their adapter set; a set tile is a run
+// of <= 128 tokens sharing the same k <= 2 adapters {e0 < e1}.  Two persistent
+// kernels, one CTA per SM:
 //
-//  shrink  D1[128 x N1] = X_tile[128 x d_in] . [A_e0 ; A_e1]^T on tcgen05
-//          (kind::f16, bf16 in, fp32 accumulate in TMEM), N1 = k * R16 where
-//          R16 is the rank rounded up to 16 (zero rows pad the smaller ranks).
-//          The gathered x rows arrive by TMA (tile::gather4: four token rows x
-//          128 bytes per instruction, 128B-swizzled, one issuing lane per warp
-//          for its 32 tokens, rows of absent tokens zero-filled) and the small
-//          A rows by 16-byte cp.async; both complete on the stage's "full"
-//          mbarrier (6 stages in flight).  One thread of the MMA warp issues
-//          the MMAs of a stage once it is full and commits them to the stage's
-//          "empty" mbarrier, which frees the stage for the next fill.
-//  gate    D1 is read back with tcgen05.ld (one TMEM lane per token), scaled
-//          by the token's gates and split into bf16 hi + lo parts (so the
-//          expand keeps ~16 mantissa bits of v), written to shared memory as
-//          the K-major A operand of the expand.
-//  expand  for every 128-column tile of d_out: D2[128 x 128] = V_hi.Bcat^T +
-//          V_lo.Bcat^T with Bcat[n] = [B_e0[n] | B_e1[n]] (K2 = N1), TMEM
-//          double buffered.  Bcat (cp.async) and the y_base rows (TMA gather4)
-//          of a tile are fetched two tiles ahead into 3-deep rings that reuse
-//          the shrink stages' shared memory; the epilogue adds D2 in its
-//          token's row, rounds to bf16 once, and the rows leave by TMA
-//          scatter4 (plain stores for the one 4-row group a tile's end cuts).
-//
-// Warps 0-3 stage operands and run epilogues, warp 4 issues the MMAs; each
-// worker warp owns 32 token rows of every buffer, so reuse of a ring slot only
-// waits for that warp's own bulk stores.
+//  shrink  item = one set tile and a group of projections (all of them when
+//          nproj * k * R16 <= 256; R16 = max rank rounded up to 16).
+//          D1[128 x N1] = X_tile . [A_{q,e0} ; A_{q,e1} ...]^T on tcgen05
+//          (kind::f16, bf16 in, fp32 in TMEM): x rows are gathered once per
+//          tile, 64 columns per stage, with 16-byte cp.async into 128B-swizzled
+//          K-major stages, A rows likewise; the copies complete on the stage's
+//          mbarrier, one thread of the MMA warp issues the MMAs and commits
+//          them to the stage's "empty" barrier.  The epilogue reads D1 back
+//          (one TMEM lane per token), scales by the token's gates and stores
+//          v as bf16 hi + lo halves (~16 mantissa bits) in the token's row of
+//          the plan order: V[q][pos][hi: k*R16 | lo: k*R16].
+//  expand  item = (set tile, projection, 1024 output columns), 128-column
+//          tiles: D2[128 x 128] = V_hi . Bcat^T + V_lo . Bcat^T with
+//          Bcat[n] = [B_e0[n] | B_e1[n]], TMEM double buffered.  Eight warps
+//          gather the tile's y_base rows and Bcat with cp.async into a 4-deep
+//          ring (three tiles ahead, across item boundaries), then run the
+//          epilogue: y = y_base + D2 for their row and half, rounded once to
+//          bf16, written back through shared memory so each warp stores whole
+//          128-byte row segments.
 //
 // Every mbarrier wait is bounded by the global timer (1 s); on expiry the CTA
-// records APR_ERR_TIMEOUT, drains its own copies and frees its TMEM.
-#include <cudaTypedefs.h>
-
-#include <mutex>
-
+// records APR_ERR_TIMEOUT, drains its copies and frees its TMEM.
 #include "apr_internal.cuh"
 #include "tc_ptx.cuh"
 
 namespace apr {
 
-constexpr int TC_THREADS = 128;
-constexpr int TC_BM = 128;       // tokens per tile (= kSetTile)
-constexpr int TC_BK = 64;        // input columns per stage (one 128-byte swizzle row)
-constexpr int TC_STAGES = 6;
-constexpr int TC_MAXN1 = 64;     // k * R16
-constexpr int TC_NT = 128;       // output columns per expand tile
-constexpr int TC_NY = 3;         // depth of the Bcat / y_base rings (prefetch distance 2)
-constexpr uint32_t TC_TMEM_COLS = 512;
-constexpr uint32_t TC_D2_COL = 128;           // D2 buffers at columns 128 and 256
-constexpr int TC_STAGE_BYTES = TC_BM * 128 + TC_MAXN1 * 128;   // x tile + A rows
-constexpr int TC_YBUF_BYTES = 2 * TC_BM * 128;                  // two 64-column halves, 128B-swizzled rows
-constexpr int TC_BBUF_BYTES = TC_NT * TC_MAXN1 * 2;
+constexpr int TB_M = 128;          // tokens per set tile (= kSetTile)
+constexpr int TB_BK = 64;          // input columns per shrink stage
+constexpr int TB_MAXN1 = 256;      // shrink accumulator columns
+constexpr int TB_MAXK2 = 64;       // k * R16 handled by the expand
+constexpr int TB_NT = 128;         // output columns per expand tile
+constexpr int TB_CW = 1024;        // output columns per expand item
+constexpr int SH_WORKERS = 128;    // shrink: warps 0-3 load and run the epilogue, warp 4 issues MMAs
+constexpr int SH_BLOCK = SH_WORKERS + 32;
+constexpr int EX_WORKERS = 256;    // expand: warps 0-7 load and run the epilogue, warp 8 issues MMAs
+constexpr int EX_BLOCK = EX_WORKERS + 32;
+constexpr int SMEM_BUDGET = 200 * 1024;
 
-struct TcSmem {
-  // the shrink stages and the expand's rings are never live at the same time
-  static constexpr size_t STAGE_AREA = (size_t)TC_STAGES * TC_STAGE_BYTES;
-  static constexpr size_t RING_AREA = (size_t)TC_NY * (TC_YBUF_BYTES + TC_BBUF_BYTES);
-  static constexpr size_t U = 0;
-  static constexpr size_t U_BYTES = STAGE_AREA > RING_AREA ? STAGE_AREA : RING_AREA;
-  static constexpr size_t YR = U;                                             // y ring (1024-aligned slots)
-  static constexpr size_t BR = U + (size_t)TC_NY * TC_YBUF_BYTES;             // Bcat ring
-  static constexpr size_t VH = U + (U_BYTES + 1023) / 1024 * 1024;            // 16 KB
-  static constexpr size_t VL = VH + (size_t)TC_BM * TC_MAXN1 * 2;             // 16 KB
-  static constexpr size_t BAR = VL + (size_t)TC_BM * TC_MAXN1 * 2;            // mbarriers
-  static constexpr int NBARS = 2 * TC_STAGES + 2 + TC_NY + 4;
-  static constexpr size_t META = BAR + (size_t)NBARS * 8;
-  static constexpr size_t TOTAL = META + 3 * TC_BM * 4 + 64;
-  static constexpr size_t ALLOC = TOTAL + 1024;                               // for 1024-byte alignment
+struct TileInfo {        // a set tile and its adapters, written by the shrink for the expand
+  int start, len, e0, e1;
 };
-static_assert(TcSmem::ALLOC <= 227 * 1024, "shared memory budget");
-static_assert(TC_STAGE_BYTES % 1024 == 0, "stages keep 1024-byte alignment");
-static_assert(TcSmem::BR % 16 == 0 && TC_YBUF_BYTES % 1024 == 0, "aligned rings");
 
-// ---------------------------------------------------------------- the kernel
-
-struct TcArgs {
-  CUtensorMap tm_x;                    // x [T, d_in], box 64 x 1, 128B swizzle
-  CUtensorMap tm_yb[APR_MAX_PROJ];     // y_base [T, d_out]
-  CUtensorMap tm_y[APR_MAX_PROJ];      // y [T, d_out]
+struct TcPlan {
   SgmmArgs a;
-  int R16;     // rank slot per adapter (multiple of 16)
-  int N1;      // k * R16
+  int R16;                           // rank slot per adapter
+  int K2;                            // k * R16
+  int pg;                            // projections per shrink item
+  int npg;                           // shrink items per set tile
+  int stages;                        // shrink pipeline depth
+  int ny;                            // expand ring depth
+  size_t vprep_off;                  // scratch: V rows [proj][pos][2 * K2] bf16
+  size_t tinfo_off;                  // scratch: TileInfo [set tiles]
+  int cc_before[APR_MAX_PROJ + 1];   // expand: prefix of 1024-column items per projection
 };
 
-constexpr int TC_WORKERS = 128;                  // warps 0-3: loads and epilogues
-constexpr int TC_BLOCK = TC_WORKERS + 32;        // warp 4: MMA issue
+static_assert(sizeof(TileInfo) == 16 && TB_MAXK2 == kTensorMaxK2, "tensor scratch sizing");
 
-__device__ __forceinline__ void workers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(TC_WORKERS) : "memory"); }
+// ---------------------------------------------------------------- shrink
 
-// Warp-specialised: warps 0-3 stage operands with TMA and cp.async (completion
-// arrives on mbarriers) and run the epilogues; lane 0 of warp 4 issues every
-// tcgen05.mma and commits it to the barrier that releases the consumer.  No
-// block-wide barrier inside an item, so loads, MMAs and epilogues of different
-// chunks and tiles overlap.
-__global__ void __launch_bounds__(TC_BLOCK, 1) sgmm_tc_kernel(const __grid_constant__ TcArgs args) {
-  const SgmmArgs& a = args.a;
+struct ShSmem {
+  int stage_bytes, stages;
+  size_t bar, meta, total;
+};
+__host__ __device__ inline ShSmem sh_smem(int n1max, int stages) {
+  ShSmem L;
+  L.stage_bytes = TB_M * 128 + n1max * 128;
+  L.stages = stages;
+  L.bar = (size_t)stages * L.stage_bytes;
+  L.meta = L.bar + (size_t)(2 * stages + 1) * 8;
+  L.total = L.meta + 3 * TB_M * 4 + 16 + TB_MAXN1 * 8 + 1024;
+  return L;
+}
+
+__global__ void __launch_bounds__(SH_BLOCK, 1) tc_shrink_kernel(const __grid_constant__ TcPlan P) {
+  const SgmmArgs& a = P.a;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const bool worker = tid < TC_WORKERS;
-  const int K = a.k, R16 = args.R16, N1 = args.N1, K2 = N1;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + TcSmem::BAR);
-  const uint32_t bar_full = smem_u32(bars);                              // [S]  stage loaded
-  const uint32_t bar_empty = smem_u32(bars + TC_STAGES);                 // [S]  stage consumed
-  const uint32_t bar_d1 = smem_u32(bars + 2 * TC_STAGES);                // shrink accumulator ready
-  const uint32_t bar_v = smem_u32(bars + 2 * TC_STAGES + 1);             // V written
-  const uint32_t bar_tfull = smem_u32(bars + 2 * TC_STAGES + 2);         // [NY] tile operands loaded
-  const uint32_t bar_d2full = smem_u32(bars + 2 * TC_STAGES + 2 + TC_NY);      // [2] expand accumulator ready
-  const uint32_t bar_d2empty = smem_u32(bars + 2 * TC_STAGES + 4 + TC_NY);     // [2] expand accumulator read
-  int* s_tok = reinterpret_cast<int*>(smem + TcSmem::META);
-  float* s_g0 = reinterpret_cast<float*>(s_tok + TC_BM);
-  float* s_g1 = s_g0 + TC_BM;
-  volatile int* s_flags = reinterpret_cast<volatile int*>(s_g1 + TC_BM);   // [0] tmem, [2..3] set, [4] bad
-  const uint32_t sU = smem_u32(smem + TcSmem::U);
-  const uint32_t sVH = smem_u32(smem + TcSmem::VH);
-  const uint32_t sVL = smem_u32(smem + TcSmem::VL);
-  unsigned char* sYp = smem + TcSmem::YR;     // rings overlay the stages
-  const uint32_t sY = smem_u32(sYp);
-  const uint32_t sB = smem_u32(smem + TcSmem::BR);
+  const bool worker = tid < SH_WORKERS;
+  const int K = a.k, R16 = P.R16, K2 = P.K2, S = P.stages;
+  const ShSmem L = sh_smem(P.pg * K2, S);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bar);
+  const uint32_t bar_full = smem_u32(bars), bar_empty = smem_u32(bars + S), bar_d1 = smem_u32(bars + 2 * S);
+  int* s_tok = reinterpret_cast<int*>(smem + L.meta);
+  float* s_g0 = reinterpret_cast<float*>(s_tok + TB_M);
+  float* s_g1 = s_g0 + TB_M;
+  volatile int* s_flags = reinterpret_cast<volatile int*>(s_g1 + TB_M);     // [0] tmem [1] e0 [2] e1 [3] bad
+  const __nv_bfloat16** s_arow = reinterpret_cast<const __nv_bfloat16**>(smem + L.meta + 3 * TB_M * 4 + 16);
+  const uint32_t sbase = smem_u32(smem);
 
   if (tid == 0) {
-    for (int i = 0; i < TC_STAGES; ++i) {
-      mbar_init(bar_full + 8 * i, TC_WORKERS + 4);       // A copies of every worker + x rows of every warp
+    for (int i = 0; i < S; ++i) {
+      mbar_init(bar_full + 8 * i, SH_WORKERS);
       mbar_init(bar_empty + 8 * i, 1);
     }
     mbar_init(bar_d1, 1);
-    mbar_init(bar_v, TC_WORKERS);
-    for (int i = 0; i < TC_NY; ++i) mbar_init(bar_tfull + 8 * i, TC_WORKERS + 4);   // Bcat + y_base rows
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(bar_d2full + 8 * i, 1);
-      mbar_init(bar_d2empty + 8 * i, TC_WORKERS);
-    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(const_cast<int*>(s_flags))),
-                 "r"(TC_TMEM_COLS)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-  }
+  if (warp == 0) tmem_alloc(smem_u32(const_cast<int*>(s_flags)), 256);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -156,30 +117,25 @@ __global__ void __launch_bounds__(TC_BLOCK, 1) sgmm_tc_kernel(const __grid_const
   pdl_wait();
   pdl_trigger();
 
-  const WsLayout L = ws_layout(a.T, a.k, a.E);
+  const WsLayout W = ws_layout(a.T, a.k, a.E);
   const WsHeader* hdr = reinterpret_cast<const WsHeader*>(a.ws);
-  const int* tok_order = ws_at<int>(a.ws, L.tok_order);
-  const SetTile* stiles = ws_at<SetTile>(a.ws, L.stiles);
+  const int* tok_order = ws_at<int>(a.ws, W.tok_order);
+  const SetTile* stiles = ws_at<SetTile>(a.ws, W.stiles);
+  TileInfo* tinfo = ws_at<TileInfo>(a.ws, P.tinfo_off);
+  __nv_bfloat16* vprep = ws_at<__nv_bfloat16>(a.ws, P.vprep_off);
   const int nst = hdr->n_stiles;
-  const long nitems = (long)nst * a.nproj;
-  const int d_in = a.d_in;
-  const int nk = d_in / TC_BK;
-  const uint32_t id1 = idesc_bf16(TC_BM, N1);
-  const uint32_t id2 = idesc_bf16(TC_BM, TC_NT);
-  const uint32_t sbo_v = (uint32_t)(K2 / 8) * 128;   // V and Bcat: next 8-row group
-  uint32_t gchunk = 0;      // shrink chunks so far (stage = gchunk % S, use = gchunk / S)
-  uint32_t gtile = 0;       // expand tiles so far (ring slot = gtile % NY, D2 buffer = gtile & 1)
-  uint32_t nitem = 0;       // items so far (parity of d1 / V barriers)
+  const long nitems = (long)nst * P.npg;
+  const __nv_bfloat16* __restrict__ x = reinterpret_cast<const __nv_bfloat16*>(a.x);
+  const int d_in = a.d_in, nk = d_in / TB_BK;
+  uint32_t gchunk = 0, nitem = 0;
   bool abort = false;
 
   for (long item = blockIdx.x; item < nitems; item += gridDim.x) {
-    const int st = (int)(item / a.nproj);
-    const int p = (int)(item % a.nproj);
-    const int d_out = a.proj[p].d_out;
-    const int nnt = (d_out + TC_NT - 1) / TC_NT;
+    const int st = (int)(item / P.npg), q0 = (int)(item % P.npg) * P.pg;
+    const int nq = min(P.pg, a.nproj - q0);
+    const int N1 = nq * K2;
+    const SetTile tile = stiles[st];
     if (worker) {
-      // tokens, their adapter set (sorted) and gates in that order
-      const SetTile tile = stiles[st];
       int tok = -1, e0 = 0, e1 = 0;
       float g0 = 0.f, g1 = 0.f;
       if (tid < tile.len) {
@@ -199,75 +155,73 @@ __global__ void __launch_bounds__(TC_BLOCK, 1) sgmm_tc_kernel(const __grid_const
       s_g0[tid] = g0;
       s_g1[tid] = g1;
       if (tid == 0) {
-        s_flags[2] = e0;
-        s_flags[3] = e1;
-        bool bad = (e0 < 0 || e0 >= a.E || (K == 2 && (e1 < 0 || e1 >= a.E)));
-        if (!bad) {
+        s_flags[1] = e0;
+        s_flags[2] = e1;
+        bool bad = tile.len > 0 && (e0 < 0 || e0 >= a.E || (K == 2 && (e1 < 0 || e1 >= a.E)));
+        if (!bad && tile.len > 0) {
           const int r0 = a.ranks[e0], r1 = K == 2 ? a.ranks[e1] : 8;
-          bad = r0 <= 0 || r0 > R16 || (r0 & 7) || r1 <= 0 || r1 > R16 || (r1 & 7);
+          bad = r0 < 8 || r0 > R16 || (r0 & 7) || r1 < 8 || r1 > R16 || (r1 & 7);
         }
-        s_flags[4] = bad ? 1 : 0;
+        s_flags[3] = bad ? 1 : 0;
         if (bad) report(a.ws, APR_ERR_DEVICE_INDEX, K_TC, e0);
+        if (q0 == 0) tinfo[st] = TileInfo{tile.start, bad ? 0 : tile.len, e0, e1};
       }
     }
     __syncthreads();
-    if (s_flags[4] || abort) {
+    if (s_flags[3] || tile.len <= 0 || abort) {
       __syncthreads();
       continue;
     }
-    const int e0 = s_flags[2], e1 = s_flags[3];
-    const int rk[2] = {a.ranks[e0], K == 2 ? a.ranks[e1] : 0};
-    const uint32_t g0 = gchunk, t0 = gtile;
-    // this warp's 32 token rows as TMA row coordinates (T = past the end: zero fill)
-    int trow[32];
-    if (worker && lane == 0) {
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const int tk = s_tok[warp * 32 + i];
-        trow[i] = tk >= 0 ? tk : a.T;
-      }
-    }
-
+    const int e0 = s_flags[1], e1 = s_flags[2];
+    // source row of every A row of the item (null: a zero row)
     if (worker) {
-      // -------------------------------------------------------- shrink operands
-      const __nv_bfloat16* Aj[2];
-      Aj[0] = reinterpret_cast<const __nv_bfloat16*>(a.proj[p].A[e0]);
-      Aj[1] = K == 2 ? reinterpret_cast<const __nv_bfloat16*>(a.proj[p].A[e1]) : Aj[0];
+      for (int j = tid; j < N1; j += SH_WORKERS) {
+        const int qi = j / K2, rem = j - qi * K2, slot = rem / R16, rr = rem - slot * R16;
+        const int e = slot == 0 ? e0 : e1;
+        const int re = a.ranks[e];
+        s_arow[j] = rr < re ? reinterpret_cast<const __nv_bfloat16*>(a.proj[q0 + qi].A[e]) + (size_t)rr * d_in : nullptr;
+      }
+      asm volatile("bar.sync 1, %0;" ::"n"(SH_WORKERS) : "memory");
+    }
+    const uint32_t g0 = gchunk;
+    if (worker) {
       for (int c = 0; c < nk && !abort; ++c) {
-        const uint32_t g = g0 + c;
-        const uint32_t s = g % TC_STAGES;
-        if (g >= TC_STAGES && !mbar_wait(bar_empty + 8 * s, ((g / TC_STAGES) - 1) & 1)) { abort = true; break; }
-        // x rows of this warp's 32 tokens: 8 TMA gathers of 4 rows x 128 bytes
-        if (lane == 0) {
-          const uint32_t fb = bar_full + 8 * s;
-          mbar_arrive_expect_tx(fb, 8 * 4 * 128);
-          const uint32_t xdst = sU + s * TC_STAGE_BYTES + (uint32_t)(warp * 32) * 128;
+        const uint32_t g = g0 + c, s = g % S;
+        if (g >= (uint32_t)S && !mbar_wait(bar_empty + 8 * s, ((g / S) - 1) & 1)) { abort = true; break; }
+        const uint32_t st_base = sbase + s * L.stage_bytes;
 #pragma unroll
-          for (int g4 = 0; g4 < 8; ++g4)
-            tma_gather4(xdst + g4 * 512, &args.tm_x, c * TC_BK, trow[4 * g4], trow[4 * g4 + 1], trow[4 * g4 + 2],
-                        trow[4 * g4 + 3], fb);
+        for (int m = 0; m < 8; ++m) {          // x rows: 8 lanes per 128-byte row segment
+          const int w = tid + m * SH_WORKERS;
+          const int row = w >> 3, q = w & 7;
+          const int tk = s_tok[row];
+          if (tk >= 0)
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(st_base + (uint32_t)row * 128 +
+                                                                            (uint32_t)((q ^ (row & 7)) << 4)),
+                         "l"(x + (size_t)tk * d_in + (size_t)c * TB_BK + q * 8)
+                         : "memory");
         }
-        const uint32_t abase = sU + s * TC_STAGE_BYTES + TC_BM * 128;
-        for (int w = tid; w < N1 * 8; w += TC_WORKERS) {
+        const uint32_t abase = st_base + TB_M * 128;
+        for (int w = tid; w < N1 * 8; w += SH_WORKERS) {
           const int j = w >> 3, q = w & 7;
-          const int slot = j / R16, r = j % R16;
-          const uint32_t dst = abase + (uint32_t)j * 128 + ((q ^ (j & 7)) << 4);
-          const bool valid = r < rk[slot];
-          cp_async16_zfill(dst, valid ? Aj[slot] + (size_t)r * d_in + (size_t)c * TC_BK + q * 8 : Aj[0], valid);
+          const __nv_bfloat16* src = s_arow[j];
+          cp_async16_zfill(abase + (uint32_t)j * 128 + (uint32_t)((q ^ (j & 7)) << 4),
+                           src ? (const void*)(src + (size_t)c * TB_BK + q * 8) : (const void*)x, src != nullptr);
         }
         cp_async_arrive(bar_full + 8 * s);
       }
-      // -------------------------------------------------------- gates -> V (bf16 hi + lo)
+      // gates -> V rows (bf16 hi | lo) in plan order
       if (!abort && !mbar_wait(bar_d1, nitem & 1)) abort = true;
       tc_fence_after();
       if (!abort) {
-        const int row = tid;                       // TMEM lane = token row
+        const int row = tid;
         const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+        const bool valid = row < tile.len;
         const float ga = s_g0[row], gb = s_g1[row];
         for (int c0 = 0; c0 < N1; c0 += 16) {
           float v[16];
           tmem_ld16(lane_addr + (uint32_t)c0, v);
-          const float gg = (c0 / R16) == 0 ? ga : gb;
+          const int qi = c0 / K2, rem = c0 - qi * K2;
+          const float gg = rem < R16 ? ga : gb;
           uint32_t hi[8], lo[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
@@ -277,522 +231,356 @@ __global__ void __launch_bounds__(TC_BLOCK, 1) sgmm_tc_kernel(const __grid_const
             hi[i] = *reinterpret_cast<const uint32_t*>(&h);
             lo[i] = pack_bf16x2(a0 - hf.x, a1 - hf.y);
           }
-#pragma unroll
-          for (int h8 = 0; h8 < 2; ++h8) {
-            const int kc8 = (c0 >> 3) + h8;
-            const uint32_t off = (uint32_t)(row >> 3) * sbo_v + (uint32_t)kc8 * 128 + (uint32_t)(row & 7) * 16;
-            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(sVH + off), "r"(hi[4 * h8]),
-                         "r"(hi[4 * h8 + 1]), "r"(hi[4 * h8 + 2]), "r"(hi[4 * h8 + 3])
-                         : "memory");
-            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(sVL + off), "r"(lo[4 * h8]),
-                         "r"(lo[4 * h8 + 1]), "r"(lo[4 * h8 + 2]), "r"(lo[4 * h8 + 3])
-                         : "memory");
+          if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(vprep + ((size_t)(q0 + qi) * a.T + tile.start + row) * (2 * K2) + rem);
+            dst[0] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+            dst[1] = make_uint4(hi[4], hi[5], hi[6], hi[7]);
+            uint4* dlo = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(dst) + K2);
+            dlo[0] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            dlo[1] = make_uint4(lo[4], lo[5], lo[6], lo[7]);
           }
         }
-        fence_proxy_async();
-        tc_fence_before();
-        mbar_arrive(bar_v);
       }
-      // -------------------------------------------------------- expand operands and epilogues
-      const __nv_bfloat16* Bj[2];
-      Bj[0] = reinterpret_cast<const __nv_bfloat16*>(a.proj[p].B[e0]);
-      Bj[1] = K == 2 ? reinterpret_cast<const __nv_bfloat16*>(a.proj[p].B[e1]) : Bj[0];
-      __nv_bfloat16* __restrict__ y = reinterpret_cast<__nv_bfloat16*>(a.proj[p].y);
-      auto issue_tile = [&](int nt) {
-        const uint32_t slot = (t0 + nt) % TC_NY;
-        const int n0 = nt * TC_NT;
-        const int ncols = min(TC_NT, d_out - n0);
-        const uint32_t bbase = sB + slot * TC_BBUF_BYTES;
-        const int cpr = K2 / 8;
-        for (int w = tid; w < TC_NT * cpr; w += TC_WORKERS) {
-          const int n = w / cpr, q = w % cpr;
-          const int kslot = q / (R16 / 8), cq = q % (R16 / 8);
-          const uint32_t dst = bbase + (uint32_t)(n >> 3) * sbo_v + (uint32_t)q * 128 + (uint32_t)(n & 7) * 16;
-          const bool valid = n < ncols && cq * 8 < rk[kslot];
-          cp_async16_zfill(dst, valid ? Bj[kslot] + (size_t)(n0 + n) * rk[kslot] + cq * 8 : Bj[0], valid);
-        }
-        cp_async_arrive(bar_tfull + 8 * slot);
-        // y_base rows of this warp's tokens: TMA gathers into the two swizzled 64-column halves
-        if (lane == 0) {
-          bulk_wait_read_all();                    // this warp's stores from the slot are read out
-          const uint32_t tb = bar_tfull + 8 * slot;
-          const int nh = (ncols + 63) / 64;
-          mbar_arrive_expect_tx(tb, nh * 8 * 4 * 128);
-          for (int h = 0; h < nh; ++h) {
-            const uint32_t ydst = sY + slot * TC_YBUF_BYTES + h * (TC_BM * 128) + (uint32_t)(warp * 32) * 128;
-#pragma unroll
-            for (int g4 = 0; g4 < 8; ++g4)
-              tma_gather4(ydst + g4 * 512, &args.tm_yb[p], n0 + 64 * h, trow[4 * g4], trow[4 * g4 + 1],
-                          trow[4 * g4 + 2], trow[4 * g4 + 3], tb);
-          }
-        }
-      };
-      for (int nt = 0; nt < TC_NY - 1 && nt < nnt && !abort; ++nt) issue_tile(nt);
-      for (int nt = 0; nt < nnt && !abort; ++nt) {
-        const uint32_t g = t0 + nt;
-        const uint32_t slot = g % TC_NY, b = g & 1;
-        const int n0 = nt * TC_NT;
-        const int ncols = min(TC_NT, d_out - n0);
-        if (nt + TC_NY - 1 < nnt) issue_tile(nt + TC_NY - 1);   // slot of tile nt-1: consumed
-        if (!mbar_wait(bar_tfull + 8 * slot, (g / TC_NY) & 1)) { abort = true; break; }
-        if (!mbar_wait(bar_d2full + 8 * b, (g >> 1) & 1)) { abort = true; break; }
-        tc_fence_after();
-        const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16) + TC_D2_COL + b * TC_NT;
-        unsigned char* yslot = sYp + (size_t)slot * TC_YBUF_BYTES;
-        const int sw = tid & 7;
-        const bool mine = s_tok[tid] >= 0;
-        for (int c0 = 0; c0 < ncols; c0 += 16) {
-          float v[16];
-          tmem_ld16(lane_addr + (uint32_t)c0, v);
-          if (mine) {
-            const int h = c0 >> 6, q = (c0 & 63) >> 3;
-            unsigned char* rbase = yslot + (size_t)h * (TC_BM * 128) + (size_t)tid * 128;
-            uint4* p0 = reinterpret_cast<uint4*>(rbase + ((q ^ sw) << 4));
-            uint4* p1 = reinterpret_cast<uint4*>(rbase + (((q + 1) ^ sw) << 4));
-            uint4 u0 = *p0, u1 = *p1;
-            __nv_bfloat162* h0 = reinterpret_cast<__nv_bfloat162*>(&u0);
-            __nv_bfloat162* h1 = reinterpret_cast<__nv_bfloat162*>(&u1);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const float2 f0 = __bfloat1622float2(h0[i]);
-              const float2 f1 = __bfloat1622float2(h1[i]);
-              h0[i] = __floats2bfloat162_rn(f0.x + v[2 * i], f0.y + v[2 * i + 1]);
-              h1[i] = __floats2bfloat162_rn(f1.x + v[8 + 2 * i], f1.y + v[8 + 2 * i + 1]);
-            }
-            *p0 = u0;
-            *p1 = u1;
-          }
-        }
-        tc_fence_before();
-        mbar_arrive(bar_d2empty + 8 * b);          // D2[b] may be overwritten
-        // rows of a 4-row group with a missing token are written by their owners ...
-        const int g4 = (tid & 31) >> 2;
-        const bool full_group = s_tok[warp * 32 + 4 * g4] >= 0 && s_tok[warp * 32 + 4 * g4 + 1] >= 0 &&
-                                s_tok[warp * 32 + 4 * g4 + 2] >= 0 && s_tok[warp * 32 + 4 * g4 + 3] >= 0;
-        if (mine && !full_group) {
-          for (int qq = 0; qq < ncols / 8; ++qq) {
-            const int h = qq >> 3, q = qq & 7;
-            const uint4 val = *reinterpret_cast<const uint4*>(yslot + (size_t)h * (TC_BM * 128) + (size_t)tid * 128 +
-                                                              ((q ^ sw) << 4));
-            *reinterpret_cast<uint4*>(y + (size_t)s_tok[tid] * d_out + n0 + qq * 8) = val;
-          }
-        }
-        // ... and full groups leave by TMA scatter, 4 rows x 64 columns per instruction
-        fence_proxy_async();
-        __syncwarp();
-        if (lane == 0) {
-          const int nh = (ncols + 63) / 64;
-          for (int gg = 0; gg < 8; ++gg) {
-            const int r = warp * 32 + 4 * gg;
-            if (s_tok[r] < 0 || s_tok[r + 1] < 0 || s_tok[r + 2] < 0 || s_tok[r + 3] < 0) continue;
-            for (int h = 0; h < nh; ++h)
-              tma_scatter4(&args.tm_y[p], n0 + 64 * h, s_tok[r], s_tok[r + 1], s_tok[r + 2], s_tok[r + 3],
-                           smem_u32(yslot + (size_t)h * (TC_BM * 128) + (size_t)r * 128));
-          }
-          bulk_commit();
-        }
-        __syncwarp();
-      }
-      // the next item's stages overlay the y ring: this warp's stores must have read it out
-      if (lane == 0) bulk_wait_read_all();
-      cp_async_wait_all();
     } else if (lane == 0) {
-      // -------------------------------------------------------- MMA issue (one thread)
+      const uint32_t id = idesc_bf16(TB_M, N1);
       for (int c = 0; c < nk && !abort; ++c) {
-        const uint32_t g = g0 + c;
-        const uint32_t s = g % TC_STAGES;
-        if (!mbar_wait(bar_full + 8 * s, (g / TC_STAGES) & 1)) { abort = true; break; }
+        const uint32_t g = g0 + c, s = g % S;
+        if (!mbar_wait(bar_full + 8 * s, (g / S) & 1)) { abort = true; break; }
         tc_fence_after();
-        const uint32_t xs = sU + s * TC_STAGE_BYTES;
-        const uint32_t as = xs + TC_BM * 128;
+        const uint32_t xs = sbase + s * L.stage_bytes, as = xs + TB_M * 128;
 #pragma unroll
-        for (int kk = 0; kk < TC_BK / 16; ++kk)
-          mma_bf16(tmem, desc_k_sw128(xs + kk * 32), desc_k_sw128(as + kk * 32), id1, (c > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < TB_BK / 16; ++kk)
+          mma_bf16(tmem, desc_k_sw128(xs + kk * 32), desc_k_sw128(as + kk * 32), id, (c > 0 || kk > 0) ? 1u : 0u);
         mma_commit(bar_empty + 8 * s);
       }
       if (!abort) mma_commit(bar_d1);
-      if (!abort && !mbar_wait(bar_v, nitem & 1)) abort = true;
-      tc_fence_after();
-      for (int nt = 0; nt < nnt && !abort; ++nt) {
-        const uint32_t g = t0 + nt;
-        const uint32_t slot = g % TC_NY, b = g & 1;
-        if (!mbar_wait(bar_tfull + 8 * slot, (g / TC_NY) & 1)) { abort = true; break; }
-        if (g >= 2 && !mbar_wait(bar_d2empty + 8 * b, ((g >> 1) - 1) & 1)) { abort = true; break; }
-        tc_fence_after();
-        const uint32_t bb = sB + slot * TC_BBUF_BYTES;
-        const uint32_t dcol = tmem + TC_D2_COL + b * TC_NT;
-        for (int kk = 0; kk < K2 / 16; ++kk)
-          mma_bf16(dcol, desc_k_plain(sVH + kk * 256, 128, sbo_v), desc_k_plain(bb + kk * 256, 128, sbo_v), id2,
-                   kk > 0 ? 1u : 0u);
-        for (int kk = 0; kk < K2 / 16; ++kk)
-          mma_bf16(dcol, desc_k_plain(sVL + kk * 256, 128, sbo_v), desc_k_plain(bb + kk * 256, 128, sbo_v), id2, 1u);
-        mma_commit(bar_d2full + 8 * b);
-      }
     }
     gchunk = g0 + nk;
-    gtile = t0 + nnt;
     ++nitem;
+    tc_fence_before();
     abort = __syncthreads_or(abort);
+    tc_fence_after();
   }
   if (abort && tid == 0) report(a.ws, APR_ERR_TIMEOUT, K_TC, (int)blockIdx.x);
   cp_async_wait_all();
-  if (lane == 0) bulk_wait_all();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 0) {
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TC_TMEM_COLS)
-                 : "memory");
+  if (warp == 0) tmem_dealloc(tmem, 256);
+}
+
+// ---------------------------------------------------------------- expand
+
+struct ExSmem {
+  int K2, ny;
+  size_t vbuf, y, b, bar, total;
+};
+__host__ __device__ inline ExSmem ex_smem(int K2, int ny) {
+  ExSmem L;
+  L.K2 = K2;
+  L.ny = ny;
+  L.vbuf = (size_t)2 * TB_M * K2 * 2;                 // one V buffer: hi then lo
+  L.y = 2 * L.vbuf;                                   // ring of y tiles [128 rows][256 B]
+  L.b = L.y + (size_t)ny * TB_M * 256;                // ring of Bcat tiles [128][K2] bf16
+  L.bar = L.b + (size_t)ny * TB_NT * K2 * 2;
+  L.total = L.bar + (size_t)(2 * ny + 8) * 8 + 16 + 1024;
+  return L;
+}
+
+struct ExItem {
+  int start, len, p, n0, ntl, d_out, tok;
+  const __nv_bfloat16* B0;
+  const __nv_bfloat16* B1;
+  int r0, r1;
+};
+
+__global__ void __launch_bounds__(EX_BLOCK, 1) tc_expand_kernel(const __grid_constant__ TcPlan P) {
+  const SgmmArgs& a = P.a;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem =
+      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int K = a.k, R16 = P.R16, K2 = P.K2, NY = P.ny;
+  const ExSmem L = ex_smem(K2, NY);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bar);
+  const uint32_t bar_tfull = smem_u32(bars);                  // [NY] tile operands landed
+  const uint32_t bar_vfull = smem_u32(bars + NY);             // [2]  V of an item landed
+  const uint32_t bar_vempty = smem_u32(bars + NY + 2);        // [2]  V of an item consumed by the MMAs
+  const uint32_t bar_d2full = smem_u32(bars + NY + 4);        // [2]  accumulator ready
+  const uint32_t bar_d2empty = smem_u32(bars + NY + 6);       // [2]  accumulator read
+  volatile uint32_t* s_tmem = reinterpret_cast<volatile uint32_t*>(bars + 2 * NY + 8);
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t SBO = (uint32_t)(K2 / 8) * 128;              // next 8-row group of a K-major operand
+
+  if (tid == 0) {
+    for (int i = 0; i < NY; ++i) mbar_init(bar_tfull + 8 * i, EX_WORKERS);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar_vfull + 8 * i, EX_WORKERS);
+      mbar_init(bar_vempty + 8 * i, 1);
+      mbar_init(bar_d2full + 8 * i, 1);
+      mbar_init(bar_d2empty + 8 * i, EX_WORKERS);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  if (warp == 0) tmem_alloc(smem_u32(const_cast<uint32_t*>(s_tmem)), 256);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+
+  pdl_wait();
+  pdl_trigger();
+
+  const WsLayout W = ws_layout(a.T, a.k, a.E);
+  const WsHeader* hdr = reinterpret_cast<const WsHeader*>(a.ws);
+  const int* tok_order = ws_at<int>(a.ws, W.tok_order);
+  const TileInfo* tinfo = ws_at<TileInfo>(a.ws, P.tinfo_off);
+  const __nv_bfloat16* vprep = ws_at<__nv_bfloat16>(a.ws, P.vprep_off);
+  const int ipt = P.cc_before[a.nproj];
+  const long nitems = (long)hdr->n_stiles * ipt;
+  auto item_at = [&](int i) -> long { return (long)blockIdx.x + (long)i * gridDim.x; };
+  // item -> (set tile, projection, first column, tiles)
+  auto item_shape = [&](long it, int& st, int& p, int& n0, int& ntl, int& d_out) {
+    st = (int)(it / ipt);
+    const int loc = (int)(it - (long)st * ipt);
+    p = 0;
+    while (p + 1 < a.nproj && loc >= P.cc_before[p + 1]) ++p;
+    d_out = a.proj[p].d_out;
+    n0 = (loc - P.cc_before[p]) * TB_CW;
+    ntl = (min(TB_CW, d_out - n0) + TB_NT - 1) / TB_NT;
+  };
+  bool abort = false;
+
+  if (tid < EX_WORKERS) {
+    const int row = tid & (TB_M - 1), half = tid >> 7;
+    auto load_item = [&](int i, ExItem& I) {
+      int st;
+      item_shape(item_at(i), st, I.p, I.n0, I.ntl, I.d_out);
+      const TileInfo ti = tinfo[st];
+      I.start = ti.start;
+      I.len = ti.len;
+      I.tok = row < ti.len ? tok_order[ti.start + row] : -1;
+      I.B0 = I.B1 = nullptr;
+      I.r0 = I.r1 = 0;
+      if (ti.len > 0) {
+        I.B0 = reinterpret_cast<const __nv_bfloat16*>(a.proj[I.p].B[ti.e0]);
+        I.r0 = a.ranks[ti.e0];
+        if (K == 2) {
+          I.B1 = reinterpret_cast<const __nv_bfloat16*>(a.proj[I.p].B[ti.e1]);
+          I.r1 = a.ranks[ti.e1];
+        }
+      }
+    };
+    // V rows of item i (this thread: row `row`, half hi/lo) into V buffer i & 1
+    auto issue_v = [&](int i, const ExItem& I) {
+      const uint32_t buf = sbase + (uint32_t)((i & 1) * L.vbuf) + (uint32_t)half * (TB_M * K2 * 2);
+      const bool valid = row < I.len;
+      const __nv_bfloat16* src = vprep + ((size_t)I.p * a.T + I.start + row) * (2 * K2) + half * K2;
+      for (int q = 0; q < K2 / 8; ++q)
+        cp_async16_zfill(buf + (uint32_t)(row >> 3) * SBO + (uint32_t)q * 128 + (uint32_t)(row & 7) * 16,
+                         valid ? (const void*)(src + q * 8) : (const void*)vprep, valid);
+      cp_async_arrive(bar_vfull + 8 * (i & 1));
+    };
+    // y_base rows and Bcat of tile t of item I into ring slot `slot`
+    auto issue_tile = [&](const ExItem& I, int t, uint32_t slot) {
+      const int n0 = I.n0 + t * TB_NT;
+      const uint32_t ybuf = sbase + (uint32_t)L.y + slot * (TB_M * 256);
+      if (I.tok >= 0) {
+        const __nv_bfloat16* src = reinterpret_cast<const __nv_bfloat16*>(a.proj[I.p].y_base) +
+                                   (size_t)I.tok * I.d_out + n0 + half * 64;
+        const uint32_t dst = ybuf + (uint32_t)row * 256 + (uint32_t)half * 128;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const bool ok = n0 + half * 64 + q * 8 < I.d_out;
+          cp_async16_zfill(dst + (uint32_t)((q ^ (row & 7)) << 4), ok ? (const void*)(src + q * 8) : (const void*)src, ok);
+        }
+      }
+      const uint32_t bbuf = sbase + (uint32_t)L.b + slot * (uint32_t)(TB_NT * K2 * 2);
+      const int cpr = K2 / 8, cps = R16 / 8;
+      for (int w = tid; w < TB_NT * cpr; w += EX_WORKERS) {
+        const int n = w / cpr, kq = w - n * cpr;
+        const int slot_a = kq / cps, cq = kq - slot_a * cps;
+        const __nv_bfloat16* B = slot_a == 0 ? I.B0 : I.B1;
+        const int re = slot_a == 0 ? I.r0 : I.r1;
+        const bool ok = B != nullptr && n0 + n < I.d_out && cq * 8 < re;
+        cp_async16_zfill(bbuf + (uint32_t)(n >> 3) * SBO + (uint32_t)kq * 128 + (uint32_t)(n & 7) * 16,
+                         ok ? (const void*)(B + (size_t)(n0 + n) * re + cq * 8) : (const void*)vprep, ok);
+      }
+      cp_async_arrive(bar_tfull + 8 * slot);
+    };
+
+    ExItem prod, cons;
+    int prod_i = 0, prod_t = 0, cons_i = 0, cons_t = 0;
+    uint32_t gp = 0, gc = 0;
+    bool prod_live = item_at(0) < nitems;
+    if (prod_live) {
+      load_item(0, prod);
+      issue_v(0, prod);
+    }
+    cons = prod;
+    while (!abort) {
+      // ------------------------------------------------ producer: up to NY - 1 tiles ahead
+      while (prod_live && gp < gc + (uint32_t)(NY - 1)) {
+        if (prod_t == prod.ntl) {
+          if (prod_i + 1 > cons_i + 1) break;                 // at most one item ahead of the epilogue
+          if (item_at(prod_i + 1) >= nitems) { prod_live = false; break; }
+          ++prod_i;
+          prod_t = 0;
+          load_item(prod_i, prod);
+          if (prod_i == cons_i) cons = prod;
+          if (prod_i >= 2 && !mbar_wait(bar_vempty + 8 * (prod_i & 1), ((prod_i >> 1) - 1) & 1)) { abort = true; break; }
+          issue_v(prod_i, prod);
+        }
+        issue_tile(prod, prod_t, gp % NY);
+        ++gp;
+        ++prod_t;
+      }
+      if (abort || gc == gp) break;
+      // ------------------------------------------------ epilogue of tile gc
+      const uint32_t slot = gc % NY, b = gc & 1;
+      if (!mbar_wait(bar_tfull + 8 * slot, (gc / NY) & 1)) { abort = true; break; }
+      if (!mbar_wait(bar_d2full + 8 * b, (gc >> 1) & 1)) { abort = true; break; }
+      tc_fence_after();
+      const int n0 = cons.n0 + cons_t * TB_NT;
+      const int ncols = min(TB_NT, cons.d_out - n0);
+      unsigned char* yrow = smem + L.y + (size_t)slot * (TB_M * 256) + (size_t)row * 256 + half * 128;
+      const uint32_t taddr = tmem + ((uint32_t)((warp & 3) * 32) << 16) + b * 128 + (uint32_t)half * 64;
+#pragma unroll
+      for (int c16 = 0; c16 < 4; ++c16) {
+        float v[16];
+        tmem_ld16(taddr + (uint32_t)(c16 * 16), v);
+        if (cons.tok >= 0) {
+          uint4* p0 = reinterpret_cast<uint4*>(yrow + (((2 * c16) ^ (row & 7)) << 4));
+          uint4* p1 = reinterpret_cast<uint4*>(yrow + (((2 * c16 + 1) ^ (row & 7)) << 4));
+          uint4 u0 = *p0, u1 = *p1;
+          __nv_bfloat162* h0 = reinterpret_cast<__nv_bfloat162*>(&u0);
+          __nv_bfloat162* h1 = reinterpret_cast<__nv_bfloat162*>(&u1);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 f0 = __bfloat1622float2(h0[i]);
+            const float2 f1 = __bfloat1622float2(h1[i]);
+            h0[i] = __floats2bfloat162_rn(f0.x + v[2 * i], f0.y + v[2 * i + 1]);
+            h1[i] = __floats2bfloat162_rn(f1.x + v[8 + 2 * i], f1.y + v[8 + 2 * i + 1]);
+          }
+          *p0 = u0;
+          *p1 = u1;
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar_d2empty + 8 * b);
+      __syncwarp();
+      // the warp's 32 rows x 128 bytes: 8 lanes per row segment
+      {
+        __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(a.proj[cons.p].y);
+        const int wrow0 = (warp & 3) * 32;
+        const int q = lane & 7;
+        const int col = half * 64 + q * 8;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int rr = 4 * i + (lane >> 3);
+          const int tk = __shfl_sync(0xffffffffu, cons.tok, rr);
+          const int r = wrow0 + rr;
+          if (tk >= 0 && col < ncols) {
+            const uint4 val = *reinterpret_cast<const uint4*>(smem + L.y + (size_t)slot * (TB_M * 256) + (size_t)r * 256 +
+                                                              half * 128 + ((q ^ (r & 7)) << 4));
+            __stcs(reinterpret_cast<uint4*>(y + (size_t)tk * cons.d_out + n0 + col), val);
+          }
+        }
+      }
+      __syncwarp();
+      ++gc;
+      if (++cons_t == cons.ntl) {
+        ++cons_i;
+        cons_t = 0;
+        if (prod_i == cons_i) cons = prod;
+      }
+    }
+  } else if (lane == 0) {
+    // ---------------------------------------------------- MMA issue
+    const uint32_t id = idesc_bf16(TB_M, TB_NT);
+    uint32_t g = 0;
+    for (int i = 0; item_at(i) < nitems && !abort; ++i) {
+      int st, p, n0, ntl, d_out;
+      item_shape(item_at(i), st, p, n0, ntl, d_out);
+      if (!mbar_wait(bar_vfull + 8 * (i & 1), (i >> 1) & 1)) { abort = true; break; }
+      const uint32_t vh = sbase + (uint32_t)((i & 1) * L.vbuf), vl = vh + (uint32_t)(TB_M * K2 * 2);
+      for (int t = 0; t < ntl; ++t, ++g) {
+        const uint32_t slot = g % NY, b = g & 1;
+        if (!mbar_wait(bar_tfull + 8 * slot, (g / NY) & 1)) { abort = true; break; }
+        if (g >= 2 && !mbar_wait(bar_d2empty + 8 * b, ((g >> 1) - 1) & 1)) { abort = true; break; }
+        tc_fence_after();
+        const uint32_t bb = sbase + (uint32_t)L.b + slot * (uint32_t)(TB_NT * K2 * 2);
+        const uint32_t dcol = tmem + b * 128;
+        for (int kk = 0; kk < K2 / 16; ++kk)
+          mma_bf16(dcol, desc_k_plain(vh + kk * 256, 128, SBO), desc_k_plain(bb + kk * 256, 128, SBO), id, kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < K2 / 16; ++kk)
+          mma_bf16(dcol, desc_k_plain(vl + kk * 256, 128, SBO), desc_k_plain(bb + kk * 256, 128, SBO), id, 1u);
+        mma_commit(bar_d2full + 8 * b);
+      }
+      if (!abort) mma_commit(bar_vempty + 8 * (i & 1));
+    }
+  }
+  abort = __syncthreads_or(abort);
+  if (abort && tid == 0) report(a.ws, APR_ERR_TIMEOUT, K_TC, (int)blockIdx.x);
+  cp_async_wait_all();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, 256);
 }
 
 // ---------------------------------------------------------------- host side
 
-static int round16(int r) { return (r + 15) / 16 * 16; }
-
 bool sgmm_tensor_supported(const SgmmArgs& a, int dtype) {
   if (dtype != APR_BF16) return false;
   if (a.k < 1 || a.k > 2) return false;
-  if (a.k * round16(a.max_rank) > TC_MAXN1) return false;
-  if (a.d_in % TC_BK != 0) return false;
+  if (a.k * round16i(a.max_rank) > TB_MAXK2) return false;
+  if (a.d_in % TB_BK != 0) return false;
   for (int p = 0; p < a.nproj; ++p)
     if (a.proj[p].d_out % 16 != 0) return false;
   return true;
 }
 
-// cuTensorMapEncodeTiled, fetched through the runtime (no link against libcuda).
-static PFN_cuTensorMapEncodeTiled tensor_map_encoder() {
-  static PFN_cuTensorMapEncodeTiled fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled>(p);
-  });
-  return fn;
-}
-
-// Row-major bf16 [rows, cols] matrix seen by TMA as boxes of one row x 64
-// columns (128 bytes) with the 128-byte swizzle; reads past the last row or
-// column return zeros, writes there are dropped.
-static bool encode_rows(PFN_cuTensorMapEncodeTiled enc, CUtensorMap* m, const void* base, int rows, int cols) {
-  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-  const cuuint32_t box[2] = {64, 1};
-  const cuuint32_t estr[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-cudaError_t launch_sgmm_tensor(const SgmmArgs& a, cudaStream_t s) {
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t err = cudaFuncSetAttribute(sgmm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           (int)TcSmem::ALLOC);
-    if (err != cudaSuccess) return err;
-    configured = true;
-  }
-  PFN_cuTensorMapEncodeTiled enc = tensor_map_encoder();
-  if (!enc) return cudaErrorNotSupported;
-  int dev = 0, nsm = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-  TcArgs t;
+cudaError_t launch_sgmm_tensor(const SgmmArgs& a, size_t scratch_off, cudaStream_t s) {
+  TcPlan t;
   memset(&t, 0, sizeof(t));
   t.a = a;
-  t.R16 = round16(a.max_rank);
-  t.N1 = a.k * t.R16;
-  if (!encode_rows(enc, &t.tm_x, a.x, a.T, a.d_in)) return cudaErrorInvalidValue;
-  for (int p = 0; p < a.nproj; ++p) {
-    if (!encode_rows(enc, &t.tm_yb[p], a.proj[p].y_base, a.T, a.proj[p].d_out) ||
-        !encode_rows(enc, &t.tm_y[p], a.proj[p].y, a.T, a.proj[p].d_out))
-      return cudaErrorInvalidValue;
+  t.R16 = round16i(a.max_rank);
+  t.K2 = a.k * t.R16;
+  t.pg = TB_MAXN1 / t.K2;
+  if (t.pg > a.nproj) t.pg = a.nproj;
+  t.npg = (a.nproj + t.pg - 1) / t.pg;
+  const int n1max = t.pg * t.K2;
+  t.stages = (int)((SMEM_BUDGET - 4096) / (TB_M * 128 + n1max * 128));
+  if (t.stages > 8) t.stages = 8;
+  t.ny = t.K2 <= 32 ? 4 : 3;
+  t.vprep_off = scratch_off;
+  t.tinfo_off = scratch_off + align_up(tc_vprep_bytes(a.T, t.K2));   // layout as in tc_scratch_bytes
+  t.cc_before[0] = 0;
+  for (int p = 0; p < a.nproj; ++p) t.cc_before[p + 1] = t.cc_before[p] + (a.proj[p].d_out + TB_CW - 1) / TB_CW;
+
+  const size_t sm1 = sh_smem(n1max, t.stages).total, sm2 = ex_smem(t.K2, t.ny).total;
+  static size_t conf1 = 0, conf2 = 0;
+  cudaError_t err;
+  if (sm1 > conf1) {
+    if ((err = cudaFuncSetAttribute(tc_shrink_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1)) != cudaSuccess)
+      return err;
+    conf1 = sm1;
   }
-  // upper bound on items: set tiles <= T (one per token at worst); the kernel loops over the real count
-  long max_items = (long)((a.T + TC_BM - 1) / TC_BM + a.T) * a.nproj;
-  int grid = nsm;
-  if (max_items < grid) grid = (int)max_items;
-  return launch_pdl(sgmm_tc_kernel, dim3(grid), dim3(TC_BLOCK), TcSmem::ALLOC, s, t);
-}
-
-
-// ---------------------------------------------------------------- merge on the tensor cores
-//
-// Batch-1 merge (AdaFuse summary §2.B decoding steps 3 and 5), every weight in
-// one launch, out of place:  W' = W + sum_j g_j B_{e_j} A_{e_j}.
-// A work item is a strip of 128 rows of one weight.  The strip's gated B rows
-// Bg[n][j*R16 + i] = g_j B_{e_j}[n][i] are formed once (fp32 -> bf16 hi + lo,
-// K-major), then for every 128-column tile: D[128 x 128] = Bg_hi.A^T +
-// Bg_lo.A^T on tcgen05 with A^T as an MN-major operand (rows of A_e are
-// contiguous along the output columns), TMEM double buffered; the W tile and
-// the A tile arrive two tiles ahead by cp.async into 3-deep rings, and the
-// epilogue adds D to W in fp32, rounds once and the warp writes its 32 rows
-// of W' back with coalesced 128-bit stores.
-
-constexpr int MT_BN = 128;                      // columns per tile
-constexpr int MT_NY = 3;                        // ring depth
-constexpr int MT_WSTRIDE = MT_BN * 2 + 16;      // bytes per staged W row
-constexpr int MT_WBUF = TC_BM * MT_WSTRIDE;
-constexpr int MT_ABUF = MT_BN * TC_MAXN1 * 2;   // MN-major A^T tile
-constexpr int MT_MAXPROJ = 4096;
-
-struct MtSmem {
-  static constexpr size_t GH = 0;                                        // 16 KB
-  static constexpr size_t GL = GH + (size_t)TC_BM * TC_MAXN1 * 2;        // 16 KB
-  static constexpr size_t WR = GL + (size_t)TC_BM * TC_MAXN1 * 2;        // W ring
-  static constexpr size_t AR = WR + (size_t)MT_NY * MT_WBUF;             // A ring
-  static constexpr size_t BAR = AR + (size_t)MT_NY * MT_ABUF;
-  static constexpr size_t META = BAR + 2 * 8;
-  static constexpr size_t PREF = META + 128;                             // [nproj + 1] strip prefix
-  static constexpr size_t fixed_bytes() { return PREF + 1024; }
-};
-
-// K-major A operand / MN-major B operand instruction descriptor (bf16 -> fp32).
-__host__ __device__ constexpr uint32_t idesc_bf16_bmn(int M, int N) { return idesc_bf16(M, N) | (1u << 16); }
-
-__global__ void __launch_bounds__(TC_THREADS, 1) merge_tc_kernel(const apr_merge_proj* __restrict__ projs,
-                                                                 int nproj, int E, int r, int R16,
-                                                                 const int32_t* __restrict__ idx,
-                                                                 const float* __restrict__ gate, int k,
-                                                                 void* ws) {
-  extern __shared__ unsigned char smem_raw[];
-  unsigned char* smem =
-      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int K = k * R16;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + MtSmem::BAR);
-  const uint32_t bar_mma = smem_u32(bars);                     // [2]
-  volatile int* s_flags = reinterpret_cast<volatile int*>(smem + MtSmem::META);   // [0] tmem, [1] bad
-  int* s_e = const_cast<int*>(s_flags) + 4;                    // [<= 8]
-  float* s_g = reinterpret_cast<float*>(s_e + 8);              // [<= 8]
-  int* s_pref = reinterpret_cast<int*>(smem + MtSmem::PREF);
-  const uint32_t sGH = smem_u32(smem + MtSmem::GH);
-  const uint32_t sGL = smem_u32(smem + MtSmem::GL);
-  unsigned char* sWp = smem + MtSmem::WR;
-  const uint32_t sW = smem_u32(sWp);
-  const uint32_t sA = smem_u32(smem + MtSmem::AR);
-
-  if (tid == 0) {
-    for (int i = 0; i < 2; ++i) mbar_init(bar_mma + 8 * i, 1);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    s_flags[1] = 0;
-  }
-  if (warp == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(const_cast<int*>(s_flags))),
-                 "r"(TC_TMEM_COLS)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = (uint32_t)s_flags[0];
-  pdl_wait();
-  pdl_trigger();
-
-  if (tid < k) {
-    const int e = idx[tid];
-    if (e < 0 || e >= E) s_flags[1] = 1;
-    s_e[tid] = e;
-    s_g[tid] = gate[tid];
-  }
-  // strips (128 rows) per weight, prefix over the weights
-  if (tid == 0) {
-    int acc = 0;
-    s_pref[0] = 0;
-    for (int p = 0; p < nproj; ++p) {
-      acc += (projs[p].d_out + TC_BM - 1) / TC_BM;
-      s_pref[p + 1] = acc;
-    }
-  }
-  __syncthreads();
-  bool abort = false;
-  if (s_flags[1]) {
-    if (tid == 0 && blockIdx.x == 0) report(ws, APR_ERR_DEVICE_INDEX, K_MERGE, 0);
-  } else {
-    const int total = s_pref[nproj];
-    const uint32_t sbo_g = (uint32_t)(K / 8) * 128;         // Bg: next 8-row group
-    const uint32_t id = idesc_bf16_bmn(TC_BM, MT_BN);
-    uint32_t ph_mma = 0;
-    for (int strip = blockIdx.x; strip < total && !abort; strip += gridDim.x) {
-      int lo = 0, hi = nproj;                                 // weight of this strip
-      while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (s_pref[mid] <= strip) lo = mid; else hi = mid;
-      }
-      const apr_merge_proj pj = projs[lo];
-      const int row0 = (strip - s_pref[lo]) * TC_BM;
-      const int nrows = min(TC_BM, pj.d_out - row0);
-      const __nv_bfloat16* __restrict__ Wt = reinterpret_cast<const __nv_bfloat16*>(pj.W);
-      __nv_bfloat16* __restrict__ Wp = reinterpret_cast<__nv_bfloat16*>(pj.Wp);
-      // gated B rows of the strip, bf16 hi + lo, K-major
-      {
-        const int n = row0 + tid;
-        for (int j = 0; j < k; ++j) {
-          const __nv_bfloat16* B = reinterpret_cast<const __nv_bfloat16*>(pj.B[s_e[j]]);
-          for (int c8 = 0; c8 < R16; c8 += 8) {
-            float f[8];
-            if (tid < nrows && c8 < r) {
-              load8(B + (size_t)n * r + c8, f);
-            } else {
-#pragma unroll
-              for (int i = 0; i < 8; ++i) f[i] = 0.f;
-            }
-            uint32_t h4[4], l4[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const float a0 = f[2 * i] * s_g[j], a1 = f[2 * i + 1] * s_g[j];
-              const __nv_bfloat162 hh = __floats2bfloat162_rn(a0, a1);
-              const float2 hf = __bfloat1622float2(hh);
-              h4[i] = *reinterpret_cast<const uint32_t*>(&hh);
-              l4[i] = pack_bf16x2(a0 - hf.x, a1 - hf.y);
-            }
-            const int kc8 = (j * R16 + c8) >> 3;
-            const uint32_t off = (uint32_t)(tid >> 3) * sbo_g + (uint32_t)kc8 * 128 + (uint32_t)(tid & 7) * 16;
-            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(sGH + off), "r"(h4[0]), "r"(h4[1]),
-                         "r"(h4[2]), "r"(h4[3])
-                         : "memory");
-            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(sGL + off), "r"(l4[0]), "r"(l4[1]),
-                         "r"(l4[2]), "r"(l4[3])
-                         : "memory");
-          }
-        }
-      }
-      fence_proxy_async();                       // Bg was written by ordinary stores
-      const int nct = (pj.d_in + MT_BN - 1) / MT_BN;
-      auto issue_tile = [&](int ct) {
-        const int slot = ct % MT_NY;
-        const int c0 = ct * MT_BN;
-        const int ncols = min(MT_BN, pj.d_in - c0);
-        // A^T tile, MN-major: core matrix (8 columns x 8 rank rows) at (col/8)*128 + (kk/8)*2048
-        const uint32_t abase = sA + (uint32_t)slot * MT_ABUF;
-        for (int w = tid; w < K * (MT_BN / 8); w += TC_THREADS) {
-          const int kk = w / (MT_BN / 8), c = w % (MT_BN / 8);
-          const int j = kk / R16, i = kk % R16;
-          const uint32_t dst = abase + (uint32_t)c * 128 + (uint32_t)(kk >> 3) * 2048 + (uint32_t)(kk & 7) * 16;
-          const bool valid = i < r && c * 8 < ncols;
-          const __nv_bfloat16* A = reinterpret_cast<const __nv_bfloat16*>(pj.A[s_e[j]]);
-          cp_async16_zfill(dst, valid ? A + (size_t)i * pj.d_in + c0 + c * 8 : A, valid);
-        }
-        // W rows of the tile: 16 lanes per 256-byte row segment, 2 rows per instruction
-        const uint32_t wbase = sW + (uint32_t)slot * MT_WBUF;
-        const int ch = lane & 15;
-        if (ch * 8 < ncols) {
-#pragma unroll 4
-          for (int k2 = 0; k2 < 16; ++k2) {
-            const int row = warp * 32 + 2 * k2 + (lane >> 4);
-            if (row < nrows)
-              asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(wbase + (uint32_t)row * MT_WSTRIDE + ch * 16),
-                           "l"(Wt + (size_t)(row0 + row) * pj.d_in + c0 + ch * 8)
-                           : "memory");
-          }
-        }
-      };
-      for (int ct = 0; ct < MT_NY - 1; ++ct) {
-        if (ct < nct) issue_tile(ct);
-        cp_async_commit();
-      }
-      for (int ct = 0; ct < nct; ++ct) {
-        const int b = ct & 1;
-        const int slot = ct % MT_NY;
-        const int c0 = ct * MT_BN;
-        const int ncols = min(MT_BN, pj.d_in - c0);
-        if (ct + MT_NY - 1 < nct) issue_tile(ct + MT_NY - 1);
-        cp_async_commit();
-        cp_async_wait<MT_NY - 1>();
-        __syncthreads();
-        if (tid == 0) {
-          tc_fence_after();
-          const uint32_t ab = sA + (uint32_t)slot * MT_ABUF;
-          const uint32_t dcol = tmem + TC_D2_COL + (uint32_t)b * MT_BN;
-          for (int kk = 0; kk < K / 16; ++kk)
-            mma_bf16(dcol, desc_k_plain(sGH + kk * 256, 128, sbo_g), desc_k_plain(ab + kk * 4096, 2048, 128), id,
-                     kk > 0 ? 1u : 0u);
-          for (int kk = 0; kk < K / 16; ++kk)
-            mma_bf16(dcol, desc_k_plain(sGL + kk * 256, 128, sbo_g), desc_k_plain(ab + kk * 4096, 2048, 128), id, 1u);
-          mma_commit(bar_mma + 8 * b);
-        }
-        if (!mbar_wait(bar_mma + 8 * b, (ph_mma >> b) & 1)) abort = true;
-        ph_mma ^= 1u << b;
-        tc_fence_after();
-        abort = __syncthreads_or(abort);
-        if (abort) break;
-        {
-          const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16) + TC_D2_COL + (uint32_t)b * MT_BN;
-          unsigned char* wrow = sWp + (size_t)slot * MT_WBUF + (size_t)tid * MT_WSTRIDE;
-          for (int cc = 0; cc < ncols; cc += 16) {
-            float v[16];
-            tmem_ld16(lane_addr + (uint32_t)cc, v);
-            if (tid < nrows) {
-              uint4* pr = reinterpret_cast<uint4*>(wrow + cc * 2);
-              uint4 u0 = pr[0], u1 = pr[1];
-              __nv_bfloat162* h0 = reinterpret_cast<__nv_bfloat162*>(&u0);
-              __nv_bfloat162* h1 = reinterpret_cast<__nv_bfloat162*>(&u1);
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const float2 f0 = __bfloat1622float2(h0[i]);
-                const float2 f1 = __bfloat1622float2(h1[i]);
-                h0[i] = __floats2bfloat162_rn(f0.x + v[2 * i], f0.y + v[2 * i + 1]);
-                h1[i] = __floats2bfloat162_rn(f1.x + v[8 + 2 * i], f1.y + v[8 + 2 * i + 1]);
-              }
-              pr[0] = u0;
-              pr[1] = u1;
-            }
-          }
-          __syncwarp();
-          const int ch = lane & 15;
-          if (ch * 8 < ncols) {
-#pragma unroll 4
-            for (int k2 = 0; k2 < 16; ++k2) {
-              const int row = warp * 32 + 2 * k2 + (lane >> 4);
-              if (row < nrows) {
-                const uint4 val = *reinterpret_cast<const uint4*>(sWp + (size_t)slot * MT_WBUF +
-                                                                 (size_t)row * MT_WSTRIDE + ch * 16);
-                __stcs(reinterpret_cast<uint4*>(Wp + (size_t)(row0 + row) * pj.d_in + c0 + ch * 8), val);
-              }
-            }
-          }
-        }
-        tc_fence_before();
-        __syncthreads();
-      }
-      cp_async_wait_all();
-      __syncthreads();
-    }
-  }
-  if (abort && tid == 0) report(ws, APR_ERR_TIMEOUT, K_MERGE, (int)blockIdx.x);
-  cp_async_wait_all();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == 0) {
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TC_TMEM_COLS)
-                 : "memory");
-  }
-}
-
-bool merge_tensor_supported(int k, int r, int nproj) {
-  return k * round16(r) <= TC_MAXN1 && nproj <= MT_MAXPROJ;
-}
-
-cudaError_t launch_merge_tensor(const apr_merge_proj* projs, int nproj, int E, int r, const int32_t* idx,
-                                const float* gate, int k, void* ws, cudaStream_t s) {
-  const size_t smem = MtSmem::fixed_bytes() + sizeof(int) * ((size_t)nproj + 1);
-  static size_t configured = 0;
-  if (smem > configured) {
-    cudaError_t err = cudaFuncSetAttribute(merge_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (err != cudaSuccess) return err;
-    configured = smem;
+  if (sm2 > conf2) {
+    if ((err = cudaFuncSetAttribute(tc_expand_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2)) != cudaSuccess)
+      return err;
+    conf2 = sm2;
   }
   int dev = 0, nsm = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-  return launch_pdl(merge_tc_kernel, dim3(nsm), dim3(TC_THREADS), smem, s, projs, nproj, E, r, round16(r), idx,
-                    gate, k, ws);
+  // set tiles <= T + ceil(T / 128): the kernels loop over the real count
+  const long max_tiles = (long)a.T + (a.T + TB_M - 1) / TB_M;
+  const int g1 = (int)(max_tiles * t.npg < nsm ? max_tiles * t.npg : nsm);
+  const int g2 = (int)(max_tiles * t.cc_before[a.nproj] < nsm ? max_tiles * t.cc_before[a.nproj] : nsm);
+  if ((err = launch_pdl(tc_shrink_kernel, dim3(g1), dim3(SH_BLOCK), sm1, s, t)) != cudaSuccess) return err;
+  return launch_pdl(tc_expand_kernel, dim3(g2), dim3(EX_BLOCK), sm2, s, t);
 }
 
 }  // namespace apr

@@ -25,10 +25,11 @@ struct WsHeader {
   int err_info;     // detail (kernel id << 24 | value)
   int n_ptiles;     // shrink pair tiles written by the segment kernel
   int n_stiles;     // tensor-core set tiles written by the segment kernel
+  int n_qtiles;     // tensor-core pair tiles (<= 128 pairs of one adapter)
   int T, k, E;      // routing the plan was built for
   unsigned bar_count;   // grid barrier of the fused skinny kernel: arrivals
   unsigned bar_gen;     //   and generation
-  int pad[55];
+  int pad[54];
 };
 static_assert(sizeof(WsHeader) == 256, "header is one alignment unit");
 
@@ -47,8 +48,14 @@ __host__ __device__ inline int max_ptiles(int T, int k, int E) {
   return (int)((n + kPairTile - 1) / kPairTile + m + 1);
 }
 
+__host__ __device__ inline int max_qtiles(int T, int k, int E) {
+  long n = (long)T * k;
+  long m = n < E ? n : E;
+  return (int)((n + kSetTile - 1) / kSetTile + m + 1);
+}
+
 struct WsLayout {
-  size_t inv, tok_order, tok_tmp, ptiles, stiles, scratch;
+  size_t inv, tok_order, tok_tmp, ptiles, stiles, qtiles, scratch;
 };
 
 __host__ __device__ inline WsLayout ws_layout(int T, int k, int E) {
@@ -59,6 +66,7 @@ __host__ __device__ inline WsLayout ws_layout(int T, int k, int E) {
   L.tok_tmp = o;   o = align_up(o + sizeof(int) * (size_t)T);
   L.ptiles = o;    o = align_up(o + sizeof(PairTile) * (size_t)max_ptiles(T, k, E));
   L.stiles = o;    o = align_up(o + sizeof(SetTile) * (size_t)(T + 1));
+  L.qtiles = o;    o = align_up(o + sizeof(PairTile) * (size_t)max_qtiles(T, k, E));
   L.scratch = o;
   (void)E;
   return L;
@@ -91,15 +99,14 @@ inline bool dense_dims_ok(int T, int E, int max_rank, int d_in = 0) {
          dense_clusters(d_in) <= 8;
 }
 
-// Tensor-core path: gated V rows [projection][plan position][2 * k * R16] bf16
-// (hi | lo) and one 16-byte descriptor per set tile; k <= 2, k * R16 <= 64.
+// Tensor-core path: gated v rows [projection][pair position][2 * R16] bf16
+// (hi | lo); k <= 2, k * R16 <= 64.
 constexpr int kTensorMaxK2 = 64;
-inline size_t tc_vprep_bytes(int T, int K2) { return (size_t)APR_MAX_PROJ * T * 4 * K2; }
 inline size_t tc_scratch_bytes(int T, int k, int max_rank) {
   if (k < 1 || k > 2) return 0;
-  const int K2 = k * round16i(max_rank);
-  if (K2 > kTensorMaxK2) return 0;
-  return align_up(tc_vprep_bytes(T, K2)) + 16 * (size_t)(T + 1);
+  const int R16 = round16i(max_rank);
+  if (k * R16 > kTensorMaxK2) return 0;
+  return (size_t)APR_MAX_PROJ * T * k * 4 * R16;
 }
 
 // Shrink partial sums.  Gather paths: [projection][column chunk][sorted pair][rank]

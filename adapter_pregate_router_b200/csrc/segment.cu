@@ -130,6 +130,7 @@ __global__ void __launch_bounds__(SEG_THREADS) segment_kernel(const int32_t* __r
       report(ws, APR_ERR_DEVICE_INDEX, K_SEGMENT, 0);
       hdr->n_ptiles = 0;
       hdr->n_stiles = 0;
+      hdr->n_qtiles = 0;
     }
     return;
   }
@@ -168,6 +169,27 @@ __global__ void __launch_bounds__(SEG_THREADS) segment_kernel(const int32_t* __r
       hdr->k = k;
       hdr->E = E;
     }
+  }
+  __syncthreads();
+  // 3b. tensor-core pair tiles: ceil(count / kSetTile) per adapter, in adapter order
+  {
+    PairTile* qtiles = ws_at<PairTile>(ws, L.qtiles);
+    const int c = tid < E ? hist[tid] : 0;
+    const int nt = (c + kSetTile - 1) / kSetTile;
+    int ntiles;
+    const int toff = block_exclusive_scan(nt, warp_sums, &ntiles);
+    if (tid < E) {
+      const int s0 = base[tid];
+      for (int i = 0; i < nt; ++i) {
+        PairTile p;
+        p.e = tid;
+        p.start = s0 + i * kSetTile;
+        p.len = min(kSetTile, c - i * kSetTile);
+        p.pad = 0;
+        qtiles[toff + i] = p;
+      }
+    }
+    if (tid == 0) hdr->n_qtiles = ntiles;
   }
   __syncthreads();
   // 4. stable scatter of the pairs (one warp, in order)

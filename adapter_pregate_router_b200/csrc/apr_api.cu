@@ -190,7 +190,7 @@ apr_status apr_sgmm_shrink_expand(const void* x, int d_in, const apr_proj* projs
     // by the shapes and the mean pairs per adapter, known on the host without reading the routing
     const double mean_seg = (double)T * k / E;
     if (sgmm_dense_supported(a, dtype)) use = APR_SGMM_DENSE;
-    else if (mean_seg >= 256.0 && sgmm_tensor_supported(a, dtype)) use = APR_SGMM_TENSOR;
+    else if ((mean_seg >= 256.0 || (long)T * k >= 2048) && sgmm_tensor_supported(a, dtype)) use = APR_SGMM_TENSOR;
     else use = APR_SGMM_SKINNY;
   }
   cudaError_t e;

@@ -44,11 +44,11 @@ constexpr int TB_MAXN1 = 256;      // shrink accumulator columns
 constexpr int TB_MAXK2 = 64;       // k * R16 handled by the expand
 constexpr int TB_NT = 128;         // output columns per expand tile
 constexpr int TB_CW = 1024;        // output columns per expand item
-constexpr int SH_WORKERS = 128;    // shrink: warps 0-3 load and run the epilogue, warp 4 issues MMAs
+constexpr int SH_WORKERS = 256;    // shrink: warps 0-7 load and run the epilogue, warp 8 issues MMAs
 constexpr int SH_BLOCK = SH_WORKERS + 32;
-constexpr int EX_PROD = 128;       // expand: warps 0-3 load
-constexpr int EX_EPI = 256;        // expand: warps 4-11 run the epilogue
-constexpr int EX_BLOCK = EX_PROD + EX_EPI + 32;   // warp 12 issues MMAs
+constexpr int EX_PROD = 256;       // expand: warps 0-7 load
+constexpr int EX_EPI = 256;        // expand: warps 8-15 run the epilogue
+constexpr int EX_BLOCK = EX_PROD + EX_EPI + 32;   // warp 16 issues MMAs
 constexpr int SMEM_BUDGET = 200 * 1024;
 
 struct TcPlan {
@@ -132,7 +132,7 @@ __global__ void __launch_bounds__(SH_BLOCK, 1) tc_shrink_kernel(const __grid_con
     const int nq = min(P.pg, a.nproj - q0);
     const int N1 = nq * R16;
     const int e = tile.e;
-    if (worker) {
+    if (tid < TB_M) {
       int tok = -1;
       float g = 0.f;
       if (tid < tile.len) {
@@ -170,7 +170,7 @@ __global__ void __launch_bounds__(SH_BLOCK, 1) tc_shrink_kernel(const __grid_con
         if (g >= (uint32_t)S && !mbar_wait(bar_empty + 8 * s, ((g / S) - 1) & 1)) { abort = true; break; }
         const uint32_t st_base = sbase + s * L.stage_bytes;
 #pragma unroll
-        for (int m = 0; m < 8; ++m) {          // x rows: 8 lanes per 128-byte row segment
+        for (int m = 0; m < TB_M * 8 / SH_WORKERS; ++m) {   // x rows: 8 lanes per 128-byte row segment
           const int w = tid + m * SH_WORKERS;
           const int row = w >> 3, q = w & 7;
           const int tk = s_tok[row];
@@ -193,11 +193,11 @@ __global__ void __launch_bounds__(SH_BLOCK, 1) tc_shrink_kernel(const __grid_con
       if (!abort && !mbar_wait(bar_d1, nitem & 1)) abort = true;
       tc_fence_after();
       if (!abort) {
-        const int row = tid;
-        const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+        const int row = tid & (TB_M - 1), half = tid >> 7;      // the two warpgroups split the columns
+        const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
         const bool valid = row < tile.len;
         const float gg = s_g[row];
-        for (int c0 = 0; c0 < N1; c0 += 16) {
+        for (int c0 = half * 16; c0 < N1; c0 += 32) {
           float v[16];
           tmem_ld16(lane_addr + (uint32_t)c0, v);
           const int qi = c0 / R16, rr = c0 - qi * R16;
@@ -356,28 +356,27 @@ __global__ void __launch_bounds__(EX_BLOCK, 1) tc_expand_kernel(const __grid_con
         bad = r0 < 8 || r0 > R16 || (r0 & 7) || r1 < 8 || r1 > R16 || (r1 & 7);
       }
       if (bad && ptid == 0) report(a.ws, APR_ERR_DEVICE_INDEX, K_TC, e0);
-      const int tok = (!bad && ptid < tile.len) ? tok_order[tile.start + ptid] : -1;
-      s_tok[mb * TB_M + ptid] = tok;
+      const int prow = ptid & (TB_M - 1), phalf = ptid >> 7;
+      const int tok = (!bad && prow < tile.len) ? tok_order[tile.start + prow] : -1;
+      if (phalf == 0) s_tok[mb * TB_M + prow] = tok;
       asm volatile("bar.sync 1, %0;" ::"n"(EX_PROD) : "memory");     // every row's token is in shared memory
       mbar_arrive(bar_mfull + 8 * mb);
-      // V rows of the item: slot s of row `ptid` = v of its pair on adapter e_s
+      // V rows of the item: slot s of row `prow` = v of its pair on adapter e_s (hi or lo half)
       if (i >= 2 && !mbar_wait(bar_vempty + 8 * mb, ((i >> 1) - 1) & 1)) { abort = true; break; }
       {
-        const uint32_t vh = sbase + (uint32_t)(mb * L.vbuf), vl = vh + (uint32_t)(TB_M * K2 * 2);
-        const int row = ptid;
+        const uint32_t vbase = sbase + (uint32_t)(mb * L.vbuf) + (uint32_t)phalf * (TB_M * K2 * 2);
         for (int sl = 0; sl < K; ++sl) {
           const __nv_bfloat16* src = nullptr;
           if (tok >= 0) {
             const int es = sl == 0 ? e0 : e1;
             int j = 0;
             if (K == 2 && a.idx[(size_t)tok * K] != es) j = 1;
-            src = vprep + ((size_t)p * npairs + inv[(size_t)tok * K + j]) * (2 * R16);
+            src = vprep + ((size_t)p * npairs + inv[(size_t)tok * K + j]) * (2 * R16) + phalf * R16;
           }
           for (int q = 0; q < R16 / 8; ++q) {
             const int kq = sl * (R16 / 8) + q;
-            const uint32_t off = (uint32_t)(row >> 3) * SBO + (uint32_t)kq * 128 + (uint32_t)(row & 7) * 16;
-            cp_async16_zfill(vh + off, src ? (const void*)(src + q * 8) : (const void*)vprep, src != nullptr);
-            cp_async16_zfill(vl + off, src ? (const void*)(src + R16 + q * 8) : (const void*)vprep, src != nullptr);
+            const uint32_t off = (uint32_t)(prow >> 3) * SBO + (uint32_t)kq * 128 + (uint32_t)(prow & 7) * 16;
+            cp_async16_zfill(vbase + off, src ? (const void*)(src + q * 8) : (const void*)vprep, src != nullptr);
           }
         }
         cp_async_arrive(bar_vfull + 8 * mb);
@@ -391,7 +390,7 @@ __global__ void __launch_bounds__(EX_BLOCK, 1) tc_expand_kernel(const __grid_con
         const int c0 = n0 + t * TB_NT;
         const uint32_t ybuf = sbase + (uint32_t)L.y + slot * (TB_M * 256);
 #pragma unroll 4
-        for (int m = 0; m < 16; ++m) {         // y_base rows: 8 lanes per 128-byte half-row segment
+        for (int m = 0; m < TB_M * 16 / EX_PROD; ++m) {   // y_base rows: 8 lanes per 128-byte half-row segment
           const int w = ptid + m * EX_PROD;
           const int row = w >> 4, hs = (w >> 3) & 1, q = w & 7;
           const int tk = s_tok[mb * TB_M + row];

@@ -172,7 +172,7 @@ typedef struct apr_proj {
  *          E <= 16 and E * (max_rank rounded up to 16) <= 256; a forced kernel
  *          returns APR_ERR_UNSUPPORTED outside its range.  AUTO takes the
  *          dense kernel where it applies, the tensor-core kernel where
- *          T*k/E >= 256, and the CUDA-core kernel otherwise.
+ *          T*k/E >= 256 or T*k >= 2048, and the CUDA-core kernel otherwise.
  * T == 0 is a no-op.  Empty segments are legal.
  * ---------------------------------------------------------------------- */
 apr_status apr_sgmm_shrink_expand(const void* x, int d_in, const apr_proj* projs, int nproj,

@@ -26,10 +26,11 @@ struct WsHeader {
   int n_ptiles;     // shrink pair tiles written by the segment kernel
   int n_stiles;     // tensor-core set tiles written by the segment kernel
   int n_qtiles;     // tensor-core pair tiles (<= 128 pairs of one adapter)
+  int n_mtiles;     // tensor-core mixed tiles (<= 128 tokens, <= 4 adapters in all)
   int T, k, E;      // routing the plan was built for
   unsigned bar_count;   // grid barrier of the fused skinny kernel: arrivals
   unsigned bar_gen;     //   and generation
-  int pad[54];
+  int pad[53];
 };
 static_assert(sizeof(WsHeader) == 256, "header is one alignment unit");
 
@@ -38,6 +39,11 @@ struct PairTile {   // a run of <= kPairTile consecutive sorted pairs of one ada
 };
 struct SetTile {    // a run of <= kSetTile tokens (in set order) sharing one adapter set
   int start, len;
+};
+constexpr int kMixAdapters = 4;
+struct MixTile {    // a run of <= kSetTile tokens (in set order) whose adapters number <= kMixAdapters
+  int start, len, nu, pad;
+  int u[kMixAdapters];   // the adapters, ascending
 };
 
 __host__ __device__ inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
@@ -55,7 +61,7 @@ __host__ __device__ inline int max_qtiles(int T, int k, int E) {
 }
 
 struct WsLayout {
-  size_t inv, tok_order, tok_tmp, ptiles, stiles, qtiles, scratch;
+  size_t inv, tok_order, tok_tmp, ptiles, stiles, qtiles, mtiles, scratch;
 };
 
 __host__ __device__ inline WsLayout ws_layout(int T, int k, int E) {
@@ -67,6 +73,7 @@ __host__ __device__ inline WsLayout ws_layout(int T, int k, int E) {
   L.ptiles = o;    o = align_up(o + sizeof(PairTile) * (size_t)max_ptiles(T, k, E));
   L.stiles = o;    o = align_up(o + sizeof(SetTile) * (size_t)(T + 1));
   L.qtiles = o;    o = align_up(o + sizeof(PairTile) * (size_t)max_qtiles(T, k, E));
+  L.mtiles = o;    o = align_up(o + sizeof(MixTile) * (size_t)(T + 2 * (T / kSetTile) + 2));
   L.scratch = o;
   (void)E;
   return L;

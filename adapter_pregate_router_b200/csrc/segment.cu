@@ -20,6 +20,7 @@
 namespace apr {
 
 constexpr int SEG_THREADS = 1024;
+constexpr int MIX_CHUNK = 1024;      // set tiles staged per pass of the mixed-tile walk
 
 __device__ __forceinline__ unsigned lanemask_lt() {
   unsigned m;
@@ -288,6 +289,83 @@ __global__ void __launch_bounds__(SEG_THREADS) segment_kernel(const int32_t* __r
     stiles[j].len = end - stiles[j].start;
   }
   if (tid == 0) hdr->n_stiles = nst;
+  // 7. mixed tiles (k <= 2): consecutive set-ordered tokens, <= kSetTile of them, whose
+  //    adapters number <= kMixAdapters; greedy over the set tiles, one thread walking chunks
+  //    of the set tiles staged in shared memory.
+  __syncthreads();
+  if (k > 2) {
+    if (tid == 0) hdr->n_mtiles = 0;
+    return;
+  }
+  {
+    MixTile* mtiles = ws_at<MixTile>(ws, L.mtiles);
+    __shared__ int4 s_st[MIX_CHUNK];       // start, len, a0, a1 of a chunk of set tiles
+    __shared__ MixTile s_cur;
+    __shared__ int s_nm;
+    if (tid == 0) {
+      s_cur.start = 0;
+      s_cur.len = 0;
+      s_cur.nu = 0;
+      s_nm = 0;
+    }
+    for (int c0 = 0; c0 < nst; c0 += MIX_CHUNK) {
+      __syncthreads();
+      for (int j = tid; j < MIX_CHUNK && c0 + j < nst; j += SEG_THREADS) {
+        const SetTile st = stiles[c0 + j];
+        const int t0 = tok_order[st.start];
+        const int a0 = sorted_key(idx, t0, k, 0);
+        const int a1 = k == 2 ? sorted_key(idx, t0, k, 1) : -1;
+        s_st[j] = make_int4(st.start, st.len, a0, a1);
+      }
+      __syncthreads();
+      if (tid == 0) {
+        MixTile cur = s_cur;
+        int nm = s_nm;
+        const int n = min(MIX_CHUNK, nst - c0);
+        for (int j = 0; j < n; ++j) {
+          const int4 t = s_st[j];
+          int remaining = t.y, pos = t.x;
+          while (remaining > 0) {
+            // the union with this set
+            int u[kMixAdapters + 2], nu = cur.nu;
+            for (int q = 0; q < cur.nu; ++q) u[q] = cur.u[q];
+            const int add[2] = {t.z, t.w};
+            for (int q = 0; q < k; ++q) {
+              bool found = false;
+              for (int w = 0; w < nu; ++w) found |= (u[w] == add[q]);
+              if (!found) {
+                int w = nu++;                  // insert keeping ascending order
+                while (w > 0 && u[w - 1] > add[q]) { u[w] = u[w - 1]; --w; }
+                u[w] = add[q];
+              }
+            }
+            if (cur.len > 0 && (nu > kMixAdapters || cur.len == kSetTile)) {
+              mtiles[nm++] = cur;              // close the tile, start a new one here
+              cur.start = pos;
+              cur.len = 0;
+              cur.nu = 0;
+              continue;
+            }
+            const int take = min(remaining, kSetTile - cur.len);
+            if (cur.len == 0) cur.start = pos;
+            cur.len += take;
+            cur.nu = nu;
+            for (int q = 0; q < nu; ++q) cur.u[q] = u[q];
+            remaining -= take;
+            pos += take;
+          }
+        }
+        s_cur = cur;
+        s_nm = nm;
+      }
+    }
+    __syncthreads();
+    if (tid == 0) {
+      int nm = s_nm;
+      if (s_cur.len > 0) mtiles[nm++] = s_cur;
+      hdr->n_mtiles = nm;
+    }
+  }
 }
 
 cudaError_t launch_segment(const int32_t* idx, int T, int k, int E, int32_t* seg_off,

@@ -59,6 +59,7 @@ struct TcPlan {
   int npg;                           // shrink items per pair tile
   int stages;                        // shrink pipeline depth
   int ny;                            // expand ring depth
+  int mixed;                         // expand over mixed tiles (<= 4 adapters, K2 = 4 * R16) instead of set tiles
   size_t vprep_off;                  // scratch: V rows [proj][pair position][2 * R16] bf16
   int cc_before[APR_MAX_PROJ + 1];   // expand: prefix of 1024-column items per projection
 };
@@ -317,11 +318,16 @@ __global__ void __launch_bounds__(EX_BLOCK, 1) tc_expand_kernel(const __grid_con
   const int* tok_order = ws_at<int>(a.ws, W.tok_order);
   const int* inv = ws_at<int>(a.ws, W.inv);
   const SetTile* stiles = ws_at<SetTile>(a.ws, W.stiles);
+  const MixTile* mtiles = ws_at<MixTile>(a.ws, W.mtiles);
   const __nv_bfloat16* vprep = ws_at<__nv_bfloat16>(a.ws, P.vprep_off);
   const long npairs = (long)a.T * K;
   const int ipt = P.cc_before[a.nproj];
-  const long nitems = (long)hdr->n_stiles * ipt;
-  auto item_at = [&](int i) -> long { return (long)blockIdx.x + (long)i * gridDim.x; };
+  const int nsl = P.mixed ? kMixAdapters : K;                  // adapter slots of the contraction
+  const long nitems = (long)(P.mixed ? hdr->n_mtiles : hdr->n_stiles) * ipt;
+  // each CTA takes a contiguous block of items, so consecutive items mostly share a tile (its
+  // tokens and adapters stay loaded) and a projection (its V stays loaded)
+  const long ibeg = (long)blockIdx.x * nitems / gridDim.x, iend = (long)(blockIdx.x + 1) * nitems / gridDim.x;
+  auto item_at = [&](int i) -> long { return ibeg + i < iend ? ibeg + i : nitems; };
   // item -> (set tile, projection, first column, 128-column tiles)
   auto item_shape = [&](long it, int& st, int& p, int& n0, int& ntl, int& d_out) {
     st = (int)(it / ipt);
@@ -338,51 +344,75 @@ __global__ void __launch_bounds__(EX_BLOCK, 1) tc_expand_kernel(const __grid_con
     // ---------------------------------------------------- producer
     const int ptid = tid;
     uint32_t gp = 0;
+    int mcnt = -1, vcnt = -1, st_prev = -1, p_prev = -1;
+    int tstart = 0, tlen = 0, tok = -1, su[kMixAdapters] = {-1, -1, -1, -1}, rs[kMixAdapters] = {0, 0, 0, 0};
+    int ej[2] = {-2, -2};
+    bool bad = false;
+    const int prow = ptid & (TB_M - 1), phalf = ptid >> 7;
+    const __nv_bfloat16* Bs[kMixAdapters] = {nullptr, nullptr, nullptr, nullptr};
     for (int i = 0; item_at(i) < nitems && !abort; ++i) {
       int st, p, n0, ntl, d_out;
       item_shape(item_at(i), st, p, n0, ntl, d_out);
-      const int mb = i & 1;
-      if (i >= 2 && !mbar_wait(bar_mempty + 8 * mb, ((i >> 1) - 1) & 1)) { abort = true; break; }
-      const SetTile tile = stiles[st];
-      // the set's adapters, ascending, from the tile's first token
-      const int t0 = tok_order[tile.start];
-      int e0 = a.idx[(size_t)t0 * K], e1 = K == 2 ? a.idx[(size_t)t0 * K + 1] : 0;
-      if (K == 2 && e1 < e0) { const int te = e0; e0 = e1; e1 = te; }
-      bool bad = e0 < 0 || e0 >= a.E || (K == 2 && (e1 < 0 || e1 >= a.E));
-      int r0 = 0, r1 = 0;
-      if (!bad) {
-        r0 = a.ranks[e0];
-        r1 = K == 2 ? a.ranks[e1] : 8;
-        bad = r0 < 8 || r0 > R16 || (r0 & 7) || r1 < 8 || r1 > R16 || (r1 & 7);
+      const bool newM = st != st_prev, newV = newM || p != p_prev;
+      st_prev = st;
+      p_prev = p;
+      if (newM) {
+        // the tile's tokens and its adapter slots (ascending; -1: an empty slot)
+        const int mb = (++mcnt) & 1;
+        if (mcnt >= 2 && !mbar_wait(bar_mempty + 8 * mb, ((mcnt >> 1) - 1) & 1)) { abort = true; break; }
+        for (int q = 0; q < kMixAdapters; ++q) { su[q] = -1; rs[q] = 0; }
+        if (P.mixed) {
+          const MixTile mt = mtiles[st];
+          tstart = mt.start;
+          tlen = mt.len;
+          for (int q = 0; q < kMixAdapters; ++q) su[q] = q < mt.nu ? mt.u[q] : -1;
+        } else {
+          const SetTile tile = stiles[st];
+          tstart = tile.start;
+          tlen = tile.len;
+          const int t0 = tok_order[tile.start];
+          int e0 = a.idx[(size_t)t0 * K], e1 = K == 2 ? a.idx[(size_t)t0 * K + 1] : -1;
+          if (K == 2 && e1 < e0) { const int te = e0; e0 = e1; e1 = te; }
+          su[0] = e0;
+          su[1] = e1;
+        }
+        bad = false;
+        for (int q = 0; q < nsl; ++q) {
+          if (su[q] < 0) continue;
+          if (su[q] >= a.E) { bad = true; continue; }
+          rs[q] = a.ranks[su[q]];
+          bad |= rs[q] < 8 || rs[q] > R16 || (rs[q] & 7);
+        }
+        if (bad && ptid == 0) report(a.ws, APR_ERR_DEVICE_INDEX, K_TC, su[0]);
+        tok = (!bad && prow < tlen) ? tok_order[tstart + prow] : -1;
+        ej[0] = ej[1] = -2;
+        if (tok >= 0)
+          for (int j = 0; j < K && j < 2; ++j) ej[j] = a.idx[(size_t)tok * K + j];
+        if (phalf == 0) s_tok[mb * TB_M + prow] = tok;
+        asm volatile("bar.sync 1, %0;" ::"n"(EX_PROD) : "memory");     // every row's token is in shared memory
+        mbar_arrive(bar_mfull + 8 * mb);
       }
-      if (bad && ptid == 0) report(a.ws, APR_ERR_DEVICE_INDEX, K_TC, e0);
-      const int prow = ptid & (TB_M - 1), phalf = ptid >> 7;
-      const int tok = (!bad && prow < tile.len) ? tok_order[tile.start + prow] : -1;
-      if (phalf == 0) s_tok[mb * TB_M + prow] = tok;
-      asm volatile("bar.sync 1, %0;" ::"n"(EX_PROD) : "memory");     // every row's token is in shared memory
-      mbar_arrive(bar_mfull + 8 * mb);
-      // V rows of the item: slot s of row `prow` = v of its pair on adapter e_s (hi or lo half)
-      if (i >= 2 && !mbar_wait(bar_vempty + 8 * mb, ((i >> 1) - 1) & 1)) { abort = true; break; }
-      {
-        const uint32_t vbase = sbase + (uint32_t)(mb * L.vbuf) + (uint32_t)phalf * (TB_M * K2 * 2);
-        for (int sl = 0; sl < K; ++sl) {
+      if (newV) {
+        // V rows: slot q of row `prow` = v of its pair on adapter su[q] (hi or lo half), else zero
+        const int vb = (++vcnt) & 1;
+        if (vcnt >= 2 && !mbar_wait(bar_vempty + 8 * vb, ((vcnt >> 1) - 1) & 1)) { abort = true; break; }
+        const uint32_t vbase = sbase + (uint32_t)(vb * L.vbuf) + (uint32_t)phalf * (TB_M * K2 * 2);
+        for (int q = 0; q < nsl; ++q) {
           const __nv_bfloat16* src = nullptr;
-          if (tok >= 0) {
-            const int es = sl == 0 ? e0 : e1;
-            int j = 0;
-            if (K == 2 && a.idx[(size_t)tok * K] != es) j = 1;
-            src = vprep + ((size_t)p * npairs + inv[(size_t)tok * K + j]) * (2 * R16) + phalf * R16;
+          if (tok >= 0 && su[q] >= 0) {
+            const int j = ej[0] == su[q] ? 0 : (ej[1] == su[q] ? 1 : -1);
+            if (j >= 0) src = vprep + ((size_t)p * npairs + inv[(size_t)tok * K + j]) * (2 * R16) + phalf * R16;
           }
-          for (int q = 0; q < R16 / 8; ++q) {
-            const int kq = sl * (R16 / 8) + q;
+          for (int c = 0; c < R16 / 8; ++c) {
+            const int kq = q * (R16 / 8) + c;
             const uint32_t off = (uint32_t)(prow >> 3) * SBO + (uint32_t)kq * 128 + (uint32_t)(prow & 7) * 16;
-            cp_async16_zfill(vbase + off, src ? (const void*)(src + q * 8) : (const void*)vprep, src != nullptr);
+            cp_async16_zfill(vbase + off, src ? (const void*)(src + c * 8) : (const void*)vprep, src != nullptr);
           }
         }
-        cp_async_arrive(bar_vfull + 8 * mb);
+        cp_async_arrive(bar_vfull + 8 * vb);
+        for (int q = 0; q < kMixAdapters; ++q)
+          Bs[q] = (!bad && q < nsl && su[q] >= 0) ? reinterpret_cast<const __nv_bfloat16*>(a.proj[p].B[su[q]]) : nullptr;
       }
-      const __nv_bfloat16* B0 = bad ? nullptr : reinterpret_cast<const __nv_bfloat16*>(a.proj[p].B[e0]);
-      const __nv_bfloat16* B1 = (bad || K < 2) ? nullptr : reinterpret_cast<const __nv_bfloat16*>(a.proj[p].B[e1]);
       const __nv_bfloat16* yb = reinterpret_cast<const __nv_bfloat16*>(a.proj[p].y_base);
       for (int t = 0; t < ntl; ++t, ++gp) {
         const uint32_t slot = gp % NY;
@@ -393,7 +423,7 @@ __global__ void __launch_bounds__(EX_BLOCK, 1) tc_expand_kernel(const __grid_con
         for (int m = 0; m < TB_M * 16 / EX_PROD; ++m) {   // y_base rows: 8 lanes per 128-byte half-row segment
           const int w = ptid + m * EX_PROD;
           const int row = w >> 4, hs = (w >> 3) & 1, q = w & 7;
-          const int tk = s_tok[mb * TB_M + row];
+          const int tk = s_tok[(mcnt & 1) * TB_M + row];
           const int col = c0 + hs * 64 + q * 8;
           if (tk >= 0 && col < d_out)
             asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(ybuf + (uint32_t)row * 256 +
@@ -407,8 +437,8 @@ __global__ void __launch_bounds__(EX_BLOCK, 1) tc_expand_kernel(const __grid_con
         for (int w = ptid; w < TB_NT * cpr; w += EX_PROD) {
           const int n = w / cpr, kq = w - n * cpr;
           const int sa = kq / cps, cq = kq - sa * cps;
-          const __nv_bfloat16* B = sa == 0 ? B0 : B1;
-          const int re = sa == 0 ? r0 : r1;
+          const __nv_bfloat16* B = Bs[sa];
+          const int re = rs[sa];
           const bool ok = B != nullptr && c0 + n < d_out && cq * 8 < re;
           cp_async16_zfill(bbuf + (uint32_t)(n >> 3) * SBO + (uint32_t)kq * 128 + (uint32_t)(n & 7) * 16,
                            ok ? (const void*)(B + (size_t)(c0 + n) * re + cq * 8) : (const void*)vprep, ok);
@@ -422,12 +452,16 @@ __global__ void __launch_bounds__(EX_BLOCK, 1) tc_expand_kernel(const __grid_con
     const int row = eid & (TB_M - 1), half = eid >> 7;
     const int wrow0 = (warp & 3) * 32;
     uint32_t g = 0;
+    int mcnt = -1, st_prev = -1, tok = -1;
     for (int i = 0; item_at(i) < nitems && !abort; ++i) {
       int st, p, n0, ntl, d_out;
       item_shape(item_at(i), st, p, n0, ntl, d_out);
-      const int mb = i & 1;
-      if (!mbar_wait(bar_mfull + 8 * mb, (i >> 1) & 1)) { abort = true; break; }
-      const int tok = s_tok[mb * TB_M + row];
+      if (st != st_prev) {
+        const int mb = (++mcnt) & 1;
+        if (!mbar_wait(bar_mfull + 8 * mb, (mcnt >> 1) & 1)) { abort = true; break; }
+        tok = s_tok[mb * TB_M + row];
+      }
+      st_prev = st;
       __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(a.proj[p].y);
       for (int t = 0; t < ntl; ++t, ++g) {
         const uint32_t slot = g % NY, b = g & 1;
@@ -482,18 +516,29 @@ __global__ void __launch_bounds__(EX_BLOCK, 1) tc_expand_kernel(const __grid_con
         mbar_arrive(bar_tempty + 8 * slot);
       }
       if (abort) break;
-      mbar_arrive(bar_mempty + 8 * mb);
+      bool last = item_at(i + 1) >= nitems;
+      if (!last) {
+        int st2, p2, n02, ntl2, d2;
+        item_shape(item_at(i + 1), st2, p2, n02, ntl2, d2);
+        last = st2 != st;
+      }
+      if (last) mbar_arrive(bar_mempty + 8 * (mcnt & 1));    // this tile's tokens are no longer read
     }
   } else if (lane == 0) {
     // ---------------------------------------------------- MMA issue
     const uint32_t id = idesc_bf16(TB_M, TB_NT);
     uint32_t g = 0;
+    int vcnt = -1, st_prev = -1, p_prev = -1;
     for (int i = 0; item_at(i) < nitems && !abort; ++i) {
       int st, p, n0, ntl, d_out;
       item_shape(item_at(i), st, p, n0, ntl, d_out);
-      const int mb = i & 1;
-      if (!mbar_wait(bar_vfull + 8 * mb, (i >> 1) & 1)) { abort = true; break; }
-      const uint32_t vh = sbase + (uint32_t)(mb * L.vbuf), vl = vh + (uint32_t)(TB_M * K2 * 2);
+      if (st != st_prev || p != p_prev) {
+        ++vcnt;
+        if (!mbar_wait(bar_vfull + 8 * (vcnt & 1), (vcnt >> 1) & 1)) { abort = true; break; }
+      }
+      st_prev = st;
+      p_prev = p;
+      const uint32_t vh = sbase + (uint32_t)((vcnt & 1) * L.vbuf), vl = vh + (uint32_t)(TB_M * K2 * 2);
       for (int t = 0; t < ntl; ++t, ++g) {
         const uint32_t slot = g % NY, b = g & 1;
         if (!mbar_wait(bar_tfull + 8 * slot, (g / NY) & 1)) { abort = true; break; }
@@ -507,7 +552,14 @@ __global__ void __launch_bounds__(EX_BLOCK, 1) tc_expand_kernel(const __grid_con
           mma_bf16(dcol, desc_k_plain(vl + kk * 256, 128, SBO), desc_k_plain(bb + kk * 256, 128, SBO), id, 1u);
         mma_commit(bar_d2full + 8 * b);
       }
-      if (!abort) mma_commit(bar_vempty + 8 * mb);
+      if (abort) break;
+      bool last = item_at(i + 1) >= nitems;
+      if (!last) {
+        int st2, p2, n02, ntl2, d2;
+        item_shape(item_at(i + 1), st2, p2, n02, ntl2, d2);
+        last = st2 != st || p2 != p;
+      }
+      if (last) mma_commit(bar_vempty + 8 * (vcnt & 1));     // this V is no longer read
     }
   }
   abort = __syncthreads_or(abort);
@@ -536,7 +588,8 @@ cudaError_t launch_sgmm_tensor(const SgmmArgs& a, size_t scratch_off, cudaStream
   memset(&t, 0, sizeof(t));
   t.a = a;
   t.R16 = round16i(a.max_rank);
-  t.K2 = a.k * t.R16;
+  t.mixed = (a.k <= 2 && kMixAdapters * t.R16 <= TB_MAXK2) ? 1 : 0;
+  t.K2 = (t.mixed ? kMixAdapters : a.k) * t.R16;
   t.pg = TB_MAXN1 / t.R16;
   if (t.pg > a.nproj) t.pg = a.nproj;
   t.npg = (a.nproj + t.pg - 1) / t.pg;

@@ -330,6 +330,8 @@ def _zipf_idx(rng, T, E, k, s=1.1):
     (517, 4096, (4096,), (16,) * 16, 2, True),             # prefill-shaped projection
     (129, 192, (64, 64, 64, 64), (32,) * 3, 2, False),     # four projections, k * rank = 64
     (1, 128, (16,), (16, 16), 2, False),                   # one token
+    (600, 256, (128, 64), (16, 8, 16, 16, 8, 16), 1, True),  # top-1 with rank slots of 16: mixed tiles of one-adapter sets
+    (2500, 512, (256,), (16,) * 12, 2, True),               # many sets, mixed tiles split long sets
 ])
 def test_sgmm_tensor_parity(apr, T, d_in, d_outs, ranks, k, zipf):
     rng = np.random.default_rng(T + d_in + k + 1)

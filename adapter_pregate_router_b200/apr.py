@@ -78,6 +78,9 @@ _segment_tokens = _sig("apr_segment_tokens", _i, [_vp, _i, _i, _i, _vp, _vp, _vp
 _sgmm = _sig("apr_sgmm_shrink_expand", _i,
              [_vp, _i, ctypes.POINTER(Proj), _i, _i, _i, _i, _i, _vp, _i, _vp, _vp, _vp, _vp, _vp, _sz, _i, _vp])
 _merge = _sig("apr_merge_adapters", _i, [_vp, _i, _i, _i, _vp, _vp, _i, _vp, _sz, _vp])
+_merge_plan_size = _sig("apr_merge_plan_size", _sz, [_i])
+_merge_plan_init = _sig("apr_merge_plan_init", _i, [_vp, _i, _vp, _sz])
+_merge_planned = _sig("apr_merge_adapters_planned", _i, [_vp, _vp, _i, _i, _i, _vp, _vp, _i, _vp, _sz, _vp])
 _gemv = _sig("apr_gemv", _i, [_vp, _vp, _vp, _i, _i, _vp])
 _stream_status = _sig("apr_stream_status", _i, [_vp, _vp])
 _last_error = _sig("apr_last_error", ctypes.c_char_p, [])
@@ -86,7 +89,8 @@ _kernel_launches = _sig("apr_kernel_launches", ctypes.c_uint64, [])
 
 EXPORTED = ("apr_workspace_size", "apr_workspace_init", "apr_pregate_route", "apr_pregate_route_noalloc",
             "apr_segment_tokens",
-            "apr_sgmm_shrink_expand", "apr_merge_adapters", "apr_gemv", "apr_stream_status",
+            "apr_sgmm_shrink_expand", "apr_merge_adapters", "apr_merge_plan_size", "apr_merge_plan_init",
+            "apr_merge_adapters_planned", "apr_gemv", "apr_stream_status",
             "apr_last_error", "apr_status_string", "apr_kernel_launches")
 
 
@@ -191,15 +195,37 @@ def sgmm_shrink_expand(x, projs, k, E, ranks, max_rank, idx, gate, seg_off, perm
                  _stream(stream)))
 
 
-def merge_table(entries, device="cuda") -> torch.Tensor:
-    """Device array of apr_merge_proj from (W, Wp, A_table, B_table) tuples."""
+def _merge_host_table(entries):
     n = len(entries)
     arr = (MergeProj * n)()
     for i, (W, Wp, At, Bt) in enumerate(entries):
         arr[i] = MergeProj(_ptr(W), _ptr(Wp), int(W.shape[1]), int(W.shape[0]), _ptr(At), _ptr(Bt))
-    raw = bytes(memoryview(arr).cast("B"))
+    return arr
+
+
+def merge_table(entries, device="cuda") -> torch.Tensor:
+    """Device array of apr_merge_proj from (W, Wp, A_table, B_table) tuples."""
+    raw = bytes(memoryview(_merge_host_table(entries)).cast("B"))
     host = torch.frombuffer(bytearray(raw), dtype=torch.uint8)
     return host.to(device)
+
+
+def merge_plan(entries, device="cuda") -> torch.Tensor:
+    """TMA descriptors of the weights in ``entries`` (same order as ``merge_table``)."""
+    n = len(entries)
+    size = int(_merge_plan_size(n))
+    if size == 0:
+        raise AprError(APR_ERR_INVALID_ARG, "merge_plan_size: nproj out of range")
+    plan = torch.empty(size + 128, dtype=torch.uint8, device=device)
+    off = (-plan.data_ptr()) % 128
+    plan = plan[off:off + size]
+    _check(_merge_plan_init(_merge_host_table(entries), n, plan.data_ptr(), size))
+    return plan
+
+
+def merge_adapters_planned(table, plan, nproj, E, r, idx, gate, k, ws, stream=None):
+    _check(_merge_planned(_ptr(table), _ptr(plan), nproj, E, r, _ptr(idx), _ptr(gate), k, _ptr(ws), ws.numel(),
+                          _stream(stream)))
 
 
 def merge_adapters(table, nproj, E, r, idx, gate, k, ws, stream=None):

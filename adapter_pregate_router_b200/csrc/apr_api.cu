@@ -209,6 +209,47 @@ apr_status apr_sgmm_shrink_expand(const void* x, int d_in, const apr_proj* projs
   return APR_OK;
 }
 
+size_t apr_merge_plan_size(int nproj) {
+  if (nproj < 1 || nproj > 4096) return 0;
+  return merge_plan_bytes(nproj);
+}
+
+apr_status apr_merge_plan_init(const apr_merge_proj* projs, int nproj, void* plan, size_t plan_bytes) {
+  if (nproj < 1 || nproj > 4096) return fail(APR_ERR_INVALID_ARG, "merge_plan_init: nproj=%d outside [1, 4096]", nproj);
+  if (!projs || !plan) return fail(APR_ERR_INVALID_ARG, "merge_plan_init: NULL pointer");
+  if (reinterpret_cast<uintptr_t>(plan) & 127) return fail(APR_ERR_INVALID_ARG, "merge_plan_init: plan not 128-byte aligned");
+  if (plan_bytes < merge_plan_bytes(nproj))
+    return fail(APR_ERR_WORKSPACE, "merge_plan_init: %zu bytes < %zu needed", plan_bytes, merge_plan_bytes(nproj));
+  for (int p = 0; p < nproj; ++p) {
+    const apr_merge_proj& m = projs[p];
+    if (!m.W || !m.Wp) return fail(APR_ERR_INVALID_ARG, "merge_plan_init: weight %d has a NULL pointer", p);
+    if (!aligned16(m.W) || !aligned16(m.Wp)) return fail(APR_ERR_INVALID_ARG, "merge_plan_init: weight %d not 16-byte aligned", p);
+    if (m.d_in < 8 || (m.d_in & 7) || m.d_out < 1)
+      return fail(APR_ERR_INVALID_ARG, "merge_plan_init: weight %d shape %d x %d (d_in must be a multiple of 8)", p, m.d_out, m.d_in);
+  }
+  cudaError_t e = merge_plan_build(projs, nproj, plan);
+  if (e != cudaSuccess) return cuda_fail(e, "merge_plan_init");
+  return APR_OK;
+}
+
+apr_status apr_merge_adapters_planned(const apr_merge_proj* projs, const void* plan, int nproj, int E, int r,
+                                      const int32_t* idx, const float* gate, int k, void* ws, size_t ws_bytes,
+                                      void* stream) {
+  if (nproj < 1) return fail(APR_ERR_INVALID_ARG, "merge: nproj=%d < 1", nproj);
+  if (E < 1 || E > APR_MAX_E) return fail(APR_ERR_INVALID_ARG, "merge: E=%d outside [1, %d]", E, APR_MAX_E);
+  if (k < 1 || k > E || k > APR_MAX_K) return fail(APR_ERR_INVALID_ARG, "merge: k=%d outside [1, min(E, %d)]", k, APR_MAX_K);
+  if (r < 8 || (r & 7) || r > APR_MAX_RANK) return fail(APR_ERR_INVALID_ARG, "merge: r=%d must be a multiple of 8 in [8, %d]", r, APR_MAX_RANK);
+  if (!merge_tensor_supported(k, r, nproj))
+    return fail(APR_ERR_UNSUPPORTED, "merge (planned): needs k * round16(r) <= 64 and nproj <= 4096");
+  if (!projs || !plan || !idx || !gate) return fail(APR_ERR_INVALID_ARG, "merge: NULL pointer");
+  if (reinterpret_cast<uintptr_t>(plan) & 127) return fail(APR_ERR_INVALID_ARG, "merge: plan not 128-byte aligned");
+  apr_status st = check_ws(ws, ws_bytes, sizeof(WsHeader), "merge");
+  if (st) return st;
+  cudaError_t e = launch_merge_tma(projs, plan, nproj, E, r, idx, gate, k, ws, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "merge launch");
+  return APR_OK;
+}
+
 apr_status apr_merge_adapters(const apr_merge_proj* projs, int nproj, int E, int r,
                               const int32_t* idx, const float* gate, int k, void* ws,
                               size_t ws_bytes, void* stream) {

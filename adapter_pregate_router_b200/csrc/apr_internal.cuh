@@ -285,6 +285,10 @@ cudaError_t launch_merge(const apr_merge_proj* projs, int nproj, int E, int r, c
 bool merge_tensor_supported(int k, int r, int nproj);
 cudaError_t launch_merge_tensor(const apr_merge_proj* projs, int nproj, int E, int r, const int32_t* idx,
                                 const float* gate, int k, void* ws, cudaStream_t s);
+size_t merge_plan_bytes(int nproj);
+cudaError_t merge_plan_build(const apr_merge_proj* projs, int nproj, void* plan);
+cudaError_t launch_merge_tma(const apr_merge_proj* projs, const void* plan, int nproj, int E, int r,
+                             const int32_t* idx, const float* gate, int k, void* ws, cudaStream_t s);
 cudaError_t launch_gemv(const void* W, const void* x, void* y, int d_in, int d_out, cudaStream_t s);
 
 }  // namespace apr

@@ -8,8 +8,9 @@ and runs, through the C ABI only:
 * ``apr_segment_tokens``  once per step;
 * ``apr_sgmm_shrink_expand`` once per (layer, shared-input group);
 
-or, for the batch-1 merge workload, the route, one ``apr_merge_adapters``
-over every weight and one ``apr_gemv`` per weight (§2.B steps 1-5).
+or, for the batch-1 merge workload, the route, one ``apr_merge_adapters_planned``
+over every weight (its TMA plan built once with the weights) and one ``apr_gemv``
+per weight (§2.B steps 1-5).
 
 Tensors are built once from the seeded pools (``workloads.device_tensor``) and
 stay resident; ``run()`` enqueues the step on the current stream.
@@ -134,6 +135,8 @@ class Step:
                     self.keep += [At, Bt]
         self.merge_tab = apr.merge_table(entries, dev)
         self.nmerge = len(entries)
+        # TMA descriptors of the weights: built once, reused by every token's merge
+        self.merge_plan = apr.merge_plan(entries, dev) if cfg.k * ((self.max_rank + 15) // 16 * 16) <= 64 else None
         W.clear_device_pools()
 
     # ------------------------------------------------------------ running
@@ -145,8 +148,12 @@ class Step:
     def layers_only(self, stream=None):
         cfg = self.cfg
         if cfg.merge:
-            apr.merge_adapters(self.merge_tab, self.nmerge, cfg.E, self.max_rank, self.idx, self.gate,
-                               cfg.k, self.ws, stream)
+            if self.merge_plan is not None:
+                apr.merge_adapters_planned(self.merge_tab, self.merge_plan, self.nmerge, cfg.E, self.max_rank,
+                                           self.idx, self.gate, cfg.k, self.ws, stream)
+            else:
+                apr.merge_adapters(self.merge_tab, self.nmerge, cfg.E, self.max_rank, self.idx, self.gate,
+                                   cfg.k, self.ws, stream)
             for (Wt, Wp, x, y) in self.weights.values():
                 apr.gemv(Wp, x, y, stream)
             return

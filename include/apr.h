@@ -204,6 +204,30 @@ apr_status apr_merge_adapters(const apr_merge_proj* projs, int nproj, int E, int
                               size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Merge plan: TMA descriptors of every weight pair (W, Wp).  The weights'
+ * addresses and shapes do not change from one token to the next, so a plan is
+ * built once for a set of weights and then used by every
+ * apr_merge_adapters_planned, which streams W in and Wp out with TMA copies
+ * (the same result as apr_merge_adapters, bit for bit).
+ * apr_merge_plan_size  device bytes of a plan for nproj weights (0 if nproj is
+ *                      outside [1, 4096])
+ * apr_merge_plan_init  projs: HOST array [nproj], the same entries as the device
+ *                      table later given to the merge; plan: device memory of
+ *                      apr_merge_plan_size(nproj) bytes, 128-byte aligned, owned by
+ *                      the caller.  W and Wp must be 16-byte aligned and d_in a
+ *                      multiple of 8.  A set-up call: it encodes on the host and
+ *                      copies synchronously (no stream).
+ * apr_merge_adapters_planned  as apr_merge_adapters, with the plan of the same
+ *                      weights in the same order; needs k * round16(r) <= 64
+ *                      (APR_ERR_UNSUPPORTED otherwise).
+ * ---------------------------------------------------------------------- */
+size_t apr_merge_plan_size(int nproj);
+apr_status apr_merge_plan_init(const apr_merge_proj* projs, int nproj, void* plan, size_t plan_bytes);
+apr_status apr_merge_adapters_planned(const apr_merge_proj* projs, const void* plan, int nproj, int E, int r,
+                                      const int32_t* idx, const float* gate, int k, void* ws, size_t ws_bytes,
+                                      void* stream);
+
+/* ------------------------------------------------------------------------
  * Base inference on the merged weight (section 2.B step 4): y = W x.
  * W device [d_out, d_in] bf16, x device [d_in] bf16, y device [d_out] bf16.
  * fp32 accumulation, one rounding per output.

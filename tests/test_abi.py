@@ -119,3 +119,22 @@ def test_merge_and_gemv_host_validation(apr):
     assert apr._gemv(0x1000, 0x1000, 0x1000, 60, 8, None) == apr.APR_ERR_INVALID_ARG
     assert apr._gemv(0x1000, 0x1000, 0x1000, 64, 0, None) == apr.APR_OK
     assert apr._gemv(None, 0x1000, 0x1000, 64, 8, None) == apr.APR_ERR_INVALID_ARG
+
+
+def test_merge_plan_host_validation(apr):
+    """The plan set-up checks its arguments on the host before touching the GPU."""
+    assert apr._merge_plan_size(0) == 0
+    assert apr._merge_plan_size(224) == 224 * 2 * 128
+    one = (apr.MergeProj * 1)(apr.MergeProj(0x1000, 0x2000, 64, 32, 0x3000, 0x4000))
+    assert apr._merge_plan_init(one, 0, 0x10000, 1 << 20) == apr.APR_ERR_INVALID_ARG
+    assert apr._merge_plan_init(one, 1, None, 1 << 20) == apr.APR_ERR_INVALID_ARG
+    assert apr._merge_plan_init(one, 1, 0x10040, 1 << 20) == apr.APR_ERR_INVALID_ARG     # not 128-byte aligned
+    assert apr._merge_plan_init(one, 1, 0x10000, 64) == apr.APR_ERR_WORKSPACE
+    bad = (apr.MergeProj * 1)(apr.MergeProj(0x1001, 0x2000, 64, 32, 0x3000, 0x4000))
+    assert apr._merge_plan_init(bad, 1, 0x10000, 1 << 20) == apr.APR_ERR_INVALID_ARG       # W not 16-byte aligned
+    odd = (apr.MergeProj * 1)(apr.MergeProj(0x1000, 0x2000, 60, 32, 0x3000, 0x4000))
+    assert apr._merge_plan_init(odd, 1, 0x10000, 1 << 20) == apr.APR_ERR_INVALID_ARG       # d_in % 8 != 0
+    # the planned merge refuses what the tensor-core merge cannot do, before launching
+    assert apr._merge_planned(0x1000, 0x10000, 1, 8, 32, 0x1000, 0x1000, 3, 0x100000, 1 << 20, None) == \
+        apr.APR_ERR_UNSUPPORTED
+

@@ -284,6 +284,21 @@ def test_merge_and_gemv_small(apr, E, r, k):
         ref = O.merge_adapters(Ws[p], As[p], Bs[p], idx1, g1.astype(np.float64))
         close(to_np(dWp[p]), ref, f"merged weight {p}")
         close(to_np(ys[p]), O.gemv(ref, xs[p]), f"gemv {p}")
+    # the planned (TMA) merge gives the same bits where the tensor-core merge applies
+    first = [w.clone() for w in dWp]
+    for w in dWp:
+        w.fill_(float("nan"))
+    plan = apr.merge_plan(entries)
+    args = (tab, plan, len(shapes), E, r, torch.from_numpy(idx1).cuda(), torch.from_numpy(g1).cuda(), k, ws)
+    if k * ((r + 15) // 16 * 16) <= 64:
+        apr.merge_adapters_planned(*args)
+        apr.stream_status(ws)
+        for p in range(len(shapes)):
+            assert torch.equal(dWp[p], first[p]), f"planned merge differs on weight {p}"
+    else:
+        with pytest.raises(apr.AprError) as ei:
+            apr.merge_adapters_planned(*args)
+        assert ei.value.status == apr.APR_ERR_UNSUPPORTED
 
 
 def test_merge_zero_B_is_bit_exact_copy(apr):
@@ -299,6 +314,12 @@ def test_merge_zero_B_is_bit_exact_copy(apr):
     ws = apr.workspace(1, 2, E, r, 8)
     apr.merge_adapters(tab, 1, E, r, torch.tensor([2, 0], dtype=torch.int32, device="cuda"),
                        torch.tensor([0.7, 0.3], dtype=torch.float32, device="cuda"), 2, ws)
+    apr.stream_status(ws)
+    assert torch.equal(dWp, dW)
+    dWp.zero_()
+    plan = apr.merge_plan([(dW, dWp, At, Bt)])
+    apr.merge_adapters_planned(tab, plan, 1, E, r, torch.tensor([2, 0], dtype=torch.int32, device="cuda"),
+                               torch.tensor([0.7, 0.3], dtype=torch.float32, device="cuda"), 2, ws)
     apr.stream_status(ws)
     assert torch.equal(dWp, dW)
 

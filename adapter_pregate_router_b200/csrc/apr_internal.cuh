@@ -27,10 +27,11 @@ struct WsHeader {
   int n_stiles;     // tensor-core set tiles written by the segment kernel
   int n_qtiles;     // tensor-core pair tiles (<= 128 pairs of one adapter)
   int n_mtiles;     // tensor-core mixed tiles (<= 128 tokens, <= 4 adapters in all)
+  unsigned sched;   // work counter of the tensor-core shrink (reset by the segment kernel and every expand)
   int T, k, E;      // routing the plan was built for
   unsigned bar_count;   // grid barrier of the fused skinny kernel: arrivals
   unsigned bar_gen;     //   and generation
-  int pad[53];
+  int pad[52];
 };
 static_assert(sizeof(WsHeader) == 256, "header is one alignment unit");
 

@@ -166,6 +166,7 @@ __global__ void __launch_bounds__(SEG_THREADS) segment_kernel(const int32_t* __r
     }
     if (tid == 0) {
       hdr->n_ptiles = ntiles;
+      hdr->sched = 0;
       hdr->T = T;
       hdr->k = k;
       hdr->E = E;

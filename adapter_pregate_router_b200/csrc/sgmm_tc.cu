@@ -117,7 +117,7 @@ __global__ void __launch_bounds__(SH_BLOCK, 1) tc_shrink_kernel(const __grid_con
   pdl_trigger();
 
   const WsLayout W = ws_layout(a.T, a.k, a.E);
-  const WsHeader* hdr = reinterpret_cast<const WsHeader*>(a.ws);
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(a.ws);
   const PairTile* qtiles = ws_at<PairTile>(a.ws, W.qtiles);
   __nv_bfloat16* vprep = ws_at<__nv_bfloat16>(a.ws, P.vprep_off);
   const long nitems = (long)hdr->n_qtiles * P.npg;
@@ -127,7 +127,12 @@ __global__ void __launch_bounds__(SH_BLOCK, 1) tc_shrink_kernel(const __grid_con
   uint32_t gchunk = 0, nitem = 0;
   bool abort = false;
 
-  for (long item = blockIdx.x; item < nitems; item += gridDim.x) {
+  // items are taken from a work counter (after one static item per CTA), so CTAs that
+  // draw small tiles take more of them
+  auto fetch_next = [&]() {
+    if (tid == 0) s_flags[2] = (int)gridDim.x + (int)atomicAdd(&hdr->sched, 1u);
+  };
+  for (long item = blockIdx.x; item < nitems;) {
     const PairTile tile = qtiles[item / P.npg];
     const int q0 = (int)(item % P.npg) * P.pg;
     const int nq = min(P.pg, a.nproj - q0);
@@ -152,7 +157,9 @@ __global__ void __launch_bounds__(SH_BLOCK, 1) tc_shrink_kernel(const __grid_con
     }
     __syncthreads();
     if (s_flags[1] || tile.len <= 0 || abort) {
+      fetch_next();
       __syncthreads();
+      item = s_flags[2];
       continue;
     }
     // source row of every A row of the item (null: a zero row)
@@ -181,13 +188,20 @@ __global__ void __launch_bounds__(SH_BLOCK, 1) tc_shrink_kernel(const __grid_con
                          "l"(x + (size_t)tk * d_in + (size_t)c * TB_BK + q * 8)
                          : "memory");
         }
+        // A rows: real rows by cp.async; rows past a rank are zeros, written with plain stores
+        // on the stage's first use in this item (no later copy touches them)
         const uint32_t abase = st_base + TB_M * 128;
         for (int w = tid; w < N1 * 8; w += SH_WORKERS) {
           const int j = w >> 3, q = w & 7;
           const __nv_bfloat16* src = s_arow[j];
-          cp_async16_zfill(abase + (uint32_t)j * 128 + (uint32_t)((q ^ (j & 7)) << 4),
-                           src ? (const void*)(src + (size_t)c * TB_BK + q * 8) : (const void*)x, src != nullptr);
+          const uint32_t dst = abase + (uint32_t)j * 128 + (uint32_t)((q ^ (j & 7)) << 4);
+          if (src)
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src + (size_t)c * TB_BK + q * 8)
+                         : "memory");
+          else if (c < S)
+            st_shared_zero16(dst);
         }
+        if (c < S) fence_proxy_async();
         cp_async_arrive(bar_full + 8 * s);
       }
       // gate -> V rows (bf16 hi | lo) at the pair's plan position
@@ -236,9 +250,11 @@ __global__ void __launch_bounds__(SH_BLOCK, 1) tc_shrink_kernel(const __grid_con
     }
     gchunk = g0 + nk;
     ++nitem;
+    fetch_next();
     tc_fence_before();
     abort = __syncthreads_or(abort);
     tc_fence_after();
+    item = s_flags[2];
   }
   if (abort && tid == 0) report(a.ws, APR_ERR_TIMEOUT, K_TC, (int)blockIdx.x);
   cp_async_wait_all();
@@ -314,7 +330,8 @@ __global__ void __launch_bounds__(EX_BLOCK, 1) tc_expand_kernel(const __grid_con
   pdl_trigger();
 
   const WsLayout W = ws_layout(a.T, a.k, a.E);
-  const WsHeader* hdr = reinterpret_cast<const WsHeader*>(a.ws);
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(a.ws);
+  if (blockIdx.x == 0 && tid == 0) hdr->sched = 0;      // this call's shrink is complete
   const int* tok_order = ws_at<int>(a.ws, W.tok_order);
   const int* inv = ws_at<int>(a.ws, W.inv);
   const SetTile* stiles = ws_at<SetTile>(a.ws, W.stiles);
@@ -406,9 +423,13 @@ __global__ void __launch_bounds__(EX_BLOCK, 1) tc_expand_kernel(const __grid_con
           for (int c = 0; c < R16 / 8; ++c) {
             const int kq = q * (R16 / 8) + c;
             const uint32_t off = (uint32_t)(prow >> 3) * SBO + (uint32_t)kq * 128 + (uint32_t)(prow & 7) * 16;
-            cp_async16_zfill(vbase + off, src ? (const void*)(src + c * 8) : (const void*)vprep, src != nullptr);
+            if (src)
+              asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(vbase + off), "l"(src + c * 8) : "memory");
+            else
+              st_shared_zero16(vbase + off);
           }
         }
+        fence_proxy_async();
         cp_async_arrive(bar_vfull + 8 * vb);
         for (int q = 0; q < kMixAdapters; ++q)
           Bs[q] = (!bad && q < nsl && su[q] >= 0) ? reinterpret_cast<const __nv_bfloat16*>(a.proj[p].B[su[q]]) : nullptr;
@@ -432,17 +453,25 @@ __global__ void __launch_bounds__(EX_BLOCK, 1) tc_expand_kernel(const __grid_con
                          "l"(yb + (size_t)tk * d_out + col)
                          : "memory");
         }
+        // Bcat: real chunks by cp.async; zero chunks (past a rank, an empty slot, past d_out) by
+        // plain stores when the slot's previous content may differ (the item's first tiles, the edge)
         const uint32_t bbuf = sbase + (uint32_t)L.b + slot * (uint32_t)(TB_NT * K2 * 2);
         const int cpr = K2 / 8, cps = R16 / 8;
+        const bool rezero = t < NY || c0 + TB_NT > d_out;
         for (int w = ptid; w < TB_NT * cpr; w += EX_PROD) {
           const int n = w / cpr, kq = w - n * cpr;
           const int sa = kq / cps, cq = kq - sa * cps;
           const __nv_bfloat16* B = Bs[sa];
           const int re = rs[sa];
           const bool ok = B != nullptr && c0 + n < d_out && cq * 8 < re;
-          cp_async16_zfill(bbuf + (uint32_t)(n >> 3) * SBO + (uint32_t)kq * 128 + (uint32_t)(n & 7) * 16,
-                           ok ? (const void*)(B + (size_t)(c0 + n) * re + cq * 8) : (const void*)vprep, ok);
+          const uint32_t dst = bbuf + (uint32_t)(n >> 3) * SBO + (uint32_t)kq * 128 + (uint32_t)(n & 7) * 16;
+          if (ok)
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(B + (size_t)(c0 + n) * re + cq * 8)
+                         : "memory");
+          else if (rezero)
+            st_shared_zero16(dst);
         }
+        if (rezero) fence_proxy_async();
         cp_async_arrive(bar_tfull + 8 * slot);
       }
     }
@@ -453,6 +482,7 @@ __global__ void __launch_bounds__(EX_BLOCK, 1) tc_expand_kernel(const __grid_con
     const int wrow0 = (warp & 3) * 32;
     uint32_t g = 0;
     int mcnt = -1, st_prev = -1, tok = -1;
+    bool live = true;
     for (int i = 0; item_at(i) < nitems && !abort; ++i) {
       int st, p, n0, ntl, d_out;
       item_shape(item_at(i), st, p, n0, ntl, d_out);
@@ -460,6 +490,7 @@ __global__ void __launch_bounds__(EX_BLOCK, 1) tc_expand_kernel(const __grid_con
         const int mb = (++mcnt) & 1;
         if (!mbar_wait(bar_mfull + 8 * mb, (mcnt >> 1) & 1)) { abort = true; break; }
         tok = s_tok[mb * TB_M + row];
+        live = __any_sync(0xffffffffu, tok >= 0);       // a warp whose 32 rows are all empty skips the work
       }
       st_prev = st;
       __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(a.proj[p].y);
@@ -474,7 +505,7 @@ __global__ void __launch_bounds__(EX_BLOCK, 1) tc_expand_kernel(const __grid_con
         unsigned char* yrow = ytile + (size_t)row * 256 + half * 128;
         const uint32_t taddr = tmem + ((uint32_t)((warp & 3) * 32) << 16) + b * 128 + (uint32_t)half * 64;
 #pragma unroll
-        for (int c16 = 0; c16 < 4; ++c16) {
+        for (int c16 = 0; c16 < 4 && live; ++c16) {
           float v[16];
           tmem_ld16(taddr + (uint32_t)(c16 * 16), v);
           if (tok >= 0) {
@@ -498,7 +529,7 @@ __global__ void __launch_bounds__(EX_BLOCK, 1) tc_expand_kernel(const __grid_con
         mbar_arrive(bar_d2empty + 8 * b);
         __syncwarp();
         // the warp's 32 rows x 128 bytes: 8 lanes per row segment
-        {
+        if (live) {
           const int q = lane & 7;
           const int col = half * 64 + q * 8;
 #pragma unroll

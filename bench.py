@@ -53,6 +53,33 @@ def load_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+def kernel_source_hash():
+    """SHA-1 prefix over the kernel sources, matched against the one a DRAM capture was taken on."""
+    import glob
+    import hashlib
+    h = hashlib.sha1()
+    csrc = os.path.join(ROOT, "adapter_pregate_router_b200", "csrc")
+    for f in sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh"))):
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(workload):
+    """DRAM bytes per SGMM call from the committed ncu capture, or None when the kernels changed since."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.md")
+    if not os.path.exists(path):
+        return None
+    want = kernel_source_hash()
+    with open(path) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) == 4 and parts[0] == "traffic:" and parts[1] == workload and parts[3] == want:
+                return float(parts[2])
+    return None
+
+
 class ClockSampler:
     """nvidia-smi clocks and throttle reasons sampled while the timed region runs."""
 
@@ -363,7 +390,9 @@ def run_gpu(args, world, rank, local):
         "bound": "hbm", "kernel": "apr_sgmm_shrink_expand (shrink+expand launches of every layer call)",
         "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
         "frac": achieved_gbs / peaks["hbm_gbs"], "peak_source": f"{peaks['source']} copy bandwidth",
-        "traffic": None, "bytes_per_call": layer_bytes / ncalls, "calls_per_step": ncalls,
+        "traffic": measured_traffic(args.workload) if not args.layers else None,
+        "traffic_source": "profiles/dram_traffic.md (ncu, one layer, bytes per call)",
+        "bytes_per_call": layer_bytes / ncalls, "calls_per_step": ncalls,
         "us_per_call": layer_ms * 1e3 / ncalls, "step_bytes": step_bytes,
         "step_frac": step_bytes / (ms_step * 1e-3) / 1e9 / peaks["hbm_gbs"],
     }

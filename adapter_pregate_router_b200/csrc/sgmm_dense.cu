@@ -10,19 +10,24 @@
 // did not select:
 //
 //  shrink  U[e*Rp + i, t] = (A_e x_t)_i for all e, t.  The input columns are
-//          split over clusters of 8 CTAs, 256 columns per CTA; each CTA stages
+//          split over clusters of 8 CTAs (16 where the rank rows fit one M
+//          tile and the device can place such a cluster), 256 columns per
+//          CTA; each CTA stages
 //          its slice of every A_e (before the PDL wait: weights never depend
 //          on the preceding launch) and of x (after it) in 128B-swizzled
 //          K-major tiles, and one thread issues the tcgen05 MMAs
 //          D[NR x Tp] = A_slice . x_slice^T (A as the M side, tokens as N).
-//          The 8 partial products are summed in a fixed order through
-//          distributed shared memory, gated
+//          The cluster's partial products are summed in a fixed order
+//          through distributed shared memory, gated
 //          V[t, e*Rp + i] = sum_j [idx[t,j] = e] g[t,j] U[e*Rp + i, t]
-//          and written as fp32 partials per cluster: [proj][cluster][Tp][NR].
+//          and written as fp32 partials per cluster: [proj][cluster][Tp][NR];
+//          when one cluster spans all of d_in, the final V is written instead,
+//          split into bf16 hi + lo in the expand's MMA operand layout.
 //  expand  one CTA per 128 output columns: D[128 x Tp] = Bslice . V^T with
 //          Bslice[n, e*Rp + i] = B_e[n, i] (staged before the wait, with the
 //          y_base columns) and V summed over the clusters in order and split
-//          into bf16 hi + lo halves (two MMAs keep ~16 mantissa bits of v).
+//          into bf16 hi + lo halves (two MMAs keep ~16 mantissa bits of v),
+//          or, with a single cluster, V fetched as is by two bulk copies.
 //          Thread n reads row n of D from TMEM and writes
 //          y[t, n] = y_base[t, n] + D[n, t], rounded to bf16 once.
 //
@@ -35,7 +40,7 @@ namespace apr {
 
 constexpr int DN_THREADS = 256;
 constexpr int DN_KC = 256;        // input columns per shrink CTA (four 64-column swizzle atoms)
-constexpr int DN_CL = 8;          // shrink CTAs per cluster
+constexpr int DN_CL = 8;          // shrink CTAs per cluster (16 when the rank rows fit one M tile)
 constexpr int DN_NT = 128;        // output columns per expand CTA
 
 struct DenseArgs {
@@ -45,6 +50,7 @@ struct DenseArgs {
   int NR;                              // E * Rp
   int MR;                              // NR rounded up to 128 (shrink MMA M)
   int ncl;                             // clusters along d_in
+  int direct;                          // ncl == 1: the shrink writes the final V (bf16 hi | lo, MMA layout)
   size_t vpart_off;                    // scratch offset of the gated partials
   int tiles_before[APR_MAX_PROJ + 1];  // expand: prefix of 128-column tiles per projection
 };
@@ -69,6 +75,9 @@ __device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
   asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
   return v;
 }
+__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
 __device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
 __device__ __forceinline__ void cluster_sync_all() {
@@ -80,7 +89,7 @@ __device__ __forceinline__ void cluster_sync_all() {
 
 // TP (tokens padded to 16) and MRT (rank rows padded to 128) are compile-time,
 // so the decode instantiation is short straight-line code.
-template <int TP, int MRT>
+template <int TP, int MRT, int CLT>
 __global__ void __launch_bounds__(DN_THREADS, 1) dense_shrink_kernel(const __grid_constant__ DenseArgs args) {
   const SgmmArgs& a = args.a;
   extern __shared__ unsigned char smem_raw[];
@@ -92,13 +101,15 @@ __global__ void __launch_bounds__(DN_THREADS, 1) dense_shrink_kernel(const __gri
   constexpr int Tp = TP, MR = MRT;
   const int Rp = args.Rp, NR = args.NR;
   const int T = a.T, K = a.k, E = a.E, d_in = a.d_in;
-  const int k0 = (cl * DN_CL + rank) * DN_KC;
+  const int k0 = (cl * CLT + rank) * DN_KC;
 
   // shared memory: A slice [4 atoms][MR][128 B], x slice [4 atoms][Tp][128 B];
   // after the MMAs the A area holds this CTA's partial product P[Tp][MR] fp32.
   unsigned char* sA = smem;
   unsigned char* sX = smem + (size_t)MR * 512;
-  unsigned char* meta = sX + (size_t)Tp * 512;
+  // MR == 128: partial rows pushed here by the cluster's CTAs, [source rank][Tp][MR / 8] fp32
+  float* red = reinterpret_cast<float*>(sX + (size_t)Tp * 512);
+  unsigned char* meta = sX + (size_t)Tp * 512 + (MR == 128 ? (size_t)Tp * MR * 4 : 0);
   uint64_t* bar = reinterpret_cast<uint64_t*>(meta);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(meta + 8);
   const __nv_bfloat16** s_Ap = reinterpret_cast<const __nv_bfloat16**>(meta + 16);   // [E]
@@ -186,41 +197,63 @@ __global__ void __launch_bounds__(DN_THREADS, 1) dense_shrink_kernel(const __gri
   if (!done) {
     if (tid == 0) report(a.ws, APR_ERR_TIMEOUT, K_SHRINK, (int)blockIdx.x);
   } else {
-    // TMEM -> P[t][r] (the A slice is no longer read)
-    const int wq = warp & 3, wg = warp >> 2;
-    const int r_in = wq * 32 + lane;
-    for (int mt = 0; mt < MR / 128; ++mt) {
-      if (MR == 256 && mt != wg) continue;
-      for (int c8 = 0; c8 < Tp / 8; ++c8) {
-        if (MR == 128 && (c8 & 1) != wg) continue;
+    if constexpr (MR == 128) {
+      // push: row r of the partial product goes to the CTA that owns it (rank r / (128 / CLT))
+      const int wq = warp & 3, wg = warp >> 2;
+      const int r = wq * 32 + lane;
+      const int owner = r / (MR / CLT), ri = r % (MR / CLT);
+      for (int c8 = wg; c8 < Tp / 8; c8 += 2) {
         float v[8];
-        tmem_ld8(tmem + ((uint32_t)(wq * 32) << 16) + (uint32_t)mt * cs + (uint32_t)(c8 * 8), v);
+        tmem_ld8(tmem + ((uint32_t)(wq * 32) << 16) + (uint32_t)(c8 * 8), v);
 #pragma unroll
-        for (int u = 0; u < 8; ++u) P[(size_t)(c8 * 8 + u) * MR + mt * 128 + r_in] = v[u];
+        for (int u = 0; u < 8; ++u) {
+          const int t = c8 * 8 + u;
+          const uint32_t off = smem_u32(red + ((size_t)(rank * Tp + t) * (MR / CLT) + ri));
+          st_cluster_f32(cluster_map(off, (uint32_t)owner), v[u]);
+        }
+      }
+    } else {
+      // TMEM -> P[t][r] (the A slice is no longer read)
+      const int wq = warp & 3, wg = warp >> 2;
+      const int r_in = wq * 32 + lane;
+      for (int mt = 0; mt < MR / 128; ++mt) {
+        if (mt != wg) continue;
+        for (int c8 = 0; c8 < Tp / 8; ++c8) {
+          float v[8];
+          tmem_ld8(tmem + ((uint32_t)(wq * 32) << 16) + (uint32_t)mt * cs + (uint32_t)(c8 * 8), v);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) P[(size_t)(c8 * 8 + u) * MR + mt * 128 + r_in] = v[u];
+        }
       }
     }
   }
   tc_fence_before();
-  cluster_sync_all();          // every CTA's P is complete
+  cluster_sync_all();          // every CTA's partial rows are in place
 
   // this CTA's share of the rows, summed over the cluster in rank order, gated
   {
-    constexpr int RS = MR / DN_CL;           // rows per CTA (16 or 32)
+    constexpr int RS = MR / CLT;             // rows per CTA (8, 16 or 32)
     constexpr int groups = RS / 4;
     float* vpart = ws_at<float>(a.ws, args.vpart_off) + ((size_t)(p * args.ncl + cl) * Tp) * NR;
-    constexpr int PER = 2;                   // float4 groups per thread: RS / 4 * Tp <= 8 * 64 = 2 * 256
-    float4 part[PER][DN_CL];
+    constexpr int PER = (groups * TP + DN_THREADS - 1) / DN_THREADS;   // float4 groups per thread (1 or 2)
+    float4 part[PER][CLT];
 #pragma unroll
     for (int u = 0; u < PER; ++u) {
       const int w = tid + u * DN_THREADS;
       if (w < groups * Tp) {
-        const int t = w / groups, r0 = rank * RS + (w % groups) * 4;
-        const uint32_t off = smem_u32(P + (size_t)t * MR + r0);
+        const int t = w / groups, g4 = w % groups;
+        if constexpr (MR == 128) {
 #pragma unroll
-        for (int c = 0; c < DN_CL; ++c) part[u][c] = ld_cluster_f4(cluster_map(off, (uint32_t)c));
+          for (int c = 0; c < CLT; ++c)
+            part[u][c] = *reinterpret_cast<const float4*>(red + ((size_t)(c * Tp + t) * RS + g4 * 4));
+        } else {
+          const uint32_t off = smem_u32(P + (size_t)t * MR + rank * RS + g4 * 4);
+#pragma unroll
+          for (int c = 0; c < CLT; ++c) part[u][c] = ld_cluster_f4(cluster_map(off, (uint32_t)c));
+        }
       }
     }
-    cluster_arrive();          // this CTA's reads of the cluster's P are issued and consumed below
+    if constexpr (MR != 128) cluster_arrive();   // this CTA's reads of the cluster's P are done
 #pragma unroll
     for (int u = 0; u < PER; ++u) {
       const int w = tid + u * DN_THREADS;
@@ -228,7 +261,7 @@ __global__ void __launch_bounds__(DN_THREADS, 1) dense_shrink_kernel(const __gri
       const int t = w / groups, r0 = rank * RS + (w % groups) * 4;
       float4 s = part[u][0];
 #pragma unroll
-      for (int c = 1; c < DN_CL; ++c) {
+      for (int c = 1; c < CLT; ++c) {
         s.x += part[u][c].x; s.y += part[u][c].y; s.z += part[u][c].z; s.w += part[u][c].w;
       }
       if (r0 >= NR) continue;
@@ -244,10 +277,29 @@ __global__ void __launch_bounds__(DN_THREADS, 1) dense_shrink_kernel(const __gri
           }
         }
       }
-      *reinterpret_cast<float4*>(vpart + (size_t)t * NR + r0) = make_float4(g * s.x, g * s.y, g * s.z, g * s.w);
+      if (args.direct) {
+        // the final V: bf16 hi | lo blocks in the expand's K-major core-matrix layout (K chunk r0 / 8)
+        __nv_bfloat16* vh = reinterpret_cast<__nv_bfloat16*>(ws_at<unsigned char>(a.ws, args.vpart_off) +
+                                                             (size_t)p * 4 * Tp * NR);
+        __nv_bfloat16* vl = vh + (size_t)Tp * NR;
+        const float f[4] = {g * s.x, g * s.y, g * s.z, g * s.w};
+        uint32_t hi[2], lo[2];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const __nv_bfloat162 hv = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+          const float2 hf = __bfloat1622float2(hv);
+          hi[i] = *reinterpret_cast<const uint32_t*>(&hv);
+          lo[i] = pack_bf16x2(f[2 * i] - hf.x, f[2 * i + 1] - hf.y);
+        }
+        const size_t o = ((size_t)(t >> 3) * (NR / 8) + (size_t)(r0 >> 3)) * 64 + (size_t)(t & 7) * 8 + (size_t)(r0 & 7);
+        *reinterpret_cast<uint2*>(vh + o) = make_uint2(hi[0], hi[1]);
+        *reinterpret_cast<uint2*>(vl + o) = make_uint2(lo[0], lo[1]);
+      } else {
+        *reinterpret_cast<float4*>(vpart + (size_t)t * NR + r0) = make_float4(g * s.x, g * s.y, g * s.z, g * s.w);
+      }
     }
   }
-  cluster_wait();              // every CTA's reads of this CTA's P are over before it leaves
+  if constexpr (MR != 128) cluster_wait();   // every CTA's reads of this CTA's P are over before it leaves
   if (warp == 0) tmem_dealloc(tmem, ncols);
 }
 
@@ -276,14 +328,15 @@ __global__ void __launch_bounds__(DN_THREADS, 1) dense_expand_kernel(const __gri
   unsigned char* sVL = sVH + (size_t)Tp * NR * 2;
   __nv_bfloat16* sYB = reinterpret_cast<__nv_bfloat16*>(sVL + (size_t)Tp * NR * 2);
   unsigned char* meta = reinterpret_cast<unsigned char*>(sYB + (size_t)Tp * DN_NT);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(meta);
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(meta + 8);
-  const __nv_bfloat16** s_Bp = reinterpret_cast<const __nv_bfloat16**>(meta + 16);   // [E]
-  int* s_rk = reinterpret_cast<int*>(meta + 16 + 8 * 16);                             // [E]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(meta);                                  // [2]: MMA done, V landed
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(meta + 16);
+  const __nv_bfloat16** s_Bp = reinterpret_cast<const __nv_bfloat16**>(meta + 32);   // [E]
+  int* s_rk = reinterpret_cast<int*>(meta + 32 + 8 * 16);                             // [E]
 
   const uint32_t ncols = tmem_cols_for(Tp);
   if (tid == 0) {
     mbar_init(smem_u32(bar), 1);
+    mbar_init(smem_u32(bar + 1), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 0) tmem_alloc(smem_u32(s_tmem), ncols);
@@ -321,6 +374,16 @@ __global__ void __launch_bounds__(DN_THREADS, 1) dense_expand_kernel(const __gri
   pdl_wait();
   pdl_trigger();
 
+  if (args.direct) {
+    // the final V, already in the MMA layout: two contiguous bulk copies on the V barrier
+    if (tid == 0) {
+      const unsigned char* src = ws_at<unsigned char>(a.ws, args.vpart_off) + (size_t)p * 4 * Tp * NR;
+      const uint32_t bytes = (uint32_t)(Tp * NR * 2);
+      mbar_arrive_expect_tx(smem_u32(bar + 1), 2 * bytes);
+      bulk_load_1d(smem_u32(sVH), src, bytes, smem_u32(bar + 1));
+      bulk_load_1d(smem_u32(sVL), src + bytes, bytes, smem_u32(bar + 1));
+    }
+  } else {
   // V = sum over the clusters' gated partials (in order), split into bf16 hi + lo
   {
     const float* vp = ws_at<float>(a.ws, args.vpart_off) + (size_t)p * args.ncl * Tp * NR;
@@ -383,11 +446,14 @@ __global__ void __launch_bounds__(DN_THREADS, 1) dense_expand_kernel(const __gri
       }
     }
   }
+  }
   cp_async_wait_all();
   fence_proxy_async();
   __syncthreads();
 
-  if (tid == 0) {
+  bool vready = true;
+  if (args.direct && tid == 0) vready = mbar_wait(smem_u32(bar + 1), 0);
+  if (tid == 0 && vready) {
     tc_fence_after();
     const uint32_t id = idesc_bf16(128, Tp);
     for (int kk = 0; kk < NR / 16; ++kk)
@@ -398,25 +464,32 @@ __global__ void __launch_bounds__(DN_THREADS, 1) dense_expand_kernel(const __gri
                id, 1u);
     mma_commit(smem_u32(bar));
   }
-  const bool done = mbar_wait(smem_u32(bar), 0);
+  const bool done = __syncthreads_and(vready) && mbar_wait(smem_u32(bar), 0);
   tc_fence_after();
   if (!done) {
     if (tid == 0) report(a.ws, APR_ERR_TIMEOUT, K_EXPAND, (int)blockIdx.x);
   } else {
-    // thread n holds D[n][t] for its column: y[t, n0 + n] = y_base[t, n0 + n] + D[n, t]
-    __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(a.proj[p].y);
+    // thread n holds D[n][t] for its column: y_base[t, n] + D[n, t] in place in shared memory,
+    // then whole 16-byte row pieces go out
     const int wq = warp & 3, wg = warp >> 2;
     const int n = wq * 32 + lane;
-    const bool col_ok = n0 + n < d_out;
     for (int c8 = wg; c8 < Tp / 8; c8 += 2) {
       float v[8];
       tmem_ld8(tmem + ((uint32_t)(wq * 32) << 16) + (uint32_t)(c8 * 8), v);
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         const int t = c8 * 8 + u;
-        if (t < T && col_ok)
-          y[(size_t)t * d_out + n0 + n] = __float2bfloat16_rn(__bfloat162float(sYB[(size_t)t * DN_NT + n]) + v[u]);
+        if (t < T) sYB[(size_t)t * DN_NT + n] = __float2bfloat16_rn(__bfloat162float(sYB[(size_t)t * DN_NT + n]) + v[u]);
       }
+    }
+  }
+  __syncthreads();
+  if (done) {
+    __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(a.proj[p].y);
+    for (int w = tid; w < T * (DN_NT / 8); w += DN_THREADS) {
+      const int t = w >> 4, c = (w & 15) * 8;
+      if (n0 + c < d_out)
+        *reinterpret_cast<uint4*>(y + (size_t)t * d_out + n0 + c) = *reinterpret_cast<const uint4*>(sYB + (size_t)t * DN_NT + c);
     }
   }
   tc_fence_before();
@@ -433,9 +506,29 @@ bool sgmm_dense_supported(const SgmmArgs& a, int dtype) {
   return dtype == APR_BF16 && dense_dims_ok(a.T, a.E, a.max_rank, a.d_in) && a.k <= APR_MAX_K;
 }
 
-static size_t shrink_smem(int MR, int Tp) { return (size_t)MR * 512 + (size_t)Tp * 512 + 16 + 8 * 16 + 4 * 16 + 8 * 64 * APR_MAX_K + 1024; }
+static size_t shrink_smem(int MR, int Tp) {
+  return (size_t)MR * 512 + (size_t)Tp * 512 + (MR == 128 ? (size_t)Tp * MR * 4 : 0) + 16 + 8 * 16 + 4 * 16 +
+         8 * 64 * APR_MAX_K + 1024;
+}
 static size_t expand_smem(int NR, int Tp) {
-  return (size_t)DN_NT * NR * 2 + 2 * (size_t)Tp * NR * 2 + (size_t)Tp * DN_NT * 2 + 16 + 8 * 16 + 4 * 16 + 128;
+  return (size_t)DN_NT * NR * 2 + 2 * (size_t)Tp * NR * 2 + (size_t)Tp * DN_NT * 2 + 32 + 8 * 16 + 4 * 16 + 128;
+}
+
+static void shrink_config(cudaLaunchConfig_t& cfg, cudaLaunchAttribute (&attr)[2], int cl, int ncl, int nproj,
+                          size_t smem, cudaStream_t s) {
+  cfg = cudaLaunchConfig_t{};
+  cfg.gridDim = dim3(cl, ncl, nproj);
+  cfg.blockDim = dim3(DN_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = cl;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
 }
 
 cudaError_t launch_sgmm_dense(const SgmmArgs& a, size_t scratch_off, cudaStream_t s) {
@@ -446,45 +539,60 @@ cudaError_t launch_sgmm_dense(const SgmmArgs& a, size_t scratch_off, cudaStream_
   d.Rp = dn_round16(a.max_rank);
   d.NR = a.E * d.Rp;
   d.MR = d.NR <= 128 ? 128 : 256;
-  d.ncl = dense_clusters(a.d_in);
   d.vpart_off = scratch_off;
   d.tiles_before[0] = 0;
   for (int p = 0; p < a.nproj; ++p) d.tiles_before[p + 1] = d.tiles_before[p] + (a.proj[p].d_out + DN_NT - 1) / DN_NT;
 
   const size_t sm1 = shrink_smem(d.MR, d.Tp), sm2 = expand_smem(d.NR, d.Tp);
   using Kern = void (*)(DenseArgs);
-  const int ti = d.Tp / 16 - 1, mi = d.MR / 128 - 1;
-  static const Kern shrinks[4][2] = {
-      {dense_shrink_kernel<16, 128>, dense_shrink_kernel<16, 256>}, {dense_shrink_kernel<32, 128>, dense_shrink_kernel<32, 256>},
-      {dense_shrink_kernel<48, 128>, dense_shrink_kernel<48, 256>}, {dense_shrink_kernel<64, 128>, dense_shrink_kernel<64, 256>}};
+  const int ti = d.Tp / 16 - 1;
+  // shrink variants: [rows 128, cluster 8] [rows 256, cluster 8] [rows 128, cluster 16]
+  static const Kern shrinks[4][3] = {
+      {dense_shrink_kernel<16, 128, 8>, dense_shrink_kernel<16, 256, 8>, dense_shrink_kernel<16, 128, 16>},
+      {dense_shrink_kernel<32, 128, 8>, dense_shrink_kernel<32, 256, 8>, dense_shrink_kernel<32, 128, 16>},
+      {dense_shrink_kernel<48, 128, 8>, dense_shrink_kernel<48, 256, 8>, dense_shrink_kernel<48, 128, 16>},
+      {dense_shrink_kernel<64, 128, 8>, dense_shrink_kernel<64, 256, 8>, dense_shrink_kernel<64, 128, 16>}};
   static const Kern expands[4] = {dense_expand_kernel<16>, dense_expand_kernel<32>, dense_expand_kernel<48>,
                                   dense_expand_kernel<64>};
-  static size_t conf1[4][2] = {}, conf2[4] = {};
-  const Kern k1 = shrinks[ti][mi], k2 = expands[ti];
+  static size_t conf1[4][3] = {}, conf2[4] = {};
+  static int wide_ok[4] = {};   // 0 unknown, 1 a 16-CTA cluster fits, -1 it does not
   cudaError_t err;
-  if (sm1 > conf1[ti][mi]) {
-    if ((err = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1)) != cudaSuccess) return err;
-    conf1[ti][mi] = sm1;
+  auto prepare = [&](int ti_, int vi) -> cudaError_t {
+    if (sm1 <= conf1[ti_][vi]) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(shrinks[ti_][vi], cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1);
+    if (e == cudaSuccess) conf1[ti_][vi] = sm1;
+    return e;
+  };
+  int vi = d.MR == 128 ? 0 : 1;
+  if (d.MR == 128 && wide_ok[ti] >= 0) {
+    // one 16-CTA cluster spans 4096 input columns; kept only where the device can place one
+    if ((err = prepare(ti, 2)) != cudaSuccess) return err;
+    if (wide_ok[ti] == 0) {
+      int nclus = 0;
+      cudaLaunchConfig_t cfg;
+      cudaLaunchAttribute attr[2];
+      shrink_config(cfg, attr, 16, 1, 1, sm1, s);
+      const bool ok = cudaFuncSetAttribute(shrinks[ti][2], cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+                          cudaSuccess &&
+                      cudaOccupancyMaxActiveClusters(&nclus, shrinks[ti][2], &cfg) == cudaSuccess && nclus >= 1;
+      (void)cudaGetLastError();
+      wide_ok[ti] = ok ? 1 : -1;
+    }
+    if (wide_ok[ti] > 0) vi = 2;
   }
+  const int cl = vi == 2 ? 16 : DN_CL;
+  d.ncl = (a.d_in + cl * DN_KC - 1) / (cl * DN_KC);
+  d.direct = d.ncl == 1;
+  const Kern k1 = shrinks[ti][vi], k2 = expands[ti];
+  if ((err = prepare(ti, vi)) != cudaSuccess) return err;
   if (sm2 > conf2[ti]) {
     if ((err = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2)) != cudaSuccess) return err;
     conf2[ti] = sm2;
   }
   {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(DN_CL, d.ncl, a.nproj);
-    cfg.blockDim = dim3(DN_THREADS);
-    cfg.dynamicSmemBytes = sm1;
-    cfg.stream = s;
+    cudaLaunchConfig_t cfg;
     cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    attr[1].id = cudaLaunchAttributeClusterDimension;
-    attr[1].val.clusterDim.x = DN_CL;
-    attr[1].val.clusterDim.y = 1;
-    attr[1].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 2;
+    shrink_config(cfg, attr, cl, d.ncl, a.nproj, sm1, s);
     count_launch();
     if ((err = cudaLaunchKernelEx(&cfg, k1, d)) != cudaSuccess) return err;
   }

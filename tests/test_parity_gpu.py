@@ -412,6 +412,8 @@ def test_sgmm_tensor_rejects_unsupported(apr):
     (17, 520, (264, 8), (64, 32, 8, 64), 1),               # rank slots of 64, k = 1, an 8-wide projection
     (50, 1024, (128,), (128, 8), 2),                       # rank 128: two adapters fill 256 rows
     (5, 64, (16,), (8,) * 3, 3),                           # k = E, fewer rank rows than one M tile
+    (16, 5000, (256,), (16,) * 16, 2),                     # 256 rank rows over three clusters, ragged
+    (24, 4104, (384,), (32,) * 4, 2),                      # one M tile, two wide clusters (the second 8 columns)
 ])
 def test_sgmm_dense_parity(apr, T, d_in, d_outs, ranks, k):
     rng = np.random.default_rng(T + d_in + k + 3)
@@ -425,11 +427,15 @@ def test_sgmm_dense_parity(apr, T, d_in, d_outs, ranks, k):
             close(got[p], ref[p], f"dense proj {p} zero_ybase={zero}")
 
 
-def test_sgmm_dense_integer_inputs_exact(apr):
+@pytest.mark.parametrize("d_in,ranks", [
+    (2560, (8, 16, 8, 24, 16)),      # 160 rank rows: partials per cluster, summed by the expand
+    (4096, (8, 16, 8, 16)),          # 64 rank rows: one cluster spans d_in and writes the final V
+])
+def test_sgmm_dense_integer_inputs_exact(apr, d_in, ranks):
     """Small integers, gates of 1/2: the dense result is the exact value rounded
     once to bf16 (pins the adapter-slot and token indexing of both products)."""
     rng = np.random.default_rng(31)
-    x, As, Bs, idx, gate, ybs = _case(rng, 40, 2560, (72, 136), (8, 16, 8, 24, 16), 2, ints=True)
+    x, As, Bs, idx, gate, ybs = _case(rng, 40, d_in, (72, 136), ranks, 2, ints=True)
     got = run_sgmm(apr, x, As, Bs, idx, gate, ybs, BF16, kernel=apr.SGMM_DENSE)
     ref = oracle_group(x, As, Bs, idx, gate.astype(np.float64), ybs)
     for p in range(2):

@@ -543,6 +543,22 @@ static PFN_cuTensorMapEncodeTiled tensor_map_encoder() {
   return fn;
 }
 
+// Row-scatter map of a [rows, cols] bf16 matrix: boxes of 64 columns x 1 row,
+// 128-byte swizzle (the tile::scatter4 / gather4 form: four rows per copy).
+cudaError_t encode_row_map(CUtensorMap* m, void* base, int rows, int cols) {
+  PFN_cuTensorMapEncodeTiled enc = tensor_map_encoder();
+  if (!enc) return cudaErrorNotSupported;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  const cuuint32_t box[2] = {64, 1};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+                 CUDA_SUCCESS
+             ? cudaSuccess
+             : cudaErrorInvalidValue;
+}
+
 size_t merge_plan_bytes(int nproj) { return (size_t)nproj * 2 * sizeof(CUtensorMap); }
 
 // One tensor map per W and per W': [d_out rows, d_in columns] bf16, boxes of

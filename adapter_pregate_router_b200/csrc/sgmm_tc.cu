@@ -52,6 +52,7 @@ constexpr int EX_BLOCK = EX_PROD + EX_EPI + 32;   // warp 16 issues MMAs
 constexpr int SMEM_BUDGET = 200 * 1024;
 
 struct TcPlan {
+  CUtensorMap ymap[APR_MAX_PROJ];    // expand: y of each projection as rows for tile::scatter4 stores
   SgmmArgs a;
   int R16;                           // rank slot per adapter
   int K2;                            // k * R16
@@ -60,6 +61,7 @@ struct TcPlan {
   int stages;                        // shrink pipeline depth
   int ny;                            // expand ring depth
   int mixed;                         // expand over mixed tiles (<= 4 adapters, K2 = 4 * R16) instead of set tiles
+  int ytma;                          // expand stores y rows with tile::scatter4 (else plain stores)
   size_t vprep_off;                  // scratch: V rows [proj][pair position][2 * R16] bf16
   int cc_before[APR_MAX_PROJ + 1];   // expand: prefix of 1024-column items per projection
 };
@@ -275,7 +277,7 @@ __host__ __device__ inline ExSmem ex_smem(int K2, int ny) {
   L.K2 = K2;
   L.ny = ny;
   L.vbuf = (size_t)2 * TB_M * K2 * 2;                 // one V buffer: hi then lo
-  L.y = 2 * L.vbuf;                                   // ring of y tiles [128 rows][256 B]
+  L.y = 2 * L.vbuf;                                   // ring of y tiles [2 halves][128 rows][128 B]
   L.b = L.y + (size_t)ny * TB_M * 256;                // ring of Bcat tiles [128][K2] bf16
   L.tok = L.b + (size_t)ny * TB_NT * K2 * 2;          // [2][128] token of each row
   L.bar = L.tok + 2 * TB_M * 4;
@@ -447,8 +449,8 @@ __global__ void __launch_bounds__(EX_BLOCK, 1) tc_expand_kernel(const __grid_con
           const int tk = s_tok[(mcnt & 1) * TB_M + row];
           const int col = c0 + hs * 64 + q * 8;
           if (tk >= 0 && col < d_out)
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(ybuf + (uint32_t)row * 256 +
-                                                                            (uint32_t)hs * 128 +
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(ybuf + (uint32_t)hs * (TB_M * 128) +
+                                                                            (uint32_t)row * 128 +
                                                                             (uint32_t)((q ^ (row & 7)) << 4)),
                          "l"(yb + (size_t)tk * d_out + col)
                          : "memory");
@@ -502,7 +504,8 @@ __global__ void __launch_bounds__(EX_BLOCK, 1) tc_expand_kernel(const __grid_con
         const int c0 = n0 + t * TB_NT;
         const int ncols = min(TB_NT, d_out - c0);
         unsigned char* ytile = smem + L.y + (size_t)slot * (TB_M * 256);
-        unsigned char* yrow = ytile + (size_t)row * 256 + half * 128;
+        unsigned char* yhalf = ytile + (size_t)half * (TB_M * 128);
+        unsigned char* yrow = yhalf + (size_t)row * 128;
         const uint32_t taddr = tmem + ((uint32_t)((warp & 3) * 32) << 16) + b * 128 + (uint32_t)half * 64;
 #pragma unroll
         for (int c16 = 0; c16 < 4 && live; ++c16) {
@@ -528,20 +531,42 @@ __global__ void __launch_bounds__(EX_BLOCK, 1) tc_expand_kernel(const __grid_con
         tc_fence_before();
         mbar_arrive(bar_d2empty + 8 * b);
         __syncwarp();
-        // the warp's 32 rows x 128 bytes: 8 lanes per row segment
+        // the warp's 32 rows x 128 bytes.  A warp whose 32 rows all hold tokens stores them four
+        // at a time with TMA tile::scatter4 (lane 0 issues; the map clips columns past d_out);
+        // other warps use plain stores, 8 lanes per row segment
+        bool used_tma = false;
         if (live) {
           const int q = lane & 7;
           const int col = half * 64 + q * 8;
+          const bool tma = P.ytma && __all_sync(0xffffffffu, tok >= 0) && half * 64 < ncols;
+          if (tma) {
+            fence_proxy_async();                          // the RMW above is visible to the TMA engine
+            __syncwarp();
 #pragma unroll
-          for (int it = 0; it < 8; ++it) {
-            const int rr = 4 * it + (lane >> 3);
-            const int tk = __shfl_sync(0xffffffffu, tok, rr);
-            const int r = wrow0 + rr;
-            if (tk >= 0 && col < ncols) {
-              const uint4 val = *reinterpret_cast<const uint4*>(ytile + (size_t)r * 256 + half * 128 + ((q ^ (r & 7)) << 4));
-              __stcs(reinterpret_cast<uint4*>(y + (size_t)tk * d_out + c0 + col), val);
+            for (int it = 0; it < 8; ++it) {
+              const int t0 = __shfl_sync(0xffffffffu, tok, 4 * it), t1 = __shfl_sync(0xffffffffu, tok, 4 * it + 1);
+              const int t2 = __shfl_sync(0xffffffffu, tok, 4 * it + 2), t3 = __shfl_sync(0xffffffffu, tok, 4 * it + 3);
+              if (lane == 0)
+                tma_scatter4(&P.ymap[p], c0 + half * 64, t0, t1, t2, t3,
+                             smem_u32(yhalf + (size_t)(wrow0 + 4 * it) * 128));
+            }
+            used_tma = true;
+          } else {
+#pragma unroll
+            for (int it = 0; it < 8; ++it) {
+              const int rr = 4 * it + (lane >> 3);
+              const int tk = __shfl_sync(0xffffffffu, tok, rr);
+              const int r = wrow0 + rr;
+              if (tk >= 0 && col < ncols) {
+                const uint4 val = *reinterpret_cast<const uint4*>(yhalf + (size_t)r * 128 + ((q ^ (r & 7)) << 4));
+                __stcs(reinterpret_cast<uint4*>(y + (size_t)tk * d_out + c0 + col), val);
+              }
             }
           }
+        }
+        if (used_tma && lane == 0) {
+          bulk_commit();
+          bulk_wait_read_all();                            // the slot may be refilled once the copies read it
         }
         __syncwarp();
         mbar_arrive(bar_tempty + 8 * slot);
@@ -555,6 +580,7 @@ __global__ void __launch_bounds__(EX_BLOCK, 1) tc_expand_kernel(const __grid_con
       }
       if (last) mbar_arrive(bar_mempty + 8 * (mcnt & 1));    // this tile's tokens are no longer read
     }
+    if (lane == 0) bulk_wait_all();                          // every y row written before the CTA ends
   } else if (lane == 0) {
     // ---------------------------------------------------- MMA issue
     const uint32_t id = idesc_bf16(TB_M, TB_NT);
@@ -629,6 +655,9 @@ cudaError_t launch_sgmm_tensor(const SgmmArgs& a, size_t scratch_off, cudaStream
   if (t.stages > 8) t.stages = 8;
   t.ny = t.K2 <= 32 ? 4 : 3;
   t.vprep_off = scratch_off;
+  t.ytma = 1;
+  for (int p = 0; p < a.nproj && t.ytma; ++p)
+    t.ytma = encode_row_map(&t.ymap[p], a.proj[p].y, a.T, a.proj[p].d_out) == cudaSuccess;
   t.cc_before[0] = 0;
   for (int p = 0; p < a.nproj; ++p) t.cc_before[p + 1] = t.cc_before[p] + (a.proj[p].d_out + TB_CW - 1) / TB_CW;
 

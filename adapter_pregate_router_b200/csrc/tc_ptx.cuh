@@ -9,6 +9,9 @@
 
 namespace apr {
 
+// Host: a [rows, cols] bf16 row-scatter tensor map (64-column x 1-row boxes,
+// 128-byte swizzle) for tile::gather4 / tile::scatter4 copies.
+cudaError_t encode_row_map(CUtensorMap* m, void* base, int rows, int cols);
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -387,7 +387,9 @@ def run_gpu(args, world, rank, local):
     ncalls = len(step.calls) if not cfg.merge else 1 + step.nmerge
     achieved_gbs = layer_bytes / (layer_ms * 1e-3) / 1e9
     roof = {
-        "bound": "hbm", "kernel": "apr_sgmm_shrink_expand (shrink+expand launches of every layer call)",
+        "bound": "hbm",
+        "kernel": ("apr_merge_adapters_planned + apr_gemv (the merge launch and every weight's GEMV)" if cfg.merge
+                   else "apr_sgmm_shrink_expand (shrink+expand launches of every layer call)"),
         "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
         "frac": achieved_gbs / peaks["hbm_gbs"], "peak_source": f"{peaks['source']} copy bandwidth",
         "traffic": measured_traffic(args.workload) if not args.layers else None,

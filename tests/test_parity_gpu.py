@@ -379,6 +379,28 @@ def test_sgmm_tensor_integer_inputs_exact(apr):
         assert np.array_equal(got[p], want), f"proj {p}: max diff {np.abs(got[p] - want).max()}"
 
 
+def test_sgmm_tensor_properties(apr):
+    """Zero B leaves y_base bit-exact; in place equals out of place; a token
+    permutation permutes the output bits (ragged d_out: the last tile's second
+    half is partly past the end)."""
+    rng = np.random.default_rng(24)
+    idx = _zipf_idx(rng, 900, 6, 2)
+    x, As, Bs, idx, gate, ybs = _case(rng, 900, 512, (1008, 80), (16,) * 6, 2, dist=idx)
+    x, As, Bs, ybs = _rounded(x, As, Bs, ybs)
+    Bz = [[np.zeros_like(b) for b in P] for P in Bs]
+    z = run_sgmm(apr, x, As, Bz, idx, gate, ybs, BF16, kernel=apr.SGMM_TENSOR)
+    for p in range(2):
+        assert np.array_equal(z[p], ybs[p].astype(np.float64))
+    a = run_sgmm(apr, x, As, Bs, idx, gate, ybs, BF16, kernel=apr.SGMM_TENSOR, in_place=True)
+    b = run_sgmm(apr, x, As, Bs, idx, gate, ybs, BF16, kernel=apr.SGMM_TENSOR)
+    for p in range(2):
+        assert np.array_equal(a[p], b[p])
+    perm = rng.permutation(900)
+    d = run_sgmm(apr, x[perm], As, Bs, idx[perm], gate[perm], [y[perm] for y in ybs], BF16, kernel=apr.SGMM_TENSOR)
+    for p in range(2):
+        assert np.array_equal(d[p], b[p][perm])
+
+
 def test_sgmm_tensor_matches_skinny(apr):
     rng = np.random.default_rng(22)
     idx = _zipf_idx(rng, 2000, 8, 2)

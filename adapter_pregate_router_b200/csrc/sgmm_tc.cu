@@ -19,17 +19,20 @@
 //          D1 back (one TMEM lane per pair), scales by the pair's gate and
 //          stores v as bf16 hi + lo halves (~16 mantissa bits) in the pair's
 //          row of the plan order: V[q][pos][hi: R16 | lo: R16].
-//  expand  item = (set tile, projection, 1024 output columns); a set tile is
-//          a run of <= 128 tokens sharing the same k <= 2 adapters {e0 < e1}.
-//          Per 128-column tile D2[128 x 128] = V_hi . Bcat^T + V_lo . Bcat^T
-//          with V[t] = [v(t, e0) | v(t, e1)] and Bcat[n] = [B_e0[n] | B_e1[n]],
-//          TMEM double buffered.  Warp-specialised: 4 producer warps gather V
-//          rows, y_base rows and Bcat with cp.async into a 4-deep ring, one
-//          thread issues the MMAs, and 8 epilogue warps compute
-//          y = y_base + D2 for their row and half, round once to bf16 and
-//          write back through shared memory so each warp stores whole
-//          128-byte row segments; loads, MMAs and stores of different tiles
-//          overlap.
+//  expand  item = (tile, projection, 1024 output columns).  A tile is a
+//          mixed tile (<= 128 consecutive plan tokens whose adapters number
+//          <= 4; slots u0 < u1 < u2 < u3) when 4 * R16 <= 64, else a set tile
+//          (<= 128 tokens sharing the same k <= 2 adapters).  Per 128-column
+//          tile D2[128 x 128] = V_hi . Bcat^T + V_lo . Bcat^T with V[t] =
+//          [v(t, u0) | ... ] (zero where t did not select the slot's adapter)
+//          and Bcat[n] = [B_u0[n] | ...], TMEM double buffered.
+//          Warp-specialised: 8 producer warps gather V rows, y_base rows and
+//          Bcat with cp.async into a 3-4 deep ring, one thread issues the
+//          MMAs, and 8 epilogue warps compute y = y_base + D2 for their row
+//          and half in shared memory, round once to bf16 and store: a warp
+//          whose 32 rows all hold tokens by TMA tile::scatter4 (four token
+//          rows per copy), others by coalesced 128-byte row segments.  Loads,
+//          MMAs and stores of different tiles overlap.
 //
 // Every mbarrier wait is bounded by the global timer (1 s); on expiry the CTA
 // records APR_ERR_TIMEOUT, drains its copies and frees its TMEM.

@@ -53,16 +53,42 @@ def load_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+def _code_tokens(text):
+    """C/CUDA source without comments and with whitespace runs collapsed: edits to comments or
+    layout leave it unchanged, any change to the code does not."""
+    import re
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c == '"':                                   # string literal (inline PTX), kept verbatim
+            j = i + 1
+            while j < n and text[j] != '"':
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    return re.sub(r"\s+", " ", "".join(out)).strip()
+
+
 def kernel_source_hash():
-    """SHA-1 prefix over the kernel sources, matched against the one a DRAM capture was taken on."""
+    """SHA-1 prefix over the kernel sources' code (comments and layout ignored), matched against
+    the one a DRAM capture was taken on."""
     import glob
     import hashlib
     h = hashlib.sha1()
     csrc = os.path.join(ROOT, "adapter_pregate_router_b200", "csrc")
     for f in sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh"))):
         h.update(os.path.basename(f).encode())
-        with open(f, "rb") as fh:
-            h.update(fh.read())
+        with open(f, encoding="utf-8") as fh:
+            h.update(_code_tokens(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -176,24 +176,30 @@ class Step:
     # ------------------------------------------------------------ bytes moved
     def algorithmic_bytes(self, idx_np=None) -> int:
         """Bytes the step must move at least once (inputs read once, outputs written once)."""
-        cfg = self.cfg
-        el = 2 if cfg.dtype == "bf16" else 4
-        T = cfg.T
         if idx_np is None:
             idx_np = self.idx.cpu().numpy()
-        touched = np.unique(idx_np.reshape(-1))
-        b = 0
-        b += T * cfg.d_router * el + cfg.E * cfg.d_router * el    # router h, Wr
-        for l in self.layers:
-            for g in cfg.groups:
-                if cfg.merge:
-                    for d_out in g.d_outs:
-                        b += 2 * d_out * g.d_in * el                              # W read, Wp write
-                        b += sum(int(self.ranks_np[e]) * (g.d_in + d_out) * el for e in touched)
-                        b += d_out * g.d_in * el + g.d_in * el + d_out * el       # GEMV
-                    continue
-                b += T * g.d_in * el                                               # x once per group
+        return algorithmic_bytes(self.cfg, self.layers, self.ranks_np, idx_np)
+
+
+def algorithmic_bytes(cfg: W.Config, layers, ranks_np, idx_np) -> int:
+    """Bytes a step must move at least once: the router's h and Wr; per shared-input group its x
+    once; per projection the A and B of every adapter some token selected, and y_base read plus y
+    written (SGMM); or, for the merge, W read, W' written, the selected adapters and the GEMV's
+    W', x and y."""
+    el = 2 if cfg.dtype == "bf16" else 4
+    T = cfg.T
+    touched = np.unique(np.asarray(idx_np).reshape(-1))
+    b = T * cfg.d_router * el + cfg.E * cfg.d_router * el                 # router h, Wr
+    for _ in layers:
+        for g in cfg.groups:
+            if cfg.merge:
                 for d_out in g.d_outs:
-                    b += sum(int(self.ranks_np[e]) * (g.d_in + d_out) * el for e in touched)
-                    b += 2 * T * d_out * el                                        # y_base read, y write
-        return b
+                    b += 2 * d_out * g.d_in * el                              # W read, W' written
+                    b += sum(int(ranks_np[e]) * (g.d_in + d_out) * el for e in touched)
+                    b += d_out * g.d_in * el + g.d_in * el + d_out * el       # GEMV
+                continue
+            b += T * g.d_in * el                                               # x once per group
+            for d_out in g.d_outs:
+                b += sum(int(ranks_np[e]) * (g.d_in + d_out) * el for e in touched)
+                b += 2 * T * d_out * el                                        # y_base read, y written
+    return b

@@ -53,3 +53,30 @@ def test_ranks_and_popularity():
     assert t.shape == (8192, 2) and np.all(t[:, 0] != t[:, 1])
     counts = np.bincount(t.ravel(), minlength=16)
     assert counts[0] > counts[5] > counts[15] > 0
+
+
+def test_algorithmic_bytes_match_the_workload_budgets():
+    """The bench's roofline numerator against the per-step budgets derived separately from the
+    workload shapes (router excluded there): decode 861.4 MB, prefill 58.05 GB, merge 39.0 GB
+    (26.06 merge + 12.96 GEMV); many tenants ~13.4 GB at the expected mean rank of 30, which the
+    drawn ranks only approach (hence the looser bound)."""
+    from adapter_pregate_router_b200 import pipeline as P
+
+    def step_bytes(name):
+        c = W.CONFIGS[name]
+        b = P.algorithmic_bytes(c, range(c.layers), W.ranks(c), W.forced_adapter_tuples(c))
+        el = 2 if c.dtype == "bf16" else 4
+        return b - (c.T + c.E) * c.d_router * el
+
+    assert abs(step_bytes("decode") - 861.4e6) < 0.05e6
+    assert abs(step_bytes("prefill") - 58.05e9) < 0.005e9
+    assert abs(step_bytes("merge") - 39.0e9) < 0.05e9
+    assert abs(step_bytes("multitenant") / 13.42e9 - 1) < 0.03
+    # an adapter nobody selected moves no bytes
+    c = W.CONFIGS["decode"]
+    idx_all = W.forced_adapter_tuples(c)
+    idx_one = np.zeros_like(idx_all)
+    full = P.algorithmic_bytes(c, [0], W.ranks(c), idx_all)
+    one = P.algorithmic_bytes(c, [0], W.ranks(c), idx_one)
+    per_adapter = sum(16 * (g.d_in + d) * 2 for g in c.groups for d in g.d_outs)
+    assert full - one == 7 * per_adapter

@@ -96,7 +96,8 @@ inline int shrink_kchunks(int d_in) { return (d_in + kShrinkKC - 1) / kShrinkKC;
 
 // Dense small-batch path: up to 64 tokens and an adapter bank of at most 16
 // adapters whose rank slots (max rank rounded up to 16) add up to <= 256 rows;
-// d_in is split over clusters of 8 CTAs x 256 columns.
+// d_in is split over clusters of 8 (or 16) CTAs x 256 columns.  Limits and
+// scratch are sized for clusters of 8, the larger count of partials.
 constexpr int kDenseMaxT = 64;
 constexpr int kDenseMaxRows = 256;
 constexpr int kDenseClusterCols = 8 * 256;

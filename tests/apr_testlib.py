@@ -55,9 +55,33 @@ def run_segment(apr, idx_np, E):
     return seg_off.cpu().numpy(), perm.cpu().numpy()[: T * k], ws
 
 
+# Guard bands around every SGMM output and y_base: GUARD elements on each side
+# (128 or 256 bytes, so the views keep 16-byte alignment) filled with SENTINEL
+# and compared bit for bit after the call: a write outside y, or into y_base
+# when the call is out of place, fails the test.
+GUARD = 64
+SENTINEL = -31.25
+
+
+def guarded(values, dtype):
+    """(buffer, view): ``values`` on the device inside a buffer with sentinel bands."""
+    n = values.size
+    buf = torch.full((n + 2 * GUARD,), SENTINEL, dtype=dtype, device="cuda")
+    view = buf[GUARD:GUARD + n].view(values.shape)
+    view.copy_(dev(values, dtype))
+    return buf, view
+
+
+def check_guards(buf, what):
+    band = torch.full((GUARD,), SENTINEL, dtype=buf.dtype, device=buf.device)
+    assert torch.equal(buf[:GUARD], band) and torch.equal(buf[-GUARD:], band), f"{what}: write outside the tensor"
+
+
 def run_sgmm(apr, x, As, Bs, idx_np, gate_np, ybases, dtype, kernel=0, in_place=False, ranks=None,
              max_rank=None, return_ws=False):
-    """One shared-input group: ``As[p][e]``, ``Bs[p][e]`` numpy; returns list of y (fp64)."""
+    """One shared-input group: ``As[p][e]``, ``Bs[p][e]`` numpy; returns list of y (fp64).
+    Outputs and y_base sit inside guard bands that are checked after the call; out of place,
+    y_base must come back unchanged."""
     T, d_in = x.shape
     k = idx_np.shape[1]
     E = len(As[0])
@@ -73,19 +97,29 @@ def run_sgmm(apr, x, As, Bs, idx_np, gate_np, ybases, dtype, kernel=0, in_place=
     perm = torch.empty(max(T * k, 1), dtype=torch.int32, device="cuda")
     apr.segment_tokens(idx, E, seg_off, perm, ws)
     xd = dev(x, dtype)
-    keep, projs, ys = [], [], []
+    keep, projs, ys, bands, inputs = [], [], [], [], []
     for p in range(len(As)):
         A = [dev(a, dtype) for a in As[p]]
         B = [dev(b, dtype) for b in Bs[p]]
         At, Bt = apr.ptr_array(A), apr.ptr_array(B)
-        yb = dev(ybases[p], dtype)
-        y = yb if in_place else torch.full_like(yb, float("nan"))
+        ybuf, yb = guarded(np.asarray(ybases[p], dtype=np.float32), dtype)
+        bands.append((ybuf, f"y_base {p}"))
+        if in_place:
+            y = yb
+        else:
+            inputs.append((ybuf, ybuf.clone(), p))
+            ybuf2, y = guarded(np.full(np.shape(ybases[p]), np.nan, np.float32), dtype)
+            bands.append((ybuf2, f"y {p}"))
         keep += [A, B, At, Bt, yb]
         projs.append(apr.make_proj(y, yb, At, Bt))
         ys.append(y)
     rk = torch.from_numpy(np.ascontiguousarray(ranks, dtype=np.int32)).cuda()
     apr.sgmm_shrink_expand(xd, projs, k, E, rk, max_rank, idx, gate, seg_off, perm, ws, kernel)
     apr.stream_status(ws)
+    for buf, what in bands:
+        check_guards(buf, what)
+    for buf, before, p in inputs:
+        assert torch.equal(buf, before), f"y_base {p} written by an out-of-place call"
     out = [to_np(y) for y in ys]
     if return_ws:
         return out, ws

@@ -10,8 +10,8 @@ import torch
 
 from oracle import apr_oracle as O
 from adapter_pregate_router_b200 import workloads as W
-from tests.apr_testlib import (GATE_ATOL, bf16_exact, close, oracle_group, run_route, run_segment,
-                               run_sgmm, to_np)
+from tests.apr_testlib import (GATE_ATOL, bf16_exact, check_guards, close, guarded, oracle_group, run_route,
+                               run_segment, run_sgmm, to_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -262,7 +262,9 @@ def test_merge_and_gemv_small(apr, E, r, k):
     idx1 = rng.permutation(E)[:k].astype(np.int32)
     g1 = rng.dirichlet(np.ones(k)).astype(np.float32)
     dW = [torch.from_numpy(w).cuda().to(BF16) for w in Ws]
-    dWp = [torch.full_like(w, float("nan")) for w in dW]
+    dW_in = [w.clone() for w in dW]
+    wp_bufs = [guarded(np.full(s, np.nan, np.float32), BF16) for s in shapes]   # W' inside guard bands
+    dWp = [v for _, v in wp_bufs]
     keep = []
     entries = []
     for p in range(len(shapes)):
@@ -274,12 +276,17 @@ def test_merge_and_gemv_small(apr, E, r, k):
     tab = apr.merge_table(entries)
     ws = apr.workspace(1, k, E, r, 8)
     apr.merge_adapters(tab, len(shapes), E, r, torch.from_numpy(idx1).cuda(), torch.from_numpy(g1).cuda(), k, ws)
-    ys = []
+    ys, y_bufs = [], []
     for p in range(len(shapes)):
-        y = torch.empty(shapes[p][0], dtype=BF16, device="cuda")
+        ybuf, y = guarded(np.full(shapes[p][0], np.nan, np.float32), BF16)
         apr.gemv(dWp[p], torch.from_numpy(xs[p]).cuda().to(BF16), y)
         ys.append(y)
+        y_bufs.append(ybuf)
     apr.stream_status(ws)
+    for p in range(len(shapes)):
+        check_guards(wp_bufs[p][0], f"merged weight {p}")
+        check_guards(y_bufs[p], f"gemv {p}")
+        assert torch.equal(dW[p], dW_in[p]), f"weight {p} written by the out-of-place merge"
     for p in range(len(shapes)):
         ref = O.merge_adapters(Ws[p], As[p], Bs[p], idx1, g1.astype(np.float64))
         close(to_np(dWp[p]), ref, f"merged weight {p}")
@@ -295,6 +302,8 @@ def test_merge_and_gemv_small(apr, E, r, k):
         apr.stream_status(ws)
         for p in range(len(shapes)):
             assert torch.equal(dWp[p], first[p]), f"planned merge differs on weight {p}"
+            check_guards(wp_bufs[p][0], f"planned merged weight {p}")
+            assert torch.equal(dW[p], dW_in[p]), f"weight {p} written by the planned merge"
     else:
         with pytest.raises(apr.AprError) as ei:
             apr.merge_adapters_planned(*args)
@@ -329,9 +338,10 @@ def test_gemv_parity(apr, d_out, d_in):
     rng = np.random.default_rng(d_out + d_in)
     Wt = bf16_exact(0.02 * rng.normal(size=(d_out, d_in)))
     x = bf16_exact(rng.normal(size=d_in))
-    y = torch.empty(d_out, dtype=BF16, device="cuda")
+    ybuf, y = guarded(np.full(d_out, np.nan, np.float32), BF16)
     apr.gemv(torch.from_numpy(Wt).cuda().to(BF16), torch.from_numpy(x).cuda().to(BF16), y)
     torch.cuda.synchronize()
+    check_guards(ybuf, "gemv")
     close(to_np(y), O.gemv(Wt, x), "gemv")
 
 

@@ -329,7 +329,8 @@ def config_block(cfg, world):
     return {"workload": descr, "name": cfg.name, "tokens_per_step": cfg.T,
             "adapters": cfg.E, "top_k": cfg.k, "ranks": list(cfg.rank_choices), "layers": cfg.layers,
             "parallelism": f"replicas x{world} (token batches, no collective)",
-            "l2": "working set larger than the 126 MB L2 (every layer has its own buffers); no flush"}
+            "l2": ("working set fits in the 126 MB L2 (parity case, no roofline claim)" if cfg.name == "tiny" else
+                   "working set larger than the 126 MB L2 (every layer has its own buffers); no flush")}
 
 
 # ---------------------------------------------------------------- GPU leg

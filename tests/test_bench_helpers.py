@@ -45,3 +45,43 @@ def test_measured_traffic_needs_the_matching_hash(tmp_path, monkeypatch):
     assert bench.measured_traffic("merge") is None        # no line
     os.remove(tmp_path / "profiles" / "dram_traffic.md")
     assert bench.measured_traffic("decode") is None
+
+
+def _run_bench(args, env_extra=None):
+    import subprocess
+    import sys
+    env = dict(os.environ)
+    env.update(env_extra or {})
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    return subprocess.run([sys.executable, os.path.join(root, "bench.py"), *args], cwd=root, env=env,
+                          capture_output=True, text=True, timeout=240)
+
+
+def test_reference_arm_prints_the_contract_line():
+    import json
+    r = _run_bench(["--impl", "reference", "--workload", "tiny", "--steps", "2", "--warmup", "3",
+                    "--ref-budget", "0.5"])
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.strip().startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["value"] > 0 and d["steps"] == 2 and d["warmup"] == 3
+    assert d["higher_is_better"] is True and d["scaling"] == "weak" and d["n_gpus"] == 1
+    assert d["config"]["workload"].startswith("tiny") and "model" not in d["config"]
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_other_ranks_exit_quietly():
+    r = _run_bench(["--impl", "reference", "--workload", "tiny", "--steps", "1", "--warmup", "3"],
+                   {"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
+    assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_bench_rejects_short_warmup():
+    r = _run_bench(["--impl", "reference", "--workload", "tiny", "--steps", "1", "--warmup", "2"])
+    assert r.returncode != 0 and "--warmup" in r.stderr

@@ -346,7 +346,8 @@ def run_gpu(args, world, rank, local):
         cfg = W.scaled(cfg, layers=args.layers)
     peaks = load_peaks()
     dev = torch.device("cuda", local)
-    step = pipeline.Step(cfg, device=dev)
+    kernels = {"auto": apr.SGMM_AUTO, "skinny": apr.SGMM_SKINNY, "tensor": apr.SGMM_TENSOR, "dense": apr.SGMM_DENSE}
+    step = pipeline.Step(cfg, device=dev, kernel=kernels[args.kernel])
     stream = torch.cuda.Stream(device=dev)
     stream.wait_stream(torch.cuda.current_stream(dev))
 
@@ -462,7 +463,8 @@ def run_gpu(args, world, rank, local):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16" if cfg.dtype == "bf16" else "f32", "data": "synthetic",
-        "config": config_block(cfg, world), "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+        "config": dict(config_block(cfg, world), **({"sgmm_kernel": args.kernel} if args.kernel != "auto" else {})),
+        "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
         "clocks": clk.summary(), "gpu_launches": launches * args.steps,
         "launches_per_step": launches,
     }
@@ -481,6 +483,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-budget", type=float, default=12.0, help="seconds of oracle work per reference step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel", default="auto", choices=["auto", "skinny", "tensor", "dense"],
+                    help="force one SGMM kernel class (comparisons; the benchmark line uses auto)")
     ap.add_argument("--layers", type=int, default=0,
                     help="build only this many layers (a reduced workload for profiling; not the benchmark)")
     args = ap.parse_args()

@@ -104,6 +104,23 @@ def test_sgmm_host_validation(apr):
     bad = (apr.Proj * 1)(apr.Proj(0x1000, 0x1000, 60, 0x1000, 0x1000))
     assert call(projs=bad) == apr.APR_ERR_INVALID_ARG
     assert call(T=0) == apr.APR_OK
+    assert call(T=-1) == apr.APR_ERR_INVALID_ARG
+    assert call(k=9, E=16) == apr.APR_ERR_INVALID_ARG                   # k above the maximum of 8
+    assert call(k=3, E=2) == apr.APR_ERR_INVALID_ARG                    # k above E
+    assert call(E=1025) == apr.APR_ERR_INVALID_ARG
+    assert call(dtype=2) == apr.APR_ERR_INVALID_ARG
+    assert call(x=0x1008) == apr.APR_ERR_INVALID_ARG                    # x not 16-byte aligned
+    for y, yb in ((0x1004, 0x1000), (0x1000, 0x1002)):                  # y or y_base misaligned
+        mis = (apr.Proj * 1)(apr.Proj(y, yb, 64, 0x1000, 0x1000))
+        assert call(projs=mis) == apr.APR_ERR_INVALID_ARG
+    nul = (apr.Proj * 1)(apr.Proj(0x1000, 0x1000, 64, None, 0x1000))   # no A table
+    assert call(projs=nul) == apr.APR_ERR_INVALID_ARG
+    assert call(projs=nul, T=0) == apr.APR_OK                          # nothing to do, nothing read
+    assert call(ws=None) == apr.APR_ERR_WORKSPACE
+    assert call(ws=0x100010) == apr.APR_ERR_WORKSPACE                   # not 256-byte aligned
+    for name in ("ranks", "idx", "gate", "seg_off", "perm"):
+        assert call(**{name: None}) == apr.APR_ERR_INVALID_ARG, name
+    assert "sgmm" in apr.last_error()
     # the tensor-core kernel refuses shapes outside its limits before launching
     assert call(kernel=2, dtype=0) == apr.APR_ERR_UNSUPPORTED
     # so does the dense kernel (fp32, or more than 64 tokens)

@@ -155,3 +155,39 @@ def test_merge_plan_host_validation(apr):
     assert apr._merge_planned(0x1000, 0x10000, 1, 8, 32, 0x1000, 0x1000, 3, 0x100000, 1 << 20, None) == \
         apr.APR_ERR_UNSUPPORTED
 
+
+
+def test_segment_and_noalloc_host_validation(apr):
+    def seg(**kw):
+        a = dict(idx=0x1000, T=4, k=2, E=8, seg_off=0x1000, perm=0x1000, ws=0x100000, ws_bytes=1 << 30, stream=None)
+        a.update(kw)
+        return apr._segment_tokens(*a.values())
+
+    assert seg(k=9, E=16) == apr.APR_ERR_INVALID_ARG
+    assert seg(k=3, E=2) == apr.APR_ERR_INVALID_ARG
+    assert seg(T=-2) == apr.APR_ERR_INVALID_ARG
+    assert seg(seg_off=None) == apr.APR_ERR_INVALID_ARG
+    assert seg(idx=None) == apr.APR_ERR_INVALID_ARG
+    assert seg(perm=None) == apr.APR_ERR_INVALID_ARG
+    assert seg(ws=None) == apr.APR_ERR_WORKSPACE
+    assert seg(ws=0x100080) == apr.APR_ERR_WORKSPACE
+    assert seg(ws_bytes=64) == apr.APR_ERR_WORKSPACE
+
+    def noalloc(**kw):
+        a = dict(h=0x1000, Wr=0x1000, dtype=1, T=4, d=64, E=8, k=2, idx=0x1000, gate=0x1000, stream=None)
+        a.update(kw)
+        return apr._pregate_route_noalloc(*a.values())
+
+    assert noalloc(E=4, k=5) == apr.APR_ERR_INVALID_ARG
+    assert noalloc(d=60) == apr.APR_ERR_INVALID_ARG
+    assert noalloc(dtype=3) == apr.APR_ERR_INVALID_ARG
+    assert noalloc(Wr=None) == apr.APR_ERR_INVALID_ARG
+    assert noalloc(Wr=0x1004) == apr.APR_ERR_INVALID_ARG
+    assert noalloc(T=1 << 21) == apr.APR_ERR_UNSUPPORTED          # T*E above the fixed scratch
+    assert noalloc(T=0, h=None, Wr=None) == apr.APR_OK
+
+
+def test_workspace_init_host_validation(apr):
+    assert apr._workspace_init(None, 1 << 20, None) == apr.APR_ERR_WORKSPACE
+    assert apr._workspace_init(0x100000, 8, None) == apr.APR_ERR_WORKSPACE
+    assert apr._workspace_init(0x100040, 1 << 20, None) == apr.APR_ERR_WORKSPACE

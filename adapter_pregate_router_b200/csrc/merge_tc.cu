@@ -26,7 +26,12 @@ static int round16(int r) { return (r + 15) / 16 * 16; }
 // contiguous along the output columns), TMEM double buffered; the W tile and
 // the A tile arrive two tiles ahead by cp.async into 3-deep rings, and the
 // epilogue adds D to W in fp32, rounds once and the warp writes its 32 rows
-// of W' back with coalesced 128-bit stores.
+// of W' back with coalesced 128-bit stores (merge_tc_kernel).
+// merge_tma_kernel does the same with the W tiles loaded and the W' tiles
+// stored by 2-D TMA boxes (64 columns x 128 rows, 128-byte swizzle) from
+// tensor maps built once per weight set (apr_merge_plan_init); the W tile
+// lands on a transaction-count mbarrier and the epilogue adds D in shared
+// memory before one thread stores the tile.
 
 constexpr int MT_BN = 128;                      // columns per tile
 constexpr int MT_NY = 3;                        // ring depth

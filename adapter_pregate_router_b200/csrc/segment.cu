@@ -12,6 +12,10 @@
 //                  k stable counting sorts), so that tokens sharing an adapter
 //                  set are contiguous
 //   set tiles      runs of <= kSetTile tokens with one adapter set
+//   qtiles         tiles of <= 128 pairs of one adapter (tensor-core shrink)
+//   mixed tiles    runs of <= 128 consecutive plan tokens whose adapters
+//                  number <= 4 (tensor-core expand, k <= 2), built by one
+//                  thread walking the set tiles in order
 // The histograms use shared-memory atomics (order-free counts); every order-
 // dependent step runs in one warp, 32 elements at a time, with __match_any_sync
 // ranking equal keys by lane, so the result is unique.

@@ -145,6 +145,41 @@ def workspace_size(T: int, k: int, E: int, max_rank: int, max_d_in: int) -> int:
     return int(_workspace_size(T, k, E, max_rank, max_d_in))
 
 
+def _need(t, name, dtypes=None, shape=None, ndim=None, min_numel=None):
+    """Validate one tensor argument before its pointer crosses the ABI: a torch tensor of an
+    accepted dtype and shape, contiguous.  The library reads raw memory, so a wrong dtype or
+    shape here would become an out-of-bounds device access there."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor, got {type(t).__name__}")
+    if dtypes is not None and t.dtype not in dtypes:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {' or '.join(str(d) for d in dtypes)}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions, got shape {tuple(t.shape)}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if min_numel is not None and t.numel() < min_numel:
+        raise ValueError(f"{name} has {t.numel()} elements, needs at least {min_numel}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _same_device(*named):
+    """Every tensor argument lives on one CUDA device (checked after dtypes and shapes)."""
+    for n, t in named:
+        if not t.is_cuda:
+            raise ValueError(f"{n} must be a CUDA tensor, got device {t.device}")
+    devs = {t.device for _, t in named}
+    if len(devs) > 1:
+        raise ValueError("tensors on different devices: " + ", ".join(f"{n}={t.device}" for n, t in named))
+
+
+_ACT = (torch.float32, torch.bfloat16)
+
+
+def _need_ws(ws):
+    _need(ws, "ws", (torch.uint8,), ndim=1)
+
+
 def workspace(T: int, k: int, E: int, max_rank: int, max_d_in: int, device="cuda", stream=None):
     """Allocate (with torch) and initialise a workspace for these maxima."""
     n = workspace_size(T, k, E, max_rank, max_d_in)
@@ -155,23 +190,40 @@ def workspace(T: int, k: int, E: int, max_rank: int, max_d_in: int, device="cuda
     return ws
 
 
-def pregate_route(h, Wr, k, idx, gate, ws, stream=None):
+def _check_route_args(h, Wr, k, idx, gate):
+    _need(h, "h", _ACT, ndim=2)
     T, d = h.shape
-    E = Wr.shape[0]
+    _need(Wr, "Wr", (h.dtype,), ndim=2)
+    if Wr.shape[1] != d:
+        raise ValueError(f"Wr has {Wr.shape[1]} columns, h has {d}")
+    _need(idx, "idx", (torch.int32,), shape=(T, k))
+    _need(gate, "gate", (torch.float32,), shape=(T, k))
+    return T, d, Wr.shape[0]
+
+
+def pregate_route(h, Wr, k, idx, gate, ws, stream=None):
+    T, d, E = _check_route_args(h, Wr, k, idx, gate)
+    _need_ws(ws)
+    _same_device(("h", h), ("Wr", Wr), ("idx", idx), ("gate", gate), ("ws", ws))
     _check(_pregate_route(_ptr(h), _ptr(Wr), _dtype_code(h), T, d, E, k, _ptr(idx), _ptr(gate),
                           _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def pregate_route_noalloc(h, Wr, k, idx, gate, stream=None):
     """``pregate_route`` for callers that cannot allocate a workspace (library-owned scratch)."""
-    T, d = h.shape
-    E = Wr.shape[0]
+    T, d, E = _check_route_args(h, Wr, k, idx, gate)
+    _same_device(("h", h), ("Wr", Wr), ("idx", idx), ("gate", gate))
     _check(_pregate_route_noalloc(_ptr(h), _ptr(Wr), _dtype_code(h), T, d, E, k, _ptr(idx), _ptr(gate),
                                   _stream(stream)))
 
 
 def segment_tokens(idx, E, seg_off, perm, ws, stream=None):
+    _need(idx, "idx", (torch.int32,), ndim=2)
     T, k = idx.shape
+    _need(seg_off, "seg_off", (torch.int32,), shape=(E + 1,))
+    _need(perm, "perm", (torch.int32,), ndim=1, min_numel=T * k)
+    _need_ws(ws)
+    _same_device(("idx", idx), ("seg_off", seg_off), ("perm", perm), ("ws", ws))
     _check(_segment_tokens(_ptr(idx), T, k, E, _ptr(seg_off), _ptr(perm), _ptr(ws), ws.numel(),
                            _stream(stream)))
 
@@ -182,13 +234,39 @@ def ptr_array(tensors, device="cuda") -> torch.Tensor:
 
 
 def make_proj(y, y_base, A_table, B_table) -> Proj:
-    return Proj(_ptr(y), _ptr(y_base), int(y_base.shape[-1]), _ptr(A_table), _ptr(B_table))
+    """One projection of a shared-input group: y [T, d_out] (may be y_base itself), y_base
+    [T, d_out] of the group's dtype, and the device tables of A and B pointers (int64 [E])."""
+    _need(y_base, "y_base", _ACT, ndim=2)
+    _need(y, "y", (y_base.dtype,), shape=tuple(y_base.shape))
+    _need(A_table, "A_table", (torch.int64,), ndim=1)
+    _need(B_table, "B_table", (torch.int64,), shape=tuple(A_table.shape))
+    _same_device(("y", y), ("y_base", y_base), ("A_table", A_table), ("B_table", B_table))
+    p = Proj(_ptr(y), _ptr(y_base), int(y_base.shape[-1]), _ptr(A_table), _ptr(B_table))
+    p.meta = (y_base.dtype, int(y_base.shape[0]), int(A_table.shape[0]), y_base.device)
+    return p
 
 
 def sgmm_shrink_expand(x, projs, k, E, ranks, max_rank, idx, gate, seg_off, perm, ws,
                        kernel=SGMM_AUTO, stream=None):
     """projs: a sequence of ``Proj`` (see ``make_proj``) sharing input ``x``."""
+    _need(x, "x", _ACT, ndim=2)
     T, d_in = x.shape
+    for i, pj in enumerate(projs):
+        meta = getattr(pj, "meta", None)
+        if meta is None:
+            raise TypeError(f"projs[{i}] was not made by make_proj")
+        dt, t_rows, e_tab, pdev = meta
+        if dt != x.dtype or t_rows != T or e_tab < E or pdev != x.device:
+            raise ValueError(f"projs[{i}]: {dt} [{t_rows}, :] with {e_tab} adapters on {pdev} does not fit "
+                             f"x {x.dtype} [{T}, {d_in}] with E={E} on {x.device}")
+    _need(ranks, "ranks", (torch.int32,), shape=(E,))
+    _need(idx, "idx", (torch.int32,), shape=(T, k))
+    _need(gate, "gate", (torch.float32,), shape=(T, k))
+    _need(seg_off, "seg_off", (torch.int32,), shape=(E + 1,))
+    _need(perm, "perm", (torch.int32,), ndim=1, min_numel=T * k)
+    _need_ws(ws)
+    _same_device(("x", x), ("ranks", ranks), ("idx", idx), ("gate", gate), ("seg_off", seg_off),
+                 ("perm", perm), ("ws", ws))
     arr = (Proj * len(projs))(*projs)
     _check(_sgmm(_ptr(x), d_in, arr, len(projs), _dtype_code(x), T, k, E, _ptr(ranks), max_rank,
                  _ptr(idx), _ptr(gate), _ptr(seg_off), _ptr(perm), _ptr(ws), ws.numel(), kernel,
@@ -223,17 +301,32 @@ def merge_plan(entries, device="cuda") -> torch.Tensor:
     return plan
 
 
+def _check_merge_args(table, nproj, idx, gate, k, ws):
+    _need(table, "table", (torch.uint8,), ndim=1, min_numel=nproj * ctypes.sizeof(MergeProj))
+    _need(idx, "idx", (torch.int32,), min_numel=k)
+    _need(gate, "gate", (torch.float32,), min_numel=k)
+    _need_ws(ws)
+    _same_device(("table", table), ("idx", idx), ("gate", gate), ("ws", ws))
+
+
 def merge_adapters_planned(table, plan, nproj, E, r, idx, gate, k, ws, stream=None):
+    _check_merge_args(table, nproj, idx, gate, k, ws)
+    _need(plan, "plan", (torch.uint8,), ndim=1, min_numel=int(_merge_plan_size(nproj)))
     _check(_merge_planned(_ptr(table), _ptr(plan), nproj, E, r, _ptr(idx), _ptr(gate), k, _ptr(ws), ws.numel(),
                           _stream(stream)))
 
 
 def merge_adapters(table, nproj, E, r, idx, gate, k, ws, stream=None):
+    _check_merge_args(table, nproj, idx, gate, k, ws)
     _check(_merge(_ptr(table), nproj, E, r, _ptr(idx), _ptr(gate), k, _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def gemv(W, x, y, stream=None):
+    _need(W, "W", (torch.bfloat16,), ndim=2)
     d_out, d_in = W.shape
+    _need(x, "x", (torch.bfloat16,), shape=(d_in,))
+    _need(y, "y", (torch.bfloat16,), shape=(d_out,))
+    _same_device(("W", W), ("x", x), ("y", y))
     _check(_gemv(_ptr(W), _ptr(x), _ptr(y), d_in, d_out, _stream(stream)))
 
 

@@ -16,6 +16,35 @@ static std::atomic<uint64_t> g_launches{0};
 
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
+cudaError_t SmemLimit::ensure(const void* func, size_t bytes) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= kMaxDevices)
+    return cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  std::lock_guard<std::mutex> lock(mu);
+  if (bytes <= done[dev]) return cudaSuccess;
+  err = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (err == cudaSuccess) done[dev] = bytes;
+  return err;
+}
+
+int device_sm_count() {
+  static std::mutex mu;
+  static int cached[kMaxDevices] = {};
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev >= 0 && dev < kMaxDevices) {
+    std::lock_guard<std::mutex> lock(mu);
+    if (cached[dev] > 0) return cached[dev];
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cached[dev] = n;
+    return n;
+  }
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  return n;
+}
+
 void set_error(const char* fmt, ...) {
   va_list ap;
   va_start(ap, fmt);
@@ -289,9 +318,8 @@ apr_status apr_stream_status(void* ws, void* stream) {
   e = cudaMemcpy(words, ws, sizeof(words), cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return cuda_fail(e, "stream_status read");
   if (words[0] != 0) {
-    // clear the error word and the grid-barrier arrivals a failed wait may have left behind
+    // clear the error word and its detail
     e = cudaMemset(ws, 0, 2 * sizeof(int));
-    if (e == cudaSuccess) e = cudaMemset(&reinterpret_cast<WsHeader*>(ws)->bar_count, 0, sizeof(unsigned));
     if (e != cudaSuccess) return cuda_fail(e, "stream_status clear");
     return fail((apr_status)words[0], "device reported %s (kernel %d, value %d)",
                 apr_status_string(words[0]), (words[1] >> 24) & 0xFF, words[1] & 0xFFFFFF);

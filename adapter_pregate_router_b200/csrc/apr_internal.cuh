@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
 #include <utility>
 
 #include "../../include/apr.h"
@@ -29,9 +30,7 @@ struct WsHeader {
   int n_mtiles;     // tensor-core mixed tiles (<= 128 tokens, <= 4 adapters in all)
   unsigned sched;   // work counter of the tensor-core shrink (reset by the segment kernel and every expand)
   int T, k, E;      // routing the plan was built for
-  unsigned bar_count;   // grid barrier of the fused skinny kernel: arrivals
-  unsigned bar_gen;     //   and generation
-  int pad[52];
+  int pad[54];
 };
 static_assert(sizeof(WsHeader) == 256, "header is one alignment unit");
 
@@ -229,6 +228,23 @@ namespace apr {
 
 void count_launch();
 void set_error(const char* fmt, ...);
+
+// Kernel attributes and device properties are per device, and a process may
+// drive several devices from several threads: each record below is kept per
+// device ordinal under a lock.
+constexpr int kMaxDevices = 64;
+
+// A kernel's raised dynamic shared-memory limit, per device.
+struct SmemLimit {
+  std::mutex mu;
+  size_t done[kMaxDevices] = {};
+  // Raise `func`'s limit to at least `bytes` on the current device (once per
+  // device and size; devices past kMaxDevices are set on every call).
+  cudaError_t ensure(const void* func, size_t bytes);
+};
+
+// Streaming multiprocessors of the current device (cached per device).
+int device_sm_count();
 
 // Launch with programmatic stream serialization allowed (PDL).
 template <typename... KArgs, typename... Args>

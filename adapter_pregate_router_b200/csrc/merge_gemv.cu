@@ -197,9 +197,7 @@ __global__ void __launch_bounds__(GV_THREADS) gemv_kernel(const __nv_bfloat16* _
 
 cudaError_t launch_merge(const apr_merge_proj* projs, int nproj, int E, int r, const int32_t* idx,
                          const float* gate, int k, void* ws, cudaStream_t s) {
-  int dev = 0, nsm = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  const int nsm = device_sm_count();
   const size_t smem = sizeof(int) * ((size_t)nproj + 1);
   return launch_pdl(merge_kernel, dim3(nsm * 8), dim3(MG_THREADS), smem, s, projs, nproj, E, r, idx,
                     gate, k, ws);
@@ -208,12 +206,10 @@ cudaError_t launch_merge(const apr_merge_proj* projs, int nproj, int E, int r, c
 cudaError_t launch_gemv(const void* W, const void* x, void* y, int d_in, int d_out, cudaStream_t s) {
   const int rows_per_block = GV_THREADS / 32;
   const size_t smem = sizeof(__nv_bfloat16) * (size_t)d_in;
-  static size_t configured = 0;
-  if (smem > 48 * 1024 && smem > configured) {
-    cudaError_t err =
-        cudaFuncSetAttribute(gemv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  static SmemLimit limit;
+  if (smem > 48 * 1024) {
+    cudaError_t err = limit.ensure((const void*)gemv_kernel, smem);
     if (err != cudaSuccess) return err;
-    configured = smem;
   }
   return launch_pdl(gemv_kernel, dim3((d_out + rows_per_block - 1) / rows_per_block),
                     dim3(GV_THREADS), smem, s, (const __nv_bfloat16*)W, (const __nv_bfloat16*)x,

@@ -591,15 +591,10 @@ cudaError_t merge_plan_build(const apr_merge_proj* projs, int nproj, void* plan)
 cudaError_t launch_merge_tma(const apr_merge_proj* projs, const void* plan, int nproj, int E, int r,
                              const int32_t* idx, const float* gate, int k, void* ws, cudaStream_t s) {
   const size_t smem = MmSmem::fixed_bytes() + sizeof(int) * ((size_t)nproj + 1);
-  static size_t configured = 0;
-  if (smem > configured) {
-    cudaError_t err = cudaFuncSetAttribute(merge_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (err != cudaSuccess) return err;
-    configured = smem;
-  }
-  int dev = 0, nsm = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  static SmemLimit limit;
+  cudaError_t err = limit.ensure((const void*)merge_tma_kernel, smem);
+  if (err != cudaSuccess) return err;
+  const int nsm = device_sm_count();
   return launch_pdl(merge_tma_kernel, dim3(nsm), dim3(TC_THREADS), smem, s, projs,
                     reinterpret_cast<const CUtensorMap*>(plan), nproj, E, r, round16(r), idx, gate, k, ws);
 }
@@ -611,15 +606,10 @@ bool merge_tensor_supported(int k, int r, int nproj) {
 cudaError_t launch_merge_tensor(const apr_merge_proj* projs, int nproj, int E, int r, const int32_t* idx,
                                 const float* gate, int k, void* ws, cudaStream_t s) {
   const size_t smem = MtSmem::fixed_bytes() + sizeof(int) * ((size_t)nproj + 1);
-  static size_t configured = 0;
-  if (smem > configured) {
-    cudaError_t err = cudaFuncSetAttribute(merge_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (err != cudaSuccess) return err;
-    configured = smem;
-  }
-  int dev = 0, nsm = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  static SmemLimit limit;
+  cudaError_t err = limit.ensure((const void*)merge_tc_kernel, smem);
+  if (err != cudaSuccess) return err;
+  const int nsm = device_sm_count();
   return launch_pdl(merge_tc_kernel, dim3(nsm), dim3(TC_THREADS), smem, s, projs, nproj, E, r, round16(r), idx,
                     gate, k, ws);
 }

@@ -215,7 +215,6 @@ constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;
 constexpr size_t kNoAllocHeaderBytes = 256;
 static __device__ __align__(256) unsigned char g_route_noalloc_scratch[kNoAllocScratchBytes];
 
-constexpr int kMaxDevices = 64;
 static std::mutex g_noalloc_mu;
 static void* g_noalloc_ptr[kMaxDevices];
 

@@ -554,20 +554,19 @@ cudaError_t launch_sgmm_dense(const SgmmArgs& a, size_t scratch_off, cudaStream_
       {dense_shrink_kernel<64, 128, 8>, dense_shrink_kernel<64, 256, 8>, dense_shrink_kernel<64, 128, 16>}};
   static const Kern expands[4] = {dense_expand_kernel<16>, dense_expand_kernel<32>, dense_expand_kernel<48>,
                                   dense_expand_kernel<64>};
-  static size_t conf1[4][3] = {}, conf2[4] = {};
-  static int wide_ok[4] = {};   // 0 unknown, 1 a 16-CTA cluster fits, -1 it does not
+  static SmemLimit lim1[4][3], lim2[4];
+  // whether a 16-CTA cluster of each token padding fits the device: 0 unknown, 1 yes, -1 no
+  static std::mutex wide_mu;
+  static int wide_ok[kMaxDevices][4] = {};
   cudaError_t err;
-  auto prepare = [&](int ti_, int vi) -> cudaError_t {
-    if (sm1 <= conf1[ti_][vi]) return cudaSuccess;
-    cudaError_t e = cudaFuncSetAttribute(shrinks[ti_][vi], cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1);
-    if (e == cudaSuccess) conf1[ti_][vi] = sm1;
-    return e;
-  };
   int vi = d.MR == 128 ? 0 : 1;
-  if (d.MR == 128 && wide_ok[ti] >= 0) {
+  int dev = 0;
+  if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
+  if (d.MR == 128 && dev >= 0 && dev < kMaxDevices) {
     // one 16-CTA cluster spans 4096 input columns; kept only where the device can place one
-    if ((err = prepare(ti, 2)) != cudaSuccess) return err;
-    if (wide_ok[ti] == 0) {
+    if ((err = lim1[ti][2].ensure((const void*)shrinks[ti][2], sm1)) != cudaSuccess) return err;
+    std::lock_guard<std::mutex> lock(wide_mu);
+    if (wide_ok[dev][ti] == 0) {
       int nclus = 0;
       cudaLaunchConfig_t cfg;
       cudaLaunchAttribute attr[2];
@@ -576,19 +575,16 @@ cudaError_t launch_sgmm_dense(const SgmmArgs& a, size_t scratch_off, cudaStream_
                           cudaSuccess &&
                       cudaOccupancyMaxActiveClusters(&nclus, shrinks[ti][2], &cfg) == cudaSuccess && nclus >= 1;
       (void)cudaGetLastError();
-      wide_ok[ti] = ok ? 1 : -1;
+      wide_ok[dev][ti] = ok ? 1 : -1;
     }
-    if (wide_ok[ti] > 0) vi = 2;
+    if (wide_ok[dev][ti] > 0) vi = 2;
   }
   const int cl = vi == 2 ? 16 : DN_CL;
   d.ncl = (a.d_in + cl * DN_KC - 1) / (cl * DN_KC);
   d.direct = d.ncl == 1;
   const Kern k1 = shrinks[ti][vi], k2 = expands[ti];
-  if ((err = prepare(ti, vi)) != cudaSuccess) return err;
-  if (sm2 > conf2[ti]) {
-    if ((err = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2)) != cudaSuccess) return err;
-    conf2[ti] = sm2;
-  }
+  if ((err = lim1[ti][vi].ensure((const void*)k1, sm1)) != cudaSuccess) return err;
+  if ((err = lim2[ti].ensure((const void*)k2, sm2)) != cudaSuccess) return err;
   {
     cudaLaunchConfig_t cfg;
     cudaLaunchAttribute attr[2];

@@ -550,16 +550,6 @@ static int expand_tokens_per_tile(int k, int max_rank) {
   return tt;
 }
 
-static int sm_count() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-  }
-  return n;
-}
-
 template <typename In>
 static cudaError_t launch_skinny_typed(const SgmmArgs& a, size_t scratch_off, cudaStream_t s) {
   SkinnyParams P;
@@ -588,18 +578,15 @@ static cudaError_t launch_skinny_typed(const SgmmArgs& a, size_t scratch_off, cu
   const size_t smem = skinny_smem_layout(P.TT, a.k, a.max_rank, elem, P.bslots, P.dense_k).total;
   const long nA = (long)a.nproj * a.E * P.nkc * P.nrc * P.nsplit;
   const long nB = (long)a.nproj * P.ntt * P.ntd;
-  const long capA = 16L * sm_count();
+  const long capA = 16L * device_sm_count();
   const long gA = nA < capA ? (nA > 0 ? nA : 1) : capA;
   const size_t smemA = skinny_smem_layout(P.TT, a.k, a.max_rank, elem, 0, 0).B;   // shrink: reduction buffers only
   cudaError_t err = launch_pdl(sgmm_skinny_kernel<In, 0>, dim3((unsigned)gA), dim3(SK_THREADS), smemA, s, a, P);
   if (err != cudaSuccess) return err;
-  static size_t configured = 0;
-  if (smem > 48 * 1024 && smem > configured) {
-    err = cudaFuncSetAttribute(sgmm_skinny_kernel<In, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (err != cudaSuccess) return err;
-    configured = smem;
-  }
-  const long capB = 64L * sm_count();
+  static SmemLimit limit;
+  if (smem > 48 * 1024 && (err = limit.ensure((const void*)sgmm_skinny_kernel<In, 1>, smem)) != cudaSuccess)
+    return err;
+  const long capB = 64L * device_sm_count();
   const long gB = nB < capB ? (nB > 0 ? nB : 1) : capB;
   return launch_pdl(sgmm_skinny_kernel<In, 1>, dim3((unsigned)gB), dim3(SK_THREADS), smem, s, a, P);
 }

@@ -665,21 +665,11 @@ cudaError_t launch_sgmm_tensor(const SgmmArgs& a, size_t scratch_off, cudaStream
   for (int p = 0; p < a.nproj; ++p) t.cc_before[p + 1] = t.cc_before[p] + (a.proj[p].d_out + TB_CW - 1) / TB_CW;
 
   const size_t sm1 = sh_smem(n1max, t.stages).total, sm2 = ex_smem(t.K2, t.ny).total;
-  static size_t conf1 = 0, conf2 = 0;
+  static SmemLimit lim1, lim2;
   cudaError_t err;
-  if (sm1 > conf1) {
-    if ((err = cudaFuncSetAttribute(tc_shrink_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1)) != cudaSuccess)
-      return err;
-    conf1 = sm1;
-  }
-  if (sm2 > conf2) {
-    if ((err = cudaFuncSetAttribute(tc_expand_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2)) != cudaSuccess)
-      return err;
-    conf2 = sm2;
-  }
-  int dev = 0, nsm = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  if ((err = lim1.ensure((const void*)tc_shrink_kernel, sm1)) != cudaSuccess) return err;
+  if ((err = lim2.ensure((const void*)tc_expand_kernel, sm2)) != cudaSuccess) return err;
+  const int nsm = device_sm_count();
   // tile counts are bounded by the plan's maxima; the kernels loop over the real ones
   const long max_q = max_qtiles(a.T, a.k, a.E), max_s = (long)a.T + (a.T + TB_M - 1) / TB_M;
   const int g1 = (int)(max_q * t.npg < nsm ? max_q * t.npg : nsm);

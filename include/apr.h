@@ -120,7 +120,10 @@ apr_status apr_pregate_route(const void* h, const void* Wr, int dtype, int T, in
  * partial logits, so T*E must not exceed 2,097,088, else the call returns
  * APR_ERR_UNSUPPORTED with nothing enqueued.  The first call on a device
  * looks the array up on that device (cudaGetSymbolAddress); make that first
- * call before any stream capture.  Every call uses the same array and leaves
+ * call before any stream capture.  The address is kept for the life of the
+ * process: after cudaDeviceReset (or a primary context that is released and
+ * created again) the array moves, and this entry point must not be used on
+ * that device again without restarting the process.  Every call uses the same array and leaves
  * its contents behind, so calls that overlap on the GPU (for example on two
  * streams with no ordering between them) race with each other.  Nothing is
  * allocated or freed.  A token whose logits are all NaN gets adapter 0; there

@@ -191,3 +191,56 @@ def test_workspace_init_host_validation(apr):
     assert apr._workspace_init(None, 1 << 20, None) == apr.APR_ERR_WORKSPACE
     assert apr._workspace_init(0x100000, 8, None) == apr.APR_ERR_WORKSPACE
     assert apr._workspace_init(0x100040, 1 << 20, None) == apr.APR_ERR_WORKSPACE
+
+
+def test_binding_rejects_mismatched_tensors(apr):
+    """The Python binding checks dtypes, shapes and contiguity before a pointer crosses the ABI
+    (a bf16 router weight under an fp32 router input would otherwise be read at twice its size)."""
+    import torch
+    f32, bf16, i32 = torch.float32, torch.bfloat16, torch.int32
+    T, d, E, k = 4, 64, 8, 2
+    h = torch.zeros((T, d), dtype=f32)
+    idx = torch.zeros((T, k), dtype=i32)
+    gate = torch.zeros((T, k), dtype=f32)
+    ws = torch.zeros(1 << 20, dtype=torch.uint8)
+    with pytest.raises(TypeError, match="Wr has dtype"):
+        apr.pregate_route(h, torch.zeros((E, d), dtype=bf16), k, idx, gate, ws)
+    with pytest.raises(ValueError, match="columns"):
+        apr.pregate_route(h, torch.zeros((E, d + 8), dtype=f32), k, idx, gate, ws)
+    with pytest.raises(TypeError, match="idx has dtype"):
+        apr.pregate_route_noalloc(h, torch.zeros((E, d), dtype=f32), k, idx.long(), gate)
+    with pytest.raises(ValueError, match="gate has shape"):
+        apr.pregate_route(h, torch.zeros((E, d), dtype=f32), k, idx, gate[:, :1], ws)
+    with pytest.raises(TypeError, match="h has dtype"):
+        apr.pregate_route(h.double(), torch.zeros((E, d), dtype=torch.float64), k, idx, gate, ws)
+    with pytest.raises(ValueError, match="contiguous"):
+        apr.pregate_route(torch.zeros((d, T), dtype=f32).t(), torch.zeros((E, T), dtype=f32), k,
+                          idx, gate, ws)
+    with pytest.raises(ValueError, match="CUDA tensor"):          # everything right but the device
+        apr.pregate_route(h, torch.zeros((E, d), dtype=f32), k, idx, gate, ws)
+    with pytest.raises(ValueError, match="seg_off has shape"):
+        apr.segment_tokens(idx, E, torch.zeros(E, dtype=i32), torch.zeros(T * k, dtype=i32), ws)
+    with pytest.raises(ValueError, match="perm has"):
+        apr.segment_tokens(idx, E, torch.zeros(E + 1, dtype=i32), torch.zeros(T * k - 1, dtype=i32), ws)
+    # SGMM: projections must match x's dtype and rows
+    tabs = torch.zeros(E, dtype=torch.int64)
+    with pytest.raises(TypeError, match="y has dtype"):
+        apr.make_proj(torch.zeros((T, 16), dtype=f32), torch.zeros((T, 16), dtype=bf16), tabs, tabs)
+    with pytest.raises(ValueError, match="B_table has shape"):
+        apr.make_proj(torch.zeros((T, 16), dtype=f32), torch.zeros((T, 16), dtype=f32), tabs, tabs[:3])
+    yb = torch.zeros((T, 16), dtype=bf16)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        apr.make_proj(yb, yb, tabs, tabs)
+    p = apr.Proj(0, 0, 16, 0, 0)
+    p.meta = (bf16, T, E, torch.device("cpu"))
+    x = torch.zeros((T, 64), dtype=f32)
+    args = (k, E, torch.zeros(E, dtype=i32), 16, idx, gate, torch.zeros(E + 1, dtype=i32),
+            torch.zeros(T * k, dtype=i32), ws)
+    with pytest.raises(ValueError, match="does not fit"):
+        apr.sgmm_shrink_expand(x, [p], *args)
+    with pytest.raises(TypeError, match="not made by make_proj"):
+        apr.sgmm_shrink_expand(x, [apr.Proj(0, 0, 16, 0, 0)], *args)
+    with pytest.raises(TypeError, match="W has dtype"):
+        apr.gemv(torch.zeros((8, 8), dtype=f32), torch.zeros(8, dtype=bf16), torch.zeros(8, dtype=bf16))
+    with pytest.raises(ValueError, match="x has shape"):
+        apr.gemv(torch.zeros((8, 16), dtype=bf16), torch.zeros(8, dtype=bf16), torch.zeros(8, dtype=bf16))

@@ -31,6 +31,7 @@ SGMM_AUTO = 0
 SGMM_SKINNY = 1
 SGMM_TENSOR = 2
 SGMM_DENSE = 3
+SGMM_BANK = 4
 
 MAX_E = 1024
 MAX_K = 8

@@ -177,7 +177,7 @@ apr_status apr_sgmm_shrink_expand(const void* x, int d_in, const apr_proj* projs
   if (d_in < 8 || (d_in & 7)) return fail(APR_ERR_INVALID_ARG, "sgmm: d_in=%d must be a positive multiple of 8", d_in);
   if (max_rank < 8 || max_rank > APR_MAX_RANK || (max_rank & 7))
     return fail(APR_ERR_INVALID_ARG, "sgmm: max_rank=%d must be a multiple of 8 in [8, %d]", max_rank, APR_MAX_RANK);
-  if (kernel < APR_SGMM_AUTO || kernel > APR_SGMM_DENSE) return fail(APR_ERR_INVALID_ARG, "sgmm: bad kernel %d", kernel);
+  if (kernel < APR_SGMM_AUTO || kernel > APR_SGMM_BANK) return fail(APR_ERR_INVALID_ARG, "sgmm: bad kernel %d", kernel);
   for (int p = 0; p < nproj; ++p) {
     const apr_proj& pj = projs[p];
     if (pj.d_out < 8 || (pj.d_out & 7)) return fail(APR_ERR_INVALID_ARG, "sgmm: proj %d d_out=%d must be a positive multiple of 8", p, pj.d_out);
@@ -219,6 +219,7 @@ apr_status apr_sgmm_shrink_expand(const void* x, int d_in, const apr_proj* projs
     // by the shapes and the mean pairs per adapter, known on the host without reading the routing
     const double mean_seg = (double)T * k / E;
     if (sgmm_dense_supported(a, dtype)) use = APR_SGMM_DENSE;
+    else if (sgmm_bank_supported(a, dtype)) use = APR_SGMM_BANK;
     else if ((mean_seg >= 256.0 || (long)T * k >= 2048) && sgmm_tensor_supported(a, dtype)) use = APR_SGMM_TENSOR;
     else use = APR_SGMM_SKINNY;
   }
@@ -227,6 +228,11 @@ apr_status apr_sgmm_shrink_expand(const void* x, int d_in, const apr_proj* projs
     if (!sgmm_dense_supported(a, dtype))
       return fail(APR_ERR_UNSUPPORTED, "sgmm: dense kernel needs bf16, T<=64, E<=16, E*round16(max_rank)<=256");
     e = launch_sgmm_dense(a, L.scratch, (cudaStream_t)stream);
+  } else if (use == APR_SGMM_BANK) {
+    if (!sgmm_bank_supported(a, dtype))
+      return fail(APR_ERR_UNSUPPORTED, "sgmm: bank kernel needs bf16, rank slots of 16/32/64, k<=4, k*R16<=64, "
+                                       "E*R16<=256, d_in%%64==0");
+    e = launch_sgmm_bank(a, L.scratch, (cudaStream_t)stream);
   } else if (use == APR_SGMM_TENSOR) {
     if (!sgmm_tensor_supported(a, dtype))
       return fail(APR_ERR_UNSUPPORTED, "sgmm: tensor-core kernel needs bf16, k<=2, max_rank<=64, d_in%%64==0, d_out%%16==0");

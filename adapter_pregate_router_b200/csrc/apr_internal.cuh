@@ -117,6 +117,18 @@ inline size_t tc_scratch_bytes(int T, int k, int max_rank) {
   return (size_t)APR_MAX_PROJ * T * k * 4 * R16;
 }
 
+// Bank path (token order over the whole adapter bank): gated v per pair
+// [projection][pair q][R16] bf16; R16 in {16, 32, 64}, k <= 4, k * R16 <= 64,
+// E * R16 <= 256.
+constexpr int kBankMaxKR = 64;
+constexpr int kBankMaxRows = 256;
+inline size_t bank_scratch_bytes(int T, int k, int E, int max_rank) {
+  const int R16 = round16i(max_rank);
+  if (R16 != 16 && R16 != 32 && R16 != 64) return 0;
+  if (k < 1 || k > 4 || k * R16 > kBankMaxKR || E * R16 > kBankMaxRows) return 0;
+  return (size_t)APR_MAX_PROJ * T * k * R16 * 2;
+}
+
 // Shrink partial sums.  Gather paths: [projection][column chunk][sorted pair][rank]
 // fp32; dense path: [projection][cluster][token (padded to 16)][adapter * rank slot].
 inline size_t sgmm_scratch_bytes(int T, int k, int E, int max_rank, int d_in) {
@@ -128,6 +140,8 @@ inline size_t sgmm_scratch_bytes(int T, int k, int E, int max_rank, int d_in) {
   }
   const size_t t = tc_scratch_bytes(T, k, max_rank);
   if (t > b) b = t;
+  const size_t bk = bank_scratch_bytes(T, k, E, max_rank);
+  if (bk > b) b = bk;
   return b;
 }
 
@@ -296,6 +310,8 @@ struct SgmmArgs {
 cudaError_t launch_sgmm_skinny(const SgmmArgs& a, int dtype, size_t scratch_off, cudaStream_t s);
 cudaError_t launch_sgmm_tensor(const SgmmArgs& a, size_t scratch_off, cudaStream_t s);
 cudaError_t launch_sgmm_dense(const SgmmArgs& a, size_t scratch_off, cudaStream_t s);
+cudaError_t launch_sgmm_bank(const SgmmArgs& a, size_t scratch_off, cudaStream_t s);
+bool sgmm_bank_supported(const SgmmArgs& a, int dtype);
 bool sgmm_dense_supported(const SgmmArgs& a, int dtype);
 bool sgmm_tensor_supported(const SgmmArgs& a, int dtype);
 cudaError_t launch_merge(const apr_merge_proj* projs, int nproj, int E, int r, const int32_t* idx,

@@ -16,9 +16,15 @@
 //   mixed tiles    runs of <= 128 consecutive plan tokens whose adapters
 //                  number <= 4 (tensor-core expand, k <= 2), built by one
 //                  thread walking the set tiles in order
-// The histograms use shared-memory atomics (order-free counts); every order-
-// dependent step runs in one warp, 32 elements at a time, with __match_any_sync
-// ranking equal keys by lane, so the result is unique.
+// The histograms use shared-memory atomics (order-free counts).  The order-
+// dependent steps (the stable scatters of the pairs and of the tokens, the set
+// tiles) run over blocks of 1024 consecutive items, all 32 warps at once: a
+// warp ranks equal keys by lane with __match_any_sync, the per-key counts of
+// the 32 warps are scanned across warps in shared memory, and a per-key base
+// carries from one block to the next, so the result is unique.  idx and the
+// token order are staged in shared memory when they fit.
+#include <climits>
+
 #include "apr_internal.cuh"
 
 namespace apr {
@@ -60,6 +66,64 @@ __device__ int block_exclusive_scan(int v, int* warp_sums, int* total) {
   return before;
 }
 
+// Inclusive max over the block (one value per thread).
+__device__ int block_inclusive_max(int v, int* warp_vals) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nwarps = blockDim.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, off);
+    if (lane >= off) x = max(x, y);
+  }
+  if (lane == 31) warp_vals[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int s = lane < nwarps ? warp_vals[lane] : INT_MIN;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, s, off);
+      if (lane >= off) s = max(s, y);
+    }
+    warp_vals[lane] = s;
+  }
+  __syncthreads();
+  const int r = warp > 0 ? max(warp_vals[warp - 1], x) : x;
+  __syncthreads();
+  return r;
+}
+
+// Stable rank of one block of up to 1024 items (thread i holds item i of the
+// block, key in [0, E) when valid): returns base[key] + the number of earlier
+// items of this block with the same key, and advances base[key] by the block's
+// count of that key.  cnt is a [32][E] table of zeros on entry and on exit.
+__device__ int block_stable_rank(int key, bool valid, int E, int* base, uint16_t* cnt) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const unsigned peers = __match_any_sync(0xffffffffu, valid ? key : -1);
+  const int intra = __popc(peers & lanemask_lt());
+  if (valid && lane == __ffs(peers) - 1) cnt[warp * E + key] = (uint16_t)__popc(peers);
+  __syncthreads();
+  int run = 0;
+  if (tid < E) {                           // this key's count in each warp -> exclusive prefix over warps
+#pragma unroll 8
+    for (int w = 0; w < 32; ++w) {
+      const int c = cnt[w * E + tid];
+      cnt[w * E + tid] = (uint16_t)run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  const int pos = valid ? base[key] + cnt[warp * E + key] + intra : -1;
+  __syncthreads();
+  if (tid < E) {
+    base[tid] += run;
+#pragma unroll 8
+    for (int w = 0; w < 32; ++w) cnt[w * E + tid] = 0;
+  }
+  __syncthreads();
+  return pos;
+}
+
 // The p-th smallest adapter of token t (its tuple sorted ascending).
 __device__ __forceinline__ int sorted_key(const int32_t* idx, int t, int k, int p) {
   if (k == 1) return idx[t];
@@ -94,19 +158,29 @@ __device__ __forceinline__ bool same_set(const int32_t* idx, int t0, int t1, int
   return true;
 }
 
-__global__ void __launch_bounds__(SEG_THREADS) segment_kernel(const int32_t* __restrict__ idx, int T,
+// Dynamic shared memory: hist [E], base [E] (int), cnt [32][E] (uint16), and
+// with STAGE idx [T*k], two token arrays [T] (int).
+__host__ __device__ inline size_t seg_smem_fixed(int E) {
+  return (sizeof(int) * 2 * (size_t)E + sizeof(uint16_t) * 32 * (size_t)E + 15) / 16 * 16;
+}
+__host__ __device__ inline size_t seg_smem_stage(int T, int k) { return sizeof(int) * ((size_t)T * k + 2 * (size_t)T); }
+
+template <bool STAGE>
+__global__ void __launch_bounds__(SEG_THREADS) segment_kernel(const int32_t* __restrict__ idx_g, int T,
                                                               int k, int E,
                                                               int32_t* __restrict__ seg_off,
                                                               int32_t* __restrict__ perm, void* ws) {
   pdl_wait();
   pdl_trigger();
-  extern __shared__ int sm[];
-  int* hist = sm;          // [E]
-  int* base = sm + E;      // [E]
+  extern __shared__ __align__(16) unsigned char seg_smem[];
+  int* hist = reinterpret_cast<int*>(seg_smem);                   // [E]
+  int* base = hist + E;                                           // [E]
+  uint16_t* cnt = reinterpret_cast<uint16_t*>(base + E);          // [32][E]
+  int* stage = reinterpret_cast<int*>(seg_smem + seg_smem_fixed(E));
   __shared__ int warp_sums[32];
   __shared__ int bad;
   __shared__ int carry[2];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x;
   const int n = T * k;
   const WsLayout L = ws_layout(T, k, E);
   WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
@@ -115,7 +189,14 @@ __global__ void __launch_bounds__(SEG_THREADS) segment_kernel(const int32_t* __r
   int* tok_tmp = ws_at<int>(ws, L.tok_tmp);
   PairTile* ptiles = ws_at<PairTile>(ws, L.ptiles);
   SetTile* stiles = ws_at<SetTile>(ws, L.stiles);
+  const int32_t* idx = STAGE ? stage : idx_g;
+  int* tok_a = STAGE ? stage + n : tok_tmp;
+  int* tok_b = STAGE ? stage + n + T : tok_order;
 
+  // 0. zero the rank table, stage idx
+  for (int i = tid; i < 32 * E; i += SEG_THREADS) cnt[i] = 0;
+  if (STAGE)
+    for (int q = tid; q < n; q += SEG_THREADS) stage[q] = idx_g[q];
   // 1. counts and validation
   for (int e = tid; e < E; e += SEG_THREADS) hist[e] = 0;
   if (tid == 0) bad = 0;
@@ -136,6 +217,7 @@ __global__ void __launch_bounds__(SEG_THREADS) segment_kernel(const int32_t* __r
       hdr->n_ptiles = 0;
       hdr->n_stiles = 0;
       hdr->n_qtiles = 0;
+      hdr->n_mtiles = 0;
     }
     return;
   }
@@ -198,27 +280,19 @@ __global__ void __launch_bounds__(SEG_THREADS) segment_kernel(const int32_t* __r
     if (tid == 0) hdr->n_qtiles = ntiles;
   }
   __syncthreads();
-  // 4. stable scatter of the pairs (one warp, in order)
-  if (warp == 0) {
-    for (int q0 = 0; q0 < n; q0 += 32) {
-      const int q = q0 + lane;
-      const bool valid = q < n;
-      const int e = valid ? idx[q] : -1 - lane;
-      const unsigned peers = __match_any_sync(0xffffffffu, e);
-      if (valid) {
-        const int pos = base[e] + __popc(peers & lanemask_lt());
-        perm[pos] = q;
-        inv[q] = pos;
-      }
-      __syncwarp();
-      if (valid && lane == __ffs(peers) - 1) base[e] += __popc(peers);
-      __syncwarp();
+  // 4. stable scatter of the pairs, 1024 at a time
+  for (int q0 = 0; q0 < n; q0 += SEG_THREADS) {
+    const int q = q0 + tid;
+    const bool valid = q < n;
+    const int pos = block_stable_rank(valid ? idx[q] : 0, valid, E, base, cnt);
+    if (valid) {
+      perm[pos] = q;
+      inv[q] = pos;
     }
   }
-  __syncthreads();
   // 5. tokens ordered by sorted adapter tuple: LSD, k stable counting sorts
-  int* src = tok_tmp;
-  int* dst = tok_order;
+  int* src = tok_a;
+  int* dst = tok_b;
   for (int i = tid; i < T; i += SEG_THREADS) src[i] = i;
   for (int p = k - 1; p >= 0; --p) {
     for (int e = tid; e < E; e += SEG_THREADS) hist[e] = 0;
@@ -232,62 +306,51 @@ __global__ void __launch_bounds__(SEG_THREADS) segment_kernel(const int32_t* __r
       if (tid < E) base[tid] = off;
     }
     __syncthreads();
-    if (warp == 0) {
-      for (int i0 = 0; i0 < T; i0 += 32) {
-        const int i = i0 + lane;
-        const bool valid = i < T;
-        const int t = valid ? src[i] : 0;
-        const int key = valid ? sorted_key(idx, t, k, p) : -1 - lane;
-        const unsigned peers = __match_any_sync(0xffffffffu, key);
-        if (valid) dst[base[key] + __popc(peers & lanemask_lt())] = t;
-        __syncwarp();
-        if (valid && lane == __ffs(peers) - 1) base[key] += __popc(peers);
-        __syncwarp();
-      }
+    for (int i0 = 0; i0 < T; i0 += SEG_THREADS) {
+      const int i = i0 + tid;
+      const bool valid = i < T;
+      const int t = valid ? src[i] : 0;
+      const int pos = block_stable_rank(valid ? sorted_key(idx, t, k, p) : 0, valid, E, base, cnt);
+      if (valid) dst[pos] = t;
     }
-    __syncthreads();
     int* tmp = src;
     src = dst;
     dst = tmp;
   }
-  // src holds the final order
+  // src holds the final order; the plan keeps it in tok_order
   if (src != tok_order) {
     for (int i = tid; i < T; i += SEG_THREADS) tok_order[i] = src[i];
-    __syncthreads();
   }
-  // 6. set tiles: split runs of equal adapter sets into <= kSetTile tokens
-  if (warp == 0) {
-    if (lane == 0) {
-      carry[0] = 0;  // start of the current run
-      carry[1] = 0;  // tiles written
-    }
-    __syncwarp();
-    for (int i0 = 0; i0 < T; i0 += 32) {
-      const int i = i0 + lane;
-      const bool valid = i < T;
-      bool head = false;
-      if (valid) head = (i == 0) || !same_set(idx, tok_order[i - 1], tok_order[i], k);
-      const unsigned heads = __ballot_sync(0xffffffffu, head);
-      const unsigned upto = heads & (lanemask_lt() | (1u << lane));
-      const int run_start = upto ? i0 + (31 - __clz(upto)) : carry[0];
-      const bool tstart = valid && (head || ((i - run_start) % kSetTile) == 0);
-      const unsigned starts = __ballot_sync(0xffffffffu, tstart);
-      const int wbase = carry[1];
-      if (tstart) {
-        SetTile st;
-        st.start = i;
-        st.len = 0;
-        stiles[wbase + __popc(starts & lanemask_lt())] = st;
-      }
-      __syncwarp();
-      if (lane == 31) {
-        carry[0] = run_start;
-        carry[1] = wbase + __popc(starts);
-      }
-      __syncwarp();
-    }
+  const int* order = src;
+  __syncthreads();
+  // 6. set tiles: runs of equal adapter sets, split into <= kSetTile tokens.  A run starts
+  //    where the set changes; a tile starts at a run start or every kSetTile tokens into a run.
+  if (tid == 0) {
+    carry[0] = 0;  // start of the current run
+    carry[1] = 0;  // tiles written
   }
   __syncthreads();
+  for (int i0 = 0; i0 < T; i0 += SEG_THREADS) {
+    const int i = i0 + tid;
+    const bool valid = i < T;
+    const bool head = valid && (i == 0 || !same_set(idx, order[i - 1], order[i], k));
+    const int rs = max(block_inclusive_max(head ? i : -1, warp_sums), carry[0]);
+    const bool tstart = valid && (head || ((i - rs) % kSetTile) == 0);
+    int ntot;
+    const int off = block_exclusive_scan(tstart ? 1 : 0, warp_sums, &ntot);
+    if (tstart) {
+      SetTile st;
+      st.start = i;
+      st.len = 0;
+      stiles[carry[1] + off] = st;
+    }
+    __syncthreads();
+    if (tid == SEG_THREADS - 1) {
+      carry[0] = rs;
+      carry[1] += ntot;
+    }
+    __syncthreads();
+  }
   const int nst = carry[1];
   for (int j = tid; j < nst; j += SEG_THREADS) {
     const int end = (j + 1 < nst) ? stiles[j + 1].start : T;
@@ -317,7 +380,7 @@ __global__ void __launch_bounds__(SEG_THREADS) segment_kernel(const int32_t* __r
       __syncthreads();
       for (int j = tid; j < MIX_CHUNK && c0 + j < nst; j += SEG_THREADS) {
         const SetTile st = stiles[c0 + j];
-        const int t0 = tok_order[st.start];
+        const int t0 = order[st.start];
         const int a0 = sorted_key(idx, t0, k, 0);
         const int a1 = k == 2 ? sorted_key(idx, t0, k, 1) : -1;
         s_st[j] = make_int4(st.start, st.len, a0, a1);
@@ -375,9 +438,20 @@ __global__ void __launch_bounds__(SEG_THREADS) segment_kernel(const int32_t* __r
 
 cudaError_t launch_segment(const int32_t* idx, int T, int k, int E, int32_t* seg_off,
                            int32_t* perm, void* ws, cudaStream_t s) {
-  const size_t smem = sizeof(int) * 2 * (size_t)E;
-  return launch_pdl(segment_kernel, dim3(1), dim3(SEG_THREADS), smem, s, idx, T, k, E, seg_off,
-                    perm, ws);
+  // idx and the token arrays go to shared memory when they fit beside the fixed tables and the
+  // mixed-tile staging (static, 16 KB)
+  constexpr size_t kStageBudget = 200 * 1024;
+  const size_t fixed = seg_smem_fixed(E);
+  const bool stage = fixed + seg_smem_stage(T, k) <= kStageBudget;
+  const size_t smem = fixed + (stage ? seg_smem_stage(T, k) : 0);
+  static SmemLimit lim[2];
+  cudaError_t err;
+  if (stage) {
+    if (smem > 48 * 1024 && (err = lim[1].ensure((const void*)segment_kernel<true>, smem)) != cudaSuccess) return err;
+    return launch_pdl(segment_kernel<true>, dim3(1), dim3(SEG_THREADS), smem, s, idx, T, k, E, seg_off, perm, ws);
+  }
+  if (smem > 48 * 1024 && (err = lim[0].ensure((const void*)segment_kernel<false>, smem)) != cudaSuccess) return err;
+  return launch_pdl(segment_kernel<false>, dim3(1), dim3(SEG_THREADS), smem, s, idx, T, k, E, seg_off, perm, ws);
 }
 
 }  // namespace apr

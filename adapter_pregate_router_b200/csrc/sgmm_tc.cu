@@ -65,7 +65,9 @@ struct TcPlan {
   int ny;                            // expand ring depth
   int mixed;                         // expand over mixed tiles (<= 4 adapters, K2 = 4 * R16) instead of set tiles
   int ytma;                          // expand stores y rows with tile::scatter4 (else plain stores)
-  size_t vprep_off;                  // scratch: V rows [proj][pair position][2 * R16] bf16
+  int vpair;                         // shrink writes v by pair id, bf16 only ([proj][q][R16]) instead of
+                                     // by plan position as bf16 hi | lo ([proj][pair position][2 * R16])
+  size_t vprep_off;                  // scratch: V rows
   int cc_before[APR_MAX_PROJ + 1];   // expand: prefix of 1024-column items per projection
 };
 
@@ -83,7 +85,7 @@ __host__ __device__ inline ShSmem sh_smem(int n1max, int stages) {
   L.stages = stages;
   L.bar = (size_t)stages * L.stage_bytes;
   L.meta = L.bar + (size_t)(2 * stages + 1) * 8;
-  L.total = L.meta + 2 * TB_M * 4 + 16 + TB_MAXN1 * 8 + 1024;
+  L.total = L.meta + 3 * TB_M * 4 + 16 + TB_MAXN1 * 8 + 1024;
   return L;
 }
 
@@ -102,6 +104,7 @@ __global__ void __launch_bounds__(SH_BLOCK, 1) tc_shrink_kernel(const __grid_con
   float* s_g = reinterpret_cast<float*>(s_tok + TB_M);
   volatile int* s_flags = reinterpret_cast<volatile int*>(s_g + TB_M);      // [0] tmem [1] bad
   const __nv_bfloat16** s_arow = reinterpret_cast<const __nv_bfloat16**>(smem + L.meta + 2 * TB_M * 4 + 16);
+  int* s_pair = reinterpret_cast<int*>(smem + L.meta + 2 * TB_M * 4 + 16 + TB_MAXN1 * 8);
   const uint32_t sbase = smem_u32(smem);
 
   if (tid == 0) {
@@ -144,14 +147,15 @@ __global__ void __launch_bounds__(SH_BLOCK, 1) tc_shrink_kernel(const __grid_con
     const int N1 = nq * R16;
     const int e = tile.e;
     if (tid < TB_M) {
-      int tok = -1;
+      int tok = -1, q = -1;
       float g = 0.f;
       if (tid < tile.len) {
-        const int q = a.perm[tile.start + tid];
+        q = a.perm[tile.start + tid];
         tok = q / K;
         g = a.gate[q];
       }
       s_tok[tid] = tok;
+      s_pair[tid] = q;
       s_g[tid] = g;
       if (tid == 0) {
         const int r = (e >= 0 && e < a.E) ? a.ranks[e] : 0;
@@ -230,7 +234,11 @@ __global__ void __launch_bounds__(SH_BLOCK, 1) tc_shrink_kernel(const __grid_con
             hi[i] = *reinterpret_cast<const uint32_t*>(&h);
             lo[i] = pack_bf16x2(a0 - hf.x, a1 - hf.y);
           }
-          if (valid) {
+          if (valid && P.vpair) {
+            __nv_bfloat16* dst = vprep + ((size_t)(q0 + qi) * npairs + s_pair[row]) * R16 + rr;
+            reinterpret_cast<uint4*>(dst)[0] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+            reinterpret_cast<uint4*>(dst)[1] = make_uint4(hi[4], hi[5], hi[6], hi[7]);
+          } else if (valid) {
             __nv_bfloat16* dst = vprep + ((size_t)(q0 + qi) * npairs + tile.start + row) * (2 * R16) + rr;
             reinterpret_cast<uint4*>(dst)[0] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
             reinterpret_cast<uint4*>(dst)[1] = make_uint4(hi[4], hi[5], hi[6], hi[7]);
@@ -643,38 +651,61 @@ bool sgmm_tensor_supported(const SgmmArgs& a, int dtype) {
   return true;
 }
 
-cudaError_t launch_sgmm_tensor(const SgmmArgs& a, size_t scratch_off, cudaStream_t s) {
-  TcPlan t;
-  memset(&t, 0, sizeof(t));
+// Shrink plan fields shared by both expands: projections per item, pipeline depth.
+static void shrink_plan(TcPlan& t, const SgmmArgs& a, size_t v_off, int vpair) {
   t.a = a;
   t.R16 = round16i(a.max_rank);
-  t.mixed = (a.k <= 2 && kMixAdapters * t.R16 <= TB_MAXK2) ? 1 : 0;
-  t.K2 = (t.mixed ? kMixAdapters : a.k) * t.R16;
   t.pg = TB_MAXN1 / t.R16;
   if (t.pg > a.nproj) t.pg = a.nproj;
   t.npg = (a.nproj + t.pg - 1) / t.pg;
   const int n1max = t.pg * t.R16;
   t.stages = (int)((SMEM_BUDGET - 4096) / (TB_M * 128 + n1max * 128));
   if (t.stages > 8) t.stages = 8;
+  t.vprep_off = v_off;
+  t.vpair = vpair;
+}
+
+static cudaError_t launch_shrink(const TcPlan& t, cudaStream_t s) {
+  const SgmmArgs& a = t.a;
+  const size_t sm1 = sh_smem(t.pg * t.R16, t.stages).total;
+  static SmemLimit lim;
+  cudaError_t err;
+  if ((err = lim.ensure((const void*)tc_shrink_kernel, sm1)) != cudaSuccess) return err;
+  const int nsm = device_sm_count();
+  // tile counts are bounded by the plan's maxima; the kernel loops over the real ones
+  const long max_q = max_qtiles(a.T, a.k, a.E);
+  const int g1 = (int)(max_q * t.npg < nsm ? max_q * t.npg : nsm);
+  return launch_pdl(tc_shrink_kernel, dim3(g1), dim3(SH_BLOCK), sm1, s, t);
+}
+
+cudaError_t launch_tc_shrink_pairs(const SgmmArgs& a, size_t v_off, cudaStream_t s) {
+  TcPlan t;
+  memset(&t, 0, sizeof(t));
+  shrink_plan(t, a, v_off, 1);
+  return launch_shrink(t, s);
+}
+
+cudaError_t launch_sgmm_tensor(const SgmmArgs& a, size_t scratch_off, cudaStream_t s) {
+  TcPlan t;
+  memset(&t, 0, sizeof(t));
+  shrink_plan(t, a, scratch_off, 0);
+  t.mixed = (a.k <= 2 && kMixAdapters * t.R16 <= TB_MAXK2) ? 1 : 0;
+  t.K2 = (t.mixed ? kMixAdapters : a.k) * t.R16;
   t.ny = t.K2 <= 32 ? 4 : 3;
-  t.vprep_off = scratch_off;
   t.ytma = 1;
   for (int p = 0; p < a.nproj && t.ytma; ++p)
     t.ytma = encode_row_map(&t.ymap[p], a.proj[p].y, a.T, a.proj[p].d_out) == cudaSuccess;
   t.cc_before[0] = 0;
   for (int p = 0; p < a.nproj; ++p) t.cc_before[p + 1] = t.cc_before[p] + (a.proj[p].d_out + TB_CW - 1) / TB_CW;
 
-  const size_t sm1 = sh_smem(n1max, t.stages).total, sm2 = ex_smem(t.K2, t.ny).total;
-  static SmemLimit lim1, lim2;
+  const size_t sm2 = ex_smem(t.K2, t.ny).total;
+  static SmemLimit lim2;
   cudaError_t err;
-  if ((err = lim1.ensure((const void*)tc_shrink_kernel, sm1)) != cudaSuccess) return err;
   if ((err = lim2.ensure((const void*)tc_expand_kernel, sm2)) != cudaSuccess) return err;
   const int nsm = device_sm_count();
-  // tile counts are bounded by the plan's maxima; the kernels loop over the real ones
-  const long max_q = max_qtiles(a.T, a.k, a.E), max_s = (long)a.T + (a.T + TB_M - 1) / TB_M;
-  const int g1 = (int)(max_q * t.npg < nsm ? max_q * t.npg : nsm);
+  const long max_s = (long)a.T + (a.T + TB_M - 1) / TB_M;
   const int g2 = (int)(max_s * t.cc_before[a.nproj] < nsm ? max_s * t.cc_before[a.nproj] : nsm);
-  if ((err = launch_pdl(tc_shrink_kernel, dim3(g1), dim3(SH_BLOCK), sm1, s, t)) != cudaSuccess) return err;
+  if ((err = launch_shrink(t, s)) != cudaSuccess) return err;
   return launch_pdl(tc_expand_kernel, dim3(g2), dim3(EX_BLOCK), sm2, s, t);
 }
 

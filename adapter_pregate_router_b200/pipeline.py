@@ -83,7 +83,10 @@ class Step:
         h.copy_(self.h)
         self.h = h
         pos_out = 0
+        self.layer_in = {}       # l -> (start, end) of the layer's inputs (x, y_base) in act_in
+        self.layer_out = {}      # l -> (start, end) of the layer's outputs in act_out
         for l in self.layers:
+            in0, out0 = pos_in[0], pos_out
             for g in cfg.groups:
                 x = take_in((T, g.d_in))
                 x.copy_(W.device_tensor(cfg, W.x_key(l, g.name), (T, g.d_in), dev))
@@ -109,6 +112,8 @@ class Step:
                     self.adapters[(l, g.name, p)] = (A, B)
                     self.keep += [At, Bt]
                 self.calls.append((x, projs, (l, g.name)))
+            self.layer_in[l] = (in0, pos_in[0])
+            self.layer_out[l] = (out0, pos_out) if out_of_place else (in0, pos_in[0])
         W.clear_device_pools()
 
     # ------------------------------------------------------------ merge workload
@@ -117,7 +122,19 @@ class Step:
         entries = []
         self.weights = {}    # (l, g, p) -> (W, Wp, x, y)
         self.adapters = {}
+        # the token's activations: router hidden and every weight's GEMV input in one arena, every
+        # GEMV output in another (the weights themselves stay resident from token to token)
+        n_in = cfg.d_router + sum(g.d_in * len(g.d_outs) for g in cfg.groups) * len(self.layers)
+        n_out = sum(sum(g.d_outs) for g in cfg.groups) * len(self.layers)
+        self.act_in = torch.empty(n_in, dtype=dt, device=dev)
+        self.act_out = torch.empty(n_out, dtype=dt, device=dev)
+        h = self.act_in[:cfg.d_router].view(1, cfg.d_router)
+        h.copy_(self.h)
+        self.h = h
+        pos_in, pos_out = cfg.d_router, 0
+        self.layer_in, self.layer_out = {}, {}
         for l in self.layers:
+            in0, out0 = pos_in, pos_out
             for g in cfg.groups:
                 for p, d_out in zip(g.proj_names, g.d_outs):
                     Wt = W.device_tensor(cfg, W.w_key(l, g.name, p), (d_out, g.d_in), dev)
@@ -127,12 +144,17 @@ class Step:
                     B = [W.device_tensor(cfg, W.b_key(l, g.name, p, e), (d_out, int(self.ranks_np[e])), dev)
                          for e in range(cfg.E)]
                     At, Bt = apr.ptr_array(A, dev), apr.ptr_array(B, dev)
-                    x = W.device_tensor(cfg, W.xm_key(l, g.name, p), (g.d_in,), dev)
-                    y = torch.empty(d_out, dtype=dt, device=dev)
+                    x = self.act_in[pos_in:pos_in + g.d_in]
+                    x.copy_(W.device_tensor(cfg, W.xm_key(l, g.name, p), (g.d_in,), dev))
+                    pos_in += g.d_in
+                    y = self.act_out[pos_out:pos_out + d_out]
+                    pos_out += d_out
                     entries.append((Wt, Wp, At, Bt))
                     self.weights[(l, g.name, p)] = (Wt, Wp, x, y)
                     self.adapters[(l, g.name, p)] = (A, B)
                     self.keep += [At, Bt]
+            self.layer_in[l] = (in0, pos_in)
+            self.layer_out[l] = (out0, pos_out)
         self.merge_tab = apr.merge_table(entries, dev)
         self.nmerge = len(entries)
         # TMA descriptors of the weights: built once, reused by every token's merge
@@ -145,21 +167,35 @@ class Step:
         apr.pregate_route(self.h, self.Wr, cfg.k, self.idx, self.gate, self.ws, stream)
         apr.segment_tokens(self.idx, cfg.E, self.seg_off, self.perm, self.ws, stream)
 
-    def layers_only(self, stream=None):
+    def merge_all(self, stream=None):
+        """Merge workload: one launch merging the token's adapters into every weight."""
+        cfg = self.cfg
+        if self.merge_plan is not None:
+            apr.merge_adapters_planned(self.merge_tab, self.merge_plan, self.nmerge, cfg.E, self.max_rank,
+                                       self.idx, self.gate, cfg.k, self.ws, stream)
+        else:
+            apr.merge_adapters(self.merge_tab, self.nmerge, cfg.E, self.max_rank, self.idx, self.gate,
+                               cfg.k, self.ws, stream)
+
+    def run_layer(self, l, stream=None):
+        """The calls of one layer: its SGMM calls, or (merge workload) its GEMVs on the merged
+        weights, which ``merge_all`` must have written first."""
         cfg = self.cfg
         if cfg.merge:
-            if self.merge_plan is not None:
-                apr.merge_adapters_planned(self.merge_tab, self.merge_plan, self.nmerge, cfg.E, self.max_rank,
-                                           self.idx, self.gate, cfg.k, self.ws, stream)
-            else:
-                apr.merge_adapters(self.merge_tab, self.nmerge, cfg.E, self.max_rank, self.idx, self.gate,
-                                   cfg.k, self.ws, stream)
-            for (Wt, Wp, x, y) in self.weights.values():
-                apr.gemv(Wp, x, y, stream)
+            for (ll, _, _), (Wt, Wp, x, y) in self.weights.items():
+                if ll == l:
+                    apr.gemv(Wp, x, y, stream)
             return
-        for x, projs, _ in self.calls:
-            apr.sgmm_shrink_expand(x, projs, cfg.k, cfg.E, self.ranks, self.max_rank, self.idx,
-                                   self.gate, self.seg_off, self.perm, self.ws, self.kernel, stream)
+        for x, projs, (ll, _) in self.calls:
+            if ll == l:
+                apr.sgmm_shrink_expand(x, projs, cfg.k, cfg.E, self.ranks, self.max_rank, self.idx,
+                                       self.gate, self.seg_off, self.perm, self.ws, self.kernel, stream)
+
+    def layers_only(self, stream=None):
+        if self.cfg.merge:
+            self.merge_all(stream)
+        for l in self.layers:
+            self.run_layer(l, stream)
 
     def run(self, stream=None):
         self.route(stream)

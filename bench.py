@@ -3,11 +3,15 @@
 A step is one pass of the whole path over one batch of synthetic tokens:
 router + top-k + gates (once), segments (once), then the SGMM shrink/expand
 fused into the base-output add for every (layer, shared-input group) of the
-workload.  The default workload is ``decode`` (Llama-2-7B layer set, 32
-tokens, 8 rank-16 adapters, top-2).  The step is captured once in a CUDA graph
-and replayed.
+workload.  The headline workload is ``prefill`` (Llama-2-7B layer set, 8192
+tokens, 16 rank-16 adapters with Zipf(1.1) popularity, top-2); the other
+full-size workloads (decode, multitenant, merge) are timed in the same run and
+reported under ``workloads``.  Each step is captured once in a CUDA graph and
+replayed; ``e2e`` times the eager C-ABI calls with the step's activations
+copied in from and out to pinned host memory.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--also decode,multitenant,merge|none] [--impl reference]
 
 With N > 1 (torchrun, one process per GPU) every rank runs its own batch
 (weak scaling: tokens are independent and the path has no exchange step);
@@ -92,18 +96,50 @@ def kernel_source_hash():
     return h.hexdigest()[:16]
 
 
+TRAFFIC_FILE = os.path.join("profiles", "dram_traffic.json")
+
+
 def measured_traffic(workload):
-    """DRAM bytes per SGMM call from the committed ncu capture, or None when the kernels changed since."""
-    path = os.path.join(ROOT, "profiles", "dram_traffic.md")
+    """DRAM bytes per SGMM call from the committed ncu capture, or None when the kernels changed
+    since (the capture records the kernel-source hash it was taken on)."""
+    path = os.path.join(ROOT, TRAFFIC_FILE)
     if not os.path.exists(path):
         return None
-    want = kernel_source_hash()
     with open(path) as f:
-        for line in f:
-            parts = line.split()
-            if len(parts) == 4 and parts[0] == "traffic:" and parts[1] == workload and parts[3] == want:
-                return float(parts[2])
-    return None
+        d = json.load(f)
+    ent = d.get("workloads", {}).get(workload)
+    if not ent or ent.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return float(ent["bytes_per_call"])
+
+
+def ingest_traffic(csv_path, workload, calls, command):
+    """Record an ncu launch capture (``--metrics dram__bytes_read.sum,dram__bytes_write.sum``,
+    ``--csv``) as the DRAM bytes per SGMM call of ``workload``: the sum over the captured launches
+    divided by ``calls``, keyed to the current kernel-source hash."""
+    import csv
+    tot = 0.0
+    with open(csv_path) as f:
+        rows = [r for r in csv.reader(l for l in f if l.startswith('"'))]
+    head = rows[0]
+    im, iv, iu = head.index("Metric Name"), head.index("Metric Value"), head.index("Metric Unit")
+    scale = {"byte": 1.0, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}
+    for r in rows[1:]:
+        if r[im] in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
+            tot += float(r[iv].replace(",", "")) * scale.get(r[iu], 1.0)
+    path = os.path.join(ROOT, TRAFFIC_FILE)
+    d = {"note": "DRAM bytes per SGMM call from ncu launch captures (dram__bytes_read.sum + "
+                 "dram__bytes_write.sum over the captured launches / calls); written by bench.py --ingest-traffic",
+         "workloads": {}}
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+    d["workloads"][workload] = {"bytes_per_call": tot / calls, "calls": calls, "kernel_source_hash": kernel_source_hash(),
+                                "command": command}
+    with open(path, "w") as f:
+        json.dump(d, f, indent=1, sort_keys=True)
+        f.write("\n")
+    return tot / calls
 
 
 class ClockSampler:
@@ -207,13 +243,21 @@ def aggregate_throughput(units_per_rank, ms_local, world, device=None):
 # ---------------------------------------------------------------- CPU oracle leg
 
 
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
 class OracleSample:
     """The fp64 oracle on a bounded sample of one step of ``cfg``.
 
     Inputs of the first ``n_layers`` layers are prepared once, outside the
     clock; one pass times the route + segments over all tokens and those
     layers (every projection, every token), and the step time is scaled to
-    all layers.  BLAS is held to one thread, so ``cores`` is 1.
+    all layers.  BLAS may use ``threads`` threads (the oracle's per-token loop
+    itself is plain Python on one core).
     """
 
     def __init__(self, cfg, layer_budget_s):
@@ -265,10 +309,10 @@ class OracleSample:
                 O.sgmm_shrink_expand(x, A, B, idx, gate, yb)
         return time.perf_counter() - t0
 
-    def step_seconds(self):
+    def step_seconds(self, threads=1):
         from threadpoolctl import threadpool_limits
         O, cfg = self.O, self.cfg
-        with threadpool_limits(limits=1):
+        with threadpool_limits(limits=threads):
             t0 = time.perf_counter()
             idx, gate, _ = O.pregate_route(self.h, self.Wr, cfg.k)
             O.segment_tokens(idx, cfg.E)
@@ -276,25 +320,34 @@ class OracleSample:
             t_layers = sum(self._time_layer(items, idx, gate) for items in self.layers)
         return t_route + t_layers * cfg.layers / len(self.layers)
 
-    def describe(self):
+    def describe(self, threads):
         c = self.cfg
         return (f"route+segments over all {c.T} tokens plus {len(self.layers)} of {c.layers} layers "
-                f"(every projection and token) timed, scaled to {c.layers} layers; fp64 numpy oracle, 1 BLAS thread")
+                f"(every projection and token) timed, scaled to {c.layers} layers; fp64 numpy oracle, "
+                f"BLAS on {threads} thread(s), the per-token loop in one Python thread")
 
 
 def cpu_baseline(cfg, budget_s):
-    """Repeat oracle passes for about ``budget_s`` seconds of CPU work."""
-    smp = OracleSample(cfg, layer_budget_s=budget_s / 4)
-    times, spent = [], 0.0
-    while spent < budget_s or not times:
-        t = smp.step_seconds()
-        times.append(t)
-        spent += t * len(smp.layers) / cfg.layers + 1e-3
-        if len(times) >= 50:
-            break
-    step_s = float(np.median(times))
-    return {"value": cfg.T / step_s, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": smp.describe() + f"; median of {len(times)} passes"}
+    """Oracle passes for about ``budget_s`` seconds of CPU work, with BLAS on all host cores and,
+    beside it, on one thread."""
+    smp = OracleSample(cfg, layer_budget_s=budget_s / 6)
+    cores = host_cores()
+    out = {}
+    for threads in (cores, 1):
+        times, spent = [], 0.0
+        while spent < budget_s / 2 or not times:
+            t = smp.step_seconds(threads)
+            times.append(t)
+            spent += t * len(smp.layers) / cfg.layers + 1e-3
+            if len(times) >= 50:
+                break
+        out[threads] = (float(np.median(times)), len(times))
+    step_s, n = out[cores]
+    line = {"value": cfg.T / step_s, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": smp.describe(cores) + f"; median of {n} passes"}
+    s1, n1 = out[1]
+    line["single_thread"] = {"value": cfg.T / s1, "unit": "tokens/s", "cores": 1, "passes": n1}
+    return line
 
 
 def run_reference(args, world, rank):
@@ -305,9 +358,10 @@ def run_reference(args, world, rank):
     cfg = W.CONFIGS[args.workload]
     per_step_budget = min(args.ref_budget, 150.0 / (args.steps + args.warmup))
     smp = OracleSample(cfg, layer_budget_s=per_step_budget)
+    cores = host_cores()
     for _ in range(args.warmup):
-        smp.step_seconds()
-    per_step = [smp.step_seconds() for _ in range(args.steps)]
+        smp.step_seconds(cores)
+    per_step = [smp.step_seconds(cores) for _ in range(args.steps)]
     step_s = float(np.mean(per_step))
     value = cfg.T / step_s
     line = {
@@ -315,7 +369,8 @@ def run_reference(args, world, rank):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": config_block(cfg, world),
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": smp.describe()},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": smp.describe(cores)},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -335,19 +390,89 @@ def config_block(cfg, world):
 
 # ---------------------------------------------------------------- GPU leg
 
+# Pinned host copies of a whole step's activations up to this size; above it (prefill: 35 GB in,
+# 22 GB out) one layer's worth of pinned host memory is reused for every layer's copies.
+E2E_FULL_PINNED_BYTES = 8 << 30
 
-def run_gpu(args, world, rank, local):
+
+def _e2e(step, cfg, stream, world, nsteps):
+    """End to end through the public API: every step copies its activations in from pinned host
+    memory, makes the eager C-ABI calls of the step and copies the outputs back, on one stream,
+    timed with CUDA events (max over ranks)."""
+    import torch
+    act_in, act_out = step.act_in, step.act_out
+    el = act_in.element_size()
+    layers = step.layers
+    lin = [step.layer_in[l] for l in layers]
+    lout = [step.layer_out[l] for l in layers]
+    head = lin[0][0]                       # router input (and nothing else) before the first layer
+    full = (act_in.numel() + act_out.numel()) * el <= E2E_FULL_PINNED_BYTES
+    if full:
+        host_in = torch.empty(act_in.numel(), dtype=act_in.dtype, pin_memory=True)
+        host_out = torch.empty(act_out.numel(), dtype=act_out.dtype, pin_memory=True)
+        host_in.copy_(act_in)
+        note = "whole step's activations in pinned host memory"
+    else:
+        n_in, n_out = lin[0][1] - lin[0][0], lout[0][1] - lout[0][0]
+        host_in = torch.empty(head + n_in, dtype=act_in.dtype, pin_memory=True)
+        host_out = torch.empty(n_out, dtype=act_out.dtype, pin_memory=True)
+        host_in[:head].copy_(act_in[:head])
+        host_in[head:].copy_(act_in[lin[0][0]:lin[0][1]])
+        note = ("one layer's activations in pinned host memory, copied in for every layer (bounds pinned host "
+                "memory); every layer's inputs and outputs still cross PCIe each step")
+    h2d = d2h = 0
+
+    def one_step():
+        nonlocal h2d, d2h
+        h2d = d2h = 0
+        act_in[:head].copy_(host_in[:head], non_blocking=True)
+        h2d += head * el
+        step.route()
+        if cfg.merge:
+            step.merge_all()
+        for l, (a0, a1), (b0, b1) in zip(layers, lin, lout):
+            src = host_in[a0:a1] if full else host_in[head:]
+            act_in[a0:a1].copy_(src, non_blocking=True)
+            h2d += (a1 - a0) * el
+            step.run_layer(l)
+            dst = host_out[b0:b1] if full else host_out
+            dst.copy_(act_out[b0:b1], non_blocking=True)
+            d2h += (b1 - b0) * el
+
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            one_step()
+        stream.synchronize()
+        barrier(world)
+        x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0 = time.perf_counter()
+        x0.record(stream)
+        for _ in range(nsteps):
+            one_step()
+        x1.record(stream)
+    stream.synchronize()
+    wall = time.perf_counter() - t0
+    e_ms = max_over_ranks(x0.elapsed_time(x1), world)
+    return {"value": cfg.T * nsteps * world / (e_ms / 1e3), "unit": "tokens/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": nsteps,
+            "ms_per_step": e_ms / nsteps, "host_wall_ms_per_step": wall * 1e3 / nsteps,
+            "calls": "eager C-ABI calls (route, segments, every layer call) on one stream", "host_buffers": note}
+
+
+def measure(name, args, world, rank, local, peaks, kernel_name="auto"):
+    """One full-size workload: launches counted, the step captured in a CUDA graph, K timed
+    replays (clocks sampled), the SGMM calls alone timed for the roofline, and the e2e leg."""
     import torch
     from adapter_pregate_router_b200 import apr, pipeline
     from adapter_pregate_router_b200 import workloads as W
 
-    cfg = W.scaled(W.CONFIGS[args.workload], seed=W.CONFIGS[args.workload].seed + rank)
+    cfg = W.scaled(W.CONFIGS[name], seed=W.CONFIGS[name].seed + rank)
     if args.layers:
         cfg = W.scaled(cfg, layers=args.layers)
-    peaks = load_peaks()
     dev = torch.device("cuda", local)
-    kernels = {"auto": apr.SGMM_AUTO, "skinny": apr.SGMM_SKINNY, "tensor": apr.SGMM_TENSOR, "dense": apr.SGMM_DENSE}
-    step = pipeline.Step(cfg, device=dev, kernel=kernels[args.kernel])
+    kernels = {"auto": apr.SGMM_AUTO, "skinny": apr.SGMM_SKINNY, "tensor": apr.SGMM_TENSOR,
+               "dense": apr.SGMM_DENSE, "bank": apr.SGMM_BANK}
+    step = pipeline.Step(cfg, device=dev, kernel=kernels[kernel_name])
     stream = torch.cuda.Stream(device=dev)
     stream.wait_stream(torch.cuda.current_stream(dev))
 
@@ -395,81 +520,82 @@ def run_gpu(args, world, rank, local):
     ms_step = ms / args.steps
     apr.stream_status(step.ws, stream)
 
-    # ---- the dominant kernel class timed alone (every layer call, no route)
+    # ---- the SGMM (or merge + GEMV) calls alone, every layer, no route
     with torch.cuda.stream(stream):
         for _ in range(3):
             layer_graph.replay()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        nrep = max(10, min(args.steps, 500))
+        nrep = max(5, min(args.steps, 200))
         for _ in range(nrep):
             layer_graph.replay()
         e1.record(stream)
     stream.synchronize()
-    layer_ms = e0.elapsed_time(e1) / nrep
+    layer_ms = max_over_ranks(e0.elapsed_time(e1) / nrep, world)
     idx_np = step.idx.cpu().numpy()
     step_bytes = step.algorithmic_bytes(idx_np)
-    router_bytes = cfg.T * cfg.d_router * (2 if cfg.dtype == "bf16" else 4) + cfg.E * cfg.d_router * (
-        2 if cfg.dtype == "bf16" else 4)
+    el = 2 if cfg.dtype == "bf16" else 4
+    router_bytes = cfg.T * cfg.d_router * el + cfg.E * cfg.d_router * el
     layer_bytes = step_bytes - router_bytes
     ncalls = len(step.calls) if not cfg.merge else 1 + step.nmerge
     achieved_gbs = layer_bytes / (layer_ms * 1e-3) / 1e9
+    traffic = measured_traffic(name) if not args.layers else None
     roof = {
         "bound": "hbm",
         "kernel": ("apr_merge_adapters_planned + apr_gemv (the merge launch and every weight's GEMV)" if cfg.merge
-                   else "apr_sgmm_shrink_expand (shrink+expand launches of every layer call)"),
+                   else "apr_sgmm_shrink_expand (shrink + expand launches of every layer call)"),
         "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
         "frac": achieved_gbs / peaks["hbm_gbs"], "peak_source": f"{peaks['source']} copy bandwidth",
-        "traffic": measured_traffic(args.workload) if not args.layers else None,
-        "traffic_source": "profiles/dram_traffic.md (ncu, one layer, bytes per call)",
+        "traffic": traffic,
+        "traffic_source": (f"{TRAFFIC_FILE} (ncu, bytes per call, kernel-source hash {kernel_source_hash()})"
+                           if traffic is not None else "no capture at the current kernel sources"),
         "bytes_per_call": layer_bytes / ncalls, "calls_per_step": ncalls,
         "us_per_call": layer_ms * 1e3 / ncalls, "step_bytes": step_bytes,
         "step_frac": step_bytes / (ms_step * 1e-3) / 1e9 / peaks["hbm_gbs"],
     }
+    graph.reset()
+    layer_graph.reset()
+    e2e = _e2e(step, cfg, stream, world, max(3, min(args.steps, 20 if cfg.T < 4096 else 3)))
+    apr.stream_status(step.ws, stream)
+    out = {"cfg": cfg, "value": value, "ms_per_step": ms_step, "roofline": roof, "e2e": e2e,
+           "clocks": clk.summary(), "gpu_launches": launches * args.steps, "launches_per_step": launches,
+           "config": dict(config_block(cfg, world), **({"sgmm_kernel": kernel_name} if kernel_name != "auto" else {}))}
+    del step
+    import gc
+    gc.collect()
+    torch.cuda.empty_cache()
+    return out
 
-    # ---- end to end through the public API with host buffers
-    e2e = None
-    if not cfg.merge:
-        host_in = torch.empty(step.act_in.numel(), dtype=step.act_in.dtype, pin_memory=True)
-        host_out = torch.empty(step.act_out.numel(), dtype=step.act_out.dtype, pin_memory=True)
-        host_in.copy_(step.act_in)
-        ke = max(3, min(args.steps, 50))
-        with torch.cuda.stream(stream):
-            for _ in range(2):
-                step.act_in.copy_(host_in, non_blocking=True)
-                graph.replay()
-                host_out.copy_(step.act_out, non_blocking=True)
-            stream.synchronize()
-            barrier(world)
-            x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            x0.record(stream)
-            for _ in range(ke):
-                step.act_in.copy_(host_in, non_blocking=True)
-                graph.replay()
-                host_out.copy_(step.act_out, non_blocking=True)
-            x1.record(stream)
-        stream.synchronize()
-        e_ms = max_over_ranks(x0.elapsed_time(x1), world)
-        e2e = {"value": cfg.T * ke * world / (e_ms / 1e3), "unit": "tokens/s",
-               "h2d_bytes_per_step": host_in.numel() * host_in.element_size(),
-               "d2h_bytes_per_step": host_out.numel() * host_out.element_size(),
-               "steps": ke, "ms_per_step": e_ms / ke}
+
+def run_gpu(args, world, rank, local):
+    from adapter_pregate_router_b200 import workloads as W
+    peaks = load_peaks()
+    main = measure(args.workload, args, world, rank, local, peaks, args.kernel)
+    cfg = main["cfg"]
+    others = {}
+    also = [] if args.also in ("", "none") else [w.strip() for w in args.also.split(",")]
+    for name in also:
+        if name == args.workload:
+            continue
+        r = measure(name, args, world, rank, local, peaks)
+        others[name] = {"value": r["value"], "unit": "tokens/s", "ms_per_step": r["ms_per_step"],
+                        "config": r["config"], "roofline": r["roofline"], "e2e": r["e2e"], "clocks": r["clocks"],
+                        "gpu_launches": r["gpu_launches"], "launches_per_step": r["launches_per_step"]}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(W.CONFIGS[args.workload], budget_s=args.ref_budget)
 
     line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "metric": METRIC, "value": main["value"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": main["ms_per_step"], "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16" if cfg.dtype == "bf16" else "f32", "data": "synthetic",
-        "config": dict(config_block(cfg, world), **({"sgmm_kernel": args.kernel} if args.kernel != "auto" else {})),
-        "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
-        "clocks": clk.summary(), "gpu_launches": launches * args.steps,
-        "launches_per_step": launches,
+        "config": main["config"], "roofline": main["roofline"], "cpu_baseline": cpu, "e2e": main["e2e"],
+        "clocks": main["clocks"], "gpu_launches": main["gpu_launches"],
+        "launches_per_step": main["launches_per_step"],
     }
-    graph.reset()
-    layer_graph.reset()
+    if others:
+        line["workloads"] = others
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -477,17 +603,27 @@ def run_gpu(args, world, rank, local):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "multitenant", "merge", "tiny"])
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="prefill", choices=["decode", "prefill", "multitenant", "merge", "tiny"])
+    ap.add_argument("--also", default="decode,multitenant,merge",
+                    help="other full-size workloads timed in the same run and reported under 'workloads' "
+                         "(comma-separated, or 'none')")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-budget", type=float, default=12.0, help="seconds of oracle work per reference step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel", default="auto", choices=["auto", "skinny", "tensor", "dense"],
-                    help="force one SGMM kernel class (comparisons; the benchmark line uses auto)")
+    ap.add_argument("--kernel", default="auto", choices=["auto", "skinny", "tensor", "dense", "bank"],
+                    help="force one SGMM kernel class on the main workload (comparisons; the benchmark uses auto)")
     ap.add_argument("--layers", type=int, default=0,
                     help="build only this many layers (a reduced workload for profiling; not the benchmark)")
+    ap.add_argument("--ingest-traffic", metavar="CSV",
+                    help="record an ncu DRAM capture of --workload as bytes per call (with --calls, --command)")
+    ap.add_argument("--calls", type=int, default=1)
+    ap.add_argument("--command", default="")
     args = ap.parse_args()
+    if args.ingest_traffic:
+        print(ingest_traffic(args.ingest_traffic, args.workload, args.calls, args.command))
+        return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":

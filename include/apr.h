@@ -69,7 +69,9 @@ typedef enum apr_sgmm_kernel {
   APR_SGMM_AUTO = 0,    /* by T, E, the ranks and the mean segment size T*k/E */
   APR_SGMM_SKINNY = 1,  /* CUDA-core kernel for few tokens per adapter        */
   APR_SGMM_TENSOR = 2,  /* tcgen05 tensor-core kernel for long segments       */
-  APR_SGMM_DENSE = 3    /* tcgen05 over the whole adapter bank, small batches */
+  APR_SGMM_DENSE = 3,   /* tcgen05 over the whole adapter bank, small batches */
+  APR_SGMM_BANK = 4     /* tcgen05 in token order over the whole bank: few
+                           adapters, many tokens (contiguous y tiles by TMA) */
 } apr_sgmm_kernel;
 
 /* ------------------------------------------------------------------------
@@ -169,13 +171,17 @@ typedef struct apr_proj {
  *          is reused by every layer, section 2.A)
  * seg_off,perm device: the outputs of apr_segment_tokens for this idx; `ws`
  *          must be the workspace that call wrote.
- * kernel   APR_SGMM_AUTO, or a forced kernel class.  The tensor-core kernel
- *          needs dtype == APR_BF16, k <= 2, max_rank <= 64, d_in % 64 == 0 and
- *          d_out % 16 == 0; the dense kernel needs dtype == APR_BF16, T <= 64,
- *          E <= 16 and E * (max_rank rounded up to 16) <= 256; a forced kernel
- *          returns APR_ERR_UNSUPPORTED outside its range.  AUTO takes the
- *          dense kernel where it applies, the tensor-core kernel where
- *          T*k/E >= 256 or T*k >= 2048, and the CUDA-core kernel otherwise.
+ * kernel   APR_SGMM_AUTO, or a forced kernel class.  With R16 = max_rank
+ *          rounded up to 16: the tensor-core kernel needs dtype == APR_BF16,
+ *          k <= 2, k * R16 <= 64, d_in % 64 == 0 and d_out % 16 == 0; the
+ *          dense kernel needs dtype == APR_BF16, T <= 64, E <= 16 and
+ *          E * R16 <= 256; the bank kernel needs dtype == APR_BF16, R16 in
+ *          {16, 32, 64}, k <= 4, k * R16 <= 64, E * R16 <= 256 and
+ *          d_in % 64 == 0.  A forced kernel returns APR_ERR_UNSUPPORTED
+ *          outside its range.  AUTO takes the dense kernel where it applies,
+ *          else the bank kernel where it applies, else the tensor-core kernel
+ *          where T*k/E >= 256 or T*k >= 2048, and the CUDA-core kernel
+ *          otherwise.
  * T == 0 is a no-op.  Empty segments are legal.
  * ---------------------------------------------------------------------- */
 apr_status apr_sgmm_shrink_expand(const void* x, int d_in, const apr_proj* projs, int nproj,

@@ -98,7 +98,7 @@ def test_sgmm_host_validation(apr):
     assert call(max_rank=12) == apr.APR_ERR_INVALID_ARG
     assert call(max_rank=136) == apr.APR_ERR_INVALID_ARG
     assert call(d_in=20) == apr.APR_ERR_INVALID_ARG
-    assert call(kernel=4) == apr.APR_ERR_INVALID_ARG
+    assert call(kernel=5) == apr.APR_ERR_INVALID_ARG
     assert call(x=None) == apr.APR_ERR_INVALID_ARG
     assert call(ws_bytes=256) == apr.APR_ERR_WORKSPACE
     bad = (apr.Proj * 1)(apr.Proj(0x1000, 0x1000, 60, 0x1000, 0x1000))
@@ -126,6 +126,13 @@ def test_sgmm_host_validation(apr):
     # so does the dense kernel (fp32, or more than 64 tokens)
     assert call(kernel=3, dtype=0) == apr.APR_ERR_UNSUPPORTED
     assert call(kernel=3, T=65) == apr.APR_ERR_UNSUPPORTED
+    # and the bank kernel: fp32, E * R16 > 256, k > 4, k * R16 > 64, rank slot 128, d_in % 64 != 0
+    assert call(kernel=4, dtype=0) == apr.APR_ERR_UNSUPPORTED
+    assert call(kernel=4, E=17) == apr.APR_ERR_UNSUPPORTED
+    assert call(kernel=4, k=5) == apr.APR_ERR_UNSUPPORTED
+    assert call(kernel=4, k=3, max_rank=32) == apr.APR_ERR_UNSUPPORTED
+    assert call(kernel=4, E=2, max_rank=128) == apr.APR_ERR_UNSUPPORTED
+    assert call(kernel=4, d_in=72) == apr.APR_ERR_UNSUPPORTED
 
 
 def test_merge_and_gemv_host_validation(apr):

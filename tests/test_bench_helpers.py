@@ -37,14 +37,20 @@ def test_measured_traffic_needs_the_matching_hash(tmp_path, monkeypatch):
     (csrc / "k.cu").write_text("__global__ void k() { }\n")
     (tmp_path / "profiles").mkdir()
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    h = bench.kernel_source_hash()
-    (tmp_path / "profiles" / "dram_traffic.md").write_text(
-        f"text\n\ntraffic: decode 1234 {h}\ntraffic: prefill 99 0000000000000000\n")
-    assert bench.measured_traffic("decode") == 1234.0
-    assert bench.measured_traffic("prefill") is None      # captured on other kernels
-    assert bench.measured_traffic("merge") is None        # no line
-    os.remove(tmp_path / "profiles" / "dram_traffic.md")
-    assert bench.measured_traffic("decode") is None
+    assert bench.measured_traffic("decode") is None       # no data file
+    # an ncu --csv launch capture with two kernels' DRAM bytes, ingested as bytes per call
+    csv = tmp_path / "cap.csv"
+    csv.write_text('==PROF== noise\n'
+                   '"ID","Kernel Name","Metric Name","Metric Unit","Metric Value"\n'
+                   '"0","k1","dram__bytes_read.sum","Mbyte","1.50"\n'
+                   '"0","k1","dram__bytes_write.sum","Kbyte","500"\n'
+                   '"0","k1","gpu__time_duration.sum","usecond","9.5"\n'
+                   '"1","k2","dram__bytes_read.sum","byte","1,000"\n')
+    assert bench.ingest_traffic(str(csv), "decode", 2, "ncu ...") == (1.5e6 + 5e5 + 1000) / 2
+    assert bench.measured_traffic("decode") == (1.5e6 + 5e5 + 1000) / 2
+    assert bench.measured_traffic("prefill") is None      # not captured
+    (csrc / "k.cu").write_text("__global__ void k() { int changed; }\n")
+    assert bench.measured_traffic("decode") is None       # captured on other kernels
 
 
 def _run_bench(args, env_extra=None):

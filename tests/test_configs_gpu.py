@@ -90,9 +90,11 @@ def test_config_parity(mods, name, nrows):
 
 
 def test_config_parity_merge(mods):
-    """Merged weights on sampled rows for every weight; for two full layers the
-    whole merged weight and the whole GEMV output (the merged path rounds W'
-    to bf16 before the GEMV, so the GEMV is judged over its full output)."""
+    """Every one of the 224 weights: the merged weight on 64 sampled rows (all rows for two
+    layers) and the whole GEMV output, against the oracle's fp64 W' = W + sum g B A and its
+    product with x.  The device GEMV reads W' after its one rounding to bf16; that rounding
+    moves each output by about 2^-9 / sqrt(3) of its magnitude in relative Frobenius norm,
+    inside the 5e-3 bound."""
     apr, pipeline = mods
     cfg = W.CONFIGS["merge"]
     step = pipeline.Step(cfg)
@@ -103,20 +105,22 @@ def test_config_parity_merge(mods):
     e_sel = ridx[0]
     rng = np.random.default_rng(3)
     full_layers = {0, 25}
+    checked = 0
     for (l, g, p), (Wt, Wp, x, y) in step.weights.items():
         d_out, d_in = Wt.shape
-        rows = np.arange(d_out) if l in full_layers else np.sort(rng.choice(d_out, size=8, replace=False))
-        Wr_rows = W.host_rows(cfg, W.w_key(l, g, p), (d_out, d_in), rows)
-        A = {e: W.host_tensor(cfg, W.a_key(l, g, p, e), (int(ranks[e]), d_in)) for e in e_sel}
-        Bfull = {e: W.host_tensor(cfg, W.b_key(l, g, p, e), (d_out, int(ranks[e]))) for e in e_sel}
-        Al = [A.get(e) for e in range(cfg.E)]
-        Bl = [Bfull[e][rows] if e in Bfull else None for e in range(cfg.E)]
-        ref_rows = O.merge_adapters(Wr_rows, Al, Bl, e_sel, rgate[0])
+        Wfull = W.host_tensor(cfg, W.w_key(l, g, p), (d_out, d_in))
+        A = [W.host_tensor(cfg, W.a_key(l, g, p, e), (int(ranks[e]), d_in)) if e in e_sel else None
+             for e in range(cfg.E)]
+        B = [W.host_tensor(cfg, W.b_key(l, g, p, e), (d_out, int(ranks[e]))) if e in e_sel else None
+             for e in range(cfg.E)]
+        ref_W = O.merge_adapters(Wfull, A, B, e_sel, rgate[0])
+        rows = np.arange(d_out) if l in full_layers else np.sort(rng.choice(d_out, size=64, replace=False))
         got = to_np(Wp[torch.from_numpy(rows).to(Wp.device)])
-        close(got, ref_rows, f"merged {l}/{p}")
-        if l in full_layers:
-            xv = W.host_tensor(cfg, W.xm_key(l, g, p), (d_in,))
-            close(to_np(y), O.gemv(ref_rows, xv), f"gemv {l}/{p}")
+        close(got, ref_W[rows], f"merged {l}/{p}")
+        xv = W.host_tensor(cfg, W.xm_key(l, g, p), (d_in,))
+        close(to_np(y), O.gemv(ref_W, xv), f"gemv {l}/{p}")
+        checked += 1
+    assert checked == 224
 
 
 def test_graph_replay_matches_eager(mods):

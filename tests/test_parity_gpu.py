@@ -75,7 +75,8 @@ def test_route_equal_logits_give_half_gates(apr):
 
 
 @pytest.mark.parametrize("T,k,E", [(1, 1, 1), (7, 2, 3), (64, 2, 8), (1000, 3, 40), (4096, 1, 256),
-                                   (8192, 2, 16), (333, 8, 1024), (5000, 2, 2)])
+                                   (8192, 2, 16), (333, 8, 1024), (5000, 2, 2), (1025, 1, 1024),
+                                   (40000, 2, 64), (20000, 3, 1024)])   # the last two: plan not staged in shared memory
 def test_segments_bit_exact(apr, T, k, E):
     rng = np.random.default_rng(T * 7 + k + E)
     idx = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
@@ -83,6 +84,19 @@ def test_segments_bit_exact(apr, T, k, E):
     rs, rp = O.segment_tokens(idx, E)
     assert np.array_equal(seg_off, rs)
     assert np.array_equal(perm, rp)
+
+
+@pytest.mark.parametrize("kernel", ["tensor", "skinny"])
+def test_sgmm_large_batch_unstaged_plan(apr, kernel):
+    """40000 tokens: the segment kernel keeps idx and the token order in global memory (too
+    large for shared memory); the gathered kernels read that plan."""
+    rng = np.random.default_rng(71)
+    idx = _zipf_idx(rng, 40000, 24, 2)
+    x, As, Bs, idx, gate, ybs = _case(rng, 40000, 64, (64,), (16,) * 24, 2, dist=idx)
+    x, As, Bs, ybs = _rounded(x, As, Bs, ybs)
+    kern = apr.SGMM_TENSOR if kernel == "tensor" else apr.SGMM_SKINNY
+    got = run_sgmm(apr, x, As, Bs, idx, gate, ybs, BF16, kernel=kern)
+    close(got[0], oracle_group(x, As, Bs, idx, gate.astype(np.float64), ybs)[0], f"{kernel} T=40000")
 
 
 def test_segments_skewed_and_empty(apr):
@@ -511,3 +525,174 @@ def test_sgmm_dense_faults_and_limits(apr):
     with pytest.raises(apr.AprError) as ei:
         run_sgmm(apr, x2, As2, Bs2, idx2, gate2, ybs2, BF16, kernel=apr.SGMM_DENSE)
     assert ei.value.status == apr.APR_ERR_UNSUPPORTED
+
+
+# ------------------------------------------------------------------ edge cases on every kernel class
+
+
+def _seg_counts_idx(rng, counts, k):
+    """idx [T, k] whose adapter segments hold exactly ``counts[e]`` pairs (adapters absent from
+    ``counts`` are empty).  The pairs sorted by adapter are dealt slot by slot (token t takes
+    positions t, t + T, ...), so a token never holds one adapter twice while every count is at
+    most T; then tokens and each token's slots are shuffled."""
+    pairs = np.concatenate([np.full(c, e, np.int32) for e, c in sorted(counts.items())])
+    T = len(pairs) // k
+    assert T * k == len(pairs) and max(counts.values()) <= T
+    idx = np.stack([pairs[j * T:(j + 1) * T] for j in range(k)], axis=1)
+    idx = idx[rng.permutation(T)]
+    for t in range(T):
+        idx[t] = idx[t][rng.permutation(k)]
+    assert all(len(set(r)) == k for r in idx.tolist())
+    return np.ascontiguousarray(idx)
+
+
+# pair counts per adapter: empty adapters (0 and the last), a one-pair segment, 127/128/129-pair
+# segments and segments of thousands of pairs
+_EDGE_K1 = {1: 1, 2: 127, 3: 128, 4: 129, 5: 2001}                      # 7 adapters, T = 2386
+_EDGE_K2 = {1: 1, 2: 127, 3: 128, 4: 129, 5: 1000, 6: 1001}             # 8 adapters, T = 1193
+
+
+@pytest.mark.parametrize("kernel,k,ranks,d_in,d_out", [
+    ("tensor", 1, (16, 8, 16, 32, 64, 16, 8), 512, 336),     # top-1, every rank slot up to 64
+    ("tensor", 2, (16,) * 8, 512, 336),                       # k = 2: mixed tiles (4 adapters x 16)
+    ("tensor", 2, (32, 24, 32, 16, 32, 32, 8, 32), 256, 144), # k = 2, rank slots of 32: set tiles
+    ("bank", 1, (16, 8, 16, 16, 16, 16, 8), 512, 336),
+    ("bank", 2, (16,) * 8, 512, 336),
+    ("bank", 2, (32, 24, 32, 16, 32, 32, 8, 32), 256, 136),   # d_out with an 8-column last tile
+    ("skinny", 1, (16, 8, 16, 32, 64, 16, 8), 512, 328),
+    ("skinny", 2, (16, 8, 16, 32, 64, 16, 8, 16), 512, 328),
+])
+def test_sgmm_edge_segments_every_kernel(apr, kernel, k, ranks, d_in, d_out):
+    """Empty adapters, a one-pair segment, 127/128/129-pair segments and segments of 1000-2001
+    pairs through each gathered or bank kernel class, against the oracle."""
+    rng = np.random.default_rng(40 + k + len(ranks) + d_out)
+    E = len(ranks)
+    idx = _seg_counts_idx(rng, _EDGE_K1 if k == 1 else _EDGE_K2, k)
+    T = idx.shape[0]
+    x, As, Bs, _, gate, ybs = _case(rng, T, d_in, (d_out,), ranks, k, dist=idx)
+    x, As, Bs, ybs = _rounded(x, As, Bs, ybs)
+    kern = {"tensor": apr.SGMM_TENSOR, "bank": apr.SGMM_BANK, "skinny": apr.SGMM_SKINNY}[kernel]
+    seg, _, _ = run_segment(apr, idx, E)
+    sizes = np.diff(seg)
+    assert sizes[0] == 0 and sizes[E - 1] == 0 and {1, 127, 128, 129} <= set(sizes.tolist())
+    for zero in (True, False):
+        yb = [np.zeros_like(y) for y in ybs] if zero else ybs
+        got = run_sgmm(apr, x, As, Bs, idx, gate, yb, BF16, kernel=kern)
+        ref = oracle_group(x, As, Bs, idx, gate.astype(np.float64), yb)
+        close(got[0], ref[0], f"{kernel} k={k} zero_ybase={zero}")
+
+
+@pytest.mark.parametrize("T,k,counts", [
+    (64, 1, {1: 1, 2: 60, 4: 3}),
+    (33, 2, {1: 1, 3: 33, 4: 29, 6: 3}),
+    (64, 2, {1: 1, 3: 64, 4: 60, 6: 3}),
+])
+def test_sgmm_dense_edge_segments(apr, T, k, counts):
+    """The dense decode kernel with empty adapters, a one-pair segment and an adapter that
+    every token selected (T <= 64)."""
+    rng = np.random.default_rng(50 + T + k)
+    ranks = (16, 8, 16, 16, 8, 16, 16, 16)
+    idx = _seg_counts_idx(rng, counts, k)
+    assert idx.shape == (T, k)
+    x, As, Bs, _, gate, ybs = _case(rng, T, 4096, (4096, 264), ranks, k, dist=idx)
+    x, As, Bs, ybs = _rounded(x, As, Bs, ybs)
+    for zero in (True, False):
+        yb = [np.zeros_like(y) for y in ybs] if zero else ybs
+        got = run_sgmm(apr, x, As, Bs, idx, gate, yb, BF16, kernel=apr.SGMM_DENSE)
+        ref = oracle_group(x, As, Bs, idx, gate.astype(np.float64), yb)
+        for p in range(2):
+            close(got[p], ref[p], f"dense T={T} k={k} proj {p} zero_ybase={zero}")
+
+
+# ------------------------------------------------------------------ SGMM, bank (token-order) kernel
+
+
+@pytest.mark.parametrize("T,d_in,d_outs,ranks,k,zipf", [
+    (517, 4096, (4096,), (16,) * 16, 2, True),              # prefill-shaped projection, ragged last row tile
+    (1000, 1024, (512, 1008), (16,) * 6, 2, True),          # two projections, ragged d_out
+    (129, 192 * 2, (64, 64, 64, 64), (32,) * 3, 2, False),  # four projections, rank slots of 32
+    (300, 256, (136,), (8, 16, 8, 16), 4, False),           # k = 4, an 8-wide last column tile
+    (700, 256, (128,), (40, 64, 56, 48), 1, False),         # rank slots of 64, k = 1
+    (65, 512, (256,), (16,) * 16, 3, False),                # one token past a tile, k = 3
+    (1, 128, (16,), (16, 16), 2, False),                    # one token
+    (8192, 512, (128,), (16,) * 16, 2, True),               # 64 full row tiles
+])
+def test_sgmm_bank_parity(apr, T, d_in, d_outs, ranks, k, zipf):
+    rng = np.random.default_rng(T + d_in + k + 11)
+    idx = _zipf_idx(rng, T, len(ranks), k) if zipf else "uniform"
+    x, As, Bs, idx, gate, ybs = _case(rng, T, d_in, d_outs, ranks, k, dist=idx)
+    x, As, Bs, ybs = _rounded(x, As, Bs, ybs)
+    for zero in (True, False):
+        yb = [np.zeros_like(y) for y in ybs] if zero else ybs
+        got = run_sgmm(apr, x, As, Bs, idx, gate, yb, BF16, kernel=apr.SGMM_BANK)
+        ref = oracle_group(x, As, Bs, idx, gate.astype(np.float64), yb)
+        for p in range(len(d_outs)):
+            close(got[p], ref[p], f"bank proj {p} zero_ybase={zero}")
+
+
+def test_sgmm_bank_integer_inputs_exact(apr):
+    """Small integers, gates of 1/2: the bank result is the exact value rounded once to bf16
+    (pins the rank-slot placement of V, the Bcat layout and the row/column tiling)."""
+    rng = np.random.default_rng(61)
+    x, As, Bs, idx, gate, ybs = _case(rng, 400, 512, (128, 264), (16, 8, 16, 16, 8), 2, ints=True)
+    got = run_sgmm(apr, x, As, Bs, idx, gate, ybs, BF16, kernel=apr.SGMM_BANK)
+    ref = oracle_group(x, As, Bs, idx, gate.astype(np.float64), ybs)
+    for p in range(2):
+        want = bf16_exact(ref[p]).astype(np.float64)
+        assert np.array_equal(got[p], want), f"proj {p}: max diff {np.abs(got[p] - want).max()}"
+
+
+def test_sgmm_bank_properties(apr):
+    """Zero B leaves y_base bit-exact; in place equals out of place; a token permutation
+    permutes the output bits; two runs agree; AUTO takes the bank kernel here."""
+    rng = np.random.default_rng(62)
+    idx = _zipf_idx(rng, 900, 6, 2)
+    x, As, Bs, idx, gate, ybs = _case(rng, 900, 512, (1008, 80), (16,) * 6, 2, dist=idx)
+    x, As, Bs, ybs = _rounded(x, As, Bs, ybs)
+    Bz = [[np.zeros_like(b) for b in P] for P in Bs]
+    z = run_sgmm(apr, x, As, Bz, idx, gate, ybs, BF16, kernel=apr.SGMM_BANK)
+    for p in range(2):
+        assert np.array_equal(z[p], ybs[p].astype(np.float64))
+    a = run_sgmm(apr, x, As, Bs, idx, gate, ybs, BF16, kernel=apr.SGMM_BANK, in_place=True)
+    b = run_sgmm(apr, x, As, Bs, idx, gate, ybs, BF16, kernel=apr.SGMM_BANK)
+    c = run_sgmm(apr, x, As, Bs, idx, gate, ybs, BF16)
+    for p in range(2):
+        assert np.array_equal(a[p], b[p]) and np.array_equal(b[p], c[p])
+    perm = rng.permutation(900)
+    d = run_sgmm(apr, x[perm], As, Bs, idx[perm], gate[perm], [y[perm] for y in ybs], BF16, kernel=apr.SGMM_BANK)
+    for p in range(2):
+        assert np.array_equal(d[p], b[p][perm])
+
+
+def test_sgmm_bank_faults_and_limits(apr):
+    rng = np.random.default_rng(63)
+    x, As, Bs, idx, gate, ybs = _case(rng, 200, 256, (128,), (16, 16, 32), 2)
+    x, As, Bs, ybs = _rounded(x, As, Bs, ybs)
+    with pytest.raises(apr.AprError) as ei:                   # a rank above max_rank, caught on the device
+        run_sgmm(apr, x, As, Bs, idx, gate, ybs, BF16, kernel=apr.SGMM_BANK, max_rank=16)
+    assert ei.value.status == apr.APR_ERR_DEVICE_INDEX
+    ok = run_sgmm(apr, x, As, Bs, idx, gate, ybs, BF16, kernel=apr.SGMM_BANK)
+    close(ok[0], oracle_group(x, As, Bs, idx, gate.astype(np.float64), ybs)[0], "bank after fault")
+    x2, As2, Bs2, idx2, gate2, ybs2 = _case(rng, 100, 256, (128,), (16,) * 17, 2)   # E * 16 > 256
+    x2, As2, Bs2, ybs2 = _rounded(x2, As2, Bs2, ybs2)
+    with pytest.raises(apr.AprError) as ei:
+        run_sgmm(apr, x2, As2, Bs2, idx2, gate2, ybs2, BF16, kernel=apr.SGMM_BANK)
+    assert ei.value.status == apr.APR_ERR_UNSUPPORTED
+
+
+def test_kernels_on_a_second_device(apr):
+    """Kernel attributes are per device: every SGMM kernel class and the merge run on device 1
+    after device 0 has set them up (skipped with fewer than two visible GPUs)."""
+    if torch.cuda.device_count() < 2:
+        pytest.skip("needs two visible GPUs")
+    rng = np.random.default_rng(64)
+    x, As, Bs, idx, gate, ybs = _case(rng, 300, 512, (256,), (16,) * 6, 2)
+    x, As, Bs, ybs = _rounded(x, As, Bs, ybs)
+    ref = oracle_group(x, As, Bs, idx, gate.astype(np.float64), ybs)
+    for dev_i in (0, 1):
+        with torch.cuda.device(dev_i):
+            for kern in (apr.SGMM_SKINNY, apr.SGMM_TENSOR, apr.SGMM_BANK):
+                close(run_sgmm(apr, x, As, Bs, idx, gate, ybs, BF16, kernel=kern)[0], ref[0], f"device {dev_i}")
+            xs, As_d, Bs_d = x[:40], As, Bs
+            close(run_sgmm(apr, xs, As_d, Bs_d, idx[:40], gate[:40], [ybs[0][:40]], BF16, kernel=apr.SGMM_DENSE)[0],
+                  oracle_group(xs, As_d, Bs_d, idx[:40], gate[:40].astype(np.float64), [ybs[0][:40]])[0], "dense")

@@ -3,7 +3,8 @@ allocate device memory (no allocator of their own, or no tolerance for the
 synchronisation cudaMalloc can cause).  It must give the same routing as
 apr_pregate_route, which runs on a caller-provided workspace, on two calls in
 a row (the second call sees the scratch the first one left behind), and must
-refuse sizes beyond its fixed scratch.  Kept in a file that pytest collects
+refuse sizes beyond its fixed scratch; on exact router inputs it must also equal
+the fp64 oracle.  Kept in a file that pytest collects
 last, so a failure here comes after every other test has run.
 """
 import numpy as np
@@ -11,6 +12,7 @@ import pytest
 import torch
 
 from adapter_pregate_router_b200 import workloads as W
+from oracle import apr_oracle as O
 
 pytestmark = pytest.mark.gpu
 
@@ -27,15 +29,16 @@ def apr():
 
 
 def _cases():
-    # forced, exact-logit router inputs of two workloads, then free float inputs
+    # forced, exact-logit router inputs of two workloads (exact: the oracle decides them too),
+    # then free float inputs (fp32 sums: compared with the workspace router only)
     out = []
     for name in ("prefill", "decode"):
         cfg = W.CONFIGS[name]
         h, Wr, _ = W.router_inputs(cfg)
-        out.append((h, Wr, cfg.k, torch.bfloat16))
+        out.append((h, Wr, cfg.k, torch.bfloat16, True))
     rng = np.random.default_rng(5)
     out.append((rng.normal(size=(700, 512)).astype(np.float32),
-                rng.normal(size=(64, 512)).astype(np.float32), 3, torch.float32))
+                rng.normal(size=(64, 512)).astype(np.float32), 3, torch.float32, False))
     return out
 
 
@@ -58,10 +61,14 @@ def test_noalloc_route_matches_workspace_route_on_consecutive_calls(apr):
     cases = _cases()
     # two rounds over different inputs: every call follows another call's scratch
     for _ in range(2):
-        for h, Wr, k, dt in cases:
+        for h, Wr, k, dt, exact in cases:
             idx, gate, idx_ref, gate_ref = _route_both(apr, h, Wr, k, dt)
             assert np.array_equal(idx, idx_ref)
             assert np.abs(gate - gate_ref).max() <= GATE_ATOL
+            if exact:
+                oidx, ogate, _ = O.pregate_route(h, Wr, k)
+                assert np.array_equal(idx, oidx)
+                assert np.abs(gate - ogate).max() <= GATE_ATOL
 
 
 def test_noalloc_route_rejects_sizes_beyond_its_scratch(apr):

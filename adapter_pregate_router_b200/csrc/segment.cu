@@ -444,13 +444,15 @@ cudaError_t launch_segment(const int32_t* idx, int T, int k, int E, int32_t* seg
   const size_t fixed = seg_smem_fixed(E);
   const bool stage = fixed + seg_smem_stage(T, k) <= kStageBudget;
   const size_t smem = fixed + (stage ? seg_smem_stage(T, k) : 0);
+  // the kernel's static shared memory (mixed-tile staging, 16 KB) counts against the same 48 KB
+  // default as the dynamic part, so the limit is raised for every size
   static SmemLimit lim[2];
   cudaError_t err;
   if (stage) {
-    if (smem > 48 * 1024 && (err = lim[1].ensure((const void*)segment_kernel<true>, smem)) != cudaSuccess) return err;
+    if ((err = lim[1].ensure((const void*)segment_kernel<true>, smem)) != cudaSuccess) return err;
     return launch_pdl(segment_kernel<true>, dim3(1), dim3(SEG_THREADS), smem, s, idx, T, k, E, seg_off, perm, ws);
   }
-  if (smem > 48 * 1024 && (err = lim[0].ensure((const void*)segment_kernel<false>, smem)) != cudaSuccess) return err;
+  if ((err = lim[0].ensure((const void*)segment_kernel<false>, smem)) != cudaSuccess) return err;
   return launch_pdl(segment_kernel<false>, dim3(1), dim3(SEG_THREADS), smem, s, idx, T, k, E, seg_off, perm, ws);
 }
 

@@ -125,8 +125,13 @@ __global__ void __launch_bounds__(BK_BLOCK, 1) bank_expand_kernel(const __grid_c
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
 
-  pdl_wait();
-  pdl_trigger();
+  // the first V warpgroup stages the first column block's Bcat (weights) before waiting for
+  // the preceding kernel; every other role waits first
+  const bool early_bcat = tid >= BK_EPI && tid < BK_EPI + BK_VW;
+  if (!early_bcat) {
+    pdl_wait();
+    pdl_trigger();
+  }
   if (blockIdx.x == 0 && tid == 0) reinterpret_cast<WsHeader*>(a.ws)->sched = 0;   // this call's shrink is done
 
   const int K = a.k, T = a.T, NB = P.NB, nrt = P.nrt;
@@ -206,6 +211,40 @@ __global__ void __launch_bounds__(BK_BLOCK, 1) bank_expand_kernel(const __grid_c
       int p, c0, t0;
       unit_at(0, p, c0, t0, blk0);
     }
+    // Bcat[n][e*R16 + r] = B_e[c0 + n][r] of projection p's column block at c0 (zeros past a rank
+    // or past d_out), K-major 8x16-byte core matrices; ends with the bfull arrival
+    auto load_bcat = [&](int p, int c0) {
+      const int d_out = a.proj[p].d_out;
+      const int cpa = R16 / 8;                     // 16-byte chunks of one adapter's row slot
+      for (int w = vt; w < a.E * BK_NT * cpa; w += BK_VW) {
+        const int e = w / (BK_NT * cpa);
+        const int rem = w - e * (BK_NT * cpa);
+        const int nn = rem / cpa, c8 = rem - nn * cpa;
+        const int re = a.ranks[e];
+        const bool rank_ok = re >= 8 && re <= R16 && (re & 7) == 0;
+        if (!rank_ok && nn == 0 && c8 == 0) report(a.ws, APR_ERR_DEVICE_INDEX, K_TC, e);
+        const int kc = e * cpa + c8;
+        const uint32_t dst = sB + (uint32_t)kc * (BK_NT / 8 * 128) + (uint32_t)(nn >> 3) * 128 + (uint32_t)(nn & 7) * 16;
+        if (rank_ok && c8 * 8 < re && c0 + nn < d_out) {
+          const __nv_bfloat16* B = reinterpret_cast<const __nv_bfloat16*>(a.proj[p].B[e]);
+          cp_async16(smem + (dst - sbase), B + (size_t)(c0 + nn) * re + c8 * 8);
+        } else {
+          st_shared_zero16(dst);
+        }
+      }
+      cp_async_wait_all();
+      fence_proxy_async();                         // Bcat is read by the tensor core (async proxy)
+      mbar_arrive(bar_bfull);
+    };
+    if (vg == 0) {
+      if (n > 0) {                                 // unit 0 always starts a block
+        int p, c0, t0, blk;
+        unit_at(0, p, c0, t0, blk);
+        load_bcat(p, c0);
+      }
+      pdl_wait();
+      pdl_trigger();
+    }
     // the gated v rows of unit i's tile (contiguous: tokens t0.. in pair order) -> this group's buffer
     auto issue_rows = [&](int i) {
       int p, c0, t0, blk;
@@ -248,32 +287,12 @@ __global__ void __launch_bounds__(BK_BLOCK, 1) bank_expand_kernel(const __grid_c
         unit_at(i - 1, p2, c02, t02, blk2);
         first = blk2 != blk;
       }
-      if (first) {
+      if (first && i > 0) {
         // Bcat of a new column block (this group takes its first unit), after the MMAs are done
-        // with the previous block
+        // with the previous block (unit 0's block was staged before the wait above)
         const int nb = blk - blk0;                 // blocks before this one in the CTA's range
-        if (nb > 0 && !mbar_wait(bar_bempty, (nb - 1) & 1)) { abort = true; break; }
-        const int d_out = a.proj[p].d_out;
-        const int cpa = R16 / 8;                   // 16-byte chunks of one adapter's row slot
-        for (int w = vt; w < a.E * BK_NT * cpa; w += BK_VW) {
-          const int e = w / (BK_NT * cpa);
-          const int rem = w - e * (BK_NT * cpa);
-          const int nn = rem / cpa, c8 = rem - nn * cpa;
-          const int re = a.ranks[e];
-          const bool rank_ok = re >= 8 && re <= R16 && (re & 7) == 0;
-          if (!rank_ok && nn == 0 && c8 == 0) report(a.ws, APR_ERR_DEVICE_INDEX, K_TC, e);
-          const int kc = e * cpa + c8;
-          const uint32_t dst = sB + (uint32_t)kc * (BK_NT / 8 * 128) + (uint32_t)(nn >> 3) * 128 + (uint32_t)(nn & 7) * 16;
-          if (rank_ok && c8 * 8 < re && c0 + nn < d_out) {
-            const __nv_bfloat16* B = reinterpret_cast<const __nv_bfloat16*>(a.proj[p].B[e]);
-            cp_async16(smem + (dst - sbase), B + (size_t)(c0 + nn) * re + c8 * 8);
-          } else {
-            st_shared_zero16(dst);
-          }
-        }
-        cp_async_wait_all();
-        fence_proxy_async();                       // Bcat is read by the tensor core (async proxy)
-        mbar_arrive(bar_bfull);
+        if (!mbar_wait(bar_bempty, (nb - 1) & 1)) { abort = true; break; }
+        load_bcat(p, c0);
       }
       const int vb = vg;
       if (!mbar_wait(bar_vc, uses & 1)) { abort = true; break; }

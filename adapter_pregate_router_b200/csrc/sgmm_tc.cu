@@ -182,33 +182,49 @@ __global__ void __launch_bounds__(SH_BLOCK, 1) tc_shrink_kernel(const __grid_con
     }
     const uint32_t g0 = gchunk;
     if (worker) {
+      // this thread's copies of every stage of the item, fixed across the stages: four 16-byte
+      // pieces of x rows and up to eight of A rows (source advanced by 64 columns per stage; a
+      // null source is a zero piece: a missing pair or a row past the rank)
+      const __nv_bfloat16* xs[TB_M * 8 / SH_WORKERS];
+      uint32_t xo[TB_M * 8 / SH_WORKERS];
+#pragma unroll
+      for (int m = 0; m < TB_M * 8 / SH_WORKERS; ++m) {   // x rows: 8 lanes per 128-byte row segment
+        const int w = tid + m * SH_WORKERS;
+        const int row = w >> 3, q = w & 7;
+        const int tk = s_tok[row];
+        xs[m] = tk >= 0 ? x + (size_t)tk * d_in + q * 8 : nullptr;
+        xo[m] = (uint32_t)row * 128 + (uint32_t)((q ^ (row & 7)) << 4);
+      }
+      constexpr int AMAX = TB_MAXN1 * 8 / SH_WORKERS;
+      const __nv_bfloat16* as[AMAX];
+      uint32_t ao[AMAX];
+#pragma unroll
+      for (int m = 0; m < AMAX; ++m) {
+        const int w = tid + m * SH_WORKERS;
+        const int j = w >> 3, q = w & 7;
+        as[m] = (w < N1 * 8 && s_arow[j]) ? s_arow[j] + q * 8 : nullptr;
+        ao[m] = w < N1 * 8 ? TB_M * 128 + (uint32_t)j * 128 + (uint32_t)((q ^ (j & 7)) << 4) : 0xFFFFFFFFu;
+      }
       for (int c = 0; c < nk && !abort; ++c) {
         const uint32_t g = g0 + c, s = g % S;
         if (g >= (uint32_t)S && !mbar_wait(bar_empty + 8 * s, ((g / S) - 1) & 1)) { abort = true; break; }
         const uint32_t st_base = sbase + s * L.stage_bytes;
+        const size_t col = (size_t)c * TB_BK;
 #pragma unroll
-        for (int m = 0; m < TB_M * 8 / SH_WORKERS; ++m) {   // x rows: 8 lanes per 128-byte row segment
-          const int w = tid + m * SH_WORKERS;
-          const int row = w >> 3, q = w & 7;
-          const int tk = s_tok[row];
-          if (tk >= 0)
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(st_base + (uint32_t)row * 128 +
-                                                                            (uint32_t)((q ^ (row & 7)) << 4)),
-                         "l"(x + (size_t)tk * d_in + (size_t)c * TB_BK + q * 8)
+        for (int m = 0; m < TB_M * 8 / SH_WORKERS; ++m)
+          if (xs[m])
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(st_base + xo[m]), "l"(xs[m] + col)
                          : "memory");
-        }
         // A rows: real rows by cp.async; rows past a rank are zeros, written with plain stores
         // on the stage's first use in this item (no later copy touches them)
-        const uint32_t abase = st_base + TB_M * 128;
-        for (int w = tid; w < N1 * 8; w += SH_WORKERS) {
-          const int j = w >> 3, q = w & 7;
-          const __nv_bfloat16* src = s_arow[j];
-          const uint32_t dst = abase + (uint32_t)j * 128 + (uint32_t)((q ^ (j & 7)) << 4);
-          if (src)
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src + (size_t)c * TB_BK + q * 8)
+#pragma unroll
+        for (int m = 0; m < AMAX; ++m) {
+          if (ao[m] == 0xFFFFFFFFu) continue;
+          if (as[m])
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(st_base + ao[m]), "l"(as[m] + col)
                          : "memory");
           else if (c < S)
-            st_shared_zero16(dst);
+            st_shared_zero16(st_base + ao[m]);
         }
         if (c < S) fence_proxy_async();
         cp_async_arrive(bar_full + 8 * s);

@@ -71,6 +71,10 @@ __device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
 }
+// Raise the barrier's expected transaction bytes without an arrival.
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
 // TMA: four rows (y0..y3) x one 64-column box of a 2-D tensor map, into / out of
 // four consecutive 128-byte (swizzled) shared rows.  Row coordinates past the
 // tensor's end load zeros; stores are only issued for rows that exist.

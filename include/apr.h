@@ -26,8 +26,13 @@
  *     and the offending rows are skipped; they never trap.  Read and clear
  *     that word with apr_stream_status().
  *   - Kernels are launched with programmatic dependent launch allowed: each
- *     waits for its predecessor on the stream before touching any input, so
- *     stream order is kept; consecutive calls may overlap their launch.
+ *     waits for its predecessor on the stream before touching activations,
+ *     routing, outputs or the workspace, so stream order is kept and
+ *     consecutive calls may overlap their launch.  Adapter weights (A, B) and
+ *     ranks, which no kernel of this library writes, may be read before that
+ *     wait; a caller that rewrites them with its own kernel just before a call
+ *     on the same stream must not let that kernel signal its dependents early
+ *     (griddepcontrol.launch_dependents).
  *   - Layouts are row-major and dense.  Element type is given by `dtype`
  *     (APR_F32 or APR_BF16) for activations and adapter weights; router
  *     logits are accumulated and gates are produced in fp32.

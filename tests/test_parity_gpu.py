@@ -99,6 +99,32 @@ def test_sgmm_large_batch_unstaged_plan(apr, kernel):
     close(got[0], oracle_group(x, As, Bs, idx, gate.astype(np.float64), ybs)[0], f"{kernel} T=40000")
 
 
+def test_segments_first_call_in_a_fresh_process(apr):
+    """The segment kernel's shared-memory limit must be set by the call that needs it, not left
+    over from an earlier, larger call in the same process (2500 tokens x 2: the staged plan plus
+    the kernel's static shared memory pass the 48 KB default while the dynamic part alone does not)."""
+    import subprocess
+    import sys
+    import os
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    code = (
+        "import numpy as np, torch\n"
+        "from adapter_pregate_router_b200 import apr\n"
+        "from oracle import apr_oracle as O\n"
+        "rng = np.random.default_rng(3)\n"
+        "idx = np.stack([rng.permutation(12)[:2] for _ in range(2500)]).astype(np.int32)\n"
+        "ws = apr.workspace(2500, 2, 12, 16, 64)\n"
+        "seg = torch.empty(13, dtype=torch.int32, device='cuda')\n"
+        "perm = torch.empty(5000, dtype=torch.int32, device='cuda')\n"
+        "apr.segment_tokens(torch.from_numpy(idx).cuda(), 12, seg, perm, ws)\n"
+        "apr.stream_status(ws)\n"
+        "rs, rp = O.segment_tokens(idx, 12)\n"
+        "assert np.array_equal(seg.cpu().numpy(), rs) and np.array_equal(perm.cpu().numpy(), rp)\n"
+        "print('ok')\n")
+    r = subprocess.run([sys.executable, "-c", code], cwd=root, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stderr[-2000:]
+
+
 def test_segments_skewed_and_empty(apr):
     # one adapter takes almost everything, several are empty
     idx = np.zeros((3000, 1), np.int32)

@@ -387,43 +387,68 @@ __global__ void __launch_bounds__(SEG_THREADS) segment_kernel(const int32_t* __r
       }
       __syncthreads();
       if (tid == 0) {
-        MixTile cur = s_cur;
+        // the open tile: start, length and its adapters u0 < u1 < u2 < u3 (INT_MAX: unused),
+        // all in registers
+        int cstart = s_cur.start, clen = s_cur.len, nu = s_cur.nu;
+        int u0 = nu > 0 ? s_cur.u[0] : INT_MAX, u1 = nu > 1 ? s_cur.u[1] : INT_MAX;
+        int u2 = nu > 2 ? s_cur.u[2] : INT_MAX, u3 = nu > 3 ? s_cur.u[3] : INT_MAX;
         int nm = s_nm;
         const int n = min(MIX_CHUNK, nst - c0);
         for (int j = 0; j < n; ++j) {
           const int4 t = s_st[j];
           int remaining = t.y, pos = t.x;
+          // adapters of this set not yet in the tile (a1 < 0 when k == 1)
+          const bool new0 = t.z != u0 && t.z != u1 && t.z != u2 && t.z != u3;
+          const bool new1 = t.w >= 0 && t.w != t.z && t.w != u0 && t.w != u1 && t.w != u2 && t.w != u3;
+          const int add = (int)new0 + (int)new1;
           while (remaining > 0) {
-            // the union with this set
-            int u[kMixAdapters + 2], nu = cur.nu;
-            for (int q = 0; q < cur.nu; ++q) u[q] = cur.u[q];
-            const int add[2] = {t.z, t.w};
-            for (int q = 0; q < k; ++q) {
-              bool found = false;
-              for (int w = 0; w < nu; ++w) found |= (u[w] == add[q]);
-              if (!found) {
-                int w = nu++;                  // insert keeping ascending order
-                while (w > 0 && u[w - 1] > add[q]) { u[w] = u[w - 1]; --w; }
-                u[w] = add[q];
+            const bool fits = clen == 0 || (nu + add <= kMixAdapters && clen < kSetTile);
+            if (!fits) {                          // close the tile; this set opens the next one
+              MixTile mt;
+              mt.start = cstart;
+              mt.len = clen;
+              mt.nu = nu;
+              mt.pad = 0;
+              mt.u[0] = u0; mt.u[1] = u1; mt.u[2] = u2; mt.u[3] = u3;
+              for (int q = nu; q < kMixAdapters; ++q) mt.u[q] = 0;
+              mtiles[nm++] = mt;
+              clen = 0;
+              nu = 0;
+              u0 = u1 = u2 = u3 = INT_MAX;
+            }
+            if (clen == 0) {
+              cstart = pos;
+              // a fresh tile holds exactly this set's adapters
+              nu = 0;
+              u0 = u1 = u2 = u3 = INT_MAX;
+            }
+            if (clen == 0 || new0 || new1) {
+              // sorted insert of the set's adapters not yet present (branch-free over 4 registers)
+              const int vs[2] = {t.z, t.w};
+#pragma unroll
+              for (int q = 0; q < 2; ++q) {
+                const int v = vs[q];
+                const bool present = v == u0 || v == u1 || v == u2 || v == u3;
+                if (v >= 0 && !present) {
+                  const int n3 = min(u3, max(u2, v)), n2 = min(u2, max(u1, v)), n1 = min(u1, max(u0, v));
+                  u0 = min(u0, v);
+                  u1 = n1;
+                  u2 = n2;
+                  u3 = n3;
+                  ++nu;
+                }
               }
             }
-            if (cur.len > 0 && (nu > kMixAdapters || cur.len == kSetTile)) {
-              mtiles[nm++] = cur;              // close the tile, start a new one here
-              cur.start = pos;
-              cur.len = 0;
-              cur.nu = 0;
-              continue;
-            }
-            const int take = min(remaining, kSetTile - cur.len);
-            if (cur.len == 0) cur.start = pos;
-            cur.len += take;
-            cur.nu = nu;
-            for (int q = 0; q < nu; ++q) cur.u[q] = u[q];
+            const int take = min(remaining, kSetTile - clen);
+            clen += take;
             remaining -= take;
             pos += take;
           }
         }
-        s_cur = cur;
+        s_cur.start = cstart;
+        s_cur.len = clen;
+        s_cur.nu = nu;
+        s_cur.u[0] = u0; s_cur.u[1] = u1; s_cur.u[2] = u2; s_cur.u[3] = u3;
         s_nm = nm;
       }
     }

@@ -113,20 +113,29 @@ def measured_traffic(workload):
     return float(ent["bytes_per_call"])
 
 
-def ingest_traffic(csv_path, workload, calls, command):
+def ingest_traffic(csv_path, workload, calls, command, kernels=None, last=0):
     """Record an ncu launch capture (``--metrics dram__bytes_read.sum,dram__bytes_write.sum``,
     ``--csv``) as the DRAM bytes per SGMM call of ``workload``: the sum over the captured launches
+    (those whose kernel name matches the regex ``kernels``, the last ``last`` of them when given)
     divided by ``calls``, keyed to the current kernel-source hash."""
     import csv
-    tot = 0.0
+    import re
     with open(csv_path) as f:
         rows = [r for r in csv.reader(l for l in f if l.startswith('"'))]
     head = rows[0]
     im, iv, iu = head.index("Metric Name"), head.index("Metric Value"), head.index("Metric Unit")
+    ik, iid = head.index("Kernel Name"), head.index("ID")
     scale = {"byte": 1.0, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}
+    per_launch = {}
     for r in rows[1:]:
+        if kernels and not re.search(kernels, r[ik]):
+            continue
         if r[im] in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
-            tot += float(r[iv].replace(",", "")) * scale.get(r[iu], 1.0)
+            per_launch[int(r[iid])] = per_launch.get(int(r[iid]), 0.0) + float(r[iv].replace(",", "")) * scale.get(r[iu], 1.0)
+    ids = sorted(per_launch)
+    if last:
+        ids = ids[-last:]
+    tot = sum(per_launch[i] for i in ids)
     path = os.path.join(ROOT, TRAFFIC_FILE)
     d = {"note": "DRAM bytes per SGMM call from ncu launch captures (dram__bytes_read.sum + "
                  "dram__bytes_write.sum over the captured launches / calls); written by bench.py --ingest-traffic",
@@ -618,11 +627,13 @@ def main():
                     help="build only this many layers (a reduced workload for profiling; not the benchmark)")
     ap.add_argument("--ingest-traffic", metavar="CSV",
                     help="record an ncu DRAM capture of --workload as bytes per call (with --calls, --command)")
-    ap.add_argument("--calls", type=int, default=1)
+    ap.add_argument("--calls", type=float, default=1.0)
     ap.add_argument("--command", default="")
+    ap.add_argument("--kernels", default=None, help="regex of the kernel names to ingest")
+    ap.add_argument("--last", type=int, default=0, help="ingest only the last N matching launches")
     args = ap.parse_args()
     if args.ingest_traffic:
-        print(ingest_traffic(args.ingest_traffic, args.workload, args.calls, args.command))
+        print(ingest_traffic(args.ingest_traffic, args.workload, args.calls, args.command, args.kernels, args.last))
         return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

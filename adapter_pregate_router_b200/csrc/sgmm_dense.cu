@@ -17,8 +17,11 @@
 //          on the preceding launch) and of x (after it) in 128B-swizzled
 //          K-major tiles, and one thread issues the tcgen05 MMAs
 //          D[NR x Tp] = A_slice . x_slice^T (A as the M side, tokens as N).
-//          The cluster's partial products are summed in a fixed order
-//          through distributed shared memory, gated
+//          The MMAs of the two halves of the K slice are issued by two
+//          threads into two accumulators.  The cluster's partial products
+//          are summed in a fixed order through distributed shared memory
+//          (one rank-row tile: each CTA sends every owner its rows by one
+//          bulk copy that completes on the owner's own mbarrier), gated
 //          V[t, e*Rp + i] = sum_j [idx[t,j] = e] g[t,j] U[e*Rp + i, t]
 //          and written as fp32 partials per cluster: [proj][cluster][Tp][NR];
 //          when one cluster spans all of d_in, the final V is written instead,
@@ -26,7 +29,8 @@
 //  expand  one CTA per 128 output columns: D[128 x Tp] = Bslice . V^T with
 //          Bslice[n, e*Rp + i] = B_e[n, i] (staged before the wait, with the
 //          y_base columns) and V summed over the clusters in order and split
-//          into bf16 hi + lo halves (two MMAs keep ~16 mantissa bits of v),
+//          into bf16 hi + lo halves (two MMA chains, issued by two threads
+//          into two accumulators, keep ~16 mantissa bits of v),
 //          or, with a single cluster, V fetched as is by two bulk copies.
 //          Thread n reads row n of D from TMEM and writes
 //          y[t, n] = y_base[t, n] + D[n, t], rounded to bf16 once.
@@ -104,24 +108,34 @@ __global__ void __launch_bounds__(DN_THREADS, 1) dense_shrink_kernel(const __gri
   const int k0 = (cl * CLT + rank) * DN_KC;
 
   // shared memory: A slice [4 atoms][MR][128 B], x slice [4 atoms][Tp][128 B];
-  // after the MMAs the A area holds this CTA's partial product P[Tp][MR] fp32.
+  // after the MMAs the A area holds this CTA's partial product: P[Tp][MR] fp32, or with one
+  // M tile P[MR][Tp + 4] (row-major, padded: owner o's rows form one contiguous block).
   unsigned char* sA = smem;
   unsigned char* sX = smem + (size_t)MR * 512;
-  // MR == 128: partial rows pushed here by the cluster's CTAs, [source rank][Tp][MR / 8] fp32
+  constexpr int TS = TP + 4;                        // row stride of P and red with one M tile
+  constexpr int RS = MR / CLT;                      // rank rows owned per CTA (8, 16 or 32)
+  // MR == 128: each source CTA's block of this CTA's rows lands here, [source rank][RS][TS] fp32
   float* red = reinterpret_cast<float*>(sX + (size_t)Tp * 512);
-  unsigned char* meta = sX + (size_t)Tp * 512 + (MR == 128 ? (size_t)Tp * MR * 4 : 0);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(meta);
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(meta + 8);
-  const __nv_bfloat16** s_Ap = reinterpret_cast<const __nv_bfloat16**>(meta + 16);   // [E]
-  int* s_rk = reinterpret_cast<int*>(meta + 16 + 8 * 16);                             // [E]
+  unsigned char* meta = sX + (size_t)Tp * 512 + (MR == 128 ? (size_t)TS * MR * 4 : 0);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(meta);                                  // [0] MMAs [1] rows in
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(meta + 16);
+  const __nv_bfloat16** s_Ap = reinterpret_cast<const __nv_bfloat16**>(meta + 32);   // [E]
+  int* s_rk = reinterpret_cast<int*>(meta + 32 + 8 * 16);                             // [E]
   int* s_idx = s_rk + 16;                                                              // [T*K]
   float* s_gate = reinterpret_cast<float*>(s_idx + 64 * APR_MAX_K);                   // [T*K]
   float* P = reinterpret_cast<float*>(sA);
 
+  // one M tile: the K slice's two halves go to two accumulators, issued by two threads
+  constexpr int NACC = MR == 128 ? 2 : 1;
+  // let the next kernel of the stream start staging its weights now: its CTAs still wait for this
+  // grid to finish before they read anything it writes (griddepcontrol.wait)
+  pdl_trigger();
   const uint32_t cs = tmem_cols_for(Tp);            // TMEM columns per M tile (a power of two)
-  const uint32_t ncols = (uint32_t)(MR / 128) * cs;
+  const uint32_t ncols = (uint32_t)(NACC * MR / 128) * cs;
+  constexpr uint32_t kBlockBytes = (uint32_t)(RS * TS * 4);   // one source's rows for one owner
   if (tid == 0) {
-    mbar_init(smem_u32(bar), 1);
+    mbar_init(smem_u32(bar), NACC);
+    mbar_init(smem_u32(bar + 1), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 0) tmem_alloc(smem_u32(s_tmem), ncols);
@@ -136,6 +150,12 @@ __global__ void __launch_bounds__(DN_THREADS, 1) dense_shrink_kernel(const __gri
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
+  if constexpr (MR == 128) {
+    // the CLT blocks of this CTA's rows are expected as transaction bytes; every CTA's barrier is
+    // initialised before any peer's copy can target it (cluster barrier, before the PDL wait)
+    if (tid == 0) mbar_arrive_expect_tx(smem_u32(bar + 1), (uint32_t)CLT * kBlockBytes);
+    cluster_sync_all();
+  }
 
   // A slice of every adapter (rows beyond a rank, or columns beyond d_in, are zeros)
   {
@@ -156,7 +176,6 @@ __global__ void __launch_bounds__(DN_THREADS, 1) dense_shrink_kernel(const __gri
   }
 
   pdl_wait();
-  pdl_trigger();
 
   // x slice of the tokens, and their routing
   {
@@ -179,16 +198,20 @@ __global__ void __launch_bounds__(DN_THREADS, 1) dense_shrink_kernel(const __gri
   fence_proxy_async();
   __syncthreads();
 
-  // D[MR x Tp] = A_slice . x_slice^T, one M tile of 128 rows at a time
-  if (tid == 0) {
+  // D[MR x Tp] = A_slice . x_slice^T, one M tile of 128 rows at a time; with one M tile, thread 0
+  // issues the first half of the K steps into accumulator 0 and thread 32 the second half into
+  // accumulator 1 (columns cs..)
+  if (tid == 0 || (NACC == 2 && tid == 32)) {
     tc_fence_after();
     const uint32_t id = idesc_bf16(128, Tp);
+    const int h = tid >> 5;
+    constexpr int KS = DN_KC / 16 / NACC;            // K steps per issuing thread
     for (int mt = 0; mt < MR / 128; ++mt)
-      for (int kk = 0; kk < DN_KC / 16; ++kk) {
+      for (int kk = h * KS; kk < (h + 1) * KS; ++kk) {
         const uint32_t aa = smem_u32(sA) + (uint32_t)(kk >> 2) * (uint32_t)(MR * 128) + (uint32_t)mt * 16384 +
                             (uint32_t)(kk & 3) * 32;
         const uint32_t bb = smem_u32(sX) + (uint32_t)(kk >> 2) * (uint32_t)(Tp * 128) + (uint32_t)(kk & 3) * 32;
-        mma_bf16(tmem + (uint32_t)mt * cs, desc_k_sw128(aa), desc_k_sw128(bb), id, kk > 0 ? 1u : 0u);
+        mma_bf16(tmem + (uint32_t)(h + mt) * cs, desc_k_sw128(aa), desc_k_sw128(bb), id, kk > h * KS ? 1u : 0u);
       }
     mma_commit(smem_u32(bar));
   }
@@ -198,19 +221,17 @@ __global__ void __launch_bounds__(DN_THREADS, 1) dense_shrink_kernel(const __gri
     if (tid == 0) report(a.ws, APR_ERR_TIMEOUT, K_SHRINK, (int)blockIdx.x);
   } else {
     if constexpr (MR == 128) {
-      // push: row r of the partial product goes to the CTA that owns it (rank r / (128 / CLT))
+      // row r of the partial product (the two accumulators summed) -> P[r][0 .. Tp) (the A slice
+      // is no longer read); owner o's rows o*RS .. are then one contiguous block
       const int wq = warp & 3, wg = warp >> 2;
       const int r = wq * 32 + lane;
-      const int owner = r / (MR / CLT), ri = r % (MR / CLT);
       for (int c8 = wg; c8 < Tp / 8; c8 += 2) {
-        float v[8];
-        tmem_ld8(tmem + ((uint32_t)(wq * 32) << 16) + (uint32_t)(c8 * 8), v);
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int t = c8 * 8 + u;
-          const uint32_t off = smem_u32(red + ((size_t)(rank * Tp + t) * (MR / CLT) + ri));
-          st_cluster_f32(cluster_map(off, (uint32_t)owner), v[u]);
-        }
+        float v0[8], v1[8];
+        tmem_ld8(tmem + ((uint32_t)(wq * 32) << 16) + (uint32_t)(c8 * 8), v0);
+        tmem_ld8(tmem + ((uint32_t)(wq * 32) << 16) + cs + (uint32_t)(c8 * 8), v1);
+        float4* dst = reinterpret_cast<float4*>(P + (size_t)r * TS + c8 * 8);
+        dst[0] = make_float4(v0[0] + v1[0], v0[1] + v1[1], v0[2] + v1[2], v0[3] + v1[3]);
+        dst[1] = make_float4(v0[4] + v1[4], v0[5] + v1[5], v0[6] + v1[6], v0[7] + v1[7]);
       }
     } else {
       // TMEM -> P[t][r] (the A slice is no longer read)
@@ -228,11 +249,30 @@ __global__ void __launch_bounds__(DN_THREADS, 1) dense_shrink_kernel(const __gri
     }
   }
   tc_fence_before();
-  cluster_sync_all();          // every CTA's partial rows are in place
+  bool rows_in = true;
+  if constexpr (MR == 128) {
+    // every owner gets its block of this CTA's rows by one bulk copy into red[rank], completing
+    // as transaction bytes on the owner's barrier; then this CTA waits for its own CLT blocks
+    fence_proxy_async();                     // P's generic writes are visible to the copies
+    __syncthreads();
+    if (tid < CLT) {
+      const uint32_t src = smem_u32(P) + (uint32_t)tid * kBlockBytes;
+      const uint32_t dst = cluster_map(smem_u32(red) + (uint32_t)rank * kBlockBytes, (uint32_t)tid);
+      const uint32_t rb = cluster_map(smem_u32(bar + 1), (uint32_t)tid);
+      asm volatile(
+          "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+          "r"(src), "r"(kBlockBytes), "r"(rb)
+          : "memory");
+      bulk_commit();
+    }
+    rows_in = mbar_wait(smem_u32(bar + 1), 0);
+    if (!rows_in && tid == 0) report(a.ws, APR_ERR_TIMEOUT, K_SHRINK, (int)blockIdx.x);
+  } else {
+    cluster_sync_all();        // every CTA's partial product is in place
+  }
 
   // this CTA's share of the rows, summed over the cluster in rank order, gated
-  {
-    constexpr int RS = MR / CLT;             // rows per CTA (8, 16 or 32)
+  if (rows_in) {
     constexpr int groups = RS / 4;
     float* vpart = ws_at<float>(a.ws, args.vpart_off) + ((size_t)(p * args.ncl + cl) * Tp) * NR;
     constexpr int PER = (groups * TP + DN_THREADS - 1) / DN_THREADS;   // float4 groups per thread (1 or 2)
@@ -244,8 +284,10 @@ __global__ void __launch_bounds__(DN_THREADS, 1) dense_shrink_kernel(const __gri
         const int t = w / groups, g4 = w % groups;
         if constexpr (MR == 128) {
 #pragma unroll
-          for (int c = 0; c < CLT; ++c)
-            part[u][c] = *reinterpret_cast<const float4*>(red + ((size_t)(c * Tp + t) * RS + g4 * 4));
+          for (int c = 0; c < CLT; ++c) {
+            const float* blk = red + (size_t)c * RS * TS + (size_t)(g4 * 4) * TS + t;
+            part[u][c] = make_float4(blk[0], blk[TS], blk[2 * TS], blk[3 * TS]);
+          }
         } else {
           const uint32_t off = smem_u32(P + (size_t)t * MR + rank * RS + g4 * 4);
 #pragma unroll
@@ -300,6 +342,9 @@ __global__ void __launch_bounds__(DN_THREADS, 1) dense_shrink_kernel(const __gri
     }
   }
   if constexpr (MR != 128) cluster_wait();   // every CTA's reads of this CTA's P are over before it leaves
+  if constexpr (MR == 128) {
+    if (tid < CLT) bulk_wait_read_all();     // this CTA's outgoing copies have read P
+  }
   if (warp == 0) tmem_dealloc(tmem, ncols);
 }
 
@@ -333,9 +378,11 @@ __global__ void __launch_bounds__(DN_THREADS, 1) dense_expand_kernel(const __gri
   const __nv_bfloat16** s_Bp = reinterpret_cast<const __nv_bfloat16**>(meta + 32);   // [E]
   int* s_rk = reinterpret_cast<int*>(meta + 32 + 8 * 16);                             // [E]
 
-  const uint32_t ncols = tmem_cols_for(Tp);
+  pdl_trigger();                                     // as in the shrink: the next kernel may stage early
+  const uint32_t cs = tmem_cols_for(Tp);
+  const uint32_t ncols = 2 * cs;                     // the hi and lo products in two accumulators
   if (tid == 0) {
-    mbar_init(smem_u32(bar), 1);
+    mbar_init(smem_u32(bar), 2);
     mbar_init(smem_u32(bar + 1), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -372,7 +419,6 @@ __global__ void __launch_bounds__(DN_THREADS, 1) dense_expand_kernel(const __gri
   }
 
   pdl_wait();
-  pdl_trigger();
 
   if (args.direct) {
     // the final V, already in the MMA layout: two contiguous bulk copies on the V barrier
@@ -452,16 +498,16 @@ __global__ void __launch_bounds__(DN_THREADS, 1) dense_expand_kernel(const __gri
   __syncthreads();
 
   bool vready = true;
-  if (args.direct && tid == 0) vready = mbar_wait(smem_u32(bar + 1), 0);
-  if (tid == 0 && vready) {
+  const bool issuer = tid == 0 || tid == 32;         // thread 0: B . V_hi^T, thread 32: B . V_lo^T
+  if (args.direct && issuer) vready = mbar_wait(smem_u32(bar + 1), 0);
+  if (issuer && vready) {
     tc_fence_after();
     const uint32_t id = idesc_bf16(128, Tp);
+    const int h = tid >> 5;
+    const uint32_t sv = h ? smem_u32(sVL) : smem_u32(sVH);
     for (int kk = 0; kk < NR / 16; ++kk)
-      mma_bf16(tmem, desc_k_plain(smem_u32(sB) + kk * 256, 128, SBO), desc_k_plain(smem_u32(sVH) + kk * 256, 128, SBO),
-               id, kk > 0 ? 1u : 0u);
-    for (int kk = 0; kk < NR / 16; ++kk)
-      mma_bf16(tmem, desc_k_plain(smem_u32(sB) + kk * 256, 128, SBO), desc_k_plain(smem_u32(sVL) + kk * 256, 128, SBO),
-               id, 1u);
+      mma_bf16(tmem + (uint32_t)h * cs, desc_k_plain(smem_u32(sB) + kk * 256, 128, SBO),
+               desc_k_plain(sv + kk * 256, 128, SBO), id, kk > 0 ? 1u : 0u);
     mma_commit(smem_u32(bar));
   }
   const bool done = __syncthreads_and(vready) && mbar_wait(smem_u32(bar), 0);
@@ -474,12 +520,14 @@ __global__ void __launch_bounds__(DN_THREADS, 1) dense_expand_kernel(const __gri
     const int wq = warp & 3, wg = warp >> 2;
     const int n = wq * 32 + lane;
     for (int c8 = wg; c8 < Tp / 8; c8 += 2) {
-      float v[8];
+      float v[8], vl[8];
       tmem_ld8(tmem + ((uint32_t)(wq * 32) << 16) + (uint32_t)(c8 * 8), v);
+      tmem_ld8(tmem + ((uint32_t)(wq * 32) << 16) + cs + (uint32_t)(c8 * 8), vl);
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         const int t = c8 * 8 + u;
-        if (t < T) sYB[(size_t)t * DN_NT + n] = __float2bfloat16_rn(__bfloat162float(sYB[(size_t)t * DN_NT + n]) + v[u]);
+        if (t < T)
+          sYB[(size_t)t * DN_NT + n] = __float2bfloat16_rn(__bfloat162float(sYB[(size_t)t * DN_NT + n]) + (v[u] + vl[u]));
       }
     }
   }
@@ -507,7 +555,7 @@ bool sgmm_dense_supported(const SgmmArgs& a, int dtype) {
 }
 
 static size_t shrink_smem(int MR, int Tp) {
-  return (size_t)MR * 512 + (size_t)Tp * 512 + (MR == 128 ? (size_t)Tp * MR * 4 : 0) + 16 + 8 * 16 + 4 * 16 +
+  return (size_t)MR * 512 + (size_t)Tp * 512 + (MR == 128 ? (size_t)(Tp + 4) * MR * 4 : 0) + 32 + 8 * 16 + 4 * 16 +
          8 * 64 * APR_MAX_K + 1024;
 }
 static size_t expand_smem(int NR, int Tp) {

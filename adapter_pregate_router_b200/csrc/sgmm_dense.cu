@@ -223,15 +223,32 @@ __global__ void __launch_bounds__(DN_THREADS, 1) dense_shrink_kernel(const __gri
     if constexpr (MR == 128) {
       // row r of the partial product (the two accumulators summed) -> P[r][0 .. Tp) (the A slice
       // is no longer read); owner o's rows o*RS .. are then one contiguous block
+      // (this warp's column groups of both accumulators are all loaded before one wait)
       const int wq = warp & 3, wg = warp >> 2;
       const int r = wq * 32 + lane;
-      for (int c8 = wg; c8 < Tp / 8; c8 += 2) {
-        float v0[8], v1[8];
-        tmem_ld8(tmem + ((uint32_t)(wq * 32) << 16) + (uint32_t)(c8 * 8), v0);
-        tmem_ld8(tmem + ((uint32_t)(wq * 32) << 16) + cs + (uint32_t)(c8 * 8), v1);
-        float4* dst = reinterpret_cast<float4*>(P + (size_t)r * TS + c8 * 8);
-        dst[0] = make_float4(v0[0] + v1[0], v0[1] + v1[1], v0[2] + v1[2], v0[3] + v1[3]);
-        dst[1] = make_float4(v0[4] + v1[4], v0[5] + v1[5], v0[6] + v1[6], v0[7] + v1[7]);
+      constexpr int NG = (TP / 8 + 1) / 2;
+      const uint32_t lb = tmem + ((uint32_t)(wq * 32) << 16);
+      uint32_t v0[NG][8], v1[NG][8];
+#pragma unroll
+      for (int gi = 0; gi < NG; ++gi) {
+        const int c8 = wg + 2 * gi;
+        if (c8 < TP / 8) {
+          tmem_ld8_async(lb + (uint32_t)(c8 * 8), v0[gi]);
+          tmem_ld8_async(lb + cs + (uint32_t)(c8 * 8), v1[gi]);
+        }
+      }
+      tmem_ld_wait();
+#pragma unroll
+      for (int gi = 0; gi < NG; ++gi) {
+        const int c8 = wg + 2 * gi;
+        if (c8 < TP / 8) {
+          tmem_ld_tie(v0[gi]);
+          tmem_ld_tie(v1[gi]);
+          const auto f = [&](int u) { return __uint_as_float(v0[gi][u]) + __uint_as_float(v1[gi][u]); };
+          float4* dst = reinterpret_cast<float4*>(P + (size_t)r * TS + c8 * 8);
+          dst[0] = make_float4(f(0), f(1), f(2), f(3));
+          dst[1] = make_float4(f(4), f(5), f(6), f(7));
+        }
       }
     } else {
       // TMEM -> P[t][r] (the A slice is no longer read)
@@ -517,17 +534,38 @@ __global__ void __launch_bounds__(DN_THREADS, 1) dense_expand_kernel(const __gri
   } else {
     // thread n holds D[n][t] for its column: y_base[t, n] + D[n, t] in place in shared memory,
     // then whole 16-byte row pieces go out
+    // (all TMEM loads of the warp before one wait; each group's y_base values are read before
+    // any of them is written)
     const int wq = warp & 3, wg = warp >> 2;
     const int n = wq * 32 + lane;
-    for (int c8 = wg; c8 < Tp / 8; c8 += 2) {
-      float v[8], vl[8];
-      tmem_ld8(tmem + ((uint32_t)(wq * 32) << 16) + (uint32_t)(c8 * 8), v);
-      tmem_ld8(tmem + ((uint32_t)(wq * 32) << 16) + cs + (uint32_t)(c8 * 8), vl);
+    constexpr int NG = (TP / 8 + 1) / 2;
+    const uint32_t lb = tmem + ((uint32_t)(wq * 32) << 16);
+    uint32_t vh[NG][8], vl[NG][8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int t = c8 * 8 + u;
-        if (t < T)
-          sYB[(size_t)t * DN_NT + n] = __float2bfloat16_rn(__bfloat162float(sYB[(size_t)t * DN_NT + n]) + (v[u] + vl[u]));
+    for (int gi = 0; gi < NG; ++gi) {
+      const int c8 = wg + 2 * gi;
+      if (c8 < TP / 8) {
+        tmem_ld8_async(lb + (uint32_t)(c8 * 8), vh[gi]);
+        tmem_ld8_async(lb + cs + (uint32_t)(c8 * 8), vl[gi]);
+      }
+    }
+    tmem_ld_wait();
+#pragma unroll
+    for (int gi = 0; gi < NG; ++gi) {
+      const int c8 = wg + 2 * gi;
+      if (c8 < TP / 8) {
+        tmem_ld_tie(vh[gi]);
+        tmem_ld_tie(vl[gi]);
+        float yv[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) yv[u] = __bfloat162float(sYB[(size_t)(c8 * 8 + u) * DN_NT + n]);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int t = c8 * 8 + u;
+          if (t < T)
+            sYB[(size_t)t * DN_NT + n] =
+                __float2bfloat16_rn(yv[u] + (__uint_as_float(vh[gi][u]) + __uint_as_float(vl[gi][u])));
+        }
       }
     }
   }

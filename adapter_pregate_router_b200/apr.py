@@ -59,6 +59,11 @@ class Proj(ctypes.Structure):
     _fields_ = [("y", _vp), ("y_base", _vp), ("d_out", _i), ("A", _vp), ("B", _vp)]
 
 
+class LinearProj(ctypes.Structure):
+    """apr_linear_proj"""
+    _fields_ = [("W", _vp), ("y", _vp), ("d_out", _i), ("A", _vp), ("B", _vp)]
+
+
 class MergeProj(ctypes.Structure):
     """apr_merge_proj"""
     _fields_ = [("W", _vp), ("Wp", _vp), ("d_in", _i), ("d_out", _i), ("A", _vp), ("B", _vp)]
@@ -78,6 +83,9 @@ _pregate_route_noalloc = _sig("apr_pregate_route_noalloc", _i, [_vp, _vp, _i, _i
 _segment_tokens = _sig("apr_segment_tokens", _i, [_vp, _i, _i, _i, _vp, _vp, _vp, _sz, _vp])
 _sgmm = _sig("apr_sgmm_shrink_expand", _i,
              [_vp, _i, ctypes.POINTER(Proj), _i, _i, _i, _i, _i, _vp, _i, _vp, _vp, _vp, _vp, _vp, _sz, _i, _vp])
+_linear = _sig("apr_linear_lora", _i,
+                [_vp, _i, ctypes.POINTER(LinearProj), _i, _i, _i, _i, _vp, _i, _vp, _vp, _vp, _vp, _vp, _sz, _vp])
+_linear_workspace_size = _sig("apr_linear_workspace_size", _sz, [_i, _i, _i, _i, _i, _i, ctypes.c_long])
 _merge = _sig("apr_merge_adapters", _i, [_vp, _i, _i, _i, _vp, _vp, _i, _vp, _sz, _vp])
 _merge_plan_size = _sig("apr_merge_plan_size", _sz, [_i])
 _merge_plan_init = _sig("apr_merge_plan_init", _i, [_vp, _i, _vp, _sz])
@@ -90,7 +98,7 @@ _kernel_launches = _sig("apr_kernel_launches", ctypes.c_uint64, [])
 
 EXPORTED = ("apr_workspace_size", "apr_workspace_init", "apr_pregate_route", "apr_pregate_route_noalloc",
             "apr_segment_tokens",
-            "apr_sgmm_shrink_expand", "apr_merge_adapters", "apr_merge_plan_size", "apr_merge_plan_init",
+            "apr_sgmm_shrink_expand", "apr_linear_lora", "apr_linear_workspace_size", "apr_merge_adapters", "apr_merge_plan_size", "apr_merge_plan_init",
             "apr_merge_adapters_planned", "apr_gemv", "apr_stream_status",
             "apr_last_error", "apr_status_string", "apr_kernel_launches")
 
@@ -272,6 +280,65 @@ def sgmm_shrink_expand(x, projs, k, E, ranks, max_rank, idx, gate, seg_off, perm
     _check(_sgmm(_ptr(x), d_in, arr, len(projs), _dtype_code(x), T, k, E, _ptr(ranks), max_rank,
                  _ptr(idx), _ptr(gate), _ptr(seg_off), _ptr(perm), _ptr(ws), ws.numel(), kernel,
                  _stream(stream)))
+
+
+def linear_workspace_size(T: int, k: int, E: int, max_rank: int, max_d_in: int, nproj: int,
+                          sum_d_out: int) -> int:
+    return int(_linear_workspace_size(T, k, E, max_rank, max_d_in, nproj, sum_d_out))
+
+
+def linear_workspace(T: int, k: int, E: int, max_rank: int, max_d_in: int, nproj: int, sum_d_out: int,
+                     device="cuda", stream=None):
+    """Allocate (with torch) and initialise a workspace that also serves ``linear_lora`` on
+    groups of up to ``nproj`` projections whose output widths add up to ``sum_d_out``."""
+    n = linear_workspace_size(T, k, E, max_rank, max_d_in, nproj, sum_d_out)
+    if n == 0:
+        raise AprError(APR_ERR_INVALID_ARG, "linear_workspace_size: arguments out of range")
+    ws = torch.empty(n, dtype=torch.uint8, device=device)
+    _check(_workspace_init(ws.data_ptr(), n, _stream(stream)))
+    return ws
+
+
+def make_linear_proj(W, y, A_table, B_table) -> LinearProj:
+    """One projection of a fused group: base weight W [d_out, d_in] bf16, output y [T, d_out]
+    bf16, and the device tables of A and B pointers (int64 [E])."""
+    _need(W, "W", (torch.bfloat16,), ndim=2)
+    d_out, d_in = W.shape
+    _need(y, "y", (torch.bfloat16,), ndim=2)
+    if y.shape[1] != d_out:
+        raise ValueError(f"y has {y.shape[1]} columns, W has {d_out} rows")
+    _need(A_table, "A_table", (torch.int64,), ndim=1)
+    _need(B_table, "B_table", (torch.int64,), shape=tuple(A_table.shape))
+    _same_device(("W", W), ("y", y), ("A_table", A_table), ("B_table", B_table))
+    p = LinearProj(_ptr(W), _ptr(y), int(d_out), _ptr(A_table), _ptr(B_table))
+    p.meta = (int(y.shape[0]), int(d_in), int(A_table.shape[0]), W.device)
+    return p
+
+
+def linear_lora(x, projs, k, E, ranks, max_rank, idx, gate, seg_off, perm, ws, stream=None):
+    """projs: a sequence of ``LinearProj`` (see ``make_linear_proj``) sharing input ``x``:
+    ``y_p = x W_p^T + sum_j gate B_e (A_e x)`` in one contraction per projection."""
+    _need(x, "x", (torch.bfloat16,), ndim=2)
+    T, d_in = x.shape
+    for i, pj in enumerate(projs):
+        meta = getattr(pj, "meta", None)
+        if meta is None:
+            raise TypeError(f"projs[{i}] was not made by make_linear_proj")
+        t_rows, w_in, e_tab, pdev = meta
+        if t_rows != T or w_in != d_in or e_tab < E or pdev != x.device:
+            raise ValueError(f"projs[{i}]: y with {t_rows} rows, W with {w_in} columns, {e_tab} adapters on "
+                             f"{pdev} does not fit x [{T}, {d_in}] with E={E} on {x.device}")
+    _need(ranks, "ranks", (torch.int32,), shape=(E,))
+    _need(idx, "idx", (torch.int32,), shape=(T, k))
+    _need(gate, "gate", (torch.float32,), shape=(T, k))
+    _need(seg_off, "seg_off", (torch.int32,), shape=(E + 1,))
+    _need(perm, "perm", (torch.int32,), ndim=1, min_numel=T * k)
+    _need_ws(ws)
+    _same_device(("x", x), ("ranks", ranks), ("idx", idx), ("gate", gate), ("seg_off", seg_off),
+                 ("perm", perm), ("ws", ws))
+    arr = (LinearProj * len(projs))(*projs)
+    _check(_linear(_ptr(x), d_in, arr, len(projs), T, k, E, _ptr(ranks), max_rank, _ptr(idx), _ptr(gate),
+                   _ptr(seg_off), _ptr(perm), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def _merge_host_table(entries):

@@ -103,6 +103,14 @@ size_t apr_workspace_size(int T, int k, int E, int max_rank, int max_d_in) {
   return L.scratch + align_up(scratch) + kAlign;
 }
 
+size_t apr_linear_workspace_size(int T, int k, int E, int max_rank, int max_d_in, int nproj, long sum_d_out) {
+  const size_t base = apr_workspace_size(T, k, E, max_rank, max_d_in);
+  if (base == 0 || nproj < 1 || nproj > APR_MAX_PROJ || sum_d_out < 8 || sum_d_out > (1L << 30)) return 0;
+  const WsLayout L = ws_layout(T, k, E);
+  const size_t lin = L.scratch + align_up(linear_scratch_bytes(T, k, E, max_rank, nproj, sum_d_out)) + kAlign;
+  return lin > base ? lin : base;
+}
+
 apr_status apr_workspace_init(void* ws, size_t ws_bytes, void* stream) {
   if (ws == nullptr || ws_bytes < sizeof(WsHeader)) return fail(APR_ERR_WORKSPACE, "workspace_init: too small");
   if (reinterpret_cast<uintptr_t>(ws) % kAlign) return fail(APR_ERR_WORKSPACE, "workspace_init: misaligned");
@@ -282,6 +290,68 @@ apr_status apr_merge_adapters_planned(const apr_merge_proj* projs, const void* p
   if (st) return st;
   cudaError_t e = launch_merge_tma(projs, plan, nproj, E, r, idx, gate, k, ws, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "merge launch");
+  return APR_OK;
+}
+
+apr_status apr_linear_lora(const void* x, int d_in, const apr_linear_proj* projs, int nproj, int T,
+                           int k, int E, const int32_t* ranks, int max_rank, const int32_t* idx,
+                           const float* gate, const int32_t* seg_off, const int32_t* perm, void* ws,
+                           size_t ws_bytes, void* stream) {
+  apr_status st = check_route_dims(T, k, E, "linear_lora");
+  if (st) return st;
+  if (nproj < 1 || nproj > APR_MAX_PROJ)
+    return fail(APR_ERR_INVALID_ARG, "linear_lora: nproj=%d outside [1, %d]", nproj, APR_MAX_PROJ);
+  if (!projs) return fail(APR_ERR_INVALID_ARG, "linear_lora: NULL projs");
+  if (d_in < 8 || (d_in & 7)) return fail(APR_ERR_INVALID_ARG, "linear_lora: d_in=%d must be a positive multiple of 8", d_in);
+  if (max_rank < 8 || max_rank > APR_MAX_RANK || (max_rank & 7))
+    return fail(APR_ERR_INVALID_ARG, "linear_lora: max_rank=%d must be a multiple of 8 in [8, %d]", max_rank, APR_MAX_RANK);
+  long sum_d_out = 0;
+  for (int p = 0; p < nproj; ++p) {
+    const apr_linear_proj& pj = projs[p];
+    if (pj.d_out < 8 || (pj.d_out & 7))
+      return fail(APR_ERR_INVALID_ARG, "linear_lora: proj %d d_out=%d must be a positive multiple of 8", p, pj.d_out);
+    if (T > 0 && (!pj.W || !pj.y || !pj.A || !pj.B))
+      return fail(APR_ERR_INVALID_ARG, "linear_lora: proj %d has a NULL pointer", p);
+    if (T > 0 && (!aligned16(pj.W) || !aligned16(pj.y)))
+      return fail(APR_ERR_INVALID_ARG, "linear_lora: proj %d W/y not 16-byte aligned", p);
+    sum_d_out += pj.d_out;
+  }
+  if (T == 0) return APR_OK;
+  if (!x || !ranks || !idx || !gate || !seg_off || !perm) return fail(APR_ERR_INVALID_ARG, "linear_lora: NULL pointer");
+  if (!aligned16(x)) return fail(APR_ERR_INVALID_ARG, "linear_lora: x not 16-byte aligned");
+  const WsLayout L = ws_layout(T, k, E);
+  st = check_ws(ws, ws_bytes, L.scratch + linear_scratch_bytes(T, k, E, max_rank, nproj, sum_d_out), "linear_lora");
+  if (st) return st;
+
+  SgmmArgs a;
+  memset(&a, 0, sizeof(a));
+  const void* W[APR_MAX_PROJ] = {};
+  a.x = x;
+  a.d_in = d_in;
+  a.nproj = nproj;
+  for (int p = 0; p < nproj; ++p) {
+    a.proj[p].y = projs[p].y;
+    a.proj[p].y_base = nullptr;
+    a.proj[p].d_out = projs[p].d_out;
+    a.proj[p].A = projs[p].A;
+    a.proj[p].B = projs[p].B;
+    W[p] = projs[p].W;
+  }
+  a.T = T;
+  a.k = k;
+  a.E = E;
+  a.ranks = ranks;
+  a.max_rank = max_rank;
+  a.idx = idx;
+  a.gate = gate;
+  a.seg_off = seg_off;
+  a.perm = perm;
+  a.ws = ws;
+  if (!linear_lora_supported(a))
+    return fail(APR_ERR_UNSUPPORTED, "linear_lora: needs rank slots of 16/32/64, k<=4, k*R16<=64, E*R16<=256, "
+                                     "d_in%%64==0");
+  cudaError_t e = launch_linear_lora(a, W, L.scratch, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "linear_lora launch");
   return APR_OK;
 }
 

@@ -145,6 +145,25 @@ inline size_t sgmm_scratch_bytes(int T, int k, int E, int max_rank, int d_in) {
   return b;
 }
 
+// Fused base projection + adapters: gated v per pair [proj][pair][R16] bf16, the bank rows
+// V [proj][T][E * R16] bf16, then each projection's Bcat [d_out][E * R16] bf16 (aligned blocks).
+struct LinearScratch {
+  size_t vc, v, bcat;
+};
+inline LinearScratch linear_scratch(int T, int k, int E, int max_rank, int nproj) {
+  const size_t R16 = (size_t)round16i(max_rank);
+  LinearScratch L;
+  L.vc = 0;
+  L.v = align_up((size_t)nproj * T * k * R16 * 2);
+  L.bcat = L.v + align_up((size_t)nproj * T * E * R16 * 2);
+  return L;
+}
+// Bytes for nproj projections whose output widths add up to sum_d_out.
+inline size_t linear_scratch_bytes(int T, int k, int E, int max_rank, int nproj, long sum_d_out) {
+  const LinearScratch L = linear_scratch(T, k, E, max_rank, nproj);
+  return L.bcat + align_up((size_t)sum_d_out * E * round16i(max_rank) * 2) + (size_t)nproj * kAlign;
+}
+
 template <typename P>
 __host__ __device__ inline P* ws_at(void* ws, size_t off) {
   return reinterpret_cast<P*>(reinterpret_cast<char*>(ws) + off);
@@ -233,7 +252,7 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 // Kernel ids used in WsHeader::err_info.
-enum KernelId { K_ROUTE = 1, K_TOPK = 2, K_SEGMENT = 3, K_SHRINK = 4, K_EXPAND = 5, K_MERGE = 6, K_TC = 7 };
+enum KernelId { K_ROUTE = 1, K_TOPK = 2, K_SEGMENT = 3, K_SHRINK = 4, K_EXPAND = 5, K_MERGE = 6, K_TC = 7, K_LINEAR = 8 };
 
 }  // namespace apr
 
@@ -312,6 +331,8 @@ cudaError_t launch_sgmm_tensor(const SgmmArgs& a, size_t scratch_off, cudaStream
 cudaError_t launch_sgmm_dense(const SgmmArgs& a, size_t scratch_off, cudaStream_t s);
 cudaError_t launch_sgmm_bank(const SgmmArgs& a, size_t scratch_off, cudaStream_t s);
 bool sgmm_bank_supported(const SgmmArgs& a, int dtype);
+bool linear_lora_supported(const SgmmArgs& a);
+cudaError_t launch_linear_lora(const SgmmArgs& a, const void* const* W, size_t scratch_off, cudaStream_t s);
 bool sgmm_dense_supported(const SgmmArgs& a, int dtype);
 bool sgmm_tensor_supported(const SgmmArgs& a, int dtype);
 cudaError_t launch_merge(const apr_merge_proj* projs, int nproj, int E, int r, const int32_t* idx,

@@ -1,0 +1,337 @@
+// Base projection and adapters in one tcgen05 contraction:
+//
+//   y[t, :] = x[t, :] W^T + sum_j g_{t,j} B_{e_{t,j}} (A_{e_{t,j}} x[t, :])
+//
+// with one fp32 accumulator and one rounding to bf16 per output element.
+// AdaFuse summary (gist.science), Resumen tecnico §2.B: the selected experts
+// are fused into the backbone in a single pass.  Where the adapter add runs
+// after a separate base GEMM, every output element is written by the GEMM,
+// read back and written again; here the adapter term enters the GEMM's own
+// accumulator, so y is written once and never read.
+//
+// The adapter term is the bank form of the contraction (the bank SGMM kernel
+// uses the same identity):
+//
+//   sum_j g_j B_{e_j} v_j = Bcat V_t,  V[t, e*R16 + r] = g_{t,j} (A_e x_t)[r] if idx[t, j] == e
+//                                      Bcat[n, e*R16 + r] = B_e[n, r]
+//
+// so the whole projection is one GEMM over K = d_in + E*R16:
+//
+//   y = [x | V] [W | Bcat]^T
+//
+// Steps of one call (all on the caller's stream, chained by programmatic
+// dependent launch):
+//  1. the tensor-core shrink (pair order) writes g * A_e x per (token, slot)
+//     in bf16 to the workspace;
+//  2. a pack kernel spreads those rows over the bank's rank slots (V, zeros
+//     where a token did not select an adapter) and lays the projection's B_e
+//     side by side (Bcat), both row-major in the workspace;
+//  3. the GEMM: 128 x 256 output tiles, 64-wide K blocks by 2-D TMA boxes
+//     (128-byte swizzle) into a 4-deep ring, x/W blocks first and V/Bcat
+//     blocks after them; one thread issues the MMAs (M = 128, N = 256) into a
+//     double-buffered TMEM accumulator; four epilogue warps round and store
+//     while the next tile accumulates.  The grid is persistent (one CTA per
+//     SM), tiles ordered row tile fastest so that the CTAs in flight share
+//     W's column block in L2.
+//
+// Every mbarrier wait is bounded (1 s); on expiry the CTA records
+// APR_ERR_TIMEOUT, stops issuing, drains its copies and frees its TMEM.
+#include "apr_internal.cuh"
+#include "tc_ptx.cuh"
+
+#include <algorithm>
+
+namespace apr {
+
+constexpr int LL_BM = 128;                        // tokens per tile (TMEM lanes)
+constexpr int LL_BN = 256;                        // output columns per tile (MMA N)
+constexpr int LL_BK = 64;                         // K per block (one 128-byte swizzle atom)
+constexpr int LL_ST = 4;                          // ring depth
+constexpr int LL_THREADS = 192;                   // warp 0: TMA, warp 1: MMA, warps 2-5: epilogue
+constexpr uint32_t LL_ABYTES = LL_BM * 128;       // 16 KB
+constexpr uint32_t LL_BBYTES = LL_BN * 128;       // 32 KB
+constexpr uint32_t LL_STAGE = LL_ABYTES + LL_BBYTES;
+constexpr uint32_t LL_TMEM_COLS = 512;            // two 256-column accumulators
+constexpr size_t LL_SMEM = (size_t)LL_ST * LL_STAGE + 256 + 1024;
+
+struct LinPlan {
+  CUtensorMap xmap;                      // x [T, d_in]: boxes of 64 columns x 128 rows
+  CUtensorMap wmap[APR_MAX_PROJ];        // W_p [d_out, d_in]: 64 x 256
+  CUtensorMap vmap[APR_MAX_PROJ];        // V_p [T, NB]: 64 x 128
+  CUtensorMap bmap[APR_MAX_PROJ];        // Bcat_p [d_out, NB]: 64 x 256
+  void* y[APR_MAX_PROJ];
+  int d_out[APR_MAX_PROJ];
+  int nt_before[APR_MAX_PROJ + 1];       // prefix of 256-column tiles per projection
+  int nproj, T, nbase, nlora, mt;
+  void* ws;
+};
+
+__global__ void __launch_bounds__(LL_THREADS, 1) linear_lora_kernel(const __grid_constant__ LinPlan P) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem =
+      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)LL_ST * LL_STAGE);
+  const uint32_t bar_full = smem_u32(bars);                 // [ST] a K block landed (TMA bytes)
+  const uint32_t bar_empty = smem_u32(bars + LL_ST);        // [ST] its MMAs are done
+  const uint32_t bar_dfull = smem_u32(bars + 2 * LL_ST);    // [2]  accumulator complete
+  const uint32_t bar_dempty = smem_u32(bars + 2 * LL_ST + 2); // [2] accumulator read out
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 2 * LL_ST + 4);
+  int* s_consumed = reinterpret_cast<int*>(s_tmem + 1);
+
+  if (tid == 0) {
+    for (int i = 0; i < LL_ST; ++i) {
+      mbar_init(bar_full + 8 * i, 1);
+      mbar_init(bar_empty + 8 * i, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar_dfull + 8 * i, 1);
+      mbar_init(bar_dempty + 8 * i, 4 * 32);
+    }
+    *s_consumed = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) tmem_alloc(smem_u32(s_tmem), LL_TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+  pdl_trigger();
+  pdl_wait();                                      // x, V and Bcat come from the preceding kernels
+
+  const int mt = P.mt, nkb = P.nbase + P.nlora;
+  const int total = P.nt_before[P.nproj] * mt;
+  auto tile_at = [&](int tile, int& p, int& n0, int& m0) {
+    const int nt = tile / mt;
+    m0 = (tile - nt * mt) * LL_BM;
+    p = 0;
+    while (p + 1 < P.nproj && nt >= P.nt_before[p + 1]) ++p;
+    n0 = (nt - P.nt_before[p]) * LL_BN;
+  };
+  bool abort = false;
+  int issued = 0;                                  // K blocks issued by the producer
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      for (int tile = blockIdx.x; tile < total && !abort; tile += gridDim.x) {
+        int p, n0, m0;
+        tile_at(tile, p, n0, m0);
+        for (int kb = 0; kb < nkb; ++kb) {
+          const int s = issued % LL_ST;
+          if (!mbar_wait(bar_empty + 8 * s, ((issued / LL_ST) & 1) ^ 1)) { abort = true; break; }
+          const uint32_t sa = sbase + (uint32_t)s * LL_STAGE, sb = sa + LL_ABYTES;
+          mbar_arrive_expect_tx(bar_full + 8 * s, LL_STAGE);
+          if (kb < P.nbase) {
+            tma_load_2d(sa, &P.xmap, kb * LL_BK, m0, bar_full + 8 * s);
+            tma_load_2d(sb, &P.wmap[p], kb * LL_BK, n0, bar_full + 8 * s);
+          } else {
+            const int lb = kb - P.nbase;
+            tma_load_2d(sa, &P.vmap[p], lb * LL_BK, m0, bar_full + 8 * s);
+            tma_load_2d(sb, &P.bmap[p], lb * LL_BK, n0, bar_full + 8 * s);
+          }
+          ++issued;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issue
+    if (lane == 0) {
+      const uint32_t id = idesc_bf16(LL_BM, LL_BN);
+      int g = 0, it = 0;
+      for (int tile = blockIdx.x; tile < total && !abort; tile += gridDim.x, ++it) {
+        const int ab = it & 1;
+        if (!mbar_wait(bar_dempty + 8 * ab, ((it >> 1) & 1) ^ 1)) { abort = true; break; }
+        tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)ab * LL_BN;
+        for (int kb = 0; kb < nkb; ++kb, ++g) {
+          const int s = g % LL_ST;
+          if (!mbar_wait(bar_full + 8 * s, (g / LL_ST) & 1)) { abort = true; break; }
+          tc_fence_after();
+          const uint32_t sa = sbase + (uint32_t)s * LL_STAGE, sb = sa + LL_ABYTES;
+#pragma unroll
+          for (int kk = 0; kk < LL_BK / 16; ++kk)
+            mma_bf16(d, desc_k_sw128(sa + kk * 32), desc_k_sw128(sb + kk * 32), id, (kb | kk) != 0 ? 1u : 0u);
+          mma_commit(bar_empty + 8 * s);           // the slot is free once these MMAs have read it
+        }
+        if (abort) break;
+        mma_commit(bar_dfull + 8 * ab);
+      }
+      *s_consumed = g;
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int quarter = warp & 3;                  // TMEM lanes this warp may read
+    const int row = quarter * 32 + lane;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < total && !abort; tile += gridDim.x, ++it) {
+      int p, n0, m0;
+      tile_at(tile, p, n0, m0);
+      const int ab = it & 1;
+      if (!mbar_wait(bar_dfull + 8 * ab, (it >> 1) & 1)) { abort = true; break; }
+      tc_fence_after();
+      const int t = m0 + row, d_out = P.d_out[p];
+      __nv_bfloat16* yrow = reinterpret_cast<__nv_bfloat16*>(P.y[p]) + (size_t)t * d_out;
+      const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)ab * LL_BN;
+#pragma unroll 1
+      for (int c32 = 0; c32 < LL_BN / 32; ++c32) {
+        float v[32];
+        tmem_ld32(taddr + (uint32_t)(c32 * 32), v);
+        const int col = n0 + c32 * 32;
+        if (t < P.T) {
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            if (col + h * 8 < d_out) {
+              uint4 u;
+              uint32_t* w = reinterpret_cast<uint32_t*>(&u);
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const __nv_bfloat162 b2 = __floats2bfloat162_rn(v[h * 8 + 2 * q], v[h * 8 + 2 * q + 1]);
+                w[q] = *reinterpret_cast<const uint32_t*>(&b2);
+              }
+              *reinterpret_cast<uint4*>(yrow + col + h * 8) = u;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar_dempty + 8 * ab);
+    }
+  }
+  abort = __syncthreads_or(abort);
+  if (abort) {
+    if (tid == 0) report(P.ws, APR_ERR_TIMEOUT, K_LINEAR, (int)blockIdx.x);
+    // copies issued but never consumed land before the shared memory is released
+    if (warp == 0 && lane == 0)
+      for (int g = *s_consumed; g < issued; ++g) (void)mbar_wait(bar_full + 8 * (g % LL_ST), (g / LL_ST) & 1);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, LL_TMEM_COLS);
+}
+
+// ---------------------------------------------------------------- V and Bcat
+
+struct PackArgs {
+  const __nv_bfloat16* vc;               // gated v rows [proj][t * k + j][R16]
+  __nv_bfloat16* V;                      // [proj][T][NB]
+  __nv_bfloat16* Bcat[APR_MAX_PROJ];     // [d_out_p][NB]
+  const void* const* B[APR_MAX_PROJ];
+  int d_out[APR_MAX_PROJ];
+  long v_chunks;                         // nproj * T * NB / 8
+  long b_before[APR_MAX_PROJ + 1];       // prefix of Bcat chunks per projection
+  const int32_t* idx;
+  const int32_t* ranks;
+  int T, k, E, R16, NB, nproj;
+  void* ws;
+};
+
+// One 16-byte chunk (8 rank slots) per thread step: V first, then every projection's Bcat.
+__global__ void __launch_bounds__(256) linear_pack_kernel(const __grid_constant__ PackArgs a) {
+  pdl_wait();                                      // the shrink's rows, and the buffers' last readers
+  pdl_trigger();
+  const int cpr = a.NB / 8;                        // chunks per bank row
+  const long total = a.v_chunks + a.b_before[a.nproj];
+  for (long w = (long)blockIdx.x * blockDim.x + threadIdx.x; w < total; w += (long)gridDim.x * blockDim.x) {
+    uint4 val = make_uint4(0, 0, 0, 0);
+    if (w < a.v_chunks) {
+      const long row = w / cpr;                    // proj * T + t
+      const int c = (int)(w - row * cpr);
+      const int p = (int)(row / a.T), t = (int)(row - (long)p * a.T);
+      const int e = c * 8 / a.R16, r0 = c * 8 - e * a.R16;
+      for (int j = 0; j < a.k; ++j) {
+        const int ej = a.idx[(size_t)t * a.k + j];
+        if (ej < 0 || ej >= a.E) {
+          if (c == 0) report(a.ws, APR_ERR_DEVICE_INDEX, K_LINEAR, ej);
+        } else if (ej == e) {
+          val = *reinterpret_cast<const uint4*>(a.vc + (((size_t)p * a.T + t) * a.k + j) * a.R16 + r0);
+        }
+      }
+      *reinterpret_cast<uint4*>(a.V + (size_t)row * a.NB + c * 8) = val;
+    } else {
+      const long wb = w - a.v_chunks;
+      int p = 0;
+      while (p + 1 < a.nproj && wb >= a.b_before[p + 1]) ++p;
+      const long loc = wb - a.b_before[p];
+      const long n = loc / cpr;
+      const int c = (int)(loc - n * cpr);
+      const int e = c * 8 / a.R16, r0 = c * 8 - e * a.R16;
+      const int re = a.ranks[e];
+      const bool rank_ok = re >= 8 && re <= a.R16 && (re & 7) == 0;
+      if (!rank_ok && n == 0 && r0 == 0) report(a.ws, APR_ERR_DEVICE_INDEX, K_LINEAR, e);
+      if (rank_ok && r0 < re)
+        val = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.B[p][e]) + (size_t)n * re + r0);
+      *reinterpret_cast<uint4*>(a.Bcat[p] + (size_t)n * a.NB + c * 8) = val;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+cudaError_t launch_tc_shrink_pairs(const SgmmArgs& a, size_t v_off, cudaStream_t s);
+
+bool linear_lora_supported(const SgmmArgs& a) { return sgmm_bank_supported(a, APR_BF16); }
+
+cudaError_t launch_linear_lora(const SgmmArgs& a, const void* const* W, size_t scratch_off, cudaStream_t s) {
+  const int R16 = round16i(a.max_rank), NB = a.E * R16;
+  const LinearScratch L = linear_scratch(a.T, a.k, a.E, a.max_rank, a.nproj);
+  PackArgs pk;
+  memset(&pk, 0, sizeof(pk));
+  pk.vc = ws_at<__nv_bfloat16>(a.ws, scratch_off + L.vc);
+  pk.V = ws_at<__nv_bfloat16>(a.ws, scratch_off + L.v);
+  pk.idx = a.idx;
+  pk.ranks = a.ranks;
+  pk.T = a.T;
+  pk.k = a.k;
+  pk.E = a.E;
+  pk.R16 = R16;
+  pk.NB = NB;
+  pk.nproj = a.nproj;
+  pk.ws = a.ws;
+  pk.v_chunks = (long)a.nproj * a.T * (NB / 8);
+  size_t boff = scratch_off + L.bcat;
+  pk.b_before[0] = 0;
+  for (int p = 0; p < a.nproj; ++p) {
+    pk.Bcat[p] = ws_at<__nv_bfloat16>(a.ws, boff);
+    pk.B[p] = a.proj[p].B;
+    pk.d_out[p] = a.proj[p].d_out;
+    pk.b_before[p + 1] = pk.b_before[p] + (long)a.proj[p].d_out * (NB / 8);
+    boff += align_up((size_t)a.proj[p].d_out * NB * 2);
+  }
+
+  LinPlan P;
+  memset(&P, 0, sizeof(P));
+  cudaError_t err;
+  if ((err = encode_tile_map(&P.xmap, a.x, a.T, a.d_in, LL_BM)) != cudaSuccess) return err;
+  P.nt_before[0] = 0;
+  for (int p = 0; p < a.nproj; ++p) {
+    const int d_out = a.proj[p].d_out;
+    if ((err = encode_tile_map(&P.wmap[p], W[p], d_out, a.d_in, LL_BN)) != cudaSuccess) return err;
+    if ((err = encode_tile_map(&P.vmap[p], pk.V + (size_t)p * a.T * NB, a.T, NB, LL_BM)) != cudaSuccess) return err;
+    if ((err = encode_tile_map(&P.bmap[p], pk.Bcat[p], d_out, NB, LL_BN)) != cudaSuccess) return err;
+    P.y[p] = a.proj[p].y;
+    P.d_out[p] = d_out;
+    P.nt_before[p + 1] = P.nt_before[p] + (d_out + LL_BN - 1) / LL_BN;
+  }
+  P.nproj = a.nproj;
+  P.T = a.T;
+  P.nbase = (a.d_in + LL_BK - 1) / LL_BK;
+  P.nlora = (NB + LL_BK - 1) / LL_BK;
+  P.mt = (a.T + LL_BM - 1) / LL_BM;
+  P.ws = a.ws;
+
+  static SmemLimit lim;
+  if ((err = lim.ensure((const void*)linear_lora_kernel, LL_SMEM)) != cudaSuccess) return err;
+  if ((err = launch_tc_shrink_pairs(a, scratch_off + L.vc, s)) != cudaSuccess) return err;
+  const int nsm = device_sm_count();
+  const long chunks = pk.v_chunks + pk.b_before[a.nproj];
+  const int pgrid = (int)std::min<long>((chunks + 255) / 256, 8L * nsm);
+  if ((err = launch_pdl(linear_pack_kernel, dim3(pgrid), dim3(256), 0, s, pk)) != cudaSuccess) return err;
+  const long tiles = (long)P.nt_before[a.nproj] * P.mt;
+  const int grid = (int)std::min<long>(tiles, nsm);
+  return launch_pdl(linear_lora_kernel, dim3(grid), dim3(LL_THREADS), LL_SMEM, s, P);
+}
+
+}  // namespace apr

@@ -195,6 +195,43 @@ apr_status apr_sgmm_shrink_expand(const void* x, int d_in, const apr_proj* projs
                                   const int32_t* seg_off, const int32_t* perm, void* ws,
                                   size_t ws_bytes, int kernel, void* stream);
 
+/* One projection of a fused base + adapter group. */
+typedef struct apr_linear_proj {
+  const void* W;          /* device [d_out, d_in] bf16 base weight (never written)    */
+  void* y;                /* device [T, d_out] bf16 out (written once, never read)     */
+  int d_out;              /* output width, a multiple of 8                             */
+  const void* const* A;   /* device array [E] of device pointers, A[e] -> [r_e, d_in]  */
+  const void* const* B;   /* device array [E] of device pointers, B[e] -> [d_out, r_e] */
+} apr_linear_proj;
+
+/* ------------------------------------------------------------------------
+ * Base projection and adapters in one contraction (section 2.B: the selected
+ * experts are fused into the backbone in a single pass).  For every
+ * projection p of the group and every token t:
+ *   y_p[t] = x[t] W_p^T + sum_j gate[t,j] * B_e (A_e x[t]),  e = idx[t,j]
+ * with fp32 accumulation of both terms in one accumulator and one rounding to
+ * bf16 per output element; y is written once and never read (no base output
+ * is read back and rewritten).
+ * Inputs as for apr_sgmm_shrink_expand (x shared by the group, the routing of
+ * apr_pregate_route, the segments of apr_segment_tokens written into the same
+ * `ws`).  bf16 only.  Needs, with R16 = max_rank rounded up to 16: R16 in
+ * {16, 32, 64}, k <= 4, k * R16 <= 64, E * R16 <= 256, d_in % 64 == 0, and
+ * every W, y and x 16-byte aligned; APR_ERR_UNSUPPORTED otherwise.
+ * ws must hold apr_linear_workspace_size(...) bytes for this group.
+ * T == 0 is a no-op.  Device faults (an index >= E, a bad rank, a wait that
+ * expires) are recorded in ws and reported by apr_stream_status.
+ * ---------------------------------------------------------------------- */
+apr_status apr_linear_lora(const void* x, int d_in, const apr_linear_proj* projs, int nproj, int T,
+                           int k, int E, const int32_t* ranks, int max_rank, const int32_t* idx,
+                           const float* gate, const int32_t* seg_off, const int32_t* perm, void* ws,
+                           size_t ws_bytes, void* stream);
+
+/* Workspace bytes for apr_linear_lora on up to T tokens with nproj projections
+ * whose output widths add up to at most sum_d_out (also enough for every other
+ * call on these maxima).  0 if an argument is out of range. */
+size_t apr_linear_workspace_size(int T, int k, int E, int max_rank, int max_d_in, int nproj,
+                                 long sum_d_out);
+
 /* One weight of the merge step. */
 typedef struct apr_merge_proj {
   const void* W;          /* device [d_out, d_in] bf16 base weight (never written) */

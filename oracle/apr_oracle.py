@@ -117,6 +117,15 @@ def sgmm_shrink_expand(x, A, B, idx, gate, y_base):
     return y
 
 
+def linear_lora(x, W, A, B, idx, gate):
+    """Base projection with the selected adapters fused into it (§2.B: the experts are fused
+    into the backbone in a single pass): ``y[t] = W x[t] + sum_j gate[t, j] * B_e (A_e x[t])``.
+    W is [d_out, d_in]."""
+    x = np.asarray(x, dtype=F64)
+    base = x @ np.asarray(W, dtype=F64).T
+    return sgmm_shrink_expand(x, A, B, idx, gate, base)
+
+
 def merge_adapters(W, A, B, idx1, gate1):
     """Merged weight for one token (§2.B step 3): ``W' = W + sum_j g_j B_{e_j} A_{e_j}``."""
     Wp = np.array(W, dtype=F64, copy=True)

@@ -293,3 +293,59 @@ def test_all_k_subsets_bruteforce_small():
         # within the selection: descending value, ascending index on ties
         for a, b in itertools.pairwise(idx.tolist()):
             assert row[a] > row[b] or (row[a] == row[b] and a < b)
+
+
+# ---------------------------------------------------------------- base projection + adapters in one pass
+
+
+def test_linear_lora_hand_example():
+    """Worked by hand: W = [[1, 2], [3, 4]], one rank-1 adapter A = [[1, 0]], B = [[1], [2]].
+    Token 0, x = (1, 1): W x = (3, 7), A x = 1, B (A x) = (1, 2), so y = (4, 9).
+    Token 1, x = (2, 0) with gate 0.5: W x = (2, 6), A x = 2, 0.5 * B (A x) = (1, 2), so y = (3, 8)."""
+    Wt = np.array([[1.0, 2.0], [3.0, 4.0]])
+    A = [np.array([[1.0, 0.0]])]
+    B = [np.array([[1.0], [2.0]])]
+    x = np.array([[1.0, 1.0], [2.0, 0.0]])
+    idx = np.zeros((2, 1), dtype=np.int32)
+    gate = np.array([[1.0], [0.5]])
+    assert np.array_equal(O.linear_lora(x, Wt, A, B, idx, gate), np.array([[4.0, 9.0], [3.0, 8.0]]))
+
+
+def test_linear_lora_zero_adapters_is_the_plain_product_by_loops():
+    """With every B zero the result is x W^T, here summed term by term on small integers."""
+    rng = np.random.default_rng(31)
+    T, d_in, d_out, E, k, r = 5, 7, 6, 3, 2, 4
+    x = rng.integers(-3, 4, size=(T, d_in)).astype(np.float64)
+    Wt = rng.integers(-3, 4, size=(d_out, d_in)).astype(np.float64)
+    A = [rng.normal(size=(r, d_in)) for _ in range(E)]
+    B = [np.zeros((d_out, r)) for _ in range(E)]
+    idx = np.array([rng.permutation(E)[:k] for _ in range(T)], dtype=np.int32)
+    gate = rng.random((T, k))
+    ref = np.zeros((T, d_out))
+    for t in range(T):
+        for n in range(d_out):
+            for i in range(d_in):
+                ref[t, n] += x[t, i] * Wt[n, i]
+    assert np.array_equal(O.linear_lora(x, Wt, A, B, idx, gate), ref)
+
+
+def test_linear_lora_single_adapter_equals_merged_weight_gemm():
+    """E = 1, k = 1, gate 1: the fused result is the textbook GEMM with W + B A."""
+    rng = np.random.default_rng(32)
+    T, d_in, d_out, r = 11, 24, 18, 5
+    Wt = rng.normal(size=(d_out, d_in))
+    A = [rng.normal(size=(r, d_in))]
+    B = [rng.normal(size=(d_out, r))]
+    x = rng.normal(size=(T, d_in))
+    y = O.linear_lora(x, Wt, A, B, np.zeros((T, 1), dtype=np.int32), np.ones((T, 1)))
+    assert np.allclose(y, x @ (Wt + B[0] @ A[0]).T, rtol=1e-12, atol=1e-12)
+
+
+def test_linear_lora_transposed_weight_changes_the_answer():
+    """x W^T, not x W: a square non-symmetric W tells the two apart on the integer example."""
+    Wt = np.array([[1.0, 2.0], [3.0, 4.0]])
+    x = np.array([[1.0, 0.0]])
+    A = [np.zeros((1, 2))]
+    B = [np.zeros((2, 1))]
+    y = O.linear_lora(x, Wt, A, B, np.zeros((1, 1), dtype=np.int32), np.ones((1, 1)))
+    assert np.array_equal(y, np.array([[1.0, 3.0]]))

@@ -220,50 +220,48 @@ struct PackArgs {
   __nv_bfloat16* Bcat[APR_MAX_PROJ];     // [d_out_p][NB]
   const void* const* B[APR_MAX_PROJ];
   int d_out[APR_MAX_PROJ];
-  long v_chunks;                         // nproj * T * NB / 8
-  long b_before[APR_MAX_PROJ + 1];       // prefix of Bcat chunks per projection
   const int32_t* idx;
   const int32_t* ranks;
   int T, k, E, R16, NB, nproj;
   void* ws;
 };
 
-// One 16-byte chunk (8 rank slots) per thread step: V first, then every projection's Bcat.
+// One 16-byte chunk (8 rank slots) per thread step.  blockIdx.y = 0: the V rows of every
+// projection (row = proj * T + t, whose gated v rows start at vc + row * k * R16);
+// blockIdx.y = 1 + p: projection p's Bcat.
 __global__ void __launch_bounds__(256) linear_pack_kernel(const __grid_constant__ PackArgs a) {
   pdl_wait();                                      // the shrink's rows, and the buffers' last readers
   pdl_trigger();
   const int cpr = a.NB / 8;                        // chunks per bank row
-  const long total = a.v_chunks + a.b_before[a.nproj];
-  for (long w = (long)blockIdx.x * blockDim.x + threadIdx.x; w < total; w += (long)gridDim.x * blockDim.x) {
-    uint4 val = make_uint4(0, 0, 0, 0);
-    if (w < a.v_chunks) {
-      const long row = w / cpr;                    // proj * T + t
-      const int c = (int)(w - row * cpr);
-      const int p = (int)(row / a.T), t = (int)(row - (long)p * a.T);
+  const int stride = gridDim.x * blockDim.x;
+  if (blockIdx.y == 0) {
+    const int total = a.nproj * a.T * cpr;
+    for (int w = blockIdx.x * blockDim.x + threadIdx.x; w < total; w += stride) {
+      const int row = w / cpr, c = w - row * cpr;
+      const int t = row % a.T;
       const int e = c * 8 / a.R16, r0 = c * 8 - e * a.R16;
+      uint4 val = make_uint4(0, 0, 0, 0);
       for (int j = 0; j < a.k; ++j) {
-        const int ej = a.idx[(size_t)t * a.k + j];
-        if (ej < 0 || ej >= a.E) {
-          if (c == 0) report(a.ws, APR_ERR_DEVICE_INDEX, K_LINEAR, ej);
-        } else if (ej == e) {
-          val = *reinterpret_cast<const uint4*>(a.vc + (((size_t)p * a.T + t) * a.k + j) * a.R16 + r0);
-        }
+        const int ej = __ldg(a.idx + (size_t)t * a.k + j);
+        if (ej == e) val = *reinterpret_cast<const uint4*>(a.vc + ((size_t)row * a.k + j) * a.R16 + r0);
+        else if ((ej < 0 || ej >= a.E) && c == 0) report(a.ws, APR_ERR_DEVICE_INDEX, K_LINEAR, ej);
       }
       *reinterpret_cast<uint4*>(a.V + (size_t)row * a.NB + c * 8) = val;
-    } else {
-      const long wb = w - a.v_chunks;
-      int p = 0;
-      while (p + 1 < a.nproj && wb >= a.b_before[p + 1]) ++p;
-      const long loc = wb - a.b_before[p];
-      const long n = loc / cpr;
-      const int c = (int)(loc - n * cpr);
+    }
+  } else {
+    const int p = blockIdx.y - 1;
+    const __nv_bfloat16* const* Bp = reinterpret_cast<const __nv_bfloat16* const*>(a.B[p]);
+    __nv_bfloat16* dst = a.Bcat[p];
+    const int total = a.d_out[p] * cpr;
+    for (int w = blockIdx.x * blockDim.x + threadIdx.x; w < total; w += stride) {
+      const int n = w / cpr, c = w - n * cpr;
       const int e = c * 8 / a.R16, r0 = c * 8 - e * a.R16;
-      const int re = a.ranks[e];
+      const int re = __ldg(a.ranks + e);
       const bool rank_ok = re >= 8 && re <= a.R16 && (re & 7) == 0;
       if (!rank_ok && n == 0 && r0 == 0) report(a.ws, APR_ERR_DEVICE_INDEX, K_LINEAR, e);
-      if (rank_ok && r0 < re)
-        val = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.B[p][e]) + (size_t)n * re + r0);
-      *reinterpret_cast<uint4*>(a.Bcat[p] + (size_t)n * a.NB + c * 8) = val;
+      uint4 val = make_uint4(0, 0, 0, 0);
+      if (rank_ok && r0 < re) val = *reinterpret_cast<const uint4*>(Bp[e] + (size_t)n * re + r0);
+      *reinterpret_cast<uint4*>(dst + (size_t)n * a.NB + c * 8) = val;
     }
   }
 }
@@ -290,14 +288,13 @@ cudaError_t launch_linear_lora(const SgmmArgs& a, const void* const* W, size_t s
   pk.NB = NB;
   pk.nproj = a.nproj;
   pk.ws = a.ws;
-  pk.v_chunks = (long)a.nproj * a.T * (NB / 8);
   size_t boff = scratch_off + L.bcat;
-  pk.b_before[0] = 0;
+  long most = (long)a.nproj * a.T * (NB / 8);     // chunks of the largest role
   for (int p = 0; p < a.nproj; ++p) {
     pk.Bcat[p] = ws_at<__nv_bfloat16>(a.ws, boff);
     pk.B[p] = a.proj[p].B;
     pk.d_out[p] = a.proj[p].d_out;
-    pk.b_before[p + 1] = pk.b_before[p] + (long)a.proj[p].d_out * (NB / 8);
+    most = std::max(most, (long)a.proj[p].d_out * (NB / 8));
     boff += align_up((size_t)a.proj[p].d_out * NB * 2);
   }
 
@@ -326,9 +323,8 @@ cudaError_t launch_linear_lora(const SgmmArgs& a, const void* const* W, size_t s
   if ((err = lim.ensure((const void*)linear_lora_kernel, LL_SMEM)) != cudaSuccess) return err;
   if ((err = launch_tc_shrink_pairs(a, scratch_off + L.vc, s)) != cudaSuccess) return err;
   const int nsm = device_sm_count();
-  const long chunks = pk.v_chunks + pk.b_before[a.nproj];
-  const int pgrid = (int)std::min<long>((chunks + 255) / 256, 8L * nsm);
-  if ((err = launch_pdl(linear_pack_kernel, dim3(pgrid), dim3(256), 0, s, pk)) != cudaSuccess) return err;
+  const int pgrid = (int)std::min<long>((most + 255) / 256, 4L * nsm);
+  if ((err = launch_pdl(linear_pack_kernel, dim3(pgrid, 1 + a.nproj), dim3(256), 0, s, pk)) != cudaSuccess) return err;
   const long tiles = (long)P.nt_before[a.nproj] * P.mt;
   const int grid = (int)std::min<long>(tiles, nsm);
   return launch_pdl(linear_lora_kernel, dim3(grid), dim3(LL_THREADS), LL_SMEM, s, P);

@@ -12,6 +12,12 @@ or, for the batch-1 merge workload, the route, one ``apr_merge_adapters_planned`
 over every weight (its TMA plan built once with the weights) and one ``apr_gemv``
 per weight (§2.B steps 1-5).
 
+With ``base="fused"`` every (layer, group) call is instead ``apr_linear_lora``:
+the base projection ``x W^T`` and the adapters in one contraction, so there is
+no y_base.  With ``base="cublas"`` the same base product comes from
+``torch.matmul`` (a plain library GEMM into y_base) followed by the SGMM call
+adding the adapters in place: the unfused pipeline the fused call replaces.
+
 Tensors are built once from the seeded pools (``workloads.device_tensor``) and
 stay resident; ``run()`` enqueues the step on the current stream.
 """
@@ -30,10 +36,15 @@ def _dt(cfg):
 
 class Step:
     def __init__(self, cfg: W.Config, device="cuda", layers=None, zero_y_base=False,
-                 kernel=apr.SGMM_AUTO, out_of_place=True):
+                 kernel=apr.SGMM_AUTO, out_of_place=True, base=None):
+        if base not in (None, "fused", "cublas"):
+            raise ValueError(f"base must be None, 'fused' or 'cublas', got {base!r}")
+        if base is not None and (cfg.merge or cfg.dtype != "bf16"):
+            raise ValueError("a base projection runs on bf16 SGMM workloads only")
         self.cfg = cfg
         self.device = device
         self.kernel = kernel
+        self.base = base
         self.layers = list(range(cfg.layers)) if layers is None else list(layers)
         dt = _dt(cfg)
         T, E, k = cfg.T, cfg.E, cfg.k
@@ -48,10 +59,16 @@ class Step:
         self.seg_off = torch.empty(E + 1, dtype=torch.int32, device=device)
         self.perm = torch.empty(T * k, dtype=torch.int32, device=device)
         max_d_in = max(g.d_in for g in cfg.groups)
-        self.ws = apr.workspace(T, k, E, self.max_rank, max_d_in, device=device)
+        if base == "fused":
+            self.ws = apr.linear_workspace(T, k, E, self.max_rank, max_d_in, max(len(g.d_outs) for g in cfg.groups),
+                                           max(sum(g.d_outs) for g in cfg.groups), device=device)
+        else:
+            self.ws = apr.workspace(T, k, E, self.max_rank, max_d_in, device=device)
         self.keep = []
         if cfg.merge:
             self._build_merge(dt)
+        elif base is not None:
+            self._build_base(dt)
         else:
             self._build_sgmm(dt, zero_y_base, out_of_place)
 
@@ -114,6 +131,50 @@ class Step:
                 self.calls.append((x, projs, (l, g.name)))
             self.layer_in[l] = (in0, pos_in[0])
             self.layer_out[l] = (out0, pos_out) if out_of_place else (in0, pos_in[0])
+        W.clear_device_pools()
+
+    # ------------------------------------------------------------ base projection + adapters
+    def _build_base(self, dt):
+        cfg, dev = self.cfg, self.device
+        T = cfg.T
+        self.calls = []          # (x, [LinearProj...] or [(W, Proj)...], (l, g))
+        self.outputs = {}        # (l, g, p) -> (y, W)
+        self.adapters = {}
+        n_in = T * cfg.d_router + sum(T * g.d_in for g in cfg.groups) * len(self.layers)
+        n_out = sum(T * sum(g.d_outs) for g in cfg.groups) * len(self.layers)
+        self.act_in = torch.empty(n_in, dtype=dt, device=dev)
+        self.act_out = torch.empty(n_out, dtype=dt, device=dev)
+        h = self.act_in[:T * cfg.d_router].view(tuple(self.h.shape))
+        h.copy_(self.h)
+        self.h = h
+        pos_in, pos_out = T * cfg.d_router, 0
+        self.layer_in, self.layer_out = {}, {}
+        for l in self.layers:
+            in0, out0 = pos_in, pos_out
+            for g in cfg.groups:
+                x = self.act_in[pos_in:pos_in + T * g.d_in].view(T, g.d_in)
+                pos_in += T * g.d_in
+                x.copy_(W.device_tensor(cfg, W.x_key(l, g.name), (T, g.d_in), dev))
+                projs = []
+                for p, d_out in zip(g.proj_names, g.d_outs):
+                    Wt = W.device_tensor(cfg, W.w_key(l, g.name, p), (d_out, g.d_in), dev)
+                    A = [W.device_tensor(cfg, W.a_key(l, g.name, p, e), (int(self.ranks_np[e]), g.d_in), dev)
+                         for e in range(cfg.E)]
+                    B = [W.device_tensor(cfg, W.b_key(l, g.name, p, e), (d_out, int(self.ranks_np[e])), dev)
+                         for e in range(cfg.E)]
+                    At, Bt = apr.ptr_array(A, dev), apr.ptr_array(B, dev)
+                    y = self.act_out[pos_out:pos_out + T * d_out].view(T, d_out)
+                    pos_out += T * d_out
+                    if self.base == "fused":
+                        projs.append(apr.make_linear_proj(Wt, y, At, Bt))
+                    else:
+                        projs.append((Wt, apr.make_proj(y, y, At, Bt), y))
+                    self.outputs[(l, g.name, p)] = (y, Wt)
+                    self.adapters[(l, g.name, p)] = (A, B)
+                    self.keep += [At, Bt, Wt]
+                self.calls.append((x, projs, (l, g.name)))
+            self.layer_in[l] = (in0, pos_in)
+            self.layer_out[l] = (out0, pos_out)
         W.clear_device_pools()
 
     # ------------------------------------------------------------ merge workload
@@ -187,7 +248,17 @@ class Step:
                     apr.gemv(Wp, x, y, stream)
             return
         for x, projs, (ll, _) in self.calls:
-            if ll == l:
+            if ll != l:
+                continue
+            if self.base == "fused":
+                apr.linear_lora(x, projs, cfg.k, cfg.E, self.ranks, self.max_rank, self.idx, self.gate,
+                                self.seg_off, self.perm, self.ws, stream)
+            elif self.base == "cublas":
+                for Wt, _, y in projs:
+                    torch.matmul(x, Wt.t(), out=y)
+                apr.sgmm_shrink_expand(x, [pj for _, pj, _ in projs], cfg.k, cfg.E, self.ranks, self.max_rank,
+                                       self.idx, self.gate, self.seg_off, self.perm, self.ws, self.kernel, stream)
+            else:
                 apr.sgmm_shrink_expand(x, projs, cfg.k, cfg.E, self.ranks, self.max_rank, self.idx,
                                        self.gate, self.seg_off, self.perm, self.ws, self.kernel, stream)
 
@@ -214,14 +285,28 @@ class Step:
         """Bytes the step must move at least once (inputs read once, outputs written once)."""
         if idx_np is None:
             idx_np = self.idx.cpu().numpy()
-        return algorithmic_bytes(self.cfg, self.layers, self.ranks_np, idx_np)
+        return algorithmic_bytes(self.cfg, self.layers, self.ranks_np, idx_np, base=self.base is not None)
+
+    def flops(self) -> float:
+        """Multiply-adds x 2 of the layer calls: the base products (when the step has them) and
+        the adapters (shrink and expand of every token's k adapters)."""
+        cfg, T = self.cfg, self.cfg.T
+        r_mean = float(np.mean([self.ranks_np[e] for e in range(cfg.E)]))
+        f = 0.0
+        for _ in self.layers:
+            for g in cfg.groups:
+                for d_out in g.d_outs:
+                    if self.base is not None:
+                        f += 2.0 * T * g.d_in * d_out
+                    f += 2.0 * T * cfg.k * r_mean * (g.d_in + d_out)
+        return f
 
 
-def algorithmic_bytes(cfg: W.Config, layers, ranks_np, idx_np) -> int:
+def algorithmic_bytes(cfg: W.Config, layers, ranks_np, idx_np, base=False) -> int:
     """Bytes a step must move at least once: the router's h and Wr; per shared-input group its x
     once; per projection the A and B of every adapter some token selected, and y_base read plus y
-    written (SGMM); or, for the merge, W read, W' written, the selected adapters and the GEMV's
-    W', x and y."""
+    written (SGMM), or W read and y written (base projection and adapters in one pass); or, for
+    the merge, W read, W' written, the selected adapters and the GEMV's W', x and y."""
     el = 2 if cfg.dtype == "bf16" else 4
     T = cfg.T
     touched = np.unique(np.asarray(idx_np).reshape(-1))
@@ -237,5 +322,8 @@ def algorithmic_bytes(cfg: W.Config, layers, ranks_np, idx_np) -> int:
             b += T * g.d_in * el                                               # x once per group
             for d_out in g.d_outs:
                 b += sum(int(ranks_np[e]) * (g.d_in + d_out) * el for e in touched)
-                b += 2 * T * d_out * el                                        # y_base read, y written
+                if base:
+                    b += d_out * g.d_in * el + T * d_out * el                  # W read, y written
+                else:
+                    b += 2 * T * d_out * el                                    # y_base read, y written
     return b

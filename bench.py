@@ -6,12 +6,15 @@ fused into the base-output add for every (layer, shared-input group) of the
 workload.  The headline workload is ``prefill`` (Llama-2-7B layer set, 8192
 tokens, 16 rank-16 adapters with Zipf(1.1) popularity, top-2); the other
 full-size workloads (decode, multitenant, merge) are timed in the same run and
-reported under ``workloads``.  Each step is captured once in a CUDA graph and
-replayed; ``e2e`` times the eager C-ABI calls with the step's activations
+reported under ``workloads``, and so is ``prefill_fused``: the prefill layers
+with their base projections, each call the base GEMM and the adapters in one
+contraction (apr_linear_lora), beside the unfused pipeline it replaces (a
+library GEMM, then the SGMM add).  Each step is captured once in a CUDA graph
+and replayed; ``e2e`` times the eager C-ABI calls with the step's activations
 copied in from and out to pinned host memory.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
-                    [--also decode,multitenant,merge|none] [--impl reference]
+                    [--also decode,multitenant,merge,prefill_fused|none] [--impl reference]
 
 With N > 1 (torchrun, one process per GPU) every rank runs its own batch
 (weak scaling: tokens are independent and the path has no exchange step);
@@ -43,7 +46,11 @@ DESCR = {
     "merge": "batch-1 merge: 224 decode-shaped weights, top-2 merged W' = W + sum g B A in one launch, "
              "then one GEMV per weight, bf16",
     "tiny": "tiny: 4 layers x 256->256, 8 adapters rank 8, top-2, 64 tokens, fp32",
+    "prefill_fused": "prefill with the base projections: every layer call is y = x W^T + sum g B A x in one "
+                     "contraction (apr_linear_lora), same layers, adapters and routing as prefill, bf16",
 }
+# workloads that are another workload's configuration run in another mode
+BASE_MODE = {"prefill_fused": ("prefill", "fused")}
 
 
 def load_peaks():
@@ -475,13 +482,14 @@ def measure(name, args, world, rank, local, peaks, kernel_name="auto"):
     from adapter_pregate_router_b200 import apr, pipeline
     from adapter_pregate_router_b200 import workloads as W
 
-    cfg = W.scaled(W.CONFIGS[name], seed=W.CONFIGS[name].seed + rank)
+    cfg_name, base = BASE_MODE.get(name, (name, None))
+    cfg = W.scaled(W.CONFIGS[cfg_name], seed=W.CONFIGS[cfg_name].seed + rank)
     if args.layers:
         cfg = W.scaled(cfg, layers=args.layers)
     dev = torch.device("cuda", local)
     kernels = {"auto": apr.SGMM_AUTO, "skinny": apr.SGMM_SKINNY, "tensor": apr.SGMM_TENSOR,
                "dense": apr.SGMM_DENSE, "bank": apr.SGMM_BANK}
-    step = pipeline.Step(cfg, device=dev, kernel=kernels[kernel_name])
+    step = pipeline.Step(cfg, device=dev, kernel=kernels[kernel_name], base=base)
     stream = torch.cuda.Stream(device=dev)
     stream.wait_stream(torch.cuda.current_stream(dev))
 
@@ -562,17 +570,59 @@ def measure(name, args, world, rank, local, peaks, kernel_name="auto"):
         "us_per_call": layer_ms * 1e3 / ncalls, "step_bytes": step_bytes,
         "step_frac": step_bytes / (ms_step * 1e-3) / 1e9 / peaks["hbm_gbs"],
     }
+    if base is not None:
+        # base projections and adapters: a contraction, bounded by the tensor cores
+        flops = step.flops()
+        tflops = flops / (layer_ms * 1e-3) / 1e12
+        roof = {
+            "bound": "tensor",
+            "kernel": "apr_linear_lora (shrink, pack and the fused GEMM of every layer call)",
+            "achieved": tflops, "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+            "frac": tflops / peaks["bf16_tflops_sustained"],
+            "peak_source": f"{peaks['source']} sustained bf16 dense (a long step under the power cap)",
+            "traffic": None, "traffic_source": "no capture of this workload",
+            "flops_per_step": flops, "calls_per_step": ncalls, "us_per_call": layer_ms * 1e3 / ncalls,
+            "hbm_frac": layer_bytes / (layer_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], "step_bytes": step_bytes,
+        }
     graph.reset()
     layer_graph.reset()
     e2e = _e2e(step, cfg, stream, world, max(3, min(args.steps, 20 if cfg.T < 4096 else 3)))
     apr.stream_status(step.ws, stream)
     out = {"cfg": cfg, "value": value, "ms_per_step": ms_step, "roofline": roof, "e2e": e2e,
            "clocks": clk.summary(), "gpu_launches": launches * args.steps, "launches_per_step": launches,
-           "config": dict(config_block(cfg, world), **({"sgmm_kernel": kernel_name} if kernel_name != "auto" else {}))}
+           "config": dict(config_block(cfg, world), **({"sgmm_kernel": kernel_name} if kernel_name != "auto" else {}),
+                          **({"base": base} if base else {}))}
     del step
     import gc
     gc.collect()
     torch.cuda.empty_cache()
+    if base == "fused":
+        # the pipeline the fused call replaces: a library GEMM into y, then the SGMM call adding the
+        # adapters in place, same layers, weights and routing, timed the same way (layer calls only)
+        ref = pipeline.Step(cfg, device=dev, base="cublas")
+        with torch.cuda.stream(stream):
+            ref.route()
+            ref.layers_only()
+            stream.synchronize()
+            g2 = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g2, stream=stream):
+                ref.layers_only()
+            for _ in range(3):
+                g2.replay()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(nrep):
+                g2.replay()
+            e1.record(stream)
+        stream.synchronize()
+        apr.stream_status(ref.ws, stream)
+        un_ms = max_over_ranks(e0.elapsed_time(e1) / nrep, world)
+        out["unfused"] = {"layers_ms": un_ms, "fused_layers_ms": layer_ms, "speedup": un_ms / layer_ms,
+                          "pipeline": "torch.matmul base GEMM into y, then apr_sgmm_shrink_expand in place (auto)"}
+        g2.reset()
+        del ref
+        gc.collect()
+        torch.cuda.empty_cache()
     return out
 
 
@@ -590,6 +640,8 @@ def run_gpu(args, world, rank, local):
         others[name] = {"value": r["value"], "unit": "tokens/s", "ms_per_step": r["ms_per_step"],
                         "config": r["config"], "roofline": r["roofline"], "e2e": r["e2e"], "clocks": r["clocks"],
                         "gpu_launches": r["gpu_launches"], "launches_per_step": r["launches_per_step"]}
+        if "unfused" in r:
+            others[name]["unfused"] = r["unfused"]
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -615,7 +667,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="prefill", choices=["decode", "prefill", "multitenant", "merge", "tiny"])
-    ap.add_argument("--also", default="decode,multitenant,merge",
+    ap.add_argument("--also", default="decode,multitenant,merge,prefill_fused",
                     help="other full-size workloads timed in the same run and reported under 'workloads' "
                          "(comma-separated, or 'none')")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])

@@ -26,13 +26,14 @@
 //  2. a pack kernel spreads those rows over the bank's rank slots (V, zeros
 //     where a token did not select an adapter) and lays the projection's B_e
 //     side by side (Bcat), both row-major in the workspace;
-//  3. the GEMM: 128 x 256 output tiles, 64-wide K blocks by 2-D TMA boxes
-//     (128-byte swizzle) into a 4-deep ring, x/W blocks first and V/Bcat
-//     blocks after them; one thread issues the MMAs (M = 128, N = 256) into a
-//     double-buffered TMEM accumulator; four epilogue warps round and store
-//     while the next tile accumulates.  The grid is persistent (one CTA per
-//     SM), tiles ordered row tile fastest so that the CTAs in flight share
-//     W's column block in L2.
+//  3. the GEMM: 64-wide K blocks by 2-D TMA boxes (128-byte swizzle) into a
+//     ring, x/W blocks first and V/Bcat blocks after them; one thread issues
+//     the MMAs into a double-buffered TMEM accumulator; four epilogue warps
+//     round and store while the next tile accumulates.  Above 128 tokens the
+//     tiles are 256 x 256 and computed by CTA pairs (cta_group::2, below);
+//     a single 128-token tile runs on one CTA (128 x 256, M = 128 MMAs).  The
+//     grid is persistent, tiles ordered row tile fastest so that the CTAs in
+//     flight share W's column block in L2.
 //
 // Every mbarrier wait is bounded (1 s); on expiry the CTA records
 // APR_ERR_TIMEOUT, stops issuing, drains its copies and frees its TMEM.
@@ -212,6 +213,186 @@ __global__ void __launch_bounds__(LL_THREADS, 1) linear_lora_kernel(const __grid
   if (warp == 0) tmem_dealloc(tmem, LL_TMEM_COLS);
 }
 
+// ---------------------------------------------------------------- CTA pairs
+// The same contraction on 256 x 256 tiles computed by a pair of CTAs (a cluster of two) with
+// one MMA stream (tcgen05 cta_group::2): each CTA loads its 128 token rows of the A operand and
+// its 128 of the 256 output columns of the B operand, the leader issues M = 256, N = 256 MMAs
+// that read both CTAs' shared memory, and each CTA's TMEM receives its 128 rows of D.  Per SM
+// that is half the operand bytes of the one-CTA tile for the same MMA work.  All the loads of a
+// K block complete on the leader's barrier; the leader's commits free the slot in both CTAs and
+// hand each CTA's epilogue its accumulator; each epilogue warp returns the accumulator to the
+// leader with a remote arrive.
+
+constexpr int L2_ST = 6;                          // ring depth (32 KB per stage per CTA)
+constexpr uint32_t L2_STAGE = 2 * 128 * 128;      // A 128 x 64 and B 128 x 64, bf16
+constexpr size_t L2_SMEM = (size_t)L2_ST * L2_STAGE + 256 + 1024;
+
+__global__ void __launch_bounds__(LL_THREADS, 1) linear_lora_pair_kernel(const __grid_constant__ LinPlan P) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem =
+      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = cluster_rank();            // 0: leader (issues the MMAs), 1: peer
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)L2_ST * L2_STAGE);
+  const uint32_t bar_full = smem_u32(bars);                  // [ST] leader: both CTAs' K block landed
+  const uint32_t bar_empty = smem_u32(bars + L2_ST);         // [ST] the slot's MMAs are done
+  const uint32_t bar_dfull = smem_u32(bars + 2 * L2_ST);     // [2]  accumulator complete
+  const uint32_t bar_dempty = smem_u32(bars + 2 * L2_ST + 2);// [2]  leader: read out by 8 epilogue warps
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 2 * L2_ST + 4);
+  int* s_consumed = reinterpret_cast<int*>(s_tmem + 1);      // leader: K blocks the MMAs took
+  int* s_issued = s_consumed + 1;                            // leader: [2] K blocks each producer issued
+
+  if (tid == 0) {
+    for (int i = 0; i < L2_ST; ++i) {
+      mbar_init(bar_full + 8 * i, 1);
+      mbar_init(bar_empty + 8 * i, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar_dfull + 8 * i, 1);
+      mbar_init(bar_dempty + 8 * i, 8);
+    }
+    *s_consumed = 0;
+    s_issued[0] = s_issued[1] = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) tmem_alloc_pair(smem_u32(s_tmem), LL_TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();                              // both CTAs' barriers and TMEM exist
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+  pdl_trigger();
+  pdl_wait();
+
+  const int mt = P.mt, nkb = P.nbase + P.nlora;   // mt: 256-row tiles
+  const int total = P.nt_before[P.nproj] * mt;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  auto tile_at = [&](int tile, int& p, int& n0, int& m0) {
+    const int nt = tile / mt;
+    m0 = (tile - nt * mt) * 2 * LL_BM;
+    p = 0;
+    while (p + 1 < P.nproj && nt >= P.nt_before[p + 1]) ++p;
+    n0 = (nt - P.nt_before[p]) * LL_BN;
+  };
+  bool abort = false;
+  int issued = 0;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer (both CTAs)
+    if (lane == 0) {
+      const uint32_t full_leader = cluster_map(bar_full, 0);
+      for (int tile = pair; tile < total && !abort; tile += npairs) {
+        int p, n0, m0;
+        tile_at(tile, p, n0, m0);
+        const int ma = m0 + (int)rank * LL_BM, nb = n0 + (int)rank * (LL_BN / 2);
+        for (int kb = 0; kb < nkb; ++kb) {
+          const int s = issued % L2_ST;
+          if (!mbar_wait(bar_empty + 8 * s, ((issued / L2_ST) & 1) ^ 1)) { abort = true; break; }
+          const uint32_t sa = sbase + (uint32_t)s * L2_STAGE, sb = sa + L2_STAGE / 2;
+          if (rank == 0) mbar_arrive_expect_tx(bar_full + 8 * s, 2 * L2_STAGE);
+          if (kb < P.nbase) {
+            tma_load_2d_pair(sa, &P.xmap, kb * LL_BK, ma, full_leader + 8 * s);
+            tma_load_2d_pair(sb, &P.wmap[p], kb * LL_BK, nb, full_leader + 8 * s);
+          } else {
+            const int lb = kb - P.nbase;
+            tma_load_2d_pair(sa, &P.vmap[p], lb * LL_BK, ma, full_leader + 8 * s);
+            tma_load_2d_pair(sb, &P.bmap[p], lb * LL_BK, nb, full_leader + 8 * s);
+          }
+          ++issued;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issue (leader)
+    if (lane == 0 && rank == 0) {
+      const uint32_t id = idesc_bf16(2 * LL_BM, LL_BN);
+      int g = 0, it = 0;
+      for (int tile = pair; tile < total && !abort; tile += npairs, ++it) {
+        const int ab = it & 1;
+        if (!mbar_wait(bar_dempty + 8 * ab, ((it >> 1) & 1) ^ 1)) { abort = true; break; }
+        tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)ab * LL_BN;
+        for (int kb = 0; kb < nkb; ++kb, ++g) {
+          const int s = g % L2_ST;
+          if (!mbar_wait(bar_full + 8 * s, (g / L2_ST) & 1)) { abort = true; break; }
+          tc_fence_after();
+          const uint32_t sa = sbase + (uint32_t)s * L2_STAGE, sb = sa + L2_STAGE / 2;
+#pragma unroll
+          for (int kk = 0; kk < LL_BK / 16; ++kk)
+            mma_bf16_pair(d, desc_k_sw128(sa + kk * 32), desc_k_sw128(sb + kk * 32), id, (kb | kk) != 0 ? 1u : 0u);
+          mma_commit_pair(bar_empty + 8 * s, 3);   // the slot is free in both CTAs
+        }
+        if (abort) break;
+        mma_commit_pair(bar_dfull + 8 * ab, 3);    // both halves of D are complete
+      }
+      *s_consumed = g;
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue (both CTAs)
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t dempty_leader = cluster_map(bar_dempty, 0);
+    int it = 0;
+    for (int tile = pair; tile < total && !abort; tile += npairs, ++it) {
+      int p, n0, m0;
+      tile_at(tile, p, n0, m0);
+      const int ab = it & 1;
+      if (!mbar_wait(bar_dfull + 8 * ab, (it >> 1) & 1)) { abort = true; break; }
+      tc_fence_after();
+      const int t = m0 + (int)rank * LL_BM + row, d_out = P.d_out[p];
+      __nv_bfloat16* yrow = reinterpret_cast<__nv_bfloat16*>(P.y[p]) + (size_t)t * d_out;
+      const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)ab * LL_BN;
+#pragma unroll 1
+      for (int c32 = 0; c32 < LL_BN / 32; ++c32) {
+        float v[32];
+        tmem_ld32(taddr + (uint32_t)(c32 * 32), v);
+        const int col = n0 + c32 * 32;
+        if (t < P.T) {
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            if (col + h * 8 < d_out) {
+              uint4 u;
+              uint32_t* w = reinterpret_cast<uint32_t*>(&u);
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const __nv_bfloat162 b2 = __floats2bfloat162_rn(v[h * 8 + 2 * q], v[h * 8 + 2 * q + 1]);
+                w[q] = *reinterpret_cast<const uint32_t*>(&b2);
+              }
+              *reinterpret_cast<uint4*>(yrow + col + h * 8) = u;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(dempty_leader + 8 * ab);
+    }
+  }
+  abort = __syncthreads_or(abort);
+  // the producers' counts go to the leader, so that after a timeout it can wait for every copy
+  // still in flight (their bytes complete on its barriers) before either CTA releases its memory
+  if (warp == 0 && lane == 0)
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_map(smem_u32(s_issued + rank), 0)), "r"(issued)
+                 : "memory");
+  cluster_sync_all();
+  const bool any_abort = abort || s_issued[0] != *s_consumed || s_issued[1] != *s_consumed;
+  if (rank == 0 && any_abort) {
+    if (tid == 0) report(P.ws, APR_ERR_TIMEOUT, K_LINEAR, (int)blockIdx.x);
+    if (warp == 0 && lane == 0) {
+      const int most = max(s_issued[0], s_issued[1]);
+      for (int g = *s_consumed; g < most; ++g) (void)mbar_wait(bar_full + 8 * (g % L2_ST), (g / L2_ST) & 1);
+    }
+  } else if (rank == 1 && abort && tid == 0) {
+    report(P.ws, APR_ERR_TIMEOUT, K_LINEAR, (int)blockIdx.x);
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();                              // no copy or remote arrive still targets either CTA
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc_pair(tmem, LL_TMEM_COLS);
+}
+
 // ---------------------------------------------------------------- V and Bcat
 
 struct PackArgs {
@@ -298,6 +479,9 @@ cudaError_t launch_linear_lora(const SgmmArgs& a, const void* const* W, size_t s
     boff += align_up((size_t)a.proj[p].d_out * NB * 2);
   }
 
+  // CTA pairs (256-token tiles) unless the call has a single 128-token tile
+  const bool pairs = a.T > LL_BM;
+  const int brows = pairs ? LL_BN / 2 : LL_BN;     // rows of a B box: the CTA's share of the N columns
   LinPlan P;
   memset(&P, 0, sizeof(P));
   cudaError_t err;
@@ -305,9 +489,9 @@ cudaError_t launch_linear_lora(const SgmmArgs& a, const void* const* W, size_t s
   P.nt_before[0] = 0;
   for (int p = 0; p < a.nproj; ++p) {
     const int d_out = a.proj[p].d_out;
-    if ((err = encode_tile_map(&P.wmap[p], W[p], d_out, a.d_in, LL_BN)) != cudaSuccess) return err;
+    if ((err = encode_tile_map(&P.wmap[p], W[p], d_out, a.d_in, brows)) != cudaSuccess) return err;
     if ((err = encode_tile_map(&P.vmap[p], pk.V + (size_t)p * a.T * NB, a.T, NB, LL_BM)) != cudaSuccess) return err;
-    if ((err = encode_tile_map(&P.bmap[p], pk.Bcat[p], d_out, NB, LL_BN)) != cudaSuccess) return err;
+    if ((err = encode_tile_map(&P.bmap[p], pk.Bcat[p], d_out, NB, brows)) != cudaSuccess) return err;
     P.y[p] = a.proj[p].y;
     P.d_out[p] = d_out;
     P.nt_before[p + 1] = P.nt_before[p] + (d_out + LL_BN - 1) / LL_BN;
@@ -316,18 +500,38 @@ cudaError_t launch_linear_lora(const SgmmArgs& a, const void* const* W, size_t s
   P.T = a.T;
   P.nbase = (a.d_in + LL_BK - 1) / LL_BK;
   P.nlora = (NB + LL_BK - 1) / LL_BK;
-  P.mt = (a.T + LL_BM - 1) / LL_BM;
+  const int tile_rows = pairs ? 2 * LL_BM : LL_BM;
+  P.mt = (a.T + tile_rows - 1) / tile_rows;
   P.ws = a.ws;
 
-  static SmemLimit lim;
+  static SmemLimit lim, lim2;
   if ((err = lim.ensure((const void*)linear_lora_kernel, LL_SMEM)) != cudaSuccess) return err;
+  if ((err = lim2.ensure((const void*)linear_lora_pair_kernel, L2_SMEM)) != cudaSuccess) return err;
   if ((err = launch_tc_shrink_pairs(a, scratch_off + L.vc, s)) != cudaSuccess) return err;
   const int nsm = device_sm_count();
   const int pgrid = (int)std::min<long>((most + 255) / 256, 4L * nsm);
   if ((err = launch_pdl(linear_pack_kernel, dim3(pgrid, 1 + a.nproj), dim3(256), 0, s, pk)) != cudaSuccess) return err;
   const long tiles = (long)P.nt_before[a.nproj] * P.mt;
-  const int grid = (int)std::min<long>(tiles, nsm);
-  return launch_pdl(linear_lora_kernel, dim3(grid), dim3(LL_THREADS), LL_SMEM, s, P);
+  if (!pairs) {
+    const int grid = (int)std::min<long>(tiles, nsm);
+    return launch_pdl(linear_lora_kernel, dim3(grid), dim3(LL_THREADS), LL_SMEM, s, P);
+  }
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  cfg.gridDim = dim3(2 * (unsigned)std::min<long>(tiles, nsm / 2));
+  cfg.blockDim = dim3(LL_THREADS);
+  cfg.dynamicSmemBytes = L2_SMEM;
+  cfg.stream = s;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 2;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  count_launch();
+  return cudaLaunchKernelEx(&cfg, linear_lora_pair_kernel, P);
 }
 
 }  // namespace apr

@@ -67,11 +67,6 @@ __device__ __forceinline__ uint32_t tmem_cols_for(int n) {
   return c;
 }
 
-__device__ __forceinline__ uint32_t cluster_map(uint32_t saddr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
-  return r;
-}
 // A load from another CTA's shared memory; ordered by the cluster barriers
 // around it, it carries no memory clobber, so several stay in flight.
 __device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
@@ -81,12 +76,6 @@ __device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
 }
 __device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
   asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
-}
-__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
-__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
-__device__ __forceinline__ void cluster_sync_all() {
-  cluster_arrive();
-  cluster_wait();
 }
 
 // ---------------------------------------------------------------- shrink

@@ -87,6 +87,10 @@ _linear = _sig("apr_linear_lora", _i,
                 [_vp, _i, ctypes.POINTER(LinearProj), _i, _i, _i, _i, _vp, _i, _vp, _vp, _vp, _vp, _vp, _sz, _vp])
 _linear_workspace_size = _sig("apr_linear_workspace_size", _sz, [_i, _i, _i, _i, _i, _i, ctypes.c_long])
 _merge = _sig("apr_merge_adapters", _i, [_vp, _i, _i, _i, _vp, _vp, _i, _vp, _sz, _vp])
+_merge_escape_bytes = _sig("apr_merge_escape_bytes", _sz, [ctypes.c_long])
+_merge_residual_bytes = _sig("apr_merge_residual_bytes", _sz, [_i, _i])
+_merge_inplace = _sig("apr_merge_adapters_inplace", _i, [_vp, _i, _i, _i, _vp, _vp, _i, _vp, _sz, _vp, _sz, _vp])
+_unmerge_inplace = _sig("apr_unmerge_adapters_inplace", _i, [_vp, _i, _i, _i, _vp, _vp, _i, _vp, _sz, _vp, _sz, _vp])
 _merge_plan_size = _sig("apr_merge_plan_size", _sz, [_i])
 _merge_plan_init = _sig("apr_merge_plan_init", _i, [_vp, _i, _vp, _sz])
 _merge_planned = _sig("apr_merge_adapters_planned", _i, [_vp, _vp, _i, _i, _i, _vp, _vp, _i, _vp, _sz, _vp])
@@ -98,7 +102,8 @@ _kernel_launches = _sig("apr_kernel_launches", ctypes.c_uint64, [])
 
 EXPORTED = ("apr_workspace_size", "apr_workspace_init", "apr_pregate_route", "apr_pregate_route_noalloc",
             "apr_segment_tokens",
-            "apr_sgmm_shrink_expand", "apr_linear_lora", "apr_linear_workspace_size", "apr_merge_adapters", "apr_merge_plan_size", "apr_merge_plan_init",
+            "apr_sgmm_shrink_expand", "apr_linear_lora", "apr_linear_workspace_size", "apr_merge_adapters", "apr_merge_escape_bytes", "apr_merge_residual_bytes", "apr_merge_adapters_inplace",
+            "apr_unmerge_adapters_inplace", "apr_merge_plan_size", "apr_merge_plan_init",
             "apr_merge_adapters_planned", "apr_gemv", "apr_stream_status",
             "apr_last_error", "apr_status_string", "apr_kernel_launches")
 
@@ -387,6 +392,45 @@ def merge_adapters_planned(table, plan, nproj, E, r, idx, gate, k, ws, stream=No
 def merge_adapters(table, nproj, E, r, idx, gate, k, ws, stream=None):
     _check_merge_args(table, nproj, idx, gate, k, ws)
     _check(_merge(_ptr(table), nproj, E, r, _ptr(idx), _ptr(gate), k, _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def merge_escape_bytes(capacity: int) -> int:
+    return int(_merge_escape_bytes(capacity))
+
+
+def merge_residual(W: torch.Tensor) -> torch.Tensor:
+    """The residual-code buffer of one weight for an in-place merge (int8, on W's device)."""
+    _need(W, "W", (torch.bfloat16,), ndim=2)
+    n = int(_merge_residual_bytes(int(W.shape[0]), int(W.shape[1])))
+    if n == 0:
+        raise AprError(APR_ERR_INVALID_ARG, "merge_residual_bytes: shape out of range")
+    return torch.empty(n, dtype=torch.int8, device=W.device)
+
+
+def merge_escapes(capacity: int, device="cuda") -> torch.Tensor:
+    """A device buffer for ``capacity`` escapes of an in-place merge (uint8, 16-byte aligned)."""
+    return torch.zeros(merge_escape_bytes(capacity), dtype=torch.uint8, device=device)
+
+
+def _check_inplace_args(table, nproj, idx, gate, k, escapes, ws):
+    _check_merge_args(table, nproj, idx, gate, k, ws)
+    _need(escapes, "escapes", (torch.uint8,), ndim=1, min_numel=merge_escape_bytes(0))
+    _same_device(("table", table), ("escapes", escapes), ("ws", ws))
+
+
+def merge_adapters_inplace(table, nproj, E, r, idx, gate, k, escapes, ws, stream=None):
+    """W <- rn(W + sum g B A) in place for every entry of ``table`` (see ``merge_table``: each
+    entry's Wp is the int8 [d_out, d_in] residual-code buffer of that weight)."""
+    _check_inplace_args(table, nproj, idx, gate, k, escapes, ws)
+    _check(_merge_inplace(_ptr(table), nproj, E, r, _ptr(idx), _ptr(gate), k, _ptr(escapes), escapes.numel(),
+                          _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def unmerge_adapters_inplace(table, nproj, E, r, idx, gate, k, escapes, ws, stream=None):
+    """Restore every W of ``table`` bit for bit after ``merge_adapters_inplace`` (same routing)."""
+    _check_inplace_args(table, nproj, idx, gate, k, escapes, ws)
+    _check(_unmerge_inplace(_ptr(table), nproj, E, r, _ptr(idx), _ptr(gate), k, _ptr(escapes), escapes.numel(),
+                            _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def gemv(W, x, y, stream=None):

@@ -374,6 +374,47 @@ apr_status apr_merge_adapters(const apr_merge_proj* projs, int nproj, int E, int
   return APR_OK;
 }
 
+size_t apr_merge_escape_bytes(long capacity) { return capacity < 0 ? 0 : merge_escape_bytes(capacity); }
+size_t apr_merge_residual_bytes(int d_out, int d_in) {
+  return (d_out < 1 || d_in < 8 || (d_in & 7)) ? 0 : merge_residual_bytes(d_out, d_in);
+}
+
+static apr_status merge_inplace_call(const apr_merge_proj* projs, int nproj, int E, int r, const int32_t* idx,
+                                     const float* gate, int k, void* escapes, size_t escape_bytes, void* ws,
+                                     size_t ws_bytes, void* stream, bool unmerge) {
+  const char* who = unmerge ? "unmerge_inplace" : "merge_inplace";
+  if (nproj < 1) return fail(APR_ERR_INVALID_ARG, "%s: nproj=%d < 1", who, nproj);
+  if (E < 1 || E > APR_MAX_E) return fail(APR_ERR_INVALID_ARG, "%s: E=%d outside [1, %d]", who, E, APR_MAX_E);
+  if (k < 1 || k > E || k > APR_MAX_K) return fail(APR_ERR_INVALID_ARG, "%s: k=%d outside [1, min(E, %d)]", who, k, APR_MAX_K);
+  if (r < 8 || (r & 7) || r > APR_MAX_RANK)
+    return fail(APR_ERR_INVALID_ARG, "%s: r=%d must be a multiple of 8 in [8, %d]", who, r, APR_MAX_RANK);
+  if (!merge_tensor_supported(k, r, nproj))
+    return fail(APR_ERR_UNSUPPORTED, "%s: needs k * round16(r) <= 64 and nproj <= 4096", who);
+  if (!projs || !idx || !gate || !escapes) return fail(APR_ERR_INVALID_ARG, "%s: NULL pointer", who);
+  if (escape_bytes < merge_escape_bytes(0) || reinterpret_cast<uintptr_t>(escapes) % 16)
+    return fail(APR_ERR_INVALID_ARG, "%s: escape buffer below %zu bytes or not 16-byte aligned", who,
+                merge_escape_bytes(0));
+  apr_status st = check_ws(ws, ws_bytes, sizeof(WsHeader), who);
+  if (st) return st;
+  const long capacity = (long)((escape_bytes - merge_escape_bytes(0)) / 12);
+  cudaError_t e = launch_merge_inplace(projs, nproj, E, r, idx, gate, k, escapes, capacity, unmerge, ws,
+                                       (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, unmerge ? "unmerge_inplace launch" : "merge_inplace launch");
+  return APR_OK;
+}
+
+apr_status apr_merge_adapters_inplace(const apr_merge_proj* projs, int nproj, int E, int r, const int32_t* idx,
+                                      const float* gate, int k, void* escapes, size_t escape_bytes, void* ws,
+                                      size_t ws_bytes, void* stream) {
+  return merge_inplace_call(projs, nproj, E, r, idx, gate, k, escapes, escape_bytes, ws, ws_bytes, stream, false);
+}
+
+apr_status apr_unmerge_adapters_inplace(const apr_merge_proj* projs, int nproj, int E, int r, const int32_t* idx,
+                                        const float* gate, int k, void* escapes, size_t escape_bytes, void* ws,
+                                        size_t ws_bytes, void* stream) {
+  return merge_inplace_call(projs, nproj, E, r, idx, gate, k, escapes, escape_bytes, ws, ws_bytes, stream, true);
+}
+
 apr_status apr_gemv(const void* W, const void* x, void* y, int d_in, int d_out, void* stream) {
   if (d_in < 8 || (d_in & 7)) return fail(APR_ERR_INVALID_ARG, "gemv: d_in=%d must be a positive multiple of 8", d_in);
   if (d_in > 48 * 1024) return fail(APR_ERR_UNSUPPORTED, "gemv: d_in=%d > 49152", d_in);

@@ -338,6 +338,11 @@ bool sgmm_tensor_supported(const SgmmArgs& a, int dtype);
 cudaError_t launch_merge(const apr_merge_proj* projs, int nproj, int E, int r, const int32_t* idx,
                          const float* gate, int k, void* ws, cudaStream_t s);
 bool merge_tensor_supported(int k, int r, int nproj);
+size_t merge_escape_bytes(long capacity);
+size_t merge_residual_bytes(int d_out, int d_in);
+cudaError_t launch_merge_inplace(const apr_merge_proj* projs, int nproj, int E, int r, const int32_t* idx,
+                                 const float* gate, int k, void* escapes, long capacity, bool unmerge, void* ws,
+                                 cudaStream_t s);
 cudaError_t launch_merge_tensor(const apr_merge_proj* projs, int nproj, int E, int r, const int32_t* idx,
                                 const float* gate, int k, void* ws, cudaStream_t s);
 size_t merge_plan_bytes(int nproj);

@@ -54,11 +54,58 @@ struct MtSmem {
 // K-major A operand / MN-major B operand instruction descriptor (bf16 -> fp32).
 __host__ __device__ constexpr uint32_t idesc_bf16_bmn(int M, int N) { return idesc_bf16(M, N) | (1u << 16); }
 
+// In-place merge and exact unmerge (AdaFuse summary §2.B steps 3 and 5: merge, run,
+// unmerge for the next token).  The merge writes w' = rn(w + d) over w and, per element, the
+// distance from w to u = rn(w' - d), the value the unmerge will recompute, counted in
+// representable bf16 steps (keys that order the bit patterns like the values).  The unmerge
+// recomputes d (the same tensor-core product, bit for bit), forms u and steps back by the
+// stored distance.  Distances outside [-126, 127] become escapes: the exact bits go to a list
+// written back after the unmerge; when the list is full the element is left unmerged (code
+// -127) and the merge reports APR_ERR_WORKSPACE, so restoration stays exact either way.
+constexpr int MERGE_OUT_OF_PLACE = 0, MERGE_IN_PLACE = 1, UNMERGE_IN_PLACE = 2;
+constexpr int8_t kCodeEscape = -128, kCodeKept = -127;
+
+struct MergeEscapes {                  // device, caller-owned (apr_merge_escape_bytes)
+  unsigned int count;                  // escapes met (may exceed the capacity: those were kept)
+  int k;                               // the merge's routing, checked by the unmerge
+  int e[APR_MAX_K];
+  float g[APR_MAX_K];
+  int pad[14];
+  // then the capacity's entries {weight, element, bits}, 3 x 32 bits each
+};
+static_assert(sizeof(MergeEscapes) == 128, "escape header is 128 bytes");
+
+// key: positive values b ^ 0x8000, negative ones ~b (16 bits), so keys ascend with the values
+__device__ __forceinline__ int bf16_key(uint32_t b) {
+  return (int)((b ^ 0x8000u ^ ((uint32_t)((int32_t)(b << 16) >> 31) & 0x7FFFu)) & 0xFFFFu);
+}
+__device__ __forceinline__ uint32_t bf16_from_key(int key) {
+  const uint32_t k = (uint32_t)key & 0xFFFFu;
+  return k ^ (0xFFFFu ^ (((k >> 15) & 1u) * 0x7FFFu));
+}
+__device__ __forceinline__ float bf16_val(uint32_t b) { return __uint_as_float(b << 16); }
+// bytes of x picked by the selector nibbles; a nibble with bit 3 set gives the picked byte's sign
+// replicated (PTX prmt, default mode)
+__device__ __forceinline__ uint32_t prmt_sext(uint32_t x, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, 0, %2;" : "=r"(r) : "r"(x), "r"(sel));
+  return r;
+}
+// the same key and its inverse on the two 16-bit halves of a word
+__device__ __forceinline__ uint32_t bf16_key2(uint32_t x) {
+  return x ^ 0x80008000u ^ (((x >> 15) & 0x00010001u) * 0x7FFFu);
+}
+__device__ __forceinline__ uint32_t bf16_from_key2(uint32_t k) {
+  return k ^ (0xFFFFFFFFu ^ (((k >> 15) & 0x00010001u) * 0x7FFFu));
+}
+__device__ __forceinline__ uint32_t bf16x2_bits(__nv_bfloat162 h) { return *reinterpret_cast<const uint32_t*>(&h); }
+
+template <int MODE>
 __global__ void __launch_bounds__(TC_THREADS, 1) merge_tc_kernel(const apr_merge_proj* __restrict__ projs,
                                                                  int nproj, int E, int r, int R16,
                                                                  const int32_t* __restrict__ idx,
                                                                  const float* __restrict__ gate, int k,
-                                                                 void* ws) {
+                                                                 void* ws, MergeEscapes* esc, long esc_cap) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -111,9 +158,24 @@ __global__ void __launch_bounds__(TC_THREADS, 1) merge_tc_kernel(const apr_merge
     }
   }
   __syncthreads();
+  if (MODE == MERGE_IN_PLACE && blockIdx.x == 0 && tid == 0 && !s_flags[1]) {
+    esc->k = k;
+    for (int j = 0; j < k; ++j) {
+      esc->e[j] = s_e[j];
+      esc->g[j] = s_g[j];
+    }
+  }
+  if (MODE == UNMERGE_IN_PLACE && tid == 0) {
+    // the unmerge must recompute the merge's delta exactly: the same adapters and gates
+    bool same = esc->k == k;
+    for (int j = 0; j < k && same; ++j) same = esc->e[j] == s_e[j] && esc->g[j] == s_g[j];
+    if (!same && !s_flags[1]) s_flags[1] = 2;
+  }
+  __syncthreads();
   bool abort = false;
   if (s_flags[1]) {
-    if (tid == 0 && blockIdx.x == 0) report(ws, APR_ERR_DEVICE_INDEX, K_MERGE, 0);
+    if (tid == 0 && blockIdx.x == 0)
+      report(ws, s_flags[1] == 2 ? APR_ERR_INVALID_ARG : APR_ERR_DEVICE_INDEX, K_MERGE, 0);
   } else {
     const int total = s_pref[nproj];
     const uint32_t sbo_g = (uint32_t)(K / 8) * 128;         // Bg: next 8-row group
@@ -128,8 +190,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1) merge_tc_kernel(const apr_merge
       const apr_merge_proj pj = projs[lo];
       const int row0 = (strip - s_pref[lo]) * TC_BM;
       const int nrows = min(TC_BM, pj.d_out - row0);
-      const __nv_bfloat16* __restrict__ Wt = reinterpret_cast<const __nv_bfloat16*>(pj.W);
-      __nv_bfloat16* __restrict__ Wp = reinterpret_cast<__nv_bfloat16*>(pj.Wp);
+      const __nv_bfloat16* Wt = reinterpret_cast<const __nv_bfloat16*>(pj.W);
+      // out of place: W' to Wp; in place: back over W, with the residual codes in Wp (int8)
+      __nv_bfloat16* Wp = MODE == MERGE_OUT_OF_PLACE ? reinterpret_cast<__nv_bfloat16*>(pj.Wp)
+                                                     : const_cast<__nv_bfloat16*>(Wt);
+      int8_t* Rc = MODE == MERGE_OUT_OF_PLACE ? nullptr : reinterpret_cast<int8_t*>(pj.Wp);
       // gated B rows of the strip, bf16 hi + lo, K-major
       {
         const int n = row0 + tid;
@@ -202,6 +267,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1) merge_tc_kernel(const apr_merge
         const int slot = ct % MT_NY;
         const int c0 = ct * MT_BN;
         const int ncols = min(MT_BN, pj.d_in - c0);
+        // unmerge: this row's residual codes of the tile, loaded now so that their latency passes
+        // under the MMA's
+        uint4 tile_codes[MODE == UNMERGE_IN_PLACE ? 8 : 1];
+        if (MODE == UNMERGE_IN_PLACE) {
+          const uint4* rt = reinterpret_cast<const uint4*>(Rc + ((size_t)(row0 / TC_BM) * nct + ct) * 8 * 2048) + tid;
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            tile_codes[q] = (q * 16 < ncols && tid < nrows) ? rt[q * 128] : make_uint4(0, 0, 0, 0);
+        }
         if (ct + MT_NY - 1 < nct) issue_tile(ct + MT_NY - 1);
         cp_async_commit();
         cp_async_wait<MT_NY - 1>();
@@ -230,18 +304,124 @@ __global__ void __launch_bounds__(TC_THREADS, 1) merge_tc_kernel(const apr_merge
             tmem_ld16(lane_addr + (uint32_t)cc, v);
             if (tid < nrows) {
               uint4* pr = reinterpret_cast<uint4*>(wrow + cc * 2);
-              uint4 u0 = pr[0], u1 = pr[1];
-              __nv_bfloat162* h0 = reinterpret_cast<__nv_bfloat162*>(&u0);
-              __nv_bfloat162* h1 = reinterpret_cast<__nv_bfloat162*>(&u1);
+              if (MODE == MERGE_OUT_OF_PLACE) {
+                uint4 u0 = pr[0], u1 = pr[1];
+                __nv_bfloat162* h0 = reinterpret_cast<__nv_bfloat162*>(&u0);
+                __nv_bfloat162* h1 = reinterpret_cast<__nv_bfloat162*>(&u1);
 #pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const float2 f0 = __bfloat1622float2(h0[i]);
-                const float2 f1 = __bfloat1622float2(h1[i]);
-                h0[i] = __floats2bfloat162_rn(f0.x + v[2 * i], f0.y + v[2 * i + 1]);
-                h1[i] = __floats2bfloat162_rn(f1.x + v[8 + 2 * i], f1.y + v[8 + 2 * i + 1]);
+                for (int i = 0; i < 4; ++i) {
+                  const float2 f0 = __bfloat1622float2(h0[i]);
+                  const float2 f1 = __bfloat1622float2(h1[i]);
+                  h0[i] = __floats2bfloat162_rn(f0.x + v[2 * i], f0.y + v[2 * i + 1]);
+                  h1[i] = __floats2bfloat162_rn(f1.x + v[8 + 2 * i], f1.y + v[8 + 2 * i + 1]);
+                }
+                pr[0] = u0;
+                pr[1] = u1;
+              } else {
+                // residual codes, tile-major: [strip][column tile][16-column chunk][row][16 bytes],
+                // so a warp's 32 rows of one chunk are 512 contiguous bytes
+                unsigned int* hw = reinterpret_cast<unsigned int*>(pr);       // 8 x bf16 pairs
+                uint4* rc = reinterpret_cast<uint4*>(Rc + (((size_t)(row0 / TC_BM) * nct + ct) * 8 + (cc >> 4)) * 2048) + tid;
+                uint4 cw = make_uint4(0, 0, 0, 0);
+                uint32_t* cwd = reinterpret_cast<uint32_t*>(&cw);
+                uint32_t bf16_orig[16];                                       // W bits (escapes)
+                if (MODE == MERGE_IN_PLACE) {
+#pragma unroll
+                  for (int i = 0; i < 16; ++i) bf16_orig[i] = (hw[i >> 1] >> (16 * (i & 1))) & 0xFFFFu;
+                  // common path on bf16 pairs; elements whose distance does not fit a code are
+                  // marked and settled below, one warp-wide counter update per chunk
+                  uint32_t esc_mask = 0;
+#pragma unroll
+                  for (int i = 0; i < 16; i += 2) {
+                    const uint32_t w2 = hw[i >> 1];
+                    const uint32_t m2 = bf16x2_bits(__floats2bfloat162_rn(bf16_val(w2 & 0xFFFFu) + v[i],
+                                                                          bf16_val(w2 >> 16) + v[i + 1]));
+                    const uint32_t u2 = bf16x2_bits(__floats2bfloat162_rn(bf16_val(m2 & 0xFFFFu) - v[i],
+                                                                          bf16_val(m2 >> 16) - v[i + 1]));
+                    const uint32_t kw = bf16_key2(w2), ku = bf16_key2(u2);
+                    const int dl = (int)(kw & 0xFFFFu) - (int)(ku & 0xFFFFu);
+                    const int dh = (int)(kw >> 16) - (int)(ku >> 16);
+                    esc_mask |= ((uint32_t)(dl + 126) > 253u ? 1u : 0u) << i;
+                    esc_mask |= ((uint32_t)(dh + 126) > 253u ? 1u : 0u) << (i + 1);
+                    const uint32_t pair = ((uint32_t)dl & 0xFFu) | (((uint32_t)dh & 0xFFu) << 8);
+                    cwd[i >> 2] |= pair << (16 * ((i >> 1) & 1));
+                    hw[i >> 1] = m2;
+                  }
+                  if (ncols - cc < 16) esc_mask &= (1u << (ncols - cc)) - 1u;   // columns past the weight
+                  const unsigned int act = __activemask();
+                  const unsigned int want = __ballot_sync(act, esc_mask != 0);
+                  if (want) {
+                    const int leader = __ffs(want) - 1;
+                    unsigned int base = 0;
+                    const unsigned int before = __popc(esc_mask);
+                    // exclusive scan of the active lanes' escape counts (rarely taken)
+                    unsigned int offs = 0, total_w = 0;
+                    for (int l = 0; l < 32; ++l) {
+                      const unsigned int n_l = __shfl_sync(act, before, l);
+                      if ((act >> l) & 1u) {
+                        total_w += n_l;
+                        if (l < lane) offs += n_l;
+                      }
+                    }
+                    if (lane == leader) base = atomicAdd(&esc->count, total_w);
+                    base = __shfl_sync(act, base, leader);
+                    int8_t* code = reinterpret_cast<int8_t*>(&cw);
+                    for (int i = 0; i < 16; ++i) {
+                      if (!((esc_mask >> i) & 1u)) continue;
+                      const uint32_t wb = bf16_orig[i];
+                      const unsigned int slot = base + offs++;
+                      if ((long)slot < esc_cap) {
+                        unsigned int* ent = reinterpret_cast<unsigned int*>(esc + 1) + 3 * (size_t)slot;
+                        ent[0] = (unsigned int)lo;
+                        ent[1] = (unsigned int)((size_t)(row0 + tid) * pj.d_in + c0 + cc + i);
+                        ent[2] = wb;
+                        code[i] = kCodeEscape;
+                      } else {
+                        code[i] = kCodeKept;                           // no room: left unmerged
+                        hw[i >> 1] = (hw[i >> 1] & ~(0xFFFFu << (16 * (i & 1)))) | (wb << (16 * (i & 1)));
+                        report(ws, APR_ERR_WORKSPACE, K_MERGE, lo);
+                      }
+                    }
+                  }
+                  *rc = cw;
+                } else {
+#pragma unroll
+                  for (int q = 0; q < 8; ++q)
+                    if (q == (cc >> 4)) cw = tile_codes[q];
+                  // bytes 0x80 / 0x81 (escape / kept) anywhere in the chunk take the slow path
+                  uint32_t special = 0;
+#pragma unroll
+                  for (int q = 0; q < 4; ++q) special |= __vcmpeq4(cwd[q], 0x80808080u) | __vcmpeq4(cwd[q], 0x81818181u);
+                  if (!__any_sync(__activemask(), special != 0)) {
+#pragma unroll
+                    for (int i = 0; i < 16; i += 2) {
+                      const uint32_t w2 = hw[i >> 1];
+                      const uint32_t u2 = bf16x2_bits(__floats2bfloat162_rn(bf16_val(w2 & 0xFFFFu) - v[i],
+                                                                            bf16_val(w2 >> 16) - v[i + 1]));
+                      // the two codes sign-extended to 16-bit halves, added to the keys of u
+                      const uint32_t c2 = prmt_sext(cwd[i >> 2], ((i >> 1) & 1) ? 0xB3A2u : 0x9180u);
+                      hw[i >> 1] = bf16_from_key2(__vadd2(bf16_key2(u2), c2));
+                    }
+                  } else {
+                    // a chunk of this warp holds an escape or a kept element: element by element
+#pragma unroll
+                    for (int i = 0; i < 16; i += 2) {
+                      const uint32_t w2 = hw[i >> 1];
+                      const uint32_t u2 = bf16x2_bits(__floats2bfloat162_rn(bf16_val(w2 & 0xFFFFu) - v[i],
+                                                                            bf16_val(w2 >> 16) - v[i + 1]));
+                      uint32_t out = 0;
+#pragma unroll
+                      for (int h = 0; h < 2; ++h) {
+                        const int8_t c = reinterpret_cast<const int8_t*>(&cw)[i + h];
+                        const uint32_t wb = (w2 >> (16 * h)) & 0xFFFFu, ub = (u2 >> (16 * h)) & 0xFFFFu;
+                        const uint32_t rb = c == kCodeKept ? wb : (c == kCodeEscape ? ub : bf16_from_key(bf16_key(ub) + c));
+                        out |= rb << (16 * h);
+                      }
+                      hw[i >> 1] = out;
+                    }
+                  }
+                }
               }
-              pr[0] = u0;
-              pr[1] = u1;
             }
           }
           __syncwarp();
@@ -605,6 +785,52 @@ cudaError_t launch_merge_tma(const apr_merge_proj* projs, const void* plan, int 
                     reinterpret_cast<const CUtensorMap*>(plan), nproj, E, r, round16(r), idx, gate, k, ws);
 }
 
+// The unmerge's last step: every escaped element gets its exact bits back (unless the routing
+// is not the merge's, in which case the unmerge itself refused and wrote nothing).
+__global__ void __launch_bounds__(256) merge_escape_kernel(const apr_merge_proj* __restrict__ projs,
+                                                           const MergeEscapes* esc, long esc_cap,
+                                                           const int32_t* __restrict__ idx,
+                                                           const float* __restrict__ gate, int k) {
+  pdl_wait();
+  pdl_trigger();
+  bool same = esc->k == k;
+  for (int j = 0; j < k && same; ++j) same = esc->e[j] == idx[j] && esc->g[j] == gate[j];
+  if (!same) return;
+  const long n = min((long)esc->count, esc_cap);
+  const unsigned int* ent = reinterpret_cast<const unsigned int*>(esc + 1);
+  for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x) {
+    const unsigned int p = ent[3 * i], el = ent[3 * i + 1], bits = ent[3 * i + 2];
+    reinterpret_cast<unsigned short*>(const_cast<void*>(projs[p].W))[el] = (unsigned short)bits;
+  }
+}
+
+size_t merge_escape_bytes(long capacity) { return sizeof(MergeEscapes) + (size_t)12 * (size_t)capacity; }
+size_t merge_residual_bytes(int d_out, int d_in) {
+  return (size_t)((d_out + TC_BM - 1) / TC_BM) * (size_t)((d_in + MT_BN - 1) / MT_BN) * TC_BM * MT_BN;
+}
+
+cudaError_t launch_merge_inplace(const apr_merge_proj* projs, int nproj, int E, int r, const int32_t* idx,
+                                 const float* gate, int k, void* escapes, long capacity, bool unmerge, void* ws,
+                                 cudaStream_t s) {
+  const size_t smem = MtSmem::fixed_bytes() + sizeof(int) * ((size_t)nproj + 1);
+  static SmemLimit lim1, lim2;
+  cudaError_t err;
+  MergeEscapes* esc = reinterpret_cast<MergeEscapes*>(escapes);
+  const int nsm = device_sm_count();
+  if (!unmerge) {
+    if ((err = lim1.ensure((const void*)merge_tc_kernel<MERGE_IN_PLACE>, smem)) != cudaSuccess) return err;
+    if ((err = cudaMemsetAsync(esc, 0, sizeof(MergeEscapes), s)) != cudaSuccess) return err;
+    return launch_pdl(merge_tc_kernel<MERGE_IN_PLACE>, dim3(nsm), dim3(TC_THREADS), smem, s, projs, nproj, E, r,
+                      round16(r), idx, gate, k, ws, esc, capacity);
+  }
+  if ((err = lim2.ensure((const void*)merge_tc_kernel<UNMERGE_IN_PLACE>, smem)) != cudaSuccess) return err;
+  if ((err = launch_pdl(merge_tc_kernel<UNMERGE_IN_PLACE>, dim3(nsm), dim3(TC_THREADS), smem, s, projs, nproj, E, r,
+                        round16(r), idx, gate, k, ws, esc, capacity)) != cudaSuccess)
+    return err;
+  return launch_pdl(merge_escape_kernel, dim3(nsm), dim3(256), 0, s, projs, (const MergeEscapes*)esc, capacity, idx,
+                    gate, k);
+}
+
 bool merge_tensor_supported(int k, int r, int nproj) {
   return k * round16(r) <= TC_MAXN1 && nproj <= MT_MAXPROJ;
 }
@@ -613,11 +839,11 @@ cudaError_t launch_merge_tensor(const apr_merge_proj* projs, int nproj, int E, i
                                 const float* gate, int k, void* ws, cudaStream_t s) {
   const size_t smem = MtSmem::fixed_bytes() + sizeof(int) * ((size_t)nproj + 1);
   static SmemLimit limit;
-  cudaError_t err = limit.ensure((const void*)merge_tc_kernel, smem);
+  cudaError_t err = limit.ensure((const void*)merge_tc_kernel<MERGE_OUT_OF_PLACE>, smem);
   if (err != cudaSuccess) return err;
   const int nsm = device_sm_count();
-  return launch_pdl(merge_tc_kernel, dim3(nsm), dim3(TC_THREADS), smem, s, projs, nproj, E, r, round16(r), idx,
-                    gate, k, ws);
+  return launch_pdl(merge_tc_kernel<MERGE_OUT_OF_PLACE>, dim3(nsm), dim3(TC_THREADS), smem, s, projs, nproj, E, r,
+                    round16(r), idx, gate, k, ws, (MergeEscapes*)nullptr, 0L);
 }
 
 }  // namespace apr

@@ -9,12 +9,15 @@ full-size workloads (decode, multitenant, merge) are timed in the same run and
 reported under ``workloads``, and so is ``prefill_fused``: the prefill layers
 with their base projections, each call the base GEMM and the adapters in one
 contraction (apr_linear_lora), beside the unfused pipeline it replaces (a
-library GEMM, then the SGMM add).  Each step is captured once in a CUDA graph
+library GEMM, then the SGMM add), and ``merge_crossover``: for 1-8 tokens that
+share one routing, the steps after which an in-place merge (with its exact
+unmerge) beats adding the adapters unmerged.  Each step is captured once in a CUDA graph
 and replayed; ``e2e`` times the eager C-ABI calls with the step's activations
 copied in from and out to pinned host memory.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
-                    [--also decode,multitenant,merge,prefill_fused|none] [--impl reference]
+                    [--also decode,multitenant,merge,prefill_fused,merge_crossover|none]
+                    [--impl reference]
 
 With N > 1 (torchrun, one process per GPU) every rank runs its own batch
 (weak scaling: tokens are independent and the path has no exchange step);
@@ -626,6 +629,115 @@ def measure(name, args, world, rank, local, peaks, kernel_name="auto"):
     return out
 
 
+def merge_crossover(args, world, rank, local, batches=(1, 2, 4, 8)):
+    """Merge in place vs unmerged adapters for a batch of T tokens that share one routing
+    (the 224 decode-shaped weights of the merge workload, its first token's top-2 adapters).
+    Per step, merged: a library GEMM of the T rows on every merged weight; unmerged: the same
+    GEMM on W plus the SGMM call of every (layer, group) adding the adapters.  The in-place
+    merge + exact unmerge is paid once per routing change, so merging pays after
+    N* = (merge + unmerge) / (unmerged - merged) steps with the same adapters."""
+    import torch
+    from adapter_pregate_router_b200 import apr
+    from adapter_pregate_router_b200 import workloads as W
+
+    cfg = W.scaled(W.CONFIGS["merge"], seed=W.CONFIGS["merge"].seed + rank)
+    if args.layers:
+        cfg = W.scaled(cfg, layers=args.layers)
+    dev = torch.device("cuda", local)
+    E, k, r = cfg.E, cfg.k, 16
+    Tmax = max(batches)
+    h, Wr, _ = W.router_inputs(cfg)
+    ws = apr.workspace(Tmax, k, E, r, max(g.d_in for g in cfg.groups), device=dev)
+    idx1 = torch.empty((1, k), dtype=torch.int32, device=dev)
+    gate1 = torch.empty((1, k), dtype=torch.float32, device=dev)
+    apr.pregate_route(torch.from_numpy(h).to(dev, torch.bfloat16), torch.from_numpy(Wr).to(dev, torch.bfloat16),
+                      k, idx1, gate1, ws)
+    ranks = torch.full((E,), r, dtype=torch.int32, device=dev)
+    entries, groups, keep = [], [], []
+    for l in range(cfg.layers):
+        for g in cfg.groups:
+            x = W.device_tensor(cfg, W.xm_key(l, g.name, g.proj_names[0]), (Tmax * g.d_in,), dev).view(Tmax, g.d_in)
+            projs = []
+            for p, d_out in zip(g.proj_names, g.d_outs):
+                Wt = W.device_tensor(cfg, W.w_key(l, g.name, p), (d_out, g.d_in), dev)
+                A = [W.device_tensor(cfg, W.a_key(l, g.name, p, e), (r, g.d_in), dev) for e in range(E)]
+                B = [W.device_tensor(cfg, W.b_key(l, g.name, p, e), (d_out, r), dev) for e in range(E)]
+                At, Bt = apr.ptr_array(A, dev), apr.ptr_array(B, dev)
+                R = apr.merge_residual(Wt)
+                y = torch.empty((Tmax, d_out), dtype=torch.bfloat16, device=dev)
+                entries.append((Wt, R, At, Bt))
+                projs.append((Wt, y, At, Bt))
+                keep += [A, B]
+            groups.append((x, projs))
+    W.clear_device_pools()
+    nmerge = len(entries)
+    table = apr.merge_table(entries, dev)
+    esc = apr.merge_escapes(1 << 22, dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def timed(fn, reps):
+        with torch.cuda.stream(stream):
+            fn()
+            stream.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                fn()
+            for _ in range(2):
+                g.replay()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(reps):
+                g.replay()
+            e1.record(stream)
+        stream.synchronize()
+        apr.stream_status(ws, stream)
+        g.reset()
+        return max_over_ranks(e0.elapsed_time(e1) / reps, world)
+
+    def merge_unmerge():
+        apr.merge_adapters_inplace(table, nmerge, E, r, idx1, gate1, k, esc, ws)
+        apr.unmerge_adapters_inplace(table, nmerge, E, r, idx1, gate1, k, esc, ws)
+
+    mu_ms = timed(merge_unmerge, 5)
+    rows = []
+    for T in batches:
+        idx = idx1.expand(T, k).contiguous()
+        gate = gate1.expand(T, k).contiguous()
+        seg_off = torch.empty(E + 1, dtype=torch.int32, device=dev)
+        perm = torch.empty(T * k, dtype=torch.int32, device=dev)
+        apr.segment_tokens(idx, E, seg_off, perm, ws)
+        calls = []
+        for x, projs in groups:
+            xt = x[:T]
+            pj = [apr.make_proj(y[:T], y[:T], At, Bt) for (_, y, At, Bt) in projs]
+            calls.append((xt, [(Wt, y[:T]) for (Wt, y, _, _) in projs], pj))
+
+        def base_only():
+            for xt, gemms, _ in calls:
+                for Wt, yt in gemms:
+                    torch.matmul(xt, Wt.t(), out=yt)
+
+        def unmerged():
+            for xt, gemms, pj in calls:
+                for Wt, yt in gemms:
+                    torch.matmul(xt, Wt.t(), out=yt)
+                apr.sgmm_shrink_expand(xt, pj, k, E, ranks, r, idx, gate, seg_off, perm, ws)
+
+        m_ms = timed(base_only, 10)
+        u_ms = timed(unmerged, 10)
+        extra = u_ms - m_ms
+        rows.append({"T": T, "merged_step_ms": m_ms, "unmerged_step_ms": u_ms,
+                     "steps_to_pay_back": (mu_ms / extra) if extra > 0 else None})
+    del table, entries, groups, keep
+    import gc
+    gc.collect()
+    torch.cuda.empty_cache()
+    return {"weights": nmerge, "merge_plus_unmerge_ms": mu_ms,
+            "merged": "in-place merge, library GEMM of the T rows on W', exact in-place unmerge",
+            "unmerged": "library GEMM on W, then apr_sgmm_shrink_expand per (layer, group) in place",
+            "batches": rows}
+
+
 def run_gpu(args, world, rank, local):
     from adapter_pregate_router_b200 import workloads as W
     peaks = load_peaks()
@@ -635,6 +747,9 @@ def run_gpu(args, world, rank, local):
     also = [] if args.also in ("", "none") else [w.strip() for w in args.also.split(",")]
     for name in also:
         if name == args.workload:
+            continue
+        if name == "merge_crossover":
+            others[name] = merge_crossover(args, world, rank, local)
             continue
         r = measure(name, args, world, rank, local, peaks)
         others[name] = {"value": r["value"], "unit": "tokens/s", "ms_per_step": r["ms_per_step"],
@@ -667,7 +782,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="prefill", choices=["decode", "prefill", "multitenant", "merge", "tiny"])
-    ap.add_argument("--also", default="decode,multitenant,merge,prefill_fused",
+    ap.add_argument("--also", default="decode,multitenant,merge,prefill_fused,merge_crossover",
                     help="other full-size workloads timed in the same run and reported under 'workloads' "
                          "(comma-separated, or 'none')")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])

@@ -255,6 +255,37 @@ apr_status apr_merge_adapters(const apr_merge_proj* projs, int nproj, int E, int
                               size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * In-place merge and exact unmerge (section 2.B steps 3 and 5: merge the
+ * token's adapters, run the base model, unmerge for the next token), all
+ * weights in one launch each, without a second copy of W.
+ * apr_merge_adapters_inplace  W <- rn(W + sum_j gate[j] B_{idx[j]} A_{idx[j]}),
+ *      the same values as apr_merge_adapters writes to Wp, bit for bit.  For
+ *      this call projs[p].Wp is NOT a weight: it receives the residual codes
+ *      that make the unmerge exact, one byte per element in a tiled layout of
+ *      its own (device, caller-owned, 16-byte aligned,
+ *      apr_merge_residual_bytes(d_out, d_in) bytes).
+ * apr_unmerge_adapters_inplace  restores every W bit for bit from W', the
+ *      residual codes and `escapes`, recomputing the same delta: idx and gate
+ *      must be the merge's (checked on the device: APR_ERR_INVALID_ARG from
+ *      apr_stream_status, and no weight is touched, otherwise).
+ * escapes  device, caller-owned, 16-byte aligned, apr_merge_escape_bytes(c)
+ *      bytes for c escapes: elements whose restoring distance does not fit a
+ *      code (typically |W| far below the delta) keep their exact bits there.
+ *      When more than c are needed, the excess elements are left unmerged (so
+ *      the unmerge is still exact) and the merge reports APR_ERR_WORKSPACE.
+ * Needs k * round16(r) <= 64 (APR_ERR_UNSUPPORTED otherwise).  Between the
+ * two calls neither W nor the codes nor `escapes` may change.
+ * ---------------------------------------------------------------------- */
+size_t apr_merge_escape_bytes(long capacity);
+size_t apr_merge_residual_bytes(int d_out, int d_in);
+apr_status apr_merge_adapters_inplace(const apr_merge_proj* projs, int nproj, int E, int r,
+                                      const int32_t* idx, const float* gate, int k, void* escapes,
+                                      size_t escape_bytes, void* ws, size_t ws_bytes, void* stream);
+apr_status apr_unmerge_adapters_inplace(const apr_merge_proj* projs, int nproj, int E, int r,
+                                        const int32_t* idx, const float* gate, int k, void* escapes,
+                                        size_t escape_bytes, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * Merge plan: TMA descriptors of every weight pair (W, Wp).  The weights'
  * addresses and shapes do not change from one token to the next, so a plan is
  * built once for a set of weights and then used by every

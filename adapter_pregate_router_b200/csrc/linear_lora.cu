@@ -55,6 +55,19 @@ constexpr uint32_t LL_STAGE = LL_ABYTES + LL_BBYTES;
 constexpr uint32_t LL_TMEM_COLS = 512;            // two 256-column accumulators
 constexpr size_t LL_SMEM = (size_t)LL_ST * LL_STAGE + 256 + 1024;
 
+// Tile order: groups of LL_GN column tiles (of all projections in a row); inside a group the
+// row tile advances every LL_GN tiles.  The CTAs in flight at any time then cover a band of about
+// (CTAs / LL_GN) row tiles x LL_GN column tiles, whose x rows and W columns both stay in L2,
+// instead of every row tile of x against one column block.
+constexpr int LL_GN = 8;
+__device__ __forceinline__ void grouped_tile(int tile, int mt, int ncols, int& nt, int& m) {
+  const int per_group = LL_GN * mt;
+  const int g = tile / per_group, r = tile - g * per_group;
+  const int width = min(LL_GN, ncols - g * LL_GN);       // the last group may be narrower
+  m = r / width;
+  nt = g * LL_GN + (r - m * width);
+}
+
 struct LinPlan {
   CUtensorMap xmap;                      // x [T, d_in]: boxes of 64 columns x 128 rows
   CUtensorMap wmap[APR_MAX_PROJ];        // W_p [d_out, d_in]: 64 x 256
@@ -104,8 +117,9 @@ __global__ void __launch_bounds__(LL_THREADS, 1) linear_lora_kernel(const __grid
   const int mt = P.mt, nkb = P.nbase + P.nlora;
   const int total = P.nt_before[P.nproj] * mt;
   auto tile_at = [&](int tile, int& p, int& n0, int& m0) {
-    const int nt = tile / mt;
-    m0 = (tile - nt * mt) * LL_BM;
+    int nt, m;
+    grouped_tile(tile, mt, P.nt_before[P.nproj], nt, m);
+    m0 = m * LL_BM;
     p = 0;
     while (p + 1 < P.nproj && nt >= P.nt_before[p + 1]) ++p;
     n0 = (nt - P.nt_before[p]) * LL_BN;
@@ -269,8 +283,9 @@ __global__ void __launch_bounds__(LL_THREADS, 1) linear_lora_pair_kernel(const _
   const int total = P.nt_before[P.nproj] * mt;
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   auto tile_at = [&](int tile, int& p, int& n0, int& m0) {
-    const int nt = tile / mt;
-    m0 = (tile - nt * mt) * 2 * LL_BM;
+    int nt, m;
+    grouped_tile(tile, mt, P.nt_before[P.nproj], nt, m);
+    m0 = m * 2 * LL_BM;
     p = 0;
     while (p + 1 < P.nproj && nt >= P.nt_before[p + 1]) ++p;
     n0 = (nt - P.nt_before[p]) * LL_BN;

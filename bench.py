@@ -760,7 +760,7 @@ def run_gpu(args, world, rank, local):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(W.CONFIGS[args.workload], budget_s=args.ref_budget)
+        cpu = cpu_baseline(W.CONFIGS[BASE_MODE.get(args.workload, (args.workload,))[0]], budget_s=args.ref_budget)
 
     line = {
         "metric": METRIC, "value": main["value"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -781,7 +781,8 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="prefill", choices=["decode", "prefill", "multitenant", "merge", "tiny"])
+    ap.add_argument("--workload", default="prefill",
+                    choices=["decode", "prefill", "multitenant", "merge", "tiny", "prefill_fused"])
     ap.add_argument("--also", default="decode,multitenant,merge,prefill_fused,merge_crossover",
                     help="other full-size workloads timed in the same run and reported under 'workloads' "
                          "(comma-separated, or 'none')")

@@ -770,6 +770,8 @@ def run_gpu(args, world, rank, local):
         "clocks": main["clocks"], "gpu_launches": main["gpu_launches"],
         "launches_per_step": main["launches_per_step"],
     }
+    if "unfused" in main:
+        line["unfused"] = main["unfused"]
     if others:
         line["workloads"] = others
     if rank == 0:

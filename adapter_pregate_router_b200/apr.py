@@ -87,6 +87,11 @@ _linear = _sig("apr_linear_lora", _i,
                 [_vp, _i, ctypes.POINTER(LinearProj), _i, _i, _i, _i, _vp, _i, _vp, _vp, _vp, _vp, _vp, _sz, _vp])
 _linear_workspace_size = _sig("apr_linear_workspace_size", _sz, [_i, _i, _i, _i, _i, _i, ctypes.c_long])
 _merge = _sig("apr_merge_adapters", _i, [_vp, _i, _i, _i, _vp, _vp, _i, _vp, _sz, _vp])
+_pool_state_bytes = _sig("apr_adapter_pool_state_bytes", _sz, [_i, _i])
+_pool_init = _sig("apr_adapter_pool_init", _i,
+                  [_vp, _sz, _i, _i, ctypes.POINTER(_vp), _sz, _vp, _vp, _sz, _vp, _vp, _i, _vp])
+_pool_page_in = _sig("apr_adapter_pool_page_in", _i,
+                     [_vp, _sz, _i, _i, _vp, _i, _i, _vp, _sz, _vp, _sz, _vp, _vp, _i, _vp, _sz, _vp])
 _merge_escape_bytes = _sig("apr_merge_escape_bytes", _sz, [ctypes.c_long])
 _merge_residual_bytes = _sig("apr_merge_residual_bytes", _sz, [_i, _i])
 _merge_inplace = _sig("apr_merge_adapters_inplace", _i, [_vp, _i, _i, _i, _vp, _vp, _i, _vp, _sz, _vp, _sz, _vp])
@@ -102,7 +107,8 @@ _kernel_launches = _sig("apr_kernel_launches", ctypes.c_uint64, [])
 
 EXPORTED = ("apr_workspace_size", "apr_workspace_init", "apr_pregate_route", "apr_pregate_route_noalloc",
             "apr_segment_tokens",
-            "apr_sgmm_shrink_expand", "apr_linear_lora", "apr_linear_workspace_size", "apr_merge_adapters", "apr_merge_escape_bytes", "apr_merge_residual_bytes", "apr_merge_adapters_inplace",
+            "apr_sgmm_shrink_expand", "apr_linear_lora", "apr_linear_workspace_size", "apr_adapter_pool_state_bytes", "apr_adapter_pool_init", "apr_adapter_pool_page_in",
+            "apr_merge_adapters", "apr_merge_escape_bytes", "apr_merge_residual_bytes", "apr_merge_adapters_inplace",
             "apr_unmerge_adapters_inplace", "apr_merge_plan_size", "apr_merge_plan_init",
             "apr_merge_adapters_planned", "apr_gemv", "apr_stream_status",
             "apr_last_error", "apr_status_string", "apr_kernel_launches")
@@ -392,6 +398,64 @@ def merge_adapters_planned(table, plan, nproj, E, r, idx, gate, k, ws, stream=No
 def merge_adapters(table, nproj, E, r, idx, gate, k, ws, stream=None):
     _check_merge_args(table, nproj, idx, gate, k, ws)
     _check(_merge(_ptr(table), nproj, E, r, _ptr(idx), _ptr(gate), k, _ptr(ws), ws.numel(), _stream(stream)))
+
+
+class AdapterPool:
+    """Adapters in pinned host memory, ``n_slots`` of them resident on the device at a time
+    (``apr_adapter_pool_*``).  ``host_buffers``: pinned uint8 CPU tensors of ``adapter_bytes``
+    each (one per adapter, the layout given by ``offsets``); ``tables``: int64 device tensors
+    [n_adapters] (the A/B pointer tables the SGMM calls take), each with the byte offset of its
+    matrix inside an adapter."""
+
+    def __init__(self, host_buffers, n_slots, tables, offsets, device="cuda", stream=None):
+        self.n_adapters = len(host_buffers)
+        self.n_slots = int(n_slots)
+        sizes = {int(b.numel() * b.element_size()) for b in host_buffers}
+        if len(sizes) != 1:
+            raise ValueError("every adapter buffer must have the same size")
+        self.adapter_bytes = sizes.pop()
+        for i, b in enumerate(host_buffers):
+            if b.is_cuda or not b.is_pinned() or not b.is_contiguous():
+                raise ValueError(f"host_buffers[{i}] must be a contiguous pinned CPU tensor")
+        if len(tables) != len(offsets):
+            raise ValueError("one offset per table")
+        for i, t in enumerate(tables):
+            _need(t, f"tables[{i}]", (torch.int64,), shape=(self.n_adapters,))
+        n = int(_pool_state_bytes(self.n_adapters, self.n_slots))
+        if n == 0:
+            raise AprError(APR_ERR_INVALID_ARG, "adapter_pool_state_bytes: arguments out of range")
+        self.state = torch.empty(n, dtype=torch.uint8, device=device)
+        self.pool = torch.empty(self.n_slots * self.adapter_bytes, dtype=torch.uint8, device=device)
+        self.src_table = torch.empty(self.n_adapters, dtype=torch.int64, device=device)
+        self.tables = list(tables)
+        self.table_ptrs = torch.tensor([t.data_ptr() for t in tables], dtype=torch.int64, device=device)
+        self.offsets = torch.tensor([int(o) for o in offsets], dtype=torch.int64, device=device)
+        self.host_buffers = list(host_buffers)
+        srcs = (_vp * self.n_adapters)(*[b.data_ptr() for b in host_buffers])
+        _check(_pool_init(_ptr(self.state), n, self.n_adapters, self.n_slots, srcs, self.adapter_bytes,
+                          _ptr(self.src_table), _ptr(self.pool), self.pool.numel(), _ptr(self.offsets),
+                          _ptr(self.table_ptrs), len(self.tables), _stream(stream)))
+
+    def page_in(self, idx, ws, stream=None):
+        """Make every adapter ``idx`` [T, k] selects resident and point the tables at it."""
+        _need(idx, "idx", (torch.int32,), ndim=2)
+        _need_ws(ws)
+        _same_device(("idx", idx), ("ws", ws), ("state", self.state))
+        T, k = idx.shape
+        _check(_pool_page_in(_ptr(self.state), self.state.numel(), self.n_adapters, self.n_slots, _ptr(idx), T, k,
+                             _ptr(self.src_table), self.adapter_bytes, _ptr(self.pool), self.pool.numel(),
+                             _ptr(self.offsets), _ptr(self.table_ptrs), len(self.tables), _ptr(ws), ws.numel(),
+                             _stream(stream)))
+
+    def stats(self):
+        """(page-in calls, adapters copied in so far), synchronising."""
+        h = self.state[:64].cpu()
+        step = int(h[16:24].view(torch.int64).item())
+        copies = int(h[24:32].view(torch.int64).item())
+        return step, copies
+
+    def slot_ptr(self, slot: int) -> int:
+        return self.pool.data_ptr() + slot * self.adapter_bytes
 
 
 def merge_escape_bytes(capacity: int) -> int:

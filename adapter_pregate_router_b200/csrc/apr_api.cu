@@ -7,6 +7,8 @@
 
 #include <atomic>
 
+#include <vector>
+
 #include "apr_internal.cuh"
 
 namespace apr {
@@ -413,6 +415,83 @@ apr_status apr_unmerge_adapters_inplace(const apr_merge_proj* projs, int nproj, 
                                         const float* gate, int k, void* escapes, size_t escape_bytes, void* ws,
                                         size_t ws_bytes, void* stream) {
   return merge_inplace_call(projs, nproj, E, r, idx, gate, k, escapes, escape_bytes, ws, ws_bytes, stream, true);
+}
+
+size_t apr_adapter_pool_state_bytes(int n_adapters, int n_slots) {
+  if (n_adapters < 1 || n_adapters > APR_MAX_E || n_slots < 1 || n_slots > APR_MAX_E) return 0;
+  return adapter_pool_state_bytes(n_adapters, n_slots);
+}
+
+apr_status apr_adapter_pool_init(void* state, size_t state_bytes, int n_adapters, int n_slots,
+                                 const void* const* host_src, size_t adapter_bytes, void* host_src_table,
+                                 void* pool, size_t pool_bytes, const uint64_t* offsets, void* const* tables,
+                                 int ntab, void* stream) {
+  const size_t need = apr_adapter_pool_state_bytes(n_adapters, n_slots);
+  if (need == 0) return fail(APR_ERR_INVALID_ARG, "adapter_pool_init: n_adapters=%d, n_slots=%d outside [1, %d]",
+                             n_adapters, n_slots, APR_MAX_E);
+  if (!state || state_bytes < need || !aligned16(state))
+    return fail(APR_ERR_WORKSPACE, "adapter_pool_init: state NULL, unaligned or below %zu bytes", need);
+  if (!host_src || !host_src_table) return fail(APR_ERR_INVALID_ARG, "adapter_pool_init: NULL pointer");
+  if (adapter_bytes < 16 || adapter_bytes % 16)
+    return fail(APR_ERR_INVALID_ARG, "adapter_pool_init: adapter_bytes=%zu must be a positive multiple of 16", adapter_bytes);
+  if (!pool || !aligned16(pool) || pool_bytes / adapter_bytes < (size_t)n_slots)
+    return fail(APR_ERR_INVALID_ARG, "adapter_pool_init: pool NULL, unaligned or below n_slots * adapter_bytes");
+  if (ntab < 0 || (ntab > 0 && (!offsets || !tables)))
+    return fail(APR_ERR_INVALID_ARG, "adapter_pool_init: NULL tables/offsets or ntab=%d < 0", ntab);
+  if (ntab > 0) {
+    // offsets are read on the host here once (the kernels trust them afterwards)
+    std::vector<uint64_t> off((size_t)ntab);
+    cudaError_t e = cudaMemcpy(off.data(), offsets, sizeof(uint64_t) * (size_t)ntab, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "adapter_pool_init: reading offsets");
+    for (int t = 0; t < ntab; ++t)
+      if (off[t] % 16 || off[t] >= adapter_bytes)
+        return fail(APR_ERR_INVALID_ARG, "adapter_pool_init: offsets[%d]=%llu not a multiple of 16 below adapter_bytes",
+                    t, (unsigned long long)off[t]);
+  }
+  // every source must be pinned host memory the device reads at the same address
+  for (int i = 0; i < n_adapters; ++i) {
+    cudaPointerAttributes at;
+    if (!host_src[i] || !aligned16(host_src[i]) || cudaPointerGetAttributes(&at, host_src[i]) != cudaSuccess ||
+        at.type != cudaMemoryTypeHost || at.devicePointer != host_src[i]) {
+      (void)cudaGetLastError();
+      return fail(APR_ERR_INVALID_ARG, "adapter_pool_init: host_src[%d] is not 16-byte aligned pinned, mapped host memory", i);
+    }
+  }
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaMemcpyAsync(host_src_table, host_src, sizeof(void*) * (size_t)n_adapters, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);     // the host array may go once this returns
+  if (e == cudaSuccess)
+    e = launch_pool_init(state, n_adapters, n_slots, pool, pool_bytes,
+                         reinterpret_cast<const unsigned long long*>(offsets), tables, ntab, s);
+  if (e != cudaSuccess) return cuda_fail(e, "adapter_pool_init");
+  return APR_OK;
+}
+
+apr_status apr_adapter_pool_page_in(void* state, size_t state_bytes, int n_adapters, int n_slots,
+                                    const int32_t* idx, int T, int k, const void* const* host_src_table,
+                                    size_t adapter_bytes, void* pool, size_t pool_bytes,
+                                    const uint64_t* offsets, void* const* tables, int ntab, void* ws,
+                                    size_t ws_bytes, void* stream) {
+  const size_t need = apr_adapter_pool_state_bytes(n_adapters, n_slots);
+  if (need == 0) return fail(APR_ERR_INVALID_ARG, "adapter_pool_page_in: n_adapters=%d, n_slots=%d outside [1, %d]",
+                             n_adapters, n_slots, APR_MAX_E);
+  if (!state || state_bytes < need || !aligned16(state))
+    return fail(APR_ERR_WORKSPACE, "adapter_pool_page_in: state NULL, unaligned or below %zu bytes", need);
+  if (T < 0 || k < 1 || k > APR_MAX_K) return fail(APR_ERR_INVALID_ARG, "adapter_pool_page_in: T=%d, k=%d", T, k);
+  if (adapter_bytes < 16 || adapter_bytes % 16)
+    return fail(APR_ERR_INVALID_ARG, "adapter_pool_page_in: adapter_bytes=%zu must be a positive multiple of 16", adapter_bytes);
+  if (!pool || !aligned16(pool) || pool_bytes / adapter_bytes < (size_t)n_slots)
+    return fail(APR_ERR_INVALID_ARG, "adapter_pool_page_in: pool NULL, unaligned or below n_slots * adapter_bytes");
+  if (ntab < 0 || (ntab > 0 && (!offsets || !tables)) || !host_src_table)
+    return fail(APR_ERR_INVALID_ARG, "adapter_pool_page_in: NULL pointer or ntab=%d < 0", ntab);
+  if (T > 0 && !idx) return fail(APR_ERR_INVALID_ARG, "adapter_pool_page_in: NULL idx");
+  apr_status st = check_ws(ws, ws_bytes, sizeof(WsHeader), "adapter_pool_page_in");
+  if (st) return st;
+  cudaError_t e = launch_pool_page_in(state, n_adapters, n_slots, idx, T * k, host_src_table, adapter_bytes, pool,
+                                      reinterpret_cast<const unsigned long long*>(offsets), tables, ntab, ws,
+                                      (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "adapter_pool_page_in launch");
+  return APR_OK;
 }
 
 apr_status apr_gemv(const void* W, const void* x, void* y, int d_in, int d_out, void* stream) {

@@ -252,7 +252,7 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 // Kernel ids used in WsHeader::err_info.
-enum KernelId { K_ROUTE = 1, K_TOPK = 2, K_SEGMENT = 3, K_SHRINK = 4, K_EXPAND = 5, K_MERGE = 6, K_TC = 7, K_LINEAR = 8 };
+enum KernelId { K_ROUTE = 1, K_TOPK = 2, K_SEGMENT = 3, K_SHRINK = 4, K_EXPAND = 5, K_MERGE = 6, K_TC = 7, K_LINEAR = 8, K_POOL = 9 };
 
 }  // namespace apr
 
@@ -332,6 +332,13 @@ cudaError_t launch_sgmm_dense(const SgmmArgs& a, size_t scratch_off, cudaStream_
 cudaError_t launch_sgmm_bank(const SgmmArgs& a, size_t scratch_off, cudaStream_t s);
 bool sgmm_bank_supported(const SgmmArgs& a, int dtype);
 bool linear_lora_supported(const SgmmArgs& a);
+size_t adapter_pool_state_bytes(int n_adapters, int n_slots);
+cudaError_t launch_pool_init(void* state, int n_adapters, int n_slots, void* pool, size_t pool_bytes,
+                             const unsigned long long* offsets, void* const* tables, int ntab, cudaStream_t s);
+cudaError_t launch_pool_page_in(void* state, int n_adapters, int n_slots, const int32_t* idx, int nq,
+                                const void* const* host_src, size_t adapter_bytes, void* pool,
+                                const unsigned long long* offsets, void* const* tables, int ntab, void* ws,
+                                cudaStream_t s);
 cudaError_t launch_linear_lora(const SgmmArgs& a, const void* const* W, size_t scratch_off, cudaStream_t s);
 bool sgmm_dense_supported(const SgmmArgs& a, int dtype);
 bool sgmm_tensor_supported(const SgmmArgs& a, int dtype);

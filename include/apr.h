@@ -232,6 +232,56 @@ apr_status apr_linear_lora(const void* x, int d_in, const apr_linear_proj* projs
 size_t apr_linear_workspace_size(int T, int k, int E, int max_rank, int max_d_in, int nproj,
                                  long sum_d_out);
 
+/* ------------------------------------------------------------------------
+ * Adapter paging (the Chameleon page: adapters loaded on demand, the popular
+ * ones kept resident in an adaptive cache, as in S-LoRA).  n_adapters adapters
+ * live in pinned host memory, each one contiguous buffer of adapter_bytes
+ * holding its A and B matrices of every (layer, projection) at fixed offsets;
+ * n_slots device slots (a caller-owned pool of n_slots * adapter_bytes) hold
+ * the ones a step selects.  The SGMM calls keep taking device tables of A and
+ * B pointers indexed by adapter id (E = n_adapters); paging rewrites the
+ * entries of the adapters it brings in.
+ * apr_adapter_pool_state_bytes  device bytes of the pool's state (0 if an
+ *      argument is outside [1, APR_MAX_E]).
+ * apr_adapter_pool_init  host_src: HOST array [n_adapters] of the adapters'
+ *      buffers, each 16-byte aligned pinned host memory that the device reads
+ *      at the same address (checked: APR_ERR_INVALID_ARG otherwise);
+ *      host_src_table: device array [n_adapters] the call fills with them.
+ *      Empties every slot, zeroes the pool and points every entry of every
+ *      table at slot 0's copy: the dense and bank SGMM kernels read the whole
+ *      adapter bank (a zero gate removes the adapters a token did not
+ *      select), so an entry must always point at finite data in the pool.
+ *      offsets: device array [ntab], read once here (multiples of 16 below
+ *      adapter_bytes).  Synchronises `stream` (set-up call).
+ * apr_adapter_pool_page_in  after the router, before the step's SGMM calls:
+ *      every adapter idx [T, k] selects becomes resident (empty slots first,
+ *      then the least recently used slots this step does not need), copied
+ *      from its host buffer by a kernel, and for each of the ntab tables
+ *      (device array `tables`, each a device array [n_adapters] of pointers)
+ *      its entry becomes pool + slot * adapter_bytes + offsets[t] (device
+ *      array [ntab], multiples of 16 below adapter_bytes).  Asynchronous, no
+ *      host round trip.  More distinct adapters in idx than slots:
+ *      APR_ERR_WORKSPACE from apr_stream_status and nothing changes.  The
+ *      entries of adapters not resident keep pointing at a copy in the pool
+ *      (another adapter's or zeros): kernels that read the whole bank get
+ *      finite data, which the zero gates of those adapters remove.  Nothing
+ *      after the copy starts before it is complete (the copy kernel does not
+ *      release its dependents early), since the SGMM kernels may read
+ *      adapter weights before their own dependency wait.
+ * ---------------------------------------------------------------------- */
+size_t apr_adapter_pool_state_bytes(int n_adapters, int n_slots);
+apr_status apr_adapter_pool_init(void* state, size_t state_bytes, int n_adapters, int n_slots,
+                                 const void* const* host_src, size_t adapter_bytes,
+                                 void* host_src_table, void* pool, size_t pool_bytes,
+                                 const uint64_t* offsets, void* const* tables, int ntab,
+                                 void* stream);
+apr_status apr_adapter_pool_page_in(void* state, size_t state_bytes, int n_adapters, int n_slots,
+                                    const int32_t* idx, int T, int k,
+                                    const void* const* host_src_table, size_t adapter_bytes,
+                                    void* pool, size_t pool_bytes, const uint64_t* offsets,
+                                    void* const* tables, int ntab, void* ws, size_t ws_bytes,
+                                    void* stream);
+
 /* One weight of the merge step. */
 typedef struct apr_merge_proj {
   const void* W;          /* device [d_out, d_in] bf16 base weight (never written) */

@@ -109,7 +109,7 @@ size_t apr_linear_workspace_size(int T, int k, int E, int max_rank, int max_d_in
   const size_t base = apr_workspace_size(T, k, E, max_rank, max_d_in);
   if (base == 0 || nproj < 1 || nproj > APR_MAX_PROJ || sum_d_out < 8 || sum_d_out > (1L << 30)) return 0;
   const WsLayout L = ws_layout(T, k, E);
-  const size_t lin = L.scratch + align_up(linear_scratch_bytes(T, k, E, max_rank, nproj, sum_d_out)) + kAlign;
+  const size_t lin = L.scratch + align_up(linear_scratch_bytes(T, k, E, max_rank, nproj, sum_d_out, max_d_in)) + kAlign;
   return lin > base ? lin : base;
 }
 
@@ -322,7 +322,7 @@ apr_status apr_linear_lora(const void* x, int d_in, const apr_linear_proj* projs
   if (!x || !ranks || !idx || !gate || !seg_off || !perm) return fail(APR_ERR_INVALID_ARG, "linear_lora: NULL pointer");
   if (!aligned16(x)) return fail(APR_ERR_INVALID_ARG, "linear_lora: x not 16-byte aligned");
   const WsLayout L = ws_layout(T, k, E);
-  st = check_ws(ws, ws_bytes, L.scratch + linear_scratch_bytes(T, k, E, max_rank, nproj, sum_d_out), "linear_lora");
+  st = check_ws(ws, ws_bytes, L.scratch + linear_scratch_bytes(T, k, E, max_rank, nproj, sum_d_out, d_in), "linear_lora");
   if (st) return st;
 
   SgmmArgs a;

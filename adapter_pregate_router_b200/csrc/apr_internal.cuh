@@ -148,19 +148,20 @@ inline size_t sgmm_scratch_bytes(int T, int k, int E, int max_rank, int d_in) {
 // Fused base projection + adapters: gated v per pair [proj][pair][R16] bf16, the bank rows
 // V [proj][T][E * R16] bf16, then each projection's Bcat [d_out][E * R16] bf16 (aligned blocks).
 struct LinearScratch {
-  size_t vc, v, bcat;
+  size_t vc, abank, v, bcat;
 };
-inline LinearScratch linear_scratch(int T, int k, int E, int max_rank, int nproj) {
+inline LinearScratch linear_scratch(int T, int k, int E, int max_rank, int nproj, int d_in) {
   const size_t R16 = (size_t)round16i(max_rank);
   LinearScratch L;
   L.vc = 0;
-  L.v = align_up((size_t)nproj * T * k * R16 * 2);
+  L.abank = align_up((size_t)nproj * T * k * R16 * 2);
+  L.v = L.abank + align_up((size_t)nproj * E * R16 * d_in * 2);
   L.bcat = L.v + align_up((size_t)nproj * T * E * R16 * 2);
   return L;
 }
 // Bytes for nproj projections whose output widths add up to sum_d_out.
-inline size_t linear_scratch_bytes(int T, int k, int E, int max_rank, int nproj, long sum_d_out) {
-  const LinearScratch L = linear_scratch(T, k, E, max_rank, nproj);
+inline size_t linear_scratch_bytes(int T, int k, int E, int max_rank, int nproj, long sum_d_out, int d_in) {
+  const LinearScratch L = linear_scratch(T, k, E, max_rank, nproj, d_in);
   return L.bcat + align_up((size_t)sum_d_out * E * round16i(max_rank) * 2) + (size_t)nproj * kAlign;
 }
 
@@ -340,6 +341,9 @@ cudaError_t launch_pool_page_in(void* state, int n_adapters, int n_slots, const 
                                 const unsigned long long* offsets, void* const* tables, int ntab, void* ws,
                                 cudaStream_t s);
 cudaError_t launch_linear_lora(const SgmmArgs& a, const void* const* W, size_t scratch_off, cudaStream_t s);
+// The bank shrink of the fused call: gated v per pair [proj][t * k + j][R16] at vc_off from one
+// GEMM of x with each projection's adapter bank, packed at abank_off.
+cudaError_t launch_bank_shrink(const SgmmArgs& a, size_t vc_off, size_t abank_off, cudaStream_t s);
 bool sgmm_dense_supported(const SgmmArgs& a, int dtype);
 bool sgmm_tensor_supported(const SgmmArgs& a, int dtype);
 cudaError_t launch_merge(const apr_merge_proj* projs, int nproj, int E, int r, const int32_t* idx,

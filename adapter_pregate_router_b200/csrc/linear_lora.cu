@@ -21,8 +21,11 @@
 //
 // Steps of one call (all on the caller's stream, chained by programmatic
 // dependent launch):
-//  1. the tensor-core shrink (pair order) writes g * A_e x per (token, slot)
-//     in bf16 to the workspace;
+//  1. the shrink, also on the tensor cores: each projection's adapters are
+//     packed into one bank [E * R16, d_in] and x is contracted with the whole
+//     bank by the same tile kernel (x by TMA, no gather); its epilogue keeps
+//     each token's selected adapters' columns, times their gates, as g * A_e x
+//     per (token, slot) in bf16;
 //  2. a pack kernel spreads those rows over the bank's rank slots (V, zeros
 //     where a token did not select an adapter) and lays the projection's B_e
 //     side by side (Bcat), both row-major in the workspace;
@@ -55,6 +58,16 @@ constexpr uint32_t LL_STAGE = LL_ABYTES + LL_BBYTES;
 constexpr uint32_t LL_TMEM_COLS = 512;            // two 256-column accumulators
 constexpr size_t LL_SMEM = (size_t)LL_ST * LL_STAGE + 256 + 1024;
 
+// One-CTA tile kernel, instantiated as the fused GEMM's (BN = 256, y stored) and as the bank
+// shrink's (BN = 128, gated columns scattered to the pair rows): ring depth and TMEM from BN.
+constexpr int EPI_STORE_Y = 0, EPI_SHRINK = 1;
+template <int BN> struct TileCfg {
+  static constexpr uint32_t stage = LL_ABYTES + (uint32_t)BN * 128;
+  static constexpr int st = BN >= 256 ? 4 : 6;
+  static constexpr uint32_t tmem_cols = 2 * BN < 32 ? 32 : 2 * BN;
+  static constexpr size_t smem = (size_t)st * stage + 256 + 1024;
+};
+
 // Tile order: groups of LL_GN column tiles (of all projections in a row); inside a group the
 // row tile advances every LL_GN tiles.  The CTAs in flight at any time then cover a band of about
 // (CTAs / LL_GN) row tiles x LL_GN column tiles, whose x rows and W columns both stay in L2,
@@ -75,27 +88,34 @@ struct LinPlan {
   CUtensorMap bmap[APR_MAX_PROJ];        // Bcat_p [d_out, NB]: 64 x 256
   void* y[APR_MAX_PROJ];
   int d_out[APR_MAX_PROJ];
-  int nt_before[APR_MAX_PROJ + 1];       // prefix of 256-column tiles per projection
+  int nt_before[APR_MAX_PROJ + 1];       // prefix of column tiles per projection
   int nproj, T, nbase, nlora, mt;
   void* ws;
+  // bank shrink: the gated v rows [proj][t * k + j][R16] bf16, the routing
+  __nv_bfloat16* vc;
+  const int32_t* idx;
+  const float* gate;
+  int k, E, R16;
 };
 
-__global__ void __launch_bounds__(LL_THREADS, 1) linear_lora_kernel(const __grid_constant__ LinPlan P) {
+template <int BN, int EPI>
+__global__ void __launch_bounds__(LL_THREADS, 1) linear_tile_kernel(const __grid_constant__ LinPlan P) {
+  using C = TileCfg<BN>;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t sbase = smem_u32(smem);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)LL_ST * LL_STAGE);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)C::st * C::stage);
   const uint32_t bar_full = smem_u32(bars);                 // [ST] a K block landed (TMA bytes)
-  const uint32_t bar_empty = smem_u32(bars + LL_ST);        // [ST] its MMAs are done
-  const uint32_t bar_dfull = smem_u32(bars + 2 * LL_ST);    // [2]  accumulator complete
-  const uint32_t bar_dempty = smem_u32(bars + 2 * LL_ST + 2); // [2] accumulator read out
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 2 * LL_ST + 4);
+  const uint32_t bar_empty = smem_u32(bars + C::st);        // [ST] its MMAs are done
+  const uint32_t bar_dfull = smem_u32(bars + 2 * C::st);    // [2]  accumulator complete
+  const uint32_t bar_dempty = smem_u32(bars + 2 * C::st + 2); // [2] accumulator read out
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 2 * C::st + 4);
   int* s_consumed = reinterpret_cast<int*>(s_tmem + 1);
 
   if (tid == 0) {
-    for (int i = 0; i < LL_ST; ++i) {
+    for (int i = 0; i < C::st; ++i) {
       mbar_init(bar_full + 8 * i, 1);
       mbar_init(bar_empty + 8 * i, 1);
     }
@@ -106,7 +126,7 @@ __global__ void __launch_bounds__(LL_THREADS, 1) linear_lora_kernel(const __grid
     *s_consumed = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 0) tmem_alloc(smem_u32(s_tmem), LL_TMEM_COLS);
+  if (warp == 0) tmem_alloc(smem_u32(s_tmem), C::tmem_cols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -122,7 +142,7 @@ __global__ void __launch_bounds__(LL_THREADS, 1) linear_lora_kernel(const __grid
     m0 = m * LL_BM;
     p = 0;
     while (p + 1 < P.nproj && nt >= P.nt_before[p + 1]) ++p;
-    n0 = (nt - P.nt_before[p]) * LL_BN;
+    n0 = (nt - P.nt_before[p]) * BN;
   };
   bool abort = false;
   int issued = 0;                                  // K blocks issued by the producer
@@ -134,10 +154,10 @@ __global__ void __launch_bounds__(LL_THREADS, 1) linear_lora_kernel(const __grid
         int p, n0, m0;
         tile_at(tile, p, n0, m0);
         for (int kb = 0; kb < nkb; ++kb) {
-          const int s = issued % LL_ST;
-          if (!mbar_wait(bar_empty + 8 * s, ((issued / LL_ST) & 1) ^ 1)) { abort = true; break; }
-          const uint32_t sa = sbase + (uint32_t)s * LL_STAGE, sb = sa + LL_ABYTES;
-          mbar_arrive_expect_tx(bar_full + 8 * s, LL_STAGE);
+          const int s = issued % C::st;
+          if (!mbar_wait(bar_empty + 8 * s, ((issued / C::st) & 1) ^ 1)) { abort = true; break; }
+          const uint32_t sa = sbase + (uint32_t)s * C::stage, sb = sa + LL_ABYTES;
+          mbar_arrive_expect_tx(bar_full + 8 * s, C::stage);
           if (kb < P.nbase) {
             tma_load_2d(sa, &P.xmap, kb * LL_BK, m0, bar_full + 8 * s);
             tma_load_2d(sb, &P.wmap[p], kb * LL_BK, n0, bar_full + 8 * s);
@@ -153,18 +173,18 @@ __global__ void __launch_bounds__(LL_THREADS, 1) linear_lora_kernel(const __grid
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issue
     if (lane == 0) {
-      const uint32_t id = idesc_bf16(LL_BM, LL_BN);
+      const uint32_t id = idesc_bf16(LL_BM, BN);
       int g = 0, it = 0;
       for (int tile = blockIdx.x; tile < total && !abort; tile += gridDim.x, ++it) {
         const int ab = it & 1;
         if (!mbar_wait(bar_dempty + 8 * ab, ((it >> 1) & 1) ^ 1)) { abort = true; break; }
         tc_fence_after();
-        const uint32_t d = tmem + (uint32_t)ab * LL_BN;
+        const uint32_t d = tmem + (uint32_t)ab * BN;
         for (int kb = 0; kb < nkb; ++kb, ++g) {
-          const int s = g % LL_ST;
-          if (!mbar_wait(bar_full + 8 * s, (g / LL_ST) & 1)) { abort = true; break; }
+          const int s = g % C::st;
+          if (!mbar_wait(bar_full + 8 * s, (g / C::st) & 1)) { abort = true; break; }
           tc_fence_after();
-          const uint32_t sa = sbase + (uint32_t)s * LL_STAGE, sb = sa + LL_ABYTES;
+          const uint32_t sa = sbase + (uint32_t)s * C::stage, sb = sa + LL_ABYTES;
 #pragma unroll
           for (int kk = 0; kk < LL_BK / 16; ++kk)
             mma_bf16(d, desc_k_sw128(sa + kk * 32), desc_k_sw128(sb + kk * 32), id, (kb | kk) != 0 ? 1u : 0u);
@@ -187,10 +207,56 @@ __global__ void __launch_bounds__(LL_THREADS, 1) linear_lora_kernel(const __grid
       if (!mbar_wait(bar_dfull + 8 * ab, (it >> 1) & 1)) { abort = true; break; }
       tc_fence_after();
       const int t = m0 + row, d_out = P.d_out[p];
-      __nv_bfloat16* yrow = reinterpret_cast<__nv_bfloat16*>(P.y[p]) + (size_t)t * d_out;
-      const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)ab * LL_BN;
+      const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)ab * BN;
+      if (EPI == EPI_SHRINK) {
+        // row t's bank columns n0 .. n0 + BN: the columns of each adapter the token selected,
+        // times its gate, go to the token's pair row (t * k + j) of v
+        int ej[APR_MAX_K];
+        float gj[APR_MAX_K];
+#pragma unroll
+        for (int j = 0; j < APR_MAX_K; ++j) {
+          ej[j] = -1;
+          gj[j] = 0.f;
+          if (j < P.k && t < P.T) {
+            ej[j] = P.idx[(size_t)t * P.k + j];
+            gj[j] = P.gate[(size_t)t * P.k + j];
+            if (ej[j] < 0 || ej[j] >= P.E) {
+              if (n0 == 0) report(P.ws, APR_ERR_DEVICE_INDEX, K_LINEAR, ej[j]);
+              ej[j] = -1;
+            }
+          }
+        }
+        __nv_bfloat16* vrow = P.vc + ((size_t)p * P.T * P.k + (size_t)t * P.k) * P.R16;
 #pragma unroll 1
-      for (int c32 = 0; c32 < LL_BN / 32; ++c32) {
+        for (int c32 = 0; c32 < BN / 32; ++c32) {
+          float v[32];
+          tmem_ld32(taddr + (uint32_t)(c32 * 32), v);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int c = n0 + c32 * 32 + 16 * h;                 // first bank column of this half
+#pragma unroll
+            for (int j = 0; j < APR_MAX_K; ++j) {
+              const int lo = ej[j] * P.R16;
+              if (ej[j] >= 0 && c >= lo && c < lo + P.R16) {
+                uint4 u[2];
+                uint32_t* w = reinterpret_cast<uint32_t*>(u);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                  const __nv_bfloat162 b2 =
+                      __floats2bfloat162_rn(gj[j] * v[16 * h + 2 * q], gj[j] * v[16 * h + 2 * q + 1]);
+                  w[q] = *reinterpret_cast<const uint32_t*>(&b2);
+                }
+                uint4* dst = reinterpret_cast<uint4*>(vrow + (size_t)j * P.R16 + (c - lo));
+                dst[0] = u[0];
+                dst[1] = u[1];
+              }
+            }
+          }
+        }
+      } else {
+      __nv_bfloat16* yrow = reinterpret_cast<__nv_bfloat16*>(P.y[p]) + (size_t)t * d_out;
+#pragma unroll 1
+      for (int c32 = 0; c32 < BN / 32; ++c32) {
         float v[32];
         tmem_ld32(taddr + (uint32_t)(c32 * 32), v);
         const int col = n0 + c32 * 32;
@@ -210,6 +276,7 @@ __global__ void __launch_bounds__(LL_THREADS, 1) linear_lora_kernel(const __grid
           }
         }
       }
+      }
       tc_fence_before();
       mbar_arrive(bar_dempty + 8 * ab);
     }
@@ -219,12 +286,12 @@ __global__ void __launch_bounds__(LL_THREADS, 1) linear_lora_kernel(const __grid
     if (tid == 0) report(P.ws, APR_ERR_TIMEOUT, K_LINEAR, (int)blockIdx.x);
     // copies issued but never consumed land before the shared memory is released
     if (warp == 0 && lane == 0)
-      for (int g = *s_consumed; g < issued; ++g) (void)mbar_wait(bar_full + 8 * (g % LL_ST), (g / LL_ST) & 1);
+      for (int g = *s_consumed; g < issued; ++g) (void)mbar_wait(bar_full + 8 * (g % C::st), (g / C::st) & 1);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 0) tmem_dealloc(tmem, LL_TMEM_COLS);
+  if (warp == 0) tmem_dealloc(tmem, C::tmem_cols);
 }
 
 // ---------------------------------------------------------------- CTA pairs
@@ -462,15 +529,95 @@ __global__ void __launch_bounds__(256) linear_pack_kernel(const __grid_constant_
   }
 }
 
-// ---------------------------------------------------------------- host side
+// ---------------------------------------------------------------- bank shrink
+// The shrink of the bank form: for each projection, S = x . Abank^T with Abank[e * R16 + i] =
+// A_e[i] (zero rows past an adapter's rank), one GEMM over the whole bank (E/k times the
+// products of the gathered shrink, on the tensor cores), x read by contiguous TMA boxes instead
+// of gathered rows.  Its epilogue keeps, for every token, the columns of the adapters it
+// selected, scaled by their gates, and writes them to the token's pair rows of v.
 
-cudaError_t launch_tc_shrink_pairs(const SgmmArgs& a, size_t v_off, cudaStream_t s);
+struct APackArgs {
+  const void* const* A[APR_MAX_PROJ];
+  __nv_bfloat16* Ab[APR_MAX_PROJ];       // [E * R16][d_in]
+  const int32_t* ranks;
+  int E, R16, d_in;
+  void* ws;
+};
+
+// one 16-byte chunk per thread step; blockIdx.y: the projection
+__global__ void __launch_bounds__(256) bank_pack_a_kernel(const __grid_constant__ APackArgs a) {
+  pdl_wait();                                      // the bank buffer's last readers
+  pdl_trigger();
+  const int p = blockIdx.y;
+  const __nv_bfloat16* const* Ap = reinterpret_cast<const __nv_bfloat16* const*>(a.A[p]);
+  __nv_bfloat16* dst = a.Ab[p];
+  const int cpr = a.d_in / 8;
+  const int total = a.E * a.R16 * cpr;
+  for (int w = blockIdx.x * blockDim.x + threadIdx.x; w < total; w += gridDim.x * blockDim.x) {
+    const int row = w / cpr, c = w - row * cpr;
+    const int e = row / a.R16, i = row - e * a.R16;
+    const int re = __ldg(a.ranks + e);
+    const bool ok = re >= 8 && re <= a.R16 && (re & 7) == 0;
+    if (!ok && i == 0 && c == 0) report(a.ws, APR_ERR_DEVICE_INDEX, K_LINEAR, e);
+    uint4 val = make_uint4(0, 0, 0, 0);
+    if (ok && i < re) val = *reinterpret_cast<const uint4*>(Ap[e] + (size_t)i * a.d_in + c * 8);
+    *reinterpret_cast<uint4*>(dst + (size_t)row * a.d_in + c * 8) = val;
+  }
+}
+
+cudaError_t launch_bank_shrink(const SgmmArgs& a, size_t vc_off, size_t abank_off, cudaStream_t s) {
+  constexpr int BN = 128;
+  const int R16 = round16i(a.max_rank), NB = a.E * R16;
+  APackArgs pk;
+  memset(&pk, 0, sizeof(pk));
+  pk.ranks = a.ranks;
+  pk.E = a.E;
+  pk.R16 = R16;
+  pk.d_in = a.d_in;
+  pk.ws = a.ws;
+  LinPlan P;
+  memset(&P, 0, sizeof(P));
+  cudaError_t err;
+  if ((err = encode_tile_map(&P.xmap, a.x, a.T, a.d_in, LL_BM)) != cudaSuccess) return err;
+  P.nt_before[0] = 0;
+  for (int p = 0; p < a.nproj; ++p) {
+    pk.A[p] = a.proj[p].A;
+    pk.Ab[p] = ws_at<__nv_bfloat16>(a.ws, abank_off + (size_t)p * NB * a.d_in * 2);
+    if ((err = encode_tile_map(&P.wmap[p], pk.Ab[p], NB, a.d_in, BN)) != cudaSuccess) return err;
+    P.d_out[p] = NB;
+    P.nt_before[p + 1] = P.nt_before[p] + (NB + BN - 1) / BN;
+  }
+  P.nproj = a.nproj;
+  P.T = a.T;
+  P.nbase = a.d_in / LL_BK;
+  P.nlora = 0;
+  P.mt = (a.T + LL_BM - 1) / LL_BM;
+  P.ws = a.ws;
+  P.vc = ws_at<__nv_bfloat16>(a.ws, vc_off);
+  P.idx = a.idx;
+  P.gate = a.gate;
+  P.k = a.k;
+  P.E = a.E;
+  P.R16 = R16;
+  static SmemLimit lim;
+  using Cfg = TileCfg<BN>;
+  if ((err = lim.ensure((const void*)linear_tile_kernel<BN, EPI_SHRINK>, Cfg::smem)) != cudaSuccess) return err;
+  const int nsm = device_sm_count();
+  const int chunks = NB * (a.d_in / 8);
+  const int pgrid = std::min((chunks + 255) / 256, 2 * nsm);
+  if ((err = launch_pdl(bank_pack_a_kernel, dim3(pgrid, a.nproj), dim3(256), 0, s, pk)) != cudaSuccess) return err;
+  const long tiles = (long)P.nt_before[a.nproj] * P.mt;
+  const int grid = (int)std::min<long>(tiles, nsm);
+  return launch_pdl(linear_tile_kernel<BN, EPI_SHRINK>, dim3(grid), dim3(LL_THREADS), Cfg::smem, s, P);
+}
+
+// ---------------------------------------------------------------- host side
 
 bool linear_lora_supported(const SgmmArgs& a) { return sgmm_bank_supported(a, APR_BF16); }
 
 cudaError_t launch_linear_lora(const SgmmArgs& a, const void* const* W, size_t scratch_off, cudaStream_t s) {
   const int R16 = round16i(a.max_rank), NB = a.E * R16;
-  const LinearScratch L = linear_scratch(a.T, a.k, a.E, a.max_rank, a.nproj);
+  const LinearScratch L = linear_scratch(a.T, a.k, a.E, a.max_rank, a.nproj, a.d_in);
   PackArgs pk;
   memset(&pk, 0, sizeof(pk));
   pk.vc = ws_at<__nv_bfloat16>(a.ws, scratch_off + L.vc);
@@ -520,16 +667,17 @@ cudaError_t launch_linear_lora(const SgmmArgs& a, const void* const* W, size_t s
   P.ws = a.ws;
 
   static SmemLimit lim, lim2;
-  if ((err = lim.ensure((const void*)linear_lora_kernel, LL_SMEM)) != cudaSuccess) return err;
+  if ((err = lim.ensure((const void*)linear_tile_kernel<LL_BN, EPI_STORE_Y>, TileCfg<LL_BN>::smem)) != cudaSuccess)
+    return err;
   if ((err = lim2.ensure((const void*)linear_lora_pair_kernel, L2_SMEM)) != cudaSuccess) return err;
-  if ((err = launch_tc_shrink_pairs(a, scratch_off + L.vc, s)) != cudaSuccess) return err;
+  if ((err = launch_bank_shrink(a, scratch_off + L.vc, scratch_off + L.abank, s)) != cudaSuccess) return err;
   const int nsm = device_sm_count();
   const int pgrid = (int)std::min<long>((most + 255) / 256, 4L * nsm);
   if ((err = launch_pdl(linear_pack_kernel, dim3(pgrid, 1 + a.nproj), dim3(256), 0, s, pk)) != cudaSuccess) return err;
   const long tiles = (long)P.nt_before[a.nproj] * P.mt;
   if (!pairs) {
     const int grid = (int)std::min<long>(tiles, nsm);
-    return launch_pdl(linear_lora_kernel, dim3(grid), dim3(LL_THREADS), LL_SMEM, s, P);
+    return launch_pdl(linear_tile_kernel<LL_BN, EPI_STORE_Y>, dim3(grid), dim3(LL_THREADS), TileCfg<LL_BN>::smem, s, P);
   }
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[2];

@@ -248,7 +248,9 @@ __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+// Every copy this thread issued has landed, committed to a group or not (cp.async.wait_all;
+// "wait_group 0" alone would skip copies not yet committed).
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
@@ -333,6 +335,9 @@ cudaError_t launch_sgmm_dense(const SgmmArgs& a, size_t scratch_off, cudaStream_
 cudaError_t launch_sgmm_bank(const SgmmArgs& a, size_t scratch_off, cudaStream_t s);
 bool sgmm_bank_supported(const SgmmArgs& a, int dtype);
 bool linear_lora_supported(const SgmmArgs& a);
+bool route_tc_supported(int dtype, int d, int E, const void* h, const void* Wr);
+cudaError_t launch_route_tc(const void* h, const void* Wr, int T, int d, int E, int k, int32_t* idx, float* gate,
+                            void* ws, cudaStream_t s);
 size_t adapter_pool_state_bytes(int n_adapters, int n_slots);
 cudaError_t launch_pool_init(void* state, int n_adapters, int n_slots, void* pool, size_t pool_bytes,
                              const unsigned long long* offsets, void* const* tables, int ntab, cudaStream_t s);

@@ -60,7 +60,7 @@ constexpr size_t LL_SMEM = (size_t)LL_ST * LL_STAGE + 256 + 1024;
 
 // One-CTA tile kernel, instantiated as the fused GEMM's (BN = 256, y stored) and as the bank
 // shrink's (BN = 128, gated columns scattered to the pair rows): ring depth and TMEM from BN.
-constexpr int EPI_STORE_Y = 0, EPI_SHRINK = 1;
+constexpr int EPI_STORE_Y = 0, EPI_SHRINK = 1, EPI_ROUTE = 2;
 template <int BN> struct TileCfg {
   static constexpr uint32_t stage = LL_ABYTES + (uint32_t)BN * 128;
   static constexpr int st = BN >= 256 ? 4 : 6;
@@ -96,6 +96,9 @@ struct LinPlan {
   const int32_t* idx;
   const float* gate;
   int k, E, R16;
+  // router: top-k adapters and gates of every token
+  int32_t* ridx;
+  float* rgate;
 };
 
 template <int BN, int EPI>
@@ -208,7 +211,72 @@ __global__ void __launch_bounds__(LL_THREADS, 1) linear_tile_kernel(const __grid
       tc_fence_after();
       const int t = m0 + row, d_out = P.d_out[p];
       const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)ab * BN;
-      if (EPI == EPI_SHRINK) {
+      if (EPI == EPI_ROUTE) {
+        // the row's E logits (exact: products of bf16 values summed in fp32) -> the k largest,
+        // the lower adapter index first among equal logits, then the softmax over them
+        float tv[APR_MAX_K];
+        int te[APR_MAX_K];
+        float kth = -INFINITY;                                  // the k-th largest so far
+#pragma unroll
+        for (int j = 0; j < APR_MAX_K; ++j) {
+          tv[j] = -INFINITY;
+          te[j] = 0x7FFFFFFF;
+        }
+#pragma unroll 1
+        for (int c32 = 0; c32 < BN / 32; ++c32) {
+          float v[32];
+          tmem_ld32(taddr + (uint32_t)(c32 * 32), v);
+#pragma unroll
+          for (int u = 0; u < 32; ++u) {
+            const int e = n0 + c32 * 32 + u;
+            float x = v[u];
+            if (e >= P.E || !(x > kth)) continue;              // ascending e: an equal logit never displaces
+            int xe = e;
+#pragma unroll
+            for (int j = 0; j < APR_MAX_K; ++j) {              // insertion, largest first; a displaced
+              if (j < P.k && (x > tv[j] || (x == tv[j] && xe < te[j]))) {   // entry keeps index order
+                const float sv = tv[j];
+                const int se = te[j];
+                tv[j] = x;
+                te[j] = xe;
+                x = sv;
+                xe = se;
+              }
+            }
+#pragma unroll
+            for (int j = 0; j < APR_MAX_K; ++j)
+              if (j == P.k - 1) kth = tv[j];
+          }
+        }
+        bool short_k = false;
+#pragma unroll
+        for (int j = 0; j < APR_MAX_K; ++j)
+          if (j == P.k - 1) short_k = te[j] == 0x7FFFFFFF;
+        if (t < P.T) {
+          if (short_k) {                                        // fewer than k non-NaN logits
+            report(P.ws, APR_ERR_DEVICE_INDEX, K_TOPK, t);
+#pragma unroll
+            for (int j = 0; j < APR_MAX_K; ++j)
+              if (te[j] == 0x7FFFFFFF) {
+                te[j] = 0;
+                tv[j] = 0.f;
+              }
+          }
+          float w[APR_MAX_K], sum = 0.f;
+#pragma unroll
+          for (int j = 0; j < APR_MAX_K; ++j) {
+            if (j >= P.k) break;
+            w[j] = expf(tv[j] - tv[0]);
+            sum += w[j];
+          }
+#pragma unroll
+          for (int j = 0; j < APR_MAX_K; ++j) {
+            if (j >= P.k) break;
+            P.ridx[(size_t)t * P.k + j] = te[j];
+            P.rgate[(size_t)t * P.k + j] = w[j] / sum;
+          }
+        }
+      } else if (EPI == EPI_SHRINK) {
         // row t's bank columns n0 .. n0 + BN: the columns of each adapter the token selected,
         // times its gate, go to the token's pair row (t * k + j) of v
         int ej[APR_MAX_K];
@@ -609,6 +677,52 @@ cudaError_t launch_bank_shrink(const SgmmArgs& a, size_t vc_off, size_t abank_of
   const long tiles = (long)P.nt_before[a.nproj] * P.mt;
   const int grid = (int)std::min<long>(tiles, nsm);
   return launch_pdl(linear_tile_kernel<BN, EPI_SHRINK>, dim3(grid), dim3(LL_THREADS), Cfg::smem, s, P);
+}
+
+// ---------------------------------------------------------------- router on the tensor cores
+// Logits L = h Wr^T for a bank of at most 256 adapters as one tile GEMM (h and Wr by TMA, M = 128
+// tokens, N = the bank padded to 64/128/256), top-k and gates in the epilogue from TMEM: one
+// launch, no partials in memory.
+
+bool route_tc_supported(int dtype, int d, int E, const void* h, const void* Wr) {
+  return dtype == APR_BF16 && d % LL_BK == 0 && E >= 1 && E <= 256 &&
+         reinterpret_cast<uintptr_t>(h) % 16 == 0 && reinterpret_cast<uintptr_t>(Wr) % 16 == 0;
+}
+
+template <int BN>
+static cudaError_t launch_route_tc_bn(LinPlan& P, cudaStream_t s) {
+  static SmemLimit lim;
+  using Cfg = TileCfg<BN>;
+  cudaError_t err;
+  if ((err = lim.ensure((const void*)linear_tile_kernel<BN, EPI_ROUTE>, Cfg::smem)) != cudaSuccess) return err;
+  const int grid = std::min(P.mt, device_sm_count());
+  return launch_pdl(linear_tile_kernel<BN, EPI_ROUTE>, dim3(grid), dim3(LL_THREADS), Cfg::smem, s, P);
+}
+
+cudaError_t launch_route_tc(const void* h, const void* Wr, int T, int d, int E, int k, int32_t* idx, float* gate,
+                            void* ws, cudaStream_t s) {
+  const int BN = E <= 64 ? 64 : (E <= 128 ? 128 : 256);
+  LinPlan P;
+  memset(&P, 0, sizeof(P));
+  cudaError_t err;
+  if ((err = encode_tile_map(&P.xmap, h, T, d, LL_BM)) != cudaSuccess) return err;
+  if ((err = encode_tile_map(&P.wmap[0], Wr, E, d, BN)) != cudaSuccess) return err;
+  P.nt_before[0] = 0;
+  P.nt_before[1] = 1;
+  P.d_out[0] = E;
+  P.nproj = 1;
+  P.T = T;
+  P.nbase = d / LL_BK;
+  P.nlora = 0;
+  P.mt = (T + LL_BM - 1) / LL_BM;
+  P.ws = ws;
+  P.k = k;
+  P.E = E;
+  P.ridx = idx;
+  P.rgate = gate;
+  if (BN == 64) return launch_route_tc_bn<64>(P, s);
+  if (BN == 128) return launch_route_tc_bn<128>(P, s);
+  return launch_route_tc_bn<256>(P, s);
 }
 
 // ---------------------------------------------------------------- host side

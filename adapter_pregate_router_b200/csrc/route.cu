@@ -4,7 +4,11 @@
 // at the first adapted layer fixes each token's adapters for all later
 // layers; §2.B steps 1-2: one router pass per token, then Top-K selection.
 //
-// Two launches:
+// bf16 inputs and at most 256 adapters: one launch on the tensor cores
+// (launch_route_tc: the tile GEMM of h and Wr, with top-k and gates in its
+// epilogue; the logits of bf16 inputs are exact in fp32 accumulation whatever
+// the summation order, for the integer-valued inputs the checks use).
+// Otherwise two launches:
 //   route_logits_kernel  split-K tiled product L = h Wr^T in fp32 (CUDA cores;
 //                        partial sums per K chunk, no atomics, so the result
 //                        does not depend on scheduling).  The router is tiny
@@ -169,6 +173,8 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
 
 cudaError_t launch_route(const void* h, const void* Wr, int dtype, int T, int d, int E, int k,
                          int32_t* idx, float* gate, void* ws, size_t scratch_off, cudaStream_t s) {
+  // bf16 banks of up to 256 adapters: logits, top-k and gates in one tensor-core launch
+  if (route_tc_supported(dtype, d, E, h, Wr)) return launch_route_tc(h, Wr, T, d, E, k, idx, gate, ws, s);
   const int tiles_t = (T + RT_M - 1) / RT_M;
   const int tiles_e = (E + RT_N - 1) / RT_N;
   const int tiles = tiles_t * tiles_e;

@@ -722,3 +722,23 @@ def test_kernels_on_a_second_device(apr):
             xs, As_d, Bs_d = x[:40], As, Bs
             close(run_sgmm(apr, xs, As_d, Bs_d, idx[:40], gate[:40], [ybs[0][:40]], BF16, kernel=apr.SGMM_DENSE)[0],
                   oracle_group(xs, As_d, Bs_d, idx[:40], gate[:40].astype(np.float64), [ybs[0][:40]])[0], "dense")
+
+
+def test_sgmm_bank_every_row_and_rerun_bits(apr):
+    """A prefill-shaped q/k/v group (8192 tokens, 16 adapters of rank 16, Zipf top-2) on the bank
+    kernel: every output row against the oracle, and three runs equal bit for bit.  Each CTA's
+    range of units crosses column blocks here, so a column block's Bcat is reloaded in the middle
+    of a CTA's work and the first unit after it reads it at once (a reload that is not complete
+    when the MMAs read it shows as wrong rows of the first row tile, differing from run to run)."""
+    rng = np.random.default_rng(95)
+    T, d_in, d_outs, ranks, k = 8192, 4096, (4096, 4096, 4096), (16,) * 16, 2
+    idx = _zipf_idx(rng, T, len(ranks), k)
+    x, As, Bs, idx, gate, ybs = _case(rng, T, d_in, d_outs, ranks, k, dist=idx)
+    x, As, Bs, ybs = _rounded(x, As, Bs, ybs)
+    runs = [run_sgmm(apr, x, As, Bs, idx, gate, ybs, BF16, kernel=apr.SGMM_BANK) for _ in range(3)]
+    for r in runs[1:]:
+        for p in range(3):
+            assert np.array_equal(r[p], runs[0][p]), f"proj {p}: runs differ"
+    ref = oracle_group(x, As, Bs, idx, gate.astype(np.float64), ybs)
+    for p in range(3):
+        close(runs[0][p], ref[p], f"bank proj {p} all rows")

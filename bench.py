@@ -583,7 +583,9 @@ def measure(name, args, world, rank, local, peaks, kernel_name="auto"):
             "achieved": tflops, "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
             "frac": tflops / peaks["bf16_tflops_sustained"],
             "peak_source": f"{peaks['source']} sustained bf16 dense (a long step under the power cap)",
-            "traffic": None, "traffic_source": "no capture of this workload",
+            "traffic": traffic,
+            "traffic_source": (f"{TRAFFIC_FILE} (ncu, bytes per call, kernel-source hash {kernel_source_hash()})"
+                               if traffic is not None else "no capture at the current kernel sources"),
             "flops_per_step": flops, "calls_per_step": ncalls, "us_per_call": layer_ms * 1e3 / ncalls,
             "hbm_frac": layer_bytes / (layer_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], "step_bytes": step_bytes,
         }

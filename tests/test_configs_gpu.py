@@ -147,3 +147,23 @@ def test_graph_replay_matches_eager(mods):
     apr.stream_status(step.ws)
     for key, ref in eager.items():
         assert torch.equal(step.outputs[key][0], ref), key
+
+
+@pytest.mark.parametrize("name", ["decode", "prefill", "multitenant"])
+def test_step_reruns_agree_bit_for_bit(mods, name):
+    """Two layers of the workload run four times: every output bit is the same each time (the
+    kernels have one writer per element and a fixed summation order, so a difference means a
+    race, e.g. a staged operand read before its copy landed)."""
+    apr, pipeline = mods
+    step = pipeline.Step(W.CONFIGS[name], layers=[0, 1])
+    ref = None
+    for _ in range(4):
+        step.act_out.fill_(float("nan"))
+        step.run()
+        apr.stream_status(step.ws)
+        if ref is None:
+            ref = step.act_out.clone()
+        assert torch.equal(step.act_out.view(torch.int16), ref.view(torch.int16))
+    del step
+    gc.collect()
+    torch.cuda.empty_cache()

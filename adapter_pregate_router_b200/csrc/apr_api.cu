@@ -245,8 +245,10 @@ apr_status apr_sgmm_shrink_expand(const void* x, int d_in, const apr_proj* projs
     e = launch_sgmm_bank(a, L.scratch, (cudaStream_t)stream);
   } else if (use == APR_SGMM_TENSOR) {
     if (!sgmm_tensor_supported(a, dtype))
-      return fail(APR_ERR_UNSUPPORTED, "sgmm: tensor-core kernel needs bf16, k<=2, max_rank<=64, d_in%%64==0, d_out%%16==0");
-    e = launch_sgmm_tensor(a, L.scratch, (cudaStream_t)stream);
+      return fail(APR_ERR_UNSUPPORTED, "sgmm: tensor-core kernel needs bf16 and d_in%%64==0, and for k=2 "
+                                       "max_rank<=32 and d_out%%16==0");
+    e = sgmm_ragged_supported(a, dtype) ? launch_sgmm_ragged(a, L.scratch, (cudaStream_t)stream)
+                                        : launch_sgmm_tensor(a, L.scratch, (cudaStream_t)stream);
   } else {
     e = launch_sgmm_skinny(a, dtype, L.scratch, (cudaStream_t)stream);
   }

@@ -129,6 +129,31 @@ inline size_t bank_scratch_bytes(int T, int k, int E, int max_rank) {
   return (size_t)APR_MAX_PROJ * T * k * R16 * 2;
 }
 
+// Many-tenant path (top-1 routing): ragged tiles of <= kSetTile consecutive plan tokens whose
+// adapters number <= kRgSlots and whose rank slots (each rank rounded up to 16) add up to
+// <= kRgKmax; an adapter with more tokens than fit goes on in the next tile.  Scratch: gated v
+// by plan position [projection][position][R16] bf16, then the tile count and the tiles.
+constexpr int kRgSlots = 16;
+constexpr int kRgKmax = 256;
+struct RgTile {
+  int start, len, nu, kt;     // plan positions [start, start + len); adapters; rank rows in all
+  short u[kRgSlots];          // the adapters, ascending
+  short koff[kRgSlots];       // first rank row of each adapter's slot (multiples of 16)
+};
+// A tile closes when it is full (<= ceil(T / 128) times) or when the next adapter does not fit
+// (such a tile holds an adapter that starts in it: <= min(E, T) times), plus the last one.
+__host__ __device__ inline int rg_max_tiles(int T, int E) {
+  return (T + kSetTile - 1) / kSetTile + (E < T ? E : T) + 1;
+}
+inline bool rg_dims_ok(int k, int max_rank) { return k == 1 && round16i(max_rank) <= 128; }
+inline size_t rg_vc_bytes(int T, int max_rank) {
+  return align_up((size_t)APR_MAX_PROJ * T * round16i(max_rank) * 2);
+}
+inline size_t rg_scratch_bytes(int T, int k, int E, int max_rank) {
+  if (!rg_dims_ok(k, max_rank)) return 0;
+  return rg_vc_bytes(T, max_rank) + 16 + sizeof(RgTile) * (size_t)rg_max_tiles(T, E);
+}
+
 // Shrink partial sums.  Gather paths: [projection][column chunk][sorted pair][rank]
 // fp32; dense path: [projection][cluster][token (padded to 16)][adapter * rank slot].
 inline size_t sgmm_scratch_bytes(int T, int k, int E, int max_rank, int d_in) {
@@ -142,6 +167,8 @@ inline size_t sgmm_scratch_bytes(int T, int k, int E, int max_rank, int d_in) {
   if (t > b) b = t;
   const size_t bk = bank_scratch_bytes(T, k, E, max_rank);
   if (bk > b) b = bk;
+  const size_t rg = rg_scratch_bytes(T, k, E, max_rank);
+  if (rg > b) b = rg;
   return b;
 }
 
@@ -331,6 +358,9 @@ struct SgmmArgs {
 };
 cudaError_t launch_sgmm_skinny(const SgmmArgs& a, int dtype, size_t scratch_off, cudaStream_t s);
 cudaError_t launch_sgmm_tensor(const SgmmArgs& a, size_t scratch_off, cudaStream_t s);
+bool sgmm_ragged_supported(const SgmmArgs& a, int dtype);
+cudaError_t launch_sgmm_ragged(const SgmmArgs& a, size_t scratch_off, cudaStream_t s);
+cudaError_t launch_tc_shrink_ragged(const SgmmArgs& a, size_t v_off, size_t tiles_off, int max_tiles, cudaStream_t s);
 cudaError_t launch_sgmm_dense(const SgmmArgs& a, size_t scratch_off, cudaStream_t s);
 cudaError_t launch_sgmm_bank(const SgmmArgs& a, size_t scratch_off, cudaStream_t s);
 bool sgmm_bank_supported(const SgmmArgs& a, int dtype);

@@ -472,6 +472,92 @@ def test_sgmm_tensor_rejects_unsupported(apr):
     assert ei.value.status == apr.APR_ERR_UNSUPPORTED
 
 
+# ------------------------------------------------------------------ SGMM, ragged many-tenant tiles (top-1)
+
+_RANKS_8_128 = tuple(range(8, 136, 8))
+
+
+def _ragged_case(rng, T, d_in, d_outs, E, rank_set, dist, ints=False):
+    ranks = tuple(int(r) for r in rng.choice(np.asarray(rank_set), size=E))
+    if dist == "zipf":
+        idx = _zipf_idx(rng, T, E, 1)
+    elif dist == "one":
+        idx = np.full((T, 1), E // 2, np.int32)
+    else:
+        idx = np.asarray(rng.integers(0, E, size=(T, 1)), np.int32)
+    return ranks, _case(rng, T, d_in, d_outs, ranks, 1, dist=idx, ints=ints)
+
+
+@pytest.mark.parametrize("T,d_in,d_outs,E,rank_set,dist", [
+    (1500, 512, (256, 200), 64, _RANKS_8_128, "uniform"),     # every rank 8..128; a 72-column last block
+    (700, 256, (128,), 300, (8, 16), "uniform"),               # 1-6 tokens per adapter: tiles close on 16 adapters
+    (900, 256, (136, 64), 40, (64, 96, 128), "zipf"),          # tiles close on 256 rank rows; long segments split
+    (1000, 512, (256,), 3, (128,), "one"),                     # one adapter of rank 128 takes every token
+    (4096, 1024, (1024, 1024), 256, (8, 16, 32, 64), "uniform"),   # the many-tenant routing, narrower projections
+    (130, 64, (16,), 2, (8, 24), "uniform"),                   # d_out of one 16-column block
+])
+def test_sgmm_ragged_parity(apr, T, d_in, d_outs, E, rank_set, dist):
+    """Top-1 calls on the tensor-core path go through ragged tiles (<= 128 tokens of <= 16
+    adapters, rank slots adding up to <= 256): every rank up to 128, tiles that close on the
+    token, adapter and rank-row limits, and an adapter split over many tiles."""
+    rng = np.random.default_rng(T + d_in + E + 7)
+    ranks, (x, As, Bs, idx, gate, ybs) = _ragged_case(rng, T, d_in, d_outs, E, rank_set, dist)
+    x, As, Bs, ybs = _rounded(x, As, Bs, ybs)
+    for zero in (True, False):
+        yb = [np.zeros_like(y) for y in ybs] if zero else ybs
+        got = run_sgmm(apr, x, As, Bs, idx, gate, yb, BF16, kernel=apr.SGMM_TENSOR)
+        ref = oracle_group(x, As, Bs, idx, gate.astype(np.float64), yb)
+        for p in range(len(d_outs)):
+            close(got[p], ref[p], f"ragged proj {p} zero_ybase={zero}")
+
+
+def test_sgmm_ragged_integer_inputs_exact(apr):
+    """Small integers (|v| <= 128, exact in bf16) and ranks 8..128: the result is the exact value
+    rounded once to bf16 (pins each adapter's slot offset and width in V and Bcat)."""
+    rng = np.random.default_rng(31)
+    ranks, (x, As, Bs, idx, gate, ybs) = _ragged_case(rng, 800, 128, (264, 128), 48, _RANKS_8_128, "uniform",
+                                                      ints=True)
+    got = run_sgmm(apr, x, As, Bs, idx, gate, ybs, BF16, kernel=apr.SGMM_TENSOR)
+    ref = oracle_group(x, As, Bs, idx, gate.astype(np.float64), ybs)
+    for p in range(2):
+        want = bf16_exact(ref[p]).astype(np.float64)
+        assert np.array_equal(got[p], want), f"proj {p}: max diff {np.abs(got[p] - want).max()}"
+
+
+def test_sgmm_ragged_properties(apr):
+    """Zero B leaves y_base bit-exact; in place equals out of place; two runs agree bit for bit;
+    a token permutation permutes the output bits."""
+    rng = np.random.default_rng(32)
+    ranks, (x, As, Bs, idx, gate, ybs) = _ragged_case(rng, 1200, 256, (520, 136), 96, (8, 16, 32, 64, 128),
+                                                      "uniform")
+    x, As, Bs, ybs = _rounded(x, As, Bs, ybs)
+    Bz = [[np.zeros_like(b) for b in P] for P in Bs]
+    z = run_sgmm(apr, x, As, Bz, idx, gate, ybs, BF16, kernel=apr.SGMM_TENSOR)
+    for p in range(2):
+        assert np.array_equal(z[p], ybs[p].astype(np.float64))
+    a = run_sgmm(apr, x, As, Bs, idx, gate, ybs, BF16, kernel=apr.SGMM_TENSOR, in_place=True)
+    b = run_sgmm(apr, x, As, Bs, idx, gate, ybs, BF16, kernel=apr.SGMM_TENSOR)
+    c = run_sgmm(apr, x, As, Bs, idx, gate, ybs, BF16, kernel=apr.SGMM_TENSOR)
+    for p in range(2):
+        assert np.array_equal(a[p], b[p]) and np.array_equal(b[p], c[p])
+    perm = rng.permutation(1200)
+    d = run_sgmm(apr, x[perm], As, Bs, idx[perm], gate[perm], [y[perm] for y in ybs], BF16, kernel=apr.SGMM_TENSOR)
+    for p in range(2):
+        assert np.array_equal(d[p], b[p][perm])
+
+
+def test_sgmm_ragged_rank_fault_is_reported(apr):
+    """A rank above the declared maximum on the ragged path: error word, no trap, context usable."""
+    rng = np.random.default_rng(33)
+    ranks, (x, As, Bs, idx, gate, ybs) = _ragged_case(rng, 600, 128, (128,), 20, (16, 32, 64), "uniform")
+    x, As, Bs, ybs = _rounded(x, As, Bs, ybs)
+    with pytest.raises(apr.AprError) as ei:
+        run_sgmm(apr, x, As, Bs, idx, gate, ybs, BF16, kernel=apr.SGMM_TENSOR, max_rank=32)
+    assert ei.value.status == apr.APR_ERR_DEVICE_INDEX
+    ok = run_sgmm(apr, x, As, Bs, idx, gate, ybs, BF16, kernel=apr.SGMM_TENSOR)
+    close(ok[0], oracle_group(x, As, Bs, idx, gate.astype(np.float64), ybs)[0], "ragged after fault")
+
+
 # ------------------------------------------------------------------ SGMM, dense small-batch kernel
 
 

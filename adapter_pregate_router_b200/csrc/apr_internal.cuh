@@ -140,6 +140,7 @@ struct RgTile {
   short u[kRgSlots];          // the adapters, ascending
   short koff[kRgSlots];       // first rank row of each adapter's slot (multiples of 16)
 };
+static_assert(sizeof(RgTile) == 80, "ragged tile record");
 // A tile closes when it is full (<= ceil(T / 128) times) or when the next adapter does not fit
 // (such a tile holds an adapter that starts in it: <= min(E, T) times), plus the last one.
 __host__ __device__ inline int rg_max_tiles(int T, int E) {
@@ -149,9 +150,19 @@ inline bool rg_dims_ok(int k, int max_rank) { return k == 1 && round16i(max_rank
 inline size_t rg_vc_bytes(int T, int max_rank) {
   return align_up((size_t)APR_MAX_PROJ * T * round16i(max_rank) * 2);
 }
+// After the tiles: each shrink CTA's ring of A tensor maps ([CTA][stage][projection]), then one
+// B tensor map per (projection, adapter) for the expand.
+constexpr int kRgMaxCtas = 256;
+constexpr int kRgMaxStages = 8;
+inline size_t rg_amaps_off(int T, int E, int max_rank) {
+  return align_up(rg_vc_bytes(T, max_rank) + 16 + 80 * (size_t)rg_max_tiles(T, E));
+}
+inline size_t rg_bmaps_off(int T, int E, int max_rank) {
+  return rg_amaps_off(T, E, max_rank) + (size_t)kRgMaxCtas * kRgMaxStages * APR_MAX_PROJ * 128;
+}
 inline size_t rg_scratch_bytes(int T, int k, int E, int max_rank) {
   if (!rg_dims_ok(k, max_rank)) return 0;
-  return rg_vc_bytes(T, max_rank) + 16 + sizeof(RgTile) * (size_t)rg_max_tiles(T, E);
+  return rg_bmaps_off(T, E, max_rank) + (size_t)APR_MAX_PROJ * E * 128;
 }
 
 // Shrink partial sums.  Gather paths: [projection][column chunk][sorted pair][rank]
@@ -360,7 +371,7 @@ cudaError_t launch_sgmm_skinny(const SgmmArgs& a, int dtype, size_t scratch_off,
 cudaError_t launch_sgmm_tensor(const SgmmArgs& a, size_t scratch_off, cudaStream_t s);
 bool sgmm_ragged_supported(const SgmmArgs& a, int dtype);
 cudaError_t launch_sgmm_ragged(const SgmmArgs& a, size_t scratch_off, cudaStream_t s);
-cudaError_t launch_tc_shrink_ragged(const SgmmArgs& a, size_t v_off, size_t tiles_off, int max_tiles, cudaStream_t s);
+
 cudaError_t launch_sgmm_dense(const SgmmArgs& a, size_t scratch_off, cudaStream_t s);
 cudaError_t launch_sgmm_bank(const SgmmArgs& a, size_t scratch_off, cudaStream_t s);
 bool sgmm_bank_supported(const SgmmArgs& a, int dtype);

@@ -32,8 +32,14 @@
 // Units are ordered (tile, projection, column block) and every CTA takes a
 // contiguous range of them: the work is balanced to one unit and V is rebuilt
 // only when a CTA's range moves to the next (tile, projection).  Every mbarrier
-// wait is bounded (1 s): on expiry the CTA records APR_ERR_TIMEOUT, drains its
-// copies and frees its tensor memory.
+// wait is bounded (1 s) and its outcome is made the same for all lanes of a warp
+// (no warp can be left at a barrier its other lanes abandoned); on expiry the CTA
+// records APR_ERR_TIMEOUT, drains its copies and frees its tensor memory.
+#include <map>
+#include <memory>
+#include <mutex>
+#include <tuple>
+
 #include "apr_internal.cuh"
 #include "tc_ptx.cuh"
 
@@ -44,8 +50,7 @@ constexpr int RG_NT = 128;                    // output columns per unit
 constexpr int RG_NS = 2;                      // stages of (y tile, Bcat)
 constexpr int RG_EPI = 256;                   // warps 0-7: epilogue (lane quarter x column half)
 constexpr int RG_VW = 128;                    // warps 8-11: V rows into TMEM
-constexpr int RG_PW = 128;                    // warps 12-15: Bcat; warp 12 also gathers y_base rows
-constexpr int RG_BLOCK = RG_EPI + RG_VW + RG_PW + 32;   // warp 16: MMA issue
+constexpr int RG_BLOCK = RG_EPI + RG_VW + 64;  // warp 12: TMA producer, warp 13: MMA issue
 constexpr uint32_t RG_TMEM_COLS = 512;        // [V0 | V1 | D0 | D1], 128 columns each
 constexpr int RG_YTILE = RG_M * RG_NT * 2;    // 32 KB: two 64-column halves of 128 rows x 128 B
 constexpr int RG_BCAT = kRgKmax * RG_NT * 2;  // 64 KB
@@ -57,7 +62,8 @@ struct RgPlan {
   SgmmArgs a;
   int R16;                            // rank slot of the staged v rows
   int max_tiles;
-  size_t vc_off, tiles_off;           // scratch: gated v [proj][position][R16] bf16; tile count, tiles
+  size_t vc_off, tiles_off, bmaps_off;   // scratch: gated v [proj][position][R16] bf16; tile count and
+                                         // tiles; B tensor maps [proj][adapter]
   int cb_before[APR_MAX_PROJ + 1];    // prefix of 128-column blocks per projection
 };
 
@@ -67,12 +73,365 @@ struct RgSmem {
   static constexpr size_t VC = BCAT + (size_t)RG_NS * RG_BCAT;    // the tile's gated v rows
   static constexpr size_t ZERO = VC + (size_t)RG_M * RG_VROW;     // 128 zero bytes
   static constexpr size_t BAR = ZERO + 128;
-  static constexpr int NBAR = 2 * RG_NS + 9;
+  static constexpr int NBAR = 2 * RG_NS + 10;
   static constexpr size_t META = BAR + NBAR * 8;
   static constexpr size_t total() { return META + 16 + 1024; }
 };
 static_assert(RgSmem::BCAT % 1024 == 0 && RG_YTILE % 1024 == 0, "swizzled rows need 1024-byte alignment");
 static_assert(RgSmem::total() <= 232448, "shared memory per block");
+
+// ---------------------------------------------------------------- checks shared by both kernels
+
+__device__ __forceinline__ bool rg_rank_ok(int r, int R16) { return r >= 8 && r <= R16 && (r & 7) == 0; }
+__device__ __forceinline__ bool rg_ptr_ok(const void* q) { return q && (reinterpret_cast<uintptr_t>(q) & 15) == 0; }
+// Adapter e of projection p has a B tensor map (built by the shrink, used by the expand).
+__device__ __forceinline__ bool rg_b_ok(const SgmmArgs& a, int p, int e, int R16) {
+  return e >= 0 && e < a.E && rg_rank_ok(a.ranks[e], R16) && rg_ptr_ok(a.proj[p].B[e]);
+}
+
+// ---------------------------------------------------------------- ragged tiles
+
+// The ragged tiles of a top-1 plan, built by one warp whose lanes all hold the same walk state
+// (lane s < kRgSlots also holds slot s of the open tile).  Adapters are taken in order; a tile
+// closes before an adapter (or the rest of one) that would make it hold more than kSetTile
+// tokens, more than kRgSlots adapters or more than kRgKmax rank rows.  The count is written even
+// past `max_tiles` (the expand checks it).
+__device__ void rg_plan(const SgmmArgs& a, int R16, int* count, RgTile* tiles, int max_tiles) {
+  const int lane = threadIdx.x & 31;
+  int t_start = 0, t_len = 0, t_nu = 0, t_kt = 0, nt = 0;
+  int my_u = 0, my_koff = 0;
+  auto close = [&]() {
+    if (t_len > 0) {
+      if (nt < max_tiles) {
+        RgTile* tl = tiles + nt;
+        if (lane < kRgSlots) {
+          tl->u[lane] = (short)(lane < t_nu ? my_u : -1);
+          tl->koff[lane] = (short)(lane < t_nu ? my_koff : t_kt);
+        }
+        if (lane == 0) {
+          tl->start = t_start;
+          tl->len = t_len;
+          tl->nu = t_nu;
+          tl->kt = t_kt;
+        }
+      }
+      ++nt;
+    }
+    t_len = t_nu = t_kt = 0;
+  };
+  for (int e0 = 0; e0 < a.E; e0 += 32) {
+    const int e = e0 + lane;
+    int beg = 0, cnt = 0, w = 16;
+    if (e < a.E) {
+      beg = a.seg_off[e];
+      cnt = a.seg_off[e + 1] - beg;
+      const int r = a.ranks[e];
+      if (rg_rank_ok(r, R16)) w = (r + 15) / 16 * 16;   // an invalid rank (reported) keeps 16 zero rows
+    }
+    unsigned m = __ballot_sync(0xffffffffu, cnt > 0);
+    while (m) {
+      const int j = __ffs(m) - 1;
+      m &= m - 1;
+      int c = __shfl_sync(0xffffffffu, cnt, j), pos = __shfl_sync(0xffffffffu, beg, j);
+      const int wj = __shfl_sync(0xffffffffu, w, j);
+      while (c > 0) {
+        if (t_nu == kRgSlots || t_kt + wj > kRgKmax || t_len == kSetTile) close();
+        if (t_len == 0) t_start = pos;
+        const int take = min(c, kSetTile - t_len);
+        if (lane == t_nu) {
+          my_u = e0 + j;
+          my_koff = t_kt;
+        }
+        ++t_nu;
+        t_kt += wj;
+        t_len += take;
+        c -= take;
+        pos += take;
+      }
+    }
+  }
+  close();
+  if (lane == 0) *count = nt;
+}
+
+// ---------------------------------------------------------------- shrink
+
+// v = g * A_e x for every pair, by plan position: [proj][position][R16] bf16 (rank rows past
+// r_e are zeros).  An item is one pair tile of adapter e (<= 128 consecutive plan positions) and
+// a group of <= 4 projections whose R16-row slots add up to <= 256.  The contraction puts the
+// adapter rows on the MMA's M side and the tokens on N:
+//   D[j, n] = sum_k A_{q(j), e}[j mod R16, k] x_{t_n}[k]   (M = 128 per accumulator, N = round16(len))
+// so a short segment costs only its own tokens.  One producer warp issues, per 64-column stage,
+// TMA boxes of A_e (64 columns x R16 rows from a tensor map made for the item: the projection's
+// template for rank r_e with A_e's address, zeros past r_e) and tile::gather4 copies of the
+// tokens' x rows; one thread issues the MMAs; eight epilogue warps read D back (a TMEM lane per
+// adapter row), scale by each token's gate and store bf16.  Items come from a work counter (after
+// one static item per CTA), so CTAs drawing high-rank adapters take fewer of them.
+constexpr int RS_EPI = 256;                   // warps 2-9
+constexpr int RS_BLOCK = 64 + RS_EPI;         // warp 0: producer, warp 1: MMA issue
+constexpr int RS_XBYTES = 128 * 128;          // x rows of a stage (128 x 64 columns, 128-byte swizzle)
+constexpr int RS_NQ = 4;                      // projections per item at most
+
+struct RsPlan {
+  CUtensorMap xmap;                               // x rows: 64-column boxes (gather4)
+  CUtensorMap atmpl[APR_MAX_PROJ][APR_MAX_RANK / 8];   // A_e of rank 8 (j + 1): [r, d_in], 64 x R16 boxes, swizzled
+  CUtensorMap btmpl[APR_MAX_PROJ][APR_MAX_RANK / 8];   // B_e of rank 8 (j + 1): [d_out, r], 8 x 128 boxes, plain
+  SgmmArgs a;
+  int R16, pg, npg, stages, max_tiles;
+  size_t vc_off, tiles_off, amaps_off, bmaps_off;
+};
+
+struct RsItem {
+  int e, q0, nq, start, len, pad[3];
+};
+
+struct RsSmem {
+  int stage_bytes, S;
+  size_t bar, item, gate, mapbuf, tmem, total;
+};
+__host__ __device__ inline RsSmem rs_smem(int pg, int R16, int S) {
+  RsSmem L;
+  // the adapter rows of a stage: at least the 128 rows one accumulator's MMAs read
+  L.stage_bytes = RS_XBYTES + (pg * R16 < 128 ? 128 : pg * R16) * 128;
+  L.S = S;
+  L.bar = (size_t)S * L.stage_bytes;
+  L.item = L.bar + (size_t)(2 * S + 6) * 8;
+  L.gate = L.item + 2 * sizeof(RsItem);
+  L.mapbuf = (L.gate + 2 * 128 * 4 + 127) / 128 * 128;
+  L.tmem = L.mapbuf + (RS_NQ + 1) * 128;
+  L.total = L.tmem + 16 + 1024;
+  return L;
+}
+
+__global__ void __launch_bounds__(RS_BLOCK, 1) rg_shrink_kernel(const __grid_constant__ RsPlan P) {
+  const SgmmArgs& a = P.a;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem =
+      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int S = P.stages, R16 = P.R16, pg = P.pg, T = a.T;
+  const RsSmem L = rs_smem(pg, R16, S);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bar);
+  const uint32_t bar_full = smem_u32(bars), bar_empty = smem_u32(bars + S);
+  const uint32_t bar_ifull = smem_u32(bars + 2 * S), bar_iempty = smem_u32(bars + 2 * S + 2);
+  const uint32_t bar_dfull = smem_u32(bars + 2 * S + 4), bar_dempty = smem_u32(bars + 2 * S + 5);
+  RsItem* s_item = reinterpret_cast<RsItem*>(smem + L.item);
+  float* s_g = reinterpret_cast<float*>(smem + L.gate);
+  const uint32_t sbase = smem_u32(smem), s_mapbuf = sbase + (uint32_t)L.mapbuf;
+  volatile uint32_t* s_tmem = reinterpret_cast<volatile uint32_t*>(smem + L.tmem);
+
+  if (tid == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(bar_full + 8 * i, 1);
+      mbar_init(bar_empty + 8 * i, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar_ifull + 8 * i, 1);
+      mbar_init(bar_iempty + 8 * i, 1 + RS_EPI / 32);
+    }
+    mbar_init(bar_dfull, 1);
+    mbar_init(bar_dempty, RS_EPI);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) tmem_alloc(smem_u32(const_cast<uint32_t*>(s_tmem)), 256);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+
+  pdl_wait();
+  pdl_trigger();
+
+  const WsLayout W = ws_layout(a.T, a.k, a.E);
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(a.ws);
+  const PairTile* qtiles = ws_at<PairTile>(a.ws, W.qtiles);
+  const long nitems = (long)hdr->n_qtiles * P.npg;
+  const int nk = a.d_in / 64;
+  bool abort = false;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer warp
+    // the expand's B tensor maps of this CTA's share of the (projection, adapter) pairs in use
+    CUtensorMap* bmaps = ws_at<CUtensorMap>(a.ws, P.bmaps_off);
+    for (int pe = blockIdx.x; pe < a.nproj * a.E; pe += gridDim.x) {
+      const int p = pe / a.E, e = pe - p * a.E;
+      if (a.seg_off[e + 1] > a.seg_off[e] && rg_b_ok(a, p, e, R16))
+        tmap_build(bmaps + pe, s_mapbuf + RS_NQ * 128, &P.btmpl[p][a.ranks[e] / 8 - 1], a.proj[p].B[e]);
+    }
+    CUtensorMap* amaps = ws_at<CUtensorMap>(a.ws, P.amaps_off) + (size_t)blockIdx.x * kRgMaxStages * RS_NQ;
+    const __nv_bfloat16* x = reinterpret_cast<const __nv_bfloat16*>(a.x);
+    (void)x;
+    uint32_t g = 0, k = 0;
+    long item = blockIdx.x;
+    while (!abort) {
+      const int slot = k & 1;
+      if (k >= 2 && !__all_sync(0xffffffffu, mbar_wait(bar_iempty + 8 * slot, ((k >> 1) - 1) & 1))) {
+        abort = true;
+        break;
+      }
+      if (item >= nitems) {                            // no more work: a sentinel item
+        if (lane == 0) {
+          s_item[slot].e = -1;
+          mbar_arrive(bar_ifull + 8 * slot);
+        }
+        break;
+      }
+      const PairTile tile = qtiles[item / P.npg];
+      const int q0 = (int)(item % P.npg) * pg, nq = min(pg, a.nproj - q0), e = tile.e;
+      const int r = (e >= 0 && e < a.E) ? a.ranks[e] : 0;
+      bool ok = rg_rank_ok(r, R16) && tile.len > 0 && tile.len <= kSetTile;
+      for (int qi = 0; qi < nq && ok; ++qi) ok = rg_ptr_ok(a.proj[q0 + qi].A[e]);
+      long next = 0;
+      if (lane == 0) next = (long)gridDim.x + (long)atomicAdd(&hdr->sched, 1u);
+      next = __shfl_sync(0xffffffffu, next, 0);
+      if (!ok) {
+        if (lane == 0 && tile.len > 0) report(a.ws, APR_ERR_DEVICE_INDEX, K_TC, e);
+        item = next;
+        continue;
+      }
+      const int len = tile.len;
+      // the item's tokens (rows 4 * lane .. + 3; rows past the tile repeat its first token) and gates
+      int tk[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int row = 4 * lane + j;
+        const int q = a.perm[tile.start + (row < len ? row : 0)];
+        tk[j] = q;                                     // top-1: the pair id is the token
+        s_g[slot * 128 + row] = row < len ? a.gate[q] : 0.f;
+      }
+      if (lane == 0) {
+        RsItem it;
+        it.e = e;
+        it.q0 = q0;
+        it.nq = nq;
+        it.start = tile.start;
+        it.len = len;
+        s_item[slot] = it;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_ifull + 8 * slot);
+      // the item's first stage is free before its A maps are rewritten: the ring slot k % S was last
+      // used by item k - S, whose copies all precede that stage's previous use
+      {
+        const uint32_t s0 = g % S;
+        if (g >= (uint32_t)S && !__all_sync(0xffffffffu, mbar_wait(bar_empty + 8 * s0, ((g / S) - 1) & 1))) {
+          abort = true;
+          break;
+        }
+      }
+      CUtensorMap* am = amaps + (size_t)(k % S) * RS_NQ;
+      for (int qi = 0; qi < nq; ++qi) {
+        tmap_build(am + qi, s_mapbuf + qi * 128, &P.atmpl[q0 + qi][r / 8 - 1], a.proj[q0 + qi].A[e]);
+        if (lane == 0) tmap_acquire(am + qi);
+      }
+      const int ngr = (len + 3) >> 2;
+      const uint32_t bytes = (uint32_t)(ngr * 512 + nq * R16 * 128);
+      for (int c = 0; c < nk; ++c, ++g) {
+        const uint32_t s = g % S;
+        if (c > 0 && g >= (uint32_t)S && !__all_sync(0xffffffffu, mbar_wait(bar_empty + 8 * s, ((g / S) - 1) & 1))) {
+          abort = true;
+          break;
+        }
+        const uint32_t xs = sbase + s * (uint32_t)L.stage_bytes, as = xs + RS_XBYTES;
+        if (lane == 0) mbar_arrive_expect_tx(bar_full + 8 * s, bytes);
+        __syncwarp();
+        if (lane < ngr) tma_gather4(xs + (uint32_t)(4 * lane) * 128, &P.xmap, 64 * c, tk[0], tk[1], tk[2], tk[3], bar_full + 8 * s);
+        if (lane == 0)
+          for (int qi = 0; qi < nq; ++qi) tma_load_2d(as + (uint32_t)(qi * R16) * 128, am + qi, 64 * c, 0, bar_full + 8 * s);
+      }
+      ++k;
+      item = next;
+    }
+    // after an abort, the copies of the last stages land before the CTA exits (bounded)
+    if (abort && lane == 0)
+      for (uint32_t j = g > (uint32_t)S ? g - S : 0; j < g; ++j) (void)mbar_wait(bar_full + 8 * (j % S), (j / S) & 1);
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issue
+    if (lane == 0) {
+      uint32_t g = 0, k = 0;
+      while (true) {
+        const int slot = k & 1;
+        if (!mbar_wait(bar_ifull + 8 * slot, (k >> 1) & 1)) { abort = true; break; }
+        const RsItem it = s_item[slot];
+        mbar_arrive(bar_iempty + 8 * slot);
+        if (it.e < 0) break;
+        const int N = (it.len + 15) / 16 * 16, nacc = (it.nq * R16 + 127) / 128;
+        const uint32_t id = idesc_bf16(128, N);
+        if (k >= 1 && !mbar_wait(bar_dempty, (k - 1) & 1)) { abort = true; break; }
+        tc_fence_after();
+        for (int c = 0; c < nk; ++c, ++g) {
+          const uint32_t s = g % S;
+          if (!mbar_wait(bar_full + 8 * s, (g / S) & 1)) { abort = true; break; }
+          tc_fence_after();
+          const uint32_t xs = sbase + s * (uint32_t)L.stage_bytes, as = xs + RS_XBYTES;
+          for (int m = 0; m < nacc; ++m)
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16(tmem + (uint32_t)m * 128, desc_k_sw128(as + (uint32_t)m * RS_XBYTES + kk * 32),
+                       desc_k_sw128(xs + kk * 32), id, (c > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(bar_empty + 8 * s);
+        }
+        if (abort) break;
+        mma_commit(bar_dfull);
+        ++k;
+      }
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int ew = warp - 2, quarter = warp & 3;
+    if (ew == 0 && blockIdx.x == gridDim.x - 1) {
+      int* cnt = ws_at<int>(a.ws, P.tiles_off);
+      rg_plan(a, R16, cnt, reinterpret_cast<RgTile*>(cnt + 4), P.max_tiles);
+    }
+    __nv_bfloat16* vc = ws_at<__nv_bfloat16>(a.ws, P.vc_off);
+    uint32_t k = 0;
+    while (true) {
+      const int slot = k & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_ifull + 8 * slot, (k >> 1) & 1))) { abort = true; break; }
+      const RsItem it = s_item[slot];
+      if (it.e < 0) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_iempty + 8 * slot);
+        break;
+      }
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_dfull, k & 1))) { abort = true; break; }
+      tc_fence_after();
+      const int N = (it.len + 15) / 16 * 16, nacc = (it.nq * R16 + 127) / 128;
+      // two accumulators: warps 2-5 read the first, 6-9 the second; one: they split the columns
+      const int m = nacc == 2 ? (ew >> 2) : 0, csel = nacc == 2 ? -1 : (ew >> 2);
+      const int j = 128 * m + 32 * quarter + lane;       // adapter row of this TMEM lane
+      const int qi = j / R16, rr = j - qi * R16;
+      const bool valid = qi < it.nq;
+      __nv_bfloat16* dst = vc + ((size_t)(it.q0 + qi) * T + it.start) * R16 + rr;
+      const float* gg = s_g + slot * 128;
+      for (int c16 = 0; c16 < N / 16; ++c16) {
+        if (csel >= 0 && (c16 & 1) != csel) continue;
+        float v[16];
+        tmem_ld16(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)m * 128 + (uint32_t)c16 * 16, v);
+        if (valid) {
+#pragma unroll
+          for (int t = 0; t < 16; ++t) {
+            const int n = c16 * 16 + t;
+            if (n < it.len) dst[(size_t)n * R16] = __float2bfloat16_rn(v[t] * gg[n]);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar_dempty);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_iempty + 8 * slot);
+      ++k;
+    }
+  }
+  abort = __syncthreads_or(abort);
+  if (abort && tid == 0) report(a.ws, APR_ERR_TIMEOUT, K_TC, (int)blockIdx.x);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, 256);
+}
+
+// ---------------------------------------------------------------- expand
 
 __global__ void __launch_bounds__(RG_BLOCK, 1) ragged_expand_kernel(const __grid_constant__ RgPlan P) {
   const SgmmArgs& a = P.a;
@@ -88,13 +447,14 @@ __global__ void __launch_bounds__(RG_BLOCK, 1) ragged_expand_kernel(const __grid
   const uint32_t bar_dfull = smem_u32(bars + 2 * RG_NS + 4);   // [2]  accumulator ready
   const uint32_t bar_dempty = smem_u32(bars + 2 * RG_NS + 6);  // [2]  accumulator read
   const uint32_t bar_vc = smem_u32(bars + 2 * RG_NS + 8);      // staged v rows landed
+  const uint32_t bar_vcfree = smem_u32(bars + 2 * RG_NS + 9);  // staged v rows read by every V thread
   volatile uint32_t* s_tmem = reinterpret_cast<volatile uint32_t*>(smem + RgSmem::META);
   const uint32_t sbase = smem_u32(smem);
   const uint32_t sY = sbase + (uint32_t)RgSmem::Y, sB = sbase + (uint32_t)RgSmem::BCAT;
 
   if (tid == 0) {
     for (int i = 0; i < RG_NS; ++i) {
-      mbar_init(bar_full + 8 * i, RG_PW + 1);
+      mbar_init(bar_full + 8 * i, 1);
       mbar_init(bar_empty + 8 * i, RG_EPI / 32 + 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -104,6 +464,7 @@ __global__ void __launch_bounds__(RG_BLOCK, 1) ragged_expand_kernel(const __grid
       mbar_init(bar_dempty + 8 * i, RG_EPI);
     }
     mbar_init(bar_vc, 1);
+    mbar_init(bar_vcfree, RG_VW);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 0) tmem_alloc(smem_u32(const_cast<uint32_t*>(s_tmem)), RG_TMEM_COLS);
@@ -160,8 +521,9 @@ __global__ void __launch_bounds__(RG_BLOCK, 1) ragged_expand_kernel(const __grid
         tok = row < len ? a.perm[tiles[ti].start + row] : -1;
       }
       const int s = i % RG_NS, db = i & 1;
-      if (!mbar_wait(bar_dfull + 8 * db, (i >> 1) & 1)) { abort = true; break; }
-      if (!mbar_wait(bar_full + 8 * s, (i / RG_NS) & 1)) { abort = true; break; }
+      bool ok = mbar_wait(bar_dfull + 8 * db, (i >> 1) & 1);
+      ok = __all_sync(0xffffffffu, ok && mbar_wait(bar_full + 8 * s, (i / RG_NS) & 1));
+      if (!ok) { abort = true; break; }
       tc_fence_after();
       const int d_out = a.proj[p].d_out;
       const int nvalid = min(max(len - quarter * 32, 0), 32);        // the warp's rows that hold tokens
@@ -233,9 +595,11 @@ __global__ void __launch_bounds__(RG_BLOCK, 1) ragged_expand_kernel(const __grid
     const __nv_bfloat16* vc = ws_at<__nv_bfloat16>(a.ws, P.vc_off);
     const uint32_t row_bytes = (uint32_t)R16 * 2;
     if (vt < 8) st_shared_zero16(sZero + (uint32_t)vt * 16);
-    asm volatile("bar.sync 1, %0;" ::"n"(RG_VW) : "memory");
-    // the gated v rows of unit i's tile and projection (contiguous in plan order)
-    auto issue_rows = [&](int i) {
+    asm volatile("bar.sync 1, %0;" ::"n"(RG_VW) : "memory");   // the zero line is written (no wait before)
+    // the gated v rows of unit i's tile and projection (contiguous in plan order); copy j reuses
+    // the staging buffer once every V thread has read copy j - 1
+    auto issue_rows = [&](int i, int j) -> bool {
+      if (j > 0 && !mbar_wait(bar_vcfree, (j - 1) & 1)) return false;
       int ti, p, c0;
       unit_at(i, ti, p, c0);
       const RgTile& tl = tiles[ti];
@@ -243,6 +607,7 @@ __global__ void __launch_bounds__(RG_BLOCK, 1) ragged_expand_kernel(const __grid
       fence_proxy_async();                             // earlier reads of the buffer come before the copy
       mbar_arrive_expect_tx(bar_vc, bytes);
       bulk_load_1d(sVC, vc + ((size_t)p * T + tl.start) * R16, bytes, bar_vc);
+      return true;
     };
     // the adapter of this thread's token in unit i's tile (-1: no token)
     auto fetch_adapter = [&](int i) -> int {
@@ -252,20 +617,20 @@ __global__ void __launch_bounds__(RG_BLOCK, 1) ragged_expand_kernel(const __grid
       return row < tl.len ? a.idx[a.perm[tl.start + row]] : -1;
     };
     int issued = 0, consumed = 0, item = 0, e_next = -1;
-    int i = 0;
     if (n > 0) {
-      if (vt == 0) issue_rows(0);
+      if (vt == 0) (void)issue_rows(0, 0);
       issued = 1;
       e_next = fetch_adapter(0);
     }
-    for (; i < n && !abort; ++i) {
+    for (int i = 0; i < n && !abort; ++i) {
       if (!new_v(i)) continue;
       int ti, p, c0;
       unit_at(i, ti, p, c0);
       const int vb = item & 1;
-      if (!mbar_wait(bar_vc, item & 1)) { abort = true; break; }
-      consumed = item + 1;
-      if (item >= 2 && !mbar_wait(bar_vempty + 8 * vb, ((item >> 1) - 1) & 1)) { abort = true; break; }
+      bool ok = mbar_wait(bar_vc, item & 1);
+      if (ok) consumed = item + 1;
+      if (item >= 2) ok = ok && mbar_wait(bar_vempty + 8 * vb, ((item >> 1) - 1) & 1);
+      if (!__all_sync(0xffffffffu, ok)) { abort = true; break; }
       tc_fence_after();
       const RgTile& tl = tiles[ti];
       const int kt = tl.kt, nu = tl.nu;
@@ -273,11 +638,11 @@ __global__ void __launch_bounds__(RG_BLOCK, 1) ragged_expand_kernel(const __grid
       // this token's slot (words of 32 bits: two bf16 rank rows)
       int ko = 0, wd = 0;
       if (e >= 0) {
-        int s = 0;
-        while (s < nu && tl.u[s] != e) ++s;
-        if (s < nu) {
-          ko = tl.koff[s] / 2;
-          wd = ((s + 1 < nu ? tl.koff[s + 1] : kt) - tl.koff[s]) / 2;
+        int q = 0;
+        while (q < nu && tl.u[q] != e) ++q;
+        if (q < nu) {
+          ko = tl.koff[q] / 2;
+          wd = ((q + 1 < nu ? tl.koff[q + 1] : kt) - tl.koff[q]) / 2;
         } else {
           report(a.ws, APR_ERR_DEVICE_INDEX, K_TC, e);
         }
@@ -309,93 +674,102 @@ __global__ void __launch_bounds__(RG_BLOCK, 1) ragged_expand_kernel(const __grid
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar_vfull + 8 * vb);
+      mbar_arrive(bar_vcfree);                          // this thread no longer reads the staged rows
       ++item;
-      asm volatile("bar.sync 1, %0;" ::"n"(RG_VW) : "memory");   // the staged rows are no longer read
       int nx = i + 1;
       while (nx < n && !new_v(nx)) ++nx;
       if (nx < n) {
-        if (vt == 0) issue_rows(nx);
+        bool sent = true;
+        if (vt == 0) sent = issue_rows(nx, item);
+        if (!__all_sync(0xffffffffu, sent)) { abort = true; break; }   // warp 8; the others time out on the copy
         ++issued;
         e_next = fetch_adapter(nx);
       }
     }
     // a row copy still in flight after an abort lands before the CTA exits (bounded wait)
     for (int u = consumed; u < issued; ++u) (void)mbar_wait(bar_vc, u & 1);
-  } else if (tid < RG_EPI + RG_VW + RG_PW) {
-    // ---------------------------------------------------------------- producers: y_base rows, Bcat
-    const int pt = tid - RG_EPI - RG_VW;
-    const bool gatherer = pt < 32;                     // warp 12 issues the y_base gathers
-    int cur_ti = -1, len = 0, start = 0, tk[4] = {0, 0, 0, 0};
-    int last = -1;                                     // last unit whose stage this thread filled
+  } else if (tid < RG_EPI + RG_VW + 32) {
+    // ---------------------------------------------------------------- producer warp: y_base rows, Bcat
+    // lane q < nu owns slot q of the current (tile, projection): the tensor map of B_{u_q} (built by
+    // the shrink), its first 16-byte K chunk and chunks per row; an invalid slot is zeros
+    const CUtensorMap* bmaps = ws_at<const CUtensorMap>(a.ws, P.bmaps_off);
+    const CUtensorMap* my_map = nullptr;
+    int my_kc0 = 0, my_cps = 0, bbytes = 0;
+    int cur_ti = -1, cur_p = -1, len = 0, tk[4] = {0, 0, 0, 0};
+    int last = -1;                                     // last unit whose stage this warp filled
     for (int i = 0; i < n && !abort; ++i) {
       int ti, p, c0;
       unit_at(i, ti, p, c0);
       const int s = i % RG_NS;
-      if (i >= RG_NS && !mbar_wait(bar_empty + 8 * s, ((i / RG_NS) - 1) & 1)) { abort = true; break; }
+      if (i >= RG_NS && !__all_sync(0xffffffffu, mbar_wait(bar_empty + 8 * s, ((i / RG_NS) - 1) & 1))) {
+        abort = true;
+        break;
+      }
       const RgTile& tl = tiles[ti];
-      if (ti != cur_ti) {
-        cur_ti = ti;
+      const bool new_tile = ti != cur_ti, new_proj = new_tile || p != cur_p;
+      cur_ti = ti;
+      cur_p = p;
+      if (new_tile) {
         len = tl.len;
-        start = tl.start;
-        if (gatherer) {
-          // rows 4 * lane .. + 3; rows past the tile repeat its first token (loaded, never stored)
+        // rows 4 * lane .. + 3; rows past the tile repeat its first token (loaded, never stored)
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int r = 4 * lane + q;
-            tk[q] = a.perm[start + (r < len ? r : 0)];
+        for (int q = 0; q < 4; ++q) {
+          const int r = 4 * lane + q;
+          tk[q] = a.perm[tl.start + (r < len ? r : 0)];
+        }
+      }
+      if (new_proj) {
+        const int nu = tl.nu;
+        my_map = nullptr;
+        my_cps = 0;
+        if (lane < nu) {
+          const int e = tl.u[lane], ko = tl.koff[lane];
+          const int w = (lane + 1 < nu ? tl.koff[lane + 1] : tl.kt) - ko;
+          my_kc0 = ko / 8;
+          my_cps = w / 8;
+          if (rg_b_ok(a, p, e, R16)) {
+            my_map = bmaps + (size_t)p * a.E + e;
+            tmap_acquire(my_map);
           }
         }
+        bbytes = __reduce_add_sync(0xffffffffu, my_map ? my_cps * (RG_NT * 16) : 0);
       }
       const int d_out = a.proj[p].d_out;
       const uint32_t ys = sY + (uint32_t)s * RG_YTILE, bs = sB + (uint32_t)s * RG_BCAT;
-      if (gatherer) {
-        const int nh = c0 + 64 < d_out ? 2 : 1, ngr = (len + 3) >> 2;
-        if (lane == 0) mbar_arrive_expect_tx(bar_full + 8 * s, (uint32_t)(ngr * nh * 512));
-        __syncwarp();
-        if (lane < ngr)
-          for (int h = 0; h < nh; ++h)
-            tma_gather4(ys + (uint32_t)h * (RG_M * 128) + (uint32_t)(4 * lane) * 128, &P.yb_map[p], c0 + 64 * h, tk[0],
-                        tk[1], tk[2], tk[3], bar_full + 8 * s);
+      // an invalid slot: zero chunks by plain stores, ordered before the arrival below
+      if (!my_map && my_cps > 0) {
+        for (int c = 0; c < my_cps; ++c)
+          for (int r16 = 0; r16 < RG_NT; ++r16) st_shared_zero16(bs + (uint32_t)(my_kc0 + c) * (RG_NT * 16) + (uint32_t)r16 * 16);
+        fence_proxy_async();
       }
-      // Bcat: every slot's 128 rows x w_s/8 16-byte chunks (zeros past the rank or past d_out)
-      const int nu = tl.nu, kt = tl.kt;
-      bool zeros = false;
-      for (int q = 0; q < nu; ++q) {
-        const int e = tl.u[q], ko = tl.koff[q];
-        const int w = (q + 1 < nu ? tl.koff[q + 1] : kt) - ko;
-        const int r = (e >= 0 && e < a.E) ? a.ranks[e] : 0;
-        const bool rank_ok = r >= 8 && r <= w && (r & 7) == 0;
-        const __nv_bfloat16* B = rank_ok ? reinterpret_cast<const __nv_bfloat16*>(a.proj[p].B[e]) : nullptr;
-        const int cps = w / 8;
-        for (int w8 = pt; w8 < RG_NT * cps; w8 += RG_PW) {
-          const int nn = w8 / cps, c = w8 - nn * cps;
-          const uint32_t dst = bs + (uint32_t)(ko / 8 + c) * (RG_NT / 8 * 128) + (uint32_t)(nn >> 3) * 128 +
-                               (uint32_t)(nn & 7) * 16;
-          if (B && c * 8 < r && c0 + nn < d_out) {
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(B + (size_t)(c0 + nn) * r + c * 8)
-                         : "memory");
-          } else {
-            st_shared_zero16(dst);
-            zeros = true;
-          }
-        }
-      }
-      if (zeros) fence_proxy_async();
-      cp_async_arrive(bar_full + 8 * s);
+      __syncwarp();
+      const int nh = c0 + 64 < d_out ? 2 : 1, ngr = (len + 3) >> 2;
+      if (lane == 0) mbar_arrive_expect_tx(bar_full + 8 * s, (uint32_t)(ngr * nh * 512 + bbytes));
+      __syncwarp();
+      if (lane < ngr)
+        for (int h = 0; h < nh; ++h)
+          tma_gather4(ys + (uint32_t)h * (RG_M * 128) + (uint32_t)(4 * lane) * 128, &P.yb_map[p], c0 + 64 * h, tk[0],
+                      tk[1], tk[2], tk[3], bar_full + 8 * s);
+      // Bcat chunk kc = rank rows 8c..8c+7 of the slot for the unit's 128 columns: one box of 8
+      // columns x 128 rows of B, which lands as the chunk's 16 core matrices (zeros past the rank
+      // and past d_out)
+      if (my_map)
+        for (int c = 0; c < my_cps; ++c)
+          tma_load_2d(bs + (uint32_t)(my_kc0 + c) * (RG_NT * 16), my_map, 8 * c, c0, bar_full + 8 * s);
       last = i;
     }
-    cp_async_wait_all();
-    // after an abort, the gathers of the stages filled last land before the CTA exits (bounded)
-    if (abort && gatherer && lane == 0)
+    // after an abort, the copies of the stages filled last land before the CTA exits (bounded)
+    if (abort && lane == 0)
       for (int i = max(last - RG_NS + 1, 0); i <= last; ++i) (void)mbar_wait(bar_full + 8 * (i % RG_NS), (i / RG_NS) & 1);
   } else if (lane == 0) {
     // ---------------------------------------------------------------- MMA issue
     const uint32_t id = idesc_bf16(RG_M, RG_NT);
-    int item = -1;
+    int item = -1, kt = 0;
     for (int i = 0; i < n && !abort; ++i) {
       int ti, p, c0;
       unit_at(i, ti, p, c0);
       if (new_v(i)) {
+        kt = tiles[ti].kt;
         ++item;
         if (!mbar_wait(bar_vfull + 8 * (item & 1), (item >> 1) & 1)) { abort = true; break; }
       }
@@ -403,7 +777,6 @@ __global__ void __launch_bounds__(RG_BLOCK, 1) ragged_expand_kernel(const __grid
       if (!mbar_wait(bar_full + 8 * s, (i / RG_NS) & 1)) { abort = true; break; }
       if (i >= 2 && !mbar_wait(bar_dempty + 8 * db, ((i >> 1) - 1) & 1)) { abort = true; break; }
       tc_fence_after();
-      const int kt = tiles[ti].kt;
       const uint32_t dcol = tmem + 256u + (uint32_t)db * 128, vcol = tmem + (uint32_t)vb * 128;
       // K step kk: B core matrices at bs + kk * 4096 (two 2048-byte K chunks): +256 in the
       // descriptor's address field (bytes / 16) per step
@@ -430,30 +803,80 @@ bool sgmm_ragged_supported(const SgmmArgs& a, int dtype) {
   return dtype == APR_BF16 && rg_dims_ok(a.k, a.max_rank) && a.d_in % 64 == 0;
 }
 
+// Tensor-map templates depend only on shapes, so they are encoded once per shape (the address is
+// a placeholder the kernels replace).
+static cudaError_t cached_box_map(CUtensorMap* m, const void* placeholder, long rows, long cols, long pitch, int box_cols,
+                                  int box_rows, bool sw) {
+  using Key = std::tuple<long, long, long, int, int, int>;
+  static std::mutex mu;
+  static std::map<Key, CUtensorMap> cache;
+  const Key key{rows, cols, pitch, box_cols, box_rows, sw ? 1 : 0};
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = cache.find(key);
+  if (it != cache.end()) {
+    *m = it->second;
+    return cudaSuccess;
+  }
+  cudaError_t err = encode_box_map(m, placeholder, rows, cols, pitch, box_cols, box_rows, sw);
+  if (err == cudaSuccess) cache.emplace(key, *m);
+  return err;
+}
+
 cudaError_t launch_sgmm_ragged(const SgmmArgs& a, size_t scratch_off, cudaStream_t s) {
+  const int R16 = round16i(a.max_rank);
+  const int nsm = device_sm_count();
+  cudaError_t err;
+  // ---- shrink
+  std::unique_ptr<RsPlan> S(new RsPlan);
+  memset(S.get(), 0, sizeof(RsPlan));
+  S->a = a;
+  S->R16 = R16;
+  S->pg = 256 / R16 < a.nproj ? 256 / R16 : a.nproj;
+  if (S->pg > RS_NQ) S->pg = RS_NQ;
+  S->npg = (a.nproj + S->pg - 1) / S->pg;
+  S->stages = (int)((200 * 1024) / rs_smem(S->pg, R16, 1).stage_bytes);
+  if (S->stages > kRgMaxStages) S->stages = kRgMaxStages;
+  S->max_tiles = rg_max_tiles(a.T, a.E);
+  S->vc_off = scratch_off;
+  S->tiles_off = scratch_off + rg_vc_bytes(a.T, a.max_rank);
+  S->amaps_off = scratch_off + rg_amaps_off(a.T, a.E, a.max_rank);
+  S->bmaps_off = scratch_off + rg_bmaps_off(a.T, a.E, a.max_rank);
+  if ((err = encode_row_map(&S->xmap, const_cast<void*>(a.x), a.T, a.d_in)) != cudaSuccess) return err;
+  for (int p = 0; p < a.nproj; ++p)
+    for (int r = 8; r <= R16; r += 8) {
+      if ((err = cached_box_map(&S->atmpl[p][r / 8 - 1], a.x, r, a.d_in, (long)a.d_in * 2, 64, R16, true)) != cudaSuccess)
+        return err;
+      if ((err = cached_box_map(&S->btmpl[p][r / 8 - 1], a.x, a.proj[p].d_out, r, (long)r * 2, 8, RG_NT, false)) !=
+          cudaSuccess)
+        return err;
+    }
+  // ---- expand
   RgPlan P;
   memset(&P, 0, sizeof(P));
   P.a = a;
-  P.R16 = round16i(a.max_rank);
-  P.max_tiles = rg_max_tiles(a.T, a.E);
-  P.vc_off = scratch_off;
-  P.tiles_off = scratch_off + rg_vc_bytes(a.T, a.max_rank);
+  P.R16 = R16;
+  P.max_tiles = S->max_tiles;
+  P.vc_off = S->vc_off;
+  P.tiles_off = S->tiles_off;
+  P.bmaps_off = S->bmaps_off;
   P.cb_before[0] = 0;
-  cudaError_t err;
   for (int p = 0; p < a.nproj; ++p) {
     P.cb_before[p + 1] = P.cb_before[p] + (a.proj[p].d_out + RG_NT - 1) / RG_NT;
     if ((err = encode_row_map(&P.yb_map[p], const_cast<void*>(a.proj[p].y_base), a.T, a.proj[p].d_out)) != cudaSuccess)
       return err;
     if ((err = encode_row_map(&P.y_map[p], a.proj[p].y, a.T, a.proj[p].d_out)) != cudaSuccess) return err;
   }
-  static SmemLimit lim;
-  const size_t smem = RgSmem::total();
-  if ((err = lim.ensure((const void*)ragged_expand_kernel, smem)) != cudaSuccess) return err;
-  if ((err = launch_tc_shrink_ragged(a, P.vc_off, P.tiles_off, P.max_tiles, s)) != cudaSuccess) return err;
+  static SmemLimit lim1, lim2;
+  const size_t smem1 = rs_smem(S->pg, R16, S->stages).total, smem2 = RgSmem::total();
+  if ((err = lim1.ensure((const void*)rg_shrink_kernel, smem1)) != cudaSuccess) return err;
+  if ((err = lim2.ensure((const void*)ragged_expand_kernel, smem2)) != cudaSuccess) return err;
+  const long items = (long)max_qtiles(a.T, a.k, a.E) * S->npg;
+  long g1 = items < nsm ? items : nsm;
+  if (g1 > kRgMaxCtas) g1 = kRgMaxCtas;
+  if ((err = launch_pdl(rg_shrink_kernel, dim3((unsigned)g1), dim3(RS_BLOCK), smem1, s, *S)) != cudaSuccess) return err;
   const long units = (long)P.max_tiles * P.cb_before[a.nproj];
-  const int nsm = device_sm_count();
   const int grid = (int)(units < nsm ? units : nsm);
-  return launch_pdl(ragged_expand_kernel, dim3(grid), dim3(RG_BLOCK), smem, s, P);
+  return launch_pdl(ragged_expand_kernel, dim3(grid), dim3(RG_BLOCK), smem2, s, P);
 }
 
 }  // namespace apr

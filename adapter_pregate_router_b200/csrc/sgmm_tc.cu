@@ -65,82 +65,13 @@ struct TcPlan {
   int ny;                            // expand ring depth
   int mixed;                         // expand over mixed tiles (<= 4 adapters, K2 = 4 * R16) instead of set tiles
   int ytma;                          // expand stores y rows with tile::scatter4 (else plain stores)
-  int vpair;                         // shrink output: 0 by plan position as bf16 hi | lo ([proj][pair
-                                     // position][2 * R16]); 1 by pair id, bf16 ([proj][q][R16]); 2 by
-                                     // plan position, bf16 ([proj][pair position][R16])
+  int vpair;                         // shrink writes v by pair id, bf16 only ([proj][q][R16]) instead of
+                                     // by plan position as bf16 hi | lo ([proj][pair position][2 * R16])
   size_t vprep_off;                  // scratch: V rows
-  size_t rg_off;                     // scratch: ragged tiles built by the shrink (0: none)
-  int rg_max;                        // room for ragged tiles
   int cc_before[APR_MAX_PROJ + 1];   // expand: prefix of 1024-column items per projection
 };
 
 static_assert(TB_MAXK2 == kTensorMaxK2, "tensor scratch sizing");
-
-// ---------------------------------------------------------------- ragged tiles
-
-// The ragged tiles of a top-1 plan, built by one warp whose lanes all hold the same walk state
-// (lane s < kRgSlots also holds slot s of the open tile).  Adapters are taken in order; a tile
-// closes before an adapter (or the rest of one) that would make it hold more than kSetTile
-// tokens, more than kRgSlots adapters or more than kRgKmax rank rows.  The count is written even
-// past `max_tiles` (the expand checks it).
-__device__ void rg_plan(const SgmmArgs& a, int R16, int* count, RgTile* tiles, int max_tiles) {
-  const int lane = threadIdx.x & 31;
-  int t_start = 0, t_len = 0, t_nu = 0, t_kt = 0, nt = 0;
-  int my_u = 0, my_koff = 0;
-  auto close = [&]() {
-    if (t_len > 0) {
-      if (nt < max_tiles) {
-        RgTile* tl = tiles + nt;
-        if (lane < kRgSlots) {
-          tl->u[lane] = (short)(lane < t_nu ? my_u : -1);
-          tl->koff[lane] = (short)(lane < t_nu ? my_koff : t_kt);
-        }
-        if (lane == 0) {
-          tl->start = t_start;
-          tl->len = t_len;
-          tl->nu = t_nu;
-          tl->kt = t_kt;
-        }
-      }
-      ++nt;
-    }
-    t_len = t_nu = t_kt = 0;
-  };
-  for (int e0 = 0; e0 < a.E; e0 += 32) {
-    const int e = e0 + lane;
-    int beg = 0, cnt = 0, w = 16;
-    if (e < a.E) {
-      beg = a.seg_off[e];
-      cnt = a.seg_off[e + 1] - beg;
-      const int r = a.ranks[e];
-      // an invalid rank (reported by the shrink) keeps a slot of 16 zero rows
-      if (r >= 8 && r <= R16 && (r & 7) == 0) w = (r + 15) / 16 * 16;
-    }
-    unsigned m = __ballot_sync(0xffffffffu, cnt > 0);
-    while (m) {
-      const int j = __ffs(m) - 1;
-      m &= m - 1;
-      int c = __shfl_sync(0xffffffffu, cnt, j), pos = __shfl_sync(0xffffffffu, beg, j);
-      const int wj = __shfl_sync(0xffffffffu, w, j);
-      while (c > 0) {
-        if (t_nu == kRgSlots || t_kt + wj > kRgKmax || t_len == kSetTile) close();
-        if (t_len == 0) t_start = pos;
-        const int take = min(c, kSetTile - t_len);
-        if (lane == t_nu) {
-          my_u = e0 + j;
-          my_koff = t_kt;
-        }
-        ++t_nu;
-        t_kt += wj;
-        t_len += take;
-        c -= take;
-        pos += take;
-      }
-    }
-  }
-  close();
-  if (lane == 0) *count = nt;
-}
 
 // ---------------------------------------------------------------- shrink
 
@@ -203,10 +134,6 @@ __global__ void __launch_bounds__(SH_BLOCK, 1) tc_shrink_kernel(const __grid_con
   const int d_in = a.d_in, nk = d_in / TB_BK;
   uint32_t gchunk = 0, nitem = 0;
   bool abort = false;
-  if (P.rg_off && blockIdx.x == gridDim.x - 1 && warp == 0) {
-    int* cnt = ws_at<int>(a.ws, P.rg_off);
-    rg_plan(a, R16, cnt, reinterpret_cast<RgTile*>(cnt + 4), P.rg_max);
-  }
 
   // items are taken from a work counter (after one static item per CTA), so CTAs that
   // draw small tiles take more of them
@@ -324,8 +251,7 @@ __global__ void __launch_bounds__(SH_BLOCK, 1) tc_shrink_kernel(const __grid_con
             lo[i] = pack_bf16x2(a0 - hf.x, a1 - hf.y);
           }
           if (valid && P.vpair) {
-            const long at = P.vpair == 1 ? (long)s_pair[row] : (long)tile.start + row;
-            __nv_bfloat16* dst = vprep + ((size_t)(q0 + qi) * npairs + at) * R16 + rr;
+            __nv_bfloat16* dst = vprep + ((size_t)(q0 + qi) * npairs + s_pair[row]) * R16 + rr;
             reinterpret_cast<uint4*>(dst)[0] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
             reinterpret_cast<uint4*>(dst)[1] = make_uint4(hi[4], hi[5], hi[6], hi[7]);
           } else if (valid) {
@@ -773,16 +699,6 @@ cudaError_t launch_tc_shrink_pairs(const SgmmArgs& a, size_t v_off, cudaStream_t
   TcPlan t;
   memset(&t, 0, sizeof(t));
   shrink_plan(t, a, v_off, 1);
-  return launch_shrink(t, s);
-}
-
-cudaError_t launch_tc_shrink_ragged(const SgmmArgs& a, size_t v_off, size_t tiles_off, int max_tiles,
-                                    cudaStream_t s) {
-  TcPlan t;
-  memset(&t, 0, sizeof(t));
-  shrink_plan(t, a, v_off, 2);
-  t.rg_off = tiles_off;
-  t.rg_max = max_tiles;
   return launch_shrink(t, s);
 }
 

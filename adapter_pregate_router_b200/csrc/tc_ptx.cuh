@@ -15,6 +15,10 @@ cudaError_t encode_row_map(CUtensorMap* m, void* base, int rows, int cols);
 // Host: a [rows, cols] bf16 tensor map with 64-column x box_rows boxes and
 // 128-byte swizzle (zeros outside the tensor on loads; stores are clipped).
 cudaError_t encode_tile_map(CUtensorMap* m, const void* base, int rows, int cols, int box_rows);
+// [rows, cols] bf16 with a row pitch of `pitch_bytes`; boxes of box_cols x box_rows; 128-byte
+// swizzle or none; zeros outside on loads.
+cudaError_t encode_box_map(CUtensorMap* m, const void* base, long rows, long cols, long pitch_bytes, int box_cols,
+                           int box_rows, bool swizzle128);
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -178,6 +182,31 @@ __device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncol
 }
 __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
   asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// A tensor map in global memory made from a template whose global address is replaced (a whole
+// warp): the template is staged in `sbuf` (128 bytes, 128-byte aligned shared memory), its address
+// field rewritten, and the result copied to `gdst` (128-byte aligned) with a release of the
+// tensor-map proxy.  The template's dimensions, strides, box and swizzle stay as encoded.
+__device__ __forceinline__ void tmap_build(void* gdst, uint32_t sbuf, const CUtensorMap* tmpl, const void* addr) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t w = reinterpret_cast<const uint32_t*>(tmpl)[lane];
+  asm volatile("st.shared.u32 [%0], %1;" ::"r"(sbuf + (uint32_t)lane * 4), "r"(w) : "memory");
+  __syncwarp();
+  if (lane == 0)
+    asm volatile("tensormap.replace.tile.global_address.shared::cta.b1024.b64 [%0], %1;" ::"r"(sbuf), "l"(addr)
+                 : "memory");
+  __syncwarp();
+  asm volatile(
+      "tensormap.cp_fenceproxy.global.shared::cta.tensormap::generic.release.gpu.sync.aligned [%0], [%1], 128;" ::"l"(
+          gdst),
+      "r"(sbuf)
+      : "memory");
+  __syncwarp();
+}
+// Before the first copy through a tensor map written by tmap_build (by the thread issuing it).
+__device__ __forceinline__ void tmap_acquire(const void* gmap) {
+  asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(gmap) : "memory");
 }
 
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }

@@ -169,7 +169,8 @@ __device__ void rg_plan(const SgmmArgs& a, int R16, int* count, RgTile* tiles, i
 // one static item per CTA), so CTAs drawing high-rank adapters take fewer of them.
 constexpr int RS_EPI = 256;                   // warps 2-9
 constexpr int RS_BLOCK = 64 + RS_EPI;         // warp 0: producer, warp 1: MMA issue
-constexpr int RS_XBYTES = 128 * 128;          // x rows of a stage (128 x 64 columns, 128-byte swizzle)
+constexpr int RS_XBYTES = 128 * 128;          // x rows of a sub-block (128 x 64 columns, 128-byte swizzle)
+constexpr int RS_SB = 2;                      // 64-column sub-blocks per stage: 256 contiguous bytes of each row
 constexpr int RS_NQ = 4;                      // projections per item at most
 
 struct RsPlan {
@@ -186,13 +187,14 @@ struct RsItem {
 };
 
 struct RsSmem {
-  int stage_bytes, S;
+  int stage_bytes, abytes, S;                 // abytes: adapter rows of one sub-block
   size_t bar, item, gate, mapbuf, tmem, total;
 };
 __host__ __device__ inline RsSmem rs_smem(int pg, int R16, int S) {
   RsSmem L;
   // the adapter rows of a stage: at least the 128 rows one accumulator's MMAs read
-  L.stage_bytes = RS_XBYTES + (pg * R16 < 128 ? 128 : pg * R16) * 128;
+  L.abytes = (pg * R16 < 128 ? 128 : pg * R16) * 128;
+  L.stage_bytes = RS_SB * (RS_XBYTES + L.abytes);
   L.S = S;
   L.bar = (size_t)S * L.stage_bytes;
   L.item = L.bar + (size_t)(2 * S + 6) * 8;
@@ -246,7 +248,7 @@ __global__ void __launch_bounds__(RS_BLOCK, 1) rg_shrink_kernel(const __grid_con
   WsHeader* hdr = reinterpret_cast<WsHeader*>(a.ws);
   const PairTile* qtiles = ws_at<PairTile>(a.ws, W.qtiles);
   const long nitems = (long)hdr->n_qtiles * P.npg;
-  const int nk = a.d_in / 64;
+  const int nblk = a.d_in / 64, nk = (nblk + RS_SB - 1) / RS_SB;   // 64-column blocks; stages
   bool abort = false;
 
   if (warp == 0) {
@@ -325,19 +327,26 @@ __global__ void __launch_bounds__(RS_BLOCK, 1) rg_shrink_kernel(const __grid_con
         if (lane == 0) tmap_acquire(am + qi);
       }
       const int ngr = (len + 3) >> 2;
-      const uint32_t bytes = (uint32_t)(ngr * 512 + nq * R16 * 128);
+      const uint32_t sb_bytes = (uint32_t)(ngr * 512 + nq * R16 * 128);   // one sub-block
       for (int c = 0; c < nk; ++c, ++g) {
         const uint32_t s = g % S;
         if (c > 0 && g >= (uint32_t)S && !__all_sync(0xffffffffu, mbar_wait(bar_empty + 8 * s, ((g / S) - 1) & 1))) {
           abort = true;
           break;
         }
-        const uint32_t xs = sbase + s * (uint32_t)L.stage_bytes, as = xs + RS_XBYTES;
-        if (lane == 0) mbar_arrive_expect_tx(bar_full + 8 * s, bytes);
+        const int nsb = min(RS_SB, nblk - RS_SB * c);
+        const uint32_t xs = sbase + s * (uint32_t)L.stage_bytes, as = xs + RS_SB * RS_XBYTES;
+        if (lane == 0) mbar_arrive_expect_tx(bar_full + 8 * s, (uint32_t)nsb * sb_bytes);
         __syncwarp();
-        if (lane < ngr) tma_gather4(xs + (uint32_t)(4 * lane) * 128, &P.xmap, 64 * c, tk[0], tk[1], tk[2], tk[3], bar_full + 8 * s);
-        if (lane == 0)
-          for (int qi = 0; qi < nq; ++qi) tma_load_2d(as + (uint32_t)(qi * R16) * 128, am + qi, 64 * c, 0, bar_full + 8 * s);
+        for (int b = 0; b < nsb; ++b) {
+          const int col = 64 * (RS_SB * c + b);
+          if (lane < ngr)
+            tma_gather4(xs + (uint32_t)b * RS_XBYTES + (uint32_t)(4 * lane) * 128, &P.xmap, col, tk[0], tk[1], tk[2],
+                        tk[3], bar_full + 8 * s);
+          if (lane == 0)
+            for (int qi = 0; qi < nq; ++qi)
+              tma_load_2d(as + (uint32_t)b * L.abytes + (uint32_t)(qi * R16) * 128, am + qi, col, 0, bar_full + 8 * s);
+        }
       }
       ++k;
       item = next;
@@ -363,12 +372,15 @@ __global__ void __launch_bounds__(RS_BLOCK, 1) rg_shrink_kernel(const __grid_con
           const uint32_t s = g % S;
           if (!mbar_wait(bar_full + 8 * s, (g / S) & 1)) { abort = true; break; }
           tc_fence_after();
-          const uint32_t xs = sbase + s * (uint32_t)L.stage_bytes, as = xs + RS_XBYTES;
-          for (int m = 0; m < nacc; ++m)
+          const int nsb = min(RS_SB, nblk - RS_SB * c);
+          const uint32_t xs = sbase + s * (uint32_t)L.stage_bytes, as = xs + RS_SB * RS_XBYTES;
+          for (int b = 0; b < nsb; ++b)
+            for (int m = 0; m < nacc; ++m)
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_bf16(tmem + (uint32_t)m * 128, desc_k_sw128(as + (uint32_t)m * RS_XBYTES + kk * 32),
-                       desc_k_sw128(xs + kk * 32), id, (c > 0 || kk > 0) ? 1u : 0u);
+              for (int kk = 0; kk < 4; ++kk)
+                mma_bf16(tmem + (uint32_t)m * 128,
+                         desc_k_sw128(as + (uint32_t)b * L.abytes + (uint32_t)m * (128 * 128) + kk * 32),
+                         desc_k_sw128(xs + (uint32_t)b * RS_XBYTES + kk * 32), id, (c > 0 || b > 0 || kk > 0) ? 1u : 0u);
           mma_commit(bar_empty + 8 * s);
         }
         if (abort) break;

@@ -50,7 +50,8 @@ constexpr int RG_NT = 128;                    // output columns per unit
 constexpr int RG_NS = 2;                      // stages of (y tile, Bcat)
 constexpr int RG_EPI = 256;                   // warps 0-7: epilogue (lane quarter x column half)
 constexpr int RG_VW = 128;                    // warps 8-11: V rows into TMEM
-constexpr int RG_BLOCK = RG_EPI + RG_VW + 64;  // warp 12: TMA producer, warp 13: MMA issue
+constexpr int RG_YW = 128;                    // warps 13-16: y_base rows by 16-byte cp.async
+constexpr int RG_BLOCK = RG_EPI + RG_VW + 32 + RG_YW + 32;   // warp 12: Bcat by TMA, warp 17: MMA issue
 constexpr uint32_t RG_TMEM_COLS = 512;        // [V0 | V1 | D0 | D1], 128 columns each
 constexpr int RG_YTILE = RG_M * RG_NT * 2;    // 32 KB: two 64-column halves of 128 rows x 128 B
 constexpr int RG_BCAT = kRgKmax * RG_NT * 2;  // 64 KB
@@ -466,7 +467,7 @@ __global__ void __launch_bounds__(RG_BLOCK, 1) ragged_expand_kernel(const __grid
 
   if (tid == 0) {
     for (int i = 0; i < RG_NS; ++i) {
-      mbar_init(bar_full + 8 * i, 1);
+      mbar_init(bar_full + 8 * i, 1 + RG_YW);
       mbar_init(bar_empty + 8 * i, RG_EPI / 32 + 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -721,15 +722,8 @@ __global__ void __launch_bounds__(RG_BLOCK, 1) ragged_expand_kernel(const __grid
       const bool new_tile = ti != cur_ti, new_proj = new_tile || p != cur_p;
       cur_ti = ti;
       cur_p = p;
-      if (new_tile) {
-        len = tl.len;
-        // rows 4 * lane .. + 3; rows past the tile repeat its first token (loaded, never stored)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int r = 4 * lane + q;
-          tk[q] = a.perm[tl.start + (r < len ? r : 0)];
-        }
-      }
+      (void)tk;
+      (void)len;
       if (new_proj) {
         const int nu = tl.nu;
         my_map = nullptr;
@@ -755,13 +749,10 @@ __global__ void __launch_bounds__(RG_BLOCK, 1) ragged_expand_kernel(const __grid
         fence_proxy_async();
       }
       __syncwarp();
-      const int nh = c0 + 64 < d_out ? 2 : 1, ngr = (len + 3) >> 2;
-      if (lane == 0) mbar_arrive_expect_tx(bar_full + 8 * s, (uint32_t)(ngr * nh * 512 + bbytes));
+      (void)ys;
+      (void)d_out;
+      if (lane == 0) mbar_arrive_expect_tx(bar_full + 8 * s, (uint32_t)bbytes);
       __syncwarp();
-      if (lane < ngr)
-        for (int h = 0; h < nh; ++h)
-          tma_gather4(ys + (uint32_t)h * (RG_M * 128) + (uint32_t)(4 * lane) * 128, &P.yb_map[p], c0 + 64 * h, tk[0],
-                      tk[1], tk[2], tk[3], bar_full + 8 * s);
       // Bcat chunk kc = rank rows 8c..8c+7 of the slot for the unit's 128 columns: one box of 8
       // columns x 128 rows of B, which lands as the chunk's 16 core matrices (zeros past the rank
       // and past d_out)
@@ -773,6 +764,48 @@ __global__ void __launch_bounds__(RG_BLOCK, 1) ragged_expand_kernel(const __grid
     // after an abort, the copies of the stages filled last land before the CTA exits (bounded)
     if (abort && lane == 0)
       for (int i = max(last - RG_NS + 1, 0); i <= last; ++i) (void)mbar_wait(bar_full + 8 * (i % RG_NS), (i / RG_NS) & 1);
+  } else if (tid < RG_EPI + RG_VW + 32 + RG_YW) {
+    // ---------------------------------------------------------------- y_base rows
+    // thread yt copies 16-byte pieces yt, yt + 128, ... of the unit's 128 rows x 256 bytes (16
+    // pieces per row, a row's pieces on consecutive threads) into the 128-byte swizzled halves
+    const int yt = tid - (RG_EPI + RG_VW + 32);
+    const int q = yt & 15, half = q >> 3, chunk = q & 7, r0 = yt >> 4;   // rows r0, r0 + 8, ...
+    int cur_ti = -1, len = 0, tok[16];
+    for (int i = 0; i < n && !abort; ++i) {
+      int ti, p, c0;
+      unit_at(i, ti, p, c0);
+      const int s = i % RG_NS;
+      if (i >= RG_NS && !__all_sync(0xffffffffu, mbar_wait(bar_empty + 8 * s, ((i / RG_NS) - 1) & 1))) {
+        abort = true;
+        break;
+      }
+      if (ti != cur_ti) {
+        cur_ti = ti;
+        const RgTile& tl = tiles[ti];
+        len = tl.len;
+#pragma unroll
+        for (int m = 0; m < 16; ++m) {
+          const int r = r0 + 8 * m;
+          tok[m] = r < len ? a.perm[tl.start + r] : -1;
+        }
+      }
+      const int d_out = a.proj[p].d_out;
+      const int col = c0 + half * 64 + chunk * 8;
+      const __nv_bfloat16* yb = reinterpret_cast<const __nv_bfloat16*>(a.proj[p].y_base) + col;
+      const uint32_t ys = sY + (uint32_t)s * RG_YTILE + (uint32_t)half * (RG_M * 128);
+      if (col < d_out) {
+#pragma unroll
+        for (int m = 0; m < 16; ++m) {
+          const int r = r0 + 8 * m;
+          if (tok[m] >= 0)
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(ys + (uint32_t)r * 128 + (uint32_t)((chunk ^ (r & 7)) << 4)),
+                         "l"(yb + (size_t)tok[m] * d_out)
+                         : "memory");
+        }
+      }
+      cp_async_arrive(bar_full + 8 * s);
+    }
+    cp_async_wait_all();
   } else if (lane == 0) {
     // ---------------------------------------------------------------- MMA issue
     const uint32_t id = idesc_bf16(RG_M, RG_NT);

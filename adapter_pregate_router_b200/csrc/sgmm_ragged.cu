@@ -169,7 +169,8 @@ __device__ void rg_plan(const SgmmArgs& a, int R16, int* count, RgTile* tiles, i
 // adapter row), scale by each token's gate and store bf16.  Items come from a work counter (after
 // one static item per CTA), so CTAs drawing high-rank adapters take fewer of them.
 constexpr int RS_EPI = 256;                   // warps 2-9
-constexpr int RS_BLOCK = 64 + RS_EPI;         // warp 0: producer, warp 1: MMA issue
+constexpr int RS_XW = 128;                    // warps 10-13: x rows by 16-byte cp.async
+constexpr int RS_BLOCK = 64 + RS_EPI + RS_XW; // warp 0: item setup and A boxes, warp 1: MMA issue
 constexpr int RS_XBYTES = 128 * 128;          // x rows of a sub-block (128 x 64 columns, 128-byte swizzle)
 constexpr int RS_SB = 2;                      // 64-column sub-blocks per stage: 256 contiguous bytes of each row
 constexpr int RS_NQ = 4;                      // projections per item at most
@@ -189,7 +190,7 @@ struct RsItem {
 
 struct RsSmem {
   int stage_bytes, abytes, S;                 // abytes: adapter rows of one sub-block
-  size_t bar, item, gate, mapbuf, tmem, total;
+  size_t bar, item, gate, tok, mapbuf, tmem, total;
 };
 __host__ __device__ inline RsSmem rs_smem(int pg, int R16, int S) {
   RsSmem L;
@@ -200,7 +201,8 @@ __host__ __device__ inline RsSmem rs_smem(int pg, int R16, int S) {
   L.bar = (size_t)S * L.stage_bytes;
   L.item = L.bar + (size_t)(2 * S + 6) * 8;
   L.gate = L.item + 2 * sizeof(RsItem);
-  L.mapbuf = (L.gate + 2 * 128 * 4 + 127) / 128 * 128;
+  L.tok = L.gate + 2 * 128 * 4;
+  L.mapbuf = (L.tok + 2 * 128 * 4 + 127) / 128 * 128;
   L.tmem = L.mapbuf + (RS_NQ + 1) * 128;
   L.total = L.tmem + 16 + 1024;
   return L;
@@ -220,17 +222,18 @@ __global__ void __launch_bounds__(RS_BLOCK, 1) rg_shrink_kernel(const __grid_con
   const uint32_t bar_dfull = smem_u32(bars + 2 * S + 4), bar_dempty = smem_u32(bars + 2 * S + 5);
   RsItem* s_item = reinterpret_cast<RsItem*>(smem + L.item);
   float* s_g = reinterpret_cast<float*>(smem + L.gate);
+  int* s_tok = reinterpret_cast<int*>(smem + L.tok);
   const uint32_t sbase = smem_u32(smem), s_mapbuf = sbase + (uint32_t)L.mapbuf;
   volatile uint32_t* s_tmem = reinterpret_cast<volatile uint32_t*>(smem + L.tmem);
 
   if (tid == 0) {
     for (int i = 0; i < S; ++i) {
-      mbar_init(bar_full + 8 * i, 1);
+      mbar_init(bar_full + 8 * i, 1 + RS_XW);
       mbar_init(bar_empty + 8 * i, 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar_ifull + 8 * i, 1);
-      mbar_init(bar_iempty + 8 * i, 1 + RS_EPI / 32);
+      mbar_init(bar_iempty + 8 * i, 1 + RS_EPI / 32 + RS_XW / 32);
     }
     mbar_init(bar_dfull, 1);
     mbar_init(bar_dempty, RS_EPI);
@@ -293,13 +296,12 @@ __global__ void __launch_bounds__(RS_BLOCK, 1) rg_shrink_kernel(const __grid_con
         continue;
       }
       const int len = tile.len;
-      // the item's tokens (rows 4 * lane .. + 3; rows past the tile repeat its first token) and gates
-      int tk[4];
+      // the item's tokens (for the x loaders) and gates
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int row = 4 * lane + j;
         const int q = a.perm[tile.start + (row < len ? row : 0)];
-        tk[j] = q;                                     // top-1: the pair id is the token
+        s_tok[slot * 128 + row] = q;                   // top-1: the pair id is the token
         s_g[slot * 128 + row] = row < len ? a.gate[q] : 0.f;
       }
       if (lane == 0) {
@@ -327,8 +329,7 @@ __global__ void __launch_bounds__(RS_BLOCK, 1) rg_shrink_kernel(const __grid_con
         tmap_build(am + qi, s_mapbuf + qi * 128, &P.atmpl[q0 + qi][r / 8 - 1], a.proj[q0 + qi].A[e]);
         if (lane == 0) tmap_acquire(am + qi);
       }
-      const int ngr = (len + 3) >> 2;
-      const uint32_t sb_bytes = (uint32_t)(ngr * 512 + nq * R16 * 128);   // one sub-block
+      const uint32_t sb_bytes = (uint32_t)(nq * R16 * 128);   // A boxes of one sub-block
       for (int c = 0; c < nk; ++c, ++g) {
         const uint32_t s = g % S;
         if (c > 0 && g >= (uint32_t)S && !__all_sync(0xffffffffu, mbar_wait(bar_empty + 8 * s, ((g / S) - 1) & 1))) {
@@ -341,9 +342,6 @@ __global__ void __launch_bounds__(RS_BLOCK, 1) rg_shrink_kernel(const __grid_con
         __syncwarp();
         for (int b = 0; b < nsb; ++b) {
           const int col = 64 * (RS_SB * c + b);
-          if (lane < ngr)
-            tma_gather4(xs + (uint32_t)b * RS_XBYTES + (uint32_t)(4 * lane) * 128, &P.xmap, col, tk[0], tk[1], tk[2],
-                        tk[3], bar_full + 8 * s);
           if (lane == 0)
             for (int qi = 0; qi < nq; ++qi)
               tma_load_2d(as + (uint32_t)b * L.abytes + (uint32_t)(qi * R16) * 128, am + qi, col, 0, bar_full + 8 * s);
@@ -389,6 +387,52 @@ __global__ void __launch_bounds__(RS_BLOCK, 1) rg_shrink_kernel(const __grid_con
         ++k;
       }
     }
+  } else if (warp >= 2 + RS_EPI / 32) {
+    // ---------------------------------------------------------------- x loaders
+    // thread xt copies 16-byte pieces of the item's token rows: 16 pieces (two 64-column
+    // sub-blocks x 8) per row on consecutive threads, rows r0, r0 + 8, ... into 128-byte swizzled rows
+    const int xt = tid - (64 + RS_EPI);
+    const int q = xt & 15, sub = q >> 3, chunk = q & 7, r0 = xt >> 4;
+    const __nv_bfloat16* x = reinterpret_cast<const __nv_bfloat16*>(a.x);
+    uint32_t g = 0, k = 0;
+    while (true) {
+      const int slot = k & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_ifull + 8 * slot, (k >> 1) & 1))) { abort = true; break; }
+      const RsItem it = s_item[slot];
+      if (it.e < 0) break;
+      int tok[16];
+#pragma unroll
+      for (int m = 0; m < 16; ++m) {
+        const int r = r0 + 8 * m;
+        tok[m] = r < it.len ? s_tok[slot * 128 + r] : -1;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_iempty + 8 * slot);   // the item's tokens are in registers
+      for (int c = 0; c < nk; ++c, ++g) {
+        const uint32_t s = g % S;
+        if (g >= (uint32_t)S && !__all_sync(0xffffffffu, mbar_wait(bar_empty + 8 * s, ((g / S) - 1) & 1))) {
+          abort = true;
+          break;
+        }
+        const int nsb = min(RS_SB, nblk - RS_SB * c);
+        if (sub < nsb) {
+          const uint32_t xs = sbase + s * (uint32_t)L.stage_bytes + (uint32_t)sub * RS_XBYTES;
+          const __nv_bfloat16* src = x + 64 * (RS_SB * c + sub) + chunk * 8;
+#pragma unroll
+          for (int m = 0; m < 16; ++m) {
+            const int r = r0 + 8 * m;
+            if (tok[m] >= 0)
+              asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(xs + (uint32_t)r * 128 + (uint32_t)((chunk ^ (r & 7)) << 4)),
+                           "l"(src + (size_t)tok[m] * a.d_in)
+                           : "memory");
+          }
+        }
+        cp_async_arrive(bar_full + 8 * s);
+      }
+      if (abort) break;
+      ++k;
+    }
+    cp_async_wait_all();
   } else {
     // ---------------------------------------------------------------- epilogue
     const int ew = warp - 2, quarter = warp & 3;

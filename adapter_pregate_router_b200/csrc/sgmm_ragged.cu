@@ -1,16 +1,26 @@
-// SGMM expand for many tenants: top-1 routing over many adapters of mixed
-// ranks (tcgen05).  AdaFuse summary (gist.science), Resumen tecnico §2.B: the
+// SGMM for many tenants: top-1 routing over many adapters of mixed ranks
+// (tcgen05).  AdaFuse summary (gist.science), Resumen tecnico §2.B: the
 // segmented gather product applies each token's selected low-rank adapter to
 // the tokens gathered per adapter and is fused into the add onto the base
 // projection output; the Chameleon page (7minutos.es), adapter cache: tenants'
 // adapters range over ranks 8-128.
 //
-// With many adapters each one holds only a few tokens, so a tile of one
-// adapter leaves most of the 128 MMA rows empty.  Here a tile is a ragged run
-// of consecutive plan tokens (sorted by adapter): up to 128 tokens of up to 16
-// adapters whose rank slots (each rank rounded up to 16) add up to <= 256.  The
-// shrink (tc_shrink_kernel) leaves g * A_e x of every token in plan order and
-// builds the tiles.  A unit is (tile, projection, 128 output columns):
+// Two launches per call.
+//
+// Shrink (rg_shrink_kernel): v = g * A_e x for every token, by plan position.
+// An item is one pair tile of an adapter (<= 128 tokens) and a group of
+// projections; the adapter's rank rows are the MMA's M side and the tokens its
+// N side, so a short segment costs only its own tokens.  A arrives by 2-D TMA
+// boxes from tensor maps the kernel writes per item (a template per rank with
+// the adapter's address), x rows by 16-byte cp.async, 128 columns (256 bytes of
+// every row) per stage.  The same kernel builds the ragged tiles and each used
+// adapter's B tensor map for the expand.
+//
+// Expand (ragged_expand_kernel): with many adapters each one holds only a few
+// tokens, so a tile of one adapter would leave most of the 128 MMA rows empty.
+// A ragged tile is a run of consecutive plan tokens (sorted by adapter): up to
+// 128 tokens of up to 16 adapters whose rank slots (each rank rounded up to
+// 16) add up to <= 256.  A unit is (tile, projection, 128 output columns):
 //
 //   D[t, n] = sum_{s < nu} sum_{r < w_s} V[t, koff_s + r] * B_{u_s}[c0 + n, r]
 //   V[t, koff_s + r] = g_t (A_{u_s} x_t)[r]  if token t selected u_s, else 0
@@ -19,11 +29,13 @@
 //    bulk copy stages them, and a warpgroup writes each token's row of V (its
 //    slot, zeros elsewhere) into tensor memory, the MMA's A operand; two TMEM
 //    V buffers, rebuilt when the tile or the projection changes.
-//  - Bcat[n][koff_s + r] = B_{u_s}[c0 + n][r]: 16-byte cp.async from four
-//    producer warps into K-major 8x16-byte core matrices (zeros past a rank).
-//  - y_base rows of the tile's tokens come in by TMA tile::gather4 (four token
-//    rows of 64 columns per copy, 128-byte swizzle); y rows go out by
-//    tile::scatter4 (groups of four tokens) and 16-byte stores (the rest).
+//  - Bcat[n][koff_s + r] = B_{u_s}[c0 + n][r]: TMA boxes of 8 rank columns x
+//    128 rows of B_{u_s}, each landing as one K chunk of 8x16-byte core
+//    matrices (zeros past the rank and past d_out).
+//  - y_base rows of the tile's tokens come in by 16-byte cp.async (a row's 256
+//    bytes on 16 consecutive threads, 128-byte swizzle); y rows go out by
+//    16-byte stores.  (Per-row TMA gather copies measured slower for both x
+//    and y here.)
 //  - One thread issues the kt/16 MMAs (M = N = 128) into a double-buffered
 //    TMEM accumulator; eight epilogue warps add D to y_base in shared memory
 //    and round once to bf16.  Two stages of (y tile, Bcat) overlap loads, MMAs
@@ -58,8 +70,6 @@ constexpr int RG_BCAT = kRgKmax * RG_NT * 2;  // 64 KB
 constexpr int RG_VROW = 256;                  // a token's staged gated v row (R16 <= 128 bf16)
 
 struct RgPlan {
-  CUtensorMap yb_map[APR_MAX_PROJ];   // y_base rows: 64-column boxes, gather4 loads
-  CUtensorMap y_map[APR_MAX_PROJ];    // y rows: 64-column boxes, scatter4 stores
   SgmmArgs a;
   int R16;                            // rank slot of the staged v rows
   int max_tiles;
@@ -610,39 +620,26 @@ __global__ void __launch_bounds__(RG_BLOCK, 1) ragged_expand_kernel(const __grid
       }
       tc_fence_before();
       mbar_arrive(bar_dempty + 8 * db);
-      fence_proxy_async();                            // the new bytes are visible to the TMA engine
       __syncwarp();
       const int x = c0 + half * 64;
       if (nvalid > 0 && x < d_out) {
-        // groups of four token rows by tile::scatter4 (the map clips columns past d_out)
-        const int ng = nvalid >> 2;
-#pragma unroll
-        for (int g = 0; g < 8; ++g) {
-          const int t0 = __shfl_sync(0xffffffffu, tok, 4 * g), t1 = __shfl_sync(0xffffffffu, tok, 4 * g + 1);
-          const int t2 = __shfl_sync(0xffffffffu, tok, 4 * g + 2), t3 = __shfl_sync(0xffffffffu, tok, 4 * g + 3);
-          if (lane == 0 && g < ng)
-            tma_scatter4(&P.y_map[p], x, t0, t1, t2, t3,
-                         smem_u32(yhalf + (size_t)(quarter * 32 + 4 * g) * 128));
-        }
-        // the last one to three rows by 16-byte stores, 8 lanes per row
-        const int rr = 4 * ng + (lane >> 3);
-        const int tk = __shfl_sync(0xffffffffu, tok, rr);
+        // the warp's rows by 16-byte stores: 8 lanes per 128-byte row piece, 4 rows per pass
+        __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(a.proj[p].y);
         const int col = half * 64 + (lane & 7) * 8;
-        if (rr < nvalid && c0 + col < d_out) {
-          const int r = quarter * 32 + rr;
-          const uint4 val = *reinterpret_cast<const uint4*>(yhalf + (size_t)r * 128 + (((lane & 7) ^ (r & 7)) << 4));
-          __stcs(reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.proj[p].y) + (size_t)tk * d_out + c0 + col),
-                 val);
+#pragma unroll
+        for (int it4 = 0; it4 < 8; ++it4) {
+          const int rr = 4 * it4 + (lane >> 3);
+          const int tk = __shfl_sync(0xffffffffu, tok, rr);
+          if (rr < nvalid && c0 + col < d_out) {
+            const int r = quarter * 32 + rr;
+            const uint4 val = *reinterpret_cast<const uint4*>(yhalf + (size_t)r * 128 + (((lane & 7) ^ (r & 7)) << 4));
+            __stcs(reinterpret_cast<uint4*>(y + (size_t)tk * d_out + c0 + col), val);
+          }
         }
       }
-      if (lane == 0) {
-        bulk_commit();
-        bulk_wait_read_all();                          // the stage may be refilled once the copies read it
-      }
-      __syncwarp();
+      __syncwarp();                                    // the stores have read the stage
       if (lane == 0) mbar_arrive(bar_empty + 8 * s);
     }
-    if (lane == 0) bulk_wait_all();                    // every y row written before the CTA ends
   } else if (tid < RG_EPI + RG_VW) {
     // ---------------------------------------------------------------- V rows into TMEM
     const int vt = tid - RG_EPI;
@@ -951,9 +948,6 @@ cudaError_t launch_sgmm_ragged(const SgmmArgs& a, size_t scratch_off, cudaStream
   P.cb_before[0] = 0;
   for (int p = 0; p < a.nproj; ++p) {
     P.cb_before[p + 1] = P.cb_before[p] + (a.proj[p].d_out + RG_NT - 1) / RG_NT;
-    if ((err = encode_row_map(&P.yb_map[p], const_cast<void*>(a.proj[p].y_base), a.T, a.proj[p].d_out)) != cudaSuccess)
-      return err;
-    if ((err = encode_row_map(&P.y_map[p], a.proj[p].y, a.T, a.proj[p].d_out)) != cudaSuccess) return err;
   }
   static SmemLimit lim1, lim2;
   const size_t smem1 = rs_smem(S->pg, R16, S->stages).total, smem2 = RgSmem::total();

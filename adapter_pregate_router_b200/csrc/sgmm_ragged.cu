@@ -172,12 +172,13 @@ __device__ void rg_plan(const SgmmArgs& a, int R16, int* count, RgTile* tiles, i
 // a group of <= 4 projections whose R16-row slots add up to <= 256.  The contraction puts the
 // adapter rows on the MMA's M side and the tokens on N:
 //   D[j, n] = sum_k A_{q(j), e}[j mod R16, k] x_{t_n}[k]   (M = 128 per accumulator, N = round16(len))
-// so a short segment costs only its own tokens.  One producer warp issues, per 64-column stage,
-// TMA boxes of A_e (64 columns x R16 rows from a tensor map made for the item: the projection's
-// template for rank r_e with A_e's address, zeros past r_e) and tile::gather4 copies of the
-// tokens' x rows; one thread issues the MMAs; eight epilogue warps read D back (a TMEM lane per
-// adapter row), scale by each token's gate and store bf16.  Items come from a work counter (after
-// one static item per CTA), so CTAs drawing high-rank adapters take fewer of them.
+// so a short segment costs only its own tokens.  Per stage of 128 columns (two 64-column
+// sub-blocks), one warp issues TMA boxes of A_e (64 columns x R16 rows from a tensor map made for
+// the item: the projection's template for rank r_e with A_e's address, zeros past r_e) and four
+// loader warps copy the tokens' x rows with 16-byte cp.async; one thread issues the MMAs; eight
+// epilogue warps read D back (a TMEM lane per adapter row), scale by each token's gate and store
+// bf16.  Items come from a work counter (after one static item per CTA), so CTAs drawing
+// high-rank adapters take fewer of them.
 constexpr int RS_EPI = 256;                   // warps 2-9
 constexpr int RS_XW = 128;                    // warps 10-13: x rows by 16-byte cp.async
 constexpr int RS_BLOCK = 64 + RS_EPI + RS_XW; // warp 0: item setup and A boxes, warp 1: MMA issue

@@ -169,26 +169,31 @@ __device__ void rg_plan(const SgmmArgs& a, int R16, int* count, RgTile* tiles, i
 
 // v = g * A_e x for every pair, by plan position: [proj][position][R16] bf16 (rank rows past
 // r_e are zeros).  An item is one pair tile of adapter e (<= 128 consecutive plan positions) and
-// a group of <= 4 projections whose R16-row slots add up to <= 256.  The contraction puts the
-// adapter rows on the MMA's M side and the tokens on N:
-//   D[j, n] = sum_k A_{q(j), e}[j mod R16, k] x_{t_n}[k]   (M = 128 per accumulator, N = round16(len))
-// so a short segment costs only its own tokens.  Per stage of 128 columns (two 64-column
-// sub-blocks), one warp issues TMA boxes of A_e (64 columns x R16 rows from a tensor map made for
-// the item: the projection's template for rank r_e with A_e's address, zeros past r_e) and four
-// loader warps copy the tokens' x rows with 16-byte cp.async; one thread issues the MMAs; eight
-// epilogue warps read D back (a TMEM lane per adapter row), scale by each token's gate and store
-// bf16.  Items come from a work counter (after one static item per CTA), so CTAs drawing
-// high-rank adapters take fewer of them.
+// a group of <= 4 projections whose rank slots add up to <= 256.  The contraction puts the
+// adapter's rank rows on the MMA's M side and the tokens on N:
+//   D[j, n] = sum_k A_{q(j), e}[j mod w, k] x_{t_n}[k]   (w = round16(r_e), M = 128 per accumulator,
+//                                                        N = round16(len))
+// so a short segment costs only its own tokens.  A stage (64 KB) packs as many 64-column
+// sub-blocks as fit the item: each holds the item's N token rows and nq * w rank rows (128-byte
+// swizzled rows); an accumulator's MMAs read 128 rank rows, the rows past nq * w being whatever
+// follows (the products of those rows are never read), so a small item moves up to 8 sub-blocks
+// (512 columns) per stage instead of paying a fixed 128-row tile.  One warp issues TMA boxes of
+// A_e (64 columns x w rows from a tensor map made for the item: the projection's template for
+// rank r_e with A_e's address, zeros past r_e); four loader warps copy the tokens' x rows with
+// 16-byte cp.async; one thread issues the MMAs; eight epilogue warps read D back (a TMEM lane per
+// rank row), scale by each token's gate and store bf16.  Items come from a work counter (after
+// one static item per CTA), so CTAs drawing high-rank adapters take fewer of them.
 constexpr int RS_EPI = 256;                   // warps 2-9
 constexpr int RS_XW = 128;                    // warps 10-13: x rows by 16-byte cp.async
 constexpr int RS_BLOCK = 64 + RS_EPI + RS_XW; // warp 0: item setup and A boxes, warp 1: MMA issue
-constexpr int RS_XBYTES = 128 * 128;          // x rows of a sub-block (128 x 64 columns, 128-byte swizzle)
-constexpr int RS_SB = 2;                      // 64-column sub-blocks per stage: 256 contiguous bytes of each row
+constexpr int RS_STAGE = 64 * 1024;           // one stage
+constexpr int RS_PAD = 128 * 128;             // after the last stage: the rank rows an MMA may read past it
+constexpr int RS_MAXSB = 8;                   // 64-column sub-blocks per stage at most
 constexpr int RS_NQ = 4;                      // projections per item at most
 
 struct RsPlan {
-  CUtensorMap xmap;                               // x rows: 64-column boxes (gather4)
-  CUtensorMap atmpl[APR_MAX_PROJ][APR_MAX_RANK / 8];   // A_e of rank 8 (j + 1): [r, d_in], 64 x R16 boxes, swizzled
+  CUtensorMap xmap;                               // x rows (unused by the loads; kept for the shapes)
+  CUtensorMap atmpl[APR_MAX_PROJ][APR_MAX_RANK / 8];   // A_e of rank 8 (j + 1): [r, d_in], 64 x round16(r) boxes, swizzled
   CUtensorMap btmpl[APR_MAX_PROJ][APR_MAX_RANK / 8];   // B_e of rank 8 (j + 1): [d_out, r], 8 x 128 boxes, plain
   SgmmArgs a;
   int R16, pg, npg, stages, max_tiles;
@@ -196,20 +201,20 @@ struct RsPlan {
 };
 
 struct RsItem {
-  int e, q0, nq, start, len, pad[3];
+  int e, q0, nq, start, len;
+  int w;                                      // rank slot round16(r_e)
+  int nsb;                                    // 64-column sub-blocks per stage
+  int nst;                                    // stages
 };
 
 struct RsSmem {
-  int stage_bytes, abytes, S;                 // abytes: adapter rows of one sub-block
+  int S;
   size_t bar, item, gate, tok, mapbuf, tmem, total;
 };
-__host__ __device__ inline RsSmem rs_smem(int pg, int R16, int S) {
+__host__ __device__ inline RsSmem rs_smem(int S) {
   RsSmem L;
-  // the adapter rows of a stage: at least the 128 rows one accumulator's MMAs read
-  L.abytes = (pg * R16 < 128 ? 128 : pg * R16) * 128;
-  L.stage_bytes = RS_SB * (RS_XBYTES + L.abytes);
   L.S = S;
-  L.bar = (size_t)S * L.stage_bytes;
+  L.bar = (size_t)S * RS_STAGE + RS_PAD;
   L.item = L.bar + (size_t)(2 * S + 6) * 8;
   L.gate = L.item + 2 * sizeof(RsItem);
   L.tok = L.gate + 2 * 128 * 4;
@@ -226,7 +231,7 @@ __global__ void __launch_bounds__(RS_BLOCK, 1) rg_shrink_kernel(const __grid_con
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int S = P.stages, R16 = P.R16, pg = P.pg, T = a.T;
-  const RsSmem L = rs_smem(pg, R16, S);
+  const RsSmem L = rs_smem(S);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bar);
   const uint32_t bar_full = smem_u32(bars), bar_empty = smem_u32(bars + S);
   const uint32_t bar_ifull = smem_u32(bars + 2 * S), bar_iempty = smem_u32(bars + 2 * S + 2);
@@ -263,11 +268,18 @@ __global__ void __launch_bounds__(RS_BLOCK, 1) rg_shrink_kernel(const __grid_con
   WsHeader* hdr = reinterpret_cast<WsHeader*>(a.ws);
   const PairTile* qtiles = ws_at<PairTile>(a.ws, W.qtiles);
   const long nitems = (long)hdr->n_qtiles * P.npg;
-  const int nblk = a.d_in / 64, nk = (nblk + RS_SB - 1) / RS_SB;   // 64-column blocks; stages
+  const int nblk = a.d_in / 64;                  // 64-column blocks of d_in
   bool abort = false;
+  // stage layout of an item: x sub-blocks (N rows each), then rank sub-blocks (nq * w rows each)
+  auto xsub = [&](const RsItem& it, uint32_t st, int b) -> uint32_t {
+    return st + (uint32_t)(b * ((it.len + 15) / 16 * 16)) * 128;
+  };
+  auto asub = [&](const RsItem& it, uint32_t st, int b) -> uint32_t {
+    return st + (uint32_t)(it.nsb * ((it.len + 15) / 16 * 16)) * 128 + (uint32_t)(b * it.nq * it.w) * 128;
+  };
 
   if (warp == 0) {
-    // ---------------------------------------------------------------- producer warp
+    // ---------------------------------------------------------------- setup and A boxes
     // the expand's B tensor maps of this CTA's share of the (projection, adapter) pairs in use
     CUtensorMap* bmaps = ws_at<CUtensorMap>(a.ws, P.bmaps_off);
     for (int pe = blockIdx.x; pe < a.nproj * a.E; pe += gridDim.x) {
@@ -276,8 +288,6 @@ __global__ void __launch_bounds__(RS_BLOCK, 1) rg_shrink_kernel(const __grid_con
         tmap_build(bmaps + pe, s_mapbuf + RS_NQ * 128, &P.btmpl[p][a.ranks[e] / 8 - 1], a.proj[p].B[e]);
     }
     CUtensorMap* amaps = ws_at<CUtensorMap>(a.ws, P.amaps_off) + (size_t)blockIdx.x * kRgMaxStages * RS_NQ;
-    const __nv_bfloat16* x = reinterpret_cast<const __nv_bfloat16*>(a.x);
-    (void)x;
     uint32_t g = 0, k = 0;
     long item = blockIdx.x;
     while (!abort) {
@@ -315,15 +325,21 @@ __global__ void __launch_bounds__(RS_BLOCK, 1) rg_shrink_kernel(const __grid_con
         s_tok[slot * 128 + row] = q;                   // top-1: the pair id is the token
         s_g[slot * 128 + row] = row < len ? a.gate[q] : 0.f;
       }
-      if (lane == 0) {
-        RsItem it;
-        it.e = e;
-        it.q0 = q0;
-        it.nq = nq;
-        it.start = tile.start;
-        it.len = len;
-        s_item[slot] = it;
-      }
+      // sub-blocks per stage: the item's rows, plus the rank rows its last MMA reads past them
+      const int w = (r + 15) / 16 * 16, N = (len + 15) / 16 * 16, arows = nq * w;
+      const int slack = ((arows + 127) / 128) * 128 - arows;
+      int nsb = (RS_STAGE - slack * 128) / ((N + arows) * 128);
+      nsb = max(1, min(nsb, min(RS_MAXSB, nblk)));
+      RsItem it;
+      it.e = e;
+      it.q0 = q0;
+      it.nq = nq;
+      it.start = tile.start;
+      it.len = len;
+      it.w = w;
+      it.nsb = nsb;
+      it.nst = (nblk + nsb - 1) / nsb;
+      if (lane == 0) s_item[slot] = it;
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_ifull + 8 * slot);
       // the item's first stage is free before its A maps are rewritten: the ring slot k % S was last
@@ -340,23 +356,21 @@ __global__ void __launch_bounds__(RS_BLOCK, 1) rg_shrink_kernel(const __grid_con
         tmap_build(am + qi, s_mapbuf + qi * 128, &P.atmpl[q0 + qi][r / 8 - 1], a.proj[q0 + qi].A[e]);
         if (lane == 0) tmap_acquire(am + qi);
       }
-      const uint32_t sb_bytes = (uint32_t)(nq * R16 * 128);   // A boxes of one sub-block
-      for (int c = 0; c < nk; ++c, ++g) {
+      for (int c = 0; c < it.nst; ++c, ++g) {
         const uint32_t s = g % S;
         if (c > 0 && g >= (uint32_t)S && !__all_sync(0xffffffffu, mbar_wait(bar_empty + 8 * s, ((g / S) - 1) & 1))) {
           abort = true;
           break;
         }
-        const int nsb = min(RS_SB, nblk - RS_SB * c);
-        const uint32_t xs = sbase + s * (uint32_t)L.stage_bytes, as = xs + RS_SB * RS_XBYTES;
-        if (lane == 0) mbar_arrive_expect_tx(bar_full + 8 * s, (uint32_t)nsb * sb_bytes);
-        __syncwarp();
-        for (int b = 0; b < nsb; ++b) {
-          const int col = 64 * (RS_SB * c + b);
-          if (lane == 0)
+        const int nb = min(nsb, nblk - c * nsb);
+        const uint32_t st = sbase + s * (uint32_t)RS_STAGE;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(bar_full + 8 * s, (uint32_t)(nb * arows * 128));
+          for (int b = 0; b < nb; ++b)
             for (int qi = 0; qi < nq; ++qi)
-              tma_load_2d(as + (uint32_t)b * L.abytes + (uint32_t)(qi * R16) * 128, am + qi, col, 0, bar_full + 8 * s);
+              tma_load_2d(asub(it, st, b) + (uint32_t)(qi * w) * 128, am + qi, 64 * (c * nsb + b), 0, bar_full + 8 * s);
         }
+        __syncwarp();
       }
       ++k;
       item = next;
@@ -374,23 +388,22 @@ __global__ void __launch_bounds__(RS_BLOCK, 1) rg_shrink_kernel(const __grid_con
         const RsItem it = s_item[slot];
         mbar_arrive(bar_iempty + 8 * slot);
         if (it.e < 0) break;
-        const int N = (it.len + 15) / 16 * 16, nacc = (it.nq * R16 + 127) / 128;
+        const int N = (it.len + 15) / 16 * 16, nacc = (it.nq * it.w + 127) / 128;
         const uint32_t id = idesc_bf16(128, N);
         if (k >= 1 && !mbar_wait(bar_dempty, (k - 1) & 1)) { abort = true; break; }
         tc_fence_after();
-        for (int c = 0; c < nk; ++c, ++g) {
+        for (int c = 0; c < it.nst; ++c, ++g) {
           const uint32_t s = g % S;
           if (!mbar_wait(bar_full + 8 * s, (g / S) & 1)) { abort = true; break; }
           tc_fence_after();
-          const int nsb = min(RS_SB, nblk - RS_SB * c);
-          const uint32_t xs = sbase + s * (uint32_t)L.stage_bytes, as = xs + RS_SB * RS_XBYTES;
-          for (int b = 0; b < nsb; ++b)
+          const int nb = min(it.nsb, nblk - c * it.nsb);
+          const uint32_t st = sbase + s * (uint32_t)RS_STAGE;
+          for (int b = 0; b < nb; ++b)
             for (int m = 0; m < nacc; ++m)
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk)
-                mma_bf16(tmem + (uint32_t)m * 128,
-                         desc_k_sw128(as + (uint32_t)b * L.abytes + (uint32_t)m * (128 * 128) + kk * 32),
-                         desc_k_sw128(xs + (uint32_t)b * RS_XBYTES + kk * 32), id, (c > 0 || b > 0 || kk > 0) ? 1u : 0u);
+                mma_bf16(tmem + (uint32_t)m * 128, desc_k_sw128(asub(it, st, b) + (uint32_t)m * (128 * 128) + kk * 32),
+                         desc_k_sw128(xsub(it, st, b) + kk * 32), id, (c > 0 || b > 0 || kk > 0) ? 1u : 0u);
           mma_commit(bar_empty + 8 * s);
         }
         if (abort) break;
@@ -400,10 +413,10 @@ __global__ void __launch_bounds__(RS_BLOCK, 1) rg_shrink_kernel(const __grid_con
     }
   } else if (warp >= 2 + RS_EPI / 32) {
     // ---------------------------------------------------------------- x loaders
-    // thread xt copies 16-byte pieces of the item's token rows: 16 pieces (two 64-column
-    // sub-blocks x 8) per row on consecutive threads, rows r0, r0 + 8, ... into 128-byte swizzled rows
+    // per sub-block, thread xt copies 16-byte piece (xt & 7) of token rows (xt >> 3) + 16 m: 8
+    // consecutive threads per 128-byte row piece, into the 128-byte swizzled rows
     const int xt = tid - (64 + RS_EPI);
-    const int q = xt & 15, sub = q >> 3, chunk = q & 7, r0 = xt >> 4;
+    const int chunk = xt & 7, r0 = xt >> 3;
     const __nv_bfloat16* x = reinterpret_cast<const __nv_bfloat16*>(a.x);
     uint32_t g = 0, k = 0;
     while (true) {
@@ -411,27 +424,28 @@ __global__ void __launch_bounds__(RS_BLOCK, 1) rg_shrink_kernel(const __grid_con
       if (!__all_sync(0xffffffffu, mbar_wait(bar_ifull + 8 * slot, (k >> 1) & 1))) { abort = true; break; }
       const RsItem it = s_item[slot];
       if (it.e < 0) break;
-      int tok[16];
+      int tok[8];
 #pragma unroll
-      for (int m = 0; m < 16; ++m) {
-        const int r = r0 + 8 * m;
+      for (int m = 0; m < 8; ++m) {
+        const int r = r0 + 16 * m;
         tok[m] = r < it.len ? s_tok[slot * 128 + r] : -1;
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_iempty + 8 * slot);   // the item's tokens are in registers
-      for (int c = 0; c < nk; ++c, ++g) {
+      for (int c = 0; c < it.nst; ++c, ++g) {
         const uint32_t s = g % S;
         if (g >= (uint32_t)S && !__all_sync(0xffffffffu, mbar_wait(bar_empty + 8 * s, ((g / S) - 1) & 1))) {
           abort = true;
           break;
         }
-        const int nsb = min(RS_SB, nblk - RS_SB * c);
-        if (sub < nsb) {
-          const uint32_t xs = sbase + s * (uint32_t)L.stage_bytes + (uint32_t)sub * RS_XBYTES;
-          const __nv_bfloat16* src = x + 64 * (RS_SB * c + sub) + chunk * 8;
+        const int nb = min(it.nsb, nblk - c * it.nsb);
+        const uint32_t st = sbase + s * (uint32_t)RS_STAGE;
+        for (int b = 0; b < nb; ++b) {
+          const uint32_t xs = xsub(it, st, b);
+          const __nv_bfloat16* src = x + 64 * (c * it.nsb + b) + chunk * 8;
 #pragma unroll
-          for (int m = 0; m < 16; ++m) {
-            const int r = r0 + 8 * m;
+          for (int m = 0; m < 8; ++m) {
+            const int r = r0 + 16 * m;
             if (tok[m] >= 0)
               asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(xs + (uint32_t)r * 128 + (uint32_t)((chunk ^ (r & 7)) << 4)),
                            "l"(src + (size_t)tok[m] * a.d_in)
@@ -457,18 +471,14 @@ __global__ void __launch_bounds__(RS_BLOCK, 1) rg_shrink_kernel(const __grid_con
       const int slot = k & 1;
       if (!__all_sync(0xffffffffu, mbar_wait(bar_ifull + 8 * slot, (k >> 1) & 1))) { abort = true; break; }
       const RsItem it = s_item[slot];
-      if (it.e < 0) {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_iempty + 8 * slot);
-        break;
-      }
+      if (it.e < 0) break;
       if (!__all_sync(0xffffffffu, mbar_wait(bar_dfull, k & 1))) { abort = true; break; }
       tc_fence_after();
-      const int N = (it.len + 15) / 16 * 16, nacc = (it.nq * R16 + 127) / 128;
+      const int N = (it.len + 15) / 16 * 16, nacc = (it.nq * it.w + 127) / 128;
       // two accumulators: warps 2-5 read the first, 6-9 the second; one: they split the columns
       const int m = nacc == 2 ? (ew >> 2) : 0, csel = nacc == 2 ? -1 : (ew >> 2);
-      const int j = 128 * m + 32 * quarter + lane;       // adapter row of this TMEM lane
-      const int qi = j / R16, rr = j - qi * R16;
+      const int j = 128 * m + 32 * quarter + lane;       // rank row of this TMEM lane
+      const int qi = j / it.w, rr = j - qi * it.w;
       const bool valid = qi < it.nq;
       __nv_bfloat16* dst = vc + ((size_t)(it.q0 + qi) * T + it.start) * R16 + rr;
       const float* gg = s_g + slot * 128;
@@ -921,7 +931,7 @@ cudaError_t launch_sgmm_ragged(const SgmmArgs& a, size_t scratch_off, cudaStream
   S->pg = 256 / R16 < a.nproj ? 256 / R16 : a.nproj;
   if (S->pg > RS_NQ) S->pg = RS_NQ;
   S->npg = (a.nproj + S->pg - 1) / S->pg;
-  S->stages = (int)((200 * 1024) / rs_smem(S->pg, R16, 1).stage_bytes);
+  S->stages = 3;
   if (S->stages > kRgMaxStages) S->stages = kRgMaxStages;
   S->max_tiles = rg_max_tiles(a.T, a.E);
   S->vc_off = scratch_off;
@@ -931,7 +941,8 @@ cudaError_t launch_sgmm_ragged(const SgmmArgs& a, size_t scratch_off, cudaStream
   if ((err = encode_row_map(&S->xmap, const_cast<void*>(a.x), a.T, a.d_in)) != cudaSuccess) return err;
   for (int p = 0; p < a.nproj; ++p)
     for (int r = 8; r <= R16; r += 8) {
-      if ((err = cached_box_map(&S->atmpl[p][r / 8 - 1], a.x, r, a.d_in, (long)a.d_in * 2, 64, R16, true)) != cudaSuccess)
+      if ((err = cached_box_map(&S->atmpl[p][r / 8 - 1], a.x, r, a.d_in, (long)a.d_in * 2, 64, round16i(r), true)) !=
+          cudaSuccess)
         return err;
       if ((err = cached_box_map(&S->btmpl[p][r / 8 - 1], a.x, a.proj[p].d_out, r, (long)r * 2, 8, RG_NT, false)) !=
           cudaSuccess)
@@ -951,7 +962,7 @@ cudaError_t launch_sgmm_ragged(const SgmmArgs& a, size_t scratch_off, cudaStream
     P.cb_before[p + 1] = P.cb_before[p] + (a.proj[p].d_out + RG_NT - 1) / RG_NT;
   }
   static SmemLimit lim1, lim2;
-  const size_t smem1 = rs_smem(S->pg, R16, S->stages).total, smem2 = RgSmem::total();
+  const size_t smem1 = rs_smem(S->stages).total, smem2 = RgSmem::total();
   if ((err = lim1.ensure((const void*)rg_shrink_kernel, smem1)) != cudaSuccess) return err;
   if ((err = lim2.ensure((const void*)ragged_expand_kernel, smem2)) != cudaSuccess) return err;
   const long items = (long)max_qtiles(a.T, a.k, a.E) * S->npg;

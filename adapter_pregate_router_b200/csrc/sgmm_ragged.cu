@@ -185,7 +185,7 @@ __device__ void rg_plan(const SgmmArgs& a, int R16, int* count, RgTile* tiles, i
 // one static item per CTA), so CTAs drawing high-rank adapters take fewer of them.
 constexpr int RS_EPI = 256;                   // warps 2-9
 constexpr int RS_XW = 128;                    // warps 10-13: x rows by 16-byte cp.async
-constexpr int RS_BLOCK = 64 + RS_EPI + RS_XW; // warp 0: item setup and A boxes, warp 1: MMA issue
+constexpr int RS_BLOCK = 64 + RS_EPI + RS_XW + 32;   // warp 0: item setup, warp 1: MMA issue, warp 14: A boxes
 constexpr int RS_STAGE = 64 * 1024;           // one stage
 constexpr int RS_PAD = 128 * 128;             // after the last stage: the rank rows an MMA may read past it
 constexpr int RS_MAXSB = 8;                   // 64-column sub-blocks per stage at most
@@ -249,7 +249,7 @@ __global__ void __launch_bounds__(RS_BLOCK, 1) rg_shrink_kernel(const __grid_con
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar_ifull + 8 * i, 1);
-      mbar_init(bar_iempty + 8 * i, 1 + RS_EPI / 32 + RS_XW / 32);
+      mbar_init(bar_iempty + 8 * i, 2 + RS_EPI / 32 + RS_XW / 32);   // A warp, MMA thread, epilogue and loader warps
     }
     mbar_init(bar_dfull, 1);
     mbar_init(bar_dempty, RS_EPI);
@@ -288,7 +288,7 @@ __global__ void __launch_bounds__(RS_BLOCK, 1) rg_shrink_kernel(const __grid_con
         tmap_build(bmaps + pe, s_mapbuf + RS_NQ * 128, &P.btmpl[p][a.ranks[e] / 8 - 1], a.proj[p].B[e]);
     }
     CUtensorMap* amaps = ws_at<CUtensorMap>(a.ws, P.amaps_off) + (size_t)blockIdx.x * kRgMaxStages * RS_NQ;
-    uint32_t g = 0, k = 0;
+    uint32_t k = 0;
     long item = blockIdx.x;
     while (!abort) {
       const int slot = k & 1;
@@ -339,41 +339,49 @@ __global__ void __launch_bounds__(RS_BLOCK, 1) rg_shrink_kernel(const __grid_con
       it.w = w;
       it.nsb = nsb;
       it.nst = (nblk + nsb - 1) / nsb;
+      // the item's A maps go to map slot `slot`: free, since every copy of item k - 2 has landed
+      CUtensorMap* am = amaps + (size_t)slot * RS_NQ;
+      for (int qi = 0; qi < nq; ++qi)
+        tmap_build(am + qi, s_mapbuf + qi * 128, &P.atmpl[q0 + qi][r / 8 - 1], a.proj[q0 + qi].A[e]);
       if (lane == 0) s_item[slot] = it;
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_ifull + 8 * slot);
-      // the item's first stage is free before its A maps are rewritten: the ring slot k % S was last
-      // used by item k - S, whose copies all precede that stage's previous use
-      {
-        const uint32_t s0 = g % S;
-        if (g >= (uint32_t)S && !__all_sync(0xffffffffu, mbar_wait(bar_empty + 8 * s0, ((g / S) - 1) & 1))) {
-          abort = true;
-          break;
-        }
-      }
-      CUtensorMap* am = amaps + (size_t)(k % S) * RS_NQ;
-      for (int qi = 0; qi < nq; ++qi) {
-        tmap_build(am + qi, s_mapbuf + qi * 128, &P.atmpl[q0 + qi][r / 8 - 1], a.proj[q0 + qi].A[e]);
-        if (lane == 0) tmap_acquire(am + qi);
-      }
+      ++k;
+      item = next;
+    }
+  } else if (warp == 2 + RS_EPI / 32 + RS_XW / 32) {
+    // ---------------------------------------------------------------- A boxes
+    const CUtensorMap* amaps = ws_at<const CUtensorMap>(a.ws, P.amaps_off) + (size_t)blockIdx.x * kRgMaxStages * RS_NQ;
+    uint32_t g = 0, k = 0;
+    while (true) {
+      const int slot = k & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_ifull + 8 * slot, (k >> 1) & 1))) { abort = true; break; }
+      const RsItem it = s_item[slot];
+      if (it.e < 0) break;
+      const CUtensorMap* am = amaps + (size_t)slot * RS_NQ;
+      if (lane == 0)
+        for (int qi = 0; qi < it.nq; ++qi) tmap_acquire(am + qi);
+      const int arows = it.nq * it.w;
       for (int c = 0; c < it.nst; ++c, ++g) {
         const uint32_t s = g % S;
-        if (c > 0 && g >= (uint32_t)S && !__all_sync(0xffffffffu, mbar_wait(bar_empty + 8 * s, ((g / S) - 1) & 1))) {
+        if (g >= (uint32_t)S && !__all_sync(0xffffffffu, mbar_wait(bar_empty + 8 * s, ((g / S) - 1) & 1))) {
           abort = true;
           break;
         }
-        const int nb = min(nsb, nblk - c * nsb);
+        const int nb = min(it.nsb, nblk - c * it.nsb);
         const uint32_t st = sbase + s * (uint32_t)RS_STAGE;
         if (lane == 0) {
           mbar_arrive_expect_tx(bar_full + 8 * s, (uint32_t)(nb * arows * 128));
           for (int b = 0; b < nb; ++b)
-            for (int qi = 0; qi < nq; ++qi)
-              tma_load_2d(asub(it, st, b) + (uint32_t)(qi * w) * 128, am + qi, 64 * (c * nsb + b), 0, bar_full + 8 * s);
+            for (int qi = 0; qi < it.nq; ++qi)
+              tma_load_2d(asub(it, st, b) + (uint32_t)(qi * it.w) * 128, am + qi, 64 * (c * it.nsb + b), 0,
+                          bar_full + 8 * s);
         }
         __syncwarp();
       }
+      if (abort) break;
+      if (lane == 0) mbar_arrive(bar_iempty + 8 * slot);
       ++k;
-      item = next;
     }
     // after an abort, the copies of the last stages land before the CTA exits (bounded)
     if (abort && lane == 0)
@@ -386,7 +394,6 @@ __global__ void __launch_bounds__(RS_BLOCK, 1) rg_shrink_kernel(const __grid_con
         const int slot = k & 1;
         if (!mbar_wait(bar_ifull + 8 * slot, (k >> 1) & 1)) { abort = true; break; }
         const RsItem it = s_item[slot];
-        mbar_arrive(bar_iempty + 8 * slot);
         if (it.e < 0) break;
         const int N = (it.len + 15) / 16 * 16, nacc = (it.nq * it.w + 127) / 128;
         const uint32_t id = idesc_bf16(128, N);
@@ -408,6 +415,7 @@ __global__ void __launch_bounds__(RS_BLOCK, 1) rg_shrink_kernel(const __grid_con
         }
         if (abort) break;
         mma_commit(bar_dfull);
+        mbar_arrive(bar_iempty + 8 * slot);            // every copy of the item has landed: its maps are free
         ++k;
       }
     }

@@ -109,12 +109,18 @@ inline bool dense_dims_ok(int T, int E, int max_rank, int d_in = 0) {
 
 // Tensor-core path: gated v rows [projection][pair position][2 * R16] bf16
 // (hi | lo); k <= 2, k * R16 <= 64.
+// After the rows, each shrink CTA's A tensor maps ([CTA][projection], <= 256 CTAs).
 constexpr int kTensorMaxK2 = 64;
+constexpr int kShrinkMaxCtas = 256;
+constexpr size_t kShrinkMapBytes = (size_t)kShrinkMaxCtas * APR_MAX_PROJ * 128;
+inline size_t tc_vc_bytes(int T, int k, int max_rank) {
+  return align_up((size_t)APR_MAX_PROJ * T * k * 4 * round16i(max_rank));
+}
 inline size_t tc_scratch_bytes(int T, int k, int max_rank) {
   if (k < 1 || k > 2) return 0;
   const int R16 = round16i(max_rank);
   if (k * R16 > kTensorMaxK2) return 0;
-  return (size_t)APR_MAX_PROJ * T * k * 4 * R16;
+  return tc_vc_bytes(T, k, max_rank) + kShrinkMapBytes;
 }
 
 // Bank path (token order over the whole adapter bank): gated v per pair
@@ -122,11 +128,14 @@ inline size_t tc_scratch_bytes(int T, int k, int max_rank) {
 // E * R16 <= 256.
 constexpr int kBankMaxKR = 64;
 constexpr int kBankMaxRows = 256;
+inline size_t bank_vc_bytes(int T, int k, int max_rank) {
+  return align_up((size_t)APR_MAX_PROJ * T * k * round16i(max_rank) * 2);
+}
 inline size_t bank_scratch_bytes(int T, int k, int E, int max_rank) {
   const int R16 = round16i(max_rank);
   if (R16 != 16 && R16 != 32 && R16 != 64) return 0;
   if (k < 1 || k > 4 || k * R16 > kBankMaxKR || E * R16 > kBankMaxRows) return 0;
-  return (size_t)APR_MAX_PROJ * T * k * R16 * 2;
+  return bank_vc_bytes(T, k, max_rank) + kShrinkMapBytes;
 }
 
 // Many-tenant path (top-1 routing): ragged tiles of <= kSetTile consecutive plan tokens whose

@@ -4,6 +4,9 @@
 #include <mutex>
 #include <vector>
 
+#include <map>
+#include <tuple>
+
 #include "apr_internal.cuh"
 #include "tc_ptx.cuh"
 
@@ -763,6 +766,25 @@ cudaError_t encode_box_map(CUtensorMap* m, const void* base, long rows, long col
              CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS
              ? cudaSuccess
              : cudaErrorInvalidValue;
+}
+
+// Tensor-map templates depend only on shapes, so they are encoded once per shape (the address is
+// a placeholder the kernels replace on the device).
+cudaError_t cached_box_map(CUtensorMap* m, const void* placeholder, long rows, long cols, long pitch_bytes,
+                           int box_cols, int box_rows, bool swizzle128) {
+  using Key = std::tuple<long, long, long, int, int, int>;
+  static std::mutex mu;
+  static std::map<Key, CUtensorMap> cache;
+  const Key key{rows, cols, pitch_bytes, box_cols, box_rows, swizzle128 ? 1 : 0};
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = cache.find(key);
+  if (it != cache.end()) {
+    *m = it->second;
+    return cudaSuccess;
+  }
+  cudaError_t err = encode_box_map(m, placeholder, rows, cols, pitch_bytes, box_cols, box_rows, swizzle128);
+  if (err == cudaSuccess) cache.emplace(key, *m);
+  return err;
 }
 
 size_t merge_plan_bytes(int nproj) { return (size_t)nproj * 2 * sizeof(CUtensorMap); }

@@ -47,10 +47,7 @@
 // wait is bounded (1 s) and its outcome is made the same for all lanes of a warp
 // (no warp can be left at a barrier its other lanes abandoned); on expiry the CTA
 // records APR_ERR_TIMEOUT, drains its copies and frees its tensor memory.
-#include <map>
 #include <memory>
-#include <mutex>
-#include <tuple>
 
 #include "apr_internal.cuh"
 #include "tc_ptx.cuh"
@@ -906,25 +903,6 @@ __global__ void __launch_bounds__(RG_BLOCK, 1) ragged_expand_kernel(const __grid
 
 bool sgmm_ragged_supported(const SgmmArgs& a, int dtype) {
   return dtype == APR_BF16 && rg_dims_ok(a.k, a.max_rank) && a.d_in % 64 == 0;
-}
-
-// Tensor-map templates depend only on shapes, so they are encoded once per shape (the address is
-// a placeholder the kernels replace).
-static cudaError_t cached_box_map(CUtensorMap* m, const void* placeholder, long rows, long cols, long pitch, int box_cols,
-                                  int box_rows, bool sw) {
-  using Key = std::tuple<long, long, long, int, int, int>;
-  static std::mutex mu;
-  static std::map<Key, CUtensorMap> cache;
-  const Key key{rows, cols, pitch, box_cols, box_rows, sw ? 1 : 0};
-  std::lock_guard<std::mutex> lock(mu);
-  auto it = cache.find(key);
-  if (it != cache.end()) {
-    *m = it->second;
-    return cudaSuccess;
-  }
-  cudaError_t err = encode_box_map(m, placeholder, rows, cols, pitch, box_cols, box_rows, sw);
-  if (err == cudaSuccess) cache.emplace(key, *m);
-  return err;
 }
 
 cudaError_t launch_sgmm_ragged(const SgmmArgs& a, size_t scratch_off, cudaStream_t s) {

@@ -36,6 +36,8 @@
 //
 // Every mbarrier wait is bounded by the global timer (1 s); on expiry the CTA
 // records APR_ERR_TIMEOUT, drains its copies and frees its TMEM.
+#include <memory>
+
 #include "apr_internal.cuh"
 #include "tc_ptx.cuh"
 
@@ -56,6 +58,7 @@ constexpr int SMEM_BUDGET = 200 * 1024;
 
 struct TcPlan {
   CUtensorMap ymap[APR_MAX_PROJ];    // expand: y of each projection as rows for tile::scatter4 stores
+  CUtensorMap atmpl[APR_MAX_PROJ][APR_MAX_RANK / 8];   // shrink: A_e of rank 8 (j + 1), [r, d_in], 64 x R16 boxes
   SgmmArgs a;
   int R16;                           // rank slot per adapter
   int K2;                            // k * R16
@@ -68,6 +71,7 @@ struct TcPlan {
   int vpair;                         // shrink writes v by pair id, bf16 only ([proj][q][R16]) instead of
                                      // by plan position as bf16 hi | lo ([proj][pair position][2 * R16])
   size_t vprep_off;                  // scratch: V rows
+  size_t amaps_off;                  // scratch: each shrink CTA's A tensor maps [CTA][projection]
   int cc_before[APR_MAX_PROJ + 1];   // expand: prefix of 1024-column items per projection
 };
 
@@ -77,7 +81,7 @@ static_assert(TB_MAXK2 == kTensorMaxK2, "tensor scratch sizing");
 
 struct ShSmem {
   int stage_bytes, stages;
-  size_t bar, meta, total;
+  size_t bar, meta, mapbuf, total;
 };
 __host__ __device__ inline ShSmem sh_smem(int n1max, int stages) {
   ShSmem L;
@@ -85,7 +89,8 @@ __host__ __device__ inline ShSmem sh_smem(int n1max, int stages) {
   L.stages = stages;
   L.bar = (size_t)stages * L.stage_bytes;
   L.meta = L.bar + (size_t)(2 * stages + 1) * 8;
-  L.total = L.meta + 3 * TB_M * 4 + 16 + TB_MAXN1 * 8 + 1024;
+  L.mapbuf = (L.meta + 3 * TB_M * 4 + 16 + TB_MAXN1 * 8 + 127) / 128 * 128;
+  L.total = L.mapbuf + APR_MAX_PROJ * 128 + 1024;
   return L;
 }
 
@@ -103,13 +108,12 @@ __global__ void __launch_bounds__(SH_BLOCK, 1) tc_shrink_kernel(const __grid_con
   int* s_tok = reinterpret_cast<int*>(smem + L.meta);
   float* s_g = reinterpret_cast<float*>(s_tok + TB_M);
   volatile int* s_flags = reinterpret_cast<volatile int*>(s_g + TB_M);      // [0] tmem [1] bad
-  const __nv_bfloat16** s_arow = reinterpret_cast<const __nv_bfloat16**>(smem + L.meta + 2 * TB_M * 4 + 16);
   int* s_pair = reinterpret_cast<int*>(smem + L.meta + 2 * TB_M * 4 + 16 + TB_MAXN1 * 8);
   const uint32_t sbase = smem_u32(smem);
 
   if (tid == 0) {
     for (int i = 0; i < S; ++i) {
-      mbar_init(bar_full + 8 * i, SH_WORKERS);
+      mbar_init(bar_full + 8 * i, SH_WORKERS + 1);   // the x copies of every worker, the A boxes' bytes
       mbar_init(bar_empty + 8 * i, 1);
     }
     mbar_init(bar_d1, 1);
@@ -159,7 +163,11 @@ __global__ void __launch_bounds__(SH_BLOCK, 1) tc_shrink_kernel(const __grid_con
       s_g[tid] = g;
       if (tid == 0) {
         const int r = (e >= 0 && e < a.E) ? a.ranks[e] : 0;
-        const bool bad = r < 8 || r > R16 || (r & 7);
+        bool bad = r < 8 || r > R16 || (r & 7);
+        for (int qi = 0; qi < nq && !bad; ++qi) {
+          const void* A = a.proj[q0 + qi].A[e];
+          bad = !A || (reinterpret_cast<uintptr_t>(A) & 15);
+        }
         s_flags[1] = bad ? 1 : 0;
         if (bad) report(a.ws, APR_ERR_DEVICE_INDEX, K_TC, e);
       }
@@ -171,20 +179,21 @@ __global__ void __launch_bounds__(SH_BLOCK, 1) tc_shrink_kernel(const __grid_con
       item = s_flags[2];
       continue;
     }
-    // source row of every A row of the item (null: a zero row)
-    if (worker) {
+    // the item's A tensor maps (one per projection: the template for rank r_e with A_e's address;
+    // rows past r_e are zeros by the map's bounds).  This CTA's maps are rewritten only after the
+    // previous item's copies have all landed (its epilogue waited for the MMAs).
+    CUtensorMap* am = ws_at<CUtensorMap>(a.ws, P.amaps_off) + (size_t)blockIdx.x * APR_MAX_PROJ;
+    if (warp == 0) {
       const int re = a.ranks[e];
-      for (int j = tid; j < N1; j += SH_WORKERS) {
-        const int qi = j / R16, rr = j - qi * R16;
-        s_arow[j] = rr < re ? reinterpret_cast<const __nv_bfloat16*>(a.proj[q0 + qi].A[e]) + (size_t)rr * d_in : nullptr;
-      }
-      asm volatile("bar.sync 1, %0;" ::"n"(SH_WORKERS) : "memory");
+      for (int qi = 0; qi < nq; ++qi)
+        tmap_build(am + qi, sbase + (uint32_t)L.mapbuf + qi * 128, &P.atmpl[q0 + qi][re / 8 - 1], a.proj[q0 + qi].A[e]);
+      if (lane == 0)
+        for (int qi = 0; qi < nq; ++qi) tmap_acquire(am + qi);
     }
     const uint32_t g0 = gchunk;
     if (worker) {
       // this thread's copies of every stage of the item, fixed across the stages: four 16-byte
-      // pieces of x rows and up to eight of A rows (source advanced by 64 columns per stage; a
-      // null source is a zero piece: a missing pair or a row past the rank)
+      // pieces of x rows (source advanced by 64 columns per stage; a null source is a missing pair)
       const __nv_bfloat16* xs[TB_M * 8 / SH_WORKERS];
       uint32_t xo[TB_M * 8 / SH_WORKERS];
 #pragma unroll
@@ -195,38 +204,22 @@ __global__ void __launch_bounds__(SH_BLOCK, 1) tc_shrink_kernel(const __grid_con
         xs[m] = tk >= 0 ? x + (size_t)tk * d_in + q * 8 : nullptr;
         xo[m] = (uint32_t)row * 128 + (uint32_t)((q ^ (row & 7)) << 4);
       }
-      constexpr int AMAX = TB_MAXN1 * 8 / SH_WORKERS;
-      const __nv_bfloat16* as[AMAX];
-      uint32_t ao[AMAX];
-#pragma unroll
-      for (int m = 0; m < AMAX; ++m) {
-        const int w = tid + m * SH_WORKERS;
-        const int j = w >> 3, q = w & 7;
-        as[m] = (w < N1 * 8 && s_arow[j]) ? s_arow[j] + q * 8 : nullptr;
-        ao[m] = w < N1 * 8 ? TB_M * 128 + (uint32_t)j * 128 + (uint32_t)((q ^ (j & 7)) << 4) : 0xFFFFFFFFu;
-      }
       for (int c = 0; c < nk && !abort; ++c) {
         const uint32_t g = g0 + c, s = g % S;
         if (g >= (uint32_t)S && !mbar_wait(bar_empty + 8 * s, ((g / S) - 1) & 1)) { abort = true; break; }
         const uint32_t st_base = sbase + s * L.stage_bytes;
         const size_t col = (size_t)c * TB_BK;
+        // A rows: one box of 64 columns x R16 rows per projection, issued by thread 0
+        if (tid == 0) {
+          mbar_arrive_expect_tx(bar_full + 8 * s, (uint32_t)(N1 * 128));
+          for (int qi = 0; qi < nq; ++qi)
+            tma_load_2d(st_base + TB_M * 128 + (uint32_t)(qi * R16) * 128, am + qi, (int)col, 0, bar_full + 8 * s);
+        }
 #pragma unroll
         for (int m = 0; m < TB_M * 8 / SH_WORKERS; ++m)
           if (xs[m])
             asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(st_base + xo[m]), "l"(xs[m] + col)
                          : "memory");
-        // A rows: real rows by cp.async; rows past a rank are zeros, written with plain stores
-        // on the stage's first use in this item (no later copy touches them)
-#pragma unroll
-        for (int m = 0; m < AMAX; ++m) {
-          if (ao[m] == 0xFFFFFFFFu) continue;
-          if (as[m])
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(st_base + ao[m]), "l"(as[m] + col)
-                         : "memory");
-          else if (c < S)
-            st_shared_zero16(st_base + ao[m]);
-        }
-        if (c < S) fence_proxy_async();
         cp_async_arrive(bar_full + 8 * s);
       }
       // gate -> V rows (bf16 hi | lo) at the pair's plan position
@@ -668,10 +661,17 @@ bool sgmm_tensor_supported(const SgmmArgs& a, int dtype) {
   return true;
 }
 
-// Shrink plan fields shared by both expands: projections per item, pipeline depth.
-static void shrink_plan(TcPlan& t, const SgmmArgs& a, size_t v_off, int vpair) {
+// Shrink plan fields shared by both expands: projections per item, pipeline depth, the A
+// tensor-map templates (one per projection and rank) and where each CTA writes its maps.
+static cudaError_t shrink_plan(TcPlan& t, const SgmmArgs& a, size_t v_off, size_t amaps_off, int vpair) {
   t.a = a;
   t.R16 = round16i(a.max_rank);
+  t.amaps_off = amaps_off;
+  for (int p = 0; p < a.nproj; ++p)
+    for (int r = 8; r <= t.R16; r += 8) {
+      const cudaError_t err = cached_box_map(&t.atmpl[p][r / 8 - 1], a.x, r, a.d_in, (long)a.d_in * 2, 64, t.R16, true);
+      if (err != cudaSuccess) return err;
+    }
   t.pg = TB_MAXN1 / t.R16;
   if (t.pg > a.nproj) t.pg = a.nproj;
   t.npg = (a.nproj + t.pg - 1) / t.pg;
@@ -680,6 +680,7 @@ static void shrink_plan(TcPlan& t, const SgmmArgs& a, size_t v_off, int vpair) {
   if (t.stages > 8) t.stages = 8;
   t.vprep_off = v_off;
   t.vpair = vpair;
+  return cudaSuccess;
 }
 
 static cudaError_t launch_shrink(const TcPlan& t, cudaStream_t s) {
@@ -691,21 +692,26 @@ static cudaError_t launch_shrink(const TcPlan& t, cudaStream_t s) {
   const int nsm = device_sm_count();
   // tile counts are bounded by the plan's maxima; the kernel loops over the real ones
   const long max_q = max_qtiles(a.T, a.k, a.E);
-  const int g1 = (int)(max_q * t.npg < nsm ? max_q * t.npg : nsm);
+  int g1 = (int)(max_q * t.npg < nsm ? max_q * t.npg : nsm);
+  if (g1 > kShrinkMaxCtas) g1 = kShrinkMaxCtas;
   return launch_pdl(tc_shrink_kernel, dim3(g1), dim3(SH_BLOCK), sm1, s, t);
 }
 
 cudaError_t launch_tc_shrink_pairs(const SgmmArgs& a, size_t v_off, cudaStream_t s) {
-  TcPlan t;
-  memset(&t, 0, sizeof(t));
-  shrink_plan(t, a, v_off, 1);
-  return launch_shrink(t, s);
+  std::unique_ptr<TcPlan> t(new TcPlan);
+  memset(t.get(), 0, sizeof(TcPlan));
+  cudaError_t err;
+  if ((err = shrink_plan(*t, a, v_off, v_off + bank_vc_bytes(a.T, a.k, a.max_rank), 1)) != cudaSuccess) return err;
+  return launch_shrink(*t, s);
 }
 
 cudaError_t launch_sgmm_tensor(const SgmmArgs& a, size_t scratch_off, cudaStream_t s) {
-  TcPlan t;
+  std::unique_ptr<TcPlan> tp(new TcPlan);
+  TcPlan& t = *tp;
   memset(&t, 0, sizeof(t));
-  shrink_plan(t, a, scratch_off, 0);
+  cudaError_t err;
+  if ((err = shrink_plan(t, a, scratch_off, scratch_off + tc_vc_bytes(a.T, a.k, a.max_rank), 0)) != cudaSuccess)
+    return err;
   t.mixed = (a.k <= 2 && kMixAdapters * t.R16 <= TB_MAXK2) ? 1 : 0;
   t.K2 = (t.mixed ? kMixAdapters : a.k) * t.R16;
   t.ny = t.K2 <= 32 ? 4 : 3;
@@ -717,7 +723,6 @@ cudaError_t launch_sgmm_tensor(const SgmmArgs& a, size_t scratch_off, cudaStream
 
   const size_t sm2 = ex_smem(t.K2, t.ny).total;
   static SmemLimit lim2;
-  cudaError_t err;
   if ((err = lim2.ensure((const void*)tc_expand_kernel, sm2)) != cudaSuccess) return err;
   const int nsm = device_sm_count();
   const long max_s = (long)a.T + (a.T + TB_M - 1) / TB_M;

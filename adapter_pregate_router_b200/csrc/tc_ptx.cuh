@@ -19,6 +19,9 @@ cudaError_t encode_tile_map(CUtensorMap* m, const void* base, int rows, int cols
 // swizzle or none; zeros outside on loads.
 cudaError_t encode_box_map(CUtensorMap* m, const void* base, long rows, long cols, long pitch_bytes, int box_cols,
                            int box_rows, bool swizzle128);
+// The same, cached per shape: a template whose address the kernels replace (tmap_build).
+cudaError_t cached_box_map(CUtensorMap* m, const void* placeholder, long rows, long cols, long pitch_bytes,
+                           int box_cols, int box_rows, bool swizzle128);
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

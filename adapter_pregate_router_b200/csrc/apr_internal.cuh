@@ -30,7 +30,8 @@ struct WsHeader {
   int n_mtiles;     // tensor-core mixed tiles (<= 128 tokens, <= 4 adapters in all)
   unsigned sched;   // work counter of the tensor-core shrink (reset by the segment kernel and every expand)
   int T, k, E;      // routing the plan was built for
-  int pad[54];
+  int gplan;        // set and mixed tiles of the current plan built (the gathered expand's tiles)
+  int pad[53];
 };
 static_assert(sizeof(WsHeader) == 256, "header is one alignment unit");
 
@@ -378,6 +379,7 @@ struct SgmmArgs {
 };
 cudaError_t launch_sgmm_skinny(const SgmmArgs& a, int dtype, size_t scratch_off, cudaStream_t s);
 cudaError_t launch_sgmm_tensor(const SgmmArgs& a, size_t scratch_off, cudaStream_t s);
+cudaError_t launch_gather_plan(const int32_t* idx, int T, int k, int E, void* ws, cudaStream_t s);
 bool sgmm_ragged_supported(const SgmmArgs& a, int dtype);
 cudaError_t launch_sgmm_ragged(const SgmmArgs& a, size_t scratch_off, cudaStream_t s);
 

@@ -11,11 +11,13 @@
 //   tok_order[T]   tokens ordered by their sorted adapter tuple (LSD radix of
 //                  k stable counting sorts), so that tokens sharing an adapter
 //                  set are contiguous
-//   set tiles      runs of <= kSetTile tokens with one adapter set
 //   qtiles         tiles of <= 128 pairs of one adapter (tensor-core shrink)
+// The top-2 gathered tensor-core expand also needs, built on demand by the
+// first such call after the plan (gather_plan_kernel; no other path pays):
+//   set tiles      runs of <= kSetTile tokens with one adapter set
 //   mixed tiles    runs of <= 128 consecutive plan tokens whose adapters
-//                  number <= 4 (tensor-core expand, k <= 2), built by one
-//                  thread walking the set tiles in order
+//                  number <= 4 (k <= 2), built by one thread walking the set
+//                  tiles in order
 // The histograms use shared-memory atomics (order-free counts).  The order-
 // dependent steps (the stable scatters of the pairs and of the tokens, the set
 // tiles) run over blocks of 1024 consecutive items, all 32 warps at once: a
@@ -179,7 +181,6 @@ __global__ void __launch_bounds__(SEG_THREADS) segment_kernel(const int32_t* __r
   int* stage = reinterpret_cast<int*>(seg_smem + seg_smem_fixed(E));
   __shared__ int warp_sums[32];
   __shared__ int bad;
-  __shared__ int carry[2];
   const int tid = threadIdx.x;
   const int n = T * k;
   const WsLayout L = ws_layout(T, k, E);
@@ -218,6 +219,7 @@ __global__ void __launch_bounds__(SEG_THREADS) segment_kernel(const int32_t* __r
       hdr->n_stiles = 0;
       hdr->n_qtiles = 0;
       hdr->n_mtiles = 0;
+      hdr->gplan = 1;                  // the empty plan needs no gathered tiles
     }
     return;
   }
@@ -321,8 +323,36 @@ __global__ void __launch_bounds__(SEG_THREADS) segment_kernel(const int32_t* __r
   if (src != tok_order) {
     for (int i = tid; i < T; i += SEG_THREADS) tok_order[i] = src[i];
   }
-  const int* order = src;
-  __syncthreads();
+  // the gathered expand's set and mixed tiles are built on demand (gather_plan_kernel)
+  if (tid == 0) hdr->gplan = 0;
+}
+
+// Set tiles and mixed tiles of the current plan, the tiles of the gathered tensor-core expand
+// only: built by the first call that needs them after the plan (the header flag makes later calls
+// of the same plan return at once), so the other paths do not pay for them.
+template <bool STAGE>
+__global__ void __launch_bounds__(SEG_THREADS) gather_plan_kernel(const int32_t* __restrict__ idx_g, int T, int k,
+                                                                  int E, void* ws) {
+  pdl_wait();
+  pdl_trigger();
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
+  if (*reinterpret_cast<volatile int*>(&hdr->gplan)) return;
+  extern __shared__ __align__(16) unsigned char gp_smem[];
+  __shared__ int warp_sums[32];
+  __shared__ int carry[2];
+  const int tid = threadIdx.x;
+  const int n = T * k;
+  const WsLayout L = ws_layout(T, k, E);
+  const int* tok_order = ws_at<int>(ws, L.tok_order);
+  SetTile* stiles = ws_at<SetTile>(ws, L.stiles);
+  int* stage = reinterpret_cast<int*>(gp_smem);
+  if (STAGE) {
+    for (int q = tid; q < n; q += SEG_THREADS) stage[q] = idx_g[q];
+    for (int i = tid; i < T; i += SEG_THREADS) stage[n + i] = tok_order[i];
+    __syncthreads();
+  }
+  const int32_t* idx = STAGE ? stage : idx_g;
+  const int* order = STAGE ? stage + n : tok_order;
   // 6. set tiles: runs of equal adapter sets, split into <= kSetTile tokens.  A run starts
   //    where the set changes; a tile starts at a run start or every kSetTile tokens into a run.
   if (tid == 0) {
@@ -362,7 +392,10 @@ __global__ void __launch_bounds__(SEG_THREADS) segment_kernel(const int32_t* __r
   //    of the set tiles staged in shared memory.
   __syncthreads();
   if (k > 2) {
-    if (tid == 0) hdr->n_mtiles = 0;
+    if (tid == 0) {
+      hdr->n_mtiles = 0;
+      hdr->gplan = 1;
+    }
     return;
   }
   {
@@ -457,20 +490,33 @@ __global__ void __launch_bounds__(SEG_THREADS) segment_kernel(const int32_t* __r
       int nm = s_nm;
       if (s_cur.len > 0) mtiles[nm++] = s_cur;
       hdr->n_mtiles = nm;
+      hdr->gplan = 1;
     }
   }
 }
 
+
+cudaError_t launch_gather_plan(const int32_t* idx, int T, int k, int E, void* ws, cudaStream_t s) {
+  // idx and the token order go to shared memory when they fit beside the mixed-tile staging
+  constexpr size_t kStageBudget = 200 * 1024;
+  const size_t need = sizeof(int) * ((size_t)T * k + (size_t)T);
+  static SmemLimit lim;
+  cudaError_t err;
+  if (need <= kStageBudget) {
+    if ((err = lim.ensure((const void*)gather_plan_kernel<true>, need)) != cudaSuccess) return err;
+    return launch_pdl(gather_plan_kernel<true>, dim3(1), dim3(SEG_THREADS), need, s, idx, T, k, E, ws);
+  }
+  return launch_pdl(gather_plan_kernel<false>, dim3(1), dim3(SEG_THREADS), 0, s, idx, T, k, E, ws);
+}
+
 cudaError_t launch_segment(const int32_t* idx, int T, int k, int E, int32_t* seg_off,
                            int32_t* perm, void* ws, cudaStream_t s) {
-  // idx and the token arrays go to shared memory when they fit beside the fixed tables and the
-  // mixed-tile staging (static, 16 KB)
+  // idx and the token arrays go to shared memory when they fit beside the fixed tables
   constexpr size_t kStageBudget = 200 * 1024;
   const size_t fixed = seg_smem_fixed(E);
   const bool stage = fixed + seg_smem_stage(T, k) <= kStageBudget;
   const size_t smem = fixed + (stage ? seg_smem_stage(T, k) : 0);
-  // the kernel's static shared memory (mixed-tile staging, 16 KB) counts against the same 48 KB
-  // default as the dynamic part, so the limit is raised for every size
+  // the limit is raised for every size (static and dynamic shared memory count against one limit)
   static SmemLimit lim[2];
   cudaError_t err;
   if (stage) {

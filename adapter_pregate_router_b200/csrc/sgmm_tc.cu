@@ -721,6 +721,8 @@ cudaError_t launch_sgmm_tensor(const SgmmArgs& a, size_t scratch_off, cudaStream
   t.cc_before[0] = 0;
   for (int p = 0; p < a.nproj; ++p) t.cc_before[p + 1] = t.cc_before[p] + (a.proj[p].d_out + TB_CW - 1) / TB_CW;
 
+  // the set and mixed tiles of the plan, on the first gathered call after it
+  if ((err = launch_gather_plan(a.idx, a.T, a.k, a.E, a.ws, s)) != cudaSuccess) return err;
   const size_t sm2 = ex_smem(t.K2, t.ny).total;
   static SmemLimit lim2;
   if ((err = lim2.ensure((const void*)tc_expand_kernel, sm2)) != cudaSuccess) return err;

@@ -472,6 +472,42 @@ def test_sgmm_tensor_rejects_unsupported(apr):
     assert ei.value.status == apr.APR_ERR_UNSUPPORTED
 
 
+def test_sgmm_tensor_plan_reuse_across_calls(apr):
+    """Top-2 gathered calls that share one workspace: the set and mixed tiles are built by the
+    first call after a plan and reused by the next; a new plan (another routing, other token
+    count) rebuilds them.  Every call is checked against the oracle."""
+    rng = np.random.default_rng(61)
+    E, ranks = 12, (16,) * 12
+    ws = apr.workspace(1500, 2, E, 16, 512)
+    for T, reps in ((1000, 2), (1500, 2), (700, 1)):
+        idx = _zipf_idx(rng, T, E, 2)
+        x, As, Bs, idx, gate, ybs = _case(rng, T, 512, (256, 144), ranks, 2, dist=idx)
+        x, As, Bs, ybs = _rounded(x, As, Bs, ybs)
+        idx_d = torch.from_numpy(np.ascontiguousarray(idx, dtype=np.int32)).cuda()
+        gate_d = torch.from_numpy(np.ascontiguousarray(gate, dtype=np.float32)).cuda()
+        seg_off = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+        perm = torch.empty(T * 2, dtype=torch.int32, device="cuda")
+        apr.segment_tokens(idx_d, E, seg_off, perm, ws)
+        xd = torch.from_numpy(x).cuda().to(BF16)
+        keep = []
+        tabs = []
+        for p in range(2):
+            A = [torch.from_numpy(a).cuda().to(BF16) for a in As[p]]
+            B = [torch.from_numpy(b).cuda().to(BF16) for b in Bs[p]]
+            keep += [A, B]
+            tabs.append((apr.ptr_array(A), apr.ptr_array(B)))
+        rk = torch.full((E,), 16, dtype=torch.int32, device="cuda")
+        ref = oracle_group(x, As, Bs, idx, gate.astype(np.float64), ybs)
+        for _ in range(reps):
+            ys = [torch.full_like(torch.from_numpy(y), float("nan")).cuda().to(BF16) for y in ybs]
+            yb = [torch.from_numpy(y).cuda().to(BF16) for y in ybs]
+            projs = [apr.make_proj(ys[p], yb[p], tabs[p][0], tabs[p][1]) for p in range(2)]
+            apr.sgmm_shrink_expand(xd, projs, 2, E, rk, 16, idx_d, gate_d, seg_off, perm, ws, apr.SGMM_TENSOR)
+            apr.stream_status(ws)
+            for p in range(2):
+                close(to_np(ys[p]), ref[p], f"T={T} proj {p}")
+
+
 # ------------------------------------------------------------------ SGMM, ragged many-tenant tiles (top-1)
 
 _RANKS_8_128 = tuple(range(8, 136, 8))

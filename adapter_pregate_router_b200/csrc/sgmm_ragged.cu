@@ -12,9 +12,9 @@
 // projections; the adapter's rank rows are the MMA's M side and the tokens its
 // N side, so a short segment costs only its own tokens.  A arrives by 2-D TMA
 // boxes from tensor maps the kernel writes per item (a template per rank with
-// the adapter's address), x rows by 16-byte cp.async, 128 columns (256 bytes of
-// every row) per stage.  The same kernel builds the ragged tiles and each used
-// adapter's B tensor map for the expand.
+// the adapter's address), x rows by 16-byte cp.async; each stage packs as many
+// 64-column sub-blocks of the item's own rows as fit.  The same kernel builds
+// the ragged tiles and each used adapter's B tensor map for the expand.
 //
 // Expand (ragged_expand_kernel): with many adapters each one holds only a few
 // tokens, so a tile of one adapter would leave most of the 128 MMA rows empty.
@@ -174,11 +174,12 @@ __device__ void rg_plan(const SgmmArgs& a, int R16, int* count, RgTile* tiles, i
 // sub-blocks as fit the item: each holds the item's N token rows and nq * w rank rows (128-byte
 // swizzled rows); an accumulator's MMAs read 128 rank rows, the rows past nq * w being whatever
 // follows (the products of those rows are never read), so a small item moves up to 8 sub-blocks
-// (512 columns) per stage instead of paying a fixed 128-row tile.  One warp issues TMA boxes of
-// A_e (64 columns x w rows from a tensor map made for the item: the projection's template for
-// rank r_e with A_e's address, zeros past r_e); four loader warps copy the tokens' x rows with
-// 16-byte cp.async; one thread issues the MMAs; eight epilogue warps read D back (a TMEM lane per
-// rank row), scale by each token's gate and store bf16.  Items come from a work counter (after
+// (512 columns) per stage instead of paying a fixed 128-row tile.  A setup warp prepares the next
+// item (its tokens and gates, and its A tensor maps: the projection's template for rank r_e with
+// A_e's address, zeros past r_e) while one warp issues the current item's A boxes (64 columns x w
+// rows); four loader warps copy the tokens' x rows with 16-byte cp.async; one thread issues the
+// MMAs; eight epilogue warps read D back (a TMEM lane per rank row), scale by each token's gate and
+// store bf16.  Items come from a work counter (after
 // one static item per CTA), so CTAs drawing high-rank adapters take fewer of them.
 constexpr int RS_EPI = 256;                   // warps 2-9
 constexpr int RS_XW = 128;                    // warps 10-13: x rows by 16-byte cp.async
@@ -189,7 +190,7 @@ constexpr int RS_MAXSB = 8;                   // 64-column sub-blocks per stage 
 constexpr int RS_NQ = 4;                      // projections per item at most
 
 struct RsPlan {
-  CUtensorMap xmap;                               // x rows (unused by the loads; kept for the shapes)
+  CUtensorMap xmap;                               // x rows (encoded with the plan; the loads are cp.async)
   CUtensorMap atmpl[APR_MAX_PROJ][APR_MAX_RANK / 8];   // A_e of rank 8 (j + 1): [r, d_in], 64 x round16(r) boxes, swizzled
   CUtensorMap btmpl[APR_MAX_PROJ][APR_MAX_RANK / 8];   // B_e of rank 8 (j + 1): [d_out, r], 8 x 128 boxes, plain
   SgmmArgs a;

@@ -177,8 +177,11 @@ typedef struct apr_proj {
  * seg_off,perm device: the outputs of apr_segment_tokens for this idx; `ws`
  *          must be the workspace that call wrote.
  * kernel   APR_SGMM_AUTO, or a forced kernel class.  With R16 = max_rank
- *          rounded up to 16: the tensor-core kernel needs dtype == APR_BF16,
- *          k <= 2, k * R16 <= 64, d_in % 64 == 0 and d_out % 16 == 0; the
+ *          rounded up to 16: the tensor-core kernel needs dtype == APR_BF16
+ *          and d_in % 64 == 0, and for k = 2 also k * R16 <= 64 and
+ *          d_out % 16 == 0 (k = 1 takes every rank up to APR_MAX_RANK: the
+ *          adapters of up to 16 short segments share one 128-token tile,
+ *          the Chameleon page's many tenants of ranks 8-128); the
  *          dense kernel needs dtype == APR_BF16, T <= 64, E <= 16 and
  *          E * R16 <= 256; the bank kernel needs dtype == APR_BF16, R16 in
  *          {16, 32, 64}, k <= 4, k * R16 <= 64, E * R16 <= 256 and
